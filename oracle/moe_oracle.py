@@ -1,0 +1,464 @@
+"""CPU oracle for the forward pass of a sparse Mixture-of-Experts FFN layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / reference leg of ``bench.py`` may import this module.
+It shares no code with the CUDA path and imports nothing from it; it takes
+plain numpy arrays (bf16 tensors arrive as their raw uint16 bit patterns, or
+as float32/float64 arrays holding the exact widened values).
+
+What it computes, step by step, and the passage each step follows:
+
+1. Router logits ``l = x . W_r^T (+ b)``: the router is "an FFN plus a
+   softmax layer" ("大语言模型并行策略（七）：专家并行", section
+   "Mixture of Experts (MoE)"); read here as one bias-free linear layer over
+   the routed experts.  Accumulated in float64, rounded once to fp32.
+2. Softmax gating ``p_i = exp(g_i) / sum_j exp(g_j)`` ("MoE技术演进",
+   "Adaptive Mixtures of Local Experts", gating-network equation).  Exact
+   mathematics, but evaluated by a fixed fp32 recipe (``exp_det`` and a
+   sequential ascending-expert sum) because expert-choice selection and
+   affinity-based token dropping compare probabilities across tokens: both
+   sides must take those integer decisions in the same precision.
+3. Selection:
+   a. token choice top-k by weight, lower expert index on ties ("MoE技术演进",
+      "Adaptive Mixtures of Local Experts", selector; GShard section 1 top-2);
+      optional group-limited routing (DeepSeek-V2 section 3, device-limited
+      routing: pick M groups, then top-K inside them);
+   b. expert capacity with overflow dropped to the residual (GShard
+      section 1, expert capacity C = O(N/E));
+   c. per-expert affinity-based token dropping, keep the top fraction
+      (DeepSeek-V2 section 5, token-dropping strategy);
+   d. expert choice: each expert takes its top-C tokens (LocMoE+ article,
+      token-choice vs expert-choice routers);
+   e. shared experts applied to every token with gate 1 (DeepSeekMoE
+      section 2, shared expert isolation equation).
+4. Permutation into expert-contiguous rows (the single-GPU counterpart of the
+   count-then-fill send buffers, "大语言模型并行策略（七）：专家并行",
+   section "MoE 中的 all-to-all 通信").
+5. Expert FFNs ``w_o . ReLU(w_i . x)`` (GShard section 3, FFN_e equation) or
+   SwiGLU with 3 * d_model * d_moe parameters ("大语言模型并行策略（七）",
+   parameter-count notes), and the gate-weighted combine
+   ``y_s = sum_e G_{s,e} FFN_e(x_s)`` (GShard section 3) plus the shared
+   experts' sum (DeepSeekMoE section 2).  Float64 throughout; the residual
+   ``+ u`` of the DeepSeekMoE equations is left to the caller.
+
+Readings where the pages are silent (each is repeated in the design notes):
+capacity ``C = ceil(cf * k * T / E)`` with one group; drop priority
+``q = j * T + t`` (every first choice before any second choice, lower token
+first); top-k keys are the fp32 logits; gates are the unnormalised
+probabilities unless ``renormalize``; group score = max logit in a
+contiguous group; keep-fraction keys = p, ties to the lower token, applied
+per expert after top-k; expert-choice keys = p, ties to the lower token,
+segment order ascending token; SwiGLU = ``W_down (SiLU(W_gate x) * W_up x)``.
+
+Every function here is pinned by tests under ``tests/`` against closed forms,
+brute-force enumeration, special cases that reduce to a dense FFN or a dense
+soft mixture, and invariants; none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+
+F32 = np.float32
+
+# --------------------------------------------------------------------------
+# input decoding
+# --------------------------------------------------------------------------
+
+
+def widen(a: np.ndarray) -> np.ndarray:
+    """Exact float64 values of an input array.
+
+    uint16 arrays are bf16 bit patterns (the upper half of an fp32 word);
+    float arrays are taken as they are.
+    """
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# step 2 arithmetic: a fixed fp32 exponential
+# --------------------------------------------------------------------------
+
+# Cody-Waite range reduction: ln 2 split into a 16-bit head (so n * LN2_HI is
+# exact for |n| < 256) and the fp32-rounded remainder.
+LOG2E = F32(1.4426950408889634)
+LN2_HI = F32(45426.0 / 65536.0)                       # 0.693145751953125
+LN2_LO = F32(math.log(2.0) - 45426.0 / 65536.0)       # 1.4286068e-06
+# Taylor coefficients 1/i!, i = 0..7, rounded to fp32
+EXP_COEF = tuple(F32(1.0 / math.factorial(i)) for i in range(8))
+EXP_FLUSH = F32(-87.0)     # below this exp(z) < 2**-125: returned as 0
+
+
+def exp_det(z: np.ndarray) -> np.ndarray:
+    """exp(z) for fp32 z <= 0, by one fixed sequence of rounded fp32 ops.
+
+    n = rint(z * log2 e); r = (z - n ln2_hi) - n ln2_lo; a degree-7 Taylor
+    polynomial of e^r in Horner form, each step one rounded multiply and one
+    rounded add (no fused multiply-add); then the exact scale by 2**n built
+    from exponent bits.  z < -87 returns 0.  Error against exp: a few ulp
+    (pinned in the tests).
+    """
+    z = np.asarray(z, dtype=F32)
+    with np.errstate(over="ignore", invalid="ignore"):      # flushed lanes may overflow
+        return _exp_det(z)
+
+
+def _exp_det(z: np.ndarray) -> np.ndarray:
+    n = np.rint(z * LOG2E).astype(F32)
+    r = (z - n * LN2_HI).astype(F32)
+    r = (r - n * LN2_LO).astype(F32)
+    p = np.full_like(z, EXP_COEF[7])
+    for c in EXP_COEF[6::-1]:
+        p = (p * r).astype(F32)
+        p = (p + c).astype(F32)
+    ni = np.clip(n, -126, 0).astype(np.int32)
+    scale = ((ni + 127).astype(np.uint32) << np.uint32(23)).view(F32)
+    out = (p * scale).astype(F32)
+    return np.where(z < EXP_FLUSH, F32(0.0), out).astype(F32)
+
+
+# --------------------------------------------------------------------------
+# steps 1-2
+# --------------------------------------------------------------------------
+
+
+def router_logits(x: np.ndarray, w_router: np.ndarray, bias: np.ndarray | None = None) -> np.ndarray:
+    """l[t, e] = sum_i x[t, i] W_r[e, i] (+ b[e]) in float64, rounded to fp32."""
+    acc = widen(x) @ widen(w_router).T
+    if bias is not None:
+        acc = acc + widen(bias)[None, :]
+    return acc.astype(F32)
+
+
+def softmax_det(logits: np.ndarray) -> np.ndarray:
+    """p[t, e] = exp(l - m) / sum_e' exp(l' - m), m = max_e l, in fixed fp32.
+
+    z = l - m is one rounded fp32 subtraction; exp is ``exp_det``; the
+    denominator is summed sequentially in ascending expert order in fp32;
+    the quotient is one rounded fp32 division.
+    """
+    l = np.asarray(logits, dtype=F32)
+    m = l.max(axis=1, keepdims=True)
+    z = (l - m).astype(F32)
+    e = exp_det(z)
+    s = e[:, 0].copy()
+    for j in range(1, l.shape[1]):
+        s = (s + e[:, j]).astype(F32)
+    return (e / s[:, None]).astype(F32)
+
+
+# --------------------------------------------------------------------------
+# step 3a: token-choice top-k
+# --------------------------------------------------------------------------
+
+
+def group_limited_mask(logits: np.ndarray, n_groups: int, topk_groups: int) -> np.ndarray:
+    """Boolean [T, E]: experts inside each token's top ``topk_groups`` groups.
+
+    Groups are ``n_groups`` contiguous blocks of E / n_groups experts; a
+    group's score is its largest logit; groups rank by score, lower group
+    index on ties.
+    """
+    l = np.asarray(logits, dtype=F32)
+    T, E = l.shape
+    gsz = E // n_groups
+    score = l.reshape(T, n_groups, gsz).max(axis=2)
+    order = np.argsort(-score, axis=1, kind="stable")       # stable: lower group first on ties
+    chosen = np.zeros((T, n_groups), dtype=bool)
+    np.put_along_axis(chosen, order[:, :topk_groups], True, axis=1)
+    return np.repeat(chosen, gsz, axis=1)
+
+
+def topk_route(logits: np.ndarray, probs: np.ndarray, k: int, n_groups: int = 0,
+               topk_groups: int = 0, renormalize: bool = False):
+    """Per token: the k experts with the largest logits, in rank order.
+
+    A strictly larger logit ranks first; equal logits go to the lower expert
+    index (softmax is monotone, so this is the top-k of p with exact ties
+    broken by index).  With group limits only experts of the chosen groups
+    compete.  Gate = p of the chosen expert, or p / (sum of the chosen p,
+    summed in rank order in fp32) when ``renormalize``.
+    Returns (topk_idx int32 [T, k], topk_gate fp32 [T, k]).
+    """
+    l = np.asarray(logits, dtype=F32)
+    keys = -l.astype(np.float64)
+    if n_groups > 0:
+        allowed = group_limited_mask(l, n_groups, topk_groups)
+        keys = np.where(allowed, keys, np.inf)
+    order = np.argsort(keys, axis=1, kind="stable")           # ties keep ascending expert index
+    idx = order[:, :k].astype(np.int32)
+    gate = np.take_along_axis(np.asarray(probs, dtype=F32), idx, axis=1).astype(F32)
+    if renormalize:
+        s = gate[:, 0].copy()
+        for j in range(1, k):
+            s = (s + gate[:, j]).astype(F32)
+        gate = (gate / s[:, None]).astype(F32)
+    return idx, gate
+
+
+# --------------------------------------------------------------------------
+# steps 3b-3d and 4: dispatch / permutation
+# --------------------------------------------------------------------------
+
+
+@dataclass
+class Dispatch:
+    """Expert-contiguous row layout produced by selection + permutation.
+
+    counts[e]   assignments made to expert e before any drop (token choice),
+                or the tokens it picked (expert choice)
+    kept[e]     rows expert e actually processes
+    offsets     exclusive scan of kept, length E + 1
+    row_token   token of each row, length offsets[E]
+    row_gate    gate of each row (fp32)
+    tok_rows    token choice: [T, k], the row of (t, j) or -1 when dropped;
+                expert choice: [E, T], the row of (e, t) or -1
+    n_dropped   token choice: assignments dropped by capacity / keep-fraction
+    """
+
+    counts: np.ndarray
+    kept: np.ndarray
+    offsets: np.ndarray
+    row_token: np.ndarray
+    row_gate: np.ndarray
+    tok_rows: np.ndarray
+    n_dropped: int
+
+
+def capacity_from_factor(T: int, E: int, k: int, capacity_factor: float) -> int:
+    """C = ceil(cf * k * T / E); 0 means unlimited (cf <= 0)."""
+    if capacity_factor <= 0:
+        return 0
+    return int(math.ceil(capacity_factor * k * T / E))
+
+
+def keep_count(n: np.ndarray, keep_num: int, keep_den: int) -> np.ndarray:
+    """ceil(n * num / den) in integers; num = den = 0 keeps everything."""
+    n = np.asarray(n, dtype=np.int64)
+    if keep_den <= 0:
+        return n
+    return (n * keep_num + keep_den - 1) // keep_den
+
+
+def _priority_ranks(topk_idx: np.ndarray, E: int):
+    """Stable counting sort of assignments by expert in priority order.
+
+    Assignment (t, j) has priority q = j * T + t.  Returns the expert of each
+    q, the q's grouped by expert (ascending q inside each expert), the start
+    of each expert's group, and the rank of each q inside its expert.
+    """
+    T, k = topk_idx.shape
+    e_of_q = np.asarray(topk_idx, dtype=np.int64).T.reshape(-1)     # q = j*T + t
+    by_expert = np.argsort(e_of_q, kind="stable")                   # stable: ascending q per expert
+    counts = np.bincount(e_of_q, minlength=E).astype(np.int64)
+    start = np.concatenate([[0], np.cumsum(counts)[:-1]])
+    rank = np.empty(T * k, dtype=np.int64)
+    rank[by_expert] = np.arange(T * k) - start[e_of_q[by_expert]]
+    return e_of_q, by_expert, counts, start, rank
+
+
+def dispatch_token_choice(topk_idx: np.ndarray, topk_gate: np.ndarray, probs: np.ndarray | None,
+                          E: int, capacity: int = 0, keep_num: int = 0, keep_den: int = 0) -> Dispatch:
+    """Token-choice dispatch with an optional capacity or keep-fraction.
+
+    Capacity C > 0: the assignment of priority q is kept iff fewer than C
+    assignments of smaller q went to the same expert; the rest overflow to
+    the residual and contribute nothing here.
+    Keep-fraction num/den: expert e keeps ceil(n_e * num / den) of its n_e
+    assignments, those with the largest p[t, e] (lower t on ties).
+    Rows of an expert are its kept assignments in priority order.
+    """
+    topk_idx = np.asarray(topk_idx)
+    T, k = topk_idx.shape
+    e_of_q, by_expert, counts, start, rank = _priority_ranks(topk_idx, E)
+    t_of_q = np.arange(T * k) % T
+    keep = np.ones(T * k, dtype=bool)
+    if capacity > 0:
+        keep = rank < capacity
+    elif keep_den > 0:
+        p = np.asarray(probs, dtype=F32)
+        m = keep_count(counts, keep_num, keep_den)
+        for e in range(E):
+            qs = by_expert[start[e]:start[e] + counts[e]]
+            pe = p[t_of_q[qs], e]
+            # sort by p descending, then t ascending
+            order = np.lexsort((t_of_q[qs], -pe.astype(np.float64)))
+            dropped = qs[order[m[e]:]]
+            keep[dropped] = False
+    kept = np.bincount(e_of_q[keep], minlength=E).astype(np.int64)
+    offsets = np.concatenate([[0], np.cumsum(kept)]).astype(np.int64)
+    # position among the kept rows of the same expert, in priority order
+    kept_rank = np.zeros(T * k, dtype=np.int64)
+    for e in range(E):
+        qs = by_expert[start[e]:start[e] + counts[e]]
+        qk = qs[keep[qs]]
+        kept_rank[qk] = np.arange(len(qk))
+    slot_q = np.where(keep, offsets[e_of_q] + kept_rank, -1)
+    tok_rows = slot_q.reshape(k, T).T.astype(np.int32).copy()
+    R = int(offsets[E])
+    row_token = np.empty(R, dtype=np.int32)
+    row_gate = np.empty(R, dtype=F32)
+    gate_q = np.asarray(topk_gate, dtype=F32).T.reshape(-1)
+    row_token[slot_q[keep]] = t_of_q[keep]
+    row_gate[slot_q[keep]] = gate_q[keep]
+    return Dispatch(counts.astype(np.int32), kept.astype(np.int32), offsets.astype(np.int32),
+                    row_token, row_gate, tok_rows, int(T * k - keep.sum()))
+
+
+def dispatch_expert_choice(probs: np.ndarray, C: int) -> Dispatch:
+    """Expert choice: expert e takes the C tokens with the largest p[t, e].
+
+    Ties go to the lower token index; rows of an expert are its tokens in
+    ascending token order; gate = p[t, e].  A token may be taken by any
+    number of experts, including none.
+    """
+    p = np.asarray(probs, dtype=F32)
+    T, E = p.shape
+    tok_rows = np.full((E, T), -1, dtype=np.int32)
+    row_token = np.empty(E * C, dtype=np.int32)
+    row_gate = np.empty(E * C, dtype=F32)
+    t = np.arange(T)
+    for e in range(E):
+        order = np.lexsort((t, -p[:, e].astype(np.float64)))
+        chosen = np.sort(order[:C])
+        rows = e * C + np.arange(C)
+        row_token[rows] = chosen
+        row_gate[rows] = p[chosen, e]
+        tok_rows[e, chosen] = rows
+    counts = np.full(E, C, dtype=np.int32)
+    offsets = (np.arange(E + 1) * C).astype(np.int32)
+    return Dispatch(counts, counts.copy(), offsets, row_token, row_gate, tok_rows, 0)
+
+
+def permute_rows(x: np.ndarray, d: Dispatch) -> np.ndarray:
+    """x_perm[r] = x[row_token[r]] (bit patterns copied as they are)."""
+    return np.asarray(x)[d.row_token]
+
+
+# --------------------------------------------------------------------------
+# step 5: expert FFNs and combine
+# --------------------------------------------------------------------------
+
+
+def expert_ffn(xrows: np.ndarray, w1_e, w2_e, w3_e=None, act: str = "relu") -> np.ndarray:
+    """FFN_e of a batch of rows in float64.
+
+    ReLU:   w2 . ReLU(w1 . x)                      (GShard section 3)
+    SwiGLU: w2 . (SiLU(w1 . x) * (w3 . x)),  SiLU(z) = z / (1 + e^-z)
+    Weight layout: w1, w3 [f, d]; w2 [d, f] (each output neuron's weights
+    contiguous along the input dimension).
+    """
+    xr = widen(xrows)
+    g = xr @ widen(w1_e).T
+    if act == "relu":
+        h = np.maximum(g, 0.0)
+    elif act == "swiglu":
+        u = xr @ widen(w3_e).T
+        h = g / (1.0 + np.exp(-g)) * u
+    else:
+        raise ValueError(act)
+    return h @ widen(w2_e).T
+
+
+@dataclass
+class OracleConfig:
+    """The layer's options, as the oracle sees them."""
+
+    E: int
+    S: int
+    k: int
+    act: str = "relu"
+    mode: str = "tc"
+    capacity: int = 0
+    keep_num: int = 0
+    keep_den: int = 0
+    ec_capacity: int = 0
+    n_groups: int = 0
+    topk_groups: int = 0
+    renormalize: bool = False
+
+
+@dataclass
+class OracleResult:
+    logits: np.ndarray
+    probs: np.ndarray
+    topk_idx: np.ndarray | None
+    topk_gate: np.ndarray | None
+    dispatch: Dispatch
+    tokens: np.ndarray          # tokens whose output was computed
+    y: np.ndarray               # float64 [len(tokens), d]
+
+
+def route(cfg: OracleConfig, logits: np.ndarray):
+    """Steps 2-4 from given fp32 logits: probabilities, selection, dispatch."""
+    probs = softmax_det(logits)
+    if cfg.mode == "ec":
+        return probs, None, None, dispatch_expert_choice(probs, cfg.ec_capacity)
+    idx, gate = topk_route(logits, probs, cfg.k, cfg.n_groups, cfg.topk_groups, cfg.renormalize)
+    disp = dispatch_token_choice(idx, gate, probs, cfg.E, cfg.capacity, cfg.keep_num, cfg.keep_den)
+    return probs, idx, gate, disp
+
+
+def combine_tokens(cfg: OracleConfig, x, w1, w2, w3, disp: Dispatch, tokens) -> np.ndarray:
+    """y_t = sum over t's kept (expert, gate) of gate * FFN_e(x_t) + sum_s FFN_s(x_t).
+
+    Computed per expert on the requested tokens only, in float64.  The
+    routed terms are added in the token's k-rank order (expert choice:
+    ascending expert), then the shared experts in index order.
+    """
+    tokens = np.asarray(tokens, dtype=np.int64)
+    x = np.asarray(x)
+    d = x.shape[1]
+    y = np.zeros((len(tokens), d), dtype=np.float64)
+    # (token position, slot order, expert, gate) for every routed term
+    terms = []
+    if cfg.mode == "ec":
+        for e in range(cfg.E):
+            rows = disp.tok_rows[e, tokens]
+            for i, r in enumerate(rows):
+                if r >= 0:
+                    terms.append((i, e, e, float(disp.row_gate[r])))
+    else:
+        for i, t in enumerate(tokens):
+            for j in range(disp.tok_rows.shape[1]):
+                r = disp.tok_rows[t, j]
+                if r >= 0:
+                    e = int(np.searchsorted(disp.offsets, r, side="right") - 1)
+                    terms.append((i, j, e, float(disp.row_gate[r])))
+    terms.sort(key=lambda z: (z[0], z[1]))
+    # evaluate FFN_e once per expert on the tokens that need it
+    contrib: dict[tuple[int, int], np.ndarray] = {}
+    by_e: dict[int, list] = {}
+    for (i, j, e, g) in terms:
+        by_e.setdefault(e, []).append((i, j, g))
+    for e, lst in by_e.items():
+        rows = x[tokens[[i for (i, _, _) in lst]]]
+        out = expert_ffn(rows, w1[e], w2[e], None if w3 is None else w3[e], cfg.act)
+        for n, (i, j, g) in enumerate(lst):
+            contrib[(i, j)] = g * out[n]
+    for (i, j, e, g) in terms:
+        y[i] += contrib[(i, j)]
+    for s in range(cfg.S):
+        ge = cfg.E + s
+        y += expert_ffn(x[tokens], w1[ge], w2[ge], None if w3 is None else w3[ge], cfg.act)
+    return y
+
+
+def forward(cfg: OracleConfig, x, w_router, bias, w1, w3, w2, tokens=None) -> OracleResult:
+    """The whole layer: routing for every token, outputs for ``tokens``.
+
+    Routing (steps 1-4) always covers all T tokens because capacity,
+    keep-fraction and expert choice couple tokens; the FFN and combine
+    (step 5) are evaluated only for the requested tokens (all by default).
+    """
+    logits = router_logits(x, w_router, bias)
+    probs, idx, gate, disp = route(cfg, logits)
+    T = logits.shape[0]
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    y = combine_tokens(cfg, x, w1, w2, w3, disp, tokens)
+    return OracleResult(logits, probs, idx, gate, disp, tokens, y)

@@ -1,0 +1,137 @@
+"""Planted mistakes in the oracle must trip at least one pin.
+
+Each case patches one plausible error into the oracle (on the CPU only) and
+re-runs the pin that is meant to catch it; the pin must fail.  This checks
+that the pins constrain the oracle rather than restate it.
+"""
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+from tests import test_oracle_dispatch as TD
+from tests import test_oracle_ffn as TF
+from tests import test_oracle_gating as TG
+from tests import test_oracle_selection as TS
+
+
+def _expect_pin_failure(pin, *args):
+    with pytest.raises(AssertionError):
+        pin(*args)
+
+
+def test_token_major_priority_is_caught(monkeypatch):
+    """Priority q = t*k + j (token-major) instead of j*T + t."""
+    orig = O._priority_ranks
+
+    def wrong(topk_idx, E):
+        T, k = topk_idx.shape
+        e_tok_major = np.asarray(topk_idx, np.int64).reshape(-1)          # q' = t*k + j
+        by = np.argsort(e_tok_major, kind="stable")
+        # map back to the j*T + t numbering the rest of the oracle uses
+        q_of_qp = (np.arange(T * k) % k) * T + np.arange(T * k) // k
+        e_of_q, _, counts, start, _ = orig(topk_idx, E)
+        rank = np.empty(T * k, np.int64)
+        rank[q_of_qp[by]] = np.arange(T * k) - start[e_tok_major[by]]
+        by_expert = q_of_qp[by]
+        return e_of_q, by_expert, counts, start, rank
+
+    monkeypatch.setattr(O, "_priority_ranks", wrong)
+    _expect_pin_failure(TD.test_capacity_golden)
+
+
+def test_reversed_tie_rule_is_caught(monkeypatch):
+    orig = O.topk_route
+
+    def wrong(logits, probs, k, n_groups=0, topk_groups=0, renormalize=False):
+        l = np.asarray(logits, np.float32)
+        E = l.shape[1]
+        idx, gate = orig(l[:, ::-1], np.asarray(probs)[:, ::-1], k, n_groups, topk_groups, renormalize)
+        return (E - 1 - idx).astype(np.int32), gate                    # higher index wins ties
+
+    monkeypatch.setattr(O, "topk_route", wrong)
+    _expect_pin_failure(TS.test_topk_golden)
+
+
+def test_dropped_gate_is_caught(monkeypatch):
+    orig = O.dispatch_token_choice
+
+    def wrong(topk_idx, topk_gate, probs, E, capacity=0, keep_num=0, keep_den=0):
+        return orig(topk_idx, np.ones_like(topk_gate), probs, E, capacity, keep_num, keep_den)
+
+    monkeypatch.setattr(O, "dispatch_token_choice", wrong)
+    _expect_pin_failure(TF.test_k_equals_E_is_dense_soft_mixture, "relu")
+
+
+@pytest.mark.parametrize("act", ["relu", "swiglu"])
+def test_wrong_activation_is_caught(monkeypatch, act):
+    orig = O.expert_ffn
+
+    def wrong(xrows, w1_e, w2_e, w3_e=None, act="relu"):
+        if act == "relu":                       # activation dropped
+            return O.widen(xrows) @ O.widen(w1_e).T @ O.widen(w2_e).T
+        return orig(xrows, w3_e, w2_e, w1_e, act)   # gate and up swapped
+
+    monkeypatch.setattr(O, "expert_ffn", wrong)
+    _expect_pin_failure(TF.test_single_expert_is_dense_ffn, act)
+
+
+def test_missing_shared_term_is_caught(monkeypatch):
+    orig = O.combine_tokens
+
+    def wrong(cfg, x, w1, w2, w3, disp, tokens):
+        cfg2 = O.OracleConfig(**{**cfg.__dict__, "S": 0})
+        return orig(cfg2, x, w1, w2, w3, disp, tokens)
+
+    monkeypatch.setattr(O, "combine_tokens", wrong)
+    _expect_pin_failure(TF.test_shared_experts_alone)
+
+
+def test_expert_choice_high_token_ties_is_caught(monkeypatch):
+    orig = O.dispatch_expert_choice
+
+    def wrong(probs, C):
+        p = np.asarray(probs)[::-1]
+        d = orig(p, C)
+        T = p.shape[0]
+        d.row_token = (T - 1 - d.row_token).astype(np.int32)
+        return d
+
+    monkeypatch.setattr(O, "dispatch_expert_choice", wrong)
+    _expect_pin_failure(TD.test_expert_choice_golden)
+
+
+def test_missing_low_ln2_correction_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "LN2_LO", np.float32(0.0))
+    _expect_pin_failure(TG.test_exp_det_within_two_ulp)
+
+
+def test_softmax_without_denominator_order_is_caught(monkeypatch):
+    """Normalising by the max instead of the sum."""
+    def wrong(logits):
+        l = np.asarray(logits, np.float32)
+        e = O.exp_det((l - l.max(1, keepdims=True)).astype(np.float32))
+        return e
+
+    monkeypatch.setattr(O, "softmax_det", wrong)
+    _expect_pin_failure(TG.test_softmax_golden)
+
+
+def test_keep_fraction_floor_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "keep_count", lambda n, a, b: (np.asarray(n) * a) // b if b > 0 else np.asarray(n))
+    _expect_pin_failure(TD.test_keep_fraction_golden)
+
+
+def test_group_score_sum_is_caught(monkeypatch):
+    """Group score = sum of the group's logits instead of its maximum."""
+    def wrong(logits, n_groups, topk_groups):
+        l = np.asarray(logits, np.float32)
+        T, E = l.shape
+        gsz = E // n_groups
+        score = l.reshape(T, n_groups, gsz).sum(axis=2)
+        order = np.argsort(-score, axis=1, kind="stable")
+        chosen = np.zeros((T, n_groups), bool)
+        np.put_along_axis(chosen, order[:, :topk_groups], True, axis=1)
+        return np.repeat(chosen, gsz, axis=1)
+
+    monkeypatch.setattr(O, "group_limited_mask", wrong)
+    _expect_pin_failure(TS.test_group_limited_brute_force)
