@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE FFN layer forward on B200 (tokens/s).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gshard] [--impl ours|reference]
+
+One step = one whole forward of the layer (router, gate, selection,
+permutation, expert FFNs, combine) over one batch of T tokens, inputs resident
+in HBM.  The timed loop issues the four step entry points of the C ABI
+(moe_route, moe_permute, moe_expert_ffn, moe_combine: the same launches as
+moe_forward) with CUDA events between them; L2 is flushed (256 MB memset,
+untimed) before every step.  `e2e` times moe_forward through the public
+layer object with the host->device copy of x and the device->host copy of y
+inside the timed region.  With N > 1 (torchrun), every rank runs its own
+replica on its own tokens (no collective in the forward: weak scaling); the
+time is the maximum over ranks.
+
+`--impl reference` times the CPU oracle (the only reference this layer has)
+on a bounded sample of the same workload, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mixture_experts_layer_63_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/s on 1 B200; grouped-GEMM % bf16 peak; permute GB/s"
+DEFAULT_WORKLOAD = "gshard"
+
+# dram bytes (read + write) per launch, from ncu captures summarised under
+# profiles/, with the sha256 (first 16 hex digits) of the kernel source they
+# were taken at; a value is reported only while the source is unchanged.
+NCU_TRAFFIC: dict[str, dict] = {}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _describe(w) -> str:
+    s = (f"{w.name}: T={w.T} d_model={w.d_model} E={w.E}+{w.S}shared k={w.k} "
+         f"{'SwiGLU' if w.act == 'swiglu' else 'ReLU'} d_ff={w.d_ff} {w.dtype}")
+    if w.capacity_factor > 0:
+        s += f" capacity_factor={w.capacity_factor}"
+    if w.keep_den > 0:
+        s += f" keep={w.keep_num}/{w.keep_den}"
+    if w.mode == "ec":
+        s += f" expert-choice C={w.ec_capacity}"
+    if w.n_groups > 0:
+        s += f" groups={w.topk_groups}of{w.n_groups}"
+    if w.renormalize:
+        s += " renormalized"
+    if w.zipf_s > 0:
+        s += f" zipf_bias={w.zipf_s}"
+    return s
+
+
+def _src_hash(name: str) -> str:
+    p = os.path.join(ROOT, "mixture_experts_layer_63_b200", "csrc", name)
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def launches_per_step(w) -> int:
+    """Kernels libmoe launches for one forward of this workload."""
+    n = 2                                     # router (GEMM or fp32) + gate
+    if w.mode == "ec":
+        n += 3                                # transpose, expert-choice select, gather
+    else:
+        n += 4                                # histogram, scan, rank/scatter, gather
+        if w.capacity_factor <= 0 and w.keep_den > 0:
+            n += 1                            # per-expert affinity select
+    n += 2                                    # up- and down-projection GEMMs
+    n += 1                                    # combine
+    return n
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", sel],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+class _DeviceExperts:
+    def __init__(self, t):
+        self.t = t
+
+    def __getitem__(self, e):
+        if self.t is None:
+            return None
+        v = self.t[int(e)].detach().contiguous().cpu()
+        return v.view(torch.int16).numpy().view(np.uint16) if v.dtype == torch.bfloat16 else v.numpy()
+
+
+def _np_in(t):
+    v = t.detach().contiguous().cpu()
+    return v.view(torch.int16).numpy().view(np.uint16) if v.dtype == torch.bfloat16 else v.numpy()
+
+
+class OracleTimer:
+    """The CPU oracle on one workload: full routing of all T tokens, then the
+    expert FFNs and combine of a sample of n tokens; tokens/s is extrapolated
+    as T / (t_route + t_ffn * T / n)."""
+
+    def __init__(self, w, seed: int, device: str):
+        from oracle import moe_oracle as O
+        self.O, self.w = O, w
+        inp = make_inputs(w, seed=seed, device=device, grid=False)
+        self.x = _np_in(inp.x)
+        self.w_router = _np_in(inp.w_router)
+        self.bias = None if inp.bias is None else _np_in(inp.bias)
+        # expert weights widened per use, like the oracle's own tests do
+        self.w1 = _DeviceExperts(inp.w1)
+        self.w2 = _DeviceExperts(inp.w2)
+        self.w3 = _DeviceExperts(inp.w3)
+        cap = O.capacity_from_factor(w.T, w.E, w.k, w.capacity_factor) if w.mode == "tc" else 0
+        self.cfg = O.OracleConfig(E=w.E, S=w.S, k=w.k, act=w.act, mode=w.mode, capacity=cap,
+                                  keep_num=w.keep_num, keep_den=w.keep_den,
+                                  ec_capacity=w.ec_capacity if w.mode == "ec" else 0,
+                                  n_groups=w.n_groups, topk_groups=w.topk_groups,
+                                  renormalize=w.renormalize)
+
+    def step(self, n: int, rng) -> tuple[float, float, float]:
+        O = self.O
+        t0 = time.perf_counter()
+        logits = O.router_logits(self.x, self.w_router, self.bias)
+        _, _, _, disp = O.route(self.cfg, logits)
+        t1 = time.perf_counter()
+        toks = np.sort(rng.choice(self.w.T, size=min(n, self.w.T), replace=False))
+        O.combine_tokens(self.cfg, self.x, self.w1, self.w2, self.w3, disp, toks)
+        t2 = time.perf_counter()
+        t_route, t_ffn = t1 - t0, t2 - t1
+        est = t_route + t_ffn * self.w.T / len(toks)
+        return self.w.T / est, t_route, t_ffn
+
+    def calibrate(self, budget_s: float) -> int:
+        """Largest power-of-two sample whose FFN part stays near budget_s."""
+        rng = np.random.default_rng(0)
+        n = 32
+        while True:
+            _, tr, tf = self.step(n, rng)
+            if tf >= budget_s / 2 or n >= self.w.T:
+                return n
+            n = min(self.w.T, n * 2)
+
+
+def cpu_baseline(w, seed: int, device: str, budget_s: float = 12.0) -> dict:
+    ot = OracleTimer(w, seed, device)
+    n = ot.calibrate(budget_s)
+    rng = np.random.default_rng(1)
+    v, tr, tf = ot.step(n, rng)
+    return {"value": v, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"routing of all {w.T} tokens ({tr:.2f} s) + expert FFNs and combine of "
+                      f"{min(n, w.T)} sampled tokens ({tf:.2f} s), extrapolated to {w.T} tokens"}
+
+
+def run_reference(args, w) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    ot = OracleTimer(w, args.seed, dev)
+    n = ot.calibrate(3.0)
+    rng = np.random.default_rng(2)
+    for _ in range(args.warmup):
+        ot.step(n, rng)
+    vals, t0 = [], time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(ot.step(n, rng)[0])
+    elapsed = time.perf_counter() - t0
+    v = float(statistics.mean(vals))
+    sample = (f"per step: routing of all {w.T} tokens + expert FFNs/combine of {n} sampled "
+              f"tokens, extrapolated to {w.T} tokens")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * w.T / v, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": _describe(w), "parallelism": "cpu oracle, rank 0 only"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": elapsed,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, w) -> None:
+    from mixture_experts_layer_63_b200 import api
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    # replicas: same weights on every rank, each rank its own tokens
+    inp = make_inputs(w, seed=args.seed, device="cuda", grid=False)
+    if world > 1:
+        g = torch.Generator(device="cuda")
+        g.manual_seed(args.seed * 1000 + rank + 1)
+        inp.x = torch.randn(w.T, w.d_model, generator=g, device="cuda").to(inp.x.dtype)
+    cfg = api.config_from_workload(w)
+    sizes = api.query_sizes(cfg)
+    B = api.step_buffers(cfg)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        api.moe_route(cfg, inp.x, inp.w_router, inp.bias, B.logits, B.probs, B.topk_idx,
+                      B.topk_gate, B.ws)
+        if ev:
+            ev[1].record(stream)
+        api.moe_permute(cfg, inp.x, B.topk_idx, B.topk_gate, B.probs, B.counts, B.offsets,
+                        B.tok_rows, B.row_token, B.row_gate, B.x_perm, B.n_dropped, B.ws)
+        if ev:
+            ev[2].record(stream)
+        api.moe_expert_ffn(cfg, inp.x, B.x_perm, B.offsets, B.row_gate, inp.w1, inp.w3, inp.w2,
+                           B.h, B.y_rows, B.ws)
+        if ev:
+            ev[3].record(stream)
+        api.moe_combine(cfg, B.y_rows, B.tok_rows, B.y)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    api.moe_check_device_errors(B.ws)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    api.moe_check_device_errors(B.ws)
+
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
+                    for i in range(args.steps)])          # ms: route, permute, ffn, combine
+    total_ms = float(per.sum())
+    t_max = torch.tensor([total_ms], device="cuda")
+    if dist:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    total_ms = float(t_max.item())
+    ms_step = total_ms / args.steps
+    value = world * w.T * args.steps / (total_ms / 1e3)
+
+    # algorithmic work of this batch
+    R = int(B.offsets[w.E].item())
+    es = 4 if w.dtype == "f32" else 2
+    rows = R + w.S * w.T
+    nmat = 3 if w.act == "swiglu" else 2
+    gemm_flops = 2.0 * rows * w.d_model * w.d_ff * nmat
+    permute_bytes = (w.T * w.d_model + R * w.d_model) * es
+    combine_bytes = (rows * w.d_model + w.T * w.d_model) * es
+    route_bytes = (w.T * w.d_model + w.E * w.d_model) * es + 2 * w.T * w.E * 4
+    mean = per.mean(axis=0)                                # ms per call
+    hbm, tfl, tfl_sus, peak_src = _peaks()
+    gemm_tflops = gemm_flops / (mean[2] * 1e-3) / 1e12
+    h = _src_hash("gemm_sm100.cu")
+    tr = NCU_TRAFFIC.get(w.name)
+    traffic = tr["bytes"] if tr and tr.get("src") == h else None
+
+    # end to end through the public layer object, host buffers
+    layer = api.MoELayer(cfg, inp.w_router, inp.w1, inp.w2, inp.w3, inp.bias)
+    x_host = inp.x.cpu().pin_memory()
+    y_host = torch.empty_like(x_host).pin_memory()
+    x_dev = torch.empty_like(inp.x)
+    y_dev = torch.empty_like(inp.x)
+    for _ in range(args.warmup):
+        flush.zero_()
+        x_dev.copy_(x_host, non_blocking=True)
+        layer(x_dev, out=y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        layer(x_dev, out=y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    api.moe_check_device_errors(layer.ws)
+    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in e2e_ev)], device="cuda")
+    if dist:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_value = world * w.T * args.steps / (float(e2e_ms.item()) / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args.seed, "cuda")
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32" if w.dtype == "f32" else "bf16",
+            "data": "synthetic: x ~ N(0,1), expert weights ~ N(0,1/fan_in), random init, seeded",
+            "config": {"workload": _describe(w), "T": w.T, "d_model": w.d_model, "E": w.E,
+                       "S": w.S, "k": w.k, "d_ff": w.d_ff,
+                       "parallelism": f"replicas x{world} (no collective in the forward)",
+                       "l2": "flushed before every step (256 MB memset, untimed)"},
+            "roofline": {"bound": "tensor", "kernel": "grouped GEMM (up + down projections)",
+                         "achieved": gemm_tflops, "peak": tfl, "unit": "TFLOP/s",
+                         "frac": gemm_tflops / tfl, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 burst", "algorithmic_flops": gemm_flops,
+                         "frac_of_sustained": gemm_tflops / tfl_sus if tfl_sus else None},
+            "steps_us": {"route": mean[0] * 1e3, "permute": mean[1] * 1e3,
+                         "expert_ffn": mean[2] * 1e3, "combine": mean[3] * 1e3},
+            "bandwidth_gbs": {"route": route_bytes / (mean[0] * 1e-3) / 1e9,
+                              "permute": permute_bytes / (mean[1] * 1e-3) / 1e9,
+                              "combine": combine_bytes / (mean[3] * 1e-3) / 1e9,
+                              "hbm_peak": hbm},
+            "rows": {"routed_kept": R, "shared": w.S * w.T, "capacity_rows": sizes.rows_cap},
+            "e2e": {"value": e2e_value, "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
+                    "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
+            "gpu_launches": launches_per_step(w) * args.steps,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,207 @@
+/*
+ * moe.h - C ABI of libmoe.so: the forward pass of a sparse Mixture-of-Experts
+ * FFN layer on one NVIDIA B200 (sm_100a).
+ *
+ * The layer, in five steps (all arithmetic runs in this library's CUDA
+ * kernels):
+ *   1. router logits  l = x . W_r^T (+ b)
+ *        - "大语言模型并行策略（七）：专家并行", section "Mixture of Experts (MoE)":
+ *          the router is an FFN plus a softmax layer (read: one bias-free
+ *          linear layer over the routed experts; b is an optional fixed bias).
+ *   2. softmax gating  p_i = exp(g_i) / sum_j exp(g_j)
+ *        - "MoE技术演进", "Adaptive Mixtures of Local Experts", gating equation.
+ *   3. selection: token-choice top-k (lower expert index wins ties), optional
+ *      group-limited routing, expert capacity with overflow dropped to the
+ *      residual, per-expert affinity-based token dropping, shared experts, or
+ *      expert choice (each expert takes its top-C tokens)
+ *        - "MoE技术演进": selector; GShard section 1 (top-2, capacity C = O(N/E));
+ *          DeepSeek-V2 section 3 (device-limited routing) and section 5
+ *          (token dropping); DeepSeekMoE section 2 (shared expert isolation).
+ *        - LocMoE+ article (机器之心): token-choice vs expert-choice routers.
+ *   4. permutation of the kept (token, expert) pairs into expert-contiguous rows
+ *        - the single-GPU counterpart of the count-then-fill all-to-all buffers,
+ *          "大语言模型并行策略（七）：专家并行", section "MoE 中的 all-to-all 通信".
+ *   5. expert FFNs  w_o . ReLU(w_i . x)  (GShard section 3)  or SwiGLU
+ *      w_2 . (SiLU(w_1 . x) * (w_3 . x)) with 3 * d_model * d_moe parameters
+ *      ("大语言模型并行策略（七）", parameter-count notes), then the
+ *      gate-weighted combine  y_t = sum_e G_{t,e} FFN_e(x_t) + sum_s FFN_s(x_t)
+ *      (GShard section 3; DeepSeekMoE section 2).  The residual "+ u" of the
+ *      DeepSeekMoE equations is left to the caller.
+ *
+ * Conventions that hold for every entry point:
+ *   - Ownership: the caller owns every buffer.  The library allocates no
+ *     device memory on any path; scratch lives in the caller's workspace
+ *     (moe_query_sizes gives its size).  Every tensor pointer is a DEVICE
+ *     pointer on the current CUDA device; the structs are host memory.
+ *   - Layout: row-major.  x [T, d]; w_router [E, d]; w1, w3 [E+S, f, d];
+ *     w2 [E+S, d, f] (each output neuron's weights contiguous along its input
+ *     dimension); experts 0..E-1 are routed, E..E+S-1 shared.  Element type
+ *     fp32 (MOE_F32) or bf16 (MOE_BF16) for x, weights, x_perm, h, y_rows, y.
+ *     Router logits, probabilities and gates are always fp32; indices int32.
+ *   - Alignment: tensor pointers 16-byte aligned, the workspace 256-byte
+ *     aligned.  Limits of this build (else MOE_ERR_UNSUPPORTED): E <= 256,
+ *     S <= 8, k <= 8, n_groups <= 32, topk_groups <= 8, T*k and E*C below
+ *     2^31; bf16: d and f multiples of 64; fp32: d a multiple of 4.
+ *   - Streams: every call is asynchronous on `stream` (a cudaStream_t) and
+ *     never synchronises with the host, except moe_check_device_errors.
+ *   - Errors: arguments are validated on the host before any launch; nothing
+ *     is launched when a call returns an error.  Launch failures return
+ *     MOE_ERR_CUDA.  Kernels never trap: a device-side wait that exceeds its
+ *     time limit sets a bit in the error word at the start of the workspace
+ *     and the kernel returns; moe_check_device_errors reads it.
+ *   - Reentrancy: calls may run concurrently on different streams with
+ *     different workspaces.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* same type as cudaStream_t */
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size or option               */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid layer, but outside this build's limits   */
+  MOE_ERR_WORKSPACE = 3,    /* workspace smaller than moe_query_sizes says    */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed    */
+  MOE_ERR_DEVICE_CHECK = 5, /* a kernel reported a bad index in its checks    */
+  MOE_ERR_TIMEOUT = 6       /* a kernel's bounded wait ran out                */
+} moe_status;
+
+typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+typedef enum moe_act { MOE_ACT_RELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
+typedef enum moe_mode { MOE_TOKEN_CHOICE = 0, MOE_EXPERT_CHOICE = 1 } moe_mode;
+
+/* The layer.  Capacity, keep-fraction and expert choice are exclusive. */
+typedef struct moe_config {
+  int64_t T;           /* tokens in this call (>= 1)                                */
+  int32_t d_model;     /* d                                                         */
+  int32_t E;           /* routed experts (>= 1)                                     */
+  int32_t S;           /* shared experts, gate 1 for every token (>= 0)             */
+  int32_t k;           /* experts per token, token choice (1 <= k <= E)             */
+  int32_t d_ff;        /* expert hidden size f (d_ff, or d_moe for SwiGLU)          */
+  int32_t capacity;    /* token choice: max rows per routed expert; <= 0 unlimited  */
+  int32_t keep_num;    /* token choice: expert e keeps ceil(n_e*num/den) of its n_e */
+  int32_t keep_den;    /*   assignments by affinity; den = 0: keep all              */
+  int32_t ec_capacity; /* expert choice: tokens per expert C (1 <= C <= T)          */
+  int32_t n_groups;    /* group-limited routing: E/n_groups contiguous experts per  */
+  int32_t topk_groups; /*   group, keep topk_groups groups per token; 0,0 = off     */
+  int32_t renormalize; /* 1: gate = p / (sum of the selected p)                     */
+  int32_t act;         /* moe_act                                                   */
+  int32_t mode;        /* moe_mode                                                  */
+  int32_t dtype;       /* moe_dtype                                                 */
+} moe_config;
+
+/* Buffer sizes of one configuration. */
+typedef struct moe_sizes {
+  int64_t rows_cap;        /* routed rows, worst case: T*k (token choice), E*C (expert choice) */
+  int64_t rows_total;      /* rows of h and y_rows: rows_cap + S*T                              */
+  int64_t tok_rows_len;    /* entries of tok_rows: T*k (token choice) or E*T (expert choice)     */
+  size_t step_workspace;   /* bytes of workspace the step entry points need                     */
+  size_t workspace;        /* bytes of workspace moe_forward needs (>= step_workspace)          */
+} moe_sizes;
+
+/* Sizes of every buffer for `cfg`.  Validates cfg: returns MOE_ERR_INVALID_ARG
+ * or MOE_ERR_UNSUPPORTED exactly when the compute entry points would. */
+MOE_API moe_status moe_query_sizes(const moe_config *cfg, moe_sizes *out);
+
+/* Steps 1-3a: router logits, softmax, token-choice top-k.
+ *   x [T, d], w_router [E, d] (cfg dtype); bias [E] fp32 or NULL.
+ *   out: logits [T, E], probs [T, E] fp32;
+ *        topk_idx [T, k] int32 in rank order, topk_gate [T, k] fp32
+ *        (both ignored and may be NULL in expert-choice mode).
+ *   Top-k keys are the fp32 logits: strictly larger first, lower expert index
+ *   on ties; with group limits only the topk_groups groups with the largest
+ *   maximum logit (lower group on ties) compete.  p is computed in a fixed
+ *   fp32 recipe (own exp, sequential ascending-expert sum, IEEE division) so
+ *   that it is reproducible bit for bit.
+ *   ws: workspace of at least step_workspace bytes. */
+MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const void *w_router, const float *bias,
+                     float *logits, float *probs, int32_t *topk_idx, float *topk_gate, void *ws,
+                     size_t ws_bytes, moe_stream_t stream);
+
+/* Steps 2-3a from given fp32 logits [T, E] (the same arithmetic moe_route
+ * applies after its router GEMM).  Outputs as moe_route. */
+MOE_API moe_status moe_gate(const moe_config *cfg, const float *logits, float *probs, int32_t *topk_idx,
+                    float *topk_gate, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Steps 3b-4: capacity / keep-fraction / expert choice, then permutation.
+ *   in : x [T, d]; token choice: topk_idx, topk_gate [T, k] (+ probs [T, E]
+ *        for keep-fraction); expert choice: probs [T, E] (topk_* may be NULL).
+ *   out: counts [E]    assignments per expert before drops (expert choice: C)
+ *        offsets [E+1] exclusive scan of the rows each expert keeps
+ *        tok_rows      token choice [T, k]: row of (t, j), -1 when dropped;
+ *                      expert choice [E, T]: row of (e, t), -1 when not taken
+ *        row_token [rows_cap], row_gate [rows_cap]: token and gate of each row
+ *                      (entries >= offsets[E] are unspecified)
+ *        x_perm [rows_cap, d]: x_perm[r] = x[row_token[r]] byte for byte
+ *        n_dropped [1] token-choice assignments dropped (0 in expert choice)
+ *   Token choice keeps rows of an expert in priority order q = j*T + t; with a
+ *   capacity C the assignment of priority q survives iff fewer than C earlier
+ *   ones went to its expert.  Keep-fraction keeps, per expert, the
+ *   ceil(n_e*num/den) assignments with the largest p[t, e] (lower t on ties).
+ *   Expert choice: expert e takes the C tokens with the largest p[t, e]
+ *   (lower t on ties), in ascending t; rows e*C .. e*C+C-1.
+ *   All integer outputs are deterministic and bit-exact. */
+MOE_API moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *topk_idx,
+                       const float *topk_gate, const float *probs, int32_t *counts, int32_t *offsets,
+                       int32_t *tok_rows, int32_t *row_token, float *row_gate, void *x_perm,
+                       int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Step 5a-5b: the grouped expert FFNs.
+ *   in : x [T, d] (input of the shared experts), x_perm [rows_cap, d],
+ *        offsets [E+1], row_gate [rows_cap], w1, w3 (SwiGLU; NULL for ReLU), w2.
+ *   out: h [rows_total, f]  activations (scratch the caller may read);
+ *        y_rows [rows_total, d]: routed row r = row_gate[r] * FFN_e(x_perm[r]);
+ *        shared expert s, token t at row rows_cap + s*T + t = FFN_{E+s}(x[t]).
+ *   bf16: tcgen05 tensor cores, bf16 operands, fp32 accumulation, h and y_rows
+ *   rounded to bf16.  fp32: CUDA-core fp32 arithmetic. */
+MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x, const void *x_perm,
+                          const int32_t *offsets, const float *row_gate, const void *w1,
+                          const void *w3, const void *w2, void *h, void *y_rows, void *ws,
+                          size_t ws_bytes, moe_stream_t stream);
+
+/* Step 5c: y[t] = sum of t's routed rows (token choice: in k-rank order;
+ * expert choice: ascending expert) + its shared rows, fp32 accumulation,
+ * rounded once to the layer dtype.  A token with no kept row and no shared
+ * expert gets 0. */
+MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_rows, const int32_t *tok_rows, void *y,
+                       moe_stream_t stream);
+
+/* Steps 1-5 in one call; intermediates live in the workspace (at least
+ * `workspace` bytes).  counts_out [E] (optional, may be NULL) receives the
+ * per-expert assignment counts.  Equivalent to moe_route, moe_permute,
+ * moe_expert_ffn and moe_combine in sequence. */
+MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const void *w_router,
+                       const float *bias, const void *w1, const void *w3, const void *w2, void *y,
+                       int32_t *counts_out, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Waits for `stream`, then reads and clears the workspace's device error
+ * word.  Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_CHECK; *flags (if
+ * not NULL) receives the raw bits.  This is the only call that blocks. */
+MOE_API moe_status moe_check_device_errors(void *ws, size_t ws_bytes, moe_stream_t stream, uint32_t *flags);
+
+/* Fill `ws` with the bytes the library expects in a fresh workspace (the
+ * error word cleared).  Call once after allocating a workspace. */
+MOE_API moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Static text for a status code. */
+MOE_API const char *moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -1,0 +1,288 @@
+"""Thin ctypes binding of libmoe.so (include/moe.h).
+
+Argument marshalling only: torch tensors become device pointers, the
+current torch CUDA stream becomes the call's stream, status codes become
+exceptions.  Every step of the layer runs in the library's CUDA kernels.
+There is no CPU fallback: a missing library, a CPU tensor or a machine
+without CUDA raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+from .inputs import Workload
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = 0, 1, 2, 3
+MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT = 4, 5, 6
+MOE_F32, MOE_BF16 = 0, 1
+MOE_ACT_RELU, MOE_ACT_SWIGLU = 0, 1
+MOE_TOKEN_CHOICE, MOE_EXPERT_CHOICE = 0, 1
+
+EXPORTS = ("moe_query_sizes", "moe_route", "moe_gate", "moe_permute", "moe_expert_ffn",
+           "moe_combine", "moe_forward", "moe_check_device_errors", "moe_workspace_init",
+           "moe_status_string")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d_model", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("S", ctypes.c_int32), ("k", ctypes.c_int32), ("d_ff", ctypes.c_int32),
+                ("capacity", ctypes.c_int32), ("keep_num", ctypes.c_int32),
+                ("keep_den", ctypes.c_int32), ("ec_capacity", ctypes.c_int32),
+                ("n_groups", ctypes.c_int32), ("topk_groups", ctypes.c_int32),
+                ("renormalize", ctypes.c_int32), ("act", ctypes.c_int32),
+                ("mode", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+class MoeSizes(ctypes.Structure):
+    _fields_ = [("rows_cap", ctypes.c_int64), ("rows_total", ctypes.c_int64),
+                ("tok_rows_len", ctypes.c_int64), ("step_workspace", ctypes.c_size_t),
+                ("workspace", ctypes.c_size_t)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m mixture_experts_layer_63_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, cfgp = ctypes.c_void_p, ctypes.POINTER(MoeConfig)
+        sz = ctypes.c_size_t
+        sig = {
+            "moe_query_sizes": [cfgp, ctypes.POINTER(MoeSizes)],
+            "moe_route": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_gate": [cfgp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_permute": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_expert_ffn": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_combine": [cfgp, vp, vp, vp, vp],
+            "moe_forward": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_check_device_errors": [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)],
+            "moe_workspace_init": [vp, sz, vp],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != MOE_OK:
+        raise MoeError(fn, status)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmoe takes CUDA tensors only (no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError("libmoe takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream: torch.cuda.Stream | None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ws(ws: torch.Tensor):
+    return _ptr(ws), ws.numel() * ws.element_size()
+
+
+# ---------------------------------------------------------------------------
+# configuration
+# ---------------------------------------------------------------------------
+
+def capacity_for(T: int, E: int, k: int, capacity_factor: float) -> int:
+    """Expert capacity ceil(cf * k * T / E) (GShard's C = O(N/E)); 0 = unlimited."""
+    if capacity_factor <= 0:
+        return 0
+    return int(math.ceil(capacity_factor * k * T / E))
+
+
+def config_from_workload(w: Workload, T: int | None = None) -> MoeConfig:
+    T = w.T if T is None else T
+    c = MoeConfig()
+    c.T, c.d_model, c.E, c.S, c.k, c.d_ff = T, w.d_model, w.E, w.S, w.k, w.d_ff
+    c.capacity = capacity_for(T, w.E, w.k, w.capacity_factor) if w.mode == "tc" else 0
+    c.keep_num, c.keep_den = w.keep_num, w.keep_den
+    if T != w.T:
+        w = w.with_tokens(T)
+    c.ec_capacity = w.ec_capacity if w.mode == "ec" else 0
+    c.n_groups, c.topk_groups = w.n_groups, w.topk_groups
+    c.renormalize = int(w.renormalize)
+    c.act = MOE_ACT_SWIGLU if w.act == "swiglu" else MOE_ACT_RELU
+    c.mode = MOE_EXPERT_CHOICE if w.mode == "ec" else MOE_TOKEN_CHOICE
+    c.dtype = MOE_F32 if w.dtype == "f32" else MOE_BF16
+    return c
+
+
+@dataclass
+class Sizes:
+    rows_cap: int
+    rows_total: int
+    tok_rows_len: int
+    step_workspace: int
+    workspace: int
+
+
+def query_sizes(cfg: MoeConfig) -> Sizes:
+    out = MoeSizes()
+    _check("moe_query_sizes", lib().moe_query_sizes(ctypes.byref(cfg), ctypes.byref(out)))
+    return Sizes(out.rows_cap, out.rows_total, out.tok_rows_len, out.step_workspace, out.workspace)
+
+
+def new_workspace(cfg: MoeConfig, device="cuda", step_only: bool = False) -> torch.Tensor:
+    """A zeroed workspace tensor (uint8) of the size the configuration needs."""
+    s = query_sizes(cfg)
+    n = s.step_workspace if step_only else s.workspace
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ---------------------------------------------------------------------------
+
+def moe_route(cfg, x, w_router, bias, logits, probs, topk_idx, topk_gate, ws, stream=None):
+    wp, wn = _ws(ws)
+    _check("moe_route", lib().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias),
+                                        _ptr(logits), _ptr(probs), _ptr(topk_idx), _ptr(topk_gate),
+                                        wp, wn, _stream(stream)))
+
+
+def moe_gate(cfg, logits, probs, topk_idx, topk_gate, ws, stream=None):
+    wp, wn = _ws(ws)
+    _check("moe_gate", lib().moe_gate(ctypes.byref(cfg), _ptr(logits), _ptr(probs), _ptr(topk_idx),
+                                      _ptr(topk_gate), wp, wn, _stream(stream)))
+
+
+def moe_permute(cfg, x, topk_idx, topk_gate, probs, counts, offsets, tok_rows, row_token, row_gate,
+                x_perm, n_dropped, ws, stream=None):
+    wp, wn = _ws(ws)
+    _check("moe_permute", lib().moe_permute(
+        ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(topk_gate), _ptr(probs), _ptr(counts),
+        _ptr(offsets), _ptr(tok_rows), _ptr(row_token), _ptr(row_gate), _ptr(x_perm),
+        _ptr(n_dropped), wp, wn, _stream(stream)))
+
+
+def moe_expert_ffn(cfg, x, x_perm, offsets, row_gate, w1, w3, w2, h, y_rows, ws, stream=None):
+    wp, wn = _ws(ws)
+    _check("moe_expert_ffn", lib().moe_expert_ffn(
+        ctypes.byref(cfg), _ptr(x), _ptr(x_perm), _ptr(offsets), _ptr(row_gate), _ptr(w1), _ptr(w3),
+        _ptr(w2), _ptr(h), _ptr(y_rows), wp, wn, _stream(stream)))
+
+
+def moe_combine(cfg, y_rows, tok_rows, y, stream=None):
+    _check("moe_combine", lib().moe_combine(ctypes.byref(cfg), _ptr(y_rows), _ptr(tok_rows), _ptr(y),
+                                            _stream(stream)))
+
+
+def moe_forward(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, stream=None):
+    wp, wn = _ws(ws)
+    _check("moe_forward", lib().moe_forward(
+        ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y),
+        _ptr(counts_out), wp, wn, _stream(stream)))
+
+
+def moe_check_device_errors(ws, stream=None) -> int:
+    """Blocks on the stream; returns the raw error bits and raises if any is set."""
+    wp, wn = _ws(ws)
+    flags = ctypes.c_uint32(0)
+    st = lib().moe_check_device_errors(wp, wn, _stream(stream), ctypes.byref(flags))
+    _check("moe_check_device_errors", st)
+    return flags.value
+
+
+def moe_workspace_init(ws, stream=None):
+    wp, wn = _ws(ws)
+    _check("moe_workspace_init", lib().moe_workspace_init(wp, wn, _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# convenience: buffers of the step API, and a layer object
+# ---------------------------------------------------------------------------
+
+@dataclass
+class StepBuffers:
+    logits: torch.Tensor
+    probs: torch.Tensor
+    topk_idx: torch.Tensor | None
+    topk_gate: torch.Tensor | None
+    counts: torch.Tensor
+    offsets: torch.Tensor
+    tok_rows: torch.Tensor
+    row_token: torch.Tensor
+    row_gate: torch.Tensor
+    x_perm: torch.Tensor
+    n_dropped: torch.Tensor
+    h: torch.Tensor
+    y_rows: torch.Tensor
+    y: torch.Tensor
+    ws: torch.Tensor
+
+
+def step_buffers(cfg: MoeConfig, device="cuda") -> StepBuffers:
+    s = query_sizes(cfg)
+    dt = torch.float32 if cfg.dtype == MOE_F32 else torch.bfloat16
+    T, E, d, f = cfg.T, cfg.E, cfg.d_model, cfg.d_ff
+    tc = cfg.mode == MOE_TOKEN_CHOICE
+    i32, f32 = torch.int32, torch.float32
+    return StepBuffers(
+        logits=torch.empty(T, E, dtype=f32, device=device),
+        probs=torch.empty(T, E, dtype=f32, device=device),
+        topk_idx=torch.empty(T, cfg.k, dtype=i32, device=device) if tc else None,
+        topk_gate=torch.empty(T, cfg.k, dtype=f32, device=device) if tc else None,
+        counts=torch.empty(E, dtype=i32, device=device),
+        offsets=torch.empty(E + 1, dtype=i32, device=device),
+        tok_rows=torch.empty(s.tok_rows_len, dtype=i32, device=device),
+        row_token=torch.empty(max(s.rows_cap, 1), dtype=i32, device=device),
+        row_gate=torch.empty(max(s.rows_cap, 1), dtype=f32, device=device),
+        x_perm=torch.empty(max(s.rows_cap, 1), d, dtype=dt, device=device),
+        n_dropped=torch.empty(1, dtype=i32, device=device),
+        h=torch.empty(s.rows_total, f, dtype=dt, device=device),
+        y_rows=torch.empty(s.rows_total, d, dtype=dt, device=device),
+        y=torch.empty(T, d, dtype=dt, device=device),
+        ws=new_workspace(cfg, device, step_only=True),
+    )
+
+
+class MoELayer:
+    """The layer's weights plus a workspace; ``layer(x)`` runs moe_forward."""
+
+    def __init__(self, cfg: MoeConfig, w_router, w1, w2, w3=None, bias=None):
+        self.cfg = cfg
+        self.w_router, self.w1, self.w2, self.w3, self.bias = w_router, w1, w2, w3, bias
+        self.ws = new_workspace(cfg, w1.device)
+        self.counts = torch.empty(cfg.E, dtype=torch.int32, device=w1.device)
+
+    def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        y = out if out is not None else torch.empty_like(x)
+        moe_forward(self.cfg, x, self.w_router, self.bias, self.w1, self.w3, self.w2, y,
+                    self.counts, self.ws, stream)
+        return y

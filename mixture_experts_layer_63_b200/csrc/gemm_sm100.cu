@@ -1,0 +1,596 @@
+// Grouped GEMM on the 5th-generation tensor cores (sm_100a): TMA-fed,
+// tcgen05.mma with fp32 accumulators in TMEM, fused epilogues.
+//
+// Serves three contractions of the layer:
+//   * the bf16 router  l = x . W_r^T (+ b)         one group, fp32 out
+//   * the expert up-projection, per expert segment of x_perm (and x for the
+//     shared experts): ReLU(x W_i^T) (GShard section 3 of "MoE技术演进") or
+//     SiLU(x W_1^T) * (x W_3^T) (SwiGLU, 3*d_model*d_moe parameters per
+//     "大语言模型并行策略（七）：专家并行"), bf16 out
+//   * the down-projection with the gate G_{t,e} of the combine equation
+//     y_s = sum_e G_{s,e} FFN_e(x_s) folded into its epilogue, bf16 out.
+// The "IO-aware" expert kernels of the Multi-Head LatentMoE summary batch
+// token-to-expert traffic with the expert compute; here the batching is the
+// expert-contiguous row layout and the activation / gate scaling never make
+// a round trip through HBM.
+//
+// Kernel structure (one CTA per SM, persistent, 256 threads):
+//   warp 0      TMA producer: A tile 128 x 64 and B tile BN x 64 (bf16,
+//               128-byte swizzle) per k-block into a 4-stage smem ring
+//   warp 1      MMA issuer: 4 x tcgen05.mma (M=128, N=BN, K=16) per k-block,
+//               tcgen05.commit frees the smem stage; a second commit hands
+//               a finished accumulator to the epilogue
+//   warp 2      TMEM allocation (512 columns = two 256-column accumulators)
+//   warps 4-7   epilogue: tcgen05.ld of its 32 rows, activation / gate /
+//               bias, bf16 pack, masked 16-byte stores (rows beyond the
+//               expert's segment are never written)
+// Tiles are ordered group by group, N-tile outer and M-tile inner, so CTAs
+// working at the same time share one expert's weight slice in L2.  Segment
+// sizes are read from device memory inside the kernel: no host sync.
+// Every wait is bounded; on expiry the kernel sets the timeout bit of the
+// error word, drains its own copies and MMAs (bounded), frees TMEM and
+// returns.
+#include <cuda.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "device_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;             // rows per tile (MMA M)
+constexpr int BK = 64;              // bf16 elements per 128-byte swizzled row
+constexpr int kUmmaK = 16;          // K per tcgen05.mma kind::f16
+constexpr int kStages = 4;
+constexpr int kThreads = 256;
+constexpr int kAccCols = 256;       // TMEM columns per accumulator buffer
+constexpr int kTmemCols = 512;
+constexpr int kMaxGroups = 320;
+constexpr uint32_t kABytes = BM * BK * 2;   // 16 KB
+
+struct Params {
+  int epi;
+  int K, N;
+  int bn;           // MMA N (B tile rows)
+  int bnh;          // output columns per tile (128 for SwiGLU, bn otherwise)
+  int nt;           // N-tiles per group
+  int n_routed, n_static, G;
+  int64_t rows_static, a_static_base, a_static_stride, out_static_base;
+  int64_t a_rows;
+  const int32_t *offsets;
+  void *out;
+  const float *row_gate;
+  const float *bias;
+  uint32_t *err;
+};
+
+// ------------------------------- PTX wrappers --------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of parity `parity` to complete.  Returns false
+// when the CTA is aborting or the time limit passed (then it raises the
+// timeout bit and starts the abort).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          uint32_t *err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        raise_error(err, kErrTimeout);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Wait used while draining after an abort: bounded, no further side effects.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0,
+                                            int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the
+// 128-byte swizzle: 8-row core-matrix groups 1024 bytes apart (SBO), leading
+// byte offset unused for this layout, descriptor version 1, swizzle mode 2.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, both
+// K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------- tile schedule -------------------------------
+struct Tile {
+  int g, m, n;
+};
+
+__device__ __forceinline__ Tile decode_tile(int tile, const int *prefix, int G, int nt) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {                      // largest g with prefix[g] <= tile
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= tile) lo = mid;
+    else hi = mid - 1;
+  }
+  Tile t;
+  t.g = lo;
+  const int local = tile - prefix[lo];
+  const int mt = (prefix[lo + 1] - prefix[lo]) / nt;
+  t.n = local / mt;
+  t.m = local - t.n * mt;
+  return t;
+}
+
+// --------------------------------- epilogues ---------------------------------
+__device__ __forceinline__ void store_bf16x32(void *dst, const float (&v)[32]) {
+  uint4 *p = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    p[q] = w;
+  }
+}
+
+// --------------------------------- the kernel --------------------------------
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                        const __grid_constant__ CUtensorMap map_a_static,
+                        const __grid_constant__ CUtensorMap map_b,
+                        const __grid_constant__ CUtensorMap map_b3, const Params P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ int s_prefix[kMaxGroups + 1];
+  __shared__ int s_off[kMaxGroups];
+  __shared__ int s_rows[kMaxGroups];
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  __shared__ __align__(8) uint64_t accf_bar[2];
+  __shared__ __align__(8) uint64_t acce_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ volatile int s_abort;
+
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~(uintptr_t)1023);
+  const uint32_t b_bytes = (uint32_t)P.bn * BK * 2;
+  const uint32_t stage_bytes = kABytes + b_bytes;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // group table: rows and tile prefix, warp 0
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < P.G; base += 32) {
+      const int g = base + lane;
+      int tiles = 0;
+      if (g < P.G) {
+        int off = 0, rows = 0;
+        if (g < P.n_routed) {
+          off = P.offsets[g];
+          rows = P.offsets[g + 1] - off;
+          if (rows < 0 || off < 0 || (int64_t)off + rows > P.a_rows) {
+            raise_error(P.err, kErrBadIndex);
+            rows = 0;
+            off = 0;
+          }
+        } else {
+          rows = (int)P.rows_static;
+        }
+        s_off[g] = off;
+        s_rows[g] = rows;
+        tiles = ((rows + BM - 1) / BM) * P.nt;
+      }
+      int x = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (g < P.G) s_prefix[g] = carry + x - tiles;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) s_prefix[P.G] = carry;
+  }
+  if (tid == 32) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accf_bar[a], 1);
+      mbar_init(&acce_bar[a], 4 * 32);
+    }
+    mbar_init(&drain_bar, 1);
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (tid == 0) {
+    tma_prefetch_map(&map_a);
+    tma_prefetch_map(&map_b);
+    if (P.n_static > 0) tma_prefetch_map(&map_a_static);
+    if (EPI == kEpiSwiglu) tma_prefetch_map(&map_b3);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = s_tmem_base;
+  const int total = s_prefix[P.G];
+  const int KB = P.K / BK;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0;            // bit s: full_bar[s] armed and maybe in flight
+    uint32_t armed_parity = 0;     // bit s: parity of that phase
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      const bool routed = tl.g < P.n_routed;
+      const int64_t a_row = routed ? (int64_t)s_off[tl.g] + (int64_t)tl.m * BM
+                                   : P.a_static_base + (int64_t)(tl.g - P.n_routed) * P.a_static_stride +
+                                         (int64_t)tl.m * BM;
+      const CUtensorMap *ma = routed ? &map_a : &map_a_static;
+      const int b_row = tl.g * P.N + tl.n * P.bnh;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+        uint8_t *sa = smem + (size_t)stage * stage_bytes;
+        uint8_t *sb = sa + kABytes;
+        mbar_expect_tx(&full_bar[stage], stage_bytes);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        tma_load_2d(sa, ma, &full_bar[stage], kb * BK, (int)a_row);
+        if (EPI == kEpiSwiglu) {
+          tma_load_2d(sb, &map_b, &full_bar[stage], kb * BK, b_row);
+          tma_load_2d(sb + (b_bytes >> 1), &map_b3, &full_bar[stage], kb * BK, b_row);
+        } else {
+          tma_load_2d(sb, &map_b, &full_bar[stage], kb * BK, b_row);
+        }
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok) {
+      // aborting: let the copies already issued land before the CTA exits
+      for (int s = 0; s < kStages; ++s)
+        if (armed & (1u << s)) mbar_wait_drain(&full_bar[s], (armed_parity >> s) & 1u);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------- MMA issuer -------------------------------
+    const uint32_t idesc = idesc_bf16(BM, P.bn);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&full_bar[stage], phase, &s_abort, P.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + (size_t)stage * stage_bytes);
+        const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+        for (int k = 0; k < BK / kUmmaK; ++k) {
+          umma_bf16(d_tmem, sw128_desc(a_addr + k * kUmmaK * 2), sw128_desc(b_addr + k * kUmmaK * 2),
+                    idesc, (kb > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty_bar[stage]);
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      umma_commit(&accf_bar[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    // all MMAs issued by this thread complete before TMEM can be freed
+    umma_commit(&drain_bar);
+    mbar_wait_drain(&drain_bar, 0);
+  } else if (warp >= 4) {
+    // -------------------------------- epilogue --------------------------------
+    const int ew = warp - 4;                     // TMEM lanes 32*ew .. 32*ew+31
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      if (!mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err)) break;
+      tc_fence_after();
+      const bool routed = tl.g < P.n_routed;
+      const int r_in = ew * 32 + lane;
+      const bool valid = tl.m * BM + r_in < s_rows[tl.g];
+      const int64_t out_row = (routed ? (int64_t)s_off[tl.g]
+                                      : P.out_static_base + (int64_t)(tl.g - P.n_routed) * P.rows_static) +
+                              (int64_t)tl.m * BM + r_in;
+      const int col0 = tl.n * P.bnh;
+      const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
+      uint32_t r[32];
+      float v[32];
+      if (EPI == kEpiSwiglu) {
+        __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
+#pragma unroll 1
+        for (int c = 0; c < 128 / 32; ++c) {
+          uint32_t u[32];
+          tmem_ld32(taddr + c * 32, r);
+          tmem_ld32(taddr + 128 + c * 32, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float g = __uint_as_float(r[i]);
+            v[i] = g / (1.0f + __expf(-g)) * __uint_as_float(u[i]);
+          }
+          const int col = col0 + c * 32;
+          if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
+        }
+      } else if (EPI == kEpiRelu || EPI == kEpiScale) {
+        __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
+        float scale = 1.0f;
+        if (EPI == kEpiScale && routed && valid) scale = P.row_gate[out_row];
+#pragma unroll 1
+        for (int c = 0; c < P.bn / 32; ++c) {
+          tmem_ld32(taddr + c * 32, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float a = __uint_as_float(r[i]);
+            v[i] = (EPI == kEpiRelu) ? fmaxf(a, 0.0f) : a * scale;
+          }
+          const int col = col0 + c * 32;
+          if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
+        }
+      } else {  // kEpiStoreF32
+        float *out = reinterpret_cast<float *>(P.out);
+#pragma unroll 1
+        for (int c = 0; c < P.bn / 32; ++c) {
+          tmem_ld32(taddr + c * 32, r);
+          tmem_ld_wait();
+          if (valid) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int col = col0 + c * 32 + i;
+              if (col < P.N) {
+                const float a = __uint_as_float(r[i]);
+                out[out_row * P.N + col] = P.bias ? a + P.bias[col] : a;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acce_bar[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols));
+  }
+}
+
+// ------------------------------- host helpers --------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] (inner contiguous), box [box_outer, 64].
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  if (outer == 0) outer = 1;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int device_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int EPI>
+cudaError_t launch_epi(const GroupedGemm &g, const Params &P, const CUtensorMap &ma,
+                       const CUtensorMap &mas, const CUtensorMap &mb, const CUtensorMap &mb3,
+                       int grid, size_t smem, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  grouped_gemm_kernel<EPI><<<grid, kThreads, smem, s>>>(ma, mas, mb, mb3, P);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
+  Params P{};
+  P.epi = g.epi;
+  P.K = g.K;
+  P.N = g.N;
+  if (g.epi == kEpiSwiglu) {
+    P.bn = 256;
+    P.bnh = 128;
+  } else if (g.epi == kEpiStoreF32) {
+    P.bn = std::max(32, (g.N + 31) / 32 * 32);
+    P.bnh = P.bn;
+  } else {
+    P.bn = 256;
+    P.bnh = 256;
+  }
+  P.nt = (g.N + P.bnh - 1) / P.bnh;
+  P.n_routed = g.n_routed;
+  P.n_static = g.n_static;
+  P.G = g.n_routed + g.n_static;
+  P.rows_static = g.rows_static;
+  P.a_static_base = g.a_static_base;
+  P.a_static_stride = g.a_static_stride;
+  P.out_static_base = g.out_static_base;
+  P.a_rows = g.a_rows;
+  P.offsets = g.offsets;
+  P.out = g.out;
+  P.row_gate = g.row_gate;
+  P.bias = g.bias;
+  P.err = g.err;
+  if (P.G <= 0 || P.G > kMaxGroups || P.bn > 256 || g.K % BK != 0) return cudaErrorInvalidValue;
+
+  CUtensorMap ma, mas, mb, mb3;
+  const uint32_t box_b = (g.epi == kEpiSwiglu) ? 128u : (uint32_t)P.bn;
+  if (!make_map(&ma, g.a, (uint64_t)g.K, (uint64_t)g.a_rows, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&mas, g.a_static ? g.a_static : g.a, (uint64_t)g.K,
+                (uint64_t)(g.a_static ? g.a_static_rows : g.a_rows), BM))
+    return cudaErrorInvalidValue;
+  if (!make_map(&mb, g.b, (uint64_t)g.K, (uint64_t)g.b_rows, box_b)) return cudaErrorInvalidValue;
+  if (!make_map(&mb3, g.b3 ? g.b3 : g.b, (uint64_t)g.K, (uint64_t)g.b_rows, box_b))
+    return cudaErrorInvalidValue;
+
+  // grid: one CTA per SM, fewer when there are fewer tiles
+  const int64_t mt_routed = (g.max_routed_rows + BM - 1) / BM + g.n_routed;
+  const int64_t mt_static = (int64_t)g.n_static * ((g.rows_static + BM - 1) / BM);
+  const int64_t max_tiles = (mt_routed + mt_static) * P.nt;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(device_sms(), max_tiles));
+  // at least 120 KB so that one CTA (and one 512-column TMEM allocation) fits per SM
+  const size_t smem = std::max<size_t>((size_t)kStages * (kABytes + (size_t)P.bn * BK * 2) + 1024,
+                                       (size_t)120 * 1024);
+
+  switch (g.epi) {
+    case kEpiStoreF32: return launch_epi<kEpiStoreF32>(g, P, ma, mas, mb, mb3, grid, smem, s);
+    case kEpiRelu: return launch_epi<kEpiRelu>(g, P, ma, mas, mb, mb3, grid, smem, s);
+    case kEpiSwiglu: return launch_epi<kEpiSwiglu>(g, P, ma, mas, mb, mb3, grid, smem, s);
+    case kEpiScale: return launch_epi<kEpiScale>(g, P, ma, mas, mb, mb3, grid, smem, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,373 @@
+// C ABI of libmoe.so (declared in include/moe.h): argument validation,
+// workspace layout and the launch sequence of each entry point.  All
+// arithmetic of the layer runs in the kernels of the other files.
+#include <algorithm>
+
+#include "device_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+moe_status validate(const moe_config *c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 1 || c->d_model < 1 || c->d_ff < 1 || c->E < 1 || c->S < 0) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->act != MOE_ACT_RELU && c->act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (c->mode != MOE_TOKEN_CHOICE && c->mode != MOE_EXPERT_CHOICE) return MOE_ERR_INVALID_ARG;
+  if (c->renormalize != 0 && c->renormalize != 1) return MOE_ERR_INVALID_ARG;
+  if (c->keep_den < 0 || c->keep_num < 0 || (c->keep_den > 0 && c->keep_num > c->keep_den) ||
+      (c->keep_den == 0 && c->keep_num != 0))
+    return MOE_ERR_INVALID_ARG;
+  if (c->n_groups < 0 || c->topk_groups < 0) return MOE_ERR_INVALID_ARG;
+  if (c->mode == MOE_TOKEN_CHOICE) {
+    if (c->k < 1 || c->k > c->E) return MOE_ERR_INVALID_ARG;
+    if (c->capacity > 0 && c->keep_den > 0) return MOE_ERR_INVALID_ARG;   // exclusive drop rules
+    if (c->n_groups > 0) {
+      if (c->E % c->n_groups != 0 || c->topk_groups < 1 || c->topk_groups > c->n_groups)
+        return MOE_ERR_INVALID_ARG;
+      if ((int64_t)c->topk_groups * (c->E / c->n_groups) < c->k) return MOE_ERR_INVALID_ARG;
+    } else if (c->topk_groups != 0) {
+      return MOE_ERR_INVALID_ARG;
+    }
+    if (c->T * (int64_t)c->k > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  } else {
+    if (c->ec_capacity < 1 || c->ec_capacity > c->T) return MOE_ERR_INVALID_ARG;
+    if (c->n_groups != 0 || c->topk_groups != 0 || c->capacity > 0 || c->keep_den > 0 ||
+        c->renormalize)
+      return MOE_ERR_INVALID_ARG;
+    if ((int64_t)c->E * c->ec_capacity > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  }
+  // limits of this build
+  if (c->E > kMaxExperts || c->S > 8) return MOE_ERR_UNSUPPORTED;
+  if (c->mode == MOE_TOKEN_CHOICE && (c->k > kMaxTopK || c->n_groups > 32 || c->topk_groups > 8))
+    return MOE_ERR_UNSUPPORTED;
+  if (c->T > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
+  if (c->dtype == MOE_BF16) {
+    if (c->d_model % 64 != 0 || c->d_ff % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  } else {
+    if (c->d_model % 4 != 0) return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_OK;
+}
+
+WsLayout make_layout(const moe_config *c) {
+  WsLayout L{};
+  const int64_t T = c->T;
+  const int E = c->E, S = c->S;
+  const bool tc = c->mode == MOE_TOKEN_CHOICE;
+  const int k = tc ? c->k : 0;
+  const size_t es = elem_size(c);
+  L.rows_cap = tc ? T * k : (int64_t)E * c->ec_capacity;
+  L.rows_total = L.rows_cap + (int64_t)S * T;
+  L.tok_rows_len = tc ? T * k : (int64_t)E * T;
+  L.nblk = tc ? (int)((T * k + kAssignBlock - 1) / kAssignBlock) : 0;
+  const bool keepfrac = tc && c->capacity <= 0 && c->keep_den > 0;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L.err = take(256);
+  L.hist = take((size_t)L.nblk * E * 4);
+  L.base = take((size_t)L.nblk * E * 4);
+  L.cnt_off = take((size_t)(E + 1) * 4);
+  L.kept = take((size_t)E * 4);
+  L.sorted_q = take(keepfrac ? (size_t)T * k * 4 : 0);
+  L.probs_t = take(tc ? 0 : (size_t)E * T * 4);
+  L.step_end = o;
+  L.logits = take((size_t)T * E * 4);
+  L.probs = take((size_t)T * E * 4);
+  L.topk_idx = take((size_t)T * k * 4);
+  L.topk_gate = take((size_t)T * k * 4);
+  L.counts = take((size_t)E * 4);
+  L.offsets = take((size_t)(E + 1) * 4);
+  L.n_dropped = take(4);
+  L.tok_rows = take((size_t)L.tok_rows_len * 4);
+  L.row_token = take((size_t)L.rows_cap * 4);
+  L.row_gate = take((size_t)L.rows_cap * 4);
+  L.x_perm = take((size_t)L.rows_cap * c->d_model * es);
+  L.h = take((size_t)L.rows_total * c->d_ff * es);
+  L.y_rows = take((size_t)L.rows_total * c->d_model * es);
+  L.total = o;
+  return L;
+}
+
+static moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+static moe_status check_ws(const WsLayout &L, const void *ws, size_t ws_bytes, size_t need) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE;
+  (void)L;
+  return MOE_OK;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- step bodies, shared by the step entry points and moe_forward ----------
+static cudaError_t run_route(const moe_config *c, const WsLayout &L, char *ws, const void *x,
+                             const void *w_router, const float *bias, float *logits, float *probs,
+                             int32_t *topk_idx, float *topk_gate, cudaStream_t s) {
+  cudaError_t e;
+  if (c->dtype == MOE_F32) {
+    e = launch_router_f32(c, static_cast<const float *>(x), static_cast<const float *>(w_router),
+                          bias, logits, s);
+  } else {
+    GroupedGemm g{};
+    g.epi = kEpiStoreF32;
+    g.K = c->d_model;
+    g.N = c->E;
+    g.a = x;
+    g.a_rows = c->T;
+    g.a_static = x;
+    g.a_static_rows = c->T;
+    g.b = w_router;
+    g.b3 = nullptr;
+    g.b_rows = c->E;
+    g.offsets = nullptr;
+    g.n_routed = 0;
+    g.n_static = 1;
+    g.rows_static = c->T;
+    g.a_static_base = 0;
+    g.a_static_stride = 0;
+    g.out_static_base = 0;
+    g.max_routed_rows = 0;
+    g.out = logits;
+    g.bias = bias;
+    g.err = reinterpret_cast<uint32_t *>(ws + L.err);
+    e = launch_grouped_gemm(g, s);
+  }
+  if (e != cudaSuccess) return e;
+  return launch_gate(c, logits, probs, topk_idx, topk_gate, s);
+}
+
+static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, const void *x,
+                           const void *x_perm, const int32_t *offsets, const float *row_gate,
+                           const void *w1, const void *w3, const void *w2, void *h, void *y_rows,
+                           cudaStream_t s) {
+  uint32_t *err = reinterpret_cast<uint32_t *>(ws + L.err);
+  if (c->dtype == MOE_F32)
+    return launch_ffn_f32(c, L, err, static_cast<const float *>(x),
+                          static_cast<const float *>(x_perm), offsets, row_gate,
+                          static_cast<const float *>(w1), static_cast<const float *>(w3),
+                          static_cast<const float *>(w2), static_cast<float *>(h),
+                          static_cast<float *>(y_rows), s);
+  const bool swiglu = c->act == MOE_ACT_SWIGLU;
+  GroupedGemm up{};
+  up.epi = swiglu ? kEpiSwiglu : kEpiRelu;
+  up.K = c->d_model;
+  up.N = c->d_ff;
+  up.a = x_perm;
+  up.a_rows = L.rows_cap;
+  up.a_static = x;
+  up.a_static_rows = c->T;
+  up.b = w1;
+  up.b3 = swiglu ? w3 : nullptr;
+  up.b_rows = (int64_t)(c->E + c->S) * c->d_ff;
+  up.offsets = offsets;
+  up.n_routed = c->E;
+  up.n_static = c->S;
+  up.rows_static = c->T;
+  up.a_static_base = 0;
+  up.a_static_stride = 0;
+  up.out_static_base = L.rows_cap;
+  up.max_routed_rows = L.rows_cap;
+  up.out = h;
+  up.err = err;
+  cudaError_t e = launch_grouped_gemm(up, s);
+  if (e != cudaSuccess) return e;
+  GroupedGemm dn{};
+  dn.epi = kEpiScale;
+  dn.K = c->d_ff;
+  dn.N = c->d_model;
+  dn.a = h;
+  dn.a_rows = L.rows_total;
+  dn.a_static = h;
+  dn.a_static_rows = L.rows_total;
+  dn.b = w2;
+  dn.b3 = nullptr;
+  dn.b_rows = (int64_t)(c->E + c->S) * c->d_model;
+  dn.offsets = offsets;
+  dn.n_routed = c->E;
+  dn.n_static = c->S;
+  dn.rows_static = c->T;
+  dn.a_static_base = L.rows_cap;
+  dn.a_static_stride = c->T;
+  dn.out_static_base = L.rows_cap;
+  dn.max_routed_rows = L.rows_cap;
+  dn.out = y_rows;
+  dn.row_gate = row_gate;
+  dn.err = err;
+  return launch_grouped_gemm(dn, s);
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_query_sizes(const moe_config *cfg, moe_sizes *out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  const moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  const WsLayout L = make_layout(cfg);
+  out->rows_cap = L.rows_cap;
+  out->rows_total = L.rows_total;
+  out->tok_rows_len = L.tok_rows_len;
+  out->step_workspace = L.step_end;
+  out->workspace = L.total;
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_config *cfg, const void *x, const void *w_router, const float *bias,
+                     float *logits, float *probs, int32_t *topk_idx, float *topk_gate, void *ws,
+                     size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  const WsLayout L = make_layout(cfg);
+  if ((st = check_ws(L, ws, ws_bytes, L.step_end)) != MOE_OK) return st;
+  const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
+  if (!x || !w_router || !logits || !probs || (tc && (!topk_idx || !topk_gate)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(logits) || !aligned16(probs))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(run_route(cfg, L, static_cast<char *>(ws), x, w_router, bias, logits, probs,
+                               topk_idx, topk_gate, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_gate(const moe_config *cfg, const float *logits, float *probs, int32_t *topk_idx,
+                    float *topk_gate, void *ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  const WsLayout L = make_layout(cfg);
+  if ((st = check_ws(L, ws, ws_bytes, L.step_end)) != MOE_OK) return st;
+  const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
+  if (!logits || !probs || (tc && (!topk_idx || !topk_gate))) return MOE_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_gate(cfg, logits, probs, topk_idx, topk_gate, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *topk_idx,
+                       const float *topk_gate, const float *probs, int32_t *counts, int32_t *offsets,
+                       int32_t *tok_rows, int32_t *row_token, float *row_gate, void *x_perm,
+                       int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  const WsLayout L = make_layout(cfg);
+  if ((st = check_ws(L, ws, ws_bytes, L.step_end)) != MOE_OK) return st;
+  const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
+  const bool keepfrac = tc && cfg->capacity <= 0 && cfg->keep_den > 0;
+  if (!x || !counts || !offsets || !tok_rows || !row_token || !row_gate || !x_perm || !n_dropped)
+    return MOE_ERR_INVALID_ARG;
+  if (tc && (!topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
+  if ((!tc || keepfrac) && !probs) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_permute(cfg, L, static_cast<char *>(ws), x, topk_idx, topk_gate, probs,
+                                    counts, offsets, tok_rows, row_token, row_gate, x_perm,
+                                    n_dropped, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_expert_ffn(const moe_config *cfg, const void *x, const void *x_perm,
+                          const int32_t *offsets, const float *row_gate, const void *w1,
+                          const void *w3, const void *w2, void *h, void *y_rows, void *ws,
+                          size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  const WsLayout L = make_layout(cfg);
+  if ((st = check_ws(L, ws, ws_bytes, L.step_end)) != MOE_OK) return st;
+  const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
+  if (!x || !x_perm || !offsets || !row_gate || !w1 || !w2 || !h || !y_rows || (swiglu && !w3))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm) || !aligned16(w1) || !aligned16(w2) || !aligned16(h) ||
+      !aligned16(y_rows) || (swiglu && !aligned16(w3)))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(run_ffn(cfg, L, static_cast<char *>(ws), x, x_perm, offsets, row_gate, w1, w3,
+                             w2, h, y_rows, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_combine(const moe_config *cfg, const void *y_rows, const int32_t *tok_rows, void *y,
+                       moe_stream_t stream) {
+  moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (!y_rows || !tok_rows || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_rows) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(cfg);
+  return cuda_status(launch_combine(cfg, L.rows_cap, y_rows, tok_rows, y,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_forward(const moe_config *cfg, const void *x, const void *w_router,
+                       const float *bias, const void *w1, const void *w3, const void *w2, void *y,
+                       int32_t *counts_out, void *ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  const WsLayout L = make_layout(cfg);
+  if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
+  const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
+  if (!x || !w_router || !w1 || !w2 || !y || (swiglu && !w3)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(w1) || !aligned16(w2) || !aligned16(y) ||
+      (swiglu && !aligned16(w3)))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char *w = static_cast<char *>(ws);
+  float *logits = reinterpret_cast<float *>(w + L.logits);
+  float *probs = reinterpret_cast<float *>(w + L.probs);
+  int32_t *topk_idx = reinterpret_cast<int32_t *>(w + L.topk_idx);
+  float *topk_gate = reinterpret_cast<float *>(w + L.topk_gate);
+  int32_t *counts = reinterpret_cast<int32_t *>(w + L.counts);
+  int32_t *offsets = reinterpret_cast<int32_t *>(w + L.offsets);
+  int32_t *n_dropped = reinterpret_cast<int32_t *>(w + L.n_dropped);
+  int32_t *tok_rows = reinterpret_cast<int32_t *>(w + L.tok_rows);
+  int32_t *row_token = reinterpret_cast<int32_t *>(w + L.row_token);
+  float *row_gate = reinterpret_cast<float *>(w + L.row_gate);
+  void *x_perm = w + L.x_perm;
+  void *h = w + L.h;
+  void *y_rows = w + L.y_rows;
+  cudaError_t e = run_route(cfg, L, w, x, w_router, bias, logits, probs, topk_idx, topk_gate, s);
+  if (e == cudaSuccess)
+    e = launch_permute(cfg, L, w, x, topk_idx, topk_gate, probs, counts, offsets, tok_rows,
+                       row_token, row_gate, x_perm, n_dropped, s);
+  if (e == cudaSuccess)
+    e = run_ffn(cfg, L, w, x, x_perm, offsets, row_gate, w1, w3, w2, h, y_rows, s);
+  if (e == cudaSuccess) e = launch_combine(cfg, L.rows_cap, y_rows, tok_rows, y, s);
+  if (e == cudaSuccess && counts_out)
+    e = cudaMemcpyAsync(counts_out, counts, (size_t)cfg->E * 4, cudaMemcpyDeviceToDevice, s);
+  return cuda_status(e);
+}
+
+moe_status moe_check_device_errors(void *ws, size_t ws_bytes, moe_stream_t stream, uint32_t *flags) {
+  if (!ws || ws_bytes < 4) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpy(&word, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word != 0 && cudaMemset(ws, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
+  if (flags) *flags = word;
+  if (word & kErrTimeout) return MOE_ERR_TIMEOUT;
+  if (word & kErrBadIndex) return MOE_ERR_DEVICE_CHECK;
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream) {
+  if (!ws || ws_bytes < 256) return MOE_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, 256, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+const char *moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_CHECK: return "device-side index check failed";
+    case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

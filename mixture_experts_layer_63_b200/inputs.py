@@ -60,6 +60,9 @@ class Workload:
     zipf_s: float = 0.0               # > 0: Zipf logit bias over experts
 
     def with_tokens(self, T: int) -> "Workload":
+        """Same layer on T tokens; expert choice keeps C = T * k / E."""
+        if self.mode == "ec":
+            return replace(self, T=T, ec_capacity=max(1, T * self.k // self.E))
         return replace(self, T=T)
 
 

@@ -1,0 +1,78 @@
+"""Helpers shared by the GPU parity tests: oracle configuration from a
+workload, tensor <-> numpy conversion, the output tolerance rule."""
+from __future__ import annotations
+
+from dataclasses import replace
+
+import numpy as np
+import torch
+
+from mixture_experts_layer_63_b200 import api
+from mixture_experts_layer_63_b200.inputs import WORKLOADS, Workload, make_inputs
+from oracle import moe_oracle as O
+
+# Output tolerance: max |y - y_ref| <= TOL * rms(y_ref).  bf16: 2e-2 (bf16
+# operands, bf16 h and y_rows); fp32: 1e-4 (read as relative to rms).
+TOL = {"bf16": 2e-2, "f32": 1e-4}
+
+# Shape-reduced versions of the five workloads: same routing options, sizes
+# the oracle evaluates in seconds, several M tiles, ragged tails and partial
+# N tiles (d or f not a multiple of 256 / 128).
+SMALL = {
+    "tiny_f32": WORKLOADS["tiny_f32"],
+    "gshard_s": replace(WORKLOADS["gshard"], T=700, d_model=256, d_ff=320),
+    "mixtral_s": replace(WORKLOADS["mixtral"], T=600, d_model=320, d_ff=192),
+    "dsmoe_tc_s": replace(WORKLOADS["deepseekmoe_tc"], T=1000, d_model=256, d_ff=128),
+    "dsmoe_ec_s": replace(WORKLOADS["deepseekmoe_ec"], T=1000, d_model=256, d_ff=128,
+                          ec_capacity=1000 * 6 // 64),
+    "dsv2_s": replace(WORKLOADS["deepseek_v2"], T=900, d_model=320, d_ff=192),
+}
+
+
+def oracle_config(w: Workload) -> O.OracleConfig:
+    cap = O.capacity_from_factor(w.T, w.E, w.k, w.capacity_factor) if w.mode == "tc" else 0
+    return O.OracleConfig(E=w.E, S=w.S, k=w.k, act=w.act, mode=w.mode, capacity=cap,
+                          keep_num=w.keep_num, keep_den=w.keep_den,
+                          ec_capacity=w.ec_capacity if w.mode == "ec" else 0,
+                          n_groups=w.n_groups, topk_groups=w.topk_groups,
+                          renormalize=w.renormalize)
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    """Host numpy copy; bf16 becomes its uint16 bit pattern (the oracle's input form)."""
+    t = t.detach().contiguous().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().double().cpu().numpy()
+
+
+class LazyExperts:
+    """Expert weights fetched from the device one expert at a time (the
+    oracle indexes w[e]); keeps host memory small for the large workloads."""
+
+    def __init__(self, t: torch.Tensor | None):
+        self.t = t
+        self.cache: dict[int, np.ndarray] = {}
+
+    def __getitem__(self, e: int):
+        if self.t is None:
+            return None
+        e = int(e)
+        if e not in self.cache:
+            self.cache[e] = to_np(self.t[e])
+        return self.cache[e]
+
+
+def assert_close_rms(y: np.ndarray, ref: np.ndarray, tol: float, what: str = "y"):
+    rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2)))
+    err = float(np.max(np.abs(y.astype(np.float64) - ref)))
+    assert err <= tol * rms, f"{what}: max|err| {err:.3e} > {tol} * rms {rms:.3e}"
+    return err / rms
+
+
+def gpu_inputs(w: Workload, seed: int = 0, grid: bool = True):
+    return make_inputs(w, seed=seed, device="cuda", grid=grid)

@@ -1,0 +1,127 @@
+"""The C-ABI library loads, exports every entry point include/moe.h declares,
+and validates arguments on the host (no GPU needed: validation returns
+before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_63_b200 import api
+from mixture_experts_layer_63_b200.inputs import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from mixture_experts_layer_63_b200 import build
+    build.build()
+    return api.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert len(names) >= 10
+    assert set(names) == set(api.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_struct_sizes(L):
+    assert ctypes.sizeof(api.MoeConfig) == 72
+    assert ctypes.sizeof(api.MoeSizes) == 40
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert api.status_string(s)
+    assert api.status_string(99) == "unknown status"
+
+
+def test_sizes_of_the_workloads(L):
+    for name, w in WORKLOADS.items():
+        s = api.query_sizes(api.config_from_workload(w))
+        if w.mode == "ec":
+            assert s.rows_cap == w.E * w.ec_capacity and s.tok_rows_len == w.E * w.T
+        else:
+            assert s.rows_cap == w.T * w.k and s.tok_rows_len == w.T * w.k
+        assert s.rows_total == s.rows_cap + w.S * w.T
+        assert s.workspace >= s.step_workspace >= 256
+
+
+def _cfg(**kw):
+    c = api.config_from_workload(WORKLOADS["gshard"])
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("T", 0, api.MOE_ERR_INVALID_ARG),
+    ("k", 0, api.MOE_ERR_INVALID_ARG),
+    ("k", 17, api.MOE_ERR_INVALID_ARG),
+    ("k", 9, api.MOE_ERR_UNSUPPORTED),
+    ("E", 300, api.MOE_ERR_UNSUPPORTED),
+    ("d_model", 100, api.MOE_ERR_UNSUPPORTED),
+    ("d_ff", 96, api.MOE_ERR_UNSUPPORTED),
+    ("dtype", 7, api.MOE_ERR_INVALID_ARG),
+    ("act", 3, api.MOE_ERR_INVALID_ARG),
+    ("S", 9, api.MOE_ERR_UNSUPPORTED),
+    ("n_groups", 3, api.MOE_ERR_INVALID_ARG),       # 16 experts do not split into 3 groups
+    ("keep_den", 10, api.MOE_ERR_INVALID_ARG),      # capacity and keep-fraction together
+])
+def test_invalid_configs_rejected(L, field, value, status):
+    c = _cfg(**{field: value})
+    with pytest.raises(api.MoeError) as ei:
+        api.query_sizes(c)
+    assert ei.value.status == status
+
+
+def test_group_limit_needs_enough_experts(L):
+    c = _cfg(n_groups=8, topk_groups=1, k=2, capacity=0)   # 1 group of 2 experts holds k=2: ok
+    api.query_sizes(c)
+    c = _cfg(n_groups=8, topk_groups=1, k=3, capacity=0)
+    with pytest.raises(api.MoeError):
+        api.query_sizes(c)
+
+
+def test_expert_choice_options(L):
+    w = WORKLOADS["deepseekmoe_ec"]
+    c = api.config_from_workload(w)
+    api.query_sizes(c)
+    c.ec_capacity = w.T + 1
+    with pytest.raises(api.MoeError):
+        api.query_sizes(c)
+
+
+def test_null_pointers_rejected_before_any_launch(L):
+    """Host validation returns before touching CUDA, so this runs without a GPU."""
+    c = _cfg()
+    s = api.query_sizes(c)
+    f = L.moe_route
+    st = f(ctypes.byref(c), None, None, None, None, None, None, None, None, 0, None)
+    assert st == api.MOE_ERR_INVALID_ARG
+    # workspace too small
+    buf = ctypes.create_string_buffer(4096 + 256)
+    addr = (ctypes.addressof(buf) + 255) & ~255
+    st = L.moe_forward(ctypes.byref(c), 16, 16, None, 16, None, 16, 16, None, addr, 1024, None)
+    assert st == api.MOE_ERR_WORKSPACE
+    # misaligned workspace
+    st = L.moe_forward(ctypes.byref(c), 16, 16, None, 16, None, 16, 16, None, addr + 8, s.workspace, None)
+    assert st == api.MOE_ERR_INVALID_ARG
+    st = L.moe_combine(ctypes.byref(c), None, None, None, None)
+    assert st == api.MOE_ERR_INVALID_ARG
+
+
+def test_cpu_tensors_refused(L):
+    import torch
+    c = _cfg()
+    x = torch.zeros(c.T, c.d_model, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        api.moe_combine(c, x, x, x)

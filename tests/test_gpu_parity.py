@@ -1,0 +1,317 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+* Integer / index work and the fp32 gating arithmetic are compared bit for
+  bit: router logits and routing on grid inputs (exact fp32 logits), the
+  gate from oracle-computed logits, the permutation from oracle routing.
+* Floating-point outputs are compared with max |y - y_ref| <= tol * rms(y_ref),
+  tol = 2e-2 for bf16 and 1e-4 for fp32.
+* Sizes: shape-reduced workloads (several tiles, ragged tails, partial N
+  tiles) compared element by element; the full workload sizes run
+  moe_forward exactly as the benchmark launches it and compare the full
+  routing plus a sample of output tokens.
+"""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_63_b200 import api
+from mixture_experts_layer_63_b200.inputs import WORKLOADS, make_inputs
+from oracle import moe_oracle as O
+from tests.gpu_common import (SMALL, TOL, LazyExperts, assert_close_rms, gpu_inputs,
+                              oracle_config, to_f64, to_np)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    api.lib()
+    yield
+    torch.cuda.synchronize()
+
+
+def _bias_np(inp):
+    return None if inp.bias is None else to_np(inp.bias)
+
+
+def _route_gpu(cfg, inp):
+    B = api.step_buffers(cfg)
+    api.moe_route(cfg, inp.x, inp.w_router, inp.bias, B.logits, B.probs, B.topk_idx, B.topk_gate, B.ws)
+    return B
+
+
+# ---------------------------------------------------------------------------
+# steps 1-3a
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", list(SMALL) + ["full:" + n for n in WORKLOADS])
+def test_route_bit_exact(name):
+    """Router GEMM (tcgen05 for bf16, CUDA cores for fp32) + gate, grid inputs."""
+    w = WORKLOADS[name[5:]] if name.startswith("full:") else SMALL[name]
+    inp = make_inputs(w, seed=1, device="cuda", grid=True, with_weights=False)
+    cfg = api.config_from_workload(w)
+    B = _route_gpu(cfg, inp)
+    torch.cuda.synchronize()
+    ref_l = O.router_logits(to_np(inp.x), to_np(inp.w_router), _bias_np(inp))
+    assert np.array_equal(to_np(B.logits), ref_l)
+    probs, idx, gate, _ = O.route(oracle_config(w), ref_l)
+    assert np.array_equal(to_np(B.probs), probs)
+    if w.mode == "tc":
+        assert np.array_equal(to_np(B.topk_idx), idx)
+        assert np.array_equal(to_np(B.topk_gate), gate)
+    api.moe_check_device_errors(B.ws)
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_gate_bit_exact_from_oracle_logits(name):
+    """Softmax / top-k / group limit on normal (non-grid) inputs, full size."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w, seed=2, device="cpu", grid=False, with_weights=False)
+    ref_l = O.router_logits(to_np(inp.x), to_np(inp.w_router), _bias_np(inp))
+    probs, idx, gate, _ = O.route(oracle_config(w), ref_l)
+    cfg = api.config_from_workload(w)
+    B = api.step_buffers(cfg)
+    api.moe_gate(cfg, torch.from_numpy(ref_l).cuda(), B.probs, B.topk_idx, B.topk_gate, B.ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(B.probs), probs)
+    if w.mode == "tc":
+        assert np.array_equal(to_np(B.topk_idx), idx)
+        assert np.array_equal(to_np(B.topk_gate), gate)
+
+
+# ---------------------------------------------------------------------------
+# steps 3b-4
+# ---------------------------------------------------------------------------
+
+def _permute_check(w, seed=3, bias_override=None):
+    inp = make_inputs(w, seed=seed, device="cpu", grid=False, with_weights=False)
+    bias = _bias_np(inp) if bias_override is None else bias_override
+    ref_l = O.router_logits(to_np(inp.x), to_np(inp.w_router), bias)
+    oc = oracle_config(w)
+    probs, idx, gate, disp = O.route(oc, ref_l)
+    cfg = api.config_from_workload(w)
+    B = api.step_buffers(cfg)
+    xg = inp.x.cuda()
+    tk_i = torch.from_numpy(idx).cuda() if idx is not None else None
+    tk_g = torch.from_numpy(gate).cuda() if gate is not None else None
+    api.moe_permute(cfg, xg, tk_i, tk_g, torch.from_numpy(probs).cuda(), B.counts, B.offsets,
+                    B.tok_rows, B.row_token, B.row_gate, B.x_perm, B.n_dropped, B.ws)
+    torch.cuda.synchronize()
+    R = int(disp.offsets[-1])
+    assert np.array_equal(to_np(B.counts), disp.counts)
+    assert np.array_equal(to_np(B.offsets), disp.offsets)
+    assert int(B.n_dropped.item()) == disp.n_dropped
+    assert np.array_equal(to_np(B.tok_rows), disp.tok_rows.reshape(-1))
+    assert np.array_equal(to_np(B.row_token)[:R], disp.row_token)
+    assert np.array_equal(to_np(B.row_gate)[:R], disp.row_gate)
+    # x_perm rows are byte copies of the x rows they name
+    assert torch.equal(B.x_perm[:R], xg[B.row_token[:R].long()])
+    api.moe_check_device_errors(B.ws)
+    return disp
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_permute_bit_exact_full_size(name):
+    _permute_check(WORKLOADS[name])
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_permute_bit_exact_small(name):
+    _permute_check(SMALL[name])
+
+
+def test_permute_capacity_saturated():
+    """Every token's first choice is expert 0: exactly C of them survive."""
+    w = SMALL["gshard_s"]
+    bias = np.zeros(w.E, np.float32)
+    bias[0] = 100.0
+    disp = _permute_check(w, bias_override=bias)
+    C = O.capacity_from_factor(w.T, w.E, w.k, w.capacity_factor)
+    assert disp.kept[0] == C and disp.n_dropped > 0
+
+
+def test_permute_unused_experts():
+    """Half of the experts receive no token at all (empty segments)."""
+    w = SMALL["dsmoe_tc_s"]
+    bias = np.zeros(w.E, np.float32)
+    bias[w.E // 2:] = -1.0e4
+    disp = _permute_check(w, bias_override=bias)
+    assert np.all(disp.counts[w.E // 2:] == 0)
+
+
+# ---------------------------------------------------------------------------
+# step 5
+# ---------------------------------------------------------------------------
+
+def _ffn_reference_rows(w, oc, inp_np, disp, T, lazy):
+    """Oracle y_rows: gate * FFN_e(x_t) per routed row, FFN_s(x_t) per shared row."""
+    x = inp_np
+    R = int(disp.offsets[-1])
+    rows = {}
+    for e in range(w.E):
+        a, b = int(disp.offsets[e]), int(disp.offsets[e + 1])
+        if b > a:
+            out = O.expert_ffn(x[disp.row_token[a:b]], lazy["w1"][e], lazy["w2"][e], lazy["w3"][e], w.act)
+            rows[e] = out * disp.row_gate[a:b, None].astype(np.float64)
+    shared = [O.expert_ffn(x, lazy["w1"][w.E + s], lazy["w2"][w.E + s], lazy["w3"][w.E + s], w.act)
+              for s in range(w.S)]
+    return R, rows, shared
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_expert_ffn_rows(name):
+    w = SMALL[name]
+    inp = gpu_inputs(w, seed=4, grid=True)
+    oc = oracle_config(w)
+    x_np = to_np(inp.x)
+    ref_l = O.router_logits(x_np, to_np(inp.w_router), _bias_np(inp))
+    probs, idx, gate, disp = O.route(oc, ref_l)
+    cfg = api.config_from_workload(w)
+    s = api.query_sizes(cfg)
+    B = api.step_buffers(cfg)
+    R = int(disp.offsets[-1])
+    B.offsets.copy_(torch.from_numpy(disp.offsets))
+    B.row_gate[:R].copy_(torch.from_numpy(disp.row_gate))
+    B.x_perm[:R].copy_(inp.x[torch.from_numpy(disp.row_token).long().cuda()])
+    api.moe_expert_ffn(cfg, inp.x, B.x_perm, B.offsets, B.row_gate, inp.w1, inp.w3, inp.w2, B.h,
+                       B.y_rows, B.ws)
+    torch.cuda.synchronize()
+    lazy = {"w1": LazyExperts(inp.w1), "w2": LazyExperts(inp.w2), "w3": LazyExperts(inp.w3)}
+    R, rows, shared = _ffn_reference_rows(w, oc, x_np, disp, w.T, lazy)
+    y_rows = to_f64(B.y_rows)
+    ref = np.zeros((R, w.d_model))
+    for e, out in rows.items():
+        ref[disp.offsets[e]:disp.offsets[e + 1]] = out
+    assert_close_rms(y_rows[:R], ref, TOL[w.dtype], "routed rows")
+    for si, sh in enumerate(shared):
+        base = s.rows_cap + si * w.T
+        assert_close_rms(y_rows[base:base + w.T], sh, TOL[w.dtype], f"shared expert {si}")
+    api.moe_check_device_errors(B.ws)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_combine_sums_rows_in_order(name):
+    w = SMALL[name]
+    inp = make_inputs(w, seed=5, device="cpu", grid=False, with_weights=False)
+    oc = oracle_config(w)
+    ref_l = O.router_logits(to_np(inp.x), to_np(inp.w_router), _bias_np(inp))
+    _, _, _, disp = O.route(oc, ref_l)
+    cfg = api.config_from_workload(w)
+    s = api.query_sizes(cfg)
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    y_rows = torch.randn(s.rows_total, w.d_model, generator=g, device="cuda").to(dt)
+    tok_rows = torch.from_numpy(disp.tok_rows.reshape(-1).copy()).cuda()
+    y = torch.empty(w.T, w.d_model, dtype=dt, device="cuda")
+    api.moe_combine(cfg, y_rows, tok_rows, y)
+    torch.cuda.synchronize()
+    yr = to_f64(y_rows)
+    ref = np.zeros((w.T, w.d_model))
+    for t in range(w.T):
+        rows = (disp.tok_rows[:, t] if w.mode == "ec" else disp.tok_rows[t])
+        for r in rows:
+            if r >= 0:
+                ref[t] += yr[r]
+        for si in range(w.S):
+            ref[t] += yr[s.rows_cap + si * w.T + t]
+    got = to_f64(y)
+    # fp32 accumulation then one rounding to the output type
+    ulp = 2.0 ** -8 if w.dtype == "bf16" else 2.0 ** -23
+    bound = ulp * np.abs(ref) + 1e-5 * (1 + np.abs(yr).max())
+    assert np.all(np.abs(got - ref) <= bound)
+
+
+# ---------------------------------------------------------------------------
+# steps 1-5 through moe_forward
+# ---------------------------------------------------------------------------
+
+def _forward_check(w, seed=6, tokens=None, inp=None):
+    inp = inp if inp is not None else gpu_inputs(w, seed=seed, grid=True)
+    cfg = api.config_from_workload(w)
+    ws = api.new_workspace(cfg)
+    y = torch.empty_like(inp.x)
+    counts = torch.empty(w.E, dtype=torch.int32, device="cuda")
+    api.moe_forward(cfg, inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, y, counts, ws)
+    api.moe_check_device_errors(ws)
+    oc = oracle_config(w)
+    x_np = to_np(inp.x)
+    ref_l = O.router_logits(x_np, to_np(inp.w_router), _bias_np(inp))
+    probs, idx, gate, disp = O.route(oc, ref_l)
+    assert np.array_equal(to_np(counts), disp.counts)
+    toks = np.arange(w.T) if tokens is None else np.asarray(tokens)
+    lazy = (LazyExperts(inp.w1), LazyExperts(inp.w2), LazyExperts(inp.w3))
+    ref = O.combine_tokens(oc, x_np, lazy[0], lazy[1], lazy[2], disp, toks)
+    got = to_f64(y)[toks]
+    rel = assert_close_rms(got, ref, TOL[w.dtype])
+    return rel, disp
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_small(name):
+    _forward_check(SMALL[name])
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_forward_full_size_sampled(name):
+    """The benchmark's launch configuration at full size: full routing bit-exact
+    (counts), outputs of 24 sampled tokens (first, last, 22 seeded) within tolerance."""
+    w = WORKLOADS[name]
+    rng = np.random.default_rng(11)
+    toks = np.unique(np.concatenate([[0, w.T - 1], rng.integers(0, w.T, 22)]))
+    _forward_check(w, seed=6, tokens=toks)
+    torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------
+# edge cases
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T", [1, 2, 127, 129])
+@pytest.mark.parametrize("base", ["gshard_s", "dsmoe_ec_s", "dsv2_s", "tiny_f32"])
+def test_forward_ragged_token_counts(T, base):
+    _forward_check(SMALL[base].with_tokens(T))
+
+
+def test_dense_mixture_k_equals_E():
+    w = replace(SMALL["mixtral_s"], T=200, k=8, renormalize=False)
+    _forward_check(w)
+
+
+def test_single_expert_dense_ffn():
+    w = replace(SMALL["gshard_s"], T=300, E=1, k=1, capacity_factor=0.0)
+    _forward_check(w)
+
+
+def test_all_routed_dropped_leaves_shared_experts():
+    w = replace(SMALL["dsv2_s"], T=300, keep_num=0, keep_den=1)
+    rel, disp = _forward_check(w)
+    assert disp.n_dropped == w.T * w.k
+
+
+def test_expert_choice_takes_every_token():
+    w = replace(SMALL["dsmoe_ec_s"], T=200, ec_capacity=200)
+    _forward_check(w)
+
+
+def test_bad_expert_index_sets_the_error_word():
+    """A corrupted routing index is caught by the kernel's own check: the
+    error word reports it and nothing out of range is touched."""
+    w = SMALL["gshard_s"]
+    cfg = api.config_from_workload(w)
+    B = api.step_buffers(cfg)
+    x = torch.randn(w.T, w.d_model, device="cuda").to(torch.bfloat16)
+    idx = torch.randint(0, w.E, (w.T, w.k), device="cuda", dtype=torch.int32)
+    idx[:, 1] = (idx[:, 0] + 1) % w.E
+    idx[5, 0] = w.E + 3
+    gate = torch.rand(w.T, w.k, device="cuda")
+    api.moe_permute(cfg, x, idx, gate, None, B.counts, B.offsets, B.tok_rows, B.row_token,
+                    B.row_gate, B.x_perm, B.n_dropped, B.ws)
+    with pytest.raises(api.MoeError) as ei:
+        api.moe_check_device_errors(B.ws)
+    assert ei.value.status == api.MOE_ERR_DEVICE_CHECK
+    # the word is cleared after reading
+    assert api.moe_check_device_errors(B.ws) == 0
