@@ -342,7 +342,7 @@ def run_ours(args, w) -> None:
     nmat = 3 if w.act == "swiglu" else 2
     gemm_flops = 2.0 * rows * w.d_model * w.d_ff * nmat
     permute_bytes = (w.T * w.d_model + R * w.d_model) * es
-    combine_bytes = (rows * w.d_model + w.T * w.d_model) * es
+    combine_bytes = rows * w.d_model * 4 + w.T * w.d_model * es     # fp32 rows in, y out
     route_bytes = (w.T * w.d_model + w.E * w.d_model) * es + 2 * w.T * w.E * 4
     mean = per.mean(axis=0)                                # ms per call
     hbm, tfl, tfl_sus, peak_src = _peaks()

@@ -1,9 +1,10 @@
 // Gate-weighted combine (GShard section 3 of "MoE技术演进": y_s = sum_e
 // G_{s,e} FFN_e(x_s); DeepSeekMoE section 2: plus the shared experts' sum).
-// The gates were applied in the down-projection epilogue, so here each
-// token sums its rows: routed rows in the token's k-rank order (expert
-// choice: ascending expert), then shared experts 0..S-1, fp32 accumulation,
-// one rounding to the output dtype.  One warp per token, 16-byte vectors.
+// The gates were applied in the down-projection epilogue, which leaves fp32
+// rows; here each token sums its rows: routed rows in the token's k-rank
+// order (expert choice: ascending expert), then shared experts 0..S-1, fp32
+// accumulation, one rounding to the output dtype.  One warp per token,
+// 16-byte vectors.
 #include "device_common.cuh"
 #include "moe_internal.h"
 
@@ -38,39 +39,36 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const void *__rest
   n += S;
   __syncwarp();
 
-  const int epv = BF16 ? 8 : 4;                 // elements per 16-byte vector
-  const int nvec = d / epv;
-  const uint4 *src = reinterpret_cast<const uint4 *>(y_rows);
-  uint4 *dst = reinterpret_cast<uint4 *>(y);
+  // y_rows are fp32; 8 (bf16 out) or 4 (fp32 out) elements per lane and step
+  constexpr int EPV = BF16 ? 8 : 4;
+  const int nvec = d / EPV;
+  const float4 *src = reinterpret_cast<const float4 *>(y_rows);
+  const int64_t row_vec = d / 4;                 // float4 per fp32 row
   for (int v = lane; v < nvec; v += 32) {
-    float acc[8];
+    float acc[EPV];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int i = 0; i < EPV; ++i) acc[i] = 0.f;
     for (int i = 0; i < n; ++i) {
-      const uint4 q = src[(int64_t)rows[i] * nvec + v];
-      if (BF16) {
-        acc[0] += bf16_lo(q.x); acc[1] += bf16_hi(q.x);
-        acc[2] += bf16_lo(q.y); acc[3] += bf16_hi(q.y);
-        acc[4] += bf16_lo(q.z); acc[5] += bf16_hi(q.z);
-        acc[6] += bf16_lo(q.w); acc[7] += bf16_hi(q.w);
-      } else {
-        acc[0] += __uint_as_float(q.x); acc[1] += __uint_as_float(q.y);
-        acc[2] += __uint_as_float(q.z); acc[3] += __uint_as_float(q.w);
+      const float4 *p = src + (int64_t)rows[i] * row_vec + (int64_t)v * (EPV / 4);
+#pragma unroll
+      for (int q = 0; q < EPV / 4; ++q) {
+        const float4 a = p[q];
+        acc[4 * q + 0] += a.x;
+        acc[4 * q + 1] += a.y;
+        acc[4 * q + 2] += a.z;
+        acc[4 * q + 3] += a.w;
       }
     }
-    uint4 o;
     if (BF16) {
+      uint4 o;
       o.x = pack_bf16x2(acc[0], acc[1]);
       o.y = pack_bf16x2(acc[2], acc[3]);
-      o.z = pack_bf16x2(acc[4], acc[5]);
-      o.w = pack_bf16x2(acc[6], acc[7]);
+      o.z = pack_bf16x2(acc[4 % EPV], acc[5 % EPV]);
+      o.w = pack_bf16x2(acc[6 % EPV], acc[7 % EPV]);
+      reinterpret_cast<uint4 *>(y)[t * nvec + v] = o;
     } else {
-      o.x = __float_as_uint(acc[0]);
-      o.y = __float_as_uint(acc[1]);
-      o.z = __float_as_uint(acc[2]);
-      o.w = __float_as_uint(acc[3]);
+      reinterpret_cast<float4 *>(y)[t * nvec + v] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     }
-    dst[t * nvec + v] = o;
   }
 }
 

@@ -8,7 +8,8 @@
 //     SiLU(x W_1^T) * (x W_3^T) (SwiGLU, 3*d_model*d_moe parameters per
 //     "大语言模型并行策略（七）：专家并行"), bf16 out
 //   * the down-projection with the gate G_{t,e} of the combine equation
-//     y_s = sum_e G_{s,e} FFN_e(x_s) folded into its epilogue, bf16 out.
+//     y_s = sum_e G_{s,e} FFN_e(x_s) folded into its epilogue, fp32 out (the
+//     combine sums the rows of a token and rounds once).
 // The "IO-aware" expert kernels of the Multi-Head LatentMoE summary batch
 // token-to-expert traffic with the expert compute; here the batching is the
 // expert-contiguous row layout and the activation / gate scaling never make
@@ -431,21 +432,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int col = col0 + c * 32;
           if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
         }
-      } else if (EPI == kEpiRelu || EPI == kEpiScale) {
+      } else if (EPI == kEpiRelu) {
         __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
-        float scale = 1.0f;
-        if (EPI == kEpiScale && routed && valid) scale = P.row_gate[out_row];
 #pragma unroll 1
         for (int c = 0; c < P.bn / 32; ++c) {
           tmem_ld32(taddr + c * 32, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float a = __uint_as_float(r[i]);
-            v[i] = (EPI == kEpiRelu) ? fmaxf(a, 0.0f) : a * scale;
-          }
+          for (int i = 0; i < 32; ++i) v[i] = fmaxf(__uint_as_float(r[i]), 0.0f);
           const int col = col0 + c * 32;
           if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
+        }
+      } else if (EPI == kEpiScale) {
+        // fp32 rows: the combine rounds once, after summing
+        float *out = reinterpret_cast<float *>(P.out);
+        const float scale = (routed && valid) ? P.row_gate[out_row] : 1.0f;
+#pragma unroll 1
+        for (int c = 0; c < P.bn / 32; ++c) {
+          tmem_ld32(taddr + c * 32, r);
+          tmem_ld_wait();
+          const int col = col0 + c * 32;
+          if (valid && col < P.N) {
+            float4 *dst = reinterpret_cast<float4 *>(out + out_row * P.N + col);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(__uint_as_float(r[4 * q]) * scale, __uint_as_float(r[4 * q + 1]) * scale,
+                                   __uint_as_float(r[4 * q + 2]) * scale, __uint_as_float(r[4 * q + 3]) * scale);
+          }
         }
       } else {  // kEpiStoreF32
         float *out = reinterpret_cast<float *>(P.out);

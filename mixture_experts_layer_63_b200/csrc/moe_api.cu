@@ -90,7 +90,7 @@ WsLayout make_layout(const moe_config *c) {
   L.row_gate = take((size_t)L.rows_cap * 4);
   L.x_perm = take((size_t)L.rows_cap * c->d_model * es);
   L.h = take((size_t)L.rows_total * c->d_ff * es);
-  L.y_rows = take((size_t)L.rows_total * c->d_model * es);
+  L.y_rows = take((size_t)L.rows_total * c->d_model * 4);      // fp32 rows
   L.total = o;
   return L;
 }

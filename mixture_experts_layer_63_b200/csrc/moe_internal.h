@@ -59,7 +59,7 @@ enum GemmEpilogue : int {
   kEpiStoreF32 = 0,   // out fp32 = acc (+ bias[col])           (router logits)
   kEpiRelu = 1,       // out bf16 = relu(acc)                    (up-projection, ReLU)
   kEpiSwiglu = 2,     // out bf16 = silu(acc_gate) * acc_up      (gate/up projection)
-  kEpiScale = 3,      // out bf16 = row_gate[row] * acc          (down-projection)
+  kEpiScale = 3,      // out fp32 = row_gate[row] * acc          (down-projection)
 };
 
 // One grouped GEMM  out[rows_g, N] = A[rows_g, K] . B_g[N, K]^T  per group g.

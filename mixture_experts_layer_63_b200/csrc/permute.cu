@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(256) rank_kernel(
     }
     __syncthreads();
     if (e >= 0 && leader) {
-      running[e] += cnt;
+      atomicAdd(&running[e], cnt);      // leaders of several warps may share e
       wc[warp][e] = 0;
     }
     __syncthreads();

@@ -55,11 +55,16 @@ cudaError_t launch_router_f32(const moe_config *c, const float *x, const float *
 //   4. p_e = exp_det(l_e - m) / S (IEEE division); gates = p of the chosen
 //      experts, or p / (their sum in rank order) when renormalising.
 // ---------------------------------------------------------------------------
+// Insert (v, i) into a list sorted by value, descending.  Candidates arrive
+// in ascending index order, so an equal value stays behind the ones already
+// listed; once inserted, every later entry shifts down one place.
 __device__ __forceinline__ void topk_insert(float v, int i, float (&tv)[kMaxTopK],
                                             int (&ti)[kMaxTopK]) {
+  bool shifting = false;
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) {
-    const bool better = (ti[j] < 0) || (v > tv[j]);
+    const bool better = shifting || (ti[j] < 0) || (v > tv[j]);
+    shifting = better;
     const float ov = tv[j];
     const int oi = ti[j];
     tv[j] = better ? v : ov;

@@ -11,9 +11,19 @@ from mixture_experts_layer_63_b200 import api
 from mixture_experts_layer_63_b200.inputs import WORKLOADS, Workload, make_inputs
 from oracle import moe_oracle as O
 
-# Output tolerance: max |y - y_ref| <= TOL * rms(y_ref).  bf16: 2e-2 (bf16
-# operands, bf16 h and y_rows); fp32: 1e-4 (read as relative to rms).
+# Output tolerance: max |y - y_ref| <= TOL * rms(y_ref) + half an ulp of
+# y_ref in the output format.  bf16: 2e-2, fp32: 1e-4 (read as relative to
+# rms).  The half-ulp term is the storage rounding of the output itself: a
+# bf16 value carries up to 2**-8 |y| of it, so without the term even the
+# correctly rounded exact answer would break the rule wherever |y| > 5.12 rms.
 TOL = {"bf16": 2e-2, "f32": 1e-4}
+SIG_BITS = {"bf16": 8, "f32": 24}
+
+
+def half_ulp(ref: np.ndarray, dtype: str) -> np.ndarray:
+    """Half an ulp of each |ref| in the output format (8 or 24 significant bits)."""
+    _, e = np.frexp(np.abs(ref))                 # |ref| = m * 2**e, m in [0.5, 1)
+    return np.ldexp(1.0, e - 1 - SIG_BITS[dtype])
 
 # Shape-reduced versions of the five workloads: same routing options, sizes
 # the oracle evaluates in seconds, several M tiles, ragged tails and partial
@@ -67,11 +77,16 @@ class LazyExperts:
         return self.cache[e]
 
 
-def assert_close_rms(y: np.ndarray, ref: np.ndarray, tol: float, what: str = "y"):
-    rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2)))
-    err = float(np.max(np.abs(y.astype(np.float64) - ref)))
-    assert err <= tol * rms, f"{what}: max|err| {err:.3e} > {tol} * rms {rms:.3e}"
-    return err / rms
+def assert_close_rms(y: np.ndarray, ref: np.ndarray, dtype: str, what: str = "y"):
+    """max over elements of (|y - ref| - half_ulp(ref)) <= TOL[dtype] * rms(ref)."""
+    ref = ref.astype(np.float64)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    diff = np.abs(y.astype(np.float64) - ref)
+    excess = float(np.max(diff - half_ulp(ref, dtype)))
+    tol = TOL[dtype]
+    assert excess <= tol * rms, (f"{what}: max(|err| - half ulp) {excess:.3e} > {tol} * rms "
+                                 f"{rms:.3e} (plain max|err| {diff.max():.3e})")
+    return float(diff.max()) / rms
 
 
 def gpu_inputs(w: Workload, seed: int = 0, grid: bool = True):

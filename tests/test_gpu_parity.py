@@ -3,8 +3,9 @@
 * Integer / index work and the fp32 gating arithmetic are compared bit for
   bit: router logits and routing on grid inputs (exact fp32 logits), the
   gate from oracle-computed logits, the permutation from oracle routing.
-* Floating-point outputs are compared with max |y - y_ref| <= tol * rms(y_ref),
-  tol = 2e-2 for bf16 and 1e-4 for fp32.
+* Floating-point outputs are compared with max |y - y_ref| <= tol * rms(y_ref)
+  plus half an ulp of y_ref in the output format (the output's own storage
+  rounding), tol = 2e-2 for bf16 and 1e-4 for fp32.
 * Sizes: shape-reduced workloads (several tiles, ragged tails, partial N
   tiles) compared element by element; the full workload sizes run
   moe_forward exactly as the benchmark launches it and compare the full
@@ -161,6 +162,14 @@ def _ffn_reference_rows(w, oc, inp_np, disp, T, lazy):
     return R, rows, shared
 
 
+def _assert_rows_close(y, ref, tol, what):
+    rms = np.sqrt(np.mean(ref ** 2, axis=1)) + 1e-30
+    err = np.abs(y - ref).max(axis=1)
+    worst = int(np.argmax(err / rms))
+    assert np.all(err <= tol * rms), (f"{what}: row {worst} max|err| {err[worst]:.3e} > "
+                                      f"{tol} * row rms {rms[worst]:.3e}")
+
+
 @pytest.mark.parametrize("name", list(SMALL))
 def test_expert_ffn_rows(name):
     w = SMALL[name]
@@ -185,10 +194,12 @@ def test_expert_ffn_rows(name):
     ref = np.zeros((R, w.d_model))
     for e, out in rows.items():
         ref[disp.offsets[e]:disp.offsets[e + 1]] = out
-    assert_close_rms(y_rows[:R], ref, TOL[w.dtype], "routed rows")
+    # each row is one expert's output for one token: the tolerance rule is
+    # applied per row (rows differ in scale by their gates)
+    _assert_rows_close(y_rows[:R], ref, TOL[w.dtype], "routed rows")
     for si, sh in enumerate(shared):
         base = s.rows_cap + si * w.T
-        assert_close_rms(y_rows[base:base + w.T], sh, TOL[w.dtype], f"shared expert {si}")
+        _assert_rows_close(y_rows[base:base + w.T], sh, TOL[w.dtype], f"shared expert {si}")
     api.moe_check_device_errors(B.ws)
 
 
@@ -204,7 +215,7 @@ def test_combine_sums_rows_in_order(name):
     dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
     g = torch.Generator(device="cuda")
     g.manual_seed(7)
-    y_rows = torch.randn(s.rows_total, w.d_model, generator=g, device="cuda").to(dt)
+    y_rows = torch.randn(s.rows_total, w.d_model, generator=g, device="cuda")     # fp32 rows
     tok_rows = torch.from_numpy(disp.tok_rows.reshape(-1).copy()).cuda()
     y = torch.empty(w.T, w.d_model, dtype=dt, device="cuda")
     api.moe_combine(cfg, y_rows, tok_rows, y)
@@ -246,7 +257,7 @@ def _forward_check(w, seed=6, tokens=None, inp=None):
     lazy = (LazyExperts(inp.w1), LazyExperts(inp.w2), LazyExperts(inp.w3))
     ref = O.combine_tokens(oc, x_np, lazy[0], lazy[1], lazy[2], disp, toks)
     got = to_f64(y)[toks]
-    rel = assert_close_rms(got, ref, TOL[w.dtype])
+    rel = assert_close_rms(got, ref, w.dtype)
     return rel, disp
 
 
