@@ -161,6 +161,33 @@ MOE_API moe_status moe_permute(const moe_config *cfg, const void *x, const int32
                        int32_t *tok_rows, int32_t *row_token, float *row_gate, void *x_perm,
                        int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_permute without a workspace argument.  The paper has no counterpart:
+ * this entry point is for callers that cannot allocate device memory (a
+ * plugin in a host program that is handed only its input and output buffers,
+ * or a process that must keep a fixed device footprint once started) and so
+ * cannot provide moe_permute's workspace.
+ *   Arguments, outputs and results are those of moe_permute.
+ *   Scratch: a fixed array of MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (8 MiB) compiled
+ *   into the library, held by every GPU that loads the library until the
+ *   process exits.  A configuration whose step scratch
+ *   (moe_sizes.step_workspace) exceeds it returns MOE_ERR_WORKSPACE before
+ *   any launch.  It calls no cudaMalloc, cudaFree or allocating routine.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   with that device current; make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *   call's contents (each call clears what must start at zero).  Calls that
+ *   overlap on the GPU -- other streams or threads -- race on it and give wrong
+ *   results; serialise them.
+ *   Errors: the array's error word is cleared at the start of each call; bad
+ *   expert indices are still skipped, but their report cannot be read here
+ *   (moe_permute with a workspace and moe_check_device_errors shows it). */
+#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const void *x, const int32_t *topk_idx,
+                                       const float *topk_gate, const float *probs, int32_t *counts,
+                                       int32_t *offsets, int32_t *tok_rows, int32_t *row_token,
+                                       float *row_gate, void *x_perm, int32_t *n_dropped,
+                                       moe_stream_t stream);
+
 /* Step 5a-5b: the grouped expert FFNs.
  *   in : x [T, d] (input of the shared experts), x_perm [rows_cap, d],
  *        offsets [E+1], row_gate [rows_cap], w1, w3 (SwiGLU; NULL for ReLU), w2.

@@ -28,7 +28,7 @@ MOE_TOKEN_CHOICE, MOE_EXPERT_CHOICE = 0, 1
 
 EXPORTS = ("moe_query_sizes", "moe_route", "moe_gate", "moe_permute", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_check_device_errors", "moe_workspace_init",
-           "moe_status_string")
+           "moe_status_string", "moe_permute_noalloc")
 
 
 class MoeError(RuntimeError):
@@ -286,3 +286,37 @@ class MoELayer:
         moe_forward(self.cfg, x, self.w_router, self.bias, self.w1, self.w3, self.w2, y,
                     self.counts, self.ws, stream)
         return y
+
+
+# ---------------------------------------------------------------------------
+# moe_permute without a workspace (callers that cannot allocate device memory)
+# ---------------------------------------------------------------------------
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+_noalloc_fn = None
+
+
+def _noalloc():
+    """moe_permute_noalloc with its C signature declared (once)."""
+    global _noalloc_fn
+    if _noalloc_fn is None:
+        f = lib().moe_permute_noalloc
+        f.argtypes = [ctypes.POINTER(MoeConfig)] + [ctypes.c_void_p] * 12
+        f.restype = ctypes.c_int
+        _noalloc_fn = f
+    return _noalloc_fn
+
+
+def moe_permute_noalloc(cfg, x, topk_idx, topk_gate, probs, counts, offsets, tok_rows, row_token,
+                        row_gate, x_perm, n_dropped, stream=None):
+    """moe_permute with its scratch in the library's fixed 8 MiB device array.
+
+    For callers that cannot allocate device memory (a plugin handed only its
+    inputs and outputs, or a process with a fixed footprint after start-up).
+    The first call on a device looks up the array's address: make it before
+    any stream capture.  Calls that overlap on the GPU race on the array.
+    """
+    _check("moe_permute_noalloc", _noalloc()(
+        ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(topk_gate), _ptr(probs), _ptr(counts),
+        _ptr(offsets), _ptr(tok_rows), _ptr(row_token), _ptr(row_gate), _ptr(x_perm),
+        _ptr(n_dropped), _stream(stream)))

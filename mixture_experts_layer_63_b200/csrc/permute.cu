@@ -21,6 +21,8 @@
 // (p bits << 32 | ~t), so "larger p first, lower t on ties" is decided by
 // integer comparisons alone.
 //   gather_rows   x_perm[r] = x[row_token[r]], 16-byte vectors.
+#include <mutex>
+
 #include "device_common.cuh"
 #include "moe_internal.h"
 
@@ -417,3 +419,78 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, con
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: moe_permute for callers that cannot allocate.
+//
+// Some callers cannot allocate device memory at all: a plugin inside a host
+// program that hands it only its input and output buffers, or a process that
+// must keep a fixed device footprint once it has started.  They cannot
+// provide moe_permute's workspace.  This entry point takes its scratch from
+// one fixed array compiled into the library instead.
+//
+// The array lives on every GPU that loads the library until the process
+// exits.  In host code its name is only a host-side stand-in, so its device
+// address is looked up once per device (with that device current) through
+// cudaGetSymbolAddress and passed to the kernels like a workspace pointer.
+// All calls on a device share the array and it keeps the last call's
+// contents: the kernels overwrite every scratch word they read except the
+// error word, which each call clears first.  Calls that overlap on the GPU
+// race on the array.
+// ---------------------------------------------------------------------------
+namespace moe {
+
+constexpr size_t kStaticScratchBytes = MOE_PERMUTE_NOALLOC_SCRATCH_BYTES;     // 8 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void *g_scratch_address[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device.
+cudaError_t static_scratch_address(char **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_address[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_address[dev] = p;
+  }
+  *out = static_cast<char *>(g_scratch_address[dev]);
+  return cudaSuccess;
+}
+}  // namespace
+
+}  // namespace moe
+
+extern "C" moe_status moe_permute_noalloc(const moe_config *cfg, const void *x,
+                                          const int32_t *topk_idx, const float *topk_gate,
+                                          const float *probs, int32_t *counts, int32_t *offsets,
+                                          int32_t *tok_rows, int32_t *row_token, float *row_gate,
+                                          void *x_perm, int32_t *n_dropped, moe_stream_t stream) {
+  using namespace moe;
+  const moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  const WsLayout L = make_layout(cfg);
+  if (L.step_end > kStaticScratchBytes) return MOE_ERR_WORKSPACE;   // beyond the fixed array
+  const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
+  const bool keepfrac = tc && cfg->capacity <= 0 && cfg->keep_den > 0;
+  if (!x || !counts || !offsets || !tok_rows || !row_token || !row_gate || !x_perm || !n_dropped)
+    return MOE_ERR_INVALID_ARG;
+  if (tc && (!topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
+  if ((!tc || keepfrac) && !probs) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u))
+    return MOE_ERR_INVALID_ARG;
+  char *scratch = nullptr;
+  if (static_scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch + L.err, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  const cudaError_t e = launch_permute(cfg, L, scratch, x, topk_idx, topk_gate, probs, counts,
+                                       offsets, tok_rows, row_token, row_gate, x_perm, n_dropped, s);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
