@@ -5,10 +5,9 @@
 
 One step = one whole forward of the layer (router, gate, selection,
 permutation, expert FFNs, combine) over one batch of T tokens, inputs resident
-in HBM.  The timed loop issues the four step entry points of the C ABI
-(moe_route, moe_permute, moe_expert_ffn, moe_combine: the same launches as
-moe_forward) with CUDA events between them; L2 is flushed (256 MB memset,
-untimed) before every step.  `e2e` times moe_forward through the public
+in HBM.  The timed loop calls moe_forward_timed (the launches of moe_forward,
+with CUDA events recorded at its phase boundaries on the launching stream);
+L2 is flushed (256 MB memset, untimed) before every step.  `e2e` times moe_forward through the public
 layer object with the host->device copy of x and the device->host copy of y
 inside the timed region.  With N > 1 (torchrun), every rank runs its own
 replica on its own tokens (no collective in the forward: weak scaling); the
@@ -78,14 +77,16 @@ def _src_hash(name: str) -> str:
 
 
 def launches_per_step(w) -> int:
-    """Kernels libmoe launches for one forward of this workload."""
-    n = 2                                     # router (GEMM or fp32) + gate
+    """Kernels libmoe launches for one moe_forward of this workload."""
+    fused_router = w.dtype == "f32" and w.E <= 32 and w.E * w.d_model * 4 <= 160 * 1024
+    n = 1 if fused_router else 2              # router GEMM (or fp32 router inside the gate) + gate
     if w.mode == "ec":
-        n += 3                                # transpose, expert-choice select, gather
+        n += 2                                # transpose, expert-choice select
     else:
-        n += 4                                # histogram, scan, rank/scatter, gather
+        n += 2                                # scan, rank/scatter
         if w.capacity_factor <= 0 and w.keep_den > 0:
             n += 1                            # per-expert affinity select
+    n += 1                                    # row gather
     n += 2                                    # up- and down-projection GEMMs
     n += 1                                    # combine
     return n
@@ -95,23 +96,59 @@ def launches_per_step(w) -> int:
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and throttle reasons sampled during the timed region.
+
+    Reads NVML (what nvidia-smi reports) from a background thread every 2 ms,
+    falling back to an `nvidia-smi -lms 200` process.  Reading only: no
+    setting of the GPU is touched."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device: int):
-        self.proc = None
+    def __init__(self, device: int, period_s: float = 0.002):
+        import threading
+        self.samples, self.proc, self.nvml, self.thread = [], None, None, None
+        uuid = str(torch.cuda.get_device_properties(device).uuid)
+        self.sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         try:
-            uuid = str(torch.cuda.get_device_properties(device).uuid)
-            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", sel],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(self.sel)
+            self.stop_flag = threading.Event()
+
+            def run():
+                while not self.stop_flag.is_set():
+                    sm = pynvml.nvmlDeviceGetClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+                    why = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((sm, why))
+                    time.sleep(period_s)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
         except Exception:
-            self.proc = None
+            self.nvml = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                     "-lms", "200", "-i", self.sel],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except Exception:
+                self.proc = None
 
     def stop(self) -> dict | None:
+        if self.nvml is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=2)
+            mx = self.nvml.nvmlDeviceGetMaxClockInfo(self.h, self.nvml.NVML_CLOCK_SM)
+            if not self.samples:
+                return None
+            reasons = sorted({n for _, why in self.samples for b, n in self.REASONS.items() if why & b})
+            return {"sm_mhz": statistics.median(sm for sm, _ in self.samples), "sm_max_mhz": mx,
+                    "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -137,7 +174,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------
@@ -284,34 +321,27 @@ def run_ours(args, w) -> None:
         inp.x = torch.randn(w.T, w.d_model, generator=g, device="cuda").to(inp.x.dtype)
     cfg = api.config_from_workload(w)
     sizes = api.query_sizes(cfg)
-    B = api.step_buffers(cfg)
+    ws = api.new_workspace(cfg)
+    y = torch.empty_like(inp.x)
+    counts = torch.empty(w.E, dtype=torch.int32, device="cuda")
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        api.moe_route(cfg, inp.x, inp.w_router, inp.bias, B.logits, B.probs, B.topk_idx,
-                      B.topk_gate, B.ws)
-        if ev:
-            ev[1].record(stream)
-        api.moe_permute(cfg, inp.x, B.topk_idx, B.topk_gate, B.probs, B.counts, B.offsets,
-                        B.tok_rows, B.row_token, B.row_gate, B.x_perm, B.n_dropped, B.ws)
-        if ev:
-            ev[2].record(stream)
-        api.moe_expert_ffn(cfg, inp.x, B.x_perm, B.offsets, B.row_gate, inp.w1, inp.w3, inp.w2,
-                           B.h, B.y_rows, B.ws)
-        if ev:
-            ev[3].record(stream)
-        api.moe_combine(cfg, B.y_rows, B.tok_rows, B.y)
-        if ev:
-            ev[4].record(stream)
+        if ev is None:
+            api.moe_forward(cfg, inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, y, counts, ws)
+        else:
+            api.moe_forward_timed(cfg, inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, y,
+                                  counts, ws, ev)
 
     for _ in range(args.warmup):
         flush.zero_()
         step()
-    api.moe_check_device_errors(B.ws)
+    api.moe_check_device_errors(ws)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for row in evs:                           # create the CUDA events before handing them over
+        for ev in row:
+            ev.record(stream)
     clocks = ClockSampler(local)
     torch.cuda.synchronize()
     if dist:
@@ -323,7 +353,7 @@ def run_ours(args, w) -> None:
     if dist:
         dist.barrier()
     clk = clocks.stop()
-    api.moe_check_device_errors(B.ws)
+    api.moe_check_device_errors(ws)
 
     per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
                     for i in range(args.steps)])          # ms: route, permute, ffn, combine
@@ -335,8 +365,16 @@ def run_ours(args, w) -> None:
     ms_step = total_ms / args.steps
     value = world * w.T * args.steps / (total_ms / 1e3)
 
-    # algorithmic work of this batch
-    R = int(B.offsets[w.E].item())
+    # algorithmic work of this batch: kept routed rows from the counts
+    if w.mode == "ec":
+        R = w.E * w.ec_capacity
+    elif w.capacity_factor > 0:
+        C = api.capacity_for(w.T, w.E, w.k, w.capacity_factor)
+        R = int(torch.clamp(counts.long(), max=C).sum().item())
+    elif w.keep_den > 0:
+        R = int(((counts.long() * w.keep_num + w.keep_den - 1) // w.keep_den).sum().item())
+    else:
+        R = w.T * w.k
     es = 4 if w.dtype == "f32" else 2
     rows = R + w.S * w.T
     nmat = 3 if w.act == "swiglu" else 2

@@ -216,6 +216,16 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const void 
                        const float *bias, const void *w1, const void *w3, const void *w2, void *y,
                        int32_t *counts_out, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_forward that also records caller-created CUDA events on `stream` at
+ * its phase boundaries: events[0] before step 1, [1] after steps 1-3a
+ * (routing), [2] after 3b-4 (permutation), [3] after 5a-5b (expert FFNs),
+ * [4] after 5c (combine).  events: array of 5 cudaEvent_t handles (entries may
+ * be NULL).  Same launches and results as moe_forward. */
+MOE_API moe_status moe_forward_timed(const moe_config *cfg, const void *x, const void *w_router,
+                                     const float *bias, const void *w1, const void *w3,
+                                     const void *w2, void *y, int32_t *counts_out, void *ws,
+                                     size_t ws_bytes, void *const *events, moe_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the workspace's device error
  * word.  Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_CHECK; *flags (if
  * not NULL) receives the raw bits.  This is the only call that blocks. */

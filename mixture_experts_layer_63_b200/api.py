@@ -28,7 +28,7 @@ MOE_TOKEN_CHOICE, MOE_EXPERT_CHOICE = 0, 1
 
 EXPORTS = ("moe_query_sizes", "moe_route", "moe_gate", "moe_permute", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_check_device_errors", "moe_workspace_init",
-           "moe_status_string", "moe_permute_noalloc")
+           "moe_status_string", "moe_permute_noalloc", "moe_forward_timed")
 
 
 class MoeError(RuntimeError):
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
             "moe_expert_ffn": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_combine": [cfgp, vp, vp, vp, vp],
             "moe_forward": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_forward_timed": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                  ctypes.POINTER(ctypes.c_void_p), vp],
             "moe_check_device_errors": [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)],
             "moe_workspace_init": [vp, sz, vp],
         }
@@ -208,6 +210,18 @@ def moe_forward(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, stream=No
     _check("moe_forward", lib().moe_forward(
         ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y),
         _ptr(counts_out), wp, wn, _stream(stream)))
+
+
+def moe_forward_timed(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, events, stream=None):
+    """moe_forward recording 5 torch CUDA events at its phase boundaries
+    (before routing, after routing, after permutation, after the expert FFNs,
+    after the combine).  Each event must have been recorded once before, so
+    that its CUDA handle exists."""
+    wp, wn = _ws(ws)
+    handles = (ctypes.c_void_p * 5)(*[ev.cuda_event if ev is not None else None for ev in events])
+    _check("moe_forward_timed", lib().moe_forward_timed(
+        ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y),
+        _ptr(counts_out), wp, wn, handles, _stream(stream)))
 
 
 def moe_check_device_errors(ws, stream=None) -> int:

@@ -50,6 +50,9 @@ constexpr int kThreads = 256;
 constexpr int kAccCols = 256;       // TMEM columns per accumulator buffer
 constexpr int kTmemCols = 512;
 constexpr int kMaxGroups = 320;
+#ifndef MOE_PAIR_MIN_ROWS
+#define MOE_PAIR_MIN_ROWS 384
+#endif
 constexpr uint32_t kABytes = BM * BK * 2;   // 16 KB
 
 struct Params {
@@ -65,6 +68,8 @@ struct Params {
   void *out;
   const float *row_gate;
   const float *bias;
+  int ksplit;               // K split into this many parts (router only), partial outputs
+  int64_t split_stride;     //   ksplit parts of the output, split_stride elements apart
   uint32_t *err;
 };
 
@@ -200,6 +205,68 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+
+// ---- CTA pairs (cta_group::2): two CTAs of a cluster share one MMA ----------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+// shared::cluster address of the same offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+// TMA load into this CTA's shared memory, completing on the mbarrier at
+// `bar_cluster` (the even CTA's barrier of the pair)
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster,
+                                                 int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// arrive (once each) on the barrier at this offset in both CTAs of the pair
+// when the pair's MMAs issued so far complete
+__device__ __forceinline__ void umma_commit_pair_both(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"((uint16_t)0x3)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_pair_local(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
 // ------------------------------- tile schedule -------------------------------
 struct Tile {
   int g, m, n;
@@ -232,6 +299,78 @@ __device__ __forceinline__ void store_bf16x32(void *dst, const float (&v)[32]) {
     w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
     w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
     p[q] = w;
+  }
+}
+
+// Epilogue of one accumulator: this thread's row (TMEM lane) of the tile,
+// BN columns from TMEM address `taddr`; activation / gate / bias, stores.
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, bool valid, bool routed,
+                                              int64_t out_row, int col0, int64_t out_offset = 0) {
+  uint32_t r[32];
+  float v[32];
+  if (EPI == kEpiSwiglu) {
+    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
+#pragma unroll 1
+    for (int c = 0; c < 128 / 32; ++c) {
+      uint32_t u[32];
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld32(taddr + 128 + c * 32, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float g = __uint_as_float(r[i]);
+        v[i] = g / (1.0f + __expf(-g)) * __uint_as_float(u[i]);
+      }
+      const int col = col0 + c * 32;
+      if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
+    }
+  } else if (EPI == kEpiRelu) {
+    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
+#pragma unroll 1
+    for (int c = 0; c < P.bn / 32; ++c) {
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = fmaxf(__uint_as_float(r[i]), 0.0f);
+      const int col = col0 + c * 32;
+      if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
+    }
+  } else if (EPI == kEpiScale) {
+    // fp32 rows: the combine rounds once, after summing
+    float *out = reinterpret_cast<float *>(P.out);
+    const float scale = (routed && valid) ? P.row_gate[out_row] : 1.0f;
+#pragma unroll 1
+    for (int c = 0; c < P.bn / 32; ++c) {
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+      const int col = col0 + c * 32;
+      if (valid && col < P.N) {
+        float4 *dst = reinterpret_cast<float4 *>(out + out_row * P.N + col);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          dst[q] = make_float4(__uint_as_float(r[4 * q]) * scale, __uint_as_float(r[4 * q + 1]) * scale,
+                               __uint_as_float(r[4 * q + 2]) * scale, __uint_as_float(r[4 * q + 3]) * scale);
+      }
+    }
+  } else {  // kEpiStoreF32 (a K part when the router is split: no bias, own output)
+    float *out = reinterpret_cast<float *>(P.out) + out_offset;
+    const float *bias = P.ksplit > 1 ? nullptr : P.bias;
+#pragma unroll 1
+    for (int c = 0; c < P.bn / 32; ++c) {
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+      if (valid) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int col = col0 + c * 32 + i;
+          if (col < P.N) {
+            const float a = __uint_as_float(r[i]);
+            out[out_row * P.N + col] = bias ? a + bias[col] : a;
+          }
+        }
+      }
+    }
   }
 }
 
@@ -325,8 +464,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
 
   const uint32_t tmem_base = s_tmem_base;
-  const int total = s_prefix[P.G];
+  const int base_total = s_prefix[P.G];
+  const int total = base_total * P.ksplit;          // K parts (router split) x tiles
   const int KB = P.K / BK;
+  const int KBs = (KB + P.ksplit - 1) / P.ksplit;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -336,14 +477,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t armed_parity = 0;     // bit s: parity of that phase
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      const int part = tile / base_total;
+      const Tile tl = decode_tile(tile - part * base_total, s_prefix, P.G, P.nt);
+      const int kb0 = part * KBs, kb1 = min(KB, kb0 + KBs);
       const bool routed = tl.g < P.n_routed;
       const int64_t a_row = routed ? (int64_t)s_off[tl.g] + (int64_t)tl.m * BM
                                    : P.a_static_base + (int64_t)(tl.g - P.n_routed) * P.a_static_stride +
                                          (int64_t)tl.m * BM;
       const CUtensorMap *ma = routed ? &map_a : &map_a_static;
       const int b_row = tl.g * P.N + tl.n * P.bnh;
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
         uint8_t *sa = smem + (size_t)stage * stage_bytes;
         uint8_t *sb = sa + kABytes;
@@ -374,10 +517,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const int part = tile / base_total;
+      const int kb0 = part * KBs, kb1 = min(KB, kb0 + KBs);
       if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&full_bar[stage], phase, &s_abort, P.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + (size_t)stage * stage_bytes);
@@ -385,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < BK / kUmmaK; ++k) {
           umma_bf16(d_tmem, sw128_desc(a_addr + k * kUmmaK * 2), sw128_desc(b_addr + k * kUmmaK * 2),
-                    idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                    idesc, (kb > kb0 || k > 0) ? 1u : 0u);
         }
         umma_commit(&empty_bar[stage]);
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -403,7 +548,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      const int part = tile / base_total;
+      const Tile tl = decode_tile(tile - part * base_total, s_prefix, P.G, P.nt);
       if (!mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err)) break;
       tc_fence_after();
       const bool routed = tl.g < P.n_routed;
@@ -414,70 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                               (int64_t)tl.m * BM + r_in;
       const int col0 = tl.n * P.bnh;
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
-      uint32_t r[32];
-      float v[32];
-      if (EPI == kEpiSwiglu) {
-        __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
-#pragma unroll 1
-        for (int c = 0; c < 128 / 32; ++c) {
-          uint32_t u[32];
-          tmem_ld32(taddr + c * 32, r);
-          tmem_ld32(taddr + 128 + c * 32, u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float g = __uint_as_float(r[i]);
-            v[i] = g / (1.0f + __expf(-g)) * __uint_as_float(u[i]);
-          }
-          const int col = col0 + c * 32;
-          if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
-        }
-      } else if (EPI == kEpiRelu) {
-        __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
-#pragma unroll 1
-        for (int c = 0; c < P.bn / 32; ++c) {
-          tmem_ld32(taddr + c * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = fmaxf(__uint_as_float(r[i]), 0.0f);
-          const int col = col0 + c * 32;
-          if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
-        }
-      } else if (EPI == kEpiScale) {
-        // fp32 rows: the combine rounds once, after summing
-        float *out = reinterpret_cast<float *>(P.out);
-        const float scale = (routed && valid) ? P.row_gate[out_row] : 1.0f;
-#pragma unroll 1
-        for (int c = 0; c < P.bn / 32; ++c) {
-          tmem_ld32(taddr + c * 32, r);
-          tmem_ld_wait();
-          const int col = col0 + c * 32;
-          if (valid && col < P.N) {
-            float4 *dst = reinterpret_cast<float4 *>(out + out_row * P.N + col);
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              dst[q] = make_float4(__uint_as_float(r[4 * q]) * scale, __uint_as_float(r[4 * q + 1]) * scale,
-                                   __uint_as_float(r[4 * q + 2]) * scale, __uint_as_float(r[4 * q + 3]) * scale);
-          }
-        }
-      } else {  // kEpiStoreF32
-        float *out = reinterpret_cast<float *>(P.out);
-#pragma unroll 1
-        for (int c = 0; c < P.bn / 32; ++c) {
-          tmem_ld32(taddr + c * 32, r);
-          tmem_ld_wait();
-          if (valid) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int col = col0 + c * 32 + i;
-              if (col < P.N) {
-                const float a = __uint_as_float(r[i]);
-                out[out_row * P.N + col] = P.bias ? a + P.bias[col] : a;
-              }
-            }
-          }
-        }
-      }
+      epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, (int64_t)part * P.split_stride);
       tc_fence_before();
       mbar_arrive(&acce_bar[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -489,6 +572,214 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (warp == 2) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols));
+  }
+}
+
+
+// ------------------------- the kernel, CTA-pair version -----------------------
+// Same contract as grouped_gemm_kernel, tiles of 256 rows: the two CTAs of a
+// cluster each stage 128 rows of A and half of the B tile (BN/2 rows) per
+// k-block, and the even CTA issues tcgen05.mma.cta_group::2 (M = 256), which
+// reads both CTAs' shared memory and leaves rows 0-127 of the accumulator in
+// the even CTA's TMEM and rows 128-255 in the odd CTA's.  Each CTA moves 32 KB
+// per k-block instead of 48 KB for the same MMA work.  Both CTAs' TMA loads
+// complete on the even CTA's full barrier; the MMA commits arrive on the
+// empty / accumulator-full barriers of both CTAs; both CTAs' epilogues arrive
+// on the even CTA's accumulator-empty barrier.  No load is multicast.
+constexpr int kPairStages = 6;
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
+                             const __grid_constant__ CUtensorMap map_a_static,
+                             const __grid_constant__ CUtensorMap map_b,
+                             const __grid_constant__ CUtensorMap map_b3, const Params P) {
+  constexpr int PM = 2 * BM;                         // rows per pair tile
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ int s_prefix[kMaxGroups + 1];
+  __shared__ int s_off[kMaxGroups];
+  __shared__ int s_rows[kMaxGroups];
+  __shared__ __align__(8) uint64_t full_bar[kPairStages];
+  __shared__ __align__(8) uint64_t empty_bar[kPairStages];
+  __shared__ __align__(8) uint64_t accf_bar[2];
+  __shared__ __align__(8) uint64_t acce_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ volatile int s_abort;
+
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~(uintptr_t)1023);
+  const uint32_t b_bytes = (uint32_t)(P.bn / 2) * BK * 2;       // this CTA's half of B
+  const uint32_t stage_bytes = kABytes + b_bytes;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 0; base < P.G; base += 32) {
+      const int g = base + lane;
+      int tiles = 0;
+      if (g < P.G) {
+        int off = 0, rows = 0;
+        if (g < P.n_routed) {
+          off = P.offsets[g];
+          rows = P.offsets[g + 1] - off;
+          if (rows < 0 || off < 0 || (int64_t)off + rows > P.a_rows) {
+            raise_error(P.err, kErrBadIndex);
+            rows = 0;
+            off = 0;
+          }
+        } else {
+          rows = (int)P.rows_static;
+        }
+        s_off[g] = off;
+        s_rows[g] = rows;
+        tiles = ((rows + PM - 1) / PM) * P.nt;
+      }
+      int x = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (g < P.G) s_prefix[g] = carry + x - tiles;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) s_prefix[P.G] = carry;
+  }
+  if (tid == 32) {
+    for (int st = 0; st < kPairStages; ++st) {
+      mbar_init(&full_bar[st], 1);
+      mbar_init(&empty_bar[st], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accf_bar[a], 1);
+      mbar_init(&acce_bar[a], 2 * 4 * 32);
+    }
+    mbar_init(&drain_bar, 1);
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  if (tid == 0) {
+    tma_prefetch_map(&map_a);
+    tma_prefetch_map(&map_b);
+    if (P.n_static > 0) tma_prefetch_map(&map_a_static);
+    if (EPI == kEpiSwiglu) tma_prefetch_map(&map_b3);
+  }
+  tc_fence_before();
+  cluster_sync_all();              // barriers of both CTAs initialised before any remote use
+  tc_fence_after();
+
+  const uint32_t tmem_base = s_tmem_base;
+  const int total = s_prefix[P.G];
+  const int KB = P.K / BK;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0, armed_parity = 0;
+    bool ok = true;
+    for (int tile = pair; tile < total && ok; tile += npairs) {
+      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      const bool routed = tl.g < P.n_routed;
+      const int64_t a_row = (routed ? (int64_t)s_off[tl.g]
+                                    : P.a_static_base + (int64_t)(tl.g - P.n_routed) * P.a_static_stride) +
+                            (int64_t)tl.m * PM + (int64_t)rank * BM;
+      const CUtensorMap *ma = routed ? &map_a : &map_a_static;
+      // B rows of this CTA: SwiGLU: even CTA the gate rows (W1), odd CTA the up
+      // rows (W3); otherwise the two halves of the BN-row tile
+      const CUtensorMap *mb = (EPI == kEpiSwiglu && rank == 1) ? &map_b3 : &map_b;
+      const int b_row = tl.g * P.N + tl.n * P.bnh + ((EPI == kEpiSwiglu) ? 0 : (int)rank * (P.bn / 2));
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+        uint8_t *sa = smem + (size_t)stage * stage_bytes;
+        uint8_t *sb = sa + kABytes;
+        const uint32_t fb = smem_u32(&full_bar[stage]) & 0xFEFFFFFFu;   // the even CTA's barrier
+        if (rank == 0) {
+          mbar_expect_tx(&full_bar[stage], 2 * stage_bytes);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        }
+        tma_load_2d_pair(sa, ma, fb, kb * BK, (int)a_row);
+        tma_load_2d_pair(sb, mb, fb, kb * BK, b_row);
+        if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (!ok && rank == 0) {
+      for (int st = 0; st < kPairStages; ++st)
+        if (armed & (1u << st)) mbar_wait_drain(&full_bar[st], (armed_parity >> st) & 1u);
+    }
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------ MMA issuer (even CTA only) ------------------------
+    const uint32_t idesc = idesc_bf16(PM, P.bn);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = pair; tile < total && ok; tile += npairs) {
+      if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&full_bar[stage], phase, &s_abort, P.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + (size_t)stage * stage_bytes);
+        const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+        for (int k = 0; k < BK / kUmmaK; ++k) {
+          umma_bf16_pair(d_tmem, sw128_desc(a_addr + k * kUmmaK * 2),
+                         sw128_desc(b_addr + k * kUmmaK * 2), idesc, (kb > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit_pair_both(&empty_bar[stage]);
+        if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      umma_commit_pair_both(&accf_bar[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    umma_commit_pair_local(&drain_bar);
+    mbar_wait_drain(&drain_bar, 0);
+  } else if (warp >= 4) {
+    // -------------------------------- epilogue --------------------------------
+    const int ew = warp - 4;
+    const uint32_t acce_even0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
+    const uint32_t acce_even1 = mapa_shared(smem_u32(&acce_bar[1]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < total; tile += npairs) {
+      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      if (!mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err)) break;
+      tc_fence_after();
+      const bool routed = tl.g < P.n_routed;
+      const int r_in = (int)rank * BM + ew * 32 + lane;
+      const bool valid = tl.m * PM + r_in < s_rows[tl.g];
+      const int64_t out_row = (routed ? (int64_t)s_off[tl.g]
+                                      : P.out_static_base + (int64_t)(tl.g - P.n_routed) * P.rows_static) +
+                              (int64_t)tl.m * PM + r_in;
+      const int col0 = tl.n * P.bnh;
+      const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
+      epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0);
+      tc_fence_before();
+      mbar_arrive_cluster(acc == 0 ? acce_even0 : acce_even1);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();              // neither CTA leaves while the pair may still touch it
+  tc_fence_after();
+  if (warp == 2) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(kTmemCols));
   }
 }
@@ -545,6 +836,37 @@ cudaError_t launch_epi(const GroupedGemm &g, const Params &P, const CUtensorMap 
   return cudaGetLastError();
 }
 
+// CTA-pair launch: as many 2-CTA clusters as fit at once (one CTA per SM),
+// fewer when there are fewer tiles.
+template <int EPI>
+cudaError_t launch_pair(const Params &P, const CUtensorMap &ma, const CUtensorMap &mas,
+                        const CUtensorMap &mb, const CUtensorMap &mb3, int64_t max_tiles,
+                        size_t smem, cudaStream_t s) {
+  auto kern = grouped_gemm_pair_kernel<EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  static int max_clusters[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int &mc = max_clusters[dev & 7];
+  if (mc == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = device_sms() / 2;
+    }
+    mc = n;
+  }
+  const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(mc, max_tiles));
+  kern<<<2 * pairs, kThreads, smem, s>>>(ma, mas, mb, mb3, P);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
@@ -575,11 +897,18 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   P.out = g.out;
   P.row_gate = g.row_gate;
   P.bias = g.bias;
+  P.ksplit = std::max(1, g.ksplit);
+  P.split_stride = g.split_stride;
   P.err = g.err;
   if (P.G <= 0 || P.G > kMaxGroups || P.bn > 256 || g.K % BK != 0) return cudaErrorInvalidValue;
+  if (g.ksplit > 1 && (g.epi != kEpiStoreF32 || g.n_routed != 0)) return cudaErrorInvalidValue;
 
+  // CTA pairs for the expert GEMMs whose groups are long enough that 256-row
+  // tiles waste little (average routed rows per expert >= MOE_PAIR_MIN_ROWS)
+  const bool pair = g.epi != kEpiStoreF32 && g.n_routed > 0 && P.bn == 256 &&
+                    g.max_routed_rows / g.n_routed >= MOE_PAIR_MIN_ROWS;
   CUtensorMap ma, mas, mb, mb3;
-  const uint32_t box_b = (g.epi == kEpiSwiglu) ? 128u : (uint32_t)P.bn;
+  const uint32_t box_b = (g.epi == kEpiSwiglu || pair) ? 128u : (uint32_t)P.bn;
   if (!make_map(&ma, g.a, (uint64_t)g.K, (uint64_t)g.a_rows, BM)) return cudaErrorInvalidValue;
   if (!make_map(&mas, g.a_static ? g.a_static : g.a, (uint64_t)g.K,
                 (uint64_t)(g.a_static ? g.a_static_rows : g.a_rows), BM))
@@ -591,12 +920,24 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   // grid: one CTA per SM, fewer when there are fewer tiles
   const int64_t mt_routed = (g.max_routed_rows + BM - 1) / BM + g.n_routed;
   const int64_t mt_static = (int64_t)g.n_static * ((g.rows_static + BM - 1) / BM);
-  const int64_t max_tiles = (mt_routed + mt_static) * P.nt;
+  const int64_t max_tiles = (mt_routed + mt_static) * P.nt * P.ksplit;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(device_sms(), max_tiles));
   // at least 120 KB so that one CTA (and one 512-column TMEM allocation) fits per SM
   const size_t smem = std::max<size_t>((size_t)kStages * (kABytes + (size_t)P.bn * BK * 2) + 1024,
                                        (size_t)120 * 1024);
 
+  if (pair) {
+    const int64_t pt_routed = (g.max_routed_rows + 2 * BM - 1) / (2 * BM) + g.n_routed;
+    const int64_t pt_static = (int64_t)g.n_static * ((g.rows_static + 2 * BM - 1) / (2 * BM));
+    const int64_t pair_tiles = (pt_routed + pt_static) * P.nt;
+    const size_t psmem = (size_t)kPairStages * (kABytes + (size_t)(P.bn / 2) * BK * 2) + 1024;
+    switch (g.epi) {
+      case kEpiRelu: return launch_pair<kEpiRelu>(P, ma, mas, mb, mb3, pair_tiles, psmem, s);
+      case kEpiSwiglu: return launch_pair<kEpiSwiglu>(P, ma, mas, mb, mb3, pair_tiles, psmem, s);
+      case kEpiScale: return launch_pair<kEpiScale>(P, ma, mas, mb, mb3, pair_tiles, psmem, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (g.epi) {
     case kEpiStoreF32: return launch_epi<kEpiStoreF32>(g, P, ma, mas, mb, mb3, grid, smem, s);
     case kEpiRelu: return launch_epi<kEpiRelu>(g, P, ma, mas, mb, mb3, grid, smem, s);

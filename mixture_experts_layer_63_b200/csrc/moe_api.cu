@@ -62,7 +62,8 @@ WsLayout make_layout(const moe_config *c) {
   L.rows_cap = tc ? T * k : (int64_t)E * c->ec_capacity;
   L.rows_total = L.rows_cap + (int64_t)S * T;
   L.tok_rows_len = tc ? T * k : (int64_t)E * T;
-  L.nblk = tc ? (int)((T * k + kAssignBlock - 1) / kAssignBlock) : 0;
+  L.nunit = (int)((T + kUnitTokens - 1) / kUnitTokens);
+  const int64_t hist_ints = tc ? (int64_t)k * L.nunit * E : 0;
   const bool keepfrac = tc && c->capacity <= 0 && c->keep_den > 0;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -71,12 +72,15 @@ WsLayout make_layout(const moe_config *c) {
     return at;
   };
   L.err = take(256);
-  L.hist = take((size_t)L.nblk * E * 4);
-  L.base = take((size_t)L.nblk * E * 4);
+  L.hist = take((size_t)hist_ints * 4);
+  L.base = take((size_t)(tc ? (k * L.nunit + 31) / 32 * E : 0) * 4);   // per-block unit totals
   L.cnt_off = take((size_t)(E + 1) * 4);
   L.kept = take((size_t)E * 4);
   L.sorted_q = take(keepfrac ? (size_t)T * k * 4 : 0);
   L.probs_t = take(tc ? 0 : (size_t)E * T * 4);
+  L.permute_end = o;
+  const int ks = (c->dtype == MOE_BF16 && !router_is_fused(c)) ? router_ksplit(c) : 1;
+  L.logits_part = take(ks > 1 ? (size_t)ks * T * E * 4 : 0);
   L.step_end = o;
   L.logits = take((size_t)T * E * 4);
   L.probs = take((size_t)T * E * 4);
@@ -111,6 +115,10 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 static cudaError_t run_route(const moe_config *c, const WsLayout &L, char *ws, const void *x,
                              const void *w_router, const float *bias, float *logits, float *probs,
                              int32_t *topk_idx, float *topk_gate, cudaStream_t s) {
+  int32_t *hist = c->mode == MOE_TOKEN_CHOICE ? reinterpret_cast<int32_t *>(ws + L.hist) : nullptr;
+  if (router_is_fused(c))
+    return launch_route_gate(c, nullptr, logits, x, w_router, bias, probs, topk_idx, topk_gate,
+                             hist, s);
   cudaError_t e;
   if (c->dtype == MOE_F32) {
     e = launch_router_f32(c, static_cast<const float *>(x), static_cast<const float *>(w_router),
@@ -135,13 +143,26 @@ static cudaError_t run_route(const moe_config *c, const WsLayout &L, char *ws, c
     g.a_static_stride = 0;
     g.out_static_base = 0;
     g.max_routed_rows = 0;
+    g.err = reinterpret_cast<uint32_t *>(ws + L.err);
+    const int ks = router_ksplit(c);
+    if (ks > 1) {
+      // K split over more CTAs; the gate adds the parts in order, then the bias
+      float *parts = reinterpret_cast<float *>(ws + L.logits_part);
+      g.out = parts;
+      g.ksplit = ks;
+      g.split_stride = c->T * c->E;
+      e = launch_grouped_gemm(g, s);
+      if (e != cudaSuccess) return e;
+      return launch_route_gate(c, parts, logits, nullptr, nullptr, bias, probs, topk_idx, topk_gate,
+                               hist, s, ks, c->T * c->E);
+    }
     g.out = logits;
     g.bias = bias;
-    g.err = reinterpret_cast<uint32_t *>(ws + L.err);
     e = launch_grouped_gemm(g, s);
   }
   if (e != cudaSuccess) return e;
-  return launch_gate(c, logits, probs, topk_idx, topk_gate, s);
+  return launch_route_gate(c, logits, nullptr, nullptr, nullptr, nullptr, probs, topk_idx,
+                           topk_gate, hist, s);
 }
 
 static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, const void *x,
@@ -247,8 +268,9 @@ moe_status moe_gate(const moe_config *cfg, const float *logits, float *probs, in
   if ((st = check_ws(L, ws, ws_bytes, L.step_end)) != MOE_OK) return st;
   const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
   if (!logits || !probs || (tc && (!topk_idx || !topk_gate))) return MOE_ERR_INVALID_ARG;
-  return cuda_status(
-      launch_gate(cfg, logits, probs, topk_idx, topk_gate, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_route_gate(cfg, logits, nullptr, nullptr, nullptr, nullptr, probs,
+                                       topk_idx, topk_gate, nullptr,
+                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *topk_idx,
@@ -266,7 +288,7 @@ moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *topk
   if (tc && (!topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
   if ((!tc || keepfrac) && !probs) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_permute(cfg, L, static_cast<char *>(ws), x, topk_idx, topk_gate, probs,
+  return cuda_status(launch_permute(cfg, L, static_cast<char *>(ws), false, x, topk_idx, topk_gate, probs,
                                     counts, offsets, tok_rows, row_token, row_gate, x_perm,
                                     n_dropped, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -300,9 +322,10 @@ moe_status moe_combine(const moe_config *cfg, const void *y_rows, const int32_t 
                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
-moe_status moe_forward(const moe_config *cfg, const void *x, const void *w_router,
-                       const float *bias, const void *w1, const void *w3, const void *w2, void *y,
-                       int32_t *counts_out, void *ws, size_t ws_bytes, moe_stream_t stream) {
+static moe_status forward_impl(const moe_config *cfg, const void *x, const void *w_router,
+                               const float *bias, const void *w1, const void *w3, const void *w2,
+                               void *y, int32_t *counts_out, void *ws, size_t ws_bytes,
+                               void *const *events, moe_stream_t stream) {
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const WsLayout L = make_layout(cfg);
@@ -327,16 +350,42 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const void *w_route
   void *x_perm = w + L.x_perm;
   void *h = w + L.h;
   void *y_rows = w + L.y_rows;
-  cudaError_t e = run_route(cfg, L, w, x, w_router, bias, logits, probs, topk_idx, topk_gate, s);
+  auto mark = [&](int i) -> cudaError_t {
+    if (events && events[i]) return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s);
+    return cudaSuccess;
+  };
+  cudaError_t e = mark(0);
   if (e == cudaSuccess)
-    e = launch_permute(cfg, L, w, x, topk_idx, topk_gate, probs, counts, offsets, tok_rows,
-                       row_token, row_gate, x_perm, n_dropped, s);
+    e = run_route(cfg, L, w, x, w_router, bias, logits, probs, topk_idx, topk_gate, s);
+  if (e == cudaSuccess) e = mark(1);
+  // token choice: the gate wrote the unit histogram into the workspace
+  if (e == cudaSuccess)
+    e = launch_permute(cfg, L, w, cfg->mode == MOE_TOKEN_CHOICE, x, topk_idx, topk_gate, probs,
+                       counts, offsets, tok_rows, row_token, row_gate, x_perm, n_dropped, s);
+  if (e == cudaSuccess) e = mark(2);
   if (e == cudaSuccess)
     e = run_ffn(cfg, L, w, x, x_perm, offsets, row_gate, w1, w3, w2, h, y_rows, s);
+  if (e == cudaSuccess) e = mark(3);
   if (e == cudaSuccess) e = launch_combine(cfg, L.rows_cap, y_rows, tok_rows, y, s);
+  if (e == cudaSuccess) e = mark(4);
   if (e == cudaSuccess && counts_out)
     e = cudaMemcpyAsync(counts_out, counts, (size_t)cfg->E * 4, cudaMemcpyDeviceToDevice, s);
   return cuda_status(e);
+}
+
+moe_status moe_forward(const moe_config *cfg, const void *x, const void *w_router,
+                       const float *bias, const void *w1, const void *w3, const void *w2, void *y,
+                       int32_t *counts_out, void *ws, size_t ws_bytes, moe_stream_t stream) {
+  return forward_impl(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, ws_bytes, nullptr,
+                      stream);
+}
+
+moe_status moe_forward_timed(const moe_config *cfg, const void *x, const void *w_router,
+                             const float *bias, const void *w1, const void *w3, const void *w2,
+                             void *y, int32_t *counts_out, void *ws, size_t ws_bytes,
+                             void *const *events, moe_stream_t stream) {
+  return forward_impl(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, ws_bytes, events,
+                      stream);
 }
 
 moe_status moe_check_device_errors(void *ws, size_t ws_bytes, moe_stream_t stream, uint32_t *flags) {

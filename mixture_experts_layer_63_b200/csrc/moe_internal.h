@@ -10,29 +10,35 @@
 
 namespace moe {
 
-// Assignments per histogram block of the token-choice counting sort.
-constexpr int kAssignBlock = 2048;
+// Tokens per unit of the token-choice counting sort (one warp per unit).
+constexpr int kUnitTokens = 32;
 // Upper bound on routed experts and on top-k handled by the kernels.
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;
+// The router runs inside the gate kernel when E <= 32 and W_r, widened to
+// fp32, fits this many bytes of shared memory; otherwise the tcgen05 GEMM
+// (bf16) or a CUDA-core kernel (fp32) computes the logits first.
+constexpr size_t kFusedRouterSmem = 160 * 1024;
 
 // Byte offsets into the caller's workspace.  The first region (error word +
 // step scratch) is what the step entry points use; moe_forward adds its
 // intermediates after it.
 struct WsLayout {
   size_t err;        // uint32 error word (256 B reserved)
-  size_t hist;       // int32 [nblk * E]   per-block expert histogram
-  size_t base;       // int32 [nblk * E]   exclusive scan over blocks
+  size_t hist;       // int32 [k * nunit * E]  per-unit expert histogram
+  size_t base;       // int32 [ceil(k * nunit / 32) * E]  per-expert totals of 32-unit blocks
   size_t cnt_off;    // int32 [E + 1]      exclusive scan of counts
   size_t kept;       // int32 [E]          rows kept per expert
   size_t sorted_q;   // int32 [T * k]      assignments grouped by expert (keep-fraction)
   size_t probs_t;    // fp32  [E * T]      transposed probabilities (expert choice)
+  size_t permute_end;    // end of the permutation's scratch
+  size_t logits_part;    // fp32 [ksplit][T][E] partial router logits (bf16 router with split K)
   size_t step_end;
   // moe_forward intermediates
   size_t logits, probs, topk_idx, topk_gate, counts, offsets, n_dropped;
   size_t tok_rows, row_token, row_gate, x_perm, h, y_rows;
   size_t total;
-  int nblk;          // histogram blocks
+  int nunit;         // 32-token units: ceil(T / 32)
   int64_t rows_cap, rows_total, tok_rows_len;
 };
 
@@ -42,15 +48,25 @@ WsLayout make_layout(const moe_config *c);
 inline size_t elem_size(const moe_config *c) { return c->dtype == MOE_F32 ? 4 : 2; }
 
 // --- router / gate (router_gate.cu) ---------------------------------------
+// true when the gate kernel computes the logits itself (small E)
+bool router_is_fused(const moe_config *c);
+// Gate (+ histogram for token choice).  logits_in == null: fused router from
+// x and w_router, writing logits_out; else gate on the given logits.
+// logits_in may hold nsplit partial sums split_stride floats apart (summed in
+// order, then + bias when bias is given).
+cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float *logits_out,
+                              const void *x, const void *w_router, const float *bias, float *probs,
+                              int32_t *topk_idx, float *topk_gate, int32_t *hist, cudaStream_t s,
+                              int nsplit = 1, int64_t split_stride = 0);
+// fp32 logits on CUDA cores for fp32 layers the fused router does not cover
 cudaError_t launch_router_f32(const moe_config *c, const float *x, const float *w, const float *bias,
                               float *logits, cudaStream_t s);
-cudaError_t launch_gate(const moe_config *c, const float *logits, float *probs, int32_t *topk_idx,
-                        float *topk_gate, cudaStream_t s);
 
 // --- permutation (permute.cu) ---------------------------------------------
-cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, const void *x,
-                           const int32_t *topk_idx, const float *topk_gate, const float *probs,
-                           int32_t *counts, int32_t *offsets, int32_t *tok_rows,
+// hist_ready: the gate already wrote the unit histogram into the workspace
+cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, bool hist_ready,
+                           const void *x, const int32_t *topk_idx, const float *topk_gate,
+                           const float *probs, int32_t *counts, int32_t *offsets, int32_t *tok_rows,
                            int32_t *row_token, float *row_gate, void *x_perm, int32_t *n_dropped,
                            cudaStream_t s);
 
@@ -87,11 +103,21 @@ struct GroupedGemm {
   int64_t max_routed_rows;  // host upper bound of offsets[n_routed] (grid sizing)
   void *out;                // [*, N] row-major, ld = N
   const float *row_gate;    // kEpiScale: gate per routed output row
-  const float *bias;        // kEpiStoreF32: [N] or null
+  const float *bias;        // kEpiStoreF32: [N] or null (ignored when ksplit > 1)
+  int ksplit;               // kEpiStoreF32, one static group: split K into ksplit parts and
+  int64_t split_stride;     //   write part s of the output at out + s * split_stride
   uint32_t *err;
 };
 cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s);
-
+// K parts of the bf16 router GEMM: enough CTAs to fill the GPU, >= 4 k-blocks each
+inline int router_ksplit(const moe_config *c) {
+  const int64_t mtiles = (c->T + 127) / 128;
+  const int kb = c->d_model / 64;
+  int ks = (int)(148 / mtiles);
+  if (ks > 4) ks = 4;
+  while (ks > 1 && kb / ks < 4) --ks;
+  return ks < 1 ? 1 : ks;
+}
 // --- fp32 CUDA-core expert FFN (ffn_f32.cu) ----------------------------------
 cudaError_t launch_ffn_f32(const moe_config *c, const WsLayout &L, uint32_t *err, const float *x,
                            const float *x_perm,

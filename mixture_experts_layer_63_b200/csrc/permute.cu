@@ -4,13 +4,16 @@
 // Token choice (GShard section 1 of "MoE技术演进": expert capacity C = O(N/E),
 // overflow passes through the residual): a stable counting sort of the
 // assignments by expert, in priority order q = j*T + t (every first choice
-// before any second choice, lower token first):
-//   hist_kernel   per-block expert histogram over q
-//   scan_kernel   per-expert exclusive scan over blocks, counts, kept rows
-//                 (min(n_e, C), or ceil(n_e*num/den)) and row offsets
-//   rank_kernel   stable rank of each assignment inside its expert (warp
-//                 match + per-warp prefix), then the capacity test and the
-//                 slot / row writes -- or, for keep-fraction, the grouped list
+// before any second choice, lower token first), in units of 32 tokens:
+//   hist_units    per-unit expert histogram (the gate kernel writes it when
+//                 it runs first, so moe_forward skips this launch)
+//   unit_sums     per-expert totals of each block of 32 units
+//   rank_units    per block: bases from the earlier blocks' totals and an
+//                 in-block scan, counts / kept rows (min(n_e, C) or
+//                 ceil(n_e*num/den)) / row offsets; then the stable rank of
+//                 each assignment inside its expert (warp match within the
+//                 unit), the capacity test and the slot / row writes -- or,
+//                 for keep-fraction, the expert-grouped list
 //   keep_select   per expert, the ceil(n_e*num/den) assignments with the
 //                 largest p[t, e] (DeepSeek-V2 section 5, token dropping)
 // Expert choice (LocMoE+ article: each expert picks its top-C tokens):
@@ -20,7 +23,9 @@
 // Both selections use an exact radix select over the 64-bit key
 // (p bits << 32 | ~t), so "larger p first, lower t on ties" is decided by
 // integer comparisons alone.
-//   gather_rows   x_perm[r] = x[row_token[r]], 16-byte vectors.
+//   gather_rows   x_perm[r] = x[row_token[r]], one warp per row, 16-byte
+//                 vectors.
+#include <algorithm>
 #include <mutex>
 
 #include "device_common.cuh"
@@ -29,130 +34,230 @@
 namespace moe {
 
 // ---------------------------------------------------------------------------
-// token choice: histogram
+// row gather: x_perm[r] = x[row_token[r]] for r < offsets[E], one warp per
+// row (grid-stride), 16-byte vectors, four loads in flight per lane.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) hist_kernel(const int32_t *__restrict__ topk_idx, int64_t T,
-                                                   int k, int E, int32_t *__restrict__ hist,
-                                                   uint32_t *err) {
-  __shared__ int h[kMaxExperts];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
-  __syncthreads();
-  const int64_t Q = T * k;
-  const int64_t q0 = (int64_t)blockIdx.x * kAssignBlock;
-  const int64_t q1 = min(q0 + kAssignBlock, Q);
-  for (int64_t q = q0 + threadIdx.x; q < q1; q += blockDim.x) {
-    const int64_t j = q / T, t = q - j * T;
-    const int e = topk_idx[t * k + j];
-    if (e < 0 || e >= E) { raise_error(err, kErrBadIndex); continue; }
-    atomicAdd(&h[e], 1);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = h[e];
-}
-
-// ---------------------------------------------------------------------------
-// token choice: scans
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) scan_kernel(const int32_t *__restrict__ hist, int nblk, int E,
-                                                   int64_t Q, int capacity, int keep_num,
-                                                   int keep_den, int32_t *__restrict__ base,
-                                                   int32_t *__restrict__ counts,
-                                                   int32_t *__restrict__ cnt_off,
-                                                   int32_t *__restrict__ kept,
-                                                   int32_t *__restrict__ offsets,
-                                                   int32_t *__restrict__ n_dropped) {
-  __shared__ int s_cnt[kMaxExperts];
-  __shared__ int s_kept[kMaxExperts];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = 0;
-    for (int b = 0; b < nblk; ++b) {
-      base[(int64_t)b * E + e] = run;
-      run += hist[(int64_t)b * E + e];
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restrict__ x,
+                                                          uint4 *__restrict__ x_perm,
+                                                          const int32_t *__restrict__ row_token,
+                                                          const int32_t *__restrict__ offsets, int E,
+                                                          int64_t T, int vpr, uint32_t *err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t R = offsets[E];
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += nwarps) {
+    const int64_t t = row_token[r];
+    if (t < 0 || t >= T) {
+      if (lane == 0) raise_error(err, kErrBadIndex);
+      continue;
     }
-    int kp = run;
-    if (capacity > 0) kp = min(run, capacity);
-    else if (keep_den > 0) kp = (int)(((int64_t)run * keep_num + keep_den - 1) / keep_den);
-    s_cnt[e] = run;
-    s_kept[e] = kp;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int a = 0, b = 0;
-    for (int e = 0; e < E; ++e) {
-      cnt_off[e] = a;
-      offsets[e] = b;
-      counts[e] = s_cnt[e];
-      kept[e] = s_kept[e];
-      a += s_cnt[e];
-      b += s_kept[e];
+    const uint4 *src = x + t * vpr;
+    uint4 *dst = x_perm + r * vpr;
+    int v = lane;
+    for (; v + 96 < vpr; v += 128) {
+      const uint4 a = src[v], b = src[v + 32], c = src[v + 64], d = src[v + 96];
+      dst[v] = a;
+      dst[v + 32] = b;
+      dst[v + 64] = c;
+      dst[v + 96] = d;
     }
-    cnt_off[E] = a;
-    offsets[E] = b;
-    *n_dropped = (int)(Q - b);
+    for (; v < vpr; v += 32) dst[v] = src[v];
   }
 }
 
 // ---------------------------------------------------------------------------
-// token choice: stable rank inside the expert, then slot / row writes
+// token choice: histogram of the priority order, per 32-token unit.
+// Unit u = r * nunit + b covers the rank-r choices of tokens b*32 .. b*32+31,
+// i.e. priorities q = r*T + b*32 + lane: units in index order are the
+// priority order.  (When the gate runs first it writes this histogram
+// itself; this kernel serves moe_permute called on its own.)
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) rank_kernel(
+__global__ void __launch_bounds__(256) hist_units_kernel(const int32_t *__restrict__ topk_idx,
+                                                         int64_t T, int k, int E, int nunit,
+                                                         int32_t *__restrict__ hist, uint32_t *err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t u = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (u >= (int64_t)k * nunit) return;                  // whole warp leaves together
+  const int r = (int)(u / nunit);
+  const int64_t b = u - (int64_t)r * nunit;
+  const int64_t t = b * kUnitTokens + lane;
+  int e = -1;
+  if (t < T) {
+    e = topk_idx[t * k + r];
+    if (e < 0 || e >= E) {
+      raise_error(err, kErrBadIndex);
+      e = -1;
+    }
+  }
+  int32_t *h = hist + u * E;
+  for (int i = lane; i < E; i += 32) h[i] = 0;
+  __syncwarp();
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  if (e >= 0 && (__ffs(peers) - 1) == lane) h[e] = __popc(peers);
+}
+
+// ---------------------------------------------------------------------------
+// token choice: scans, in two levels.  Units are grouped in blocks of
+// kUnitsPerBlock; unit_sums gives each block's per-expert total; the rank
+// kernel of a block then adds up the totals of the blocks before it, scans
+// its own units in shared memory, and has the per-expert base of each unit.
+// Every block also derives counts, kept rows (min(n_e, C) or
+// ceil(n_e*num/den)) and the exclusive scans over experts from the totals;
+// block 0 writes them out.
+// ---------------------------------------------------------------------------
+constexpr int kUnitsPerBlock = 32;
+
+__global__ void __launch_bounds__(1024) unit_sums_kernel(const int32_t *__restrict__ hist, int nu,
+                                                         int E, int32_t *__restrict__ bsum) {
+  __shared__ int s_part[1024];
+  const int G = max(1, (int)blockDim.x / E);
+  const int g = threadIdx.x / E, e = threadIdx.x - g * E;
+  const int u_begin = blockIdx.x * kUnitsPerBlock;
+  const int u_end = min(nu, u_begin + kUnitsPerBlock);
+  int part = 0;
+  if (g < G)
+    for (int u = u_begin + g; u < u_end; u += G) part += hist[(int64_t)u * E + e];
+  if (g < G) s_part[threadIdx.x] = part;
+  __syncthreads();
+  if (g == 0) {
+    int total = 0;
+    for (int gg = 0; gg < G; ++gg) total += s_part[gg * E + e];
+    bsum[(int64_t)blockIdx.x * E + e] = total;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// token choice: stable rank of each assignment inside its expert.  Block b
+// owns units b*32 .. b*32+31, one warp per unit: rank = per-expert base of
+// the unit + rank among equal experts inside the unit (warp match).  Then the
+// capacity test and the slot / row writes -- or, for keep-fraction, the
+// expert-grouped list of priorities.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024, 1) rank_units_kernel(
     const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_gate, int64_t T, int k,
-    int E, const int32_t *__restrict__ base, const int32_t *__restrict__ offsets,
-    const int32_t *__restrict__ cnt_off, int capacity, int keep_fraction,
+    int E, int nunit, int nb, const int32_t *__restrict__ hist, const int32_t *__restrict__ bsum,
+    int capacity, int keep_num, int keep_den, int keep_fraction, int32_t *__restrict__ counts,
+    int32_t *__restrict__ cnt_off_out, int32_t *__restrict__ kept_out,
+    int32_t *__restrict__ offsets_out, int32_t *__restrict__ n_dropped,
     int32_t *__restrict__ tok_rows, int32_t *__restrict__ row_token, float *__restrict__ row_gate,
     int32_t *__restrict__ sorted_q) {
-  __shared__ int running[kMaxExperts];
-  __shared__ int wc[8][kMaxExperts];
+  extern __shared__ int sm[];
+  int *s_base = sm;                                   // [32 units][E]
+  int *s_pre = s_base + kUnitsPerBlock * E;           // [E] totals of earlier blocks
+  int *s_tot = s_pre + E;                             // [E] totals of all blocks
+  int *s_off = s_tot + E;                             // [E+1] row offsets (exclusive scan of kept)
+  int *s_coff = s_off + E + 1;                        // [E+1] count offsets
+  int *s_part = s_coff + E + 1;                       // [1024] partial sums
+  int *s_part2 = s_part + 1024;                       // [1024]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    running[e] = base[(int64_t)blockIdx.x * E + e];
-#pragma unroll
-    for (int w = 0; w < 8; ++w) wc[w][e] = 0;
+  const int nu = k * nunit;
+  const int b = blockIdx.x;
+  const int u_begin = b * kUnitsPerBlock;
+  const int u_end = min(nu, u_begin + kUnitsPerBlock);
+
+  // 1. totals of the blocks before this one, and of all blocks
+  const int G = max(1, (int)blockDim.x / E);
+  const int g = threadIdx.x / E, e_g = threadIdx.x - g * E;
+  int pre = 0, tot = 0;
+  if (g < G) {
+    for (int bb = g; bb < nb; bb += G) {
+      const int v = bsum[(int64_t)bb * E + e_g];
+      tot += v;
+      if (bb < b) pre += v;
+    }
+    s_part[threadIdx.x] = pre;
+    s_part2[threadIdx.x] = tot;
+  }
+  // this block's unit histograms into shared memory
+  for (int i = threadIdx.x; i < (u_end - u_begin) * E; i += blockDim.x)
+    s_base[i] = hist[(int64_t)u_begin * E + i];
+  __syncthreads();
+  if (g == 0) {
+    int p = 0, t = 0;
+    for (int gg = 0; gg < G; ++gg) {
+      p += s_part[gg * E + e_g];
+      t += s_part2[gg * E + e_g];
+    }
+    s_pre[e_g] = p;
+    s_tot[e_g] = t;
   }
   __syncthreads();
-  const int64_t Q = T * k;
-  const int64_t q0 = (int64_t)blockIdx.x * kAssignBlock;
-  const int64_t q1 = min(q0 + kAssignBlock, Q);
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int64_t cq = q0; cq < q1; cq += blockDim.x) {
-    const int64_t q = cq + threadIdx.x;
-    int e = -1;
-    int64_t t = 0, j = 0;
-    if (q < q1) {
-      j = q / T;
-      t = q - j * T;
-      e = topk_idx[t * k + j];
-      if (e < 0 || e >= E) e = -1;       // reported by hist_kernel
+  // 2. per-expert exclusive scan over this block's units (in place)
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = s_pre[e];
+    for (int i = 0; i < u_end - u_begin; ++i) {
+      const int v = s_base[i * E + e];
+      s_base[i * E + e] = run;
+      run += v;
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int lane_rank = __popc(peers & lt_mask);
-    const int cnt = __popc(peers);
-    const bool leader = (__ffs(peers) - 1) == lane;
-    if (e >= 0 && leader) wc[warp][e] = cnt;
-    __syncthreads();
-    int rank = 0;
-    if (e >= 0) {
-      rank = running[e] + lane_rank;
-      for (int w = 0; w < warp; ++w) rank += wc[w][e];
+  }
+  // 3. kept rows and the exclusive scans over experts
+  if (warp == 0) {
+    int a = 0, c = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int ce = e < E ? s_tot[e] : 0;
+      int ke = ce;
+      if (capacity > 0) ke = min(ce, capacity);
+      else if (keep_den > 0) ke = (int)(((int64_t)ce * keep_num + keep_den - 1) / keep_den);
+      int xa = ce, xc = ke;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int ya = __shfl_up_sync(0xffffffffu, xa, o);
+        const int yc = __shfl_up_sync(0xffffffffu, xc, o);
+        if (lane >= o) {
+          xa += ya;
+          xc += yc;
+        }
+      }
+      if (e < E) {
+        s_coff[e] = a + xa - ce;
+        s_off[e] = c + xc - ke;
+        if (b == 0) {
+          counts[e] = ce;
+          kept_out[e] = ke;
+          cnt_off_out[e] = a + xa - ce;
+          offsets_out[e] = c + xc - ke;
+        }
+      }
+      a += __shfl_sync(0xffffffffu, xa, 31);
+      c += __shfl_sync(0xffffffffu, xc, 31);
     }
-    __syncthreads();
-    if (e >= 0 && leader) {
-      atomicAdd(&running[e], cnt);      // leaders of several warps may share e
-      wc[warp][e] = 0;
-    }
-    __syncthreads();
-    if (e < 0) continue;
-    if (keep_fraction) {
-      sorted_q[cnt_off[e] + rank] = (int32_t)q;
-    } else {
-      const bool keep = capacity <= 0 || rank < capacity;
-      const int slot = keep ? offsets[e] + rank : -1;
-      tok_rows[t * k + j] = slot;
-      if (keep) {
-        row_token[slot] = (int32_t)t;
-        row_gate[slot] = topk_gate[t * k + j];
+    if (lane == 0) {
+      s_coff[E] = a;
+      s_off[E] = c;
+      if (b == 0) {
+        cnt_off_out[E] = a;
+        offsets_out[E] = c;
+        *n_dropped = (int)((int64_t)T * k - c);
       }
     }
+  }
+  __syncthreads();
+
+  // 4. one warp per unit
+  const int u = u_begin + warp;
+  if (u >= u_end) return;
+  const int r = u / nunit;
+  const int64_t bu = u - (int64_t)r * nunit;
+  const int64_t t = bu * kUnitTokens + lane;
+  int e = -1;
+  if (t < T) {
+    e = topk_idx[t * k + r];
+    if (e < 0 || e >= E) e = -1;                         // reported by the histogram
+  }
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const int rank = e >= 0 ? s_base[warp * E + e] + __popc(peers & ((1u << lane) - 1u)) : 0;
+  if (keep_fraction) {
+    if (e >= 0) sorted_q[s_coff[e] + rank] = (int32_t)(r * T + t);
+    return;
+  }
+  const bool keep = e >= 0 && (capacity <= 0 || rank < capacity);
+  const int slot = keep ? s_off[e] + rank : -1;
+  if (e >= 0) tok_rows[t * k + r] = slot;
+  if (keep) {
+    row_token[slot] = (int32_t)t;
+    row_gate[slot] = topk_gate[t * k + r];
   }
 }
 
@@ -341,51 +446,19 @@ __global__ void __launch_bounds__(1024) ec_select_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// row gather
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restrict__ x,
-                                                          uint4 *__restrict__ x_perm,
-                                                          const int32_t *__restrict__ row_token,
-                                                          const int32_t *__restrict__ offsets, int E,
-                                                          int64_t T, int vec_per_row,
-                                                          uint32_t *err) {
-  const int lane = threadIdx.x & 31;
-  const int64_t R = offsets[E];
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += nwarps) {
-    const int64_t t = row_token[r];
-    if (t < 0 || t >= T) {
-      if (lane == 0) raise_error(err, kErrBadIndex);
-      continue;
-    }
-    const uint4 *src = x + t * vec_per_row;
-    uint4 *dst = x_perm + r * vec_per_row;
-    for (int v = lane; v < vec_per_row; v += 32) dst[v] = src[v];
-  }
-}
-
-// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-static int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
-cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, const void *x,
-                           const int32_t *topk_idx, const float *topk_gate, const float *probs,
-                           int32_t *counts, int32_t *offsets, int32_t *tok_rows,
+cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, bool hist_ready,
+                           const void *x, const int32_t *topk_idx, const float *topk_gate,
+                           const float *probs, int32_t *counts, int32_t *offsets, int32_t *tok_rows,
                            int32_t *row_token, float *row_gate, void *x_perm, int32_t *n_dropped,
                            cudaStream_t s) {
   uint32_t *err = reinterpret_cast<uint32_t *>(ws + L.err);
   const int E = c->E;
   const int64_t T = c->T;
+  const int vpr = (int)(c->d_model * elem_size(c) / 16);
+  const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+  uint4 *xp = reinterpret_cast<uint4 *>(x_perm);
   if (c->mode == MOE_EXPERT_CHOICE) {
     float *pt = reinterpret_cast<float *>(ws + L.probs_t);
     dim3 tb(32, 8), tg((unsigned)((T + 31) / 32), (unsigned)((E + 31) / 32));
@@ -393,28 +466,37 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, con
     ec_select_kernel<<<E, 1024, 0, s>>>(pt, T, E, c->ec_capacity, counts, offsets, tok_rows,
                                         row_token, row_gate, n_dropped);
   } else {
-    int32_t *hist = reinterpret_cast<int32_t *>(ws + L.hist);
-    int32_t *base = reinterpret_cast<int32_t *>(ws + L.base);
-    int32_t *cnt_off = reinterpret_cast<int32_t *>(ws + L.cnt_off);
-    int32_t *kept = reinterpret_cast<int32_t *>(ws + L.kept);
-    int32_t *sorted_q = reinterpret_cast<int32_t *>(ws + L.sorted_q);
-    const int keepfrac = (c->capacity <= 0 && c->keep_den > 0) ? 1 : 0;
-    hist_kernel<<<L.nblk, 256, 0, s>>>(topk_idx, T, c->k, E, hist, err);
-    scan_kernel<<<1, 256, 0, s>>>(hist, L.nblk, E, T * c->k, c->capacity, c->keep_num, c->keep_den,
-                                  base, counts, cnt_off, kept, offsets, n_dropped);
-    rank_kernel<<<L.nblk, 256, 0, s>>>(topk_idx, topk_gate, T, c->k, E, base, offsets, cnt_off,
-                                       c->capacity, keepfrac, tok_rows, row_token, row_gate,
-                                       sorted_q);
-    if (keepfrac)
-      keep_select_kernel<<<E, 1024, 0, s>>>(sorted_q, cnt_off, kept, offsets, probs, topk_gate, T,
-                                            c->k, E, tok_rows, row_token, row_gate);
+  int32_t *hist = reinterpret_cast<int32_t *>(ws + L.hist);
+  int32_t *bsum = reinterpret_cast<int32_t *>(ws + L.base);
+  int32_t *cnt_off = reinterpret_cast<int32_t *>(ws + L.cnt_off);
+  int32_t *kept = reinterpret_cast<int32_t *>(ws + L.kept);
+  int32_t *sorted_q = reinterpret_cast<int32_t *>(ws + L.sorted_q);
+  const int keepfrac = (c->capacity <= 0 && c->keep_den > 0) ? 1 : 0;
+  const int nu = c->k * L.nunit;
+  const int nb = (nu + kUnitsPerBlock - 1) / kUnitsPerBlock;
+  if (!hist_ready)
+    hist_units_kernel<<<(unsigned)((nu + 7) / 8), 256, 0, s>>>(topk_idx, T, c->k, E, L.nunit, hist, err);
+  unit_sums_kernel<<<nb, 1024, 0, s>>>(hist, nu, E, bsum);
+  const size_t rank_smem = ((size_t)kUnitsPerBlock * E + 4 * E + 2 + 2048) * sizeof(int);
+  if (rank_smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(rank_units_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rank_smem);
+    if (e != cudaSuccess) return e;
   }
-  const int vec_per_row = (int)(c->d_model * elem_size(c) / 16);
+  rank_units_kernel<<<nb, 1024, rank_smem, s>>>(topk_idx, topk_gate, T, c->k, E, L.nunit, nb, hist,
+                                                bsum, c->capacity, c->keep_num, c->keep_den, keepfrac,
+                                                counts, cnt_off, kept, offsets, n_dropped, tok_rows,
+                                                row_token, row_gate, sorted_q);
+  if (keepfrac)
+    keep_select_kernel<<<E, 1024, 0, s>>>(sorted_q, cnt_off, kept, offsets, probs, topk_gate, T,
+                                          c->k, E, tok_rows, row_token, row_gate);
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t want = (L.rows_cap + 7) / 8;
-  const int blocks = (int)std::min<int64_t>(want > 0 ? want : 1, (int64_t)sm_count() * 8);
-  gather_rows_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4 *>(x),
-                                            reinterpret_cast<uint4 *>(x_perm), row_token, offsets,
-                                            E, T, vec_per_row, err);
+  const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 8));
+  gather_rows_kernel<<<blocks, 256, 0, s>>>(xv, xp, row_token, offsets, E, T, vpr, err);
   return cudaGetLastError();
 }
 
@@ -477,7 +559,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_config *cfg, const void *x,
   const moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const WsLayout L = make_layout(cfg);
-  if (L.step_end > kStaticScratchBytes) return MOE_ERR_WORKSPACE;   // beyond the fixed array
+  if (L.permute_end > kStaticScratchBytes) return MOE_ERR_WORKSPACE;   // beyond the fixed array
   const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
   const bool keepfrac = tc && cfg->capacity <= 0 && cfg->keep_den > 0;
   if (!x || !counts || !offsets || !tok_rows || !row_token || !row_gate || !x_perm || !n_dropped)
@@ -490,7 +572,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_config *cfg, const void *x,
   if (static_scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(scratch + L.err, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-  const cudaError_t e = launch_permute(cfg, L, scratch, x, topk_idx, topk_gate, probs, counts,
+  const cudaError_t e = launch_permute(cfg, L, scratch, false, x, topk_idx, topk_gate, probs, counts,
                                        offsets, tok_rows, row_token, row_gate, x_perm, n_dropped, s);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -36,6 +36,10 @@ SMALL = {
     "dsmoe_ec_s": replace(WORKLOADS["deepseekmoe_ec"], T=1000, d_model=256, d_ff=128,
                           ec_capacity=1000 * 6 // 64),
     "dsv2_s": replace(WORKLOADS["deepseek_v2"], T=900, d_model=320, d_ff=192),
+    # >= 1024 rows per expert: the up/down projections run on CTA pairs
+    # (256-row tiles); ragged M tails, partial N tiles, shared experts
+    "pair_relu_s": replace(WORKLOADS["gshard"], T=2100, E=4, d_model=256, d_ff=320),
+    "pair_swiglu_s": replace(WORKLOADS["deepseekmoe_tc"], T=1400, E=8, k=6, d_model=320, d_ff=192),
 }
 
 

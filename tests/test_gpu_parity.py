@@ -48,10 +48,18 @@ def _route_gpu(cfg, inp):
 # steps 1-3a
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("name", list(SMALL) + ["full:" + n for n in WORKLOADS])
+# small cases whose router K is split over CTAs (d = 1024, few token tiles)
+ROUTE_EXTRA = {
+    "split_k_s": replace(WORKLOADS["gshard"], T=300),
+    "split_k_groups_s": replace(WORKLOADS["deepseek_v2"], T=200, d_model=1024, keep_num=0, keep_den=0),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL) + list(ROUTE_EXTRA) + ["full:" + n for n in WORKLOADS])
 def test_route_bit_exact(name):
     """Router GEMM (tcgen05 for bf16, CUDA cores for fp32) + gate, grid inputs."""
-    w = WORKLOADS[name[5:]] if name.startswith("full:") else SMALL[name]
+    w = (WORKLOADS[name[5:]] if name.startswith("full:")
+         else ROUTE_EXTRA[name] if name in ROUTE_EXTRA else SMALL[name])
     inp = make_inputs(w, seed=1, device="cuda", grid=True, with_weights=False)
     cfg = api.config_from_workload(w)
     B = _route_gpu(cfg, inp)
