@@ -42,7 +42,10 @@ DEFAULT_WORKLOAD = "gshard"
 # dram bytes (read + write) per launch, from ncu captures summarised under
 # profiles/, with the sha256 (first 16 hex digits) of the kernel source they
 # were taken at; a value is reported only while the source is unchanged.
-NCU_TRAFFIC: dict[str, dict] = {}
+NCU_TRAFFIC: dict[str, dict] = {
+    # profiles/gemm_gshard_ncu.md: up 151.0 + 39.2 MB, down 207.6 + 19.5 MB
+    "gshard": {"bytes": 417_320_704, "src": "3c68e297a84446e9"},
+}
 
 
 def _peaks():
@@ -299,11 +302,10 @@ def run_reference(args, w) -> None:
 # our arm
 # ---------------------------------------------------------------------------
 def run_ours(args, w) -> None:
-    from mixture_experts_layer_63_b200 import api
+    from mixture_experts_layer_63_b200 import api, replicas
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    info = replicas.rank_info()
+    world, rank, local = info.world, info.rank, info.local_rank
     torch.cuda.set_device(local)
     dist = None
     if world > 1:
@@ -317,7 +319,7 @@ def run_ours(args, w) -> None:
     inp = make_inputs(w, seed=args.seed, device="cuda", grid=False)
     if world > 1:
         g = torch.Generator(device="cuda")
-        g.manual_seed(args.seed * 1000 + rank + 1)
+        g.manual_seed(replicas.token_seed(args.seed, rank, world))
         inp.x = torch.randn(w.T, w.d_model, generator=g, device="cuda").to(inp.x.dtype)
     cfg = api.config_from_workload(w)
     sizes = api.query_sizes(cfg)
@@ -357,13 +359,9 @@ def run_ours(args, w) -> None:
 
     per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)]
                     for i in range(args.steps)])          # ms: route, permute, ffn, combine
-    total_ms = float(per.sum())
-    t_max = torch.tensor([total_ms], device="cuda")
-    if dist:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    total_ms = float(t_max.item())
+    total_ms = replicas.max_over_ranks(float(per.sum()), dist, device="cuda")
     ms_step = total_ms / args.steps
-    value = world * w.T * args.steps / (total_ms / 1e3)
+    value = replicas.throughput(world, w.T, args.steps, total_ms)
 
     # algorithmic work of this batch: kept routed rows from the counts
     if w.mode == "ec":
@@ -413,11 +411,10 @@ def run_ours(args, w) -> None:
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     api.moe_check_device_errors(layer.ws)
-    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in e2e_ev)], device="cuda")
+    e2e_ms = replicas.max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), dist, device="cuda")
     if dist:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_value = world * w.T * args.steps / (float(e2e_ms.item()) / 1e3)
+    e2e_value = replicas.throughput(world, w.T, args.steps, e2e_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -458,6 +455,62 @@ def run_ours(args, w) -> None:
         dist.destroy_process_group()
 
 
+def run_gemm_vs_library(args, w) -> None:
+    """The expert GEMMs of this workload's shape, all rows on one expert (a
+    dense problem), through moe_expert_ffn, next to torch.matmul (cuBLAS) on
+    the same operands.  A yardstick for the kernels only: the library GEMM is
+    never on the layer's path."""
+    from mixture_experts_layer_63_b200 import api
+    torch.cuda.set_device(0)
+    R, d, f = w.T * w.k, w.d_model, w.d_ff
+    c = api.MoeConfig()
+    c.T, c.d_model, c.E, c.S, c.k, c.d_ff = R, d, 1, 0, 1, f
+    c.act = api.MOE_ACT_SWIGLU if w.act == "swiglu" else api.MOE_ACT_RELU
+    c.mode, c.dtype = api.MOE_TOKEN_CHOICE, api.MOE_BF16
+    s = api.query_sizes(c)
+    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    x = torch.randn(R, d, generator=g, device="cuda").bfloat16()
+    w1 = (torch.randn(1, f, d, generator=g, device="cuda") * d ** -0.5).bfloat16()
+    w3 = (torch.randn(1, f, d, generator=g, device="cuda") * d ** -0.5).bfloat16() if w.act == "swiglu" else None
+    w2 = (torch.randn(1, d, f, generator=g, device="cuda") * f ** -0.5).bfloat16()
+    offsets = torch.tensor([0, R], dtype=torch.int32, device="cuda")
+    gate = torch.ones(R, device="cuda")
+    h = torch.empty(s.rows_total, f, device="cuda", dtype=torch.bfloat16)
+    y = torch.empty(s.rows_total, d, device="cuda", dtype=torch.float32)
+    ws = api.new_workspace(c, step_only=True)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def ours():
+        api.moe_expert_ffn(c, x, x, offsets, gate, w1, w3, w2, h, y, ws)
+
+    def lib():
+        a = x @ w1[0].T
+        hh = torch.relu(a) if w3 is None else torch.nn.functional.silu(a) * (x @ w3[0].T)
+        return hh @ w2[0].T
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        t = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            t += e0.elapsed_time(e1)
+        return t / args.steps
+
+    t_ours, t_lib = timed(ours), timed(lib)
+    fl = 2.0 * R * d * f * (3 if w3 is not None else 2)
+    print(json.dumps({"mode": "gemm-vs-library", "workload": _describe(w), "rows": R, "d_model": d,
+                      "d_ff": f, "ours_us": t_ours * 1e3, "ours_tflops": fl / t_ours / 1e9,
+                      "torch_matmul_us": t_lib * 1e3, "torch_matmul_tflops": fl / t_lib / 1e9,
+                      "ratio": t_lib / t_ours, "l2": "flushed before every call"}), flush=True)
+
+
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -467,10 +520,14 @@ def main() -> None:
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm-vs-library", action="store_true",
+                    help="time the expert GEMMs on this workload's dense shape next to torch.matmul")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
-    if args.impl == "reference":
+    if args.gemm_vs_library:
+        run_gemm_vs_library(args, w)
+    elif args.impl == "reference":
         run_reference(args, w)
     else:
         run_ours(args, w)
