@@ -228,11 +228,17 @@ MOE_API moe_status moe_forward_timed(const moe_config *cfg, const void *x, const
 
 /* Waits for `stream`, then reads and clears the workspace's device error
  * word.  Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_CHECK; *flags (if
- * not NULL) receives the raw bits.  This is the only call that blocks. */
+ * not NULL) receives the raw bits.  After an error it also clears the rest
+ * of the workspace's 4 KiB control block (the GEMMs' stream-K ready flags,
+ * which a timed-out launch can leave set).  This is the only call that
+ * blocks. */
 MOE_API moe_status moe_check_device_errors(void *ws, size_t ws_bytes, moe_stream_t stream, uint32_t *flags);
 
-/* Fill `ws` with the bytes the library expects in a fresh workspace (the
- * error word cleared).  Call once after allocating a workspace. */
+/* Fill `ws` with the bytes the library expects in a fresh workspace: the
+ * 4 KiB control block at its start (error word, the GEMMs' stream-K ready
+ * flags) cleared.  Call once after allocating a workspace (a zero-filled
+ * allocation needs no call).  Every launch leaves the flags at zero unless
+ * it reports an error. */
 MOE_API moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Static text for a status code. */

@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const void *__rest
   __shared__ int s_rows[kWarps][kMaxRows];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t = (int64_t)blockIdx.x * kWarps + warp;
+  pdl_wait();
+  pdl_trigger();
   if (t >= T) return;
   int *rows = s_rows[warp];
   // collect the token's rows in order
@@ -79,13 +81,9 @@ cudaError_t launch_combine(const moe_config *c, int64_t rows_cap, const void *y_
   const bool ec = c->mode == MOE_EXPERT_CHOICE;
   const int W = ec ? c->E : c->k;
   const unsigned blocks = (unsigned)((c->T + kWarps - 1) / kWarps);
-  if (c->dtype == MOE_BF16)
-    combine_kernel<true><<<blocks, kWarps * 32, 0, s>>>(y_rows, tok_rows, y, c->T, c->d_model, W,
-                                                        ec ? 1 : 0, c->S, rows_cap);
-  else
-    combine_kernel<false><<<blocks, kWarps * 32, 0, s>>>(y_rows, tok_rows, y, c->T, c->d_model, W,
-                                                         ec ? 1 : 0, c->S, rows_cap);
-  return cudaGetLastError();
+  auto kern = c->dtype == MOE_BF16 ? combine_kernel<true> : combine_kernel<false>;
+  return launch_kernel(kern, blocks, kWarps * 32, 0, s, y_rows, tok_rows, y, c->T, c->d_model, W,
+                       ec ? 1 : 0, c->S, rows_cap);
 }
 
 }  // namespace moe

@@ -25,6 +25,22 @@ __device__ __forceinline__ void raise_error(uint32_t *err, uint32_t bit) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialization (launch_kernel in moe_internal.h):
+// it may become resident while the kernel before it on the stream is still
+// running.  Each kernel therefore runs pdl_wait() in every thread before its
+// first access to global memory (it returns once the previous kernel has
+// completed and its writes are visible; at once when there is none), and no
+// thread returns before it, so the completion of a kernel implies the
+// completion of all kernels before it.  pdl_trigger() lets the next kernel
+// start its own prologue early.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // bf16 <-> fp32
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }

@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(const F32Params P) {
   __shared__ float B3s[TN][TK + 1];
   const int G = P.n_routed + P.n_static;
   const int nt = (P.N + TN - 1) / TN;
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x == 0) {
     int acc = 0;
     for (int g = 0; g < G; ++g) {
@@ -160,8 +162,7 @@ cudaError_t launch_ffn_f32(const moe_config *c, const WsLayout &L, uint32_t *err
   up.out_static_base = L.rows_cap;
   up.a_rows = L.rows_cap;
   up.err = err;
-  ffn_f32_kernel<<<grid, 256, 0, s>>>(up);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_kernel(ffn_f32_kernel, grid, 256, 0, s, up);
   if (e != cudaSuccess) return e;
   F32Params dn{};
   dn.mode = 2;
@@ -182,8 +183,7 @@ cudaError_t launch_ffn_f32(const moe_config *c, const WsLayout &L, uint32_t *err
   dn.out_static_base = L.rows_cap;
   dn.a_rows = L.rows_total;
   dn.err = err;
-  ffn_f32_kernel<<<grid, 256, 0, s>>>(dn);
-  return cudaGetLastError();
+  return launch_kernel(ffn_f32_kernel, grid, 256, 0, s, dn);
 }
 
 }  // namespace moe

@@ -54,6 +54,17 @@ constexpr int kMaxGroups = 320;
 #define MOE_PAIR_MIN_ROWS 384
 #endif
 constexpr uint32_t kABytes = BM * BK * 2;   // 16 KB
+// Stream-K tail: a piece of a split tile covers at least this many k-blocks
+constexpr int kSkMinUnits = 8;
+#ifndef MOE_STREAM_K
+#define MOE_STREAM_K 1
+#endif
+// The TMA producer also asks L2 for the k-block this many loads ahead of the
+// one it is loading (0: off), so operand fetches from HBM start earlier than
+// the shared-memory ring alone allows.
+#ifndef MOE_L2_PREFETCH
+#define MOE_L2_PREFETCH 0
+#endif
 
 struct Params {
   int epi;
@@ -70,6 +81,8 @@ struct Params {
   const float *bias;
   int ksplit;               // K split into this many parts (router only), partial outputs
   int64_t split_stride;     //   ksplit parts of the output, split_stride elements apart
+  float *sk_part;           // stream-K partial accumulators, one kSkSlotFloats slot per CTA
+  int *sk_flags;            //   and one ready flag per slot; null: no stream-K
   uint32_t *err;
 };
 
@@ -139,6 +152,14 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
+}
+
+// hint: bring one box of the tensor into L2 (no shared memory, no completion)
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap *map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map) {
@@ -288,6 +309,202 @@ __device__ __forceinline__ Tile decode_tile(int tile, const int *prefix, int G, 
   return t;
 }
 
+// Work of one CTA (or CTA pair): whole tiles dealt round-robin, then -- when
+// the tile count is not a multiple of the worker count -- a stream-K tail.
+// The last tiles (between one and two waves' worth, or all of them when
+// there are fewer tiles than workers) are cut into k-block units, laid end to
+// end and split evenly over the workers, so no worker idles through a last,
+// partly filled wave.  A tile cut between workers is summed by the worker
+// holding its first k-block (the "finalizer"; that piece is the last of its
+// range), adding the partial accumulators of the later workers (each one
+// the first piece of its range, so it is written without waiting on anyone)
+// in worker order: the result depends only on the tile count and the grid.
+struct Sched {
+  int P, w, KB;
+  int base;                      // tiles of one K part
+  int ksplit, KBs;               // router K split: parts of KBs k-blocks (no stream-K)
+  int dp_rounds, dp_limit;       // round-robin items: w + i * P < dp_limit, i < dp_rounds
+  int64_t sk_units;              // k-block units of the stream-K tail
+  int sk_workers;                // workers sharing the tail (pieces >= kSkMinUnits)
+  int64_t my_end, u;             // this worker's tail units [u, my_end)
+  int i;
+
+  __device__ __forceinline__ void init(int total, int KB_, int P_, int w_, bool sk, int ksplit_) {
+    P = P_;
+    w = w_;
+    KB = KB_;
+    base = total;
+    ksplit = ksplit_ > 1 ? ksplit_ : 1;
+    KBs = (KB + ksplit - 1) / ksplit;
+    sk_units = 0;
+    sk_workers = 1;
+    if (!sk || ksplit > 1 || total % P == 0) {
+      dp_limit = total * ksplit;
+      dp_rounds = (dp_limit + P - 1) / P;
+    } else {
+      dp_rounds = total / P - 1;
+      if (dp_rounds < 0) dp_rounds = 0;
+      dp_limit = dp_rounds * P;
+      sk_units = (int64_t)(total - dp_limit) * KB;
+      int64_t nw = sk_units / kSkMinUnits;
+      if (nw < 1) nw = 1;
+      sk_workers = (int)(nw < P ? nw : P);
+    }
+    u = start(w);
+    my_end = start(w + 1);
+    i = 0;
+  }
+  // first tail unit of worker q (the tail's end for q >= sk_workers)
+  __device__ __forceinline__ int64_t start(int q) const {
+    return q >= sk_workers ? sk_units : (int64_t)q * sk_units / sk_workers;
+  }
+  // next piece of this worker: tile, k-blocks [kb0, kb1), K part
+  __device__ __forceinline__ bool next(int &tile, int &kb0, int &kb1, int &part) {
+    while (i < dp_rounds) {
+      const int t = w + i * P;
+      ++i;
+      if (t < dp_limit) {
+        part = t / base;
+        tile = t - part * base;
+        kb0 = part * KBs;
+        kb1 = min(KB, kb0 + KBs);
+        return true;
+      }
+    }
+    if (u < my_end) {
+      part = 0;
+      tile = dp_limit + (int)(u / KB);
+      kb0 = (int)(u % KB);
+      const int64_t left = my_end - u;
+      kb1 = (int)(KB - kb0 < left ? KB : kb0 + left);
+      u += kb1 - kb0;
+      return true;
+    }
+    return false;
+  }
+  // workers [w + 1, q_end) may hold later pieces of this worker's tile
+  __device__ __forceinline__ int contributors_end(int tile) const {
+    const int64_t tile_end = (int64_t)(tile - dp_limit + 1) * KB;
+    int q = w + 1;
+    while (q < sk_workers && start(q) < tile_end) ++q;
+    return q;
+  }
+  __device__ __forceinline__ bool nonempty(int q) const { return start(q + 1) > start(q); }
+};
+
+// A second cursor over a worker's k-blocks, running ahead of the producer.
+struct Ahead {
+  Sched sc;
+  int tile, kb, kb1, part;
+  bool live;
+  __device__ __forceinline__ void init(const Sched &s, int skip) {
+    sc = s;
+    live = sc.next(tile, kb, kb1, part);
+    for (int i = 0; i < skip; ++i) step();
+  }
+  __device__ __forceinline__ void step() {
+    if (live && ++kb >= kb1) live = sc.next(tile, kb, kb1, part);
+  }
+};
+
+// Stream-K partial accumulator slot: 128 rows x 256 fp32 columns, stored as
+// float4 column groups of 128 rows, so that a warp's 32 rows x 16 bytes are
+// one contiguous 512-byte run.
+__device__ __forceinline__ float4 *sk_slot_ptr(float *part, int slot, int row, int col) {
+  return reinterpret_cast<float4 *>(part + (size_t)slot * kSkSlotFloats) + (size_t)(col >> 2) * BM + row;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add_gpu(int *p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Ready flags count rows, so no epilogue thread ever waits on another thread
+// of its own CTA: each of the 128 writer threads adds 1 after storing its row
+// (release); a finalizer thread reads a slot once the flag is >= 128
+// (acquire) and then adds 1 itself; the thread that brings it to 256 resets
+// it to 0 for the next launch, which the stream orders after this one.
+constexpr int kEpiThreads = 128;
+
+// The finalizer's view of the later pieces of its tile: slots of workers
+// q in [q0, q1) with a non-empty range, slot = q * slot_mul + slot_add.
+struct Fixup {
+  const float *part;
+  const Sched *sc;
+  int q0, q1, slot_mul, slot_add, row;
+};
+
+// v[i] += every later piece's column col + i of this row, in worker order
+__device__ __forceinline__ void add_parts(float (&v)[32], const Fixup &F, int col) {
+  for (int q = F.q0; q < F.q1; ++q) {
+    if (!F.sc->nonempty(q)) continue;
+    const float4 *p = sk_slot_ptr(const_cast<float *>(F.part), q * F.slot_mul + F.slot_add, F.row, col);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 t = p[(size_t)j * BM];
+      v[4 * j + 0] += t.x;
+      v[4 * j + 1] += t.y;
+      v[4 * j + 2] += t.z;
+      v[4 * j + 3] += t.w;
+    }
+  }
+}
+
+// A piece that does not finish its tile: this thread's row of the raw
+// accumulator (P.bn TMEM columns) into the worker's slot, then publish it.
+__device__ __forceinline__ void sk_write(const Params &P, int slot, int row, uint32_t taddr) {
+  uint32_t r[32];
+#pragma unroll 1
+  for (int c = 0; c < P.bn; c += 32) {
+    tmem_ld32(taddr + c, r);
+    tmem_ld_wait();
+    float4 *p = sk_slot_ptr(P.sk_part, slot, row, c);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      p[(size_t)j * BM] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                      __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+  }
+  red_release_add_gpu(P.sk_flags + slot, 1);
+}
+
+// Finalizer thread: bounded wait until every later piece of the tile is
+// published.  False when the CTA is aborting (timeout bit raised here).
+__device__ __forceinline__ bool sk_wait(const Params &P, const Fixup &F, volatile int *abort_flag) {
+  for (int q = F.q0; q < F.q1; ++q) {
+    if (!F.sc->nonempty(q)) continue;
+    const int *flag = P.sk_flags + q * F.slot_mul + F.slot_add;
+    if (ld_acquire_gpu(flag) >= kEpiThreads) continue;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (ld_acquire_gpu(flag) >= kEpiThreads) break;
+      if ((it & 63u) == 0) {
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          raise_error(P.err, kErrTimeout);
+          *abort_flag = 1;
+          return false;
+        }
+      }
+    }
+  }
+  return true;
+}
+
+// Finalizer thread, after its epilogue read the slots: count itself done;
+// the last of the 128 readers clears the flag.
+__device__ __forceinline__ void sk_done(const Params &P, const Fixup &F) {
+  for (int q = F.q0; q < F.q1; ++q) {
+    if (!F.sc->nonempty(q)) continue;
+    int *flag = P.sk_flags + q * F.slot_mul + F.slot_add;
+    if (atomicAdd(flag, 1) == 2 * kEpiThreads - 1) atomicExch(flag, 0);
+  }
+}
+
 // --------------------------------- epilogues ---------------------------------
 __device__ __forceinline__ void store_bf16x32(void *dst, const float (&v)[32]) {
   uint4 *p = reinterpret_cast<uint4 *>(dst);
@@ -303,10 +520,12 @@ __device__ __forceinline__ void store_bf16x32(void *dst, const float (&v)[32]) {
 }
 
 // Epilogue of one accumulator: this thread's row (TMEM lane) of the tile,
-// BN columns from TMEM address `taddr`; activation / gate / bias, stores.
+// BN columns from TMEM address `taddr`; the later stream-K pieces of the tile
+// added first when F is given; then activation / gate / bias, stores.
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, bool valid, bool routed,
-                                              int64_t out_row, int col0, int64_t out_offset = 0) {
+                                              int64_t out_row, int col0, int64_t out_offset = 0,
+                                              const Fixup *F = nullptr) {
   uint32_t r[32];
   float v[32];
   if (EPI == kEpiSwiglu) {
@@ -314,13 +533,23 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
 #pragma unroll 1
     for (int c = 0; c < 128 / 32; ++c) {
       uint32_t u[32];
+      float uf[32];
       tmem_ld32(taddr + c * 32, r);
       tmem_ld32(taddr + 128 + c * 32, u);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float g = __uint_as_float(r[i]);
-        v[i] = g / (1.0f + __expf(-g)) * __uint_as_float(u[i]);
+        v[i] = __uint_as_float(r[i]);
+        uf[i] = __uint_as_float(u[i]);
+      }
+      if (F) {
+        add_parts(v, *F, c * 32);
+        add_parts(uf, *F, 128 + c * 32);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float g = v[i];
+        v[i] = g / (1.0f + __expf(-g)) * uf[i];
       }
       const int col = col0 + c * 32;
       if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
@@ -332,7 +561,10 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
       tmem_ld32(taddr + c * 32, r);
       tmem_ld_wait();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = fmaxf(__uint_as_float(r[i]), 0.0f);
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      if (F) add_parts(v, *F, c * 32);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.0f);
       const int col = col0 + c * 32;
       if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
     }
@@ -344,13 +576,16 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
     for (int c = 0; c < P.bn / 32; ++c) {
       tmem_ld32(taddr + c * 32, r);
       tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      if (F) add_parts(v, *F, c * 32);
       const int col = col0 + c * 32;
       if (valid && col < P.N) {
         float4 *dst = reinterpret_cast<float4 *>(out + out_row * P.N + col);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          dst[q] = make_float4(__uint_as_float(r[4 * q]) * scale, __uint_as_float(r[4 * q + 1]) * scale,
-                               __uint_as_float(r[4 * q + 2]) * scale, __uint_as_float(r[4 * q + 3]) * scale);
+          dst[q] = make_float4(v[4 * q] * scale, v[4 * q + 1] * scale, v[4 * q + 2] * scale,
+                               v[4 * q + 3] * scale);
       }
     }
   } else {  // kEpiStoreF32 (a K part when the router is split: no bias, own output)
@@ -400,6 +635,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+  if (tid == 32) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accf_bar[a], 1);
+      mbar_init(&acce_bar[a], 4 * 32);
+    }
+    mbar_init(&drain_bar, 1);
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (tid == 0) {
+    tma_prefetch_map(&map_a);
+    tma_prefetch_map(&map_b);
+    if (P.n_static > 0) tma_prefetch_map(&map_a_static);
+    if (EPI == kEpiSwiglu) tma_prefetch_map(&map_b3);
+  }
+  pdl_wait();              // what earlier kernels wrote is visible from here on
+  pdl_trigger();
   // group table: rows and tile prefix, warp 0
   if (warp == 0) {
     int carry = 0;
@@ -434,40 +696,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) s_prefix[P.G] = carry;
   }
-  if (tid == 32) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&accf_bar[a], 1);
-      mbar_init(&acce_bar[a], 4 * 32);
-    }
-    mbar_init(&drain_bar, 1);
-    s_abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 2) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&s_tmem_base)),
-                 "r"(kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-  }
-  if (tid == 0) {
-    tma_prefetch_map(&map_a);
-    tma_prefetch_map(&map_b);
-    if (P.n_static > 0) tma_prefetch_map(&map_a_static);
-    if (EPI == kEpiSwiglu) tma_prefetch_map(&map_b3);
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
   const uint32_t tmem_base = s_tmem_base;
-  const int base_total = s_prefix[P.G];
-  const int total = base_total * P.ksplit;          // K parts (router split) x tiles
   const int KB = P.K / BK;
-  const int KBs = (KB + P.ksplit - 1) / P.ksplit;
+  const bool sk = EPI != kEpiStoreF32 && P.sk_part != nullptr;
+  Sched sc;
+  sc.init(s_prefix[P.G], KB, gridDim.x, blockIdx.x, sk, P.ksplit);
+  int tile, kb0, kb1, part;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -476,17 +714,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t armed = 0;            // bit s: full_bar[s] armed and maybe in flight
     uint32_t armed_parity = 0;     // bit s: parity of that phase
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const int part = tile / base_total;
-      const Tile tl = decode_tile(tile - part * base_total, s_prefix, P.G, P.nt);
-      const int kb0 = part * KBs, kb1 = min(KB, kb0 + KBs);
+    // operand coordinates of a tile
+    auto a_of = [&](const Tile &tl, int64_t &row) -> const CUtensorMap * {
       const bool routed = tl.g < P.n_routed;
-      const int64_t a_row = routed ? (int64_t)s_off[tl.g] + (int64_t)tl.m * BM
-                                   : P.a_static_base + (int64_t)(tl.g - P.n_routed) * P.a_static_stride +
-                                         (int64_t)tl.m * BM;
-      const CUtensorMap *ma = routed ? &map_a : &map_a_static;
+      row = routed ? (int64_t)s_off[tl.g] + (int64_t)tl.m * BM
+                   : P.a_static_base + (int64_t)(tl.g - P.n_routed) * P.a_static_stride +
+                         (int64_t)tl.m * BM;
+      return routed ? &map_a : &map_a_static;
+    };
+    Ahead ahead;
+    if (MOE_L2_PREFETCH > 0) ahead.init(sc, MOE_L2_PREFETCH);
+    while (ok && sc.next(tile, kb0, kb1, part)) {
+      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      int64_t a_row;
+      const CUtensorMap *ma = a_of(tl, a_row);
       const int b_row = tl.g * P.N + tl.n * P.bnh;
       for (int kb = kb0; kb < kb1; ++kb) {
+        if (MOE_L2_PREFETCH > 0 && ahead.live) {
+          const Tile pt = decode_tile(ahead.tile, s_prefix, P.G, P.nt);
+          int64_t prow;
+          const CUtensorMap *pm = a_of(pt, prow);
+          const int pb = pt.g * P.N + pt.n * P.bnh;
+          tma_prefetch_l2(pm, ahead.kb * BK, (int)prow);
+          tma_prefetch_l2(&map_b, ahead.kb * BK, pb);
+          if (EPI == kEpiSwiglu) tma_prefetch_l2(&map_b3, ahead.kb * BK, pb);
+          ahead.step();
+        }
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
         uint8_t *sa = smem + (size_t)stage * stage_bytes;
         uint8_t *sb = sa + kABytes;
@@ -516,9 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const int part = tile / base_total;
-      const int kb0 = part * KBs, kb1 = min(KB, kb0 + KBs);
+    while (ok && sc.next(tile, kb0, kb1, part)) {
       if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
@@ -545,22 +796,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     // -------------------------------- epilogue --------------------------------
     const int ew = warp - 4;                     // TMEM lanes 32*ew .. 32*ew+31
+    const int r_cta = ew * 32 + lane;            // row of the tile
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const int part = tile / base_total;
-      const Tile tl = decode_tile(tile - part * base_total, s_prefix, P.G, P.nt);
+    while (sc.next(tile, kb0, kb1, part)) {
+      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
       if (!mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err)) break;
       tc_fence_after();
-      const bool routed = tl.g < P.n_routed;
-      const int r_in = ew * 32 + lane;
-      const bool valid = tl.m * BM + r_in < s_rows[tl.g];
-      const int64_t out_row = (routed ? (int64_t)s_off[tl.g]
-                                      : P.out_static_base + (int64_t)(tl.g - P.n_routed) * P.rows_static) +
-                              (int64_t)tl.m * BM + r_in;
-      const int col0 = tl.n * P.bnh;
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
-      epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, (int64_t)part * P.split_stride);
+      const bool in_tail = sk && tile >= sc.dp_limit;
+      if (in_tail && kb0 > 0) {
+        sk_write(P, (int)blockIdx.x, r_cta, taddr);              // a later piece of the tile
+      } else {
+        const bool routed = tl.g < P.n_routed;
+        const bool valid = tl.m * BM + r_cta < s_rows[tl.g];
+        const int64_t out_row = (routed ? (int64_t)s_off[tl.g]
+                                        : P.out_static_base + (int64_t)(tl.g - P.n_routed) * P.rows_static) +
+                                (int64_t)tl.m * BM + r_cta;
+        const int col0 = tl.n * P.bnh;
+        if (in_tail && kb1 < KB) {                              // finalizer of a split tile
+          const Fixup F{P.sk_part, &sc, (int)blockIdx.x + 1, sc.contributors_end(tile), 1, 0, r_cta};
+          if (!sk_wait(P, F, &s_abort)) break;
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, 0, &F);
+          sk_done(P, F);
+        } else {
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, (int64_t)part * P.split_stride);
+        }
+      }
       tc_fence_before();
       mbar_arrive(&acce_bar[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -616,6 +878,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
+  if (tid == 32) {
+    for (int st = 0; st < kPairStages; ++st) {
+      mbar_init(&full_bar[st], 1);
+      mbar_init(&empty_bar[st], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accf_bar[a], 1);
+      mbar_init(&acce_bar[a], 2 * 4 * 32);
+    }
+    mbar_init(&drain_bar, 1);
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  if (tid == 0) {
+    tma_prefetch_map(&map_a);
+    tma_prefetch_map(&map_b);
+    if (P.n_static > 0) tma_prefetch_map(&map_a_static);
+    if (EPI == kEpiSwiglu) tma_prefetch_map(&map_b3);
+  }
+  pdl_wait();              // what earlier kernels wrote is visible from here on
+  pdl_trigger();
   if (warp == 0) {
     int carry = 0;
     for (int base = 0; base < P.G; base += 32) {
@@ -649,38 +938,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) s_prefix[P.G] = carry;
   }
-  if (tid == 32) {
-    for (int st = 0; st < kPairStages; ++st) {
-      mbar_init(&full_bar[st], 1);
-      mbar_init(&empty_bar[st], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&accf_bar[a], 1);
-      mbar_init(&acce_bar[a], 2 * 4 * 32);
-    }
-    mbar_init(&drain_bar, 1);
-    s_abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 2) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(&s_tmem_base)),
-                 "r"(kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
-  }
-  if (tid == 0) {
-    tma_prefetch_map(&map_a);
-    tma_prefetch_map(&map_b);
-    if (P.n_static > 0) tma_prefetch_map(&map_a_static);
-    if (EPI == kEpiSwiglu) tma_prefetch_map(&map_b3);
-  }
   tc_fence_before();
   cluster_sync_all();              // barriers of both CTAs initialised before any remote use
   tc_fence_after();
 
   const uint32_t tmem_base = s_tmem_base;
-  const int total = s_prefix[P.G];
   const int KB = P.K / BK;
+  const bool sk = P.sk_part != nullptr;
+  Sched sc;
+  sc.init(s_prefix[P.G], KB, npairs, pair, sk, 1);
+  int tile, kb0, kb1, part;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -688,18 +955,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     uint32_t armed = 0, armed_parity = 0;
     bool ok = true;
-    for (int tile = pair; tile < total && ok; tile += npairs) {
-      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+    // B rows of this CTA: SwiGLU: even CTA the gate rows (W1), odd CTA the up
+    // rows (W3); otherwise the two halves of the BN-row tile
+    const CUtensorMap *mb = (EPI == kEpiSwiglu && rank == 1) ? &map_b3 : &map_b;
+    auto rows_of = [&](const Tile &tl, int64_t &a_row, int &b_row) -> const CUtensorMap * {
       const bool routed = tl.g < P.n_routed;
-      const int64_t a_row = (routed ? (int64_t)s_off[tl.g]
-                                    : P.a_static_base + (int64_t)(tl.g - P.n_routed) * P.a_static_stride) +
-                            (int64_t)tl.m * PM + (int64_t)rank * BM;
-      const CUtensorMap *ma = routed ? &map_a : &map_a_static;
-      // B rows of this CTA: SwiGLU: even CTA the gate rows (W1), odd CTA the up
-      // rows (W3); otherwise the two halves of the BN-row tile
-      const CUtensorMap *mb = (EPI == kEpiSwiglu && rank == 1) ? &map_b3 : &map_b;
-      const int b_row = tl.g * P.N + tl.n * P.bnh + ((EPI == kEpiSwiglu) ? 0 : (int)rank * (P.bn / 2));
-      for (int kb = 0; kb < KB; ++kb) {
+      a_row = (routed ? (int64_t)s_off[tl.g]
+                      : P.a_static_base + (int64_t)(tl.g - P.n_routed) * P.a_static_stride) +
+              (int64_t)tl.m * PM + (int64_t)rank * BM;
+      b_row = tl.g * P.N + tl.n * P.bnh + ((EPI == kEpiSwiglu) ? 0 : (int)rank * (P.bn / 2));
+      return routed ? &map_a : &map_a_static;
+    };
+    Ahead ahead;
+    if (MOE_L2_PREFETCH > 0) ahead.init(sc, MOE_L2_PREFETCH);
+    while (ok && sc.next(tile, kb0, kb1, part)) {
+      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      int64_t a_row;
+      int b_row;
+      const CUtensorMap *ma = rows_of(tl, a_row, b_row);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (MOE_L2_PREFETCH > 0 && ahead.live) {
+          const Tile pt = decode_tile(ahead.tile, s_prefix, P.G, P.nt);
+          int64_t pa;
+          int pb;
+          const CUtensorMap *pm = rows_of(pt, pa, pb);
+          tma_prefetch_l2(pm, ahead.kb * BK, (int)pa);
+          tma_prefetch_l2(mb, ahead.kb * BK, pb);
+          ahead.step();
+        }
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
         uint8_t *sa = smem + (size_t)stage * stage_bytes;
         uint8_t *sb = sa + kABytes;
@@ -726,11 +1009,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int tile = pair; tile < total && ok; tile += npairs) {
+    while (ok && sc.next(tile, kb0, kb1, part)) {
       if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&full_bar[stage], phase, &s_abort, P.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + (size_t)stage * stage_bytes);
@@ -738,7 +1021,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int k = 0; k < BK / kUmmaK; ++k) {
           umma_bf16_pair(d_tmem, sw128_desc(a_addr + k * kUmmaK * 2),
-                         sw128_desc(b_addr + k * kUmmaK * 2), idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                         sw128_desc(b_addr + k * kUmmaK * 2), idesc, (kb > kb0 || k > 0) ? 1u : 0u);
         }
         umma_commit_pair_both(&empty_bar[stage]);
         if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
@@ -752,23 +1035,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     // -------------------------------- epilogue --------------------------------
     const int ew = warp - 4;
+    const int r_cta = ew * 32 + lane;                 // row within this CTA's half
     const uint32_t acce_even0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
     const uint32_t acce_even1 = mapa_shared(smem_u32(&acce_bar[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = pair; tile < total; tile += npairs) {
+    while (sc.next(tile, kb0, kb1, part)) {
       const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
       if (!mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err)) break;
       tc_fence_after();
-      const bool routed = tl.g < P.n_routed;
-      const int r_in = (int)rank * BM + ew * 32 + lane;
-      const bool valid = tl.m * PM + r_in < s_rows[tl.g];
-      const int64_t out_row = (routed ? (int64_t)s_off[tl.g]
-                                      : P.out_static_base + (int64_t)(tl.g - P.n_routed) * P.rows_static) +
-                              (int64_t)tl.m * PM + r_in;
-      const int col0 = tl.n * P.bnh;
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
-      epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0);
+      const bool in_tail = sk && tile >= sc.dp_limit;
+      if (in_tail && kb0 > 0) {
+        sk_write(P, 2 * pair + (int)rank, r_cta, taddr);        // a later piece of the tile
+      } else {
+        const bool routed = tl.g < P.n_routed;
+        const int r_in = (int)rank * BM + r_cta;
+        const bool valid = tl.m * PM + r_in < s_rows[tl.g];
+        const int64_t out_row = (routed ? (int64_t)s_off[tl.g]
+                                        : P.out_static_base + (int64_t)(tl.g - P.n_routed) * P.rows_static) +
+                                (int64_t)tl.m * PM + r_in;
+        const int col0 = tl.n * P.bnh;
+        if (in_tail && kb1 < KB) {                              // finalizer of a split tile
+          const Fixup F{P.sk_part, &sc, pair + 1, sc.contributors_end(tile), 2, (int)rank, r_cta};
+          if (!sk_wait(P, F, &s_abort)) break;
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, 0, &F);
+          sk_done(P, F);
+        } else {
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0);
+        }
+      }
       tc_fence_before();
       mbar_arrive_cluster(acc == 0 ? acce_even0 : acce_even1);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -832,8 +1128,7 @@ cudaError_t launch_epi(const GroupedGemm &g, const Params &P, const CUtensorMap 
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<EPI><<<grid, kThreads, smem, s>>>(ma, mas, mb, mb3, P);
-  return cudaGetLastError();
+  return launch_kernel(grouped_gemm_kernel<EPI>, grid, kThreads, smem, s, ma, mas, mb, mb3, P);
 }
 
 // CTA-pair launch: as many 2-CTA clusters as fit at once (one CTA per SM),
@@ -862,9 +1157,9 @@ cudaError_t launch_pair(const Params &P, const CUtensorMap &ma, const CUtensorMa
     }
     mc = n;
   }
-  const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(mc, max_tiles));
-  kern<<<2 * pairs, kThreads, smem, s>>>(ma, mas, mb, mb3, P);
-  return cudaGetLastError();
+  const int64_t want = P.sk_part ? mc : std::min<int64_t>(mc, max_tiles);
+  const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(want, kSkSlots / 2));
+  return launch_kernel(kern, 2 * pairs, kThreads, smem, s, ma, mas, mb, mb3, P);
 }
 
 }  // namespace
@@ -899,6 +1194,10 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   P.bias = g.bias;
   P.ksplit = std::max(1, g.ksplit);
   P.split_stride = g.split_stride;
+  // stream-K tail for the expert GEMMs (the router splits K its own way)
+  const bool sk = MOE_STREAM_K && g.epi != kEpiStoreF32 && g.sk_part && g.sk_flags;
+  P.sk_part = sk ? g.sk_part : nullptr;
+  P.sk_flags = sk ? g.sk_flags : nullptr;
   P.err = g.err;
   if (P.G <= 0 || P.G > kMaxGroups || P.bn > 256 || g.K % BK != 0) return cudaErrorInvalidValue;
   if (g.ksplit > 1 && (g.epi != kEpiStoreF32 || g.n_routed != 0)) return cudaErrorInvalidValue;
@@ -921,7 +1220,9 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   const int64_t mt_routed = (g.max_routed_rows + BM - 1) / BM + g.n_routed;
   const int64_t mt_static = (int64_t)g.n_static * ((g.rows_static + BM - 1) / BM);
   const int64_t max_tiles = (mt_routed + mt_static) * P.nt * P.ksplit;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(device_sms(), max_tiles));
+  // (with stream-K, every SM: a short problem's k-blocks are spread over all)
+  const int grid = std::min(kSkSlots, (int)std::max<int64_t>(1, std::min<int64_t>(
+                                          device_sms(), sk ? device_sms() : max_tiles)));
   // at least 120 KB so that one CTA (and one 512-column TMEM allocation) fits per SM
   const size_t smem = std::max<size_t>((size_t)kStages * (kABytes + (size_t)P.bn * BK * 2) + 1024,
                                        (size_t)120 * 1024);

@@ -71,7 +71,7 @@ WsLayout make_layout(const moe_config *c) {
     o = align256(o + bytes);
     return at;
   };
-  L.err = take(256);
+  L.err = take(kCtrlBytes);
   L.hist = take((size_t)hist_ints * 4);
   L.base = take((size_t)(tc ? (k * L.nunit + 31) / 32 * E : 0) * 4);   // per-block unit totals
   L.cnt_off = take((size_t)(E + 1) * 4);
@@ -81,6 +81,7 @@ WsLayout make_layout(const moe_config *c) {
   L.permute_end = o;
   const int ks = (c->dtype == MOE_BF16 && !router_is_fused(c)) ? router_ksplit(c) : 1;
   L.logits_part = take(ks > 1 ? (size_t)ks * T * E * 4 : 0);
+  L.sk_part = take(c->dtype == MOE_BF16 ? (size_t)kSkSlots * kSkSlotFloats * 4 : 0);
   L.step_end = o;
   L.logits = take((size_t)T * E * 4);
   L.probs = take((size_t)T * E * 4);
@@ -197,6 +198,8 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
   up.out_static_base = L.rows_cap;
   up.max_routed_rows = L.rows_cap;
   up.out = h;
+  up.sk_part = reinterpret_cast<float *>(ws + L.sk_part);
+  up.sk_flags = reinterpret_cast<int *>(ws + L.err + kSkFlagsOffset);
   up.err = err;
   cudaError_t e = launch_grouped_gemm(up, s);
   if (e != cudaSuccess) return e;
@@ -221,6 +224,8 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
   dn.max_routed_rows = L.rows_cap;
   dn.out = y_rows;
   dn.row_gate = row_gate;
+  dn.sk_part = up.sk_part;
+  dn.sk_flags = up.sk_flags;
   dn.err = err;
   return launch_grouped_gemm(dn, s);
 }
@@ -394,7 +399,9 @@ moe_status moe_check_device_errors(void *ws, size_t ws_bytes, moe_stream_t strea
   uint32_t word = 0;
   if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaMemcpy(&word, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
-  if (word != 0 && cudaMemset(ws, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
+  // after a device error the stream-K flags may be left set: clear the block
+  if (word != 0 && cudaMemset(ws, 0, std::min(ws_bytes, kCtrlBytes)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (flags) *flags = word;
   if (word & kErrTimeout) return MOE_ERR_TIMEOUT;
   if (word & kErrBadIndex) return MOE_ERR_DEVICE_CHECK;
@@ -403,7 +410,8 @@ moe_status moe_check_device_errors(void *ws, size_t ws_bytes, moe_stream_t strea
 
 moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream) {
   if (!ws || ws_bytes < 256) return MOE_ERR_INVALID_ARG;
-  return cuda_status(cudaMemsetAsync(ws, 0, 256, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(cudaMemsetAsync(ws, 0, std::min(ws_bytes, kCtrlBytes),
+                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 const char *moe_status_string(moe_status s) {

@@ -10,6 +10,29 @@
 
 namespace moe {
 
+// Launch `kern` on `s` with programmatic stream serialization, so that its
+// CTAs may start while the previous kernel on the stream finishes (the
+// kernels call pdl_wait() before touching global memory).  MOE_PDL=0 at
+// build time launches with plain stream order instead.
+#ifndef MOE_PDL
+#define MOE_PDL 1
+#endif
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = MOE_PDL ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Tokens per unit of the token-choice counting sort (one warp per unit).
 constexpr int kUnitTokens = 32;
 // Upper bound on routed experts and on top-k handled by the kernels.
@@ -23,8 +46,17 @@ constexpr size_t kFusedRouterSmem = 160 * 1024;
 // Byte offsets into the caller's workspace.  The first region (error word +
 // step scratch) is what the step entry points use; moe_forward adds its
 // intermediates after it.
+// Control block at the start of every workspace: the uint32 error word at
+// offset 0 and the stream-K ready flags (int32 [kSkSlots]) at kSkFlagsOffset.
+// All zero in a fresh workspace; kernels leave the flags at zero when they
+// finish without an error.
+constexpr size_t kCtrlBytes = 4096;
+constexpr size_t kSkFlagsOffset = 256;
+constexpr int kSkSlots = 192;                 // stream-K slots: >= CTAs of one GEMM launch
+constexpr int kSkSlotFloats = 128 * 256;      // one CTA's fp32 accumulator tile
+
 struct WsLayout {
-  size_t err;        // uint32 error word (256 B reserved)
+  size_t err;        // control block (kCtrlBytes): error word, stream-K flags
   size_t hist;       // int32 [k * nunit * E]  per-unit expert histogram
   size_t base;       // int32 [ceil(k * nunit / 32) * E]  per-expert totals of 32-unit blocks
   size_t cnt_off;    // int32 [E + 1]      exclusive scan of counts
@@ -33,6 +65,7 @@ struct WsLayout {
   size_t probs_t;    // fp32  [E * T]      transposed probabilities (expert choice)
   size_t permute_end;    // end of the permutation's scratch
   size_t logits_part;    // fp32 [ksplit][T][E] partial router logits (bf16 router with split K)
+  size_t sk_part;        // fp32 [kSkSlots][kSkSlotFloats] stream-K partial tiles (bf16 GEMMs)
   size_t step_end;
   // moe_forward intermediates
   size_t logits, probs, topk_idx, topk_gate, counts, offsets, n_dropped;
@@ -106,6 +139,8 @@ struct GroupedGemm {
   const float *bias;        // kEpiStoreF32: [N] or null (ignored when ksplit > 1)
   int ksplit;               // kEpiStoreF32, one static group: split K into ksplit parts and
   int64_t split_stride;     //   write part s of the output at out + s * split_stride
+  float *sk_part;           // stream-K partial tiles [kSkSlots][kSkSlotFloats] and their
+  int *sk_flags;            //   flags [kSkSlots] (zero between launches); null: no stream-K
   uint32_t *err;
 };
 cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s);

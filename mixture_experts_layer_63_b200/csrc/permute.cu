@@ -43,6 +43,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
                                                           const int32_t *__restrict__ offsets, int E,
                                                           int64_t T, int vpr, uint32_t *err) {
   const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
   const int64_t R = offsets[E];
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += nwarps) {
@@ -76,6 +78,8 @@ __global__ void __launch_bounds__(256) hist_units_kernel(const int32_t *__restri
                                                          int64_t T, int k, int E, int nunit,
                                                          int32_t *__restrict__ hist, uint32_t *err) {
   const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
   const int64_t u = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (u >= (int64_t)k * nunit) return;                  // whole warp leaves together
   const int r = (int)(u / nunit);
@@ -110,6 +114,8 @@ constexpr int kUnitsPerBlock = 32;
 __global__ void __launch_bounds__(1024) unit_sums_kernel(const int32_t *__restrict__ hist, int nu,
                                                          int E, int32_t *__restrict__ bsum) {
   __shared__ int s_part[1024];
+  pdl_wait();
+  pdl_trigger();
   const int G = max(1, (int)blockDim.x / E);
   const int g = threadIdx.x / E, e = threadIdx.x - g * E;
   const int u_begin = blockIdx.x * kUnitsPerBlock;
@@ -142,6 +148,8 @@ __global__ void __launch_bounds__(1024, 1) rank_units_kernel(
     int32_t *__restrict__ tok_rows, int32_t *__restrict__ row_token, float *__restrict__ row_gate,
     int32_t *__restrict__ sorted_q) {
   extern __shared__ int sm[];
+  pdl_wait();
+  pdl_trigger();
   int *s_base = sm;                                   // [32 units][E]
   int *s_pre = s_base + kUnitsPerBlock * E;           // [E] totals of earlier blocks
   int *s_tot = s_pre + E;                             // [E] totals of all blocks
@@ -340,6 +348,8 @@ __global__ void __launch_bounds__(1024) keep_select_kernel(
   __shared__ int scratch[32];
   __shared__ uint64_t s_prefix;
   __shared__ int s_remaining;
+  pdl_wait();
+  pdl_trigger();
   const int e = blockIdx.x;
   const int start = cnt_off[e];
   const int n = cnt_off[e + 1] - start;
@@ -386,6 +396,8 @@ __global__ void __launch_bounds__(1024) keep_select_kernel(
 __global__ void transpose_kernel(const float *__restrict__ in, float *__restrict__ out, int64_t T,
                                  int E) {
   __shared__ float tile[32][33];
+  pdl_wait();
+  pdl_trigger();
   const int64_t t0 = (int64_t)blockIdx.x * 32;
   const int e0 = blockIdx.y * 32;
   for (int i = threadIdx.y; i < 32; i += blockDim.y) {
@@ -409,6 +421,8 @@ __global__ void __launch_bounds__(1024) ec_select_kernel(
   __shared__ int scratch[32];
   __shared__ uint64_t s_prefix;
   __shared__ int s_remaining;
+  pdl_wait();
+  pdl_trigger();
   const int e = blockIdx.x;
   const float *pe = probs_t + (int64_t)e * T;
   auto key_of = [&](int i) -> uint64_t { return affinity_key(pe[i], (uint32_t)i); };
@@ -462,9 +476,11 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
   if (c->mode == MOE_EXPERT_CHOICE) {
     float *pt = reinterpret_cast<float *>(ws + L.probs_t);
     dim3 tb(32, 8), tg((unsigned)((T + 31) / 32), (unsigned)((E + 31) / 32));
-    transpose_kernel<<<tg, tb, 0, s>>>(probs, pt, T, E);
-    ec_select_kernel<<<E, 1024, 0, s>>>(pt, T, E, c->ec_capacity, counts, offsets, tok_rows,
-                                        row_token, row_gate, n_dropped);
+    cudaError_t e = launch_kernel(transpose_kernel, tg, tb, 0, s, probs, pt, T, E);
+    if (e != cudaSuccess) return e;
+    e = launch_kernel(ec_select_kernel, E, 1024, 0, s, pt, T, E, c->ec_capacity, counts, offsets,
+                      tok_rows, row_token, row_gate, n_dropped);
+    if (e != cudaSuccess) return e;
   } else {
   int32_t *hist = reinterpret_cast<int32_t *>(ws + L.hist);
   int32_t *bsum = reinterpret_cast<int32_t *>(ws + L.base);
@@ -474,30 +490,37 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
   const int keepfrac = (c->capacity <= 0 && c->keep_den > 0) ? 1 : 0;
   const int nu = c->k * L.nunit;
   const int nb = (nu + kUnitsPerBlock - 1) / kUnitsPerBlock;
-  if (!hist_ready)
-    hist_units_kernel<<<(unsigned)((nu + 7) / 8), 256, 0, s>>>(topk_idx, T, c->k, E, L.nunit, hist, err);
-  unit_sums_kernel<<<nb, 1024, 0, s>>>(hist, nu, E, bsum);
-  const size_t rank_smem = ((size_t)kUnitsPerBlock * E + 4 * E + 2 + 2048) * sizeof(int);
-  if (rank_smem > 48 * 1024) {
-    const cudaError_t e = cudaFuncSetAttribute(rank_units_kernel,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rank_smem);
+  cudaError_t e = cudaSuccess;
+  if (!hist_ready) {
+    e = launch_kernel(hist_units_kernel, (unsigned)((nu + 7) / 8), 256, 0, s, topk_idx, T, c->k, E,
+                      L.nunit, hist, err);
     if (e != cudaSuccess) return e;
   }
-  rank_units_kernel<<<nb, 1024, rank_smem, s>>>(topk_idx, topk_gate, T, c->k, E, L.nunit, nb, hist,
-                                                bsum, c->capacity, c->keep_num, c->keep_den, keepfrac,
-                                                counts, cnt_off, kept, offsets, n_dropped, tok_rows,
-                                                row_token, row_gate, sorted_q);
-  if (keepfrac)
-    keep_select_kernel<<<E, 1024, 0, s>>>(sorted_q, cnt_off, kept, offsets, probs, topk_gate, T,
-                                          c->k, E, tok_rows, row_token, row_gate);
+  e = launch_kernel(unit_sums_kernel, nb, 1024, 0, s, hist, nu, E, bsum);
+  if (e != cudaSuccess) return e;
+  const size_t rank_smem = ((size_t)kUnitsPerBlock * E + 4 * E + 2 + 2048) * sizeof(int);
+  if (rank_smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(rank_units_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)rank_smem);
+    if (e != cudaSuccess) return e;
+  }
+  e = launch_kernel(rank_units_kernel, nb, 1024, rank_smem, s, topk_idx, topk_gate, T, c->k, E,
+                    L.nunit, nb, hist, bsum, c->capacity, c->keep_num, c->keep_den, keepfrac, counts,
+                    cnt_off, kept, offsets, n_dropped, tok_rows, row_token, row_gate, sorted_q);
+  if (e != cudaSuccess) return e;
+  if (keepfrac) {
+    e = launch_kernel(keep_select_kernel, E, 1024, 0, s, sorted_q, cnt_off, kept, offsets, probs,
+                      topk_gate, T, c->k, E, tok_rows, row_token, row_gate);
+    if (e != cudaSuccess) return e;
+  }
   }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t want = (L.rows_cap + 7) / 8;
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 8));
-  gather_rows_kernel<<<blocks, 256, 0, s>>>(xv, xp, row_token, offsets, E, T, vpr, err);
-  return cudaGetLastError();
+  return launch_kernel(gather_rows_kernel, blocks, 256, 0, s, xv, xp, row_token, offsets, E, T, vpr,
+                       err);
 }
 
 }  // namespace moe

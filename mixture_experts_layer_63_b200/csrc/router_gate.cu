@@ -72,6 +72,8 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_gate_kernel(const GatePa
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int E = P.E, k = P.k;
+  pdl_wait();
+  pdl_trigger();
   int *s_hist = reinterpret_cast<int *>(smem);                    // [k][E]
   const int hist_ints = P.hist ? k * E : 0;
   // fused router: W_r staged as fp32 in 16-byte groups laid out so that the
@@ -291,8 +293,7 @@ cudaError_t launch_nv(int NV, const GateParams &P, int blocks, size_t smem, cuda
                                            (int)smem);                                         \
       if (e != cudaSuccess) return e;                                                          \
     }                                                                                          \
-    kern<<<blocks, kTokWarps * 32, smem, s>>>(P);                                              \
-    return cudaGetLastError();                                                                 \
+    return launch_kernel(kern, blocks, kTokWarps * 32, smem, s, P);                            \
   }
   switch (NV) {
     MOE_GATE_CASE(1)
@@ -363,8 +364,7 @@ cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float
           cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
-    kern<<<blocks, kTokWarps * 32, smem, s>>>(P);
-    return cudaGetLastError();
+    return launch_kernel(kern, blocks, kTokWarps * 32, smem, s, P);
   }
   return launch_nv(NV, P, blocks, smem, s);
 }
@@ -382,6 +382,8 @@ __global__ void __launch_bounds__(256) router_f32_kernel(const float *__restrict
                                                          int d, int E) {
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_trigger();
   if (t >= T) return;
   const float *xr = x + t * d;
   for (int e = 0; e < E; ++e) {
@@ -399,9 +401,8 @@ cudaError_t launch_router_f32(const moe_config *c, const float *x, const float *
                               const float *bias, float *logits, cudaStream_t s) {
   const int warps = 8;
   const int64_t blocks = (c->T + warps - 1) / warps;
-  router_f32_kernel<<<(unsigned)blocks, warps * 32, 0, s>>>(x, w, bias, logits, c->T, c->d_model,
-                                                            c->E);
-  return cudaGetLastError();
+  return launch_kernel(router_f32_kernel, (unsigned)blocks, warps * 32, 0, s, x, w, bias, logits,
+                       c->T, c->d_model, c->E);
 }
 
 }  // namespace moe
