@@ -30,7 +30,14 @@ What it computes, step by step, and the passage each step follows:
    d. expert choice: each expert takes its top-C tokens (LocMoE+ article,
       token-choice vs expert-choice routers);
    e. shared experts applied to every token with gate 1 (DeepSeekMoE
-      section 2, shared expert isolation equation).
+      section 2, shared expert isolation equation);
+   f. selection-key variants: DeepSeek-V3's auxiliary-loss-free balancing
+      (select on s + b, gate s + b; "MoE技术演进", DeepSeek-V3 item 1) with
+      its per-step bias update, and load-aware top-k (select on
+      g + alpha (1 - u); "MoE技术演进", interview question Q3, item 3);
+   g. GShard local group dispatching: the batch cut into G groups that
+      dispatch independently, capacity per group ("MoE技术演进", GShard
+      item 1).
 4. Permutation into expert-contiguous rows (the single-GPU counterpart of the
    count-then-fill send buffers, "大语言模型并行策略（七）：专家并行",
    section "MoE 中的 all-to-all 通信").
@@ -174,25 +181,80 @@ def group_limited_mask(logits: np.ndarray, n_groups: int, topk_groups: int) -> n
     return np.repeat(chosen, gsz, axis=1)
 
 
-def topk_route(logits: np.ndarray, probs: np.ndarray, k: int, n_groups: int = 0,
-               topk_groups: int = 0, renormalize: bool = False):
-    """Per token: the k experts with the largest logits, in rank order.
+ROUTE_RULES = ("softmax", "bias", "load")
 
-    A strictly larger logit ranks first; equal logits go to the lower expert
-    index (softmax is monotone, so this is the top-k of p with exact ties
-    broken by index).  With group limits only experts of the chosen groups
-    compete.  Gate = p of the chosen expert, or p / (sum of the chosen p,
-    summed in rank order in fp32) when ``renormalize``.
-    Returns (topk_idx int32 [T, k], topk_gate fp32 [T, k]).
+
+def selection_keys(logits: np.ndarray, probs: np.ndarray, rule: str = "softmax",
+                   state: np.ndarray | None = None, alpha: float = 0.0):
+    """Per (token, expert): the fp32 key top-k selects on and the gate a
+    chosen expert receives.
+
+    "softmax": key = the logit g, gate = p (the plain selector).
+    "bias"   : DeepSeek-V3's auxiliary-loss-free balancing ("MoE技术演进",
+               DeepSeek-V3 item 1): key = s + b_e, one rounded fp32 add,
+               with the affinity s read as the softmax probability p and
+               b = ``state`` the per-expert routing bias; the gate of a chosen
+               expert is s + b_e, as the printed formula gives it.
+    "load"   : load-aware top-k ("MoE技术演进", interview question Q3,
+               item 3): key = g_e + alpha * (1 - u_e) with g the logit and
+               u = ``state`` the expert's historical utilisation; in fp32
+               o_e = alpha * (1 - u_e) (two rounded operations), key = g + o_e
+               (one rounded add); the gate stays p.
     """
     l = np.asarray(logits, dtype=F32)
-    keys = -l.astype(np.float64)
+    p = np.asarray(probs, dtype=F32)
+    if rule == "softmax":
+        return l, p
+    st = np.asarray(state, dtype=F32)
+    if rule == "bias":
+        key = (p + st[None, :]).astype(F32)
+        return key, key
+    if rule == "load":
+        off = (F32(alpha) * (F32(1.0) - st).astype(F32)).astype(F32)
+        return (l + off[None, :]).astype(F32), p
+    raise ValueError(rule)
+
+
+def bias_update(counts: np.ndarray, bias: np.ndarray, T: int, k: int, gamma: float) -> np.ndarray:
+    """DeepSeek-V3's per-step update of the routing bias ("MoE技术演进",
+    DeepSeek-V3 item 1): an expert with more assignments than the mean T*k/E
+    (overloaded) lowers its bias by gamma, one with fewer raises it by gamma,
+    one exactly at the mean keeps it.  The load test is exact integer
+    arithmetic (c_e * E against T * k); the step is one rounded fp32 add."""
+    c = np.asarray(counts, dtype=np.int64)
+    b = np.asarray(bias, dtype=F32)
+    E = len(c)
+    g = F32(gamma)
+    over = c * E > T * k
+    under = c * E < T * k
+    out = b.copy()
+    out[over] = (b[over] - g).astype(F32)
+    out[under] = (b[under] + g).astype(F32)
+    return out
+
+
+def topk_route(logits: np.ndarray, probs: np.ndarray, k: int, n_groups: int = 0,
+               topk_groups: int = 0, renormalize: bool = False, rule: str = "softmax",
+               state: np.ndarray | None = None, alpha: float = 0.0):
+    """Per token: the k experts with the largest selection keys, in rank order.
+
+    Keys and gates come from ``selection_keys`` (plain: the logits, so by
+    monotonicity of softmax the top-k of p with exact ties broken by index).
+    A strictly larger key ranks first; equal keys go to the lower expert
+    index.  With group limits only experts of the chosen groups compete (a
+    group's score is its largest key).  Gate = that of the chosen expert, or
+    gate / (sum of the chosen gates, summed in rank order in fp32) when
+    ``renormalize``.
+    Returns (topk_idx int32 [T, k], topk_gate fp32 [T, k]).
+    """
+    key, gsrc = selection_keys(logits, probs, rule, state, alpha)
+    keys = -key.astype(np.float64)
     if n_groups > 0:
-        allowed = group_limited_mask(l, n_groups, topk_groups)
+        allowed = group_limited_mask(key, n_groups, topk_groups)
         keys = np.where(allowed, keys, np.inf)
     order = np.argsort(keys, axis=1, kind="stable")           # ties keep ascending expert index
     idx = order[:, :k].astype(np.int32)
-    gate = np.take_along_axis(np.asarray(probs, dtype=F32), idx, axis=1).astype(F32)
+    gate = np.take_along_axis(np.asarray(gsrc, dtype=F32), idx, axis=1).astype(F32)
     if renormalize:
         s = gate[:, 0].copy()
         for j in range(1, k):
@@ -245,37 +307,61 @@ def keep_count(n: np.ndarray, keep_num: int, keep_den: int) -> np.ndarray:
     return (n * keep_num + keep_den - 1) // keep_den
 
 
-def _priority_ranks(topk_idx: np.ndarray, E: int):
+def _priority_ranks(topk_idx: np.ndarray, E: int, local_groups: int = 1):
     """Stable counting sort of assignments by expert in priority order.
 
-    Assignment (t, j) has priority q = j * T + t.  Returns the expert of each
-    q, the q's grouped by expert (ascending q inside each expert), the start
-    of each expert's group, and the rank of each q inside its expert.
+    Assignment (t, j) is numbered q = j * T + t.  With one group its priority
+    is q itself.  With G local groups (tokens cut into G contiguous groups of
+    T/G) the priority is group-major: group g's assignments in the order
+    j * (T/G) + (t - g T/G), then group g + 1's.  Returns the expert of each
+    q, the q's grouped by expert (ascending priority inside each expert), the
+    start of each expert's group, the rank of each q inside its expert and
+    local group, and the local group of each q.
     """
     T, k = topk_idx.shape
+    G = max(1, int(local_groups))
+    Tg = T // G
     e_of_q = np.asarray(topk_idx, dtype=np.int64).T.reshape(-1)     # q = j*T + t
-    by_expert = np.argsort(e_of_q, kind="stable")                   # stable: ascending q per expert
+    q = np.arange(T * k)
+    t_of_q, j_of_q = q % T, q // T
+    g_of_q = t_of_q // Tg
+    prio = g_of_q * (k * Tg) + j_of_q * Tg + (t_of_q - g_of_q * Tg)
+    by_expert = np.lexsort((prio, e_of_q))                          # by expert, then priority
     counts = np.bincount(e_of_q, minlength=E).astype(np.int64)
     start = np.concatenate([[0], np.cumsum(counts)[:-1]])
     rank = np.empty(T * k, dtype=np.int64)
-    rank[by_expert] = np.arange(T * k) - start[e_of_q[by_expert]]
-    return e_of_q, by_expert, counts, start, rank
+    # rank inside (expert, group): position in the sorted list minus the
+    # position of the first assignment of the same (expert, group)
+    se, sg = e_of_q[by_expert], g_of_q[by_expert]
+    first = np.ones(T * k, dtype=bool)
+    first[1:] = (se[1:] != se[:-1]) | (sg[1:] != sg[:-1])
+    run_start = np.maximum.accumulate(np.where(first, np.arange(T * k), 0))
+    rank[by_expert] = np.arange(T * k) - run_start
+    return e_of_q, by_expert, counts, start, rank, g_of_q
 
 
 def dispatch_token_choice(topk_idx: np.ndarray, topk_gate: np.ndarray, probs: np.ndarray | None,
-                          E: int, capacity: int = 0, keep_num: int = 0, keep_den: int = 0) -> Dispatch:
+                          E: int, capacity: int = 0, keep_num: int = 0, keep_den: int = 0,
+                          local_groups: int = 1) -> Dispatch:
     """Token-choice dispatch with an optional capacity or keep-fraction.
 
     Capacity C > 0: the assignment of priority q is kept iff fewer than C
     assignments of smaller q went to the same expert; the rest overflow to
     the residual and contribute nothing here.
+    Local groups G > 1 (GShard item 1, "MoE技术演进"): the tokens form G
+    contiguous groups of T/G that dispatch independently; C is then the
+    capacity of one expert in one group, and ranks count only the group's
+    own assignments (T must be a multiple of G; capacity mode only).
     Keep-fraction num/den: expert e keeps ceil(n_e * num / den) of its n_e
     assignments, those with the largest p[t, e] (lower t on ties).
-    Rows of an expert are its kept assignments in priority order.
+    Rows of an expert are its kept assignments in priority order (group by
+    group when G > 1).
     """
     topk_idx = np.asarray(topk_idx)
     T, k = topk_idx.shape
-    e_of_q, by_expert, counts, start, rank = _priority_ranks(topk_idx, E)
+    if local_groups > 1 and (T % local_groups or capacity <= 0):
+        raise ValueError("local groups need T % G == 0 and a capacity")
+    e_of_q, by_expert, counts, start, rank, _ = _priority_ranks(topk_idx, E, local_groups)
     t_of_q = np.arange(T * k) % T
     keep = np.ones(T * k, dtype=bool)
     if capacity > 0:
@@ -381,6 +467,9 @@ class OracleConfig:
     n_groups: int = 0
     topk_groups: int = 0
     renormalize: bool = False
+    rule: str = "softmax"            # selection keys: "softmax", "bias", "load"
+    alpha: float = 0.0               # load-aware coefficient
+    local_groups: int = 1            # GShard local groups (capacity mode)
 
 
 @dataclass
@@ -394,13 +483,17 @@ class OracleResult:
     y: np.ndarray               # float64 [len(tokens), d]
 
 
-def route(cfg: OracleConfig, logits: np.ndarray):
-    """Steps 2-4 from given fp32 logits: probabilities, selection, dispatch."""
+def route(cfg: OracleConfig, logits: np.ndarray, state: np.ndarray | None = None):
+    """Steps 2-4 from given fp32 logits: probabilities, selection, dispatch.
+    ``state`` is the per-expert routing bias (rule "bias") or utilisation
+    (rule "load")."""
     probs = softmax_det(logits)
     if cfg.mode == "ec":
         return probs, None, None, dispatch_expert_choice(probs, cfg.ec_capacity)
-    idx, gate = topk_route(logits, probs, cfg.k, cfg.n_groups, cfg.topk_groups, cfg.renormalize)
-    disp = dispatch_token_choice(idx, gate, probs, cfg.E, cfg.capacity, cfg.keep_num, cfg.keep_den)
+    idx, gate = topk_route(logits, probs, cfg.k, cfg.n_groups, cfg.topk_groups, cfg.renormalize,
+                           cfg.rule, state, cfg.alpha)
+    disp = dispatch_token_choice(idx, gate, probs, cfg.E, cfg.capacity, cfg.keep_num, cfg.keep_den,
+                                 cfg.local_groups)
     return probs, idx, gate, disp
 
 
@@ -449,7 +542,8 @@ def combine_tokens(cfg: OracleConfig, x, w1, w2, w3, disp: Dispatch, tokens) -> 
     return y
 
 
-def forward(cfg: OracleConfig, x, w_router, bias, w1, w3, w2, tokens=None) -> OracleResult:
+def forward(cfg: OracleConfig, x, w_router, bias, w1, w3, w2, tokens=None,
+            state: np.ndarray | None = None) -> OracleResult:
     """The whole layer: routing for every token, outputs for ``tokens``.
 
     Routing (steps 1-4) always covers all T tokens because capacity,
@@ -457,7 +551,7 @@ def forward(cfg: OracleConfig, x, w_router, bias, w1, w3, w2, tokens=None) -> Or
     (step 5) are evaluated only for the requested tokens (all by default).
     """
     logits = router_logits(x, w_router, bias)
-    probs, idx, gate, disp = route(cfg, logits)
+    probs, idx, gate, disp = route(cfg, logits, state)
     T = logits.shape[0]
     tokens = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
     y = combine_tokens(cfg, x, w1, w2, w3, disp, tokens)

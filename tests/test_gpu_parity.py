@@ -48,9 +48,14 @@ def _route_gpu(cfg, inp):
 # steps 1-3a
 # ---------------------------------------------------------------------------
 
-# small cases whose router K is split over CTAs (d = 1024, few token tiles)
+# extra routing cases: the fused CUDA-core router (E <= 32, one and two passes
+# over the experts) and the tcgen05 router GEMM with its K split over CTAs
 ROUTE_EXTRA = {
-    "split_k_s": replace(WORKLOADS["gshard"], T=300),
+    # E <= 32: the logits come from the gate kernel's own CUDA-core router
+    "fused_router_s": replace(WORKLOADS["gshard"], T=300),
+    "fused_router_e32_s": replace(WORKLOADS["gshard"], T=200, E=32, d_model=512),
+    # E > 32: the tcgen05 router GEMM with K split over CTAs
+    "split_k_s": replace(WORKLOADS["deepseekmoe_tc"], T=300),
     "split_k_groups_s": replace(WORKLOADS["deepseek_v2"], T=200, d_model=1024, keep_num=0, keep_den=0),
 }
 

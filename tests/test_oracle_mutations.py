@@ -12,6 +12,7 @@ from tests import test_oracle_dispatch as TD
 from tests import test_oracle_ffn as TF
 from tests import test_oracle_gating as TG
 from tests import test_oracle_selection as TS
+from tests import test_oracle_routing_variants as TV
 
 
 def _expect_pin_failure(pin, *args):
@@ -23,17 +24,17 @@ def test_token_major_priority_is_caught(monkeypatch):
     """Priority q = t*k + j (token-major) instead of j*T + t."""
     orig = O._priority_ranks
 
-    def wrong(topk_idx, E):
+    def wrong(topk_idx, E, local_groups=1):
         T, k = topk_idx.shape
         e_tok_major = np.asarray(topk_idx, np.int64).reshape(-1)          # q' = t*k + j
         by = np.argsort(e_tok_major, kind="stable")
         # map back to the j*T + t numbering the rest of the oracle uses
         q_of_qp = (np.arange(T * k) % k) * T + np.arange(T * k) // k
-        e_of_q, _, counts, start, _ = orig(topk_idx, E)
+        e_of_q, _, counts, start, _, g_of_q = orig(topk_idx, E, local_groups)
         rank = np.empty(T * k, np.int64)
         rank[q_of_qp[by]] = np.arange(T * k) - start[e_tok_major[by]]
         by_expert = q_of_qp[by]
-        return e_of_q, by_expert, counts, start, rank
+        return e_of_q, by_expert, counts, start, rank, g_of_q
 
     monkeypatch.setattr(O, "_priority_ranks", wrong)
     _expect_pin_failure(TD.test_capacity_golden)
@@ -42,10 +43,13 @@ def test_token_major_priority_is_caught(monkeypatch):
 def test_reversed_tie_rule_is_caught(monkeypatch):
     orig = O.topk_route
 
-    def wrong(logits, probs, k, n_groups=0, topk_groups=0, renormalize=False):
+    def wrong(logits, probs, k, n_groups=0, topk_groups=0, renormalize=False, rule="softmax",
+              state=None, alpha=0.0):
         l = np.asarray(logits, np.float32)
         E = l.shape[1]
-        idx, gate = orig(l[:, ::-1], np.asarray(probs)[:, ::-1], k, n_groups, topk_groups, renormalize)
+        st = None if state is None else np.asarray(state)[::-1]
+        idx, gate = orig(l[:, ::-1], np.asarray(probs)[:, ::-1], k, n_groups, topk_groups, renormalize,
+                         rule, st, alpha)
         return (E - 1 - idx).astype(np.int32), gate                    # higher index wins ties
 
     monkeypatch.setattr(O, "topk_route", wrong)
@@ -55,8 +59,9 @@ def test_reversed_tie_rule_is_caught(monkeypatch):
 def test_dropped_gate_is_caught(monkeypatch):
     orig = O.dispatch_token_choice
 
-    def wrong(topk_idx, topk_gate, probs, E, capacity=0, keep_num=0, keep_den=0):
-        return orig(topk_idx, np.ones_like(topk_gate), probs, E, capacity, keep_num, keep_den)
+    def wrong(topk_idx, topk_gate, probs, E, capacity=0, keep_num=0, keep_den=0, local_groups=1):
+        return orig(topk_idx, np.ones_like(topk_gate), probs, E, capacity, keep_num, keep_den,
+                    local_groups)
 
     monkeypatch.setattr(O, "dispatch_token_choice", wrong)
     _expect_pin_failure(TF.test_k_equals_E_is_dense_soft_mixture, "relu")
@@ -135,3 +140,49 @@ def test_group_score_sum_is_caught(monkeypatch):
 
     monkeypatch.setattr(O, "group_limited_mask", wrong)
     _expect_pin_failure(TS.test_group_limited_brute_force)
+
+
+def test_bias_rule_on_logits_is_caught(monkeypatch):
+    """DeepSeek-V3 keys formed from the logits instead of the affinity p."""
+    orig = O.selection_keys
+
+    def wrong(logits, probs, rule="softmax", state=None, alpha=0.0):
+        if rule == "bias":
+            key = (np.asarray(logits, np.float32) + np.asarray(state, np.float32)[None, :]).astype(np.float32)
+            return key, key
+        return orig(logits, probs, rule, state, alpha)
+
+    monkeypatch.setattr(O, "selection_keys", wrong)
+    _expect_pin_failure(TV.test_bias_rule_brute_force, 0)
+
+
+def test_load_rule_without_complement_is_caught(monkeypatch):
+    """alpha * u instead of alpha * (1 - u)."""
+    orig = O.selection_keys
+
+    def wrong(logits, probs, rule="softmax", state=None, alpha=0.0):
+        if rule == "load":
+            off = (np.float32(alpha) * np.asarray(state, np.float32)).astype(np.float32)
+            return (np.asarray(logits, np.float32) + off[None, :]).astype(np.float32), np.asarray(probs, np.float32)
+        return orig(logits, probs, rule, state, alpha)
+
+    monkeypatch.setattr(O, "selection_keys", wrong)
+    _expect_pin_failure(TV.test_load_rule_brute_force, 0)
+
+
+def test_bias_update_sign_is_caught(monkeypatch):
+    orig = O.bias_update
+    monkeypatch.setattr(O, "bias_update", lambda c, b, T, k, g: orig(c, b, T, k, -g))
+    _expect_pin_failure(TV.test_bias_routing_golden)
+
+
+def test_global_ranks_under_local_groups_are_caught(monkeypatch):
+    """Capacity ranks counted over the whole batch instead of per group."""
+    orig = O._priority_ranks
+
+    def wrong(topk_idx, E, local_groups=1):
+        e_of_q, by_expert, counts, start, rank, g_of_q = orig(topk_idx, E, 1)
+        return e_of_q, by_expert, counts, start, rank, g_of_q
+
+    monkeypatch.setattr(O, "_priority_ranks", wrong)
+    _expect_pin_failure(TV.test_local_groups_are_independent_batches, 4)
