@@ -81,15 +81,20 @@ def _src_hash(name: str) -> str:
 
 def launches_per_step(w) -> int:
     """Kernels libmoe launches for one moe_forward of this workload."""
-    fused_router = w.dtype == "f32" and w.E <= 32 and w.E * w.d_model * 4 <= 160 * 1024
-    n = 1 if fused_router else 2              # router GEMM (or fp32 router inside the gate) + gate
+    # fp32 layers: the gate kernel computes the logits itself for E <= 32 when
+    # W_r (fp32) and the partial logits of 32 slices x 32 tokens fit 200 KB of
+    # shared memory; bf16 layers run the tcgen05 router GEMM first
+    fused_router = (w.dtype == "f32" and w.E <= 32
+                    and w.E * w.d_model * 4 + 32 * 32 * (w.E + 1) * 4 <= 200 * 1024)
+    n = 1 if fused_router else 2              # router GEMM (or the router inside the gate) + gate
     if w.mode == "ec":
         n += 2                                # transpose, expert-choice select
     else:
         n += 2                                # scan, rank/scatter
         if w.capacity_factor <= 0 and w.keep_den > 0:
             n += 1                            # per-expert affinity select
-    n += 1                                    # row gather
+    if w.dtype == "f32":
+        n += 1                                # row gather (bf16: inside the up-projection GEMM)
     n += 2                                    # up- and down-projection GEMMs
     n += 1                                    # combine
     return n
@@ -226,18 +231,22 @@ class OracleTimer:
         self.w1 = _DeviceExperts(inp.w1)
         self.w2 = _DeviceExperts(inp.w2)
         self.w3 = _DeviceExperts(inp.w3)
-        cap = O.capacity_from_factor(w.T, w.E, w.k, w.capacity_factor) if w.mode == "tc" else 0
+        Tg = w.T // max(1, w.local_groups)
+        cap = O.capacity_from_factor(Tg, w.E, w.k, w.capacity_factor) if w.mode == "tc" else 0
+        self.state = None if inp.route_state is None else inp.route_state.cpu().numpy()
         self.cfg = O.OracleConfig(E=w.E, S=w.S, k=w.k, act=w.act, mode=w.mode, capacity=cap,
                                   keep_num=w.keep_num, keep_den=w.keep_den,
                                   ec_capacity=w.ec_capacity if w.mode == "ec" else 0,
                                   n_groups=w.n_groups, topk_groups=w.topk_groups,
-                                  renormalize=w.renormalize)
+                                  renormalize=w.renormalize, rule=w.route_rule,
+                                  alpha=float(np.float32(w.route_alpha)),
+                                  local_groups=w.local_groups)
 
     def step(self, n: int, rng) -> tuple[float, float, float]:
         O = self.O
         t0 = time.perf_counter()
         logits = O.router_logits(self.x, self.w_router, self.bias)
-        _, _, _, disp = O.route(self.cfg, logits)
+        _, _, _, disp = O.route(self.cfg, logits, self.state)
         t1 = time.perf_counter()
         toks = np.sort(rng.choice(self.w.T, size=min(n, self.w.T), replace=False))
         O.combine_tokens(self.cfg, self.x, self.w1, self.w2, self.w3, disp, toks)
@@ -331,10 +340,11 @@ def run_ours(args, w) -> None:
 
     def step(ev=None):
         if ev is None:
-            api.moe_forward(cfg, inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, y, counts, ws)
+            api.moe_forward(cfg, inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, y, counts, ws,
+                            route_state=inp.route_state)
         else:
             api.moe_forward_timed(cfg, inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, y,
-                                  counts, ws, ev)
+                                  counts, ws, ev, route_state=inp.route_state)
 
     def new_events(n):
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n)] for _ in range(args.steps)]
@@ -379,16 +389,15 @@ def run_ours(args, w) -> None:
     per = np.array([[pevs[i][j].elapsed_time(pevs[i][j + 1]) for j in range(4)]
                     for i in range(args.steps)])          # ms: route, permute, ffn, combine
 
-    # algorithmic work of this batch: kept routed rows from the counts
-    if w.mode == "ec":
-        R = w.E * w.ec_capacity
-    elif w.capacity_factor > 0:
-        C = api.capacity_for(w.T, w.E, w.k, w.capacity_factor)
-        R = int(torch.clamp(counts.long(), max=C).sum().item())
-    elif w.keep_den > 0:
-        R = int(((counts.long() * w.keep_num + w.keep_den - 1) // w.keep_den).sum().item())
-    else:
-        R = w.T * w.k
+    # algorithmic work of this batch: the kept routed rows, offsets[E] of the
+    # same routing and permutation run once through the step entry points
+    B = api.step_buffers(cfg)
+    api.moe_route(cfg, inp.x, inp.w_router, inp.bias, B.logits, B.probs, B.topk_idx, B.topk_gate,
+                  B.ws, route_state=inp.route_state)
+    api.moe_permute(cfg, inp.x, B.topk_idx, B.topk_gate, B.probs, B.counts, B.offsets, B.tok_rows,
+                    B.row_token, B.row_gate, B.x_perm, B.n_dropped, B.ws)
+    R = int(B.offsets[w.E].item())
+    del B
     es = 4 if w.dtype == "f32" else 2
     rows = R + w.S * w.T
     nmat = 3 if w.act == "swiglu" else 2
@@ -404,7 +413,8 @@ def run_ours(args, w) -> None:
     traffic = tr["bytes"] if tr and tr.get("src") == h else None
 
     # end to end through the public layer object, host buffers
-    layer = api.MoELayer(cfg, inp.w_router, inp.w1, inp.w2, inp.w3, inp.bias)
+    layer = api.MoELayer(cfg, inp.w_router, inp.w1, inp.w2, inp.w3, inp.bias,
+                         route_state=inp.route_state)
     x_host = inp.x.cpu().pin_memory()
     y_host = torch.empty_like(x_host).pin_memory()
     x_dev = torch.empty_like(inp.x)

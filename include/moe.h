@@ -84,6 +84,15 @@ typedef enum moe_status {
 typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 typedef enum moe_act { MOE_ACT_RELU = 0, MOE_ACT_SWIGLU = 1 } moe_act;
 typedef enum moe_mode { MOE_TOKEN_CHOICE = 0, MOE_EXPERT_CHOICE = 1 } moe_mode;
+/* What token-choice top-k selects on ("MoE技术演进"):
+ *   SOFTMAX  key = logit g, gate = p (the plain selector);
+ *   BIAS     DeepSeek-V3 item 1, auxiliary-loss-free balancing: key = p + b_e
+ *            (one fp32 add; the affinity s read as p), gate = p + b_e as the
+ *            printed formula gives it; b = route_state [E];
+ *   LOAD     interview question Q3 item 3, load-aware top-k: key = g +
+ *            route_alpha * (1 - u_e) (fp32: o = alpha * (1 - u), key = g + o),
+ *            gate = p; u = route_state [E], the experts' utilisation. */
+typedef enum moe_route_rule { MOE_ROUTE_SOFTMAX = 0, MOE_ROUTE_BIAS = 1, MOE_ROUTE_LOAD = 2 } moe_route_rule;
 
 /* The layer.  Capacity, keep-fraction and expert choice are exclusive. */
 typedef struct moe_config {
@@ -103,6 +112,13 @@ typedef struct moe_config {
   int32_t act;         /* moe_act                                                   */
   int32_t mode;        /* moe_mode                                                  */
   int32_t dtype;       /* moe_dtype                                                 */
+  int32_t route_rule;  /* moe_route_rule (token choice; SOFTMAX in expert choice)   */
+  float route_alpha;   /* MOE_ROUTE_LOAD: alpha                                     */
+  int32_t local_groups;/* GShard local groups G (0 or 1: one group): T/G contiguous  */
+                       /*   tokens per group, each dispatching on its own with      */
+                       /*   `capacity` rows per expert; needs capacity > 0, T % G   */
+                       /*   == 0 and (T/G) % 32 == 0                                */
+  int32_t reserved;    /* 0                                                         */
 } moe_config;
 
 /* Buffer sizes of one configuration. */
@@ -119,24 +135,38 @@ typedef struct moe_sizes {
 MOE_API moe_status moe_query_sizes(const moe_config *cfg, moe_sizes *out);
 
 /* Steps 1-3a: router logits, softmax, token-choice top-k.
- *   x [T, d], w_router [E, d] (cfg dtype); bias [E] fp32 or NULL.
+ *   x [T, d], w_router [E, d] (cfg dtype); bias [E] fp32 or NULL (added to
+ *   the logits); route_state [E] fp32: the routing bias b (MOE_ROUTE_BIAS) or
+ *   the utilisation u (MOE_ROUTE_LOAD), NULL with MOE_ROUTE_SOFTMAX.
  *   out: logits [T, E], probs [T, E] fp32;
  *        topk_idx [T, k] int32 in rank order, topk_gate [T, k] fp32
  *        (both ignored and may be NULL in expert-choice mode).
- *   Top-k keys are the fp32 logits: strictly larger first, lower expert index
- *   on ties; with group limits only the topk_groups groups with the largest
- *   maximum logit (lower group on ties) compete.  p is computed in a fixed
+ *   Top-k keys are those of cfg->route_rule (the fp32 logits by default):
+ *   strictly larger first, lower expert index on ties; with group limits
+ *   only the topk_groups groups with the largest maximum key (lower group on
+ *   ties) compete.  p is computed in a fixed
  *   fp32 recipe (own exp, sequential ascending-expert sum, IEEE division) so
  *   that it is reproducible bit for bit.
  *   ws: workspace of at least step_workspace bytes. */
 MOE_API moe_status moe_route(const moe_config *cfg, const void *x, const void *w_router, const float *bias,
-                     float *logits, float *probs, int32_t *topk_idx, float *topk_gate, void *ws,
-                     size_t ws_bytes, moe_stream_t stream);
+                     const float *route_state, float *logits, float *probs, int32_t *topk_idx,
+                     float *topk_gate, void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Steps 2-3a from given fp32 logits [T, E] (the same arithmetic moe_route
  * applies after its router GEMM).  Outputs as moe_route. */
-MOE_API moe_status moe_gate(const moe_config *cfg, const float *logits, float *probs, int32_t *topk_idx,
-                    float *topk_gate, void *ws, size_t ws_bytes, moe_stream_t stream);
+MOE_API moe_status moe_gate(const moe_config *cfg, const float *logits, const float *route_state,
+                    float *probs, int32_t *topk_idx, float *topk_gate, void *ws, size_t ws_bytes,
+                    moe_stream_t stream);
+
+/* DeepSeek-V3's per-step routing-bias update ("MoE技术演进", DeepSeek-V3
+ * item 1): with counts [E] from a step (assignments per expert, as
+ * moe_permute / moe_forward report them), an expert above the mean load
+ * T*k/E lowers its bias by gamma, one below raises it by gamma, one exactly
+ * at the mean keeps it.  The load test is exact integer arithmetic
+ * (counts[e]*E against T*k); the step one fp32 add.  route_bias [E] fp32 is
+ * updated in place.  Token choice only. */
+MOE_API moe_status moe_route_bias_update(const moe_config *cfg, const int32_t *counts, float *route_bias,
+                                         float gamma, moe_stream_t stream);
 
 /* Steps 3b-4: capacity / keep-fraction / expert choice, then permutation.
  *   in : x [T, d]; token choice: topk_idx, topk_gate [T, k] (+ probs [T, E]
@@ -213,8 +243,9 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_rows, const 
  * per-expert assignment counts.  Equivalent to moe_route, moe_permute,
  * moe_expert_ffn and moe_combine in sequence. */
 MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const void *w_router,
-                       const float *bias, const void *w1, const void *w3, const void *w2, void *y,
-                       int32_t *counts_out, void *ws, size_t ws_bytes, moe_stream_t stream);
+                       const float *bias, const float *route_state, const void *w1, const void *w3,
+                       const void *w2, void *y, int32_t *counts_out, void *ws, size_t ws_bytes,
+                       moe_stream_t stream);
 
 /* moe_forward that also records caller-created CUDA events on `stream` at
  * its phase boundaries: events[0] before step 1, [1] after steps 1-3a
@@ -222,9 +253,10 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const void 
  * [4] after 5c (combine).  events: array of 5 cudaEvent_t handles (entries may
  * be NULL).  Same launches and results as moe_forward. */
 MOE_API moe_status moe_forward_timed(const moe_config *cfg, const void *x, const void *w_router,
-                                     const float *bias, const void *w1, const void *w3,
-                                     const void *w2, void *y, int32_t *counts_out, void *ws,
-                                     size_t ws_bytes, void *const *events, moe_stream_t stream);
+                                     const float *bias, const float *route_state, const void *w1,
+                                     const void *w3, const void *w2, void *y, int32_t *counts_out,
+                                     void *ws, size_t ws_bytes, void *const *events,
+                                     moe_stream_t stream);
 
 /* Waits for `stream`, then reads and clears the workspace's device error
  * word.  Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_CHECK; *flags (if

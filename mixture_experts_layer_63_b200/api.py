@@ -25,10 +25,13 @@ MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT = 4, 5, 6
 MOE_F32, MOE_BF16 = 0, 1
 MOE_ACT_RELU, MOE_ACT_SWIGLU = 0, 1
 MOE_TOKEN_CHOICE, MOE_EXPERT_CHOICE = 0, 1
+MOE_ROUTE_SOFTMAX, MOE_ROUTE_BIAS, MOE_ROUTE_LOAD = 0, 1, 2
+ROUTE_RULES = {"softmax": MOE_ROUTE_SOFTMAX, "bias": MOE_ROUTE_BIAS, "load": MOE_ROUTE_LOAD}
 
 EXPORTS = ("moe_query_sizes", "moe_route", "moe_gate", "moe_permute", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_check_device_errors", "moe_workspace_init",
-           "moe_status_string", "moe_permute_noalloc", "moe_forward_timed")
+           "moe_status_string", "moe_permute_noalloc", "moe_forward_timed",
+           "moe_route_bias_update")
 
 
 class MoeError(RuntimeError):
@@ -44,7 +47,9 @@ class MoeConfig(ctypes.Structure):
                 ("keep_den", ctypes.c_int32), ("ec_capacity", ctypes.c_int32),
                 ("n_groups", ctypes.c_int32), ("topk_groups", ctypes.c_int32),
                 ("renormalize", ctypes.c_int32), ("act", ctypes.c_int32),
-                ("mode", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+                ("mode", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("route_rule", ctypes.c_int32), ("route_alpha", ctypes.c_float),
+                ("local_groups", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class MoeSizes(ctypes.Structure):
@@ -68,13 +73,14 @@ def lib() -> ctypes.CDLL:
         sz = ctypes.c_size_t
         sig = {
             "moe_query_sizes": [cfgp, ctypes.POINTER(MoeSizes)],
-            "moe_route": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
-            "moe_gate": [cfgp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_route": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_gate": [cfgp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_route_bias_update": [cfgp, vp, vp, ctypes.c_float, vp],
             "moe_permute": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_expert_ffn": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_combine": [cfgp, vp, vp, vp, vp],
-            "moe_forward": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
-            "moe_forward_timed": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+            "moe_forward": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+            "moe_forward_timed": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                   ctypes.POINTER(ctypes.c_void_p), vp],
             "moe_check_device_errors": [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)],
             "moe_workspace_init": [vp, sz, vp],
@@ -142,6 +148,11 @@ def config_from_workload(w: Workload, T: int | None = None) -> MoeConfig:
     c.act = MOE_ACT_SWIGLU if w.act == "swiglu" else MOE_ACT_RELU
     c.mode = MOE_EXPERT_CHOICE if w.mode == "ec" else MOE_TOKEN_CHOICE
     c.dtype = MOE_F32 if w.dtype == "f32" else MOE_BF16
+    c.route_rule = ROUTE_RULES[w.route_rule]
+    c.route_alpha = w.route_alpha
+    c.local_groups = w.local_groups
+    if w.local_groups > 1:           # capacity of one expert in one group
+        c.capacity = capacity_for(T // w.local_groups, w.E, w.k, w.capacity_factor)
     return c
 
 
@@ -171,17 +182,25 @@ def new_workspace(cfg: MoeConfig, device="cuda", step_only: bool = False) -> tor
 # entry points (same names as the C ABI)
 # ---------------------------------------------------------------------------
 
-def moe_route(cfg, x, w_router, bias, logits, probs, topk_idx, topk_gate, ws, stream=None):
+def moe_route(cfg, x, w_router, bias, logits, probs, topk_idx, topk_gate, ws, stream=None, *,
+              route_state=None):
     wp, wn = _ws(ws)
     _check("moe_route", lib().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias),
-                                        _ptr(logits), _ptr(probs), _ptr(topk_idx), _ptr(topk_gate),
-                                        wp, wn, _stream(stream)))
+                                        _ptr(route_state), _ptr(logits), _ptr(probs), _ptr(topk_idx),
+                                        _ptr(topk_gate), wp, wn, _stream(stream)))
 
 
-def moe_gate(cfg, logits, probs, topk_idx, topk_gate, ws, stream=None):
+def moe_gate(cfg, logits, probs, topk_idx, topk_gate, ws, stream=None, *, route_state=None):
     wp, wn = _ws(ws)
-    _check("moe_gate", lib().moe_gate(ctypes.byref(cfg), _ptr(logits), _ptr(probs), _ptr(topk_idx),
-                                      _ptr(topk_gate), wp, wn, _stream(stream)))
+    _check("moe_gate", lib().moe_gate(ctypes.byref(cfg), _ptr(logits), _ptr(route_state), _ptr(probs),
+                                      _ptr(topk_idx), _ptr(topk_gate), wp, wn, _stream(stream)))
+
+
+def moe_route_bias_update(cfg, counts, route_bias, gamma: float, stream=None):
+    """DeepSeek-V3's bias step: route_bias[e] -/+ gamma for experts above /
+    below the mean load T*k/E, in place."""
+    _check("moe_route_bias_update", lib().moe_route_bias_update(
+        ctypes.byref(cfg), _ptr(counts), _ptr(route_bias), float(gamma), _stream(stream)))
 
 
 def moe_permute(cfg, x, topk_idx, topk_gate, probs, counts, offsets, tok_rows, row_token, row_gate,
@@ -205,14 +224,16 @@ def moe_combine(cfg, y_rows, tok_rows, y, stream=None):
                                             _stream(stream)))
 
 
-def moe_forward(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, stream=None):
+def moe_forward(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, stream=None, *,
+                route_state=None):
     wp, wn = _ws(ws)
     _check("moe_forward", lib().moe_forward(
-        ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y),
-        _ptr(counts_out), wp, wn, _stream(stream)))
+        ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(route_state), _ptr(w1), _ptr(w3),
+        _ptr(w2), _ptr(y), _ptr(counts_out), wp, wn, _stream(stream)))
 
 
-def moe_forward_timed(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, events, stream=None):
+def moe_forward_timed(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, events, stream=None, *,
+                      route_state=None):
     """moe_forward recording 5 torch CUDA events at its phase boundaries
     (before routing, after routing, after permutation, after the expert FFNs,
     after the combine).  Each event must have been recorded once before, so
@@ -220,8 +241,8 @@ def moe_forward_timed(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, eve
     wp, wn = _ws(ws)
     handles = (ctypes.c_void_p * 5)(*[ev.cuda_event if ev is not None else None for ev in events])
     _check("moe_forward_timed", lib().moe_forward_timed(
-        ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w1), _ptr(w3), _ptr(w2), _ptr(y),
-        _ptr(counts_out), wp, wn, handles, _stream(stream)))
+        ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(route_state), _ptr(w1), _ptr(w3),
+        _ptr(w2), _ptr(y), _ptr(counts_out), wp, wn, handles, _stream(stream)))
 
 
 def moe_check_device_errors(ws, stream=None) -> int:
@@ -289,17 +310,24 @@ def step_buffers(cfg: MoeConfig, device="cuda") -> StepBuffers:
 class MoELayer:
     """The layer's weights plus a workspace; ``layer(x)`` runs moe_forward."""
 
-    def __init__(self, cfg: MoeConfig, w_router, w1, w2, w3=None, bias=None):
+    def __init__(self, cfg: MoeConfig, w_router, w1, w2, w3=None, bias=None, route_state=None):
         self.cfg = cfg
         self.w_router, self.w1, self.w2, self.w3, self.bias = w_router, w1, w2, w3, bias
+        if route_state is None and cfg.route_rule != MOE_ROUTE_SOFTMAX:
+            route_state = torch.zeros(cfg.E, dtype=torch.float32, device=w1.device)
+        self.route_state = route_state     # routing bias (DeepSeek-V3) or utilisation
         self.ws = new_workspace(cfg, w1.device)
         self.counts = torch.empty(cfg.E, dtype=torch.int32, device=w1.device)
 
     def __call__(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
         y = out if out is not None else torch.empty_like(x)
         moe_forward(self.cfg, x, self.w_router, self.bias, self.w1, self.w3, self.w2, y,
-                    self.counts, self.ws, stream)
+                    self.counts, self.ws, stream, route_state=self.route_state)
         return y
+
+    def update_route_bias(self, gamma: float, stream=None):
+        """DeepSeek-V3's bias step from the last forward's counts."""
+        moe_route_bias_update(self.cfg, self.counts, self.route_state, gamma, stream)
 
 
 # ---------------------------------------------------------------------------

@@ -54,16 +54,23 @@ constexpr int kMaxGroups = 320;
 #define MOE_PAIR_MIN_ROWS 384
 #endif
 constexpr uint32_t kABytes = BM * BK * 2;   // 16 KB
+// Gathered A rows: warps 2 and 3 copy them with cp.async (16 bytes a copy,
+// 128-byte swizzle applied by hand) and report a stage full after issuing
+// this many later stages.  Deadlock-free for any lag below the ring depth;
+// the MMA then has (depth - 1 - lag) stages ready ahead of it, so the lag is
+// kept short: a lag of depth - 1 would tie every report to the completion of
+// the previous stage's MMAs.
+constexpr int kGatherThreads = 64;
+#ifndef MOE_GATHER_LAG_ONE
+#define MOE_GATHER_LAG_ONE 1
+#endif
+#ifndef MOE_GATHER_LAG_PAIR
+#define MOE_GATHER_LAG_PAIR 2
+#endif
 // Stream-K tail: a piece of a split tile covers at least this many k-blocks
 constexpr int kSkMinUnits = 8;
 #ifndef MOE_STREAM_K
 #define MOE_STREAM_K 1
-#endif
-// The TMA producer also asks L2 for the k-block this many loads ahead of the
-// one it is loading (0: off), so operand fetches from HBM start earlier than
-// the shared-memory ring alone allows.
-#ifndef MOE_L2_PREFETCH
-#define MOE_L2_PREFETCH 0
 #endif
 
 struct Params {
@@ -75,6 +82,8 @@ struct Params {
   int n_routed, n_static, G;
   int64_t rows_static, a_static_base, a_static_stride, out_static_base;
   int64_t a_rows;
+  int64_t seg_rows;         // routed segments lie in rows [0, seg_rows) (of A, or of gather_rows)
+  int reverse;              // visit the tiles last group first
   const int32_t *offsets;
   void *out;
   const float *row_gate;
@@ -83,6 +92,9 @@ struct Params {
   int64_t split_stride;     //   ksplit parts of the output, split_stride elements apart
   float *sk_part;           // stream-K partial accumulators, one kSkSlotFloats slot per CTA
   int *sk_flags;            //   and one ready flag per slot; null: no stream-K
+  const int32_t *gather_rows;  // routed A row r = gather_src[gather_rows[r]] (null: A as stored)
+  const void *gather_src;      //   bf16 [src_rows, K]
+  int64_t src_rows;
   uint32_t *err;
 };
 
@@ -117,15 +129,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// the same with acquire at cluster scope: for phases completed by arrivals
+// of the other CTA of a pair, whose shared-memory writes must be visible
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase of parity `parity` to complete.  Returns false
 // when the CTA is aborting or the time limit passed (then it raises the
 // timeout bit and starts the abort).
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           uint32_t *err) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto try_wait = [&]() {
+    return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+  };
+  if (try_wait()) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (try_wait()) return true;
     if ((i & 63u) == 0) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > kWaitLimitNs) {
@@ -152,14 +182,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
-}
-
-// hint: bring one box of the tensor into L2 (no shared memory, no completion)
-__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap *map, int c0, int c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1)
-               : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map) {
@@ -226,6 +248,66 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 16-byte global -> shared copy; src_bytes 0 fills the 16 bytes with zeros
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// make this thread's generic-proxy shared-memory writes visible to the
+// async proxy (the tensor cores read the tile through it)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Gather role: the A rows of routed tiles, one stage at a time.  Thread
+// gt = 32 w + l of kGatherThreads copies 16-byte chunk c = l mod 8 of the 16
+// tile rows r_i = 8 i + 4 w + l / 8: each warp-wide copy covers four whole
+// 128-byte rows (coalesced).  Chunk c of row r lands at
+// r * 128 + ((c ^ (r mod 8)) << 4), the 128-byte swizzle TMA would apply;
+// r mod 8 is the same for all 16 rows of a thread.  Rows past the segment
+// are zero-filled.
+struct GatherRows {
+  int32_t tok[16];             // source row of each of the thread's rows (-1: zero fill)
+
+  __device__ __forceinline__ void load(const Params &P, int seg_off, int seg_rows, int row0, int gt) {
+    const int rb = 4 * (gt >> 5) + ((gt & 31) >> 3);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int r = row0 + 8 * i + rb;
+      int t = -1;
+      if (r < seg_rows) {
+        t = P.gather_rows[seg_off + r];
+        if (t < 0 || t >= P.src_rows) {
+          raise_error(P.err, kErrBadIndex);
+          t = -1;
+        }
+      }
+      tok[i] = t;
+    }
+  }
+  __device__ __forceinline__ void clear() {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) tok[i] = -1;
+  }
+  __device__ __forceinline__ void issue(uint32_t sa, int gt, int kb, const char *xs,
+                                        int64_t row_bytes) const {
+    const int c = gt & 7;
+    const int rb = 4 * (gt >> 5) + ((gt & 31) >> 3);
+    const uint32_t dst0 = sa + (uint32_t)rb * 128u + ((uint32_t)(c ^ rb) << 4);
+    const int64_t col = (int64_t)kb * 128 + c * 16;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const bool ok = tok[i] >= 0;
+      cp_async_16(dst0 + (uint32_t)i * 1024u, ok ? xs + (int64_t)tok[i] * row_bytes + col : xs,
+                  ok ? 16u : 0u);
+    }
+  }
+};
 
 // ---- CTA pairs (cta_group::2): two CTAs of a cluster share one MMA ----------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -390,21 +472,6 @@ struct Sched {
     return q;
   }
   __device__ __forceinline__ bool nonempty(int q) const { return start(q + 1) > start(q); }
-};
-
-// A second cursor over a worker's k-blocks, running ahead of the producer.
-struct Ahead {
-  Sched sc;
-  int tile, kb, kb1, part;
-  bool live;
-  __device__ __forceinline__ void init(const Sched &s, int skip) {
-    sc = s;
-    live = sc.next(tile, kb, kb1, part);
-    for (int i = 0; i < skip; ++i) step();
-  }
-  __device__ __forceinline__ void step() {
-    if (live && ++kb >= kb1) live = sc.next(tile, kb, kb1, part);
-  }
 };
 
 // Stream-K partial accumulator slot: 128 rows x 256 fp32 columns, stored as
@@ -635,9 +702,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+  const bool gather = P.gather_rows != nullptr;
   if (tid == 32) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_bar[s], 1);
+      mbar_init(&full_bar[s], 1 + (gather ? kGatherThreads : 0));
       mbar_init(&empty_bar[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -673,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (g < P.n_routed) {
           off = P.offsets[g];
           rows = P.offsets[g + 1] - off;
-          if (rows < 0 || off < 0 || (int64_t)off + rows > P.a_rows) {
+          if (rows < 0 || off < 0 || (int64_t)off + rows > P.seg_rows) {
             raise_error(P.err, kErrBadIndex);
             rows = 0;
             off = 0;
@@ -722,31 +790,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                          (int64_t)tl.m * BM;
       return routed ? &map_a : &map_a_static;
     };
-    Ahead ahead;
-    if (MOE_L2_PREFETCH > 0) ahead.init(sc, MOE_L2_PREFETCH);
     while (ok && sc.next(tile, kb0, kb1, part)) {
-      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
       int64_t a_row;
       const CUtensorMap *ma = a_of(tl, a_row);
       const int b_row = tl.g * P.N + tl.n * P.bnh;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (MOE_L2_PREFETCH > 0 && ahead.live) {
-          const Tile pt = decode_tile(ahead.tile, s_prefix, P.G, P.nt);
-          int64_t prow;
-          const CUtensorMap *pm = a_of(pt, prow);
-          const int pb = pt.g * P.N + pt.n * P.bnh;
-          tma_prefetch_l2(pm, ahead.kb * BK, (int)prow);
-          tma_prefetch_l2(&map_b, ahead.kb * BK, pb);
-          if (EPI == kEpiSwiglu) tma_prefetch_l2(&map_b3, ahead.kb * BK, pb);
-          ahead.step();
-        }
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
         uint8_t *sa = smem + (size_t)stage * stage_bytes;
         uint8_t *sb = sa + kABytes;
-        mbar_expect_tx(&full_bar[stage], stage_bytes);
+        const bool a_by_tma = !(gather && tl.g < P.n_routed);   // else the gather warps
+        mbar_expect_tx(&full_bar[stage], a_by_tma ? stage_bytes : b_bytes);
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-        tma_load_2d(sa, ma, &full_bar[stage], kb * BK, (int)a_row);
+        if (a_by_tma) tma_load_2d(sa, ma, &full_bar[stage], kb * BK, (int)a_row);
         if (EPI == kEpiSwiglu) {
           tma_load_2d(sb, &map_b, &full_bar[stage], kb * BK, b_row);
           tma_load_2d(sb + (b_bytes >> 1), &map_b3, &full_bar[stage], kb * BK, b_row);
@@ -793,6 +850,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     // all MMAs issued by this thread complete before TMEM can be freed
     umma_commit(&drain_bar);
     mbar_wait_drain(&drain_bar, 0);
+  } else if (gather && (warp == 2 || warp == 3)) {
+    // ------------------------- gather of routed A rows -------------------------
+    constexpr int kLag = MOE_GATHER_LAG_ONE;
+    static_assert(kLag >= 0 && kLag < kStages, "gather lag below the ring depth");
+    const int gt = tid - 64;
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0, arrived = 0;
+    bool ok = true;
+    const char *xs = static_cast<const char *>(P.gather_src);
+    const int64_t row_bytes = (int64_t)P.K * 2;
+    while (ok && sc.next(tile, kb0, kb1, part)) {
+      const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
+      const bool routed = tl.g < P.n_routed;
+      GatherRows gr;
+      if (routed) gr.load(P, s_off[tl.g], s_rows[tl.g], tl.m * BM, gt);
+      else gr.clear();
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+        if (routed) gr.issue(smem_u32(smem + (size_t)stage * stage_bytes), gt, kb, xs, row_bytes);
+        cp_async_commit();
+        ++issued;
+        if (issued - arrived > kLag) {
+          cp_async_wait<kLag>();
+          fence_proxy_async_smem();
+          mbar_arrive(&full_bar[arrived % kStages]);
+          ++arrived;
+        }
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    for (; arrived < issued; ++arrived) mbar_arrive(&full_bar[arrived % kStages]);
   } else if (warp >= 4) {
     // -------------------------------- epilogue --------------------------------
     const int ew = warp - 4;                     // TMEM lanes 32*ew .. 32*ew+31
@@ -800,7 +891,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     while (sc.next(tile, kb0, kb1, part)) {
-      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
       if (!mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
@@ -878,9 +969,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
+  const bool gather = P.gather_rows != nullptr;
   if (tid == 32) {
     for (int st = 0; st < kPairStages; ++st) {
-      mbar_init(&full_bar[st], 1);
+      // the even CTA's: its expect_tx arrival, then both CTAs' gather threads
+      mbar_init(&full_bar[st], 1 + (gather ? 2 * kGatherThreads : 0));
       mbar_init(&empty_bar[st], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -915,7 +1008,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (g < P.n_routed) {
           off = P.offsets[g];
           rows = P.offsets[g + 1] - off;
-          if (rows < 0 || off < 0 || (int64_t)off + rows > P.a_rows) {
+          if (rows < 0 || off < 0 || (int64_t)off + rows > P.seg_rows) {
             raise_error(P.err, kErrBadIndex);
             rows = 0;
             off = 0;
@@ -966,33 +1059,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       b_row = tl.g * P.N + tl.n * P.bnh + ((EPI == kEpiSwiglu) ? 0 : (int)rank * (P.bn / 2));
       return routed ? &map_a : &map_a_static;
     };
-    Ahead ahead;
-    if (MOE_L2_PREFETCH > 0) ahead.init(sc, MOE_L2_PREFETCH);
     while (ok && sc.next(tile, kb0, kb1, part)) {
-      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
       int64_t a_row;
       int b_row;
       const CUtensorMap *ma = rows_of(tl, a_row, b_row);
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (MOE_L2_PREFETCH > 0 && ahead.live) {
-          const Tile pt = decode_tile(ahead.tile, s_prefix, P.G, P.nt);
-          int64_t pa;
-          int pb;
-          const CUtensorMap *pm = rows_of(pt, pa, pb);
-          tma_prefetch_l2(pm, ahead.kb * BK, (int)pa);
-          tma_prefetch_l2(mb, ahead.kb * BK, pb);
-          ahead.step();
-        }
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
         uint8_t *sa = smem + (size_t)stage * stage_bytes;
         uint8_t *sb = sa + kABytes;
         const uint32_t fb = smem_u32(&full_bar[stage]) & 0xFEFFFFFFu;   // the even CTA's barrier
+        const bool a_by_tma = !(gather && tl.g < P.n_routed);          // else the gather warps
         if (rank == 0) {
-          mbar_expect_tx(&full_bar[stage], 2 * stage_bytes);
+          mbar_expect_tx(&full_bar[stage], a_by_tma ? 2 * stage_bytes : 2 * b_bytes);
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         }
-        tma_load_2d_pair(sa, ma, fb, kb * BK, (int)a_row);
+        if (a_by_tma) tma_load_2d_pair(sa, ma, fb, kb * BK, (int)a_row);
         tma_load_2d_pair(sb, mb, fb, kb * BK, b_row);
         if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
       }
@@ -1014,7 +1097,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&full_bar[stage], phase, &s_abort, P.err)) { ok = false; break; }
+        if (!mbar_wait<true>(&full_bar[stage], phase, &s_abort, P.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + (size_t)stage * stage_bytes);
         const uint32_t b_addr = a_addr + kABytes;
@@ -1032,6 +1115,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     umma_commit_pair_local(&drain_bar);
     mbar_wait_drain(&drain_bar, 0);
+  } else if (gather && (warp == 2 || warp == 3)) {
+    // --------------- gather of this CTA's 128 routed A rows ---------------
+    constexpr int kLag = MOE_GATHER_LAG_PAIR;
+    static_assert(kLag >= 0 && kLag < kPairStages, "gather lag below the ring depth");
+    const int gt = tid - 64;
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0, arrived = 0;
+    bool ok = true;
+    const char *xs = static_cast<const char *>(P.gather_src);
+    const int64_t row_bytes = (int64_t)P.K * 2;
+    // stage s is full on the even CTA's barrier
+    auto arrive_full = [&](int s) {
+      if (rank == 0) mbar_arrive(&full_bar[s]);
+      else mbar_arrive_cluster(mapa_shared(smem_u32(&full_bar[s]), 0));
+    };
+    while (ok && sc.next(tile, kb0, kb1, part)) {
+      const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
+      const bool routed = tl.g < P.n_routed;
+      GatherRows gr;
+      if (routed) gr.load(P, s_off[tl.g], s_rows[tl.g], tl.m * PM + (int)rank * BM, gt);
+      else gr.clear();
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+        if (routed) gr.issue(smem_u32(smem + (size_t)stage * stage_bytes), gt, kb, xs, row_bytes);
+        cp_async_commit();
+        ++issued;
+        if (issued - arrived > kLag) {
+          cp_async_wait<kLag>();
+          fence_proxy_async_smem();
+          arrive_full((int)(arrived % kPairStages));
+          ++arrived;
+        }
+        if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    for (; arrived < issued; ++arrived) arrive_full((int)(arrived % kPairStages));
   } else if (warp >= 4) {
     // -------------------------------- epilogue --------------------------------
     const int ew = warp - 4;
@@ -1041,7 +1163,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     while (sc.next(tile, kb0, kb1, part)) {
-      const Tile tl = decode_tile(tile, s_prefix, P.G, P.nt);
+      const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
       if (!mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
@@ -1188,6 +1310,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   P.a_static_stride = g.a_static_stride;
   P.out_static_base = g.out_static_base;
   P.a_rows = g.a_rows;
+  P.seg_rows = g.gather_rows ? g.max_routed_rows : g.a_rows;
   P.offsets = g.offsets;
   P.out = g.out;
   P.row_gate = g.row_gate;
@@ -1198,6 +1321,12 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   const bool sk = MOE_STREAM_K && g.epi != kEpiStoreF32 && g.sk_part && g.sk_flags;
   P.sk_part = sk ? g.sk_part : nullptr;
   P.sk_flags = sk ? g.sk_flags : nullptr;
+  P.reverse = g.reverse;
+  P.gather_rows = g.gather_rows;
+  P.gather_src = g.gather_src;
+  P.src_rows = g.src_rows;
+  if (g.gather_rows && (!g.gather_src || g.epi == kEpiStoreF32 || g.n_routed == 0))
+    return cudaErrorInvalidValue;
   P.err = g.err;
   if (P.G <= 0 || P.G > kMaxGroups || P.bn > 256 || g.K % BK != 0) return cudaErrorInvalidValue;
   if (g.ksplit > 1 && (g.epi != kEpiStoreF32 || g.n_routed != 0)) return cudaErrorInvalidValue;

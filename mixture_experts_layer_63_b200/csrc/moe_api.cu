@@ -21,6 +21,16 @@ moe_status validate(const moe_config *c) {
       (c->keep_den == 0 && c->keep_num != 0))
     return MOE_ERR_INVALID_ARG;
   if (c->n_groups < 0 || c->topk_groups < 0) return MOE_ERR_INVALID_ARG;
+  if (c->route_rule < MOE_ROUTE_SOFTMAX || c->route_rule > MOE_ROUTE_LOAD || c->reserved != 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!(c->route_alpha == c->route_alpha)) return MOE_ERR_INVALID_ARG;       // NaN
+  if (c->local_groups < 0) return MOE_ERR_INVALID_ARG;
+  if (c->local_groups > 1) {
+    // GShard local groups: capacity dispatch of contiguous 32-token-aligned groups
+    if (c->mode != MOE_TOKEN_CHOICE || c->capacity <= 0) return MOE_ERR_INVALID_ARG;
+    if (c->T % c->local_groups != 0) return MOE_ERR_INVALID_ARG;
+    if ((c->T / c->local_groups) % kUnitTokens != 0) return MOE_ERR_UNSUPPORTED;
+  }
   if (c->mode == MOE_TOKEN_CHOICE) {
     if (c->k < 1 || c->k > c->E) return MOE_ERR_INVALID_ARG;
     if (c->capacity > 0 && c->keep_den > 0) return MOE_ERR_INVALID_ARG;   // exclusive drop rules
@@ -35,7 +45,7 @@ moe_status validate(const moe_config *c) {
   } else {
     if (c->ec_capacity < 1 || c->ec_capacity > c->T) return MOE_ERR_INVALID_ARG;
     if (c->n_groups != 0 || c->topk_groups != 0 || c->capacity > 0 || c->keep_den > 0 ||
-        c->renormalize)
+        c->renormalize || c->route_rule != MOE_ROUTE_SOFTMAX)
       return MOE_ERR_INVALID_ARG;
     if ((int64_t)c->E * c->ec_capacity > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
   }
@@ -51,6 +61,16 @@ moe_status validate(const moe_config *c) {
   }
   return MOE_OK;
 }
+
+// moe_forward gathers the routed rows inside the up-projection GEMM (bf16);
+// MOE_FUSED_GATHER=0 at build time runs the separate gather kernel instead
+#ifndef MOE_FUSED_GATHER
+#define MOE_FUSED_GATHER 0
+#endif
+
+#ifndef MOE_DOWN_REVERSE
+#define MOE_DOWN_REVERSE 0
+#endif
 
 WsLayout make_layout(const moe_config *c) {
   WsLayout L{};
@@ -73,7 +93,7 @@ WsLayout make_layout(const moe_config *c) {
   };
   L.err = take(kCtrlBytes);
   L.hist = take((size_t)hist_ints * 4);
-  L.base = take((size_t)(tc ? (k * L.nunit + 31) / 32 * E : 0) * 4);   // per-block unit totals
+  L.base = take((size_t)(tc ? unit_grid(c).nb * E : 0) * 4);           // per-block unit totals
   L.cnt_off = take((size_t)(E + 1) * 4);
   L.kept = take((size_t)E * 4);
   L.sorted_q = take(keepfrac ? (size_t)T * k * 4 : 0);
@@ -93,7 +113,9 @@ WsLayout make_layout(const moe_config *c) {
   L.tok_rows = take((size_t)L.tok_rows_len * 4);
   L.row_token = take((size_t)L.rows_cap * 4);
   L.row_gate = take((size_t)L.rows_cap * 4);
-  L.x_perm = take((size_t)L.rows_cap * c->d_model * es);
+  // moe_forward's x_perm: bf16 layers gather inside the up-projection GEMM
+  const bool fused_gather = c->dtype == MOE_BF16 && MOE_FUSED_GATHER;
+  L.x_perm = take(fused_gather ? 0 : (size_t)L.rows_cap * c->d_model * es);
   L.h = take((size_t)L.rows_total * c->d_ff * es);
   L.y_rows = take((size_t)L.rows_total * c->d_model * 4);      // fp32 rows
   L.total = o;
@@ -114,12 +136,13 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // ---- step bodies, shared by the step entry points and moe_forward ----------
 static cudaError_t run_route(const moe_config *c, const WsLayout &L, char *ws, const void *x,
-                             const void *w_router, const float *bias, float *logits, float *probs,
-                             int32_t *topk_idx, float *topk_gate, cudaStream_t s) {
+                             const void *w_router, const float *bias, const float *state,
+                             float *logits, float *probs, int32_t *topk_idx, float *topk_gate,
+                             cudaStream_t s) {
   int32_t *hist = c->mode == MOE_TOKEN_CHOICE ? reinterpret_cast<int32_t *>(ws + L.hist) : nullptr;
   if (router_is_fused(c))
-    return launch_route_gate(c, nullptr, logits, x, w_router, bias, probs, topk_idx, topk_gate,
-                             hist, s);
+    return launch_route_gate(c, nullptr, logits, x, w_router, bias, state, probs, topk_idx,
+                             topk_gate, hist, s);
   cudaError_t e;
   if (c->dtype == MOE_F32) {
     e = launch_router_f32(c, static_cast<const float *>(x), static_cast<const float *>(w_router),
@@ -154,22 +177,24 @@ static cudaError_t run_route(const moe_config *c, const WsLayout &L, char *ws, c
       g.split_stride = c->T * c->E;
       e = launch_grouped_gemm(g, s);
       if (e != cudaSuccess) return e;
-      return launch_route_gate(c, parts, logits, nullptr, nullptr, bias, probs, topk_idx, topk_gate,
-                               hist, s, ks, c->T * c->E);
+      return launch_route_gate(c, parts, logits, nullptr, nullptr, bias, state, probs, topk_idx,
+                               topk_gate, hist, s, ks, c->T * c->E);
     }
     g.out = logits;
     g.bias = bias;
     e = launch_grouped_gemm(g, s);
   }
   if (e != cudaSuccess) return e;
-  return launch_route_gate(c, logits, nullptr, nullptr, nullptr, nullptr, probs, topk_idx,
+  return launch_route_gate(c, logits, nullptr, nullptr, nullptr, nullptr, state, probs, topk_idx,
                            topk_gate, hist, s);
 }
 
+// row_token non-null (bf16): the up-projection gathers the routed rows of x
+// itself and x_perm is not read
 static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, const void *x,
                            const void *x_perm, const int32_t *offsets, const float *row_gate,
                            const void *w1, const void *w3, const void *w2, void *h, void *y_rows,
-                           cudaStream_t s) {
+                           cudaStream_t s, const int32_t *row_token = nullptr) {
   uint32_t *err = reinterpret_cast<uint32_t *>(ws + L.err);
   if (c->dtype == MOE_F32)
     return launch_ffn_f32(c, L, err, static_cast<const float *>(x),
@@ -182,8 +207,11 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
   up.epi = swiglu ? kEpiSwiglu : kEpiRelu;
   up.K = c->d_model;
   up.N = c->d_ff;
-  up.a = x_perm;
-  up.a_rows = L.rows_cap;
+  up.a = row_token ? x : x_perm;
+  up.a_rows = row_token ? c->T : L.rows_cap;
+  up.gather_rows = row_token;
+  up.gather_src = row_token ? x : nullptr;
+  up.src_rows = c->T;
   up.a_static = x;
   up.a_static_rows = c->T;
   up.b = w1;
@@ -224,6 +252,9 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
   dn.max_routed_rows = L.rows_cap;
   dn.out = y_rows;
   dn.row_gate = row_gate;
+  // the last groups' activations are the ones still in L2 when the
+  // up-projection ends: start the down-projection there
+  dn.reverse = MOE_DOWN_REVERSE;
   dn.sk_part = up.sk_part;
   dn.sk_flags = up.sk_flags;
   dn.err = err;
@@ -249,9 +280,14 @@ moe_status moe_query_sizes(const moe_config *cfg, moe_sizes *out) {
   return MOE_OK;
 }
 
+// the routing state array is required exactly when the rule reads it
+static bool state_ok(const moe_config *c, const float *state) {
+  return c->route_rule == MOE_ROUTE_SOFTMAX || state != nullptr;
+}
+
 moe_status moe_route(const moe_config *cfg, const void *x, const void *w_router, const float *bias,
-                     float *logits, float *probs, int32_t *topk_idx, float *topk_gate, void *ws,
-                     size_t ws_bytes, moe_stream_t stream) {
+                     const float *route_state, float *logits, float *probs, int32_t *topk_idx,
+                     float *topk_gate, void *ws, size_t ws_bytes, moe_stream_t stream) {
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const WsLayout L = make_layout(cfg);
@@ -259,23 +295,37 @@ moe_status moe_route(const moe_config *cfg, const void *x, const void *w_router,
   const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
   if (!x || !w_router || !logits || !probs || (tc && (!topk_idx || !topk_gate)))
     return MOE_ERR_INVALID_ARG;
+  if (!state_ok(cfg, route_state)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(logits) || !aligned16(probs))
     return MOE_ERR_INVALID_ARG;
-  return cuda_status(run_route(cfg, L, static_cast<char *>(ws), x, w_router, bias, logits, probs,
-                               topk_idx, topk_gate, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(run_route(cfg, L, static_cast<char *>(ws), x, w_router, bias, route_state,
+                               logits, probs, topk_idx, topk_gate,
+                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
-moe_status moe_gate(const moe_config *cfg, const float *logits, float *probs, int32_t *topk_idx,
-                    float *topk_gate, void *ws, size_t ws_bytes, moe_stream_t stream) {
+moe_status moe_gate(const moe_config *cfg, const float *logits, const float *route_state,
+                    float *probs, int32_t *topk_idx, float *topk_gate, void *ws, size_t ws_bytes,
+                    moe_stream_t stream) {
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const WsLayout L = make_layout(cfg);
   if ((st = check_ws(L, ws, ws_bytes, L.step_end)) != MOE_OK) return st;
   const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
   if (!logits || !probs || (tc && (!topk_idx || !topk_gate))) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_route_gate(cfg, logits, nullptr, nullptr, nullptr, nullptr, probs,
-                                       topk_idx, topk_gate, nullptr,
+  if (!state_ok(cfg, route_state)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_route_gate(cfg, logits, nullptr, nullptr, nullptr, nullptr, route_state,
+                                       probs, topk_idx, topk_gate, nullptr,
                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_route_bias_update(const moe_config *cfg, const int32_t *counts, float *route_bias,
+                                 float gamma, moe_stream_t stream) {
+  const moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->mode != MOE_TOKEN_CHOICE || !counts || !route_bias) return MOE_ERR_INVALID_ARG;
+  if (!(gamma == gamma)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_bias_update(cfg, counts, route_bias, gamma,
+                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *topk_idx,
@@ -328,15 +378,17 @@ moe_status moe_combine(const moe_config *cfg, const void *y_rows, const int32_t 
 }
 
 static moe_status forward_impl(const moe_config *cfg, const void *x, const void *w_router,
-                               const float *bias, const void *w1, const void *w3, const void *w2,
-                               void *y, int32_t *counts_out, void *ws, size_t ws_bytes,
-                               void *const *events, moe_stream_t stream) {
+                               const float *bias, const float *state, const void *w1,
+                               const void *w3, const void *w2, void *y, int32_t *counts_out,
+                               void *ws, size_t ws_bytes, void *const *events,
+                               moe_stream_t stream) {
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const WsLayout L = make_layout(cfg);
   if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
   const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
   if (!x || !w_router || !w1 || !w2 || !y || (swiglu && !w3)) return MOE_ERR_INVALID_ARG;
+  if (!state_ok(cfg, state)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(w1) || !aligned16(w2) || !aligned16(y) ||
       (swiglu && !aligned16(w3)))
     return MOE_ERR_INVALID_ARG;
@@ -361,15 +413,19 @@ static moe_status forward_impl(const moe_config *cfg, const void *x, const void 
   };
   cudaError_t e = mark(0);
   if (e == cudaSuccess)
-    e = run_route(cfg, L, w, x, w_router, bias, logits, probs, topk_idx, topk_gate, s);
+    e = run_route(cfg, L, w, x, w_router, bias, state, logits, probs, topk_idx, topk_gate, s);
   if (e == cudaSuccess) e = mark(1);
-  // token choice: the gate wrote the unit histogram into the workspace
+  // token choice: the gate wrote the unit histogram into the workspace.
+  // bf16: the up-projection gathers the rows of x itself (no x_perm)
+  const bool fused_gather = cfg->dtype == MOE_BF16 && MOE_FUSED_GATHER;
   if (e == cudaSuccess)
     e = launch_permute(cfg, L, w, cfg->mode == MOE_TOKEN_CHOICE, x, topk_idx, topk_gate, probs,
-                       counts, offsets, tok_rows, row_token, row_gate, x_perm, n_dropped, s);
+                       counts, offsets, tok_rows, row_token, row_gate, x_perm, n_dropped, s,
+                       !fused_gather);
   if (e == cudaSuccess) e = mark(2);
   if (e == cudaSuccess)
-    e = run_ffn(cfg, L, w, x, x_perm, offsets, row_gate, w1, w3, w2, h, y_rows, s);
+    e = run_ffn(cfg, L, w, x, x_perm, offsets, row_gate, w1, w3, w2, h, y_rows, s,
+                fused_gather ? row_token : nullptr);
   if (e == cudaSuccess) e = mark(3);
   if (e == cudaSuccess) e = launch_combine(cfg, L.rows_cap, y_rows, tok_rows, y, s);
   if (e == cudaSuccess) e = mark(4);
@@ -379,18 +435,19 @@ static moe_status forward_impl(const moe_config *cfg, const void *x, const void 
 }
 
 moe_status moe_forward(const moe_config *cfg, const void *x, const void *w_router,
-                       const float *bias, const void *w1, const void *w3, const void *w2, void *y,
-                       int32_t *counts_out, void *ws, size_t ws_bytes, moe_stream_t stream) {
-  return forward_impl(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, ws_bytes, nullptr,
-                      stream);
+                       const float *bias, const float *route_state, const void *w1, const void *w3,
+                       const void *w2, void *y, int32_t *counts_out, void *ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+  return forward_impl(cfg, x, w_router, bias, route_state, w1, w3, w2, y, counts_out, ws, ws_bytes,
+                      nullptr, stream);
 }
 
 moe_status moe_forward_timed(const moe_config *cfg, const void *x, const void *w_router,
-                             const float *bias, const void *w1, const void *w3, const void *w2,
-                             void *y, int32_t *counts_out, void *ws, size_t ws_bytes,
-                             void *const *events, moe_stream_t stream) {
-  return forward_impl(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, ws_bytes, events,
-                      stream);
+                             const float *bias, const float *route_state, const void *w1,
+                             const void *w3, const void *w2, void *y, int32_t *counts_out,
+                             void *ws, size_t ws_bytes, void *const *events, moe_stream_t stream) {
+  return forward_impl(cfg, x, w_router, bias, route_state, w1, w3, w2, y, counts_out, ws, ws_bytes,
+                      events, stream);
 }
 
 moe_status moe_check_device_errors(void *ws, size_t ws_bytes, moe_stream_t stream, uint32_t *flags) {

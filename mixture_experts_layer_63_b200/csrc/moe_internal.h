@@ -35,13 +35,33 @@ inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, 
 
 // Tokens per unit of the token-choice counting sort (one warp per unit).
 constexpr int kUnitTokens = 32;
+constexpr int kUnitsPerBlock = 32;      // units per block of the permutation's scans
+
+// Numbering of the token-choice units.  Tokens form G local groups (GShard's
+// local group dispatch; G = 1 without it) of nbg 32-token blocks each; unit
+// u = g*upg + r*nbg + bl holds the rank-r choices of block bl of group g
+// (upg = k*nbg units per group), so a group's units are contiguous and in its
+// own priority order.  Scan blocks of kUnitsPerBlock units never straddle a
+// group: bpg blocks per group, nb in all.
+struct UnitGrid {
+  int G, nbg, upg, bpg, nb;
+};
+inline UnitGrid unit_grid(const moe_config *c) {
+  UnitGrid u;
+  u.G = c->local_groups > 1 ? c->local_groups : 1;
+  u.nbg = u.G > 1 ? (int)(c->T / u.G / kUnitTokens) : (int)((c->T + kUnitTokens - 1) / kUnitTokens);
+  u.upg = (c->mode == MOE_TOKEN_CHOICE ? c->k : 0) * u.nbg;
+  u.bpg = (u.upg + kUnitsPerBlock - 1) / kUnitsPerBlock;
+  u.nb = u.G * u.bpg;
+  return u;
+}
 // Upper bound on routed experts and on top-k handled by the kernels.
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;
 // The router runs inside the gate kernel when E <= 32 and W_r, widened to
 // fp32, fits this many bytes of shared memory; otherwise the tcgen05 GEMM
 // (bf16) or a CUDA-core kernel (fp32) computes the logits first.
-constexpr size_t kFusedRouterSmem = 160 * 1024;
+constexpr size_t kFusedRouterSmem = 200 * 1024;
 
 // Byte offsets into the caller's workspace.  The first region (error word +
 // step scratch) is what the step entry points use; moe_forward adds its
@@ -87,21 +107,28 @@ bool router_is_fused(const moe_config *c);
 // x and w_router, writing logits_out; else gate on the given logits.
 // logits_in may hold nsplit partial sums split_stride floats apart (summed in
 // order, then + bias when bias is given).
+// state: the per-expert routing bias or utilisation of c->route_rule (or null).
 cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float *logits_out,
-                              const void *x, const void *w_router, const float *bias, float *probs,
-                              int32_t *topk_idx, float *topk_gate, int32_t *hist, cudaStream_t s,
-                              int nsplit = 1, int64_t split_stride = 0);
+                              const void *x, const void *w_router, const float *bias,
+                              const float *state, float *probs, int32_t *topk_idx, float *topk_gate,
+                              int32_t *hist, cudaStream_t s, int nsplit = 1,
+                              int64_t split_stride = 0);
+// DeepSeek-V3 routing-bias update from a step's counts (one block)
+cudaError_t launch_bias_update(const moe_config *c, const int32_t *counts, float *bias, float gamma,
+                               cudaStream_t s);
 // fp32 logits on CUDA cores for fp32 layers the fused router does not cover
 cudaError_t launch_router_f32(const moe_config *c, const float *x, const float *w, const float *bias,
                               float *logits, cudaStream_t s);
 
 // --- permutation (permute.cu) ---------------------------------------------
 // hist_ready: the gate already wrote the unit histogram into the workspace
+// gather = false: x_perm is not written (the up-projection GEMM gathers the
+// rows itself)
 cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, bool hist_ready,
                            const void *x, const int32_t *topk_idx, const float *topk_gate,
                            const float *probs, int32_t *counts, int32_t *offsets, int32_t *tok_rows,
                            int32_t *row_token, float *row_gate, void *x_perm, int32_t *n_dropped,
-                           cudaStream_t s);
+                           cudaStream_t s, bool gather = true);
 
 // --- tcgen05 grouped GEMM (gemm_sm100.cu) ---------------------------------
 enum GemmEpilogue : int {
@@ -141,6 +168,10 @@ struct GroupedGemm {
   int64_t split_stride;     //   write part s of the output at out + s * split_stride
   float *sk_part;           // stream-K partial tiles [kSkSlots][kSkSlotFloats] and their
   int *sk_flags;            //   flags [kSkSlots] (zero between launches); null: no stream-K
+  int reverse;              // 1: tiles in reverse order (last group first)
+  const int32_t *gather_rows;  // non-null: routed A row r is gather_src[gather_rows[r]]
+  const void *gather_src;      //   (the row gather done inside the GEMM; bf16 [src_rows, K])
+  int64_t src_rows;
   uint32_t *err;
 };
 cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s);

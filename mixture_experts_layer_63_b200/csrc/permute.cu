@@ -75,15 +75,18 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
 // itself; this kernel serves moe_permute called on its own.)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) hist_units_kernel(const int32_t *__restrict__ topk_idx,
-                                                         int64_t T, int k, int E, int nunit,
+                                                         int64_t T, int k, int E, int nu, int nbg,
                                                          int32_t *__restrict__ hist, uint32_t *err) {
   const int lane = threadIdx.x & 31;
   pdl_wait();
   pdl_trigger();
   const int64_t u = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (u >= (int64_t)k * nunit) return;                  // whole warp leaves together
-  const int r = (int)(u / nunit);
-  const int64_t b = u - (int64_t)r * nunit;
+  if (u >= nu) return;                                   // whole warp leaves together
+  // unit u = g*k*nbg + r*nbg + bl (local groups; one group: g = 0)
+  const int64_t g = u / ((int64_t)k * nbg);
+  const int64_t rem = u - g * k * nbg;
+  const int r = (int)(rem / nbg);
+  const int64_t b = g * nbg + (rem - (int64_t)r * nbg);
   const int64_t t = b * kUnitTokens + lane;
   int e = -1;
   if (t < T) {
@@ -109,17 +112,23 @@ __global__ void __launch_bounds__(256) hist_units_kernel(const int32_t *__restri
 // ceil(n_e*num/den)) and the exclusive scans over experts from the totals;
 // block 0 writes them out.
 // ---------------------------------------------------------------------------
-constexpr int kUnitsPerBlock = 32;
 
-__global__ void __launch_bounds__(1024) unit_sums_kernel(const int32_t *__restrict__ hist, int nu,
-                                                         int E, int32_t *__restrict__ bsum) {
+// units of scan block b: kUnitsPerBlock consecutive units of one local group
+__device__ __forceinline__ void block_units(int b, int upg, int bpg, int &u_begin, int &u_end) {
+  const int g = b / bpg;
+  u_begin = g * upg + (b - g * bpg) * kUnitsPerBlock;
+  u_end = min(u_begin + kUnitsPerBlock, (g + 1) * upg);
+}
+
+__global__ void __launch_bounds__(1024) unit_sums_kernel(const int32_t *__restrict__ hist, int upg,
+                                                         int bpg, int E, int32_t *__restrict__ bsum) {
   __shared__ int s_part[1024];
   pdl_wait();
   pdl_trigger();
   const int G = max(1, (int)blockDim.x / E);
   const int g = threadIdx.x / E, e = threadIdx.x - g * E;
-  const int u_begin = blockIdx.x * kUnitsPerBlock;
-  const int u_end = min(nu, u_begin + kUnitsPerBlock);
+  int u_begin, u_end;
+  block_units(blockIdx.x, upg, bpg, u_begin, u_end);
   int part = 0;
   if (g < G)
     for (int u = u_begin + g; u < u_end; u += G) part += hist[(int64_t)u * E + e];
@@ -141,8 +150,9 @@ __global__ void __launch_bounds__(1024) unit_sums_kernel(const int32_t *__restri
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024, 1) rank_units_kernel(
     const int32_t *__restrict__ topk_idx, const float *__restrict__ topk_gate, int64_t T, int k,
-    int E, int nunit, int nb, const int32_t *__restrict__ hist, const int32_t *__restrict__ bsum,
-    int capacity, int keep_num, int keep_den, int keep_fraction, int32_t *__restrict__ counts,
+    int E, int nbg, int upg, int bpg, int nb, const int32_t *__restrict__ hist,
+    const int32_t *__restrict__ bsum, int capacity, int keep_num, int keep_den, int keep_fraction,
+    int32_t *__restrict__ counts,
     int32_t *__restrict__ cnt_off_out, int32_t *__restrict__ kept_out,
     int32_t *__restrict__ offsets_out, int32_t *__restrict__ n_dropped,
     int32_t *__restrict__ tok_rows, int32_t *__restrict__ row_token, float *__restrict__ row_gate,
@@ -157,30 +167,56 @@ __global__ void __launch_bounds__(1024, 1) rank_units_kernel(
   int *s_coff = s_off + E + 1;                        // [E+1] count offsets
   int *s_part = s_coff + E + 1;                       // [1024] partial sums
   int *s_part2 = s_part + 1024;                       // [1024]
+  int *s_kept = s_part2 + 1024;                       // [E] rows kept (local groups)
+  int *s_kbefore = s_kept + E;                        // [E] rows kept by earlier groups
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nu = k * nunit;
   const int b = blockIdx.x;
-  const int u_begin = b * kUnitsPerBlock;
-  const int u_end = min(nu, u_begin + kUnitsPerBlock);
+  int u_begin, u_end;
+  block_units(b, upg, bpg, u_begin, u_end);
+  const int lgroups = nb / bpg;                       // local groups
+  const int my_group = b / bpg;
 
-  // 1. totals of the blocks before this one, and of all blocks
+  // 1. totals of the blocks before this one (in its group), and of all blocks
   const int G = max(1, (int)blockDim.x / E);
   const int g = threadIdx.x / E, e_g = threadIdx.x - g * E;
-  int pre = 0, tot = 0;
-  if (g < G) {
-    for (int bb = g; bb < nb; bb += G) {
-      const int v = bsum[(int64_t)bb * E + e_g];
-      tot += v;
-      if (bb < b) pre += v;
+  if (lgroups == 1) {
+    int pre = 0, tot = 0;
+    if (g < G) {
+      for (int bb = g; bb < nb; bb += G) {
+        const int v = bsum[(int64_t)bb * E + e_g];
+        tot += v;
+        if (bb < b) pre += v;
+      }
+      s_part[threadIdx.x] = pre;
+      s_part2[threadIdx.x] = tot;
     }
-    s_part[threadIdx.x] = pre;
-    s_part2[threadIdx.x] = tot;
+  } else {
+    // local groups: per expert, one thread walks every group's blocks
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int pre = 0, tot = 0, kept = 0, kbefore = 0;
+      for (int gg = 0; gg < lgroups; ++gg) {
+        int n = 0;
+        for (int bb = gg * bpg; bb < (gg + 1) * bpg; ++bb) {
+          const int v = bsum[(int64_t)bb * E + e];
+          n += v;
+          if (gg == my_group && bb < b) pre += v;
+        }
+        const int kg = capacity > 0 ? min(n, capacity) : n;
+        tot += n;
+        kept += kg;
+        if (gg < my_group) kbefore += kg;
+      }
+      s_pre[e] = pre;
+      s_tot[e] = tot;
+      s_kept[e] = kept;
+      s_kbefore[e] = kbefore;
+    }
   }
   // this block's unit histograms into shared memory
   for (int i = threadIdx.x; i < (u_end - u_begin) * E; i += blockDim.x)
     s_base[i] = hist[(int64_t)u_begin * E + i];
   __syncthreads();
-  if (g == 0) {
+  if (lgroups == 1 && g == 0) {
     int p = 0, t = 0;
     for (int gg = 0; gg < G; ++gg) {
       p += s_part[gg * E + e_g];
@@ -188,6 +224,7 @@ __global__ void __launch_bounds__(1024, 1) rank_units_kernel(
     }
     s_pre[e_g] = p;
     s_tot[e_g] = t;
+    s_kbefore[e_g] = 0;
   }
   __syncthreads();
   // 2. per-expert exclusive scan over this block's units (in place)
@@ -206,7 +243,8 @@ __global__ void __launch_bounds__(1024, 1) rank_units_kernel(
       const int e = e0 + lane;
       const int ce = e < E ? s_tot[e] : 0;
       int ke = ce;
-      if (capacity > 0) ke = min(ce, capacity);
+      if (lgroups > 1) ke = e < E ? s_kept[e] : 0;
+      else if (capacity > 0) ke = min(ce, capacity);
       else if (keep_den > 0) ke = (int)(((int64_t)ce * keep_num + keep_den - 1) / keep_den);
       int xa = ce, xc = ke;
 #pragma unroll
@@ -243,11 +281,12 @@ __global__ void __launch_bounds__(1024, 1) rank_units_kernel(
   }
   __syncthreads();
 
-  // 4. one warp per unit
+  // 4. one warp per unit (u = g*upg + r*nbg + bl)
   const int u = u_begin + warp;
   if (u >= u_end) return;
-  const int r = u / nunit;
-  const int64_t bu = u - (int64_t)r * nunit;
+  const int rem = u - my_group * upg;
+  const int r = rem / nbg;
+  const int64_t bu = (int64_t)my_group * nbg + (rem - r * nbg);
   const int64_t t = bu * kUnitTokens + lane;
   int e = -1;
   if (t < T) {
@@ -261,7 +300,7 @@ __global__ void __launch_bounds__(1024, 1) rank_units_kernel(
     return;
   }
   const bool keep = e >= 0 && (capacity <= 0 || rank < capacity);
-  const int slot = keep ? s_off[e] + rank : -1;
+  const int slot = keep ? s_off[e] + s_kbefore[e] + rank : -1;
   if (e >= 0) tok_rows[t * k + r] = slot;
   if (keep) {
     row_token[slot] = (int32_t)t;
@@ -466,7 +505,7 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
                            const void *x, const int32_t *topk_idx, const float *topk_gate,
                            const float *probs, int32_t *counts, int32_t *offsets, int32_t *tok_rows,
                            int32_t *row_token, float *row_gate, void *x_perm, int32_t *n_dropped,
-                           cudaStream_t s) {
+                           cudaStream_t s, bool gather) {
   uint32_t *err = reinterpret_cast<uint32_t *>(ws + L.err);
   const int E = c->E;
   const int64_t T = c->T;
@@ -488,24 +527,26 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
   int32_t *kept = reinterpret_cast<int32_t *>(ws + L.kept);
   int32_t *sorted_q = reinterpret_cast<int32_t *>(ws + L.sorted_q);
   const int keepfrac = (c->capacity <= 0 && c->keep_den > 0) ? 1 : 0;
-  const int nu = c->k * L.nunit;
-  const int nb = (nu + kUnitsPerBlock - 1) / kUnitsPerBlock;
+  const UnitGrid ug = unit_grid(c);
+  const int nu = ug.G * ug.upg;
+  const int nb = ug.nb;
   cudaError_t e = cudaSuccess;
   if (!hist_ready) {
     e = launch_kernel(hist_units_kernel, (unsigned)((nu + 7) / 8), 256, 0, s, topk_idx, T, c->k, E,
-                      L.nunit, hist, err);
+                      nu, ug.nbg, hist, err);
     if (e != cudaSuccess) return e;
   }
-  e = launch_kernel(unit_sums_kernel, nb, 1024, 0, s, hist, nu, E, bsum);
+  e = launch_kernel(unit_sums_kernel, nb, 1024, 0, s, hist, ug.upg, ug.bpg, E, bsum);
   if (e != cudaSuccess) return e;
-  const size_t rank_smem = ((size_t)kUnitsPerBlock * E + 4 * E + 2 + 2048) * sizeof(int);
+  const size_t rank_smem = ((size_t)kUnitsPerBlock * E + 6 * E + 2 + 2048) * sizeof(int);
   if (rank_smem > 48 * 1024) {
     e = cudaFuncSetAttribute(rank_units_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)rank_smem);
     if (e != cudaSuccess) return e;
   }
   e = launch_kernel(rank_units_kernel, nb, 1024, rank_smem, s, topk_idx, topk_gate, T, c->k, E,
-                    L.nunit, nb, hist, bsum, c->capacity, c->keep_num, c->keep_den, keepfrac, counts,
+                    ug.nbg, ug.upg, ug.bpg, nb, hist, bsum, c->capacity, c->keep_num, c->keep_den,
+                    keepfrac, counts,
                     cnt_off, kept, offsets, n_dropped, tok_rows, row_token, row_gate, sorted_q);
   if (e != cudaSuccess) return e;
   if (keepfrac) {
@@ -514,6 +555,7 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
     if (e != cudaSuccess) return e;
   }
   }
+  if (!gather) return cudaSuccess;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -42,8 +42,12 @@ struct GateParams {
   int32_t *hist;              // [k][nunit][E] or null
   int nsplit;                 // logits_in holds nsplit partial sums ...
   int64_t split_stride;       // ... split_stride floats apart
+  const float *state;         // [E] routing bias (rule 1) or utilisation (rule 2)
+  int rule;                   // moe_route_rule
+  float alpha;                // load-aware coefficient
   int64_t T;
   int d, E, k, n_groups, topk_groups, renormalize, nunit;
+  int nbg;                    // 32-token blocks per local group (unit numbering)
 };
 
 __device__ __forceinline__ void argmax_warp(float &v, int &i) {
@@ -76,31 +80,28 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_gate_kernel(const GatePa
   pdl_trigger();
   int *s_hist = reinterpret_cast<int *>(smem);                    // [k][E]
   const int hist_ints = P.hist ? k * E : 0;
-  // fused router: W_r staged as fp32 in 16-byte groups laid out so that the
-  // 32 lanes of a warp read 32 consecutive groups (no bank conflicts):
-  // element i of expert e -> group ((e * EPV/4 + (i % EPV) / 4) * nchunk + i / EPV)
+  // fused router: W_r widened to fp32 [E][d] and the partial logits of the
+  // 32 slices of the model dimension [32 slices][32 tokens][E + 1 (pad)]
   constexpr int EPV = BF16 ? 8 : 4;                      // x elements per 16-byte chunk
-  constexpr int GPC = EPV / 4;                           // fp32 groups per chunk
-  float4 *s_w = reinterpret_cast<float4 *>(smem + ((hist_ints * 4 + 15) & ~15));
   const int nchunk = P.d / EPV;
+  const int pstride = E + 1;                             // odd: conflict-free rows
+  float *s_w = reinterpret_cast<float *>(smem + ((hist_ints * 4 + 15) & ~15));
+  float *s_part = s_w + (FUSED ? (size_t)E * P.d : 0);
   // per-warp buffer of the exponentials, summed in order by lane 0
-  float *s_ex = reinterpret_cast<float *>(smem + ((hist_ints * 4 + 15) & ~15) +
-                                          (FUSED ? (size_t)E * P.d * 4 : 0)) + warp * E;
+  float *s_ex = s_part + (FUSED ? (size_t)32 * kTokWarps * pstride : 0) + warp * E;
 
   for (int i = threadIdx.x; i < hist_ints; i += blockDim.x) s_hist[i] = 0;
   if (FUSED) {
-    const int ngroups = E * P.d / 4;
-    for (int gi = threadIdx.x; gi < ngroups; gi += blockDim.x) {
-      const int e = gi / (P.d / 4), i0 = (gi - e * (P.d / 4)) * 4;   // 4 consecutive elements
+    const int nq = E * P.d / 4;                          // 4 consecutive elements at a time
+    for (int q = threadIdx.x; q < nq; q += blockDim.x) {
       float4 f;
       if (BF16) {
-        const uint2 w = reinterpret_cast<const uint2 *>(P.w_router)[gi];
+        const uint2 w = reinterpret_cast<const uint2 *>(P.w_router)[q];
         f = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
       } else {
-        f = reinterpret_cast<const float4 *>(P.w_router)[gi];
+        f = reinterpret_cast<const float4 *>(P.w_router)[q];
       }
-      const int c = i0 / EPV, h = (i0 % EPV) / 4;
-      s_w[(e * GPC + h) * nchunk + c] = f;
+      reinterpret_cast<float4 *>(s_w)[q] = f;
     }
   }
   __syncthreads();
@@ -111,47 +112,61 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_gate_kernel(const GatePa
   // ---- logits of this token: lane l holds experts l + 32 j ----------------
   float l[NV];
   if (FUSED) {
-    float acc[EMAX];
+    // slice `warp` of the model dimension for token t0 + lane: x chunks from
+    // global memory into registers, W_r chunks read by all lanes at once
+    // (shared-memory broadcast); per expert an fp32 chain in element order
+    // (experts in passes of up to 16, to stay within 64 registers a thread)
+    constexpr int EB = EMAX < 16 ? EMAX : 16;
+    for (int e0 = 0; e0 < E; e0 += EB) {
+      const int64_t tt = (int64_t)blockIdx.x * kTokWarps + lane;
+      const int c0 = warp * nchunk / 32, c1 = (warp + 1) * nchunk / 32;
+      float acc[EB];
 #pragma unroll
-    for (int e = 0; e < EMAX; ++e) acc[e] = 0.f;
-    if (live) {
-      const uint4 *xr = reinterpret_cast<const uint4 *>(P.x) + t * nchunk;
-      for (int c = lane; c < nchunk; c += 32) {
-        const uint4 xv = xr[c];
-        float xf[EPV];
-        if (BF16) {
-          xf[0] = bf16_lo(xv.x); xf[1] = bf16_hi(xv.x); xf[2 % EPV] = bf16_lo(xv.y); xf[3 % EPV] = bf16_hi(xv.y);
-          xf[4 % EPV] = bf16_lo(xv.z); xf[5 % EPV] = bf16_hi(xv.z); xf[6 % EPV] = bf16_lo(xv.w); xf[7 % EPV] = bf16_hi(xv.w);
-        } else {
-          xf[0] = __uint_as_float(xv.x); xf[1] = __uint_as_float(xv.y);
-          xf[2 % EPV] = __uint_as_float(xv.z); xf[3 % EPV] = __uint_as_float(xv.w);
-        }
+      for (int e = 0; e < EB; ++e) acc[e] = 0.f;
+      if (tt < P.T) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(P.x) + tt * nchunk;
+        for (int c = c0; c < c1; ++c) {
+          const uint4 xv = xr[c];
+          float xf[EPV];
+          if (BF16) {
+            xf[0] = bf16_lo(xv.x); xf[1] = bf16_hi(xv.x); xf[2 % EPV] = bf16_lo(xv.y); xf[3 % EPV] = bf16_hi(xv.y);
+            xf[4 % EPV] = bf16_lo(xv.z); xf[5 % EPV] = bf16_hi(xv.z); xf[6 % EPV] = bf16_lo(xv.w); xf[7 % EPV] = bf16_hi(xv.w);
+          } else {
+            xf[0] = __uint_as_float(xv.x); xf[1] = __uint_as_float(xv.y);
+            xf[2 % EPV] = __uint_as_float(xv.z); xf[3 % EPV] = __uint_as_float(xv.w);
+          }
+          const float4 *wc = reinterpret_cast<const float4 *>(s_w + (size_t)e0 * P.d + (size_t)c * EPV);
 #pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-          if (e < E) {
-            float a = acc[e];
+          for (int e = 0; e < EB; ++e) {
+            if (e0 + e < E) {
+              float a = acc[e];
 #pragma unroll
-            for (int h = 0; h < GPC; ++h) {
-              const float4 w = s_w[(e * GPC + h) * nchunk + c];
-              a = fmaf(xf[4 * h + 0], w.x, a);
-              a = fmaf(xf[4 * h + 1], w.y, a);
-              a = fmaf(xf[4 * h + 2], w.z, a);
-              a = fmaf(xf[4 * h + 3], w.w, a);
+              for (int h = 0; h < EPV / 4; ++h) {
+                const float4 w = wc[(size_t)e * (P.d / 4) + h];
+                a = fmaf(xf[4 * h + 0], w.x, a);
+                a = fmaf(xf[4 * h + 1], w.y, a);
+                a = fmaf(xf[4 * h + 2], w.z, a);
+                a = fmaf(xf[4 * h + 3], w.w, a);
+              }
+              acc[e] = a;
             }
-            acc[e] = a;
           }
         }
       }
+      float *pp = s_part + ((size_t)warp * kTokWarps + lane) * pstride + e0;
+#pragma unroll
+      for (int e = 0; e < EB; ++e)
+        if (e0 + e < E) pp[e] = acc[e];
     }
+    __syncthreads();
+    // token t = this warp's token: the 32 slices summed in order, then the bias
     float mine = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < EMAX; ++e) {
-      if (e < E) {
-        float v = acc[e];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == e) mine = P.bias ? __fadd_rn(v, P.bias[e]) : v;
-      }
+    if (lane < E) {
+      const float *pp = s_part + (size_t)warp * pstride + lane;
+      float v = pp[0];
+#pragma unroll 8
+      for (int sl = 1; sl < 32; ++sl) v = __fadd_rn(v, pp[(size_t)sl * kTokWarps * pstride]);
+      mine = P.bias ? __fadd_rn(v, P.bias[lane]) : v;
     }
     l[0] = mine;
     if (live && lane < E) P.logits_out[t * E + lane] = mine;
@@ -200,6 +215,27 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_gate_kernel(const GatePa
   }
   if (P.topk_idx == nullptr) return;          // expert choice: probabilities only
 
+  // ---- selection keys and gate values of the routing rule -----------------
+  //   softmax: key = logit, gate = p
+  //   bias   : key = p + b_e (one fp32 add), gate = key   (DeepSeek-V3)
+  //   load   : key = logit + alpha * (1 - u_e), gate = p   (load-aware top-k)
+  float key[NV], gsrc[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = l[j];
+    gsrc[j] = p[j];
+    if (P.rule != 0 && e < E) {
+      const float st = P.state[e];
+      if (P.rule == 1) {
+        key[j] = __fadd_rn(p[j], st);
+        gsrc[j] = key[j];
+      } else {
+        key[j] = __fadd_rn(l[j], __fmul_rn(P.alpha, __fsub_rn(1.0f, st)));
+      }
+    }
+  }
+
   // ---- group limit: groups of E/n_groups experts, keep the best topk_groups
   uint32_t allowed = 0xffffffffu;
   int grp[NV];                             // group of each slot (0 without a group limit)
@@ -213,7 +249,7 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_gate_kernel(const GatePa
 #pragma unroll
       for (int j = 0; j < NV; ++j) {
         const int e = lane + 32 * j;
-        if (e < E && grp[j] == g) gm = fmaxf(gm, l[j]);
+        if (e < E && grp[j] == g) gm = fmaxf(gm, key[j]);
       }
       gm = max_warp(gm);
       if (lane == g) my_score = gm;
@@ -245,17 +281,17 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_gate_kernel(const GatePa
       for (int j = 0; j < NV; ++j) {
         const int e = lane + 32 * j;
         const bool ok = e < E && !((taken >> j) & 1u) && ((allowed >> grp[j]) & 1u);
-        if (ok && (l[j] > bv || (l[j] == bv && e < bi))) {
-          bv = l[j];
+        if (ok && (key[j] > bv || (key[j] == bv && e < bi))) {
+          bv = key[j];
           bi = e;
         }
       }
       argmax_warp(bv, bi);
-      // probability of the chosen expert, from the lane that holds it
+      // gate of the chosen expert, from the lane that holds it
       float pv = 0.f;
 #pragma unroll
       for (int j = 0; j < NV; ++j)
-        if (j == bi / 32) pv = p[j];
+        if (j == bi / 32) pv = gsrc[j];
       pv = __shfl_sync(0xffffffffu, pv, bi & 31);
       if (lane == (bi & 31)) taken |= 1u << (bi / 32);
       idxs[r] = bi;
@@ -279,7 +315,10 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_gate_kernel(const GatePa
     __syncthreads();
     for (int i = threadIdx.x; i < hist_ints; i += blockDim.x) {
       const int r = i / E, e = i - r * E;
-      P.hist[((int64_t)r * P.nunit + blockIdx.x) * E + e] = s_hist[i];
+      // unit of (rank r, this block): group-major numbering, see unit_grid
+      const int g = blockIdx.x / P.nbg, bl = blockIdx.x - g * P.nbg;
+      const int64_t u = ((int64_t)g * P.k + r) * P.nbg + bl;
+      P.hist[u * E + e] = s_hist[i];
     }
   }
 }
@@ -315,18 +354,31 @@ cudaError_t launch_nv(int NV, const GateParams &P, int blocks, size_t smem, cuda
 #define MOE_FUSED_ROUTER_BF16 0
 #endif
 
-// fp32 layers: the gate kernel computes the logits (CUDA cores).  bf16 layers
-// use the tcgen05 router GEMM.
+// shared memory of the fused router: W_r widened to fp32 and the partial
+// logits of 32 slices x 32 tokens
+static size_t fused_router_smem(const moe_config *c) {
+  return (size_t)c->E * c->d_model * 4 + (size_t)32 * kTokWarps * (c->E + 1) * 4;
+}
+
+// fp32 layers with few experts (E <= 32) and a W_r that fits shared memory:
+// the gate kernel computes the logits itself on CUDA cores, reading x once.
+// Otherwise the tcgen05 router GEMM (bf16) or a CUDA-core kernel (fp32) runs
+// first.  (For bf16 the fused form measured slower than the router GEMM plus
+// the gate: 21 vs 18 us on the GShard-shaped layer, 78 vs 44 us on the
+// Mixtral-shaped one; MOE_FUSED_ROUTER_BF16=1 builds it.)
 bool router_is_fused(const moe_config *c) {
   if (c->dtype == MOE_BF16 && !MOE_FUSED_ROUTER_BF16) return false;
-  return c->E <= 32 && (size_t)c->E * c->d_model * 4 <= kFusedRouterSmem;
+  return c->E <= 32 && fused_router_smem(c) <= kFusedRouterSmem;
 }
 
 cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float *logits_out,
-                              const void *x, const void *w_router, const float *bias, float *probs,
-                              int32_t *topk_idx, float *topk_gate, int32_t *hist, cudaStream_t s,
-                              int nsplit, int64_t split_stride) {
+                              const void *x, const void *w_router, const float *bias,
+                              const float *state, float *probs, int32_t *topk_idx, float *topk_gate,
+                              int32_t *hist, cudaStream_t s, int nsplit, int64_t split_stride) {
   GateParams P{};
+  P.rule = c->mode == MOE_TOKEN_CHOICE ? c->route_rule : MOE_ROUTE_SOFTMAX;
+  P.state = state;
+  P.alpha = c->route_alpha;
   P.nsplit = nsplit < 1 ? 1 : nsplit;
   P.split_stride = split_stride;
   const bool tc = c->mode == MOE_TOKEN_CHOICE;
@@ -348,13 +400,14 @@ cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float
   P.topk_groups = c->topk_groups;
   P.renormalize = c->renormalize;
   P.nunit = (int)((c->T + kUnitTokens - 1) / kUnitTokens);
+  P.nbg = unit_grid(c).nbg;
   const int blocks = P.nunit;
   size_t smem = P.hist ? (size_t)P.k * P.E * 4 : 0;
   smem = (smem + 15) & ~(size_t)15;
   smem += (size_t)kTokWarps * c->E * 4;                     // per-warp exponentials
   const int NV = (c->E + 31) / 32;
   if (fused) {
-    smem += (size_t)c->E * c->d_model * 4;                  // W_r staged as fp32
+    smem += fused_router_smem(c);                           // W_r (fp32) + slice partials
     const bool bf = c->dtype == MOE_BF16;
     auto kern = c->E <= 8    ? (bf ? route_gate_kernel<1, true, true, 8> : route_gate_kernel<1, true, false, 8>)
                 : c->E <= 16 ? (bf ? route_gate_kernel<1, true, true, 16> : route_gate_kernel<1, true, false, 16>)
@@ -403,6 +456,27 @@ cudaError_t launch_router_f32(const moe_config *c, const float *x, const float *
   const int64_t blocks = (c->T + warps - 1) / warps;
   return launch_kernel(router_f32_kernel, (unsigned)blocks, warps * 32, 0, s, x, w, bias, logits,
                        c->T, c->d_model, c->E);
+}
+
+namespace {
+// DeepSeek-V3 bias update: b_e -= gamma when c_e * E > T * k, += gamma when
+// c_e * E < T * k (exact integer load test), unchanged at the mean.
+__global__ void bias_update_kernel(const int32_t *__restrict__ counts, float *__restrict__ bias,
+                                   int E, int64_t Tk, float gamma) {
+  pdl_wait();
+  pdl_trigger();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int64_t load = (int64_t)counts[e] * E;
+    if (load > Tk) bias[e] = __fsub_rn(bias[e], gamma);
+    else if (load < Tk) bias[e] = __fadd_rn(bias[e], gamma);
+  }
+}
+}  // namespace
+
+cudaError_t launch_bias_update(const moe_config *c, const int32_t *counts, float *bias, float gamma,
+                               cudaStream_t s) {
+  return launch_kernel(bias_update_kernel, 1, 256, 0, s, counts, bias, c->E, c->T * (int64_t)c->k,
+                       gamma);
 }
 
 }  // namespace moe

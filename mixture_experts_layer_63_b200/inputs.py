@@ -58,6 +58,9 @@ class Workload:
     renormalize: bool = False         # gates divided by the sum of the selected p
     router_std: float | None = None   # None: d_model ** -0.5
     zipf_s: float = 0.0               # > 0: Zipf logit bias over experts
+    route_rule: str = "softmax"       # selection keys: "softmax" | "bias" | "load"
+    route_alpha: float = 0.0          # load-aware coefficient
+    local_groups: int = 1             # GShard local groups (capacity per group)
 
     def with_tokens(self, T: int) -> "Workload":
         """Same layer on T tokens; expert choice keeps C = T * k / E."""
@@ -81,6 +84,16 @@ WORKLOADS: dict[str, Workload] = {
     "deepseek_v2": Workload("deepseek_v2", T=8192, d_model=5120, E=160, S=2, k=6,
                             d_ff=1536, act="swiglu", dtype="bf16", n_groups=8,
                             topk_groups=3, keep_num=9, keep_den=10),
+    # DeepSeek-V3's routing on the pages: 256 routed + 1 shared experts, top-8,
+    # at most 4 of 8 nodes (groups) per token, auxiliary-loss-free bias routing.
+    # The pages give no V3 hidden sizes: DeepSeek-V2's (5120 / 1536) stand in.
+    "deepseek_v3": Workload("deepseek_v3", T=8192, d_model=5120, E=256, S=1, k=8,
+                            d_ff=1536, act="swiglu", dtype="bf16", n_groups=8,
+                            topk_groups=4, route_rule="bias"),
+    # GShard with local group dispatching: 4 groups of 1024 tokens
+    "gshard_local": Workload("gshard_local", T=4096, d_model=1024, E=16, S=0, k=2, d_ff=4096,
+                             act="relu", dtype="bf16", capacity_factor=1.25, router_std=0.02,
+                             local_groups=4),
 }
 
 
@@ -94,6 +107,7 @@ class LayerInputs:
     w1: torch.Tensor                # [E+S, f, d]
     w3: torch.Tensor | None         # [E+S, f, d] (SwiGLU) or None
     w2: torch.Tensor                # [E+S, d, f]
+    route_state: torch.Tensor | None = None   # [E] fp32: routing bias or utilisation
 
 
 def torch_dtype(w: Workload) -> torch.dtype:
@@ -132,8 +146,9 @@ def make_inputs(w: Workload, seed: int = 0, device: str | torch.device = "cpu",
         b64 = torch.tensor([-w.zipf_s * math.log(e + 1.0) for e in range(E)], dtype=torch.float64)
         bias = b64.to(torch.float32).to(dev)
 
+    state = route_state(w, seed, dev, grid)
     if not with_weights:
-        return LayerInputs(x, w_router, bias, None, None, None)
+        return LayerInputs(x, w_router, bias, None, None, None, state)
 
     G = E + S
     w1 = torch.empty(G, f, d, device=dev, dtype=dt)
@@ -145,7 +160,31 @@ def make_inputs(w: Workload, seed: int = 0, device: str | torch.device = "cpu",
         if w3 is not None:
             w3[e] = (torch.randn(f, d, generator=g, device=dev, dtype=torch.float32) * s_in).to(dt)
         w2[e] = (torch.randn(d, f, generator=g, device=dev, dtype=torch.float32) * s_hid).to(dt)
-    return LayerInputs(x, w_router, bias, w1, w3, w2)
+    return LayerInputs(x, w_router, bias, w1, w3, w2, state)
+
+
+def route_state(w: Workload, seed: int, device, grid: bool = False) -> torch.Tensor | None:
+    """The per-expert routing state of the workload's rule, from a generator
+    of its own (seed + 7919), so the other draws do not move.
+
+    bias: b_e ~ N(0, (0.5 / E)^2), the scale of a softmax probability's
+          spread over E experts, as a bias that has been trained for a while
+          would be; grid: rounded to multiples of 2^-16.
+    load: u_e ~ U(0, 1), a utilisation; grid: multiples of 1/16.
+    """
+    if w.route_rule == "softmax":
+        return None
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed + 7919)
+    if w.route_rule == "bias":
+        st = torch.randn(w.E, generator=g, dtype=torch.float64) * (0.5 / w.E)
+        if grid:
+            st = torch.round(st * 65536.0) / 65536.0
+    else:
+        st = torch.rand(w.E, generator=g, dtype=torch.float64)
+        if grid:
+            st = torch.round(st * 16.0) / 16.0
+    return st.to(torch.float32).to(device)
 
 
 def router_sum_bound(inp: LayerInputs) -> float:

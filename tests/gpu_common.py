@@ -40,16 +40,25 @@ SMALL = {
     # (256-row tiles); ragged M tails, partial N tiles, shared experts
     "pair_relu_s": replace(WORKLOADS["gshard"], T=2100, E=4, d_model=256, d_ff=320),
     "pair_swiglu_s": replace(WORKLOADS["deepseekmoe_tc"], T=1400, E=8, k=6, d_model=320, d_ff=192),
+    # routing variants: DeepSeek-V3 bias routing (256 + 1 experts, top-8 of 4
+    # groups), load-aware top-k, GShard local groups
+    "dsv3_s": replace(WORKLOADS["deepseek_v3"], T=600, d_model=256, d_ff=128),
+    "load_aware_s": replace(WORKLOADS["gshard"], T=700, d_model=256, d_ff=320, route_rule="load",
+                            route_alpha=0.75, capacity_factor=0.0),
+    "local_groups_s": replace(WORKLOADS["gshard_local"], T=768, d_model=256, d_ff=320),
 }
 
 
 def oracle_config(w: Workload) -> O.OracleConfig:
     cap = O.capacity_from_factor(w.T, w.E, w.k, w.capacity_factor) if w.mode == "tc" else 0
+    if w.mode == "tc" and w.local_groups > 1:        # capacity of one expert in one group
+        cap = O.capacity_from_factor(w.T // w.local_groups, w.E, w.k, w.capacity_factor)
     return O.OracleConfig(E=w.E, S=w.S, k=w.k, act=w.act, mode=w.mode, capacity=cap,
                           keep_num=w.keep_num, keep_den=w.keep_den,
                           ec_capacity=w.ec_capacity if w.mode == "ec" else 0,
                           n_groups=w.n_groups, topk_groups=w.topk_groups,
-                          renormalize=w.renormalize)
+                          renormalize=w.renormalize, rule=w.route_rule,
+                          alpha=float(np.float32(w.route_alpha)), local_groups=w.local_groups)
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
@@ -95,3 +104,13 @@ def assert_close_rms(y: np.ndarray, ref: np.ndarray, dtype: str, what: str = "y"
 
 def gpu_inputs(w: Workload, seed: int = 0, grid: bool = True):
     return make_inputs(w, seed=seed, device="cuda", grid=grid)
+
+
+def state_dev(inp):
+    """The routing state of the inputs on the GPU (or None)."""
+    return None if inp.route_state is None else inp.route_state.cuda()
+
+
+def state_np(inp):
+    """The routing state of the inputs as a host fp32 array (or None)."""
+    return None if inp.route_state is None else inp.route_state.detach().cpu().numpy()

@@ -34,8 +34,34 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_struct_sizes(L):
-    assert ctypes.sizeof(api.MoeConfig) == 72
+    assert ctypes.sizeof(api.MoeConfig) == 88
     assert ctypes.sizeof(api.MoeSizes) == 40
+
+
+def test_struct_layout_matches_the_header(tmp_path):
+    """Every field offset of the ctypes structs equals the C compiler's
+    offsetof on include/moe.h (gcc, host only)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not found")
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "moe.h"', 'int main(void) {']
+    for st, cname in ((api.MoeConfig, "moe_config"), (api.MoeSizes, "moe_sizes")):
+        lines.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
+        for f, _ in st._fields_:
+            lines.append(f'printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
+    lines.append("return 0; }")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run(["gcc", "-I", inc, str(src), "-o", str(exe)], check=True)
+    got = dict(l.split() for l in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                  check=True).stdout.splitlines())
+    for st, cname in ((api.MoeConfig, "moe_config"), (api.MoeSizes, "moe_sizes")):
+        assert int(got[cname]) == ctypes.sizeof(st)
+        for f, _ in st._fields_:
+            assert int(got[f"{cname}.{f}"]) == getattr(st, f).offset, f
 
 
 def test_status_strings(L):
@@ -75,6 +101,11 @@ def _cfg(**kw):
     ("S", 9, api.MOE_ERR_UNSUPPORTED),
     ("n_groups", 3, api.MOE_ERR_INVALID_ARG),       # 16 experts do not split into 3 groups
     ("keep_den", 10, api.MOE_ERR_INVALID_ARG),      # capacity and keep-fraction together
+    ("route_rule", 5, api.MOE_ERR_INVALID_ARG),
+    ("reserved", 1, api.MOE_ERR_INVALID_ARG),
+    ("local_groups", 3, api.MOE_ERR_INVALID_ARG),   # 4096 tokens do not split into 3 groups
+    ("local_groups", 256, api.MOE_ERR_UNSUPPORTED), # groups of 16 tokens: below one 32-token unit
+    ("local_groups", -1, api.MOE_ERR_INVALID_ARG),
 ])
 def test_invalid_configs_rejected(L, field, value, status):
     c = _cfg(**{field: value})
@@ -98,6 +129,18 @@ def test_expert_choice_options(L):
     c.ec_capacity = w.T + 1
     with pytest.raises(api.MoeError):
         api.query_sizes(c)
+    c = api.config_from_workload(w)
+    c.route_rule = api.MOE_ROUTE_LOAD                # routing rules are token-choice options
+    with pytest.raises(api.MoeError):
+        api.query_sizes(c)
+
+
+def test_local_groups_need_a_capacity(L):
+    c = _cfg(local_groups=4)
+    api.query_sizes(c)
+    c = _cfg(local_groups=4, capacity=0)
+    with pytest.raises(api.MoeError):
+        api.query_sizes(c)
 
 
 def test_null_pointers_rejected_before_any_launch(L):
@@ -105,15 +148,26 @@ def test_null_pointers_rejected_before_any_launch(L):
     c = _cfg()
     s = api.query_sizes(c)
     f = L.moe_route
-    st = f(ctypes.byref(c), None, None, None, None, None, None, None, None, 0, None)
+    st = f(ctypes.byref(c), None, None, None, None, None, None, None, None, None, 0, None)
     assert st == api.MOE_ERR_INVALID_ARG
     # workspace too small
     buf = ctypes.create_string_buffer(4096 + 256)
     addr = (ctypes.addressof(buf) + 255) & ~255
-    st = L.moe_forward(ctypes.byref(c), 16, 16, None, 16, None, 16, 16, None, addr, 1024, None)
+    st = L.moe_forward(ctypes.byref(c), 16, 16, None, None, 16, None, 16, 16, None, addr, 1024, None)
     assert st == api.MOE_ERR_WORKSPACE
     # misaligned workspace
-    st = L.moe_forward(ctypes.byref(c), 16, 16, None, 16, None, 16, 16, None, addr + 8, s.workspace, None)
+    st = L.moe_forward(ctypes.byref(c), 16, 16, None, None, 16, None, 16, 16, None, addr + 8,
+                       s.workspace, None)
+    assert st == api.MOE_ERR_INVALID_ARG
+    # a routing rule that reads route_state, without one
+    c2 = _cfg(T=64, d_model=64, d_ff=64, capacity=8)
+    c2.route_rule = api.MOE_ROUTE_BIAS
+    ws = ctypes.create_string_buffer(api.query_sizes(c2).workspace + 256)
+    wa = (ctypes.addressof(ws) + 255) & ~255
+    st = L.moe_forward(ctypes.byref(c2), 16, 16, None, None, 16, None, 16, 16, None, wa,
+                       api.query_sizes(c2).workspace, None)
+    assert st == api.MOE_ERR_INVALID_ARG
+    st = L.moe_route_bias_update(ctypes.byref(c2), None, None, 0.001, None)
     assert st == api.MOE_ERR_INVALID_ARG
     st = L.moe_combine(ctypes.byref(c), None, None, None, None)
     assert st == api.MOE_ERR_INVALID_ARG

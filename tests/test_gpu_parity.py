@@ -21,7 +21,7 @@ from mixture_experts_layer_63_b200 import api
 from mixture_experts_layer_63_b200.inputs import WORKLOADS, make_inputs
 from oracle import moe_oracle as O
 from tests.gpu_common import (SMALL, TOL, LazyExperts, assert_close_rms, gpu_inputs,
-                              oracle_config, to_f64, to_np)
+                              oracle_config, state_dev, state_np, to_f64, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -40,7 +40,8 @@ def _bias_np(inp):
 
 def _route_gpu(cfg, inp):
     B = api.step_buffers(cfg)
-    api.moe_route(cfg, inp.x, inp.w_router, inp.bias, B.logits, B.probs, B.topk_idx, B.topk_gate, B.ws)
+    api.moe_route(cfg, inp.x, inp.w_router, inp.bias, B.logits, B.probs, B.topk_idx, B.topk_gate, B.ws,
+                  route_state=inp.route_state)
     return B
 
 
@@ -48,12 +49,16 @@ def _route_gpu(cfg, inp):
 # steps 1-3a
 # ---------------------------------------------------------------------------
 
-# extra routing cases: the fused CUDA-core router (E <= 32, one and two passes
-# over the experts) and the tcgen05 router GEMM with its K split over CTAs
+# extra routing cases: the fused CUDA-core router (fp32, E <= 32, one and two
+# passes over the experts) and the tcgen05 router GEMM, K whole or split
 ROUTE_EXTRA = {
-    # E <= 32: the logits come from the gate kernel's own CUDA-core router
-    "fused_router_s": replace(WORKLOADS["gshard"], T=300),
-    "fused_router_e32_s": replace(WORKLOADS["gshard"], T=200, E=32, d_model=512),
+    # fp32, E <= 32: the logits come from the gate kernel's own CUDA-core
+    # router (two passes over the experts for E = 32)
+    "fused_router_f32_s": replace(WORKLOADS["tiny_f32"], T=300, d_model=512),
+    "fused_router_e32_f32_s": replace(WORKLOADS["tiny_f32"], T=200, E=32, d_model=256),
+    # bf16: tcgen05 router GEMM, one K part and 16 / 32 experts
+    "router_gemm_s": replace(WORKLOADS["gshard"], T=300),
+    "router_gemm_e32_s": replace(WORKLOADS["gshard"], T=200, E=32, d_model=512),
     # E > 32: the tcgen05 router GEMM with K split over CTAs
     "split_k_s": replace(WORKLOADS["deepseekmoe_tc"], T=300),
     "split_k_groups_s": replace(WORKLOADS["deepseek_v2"], T=200, d_model=1024, keep_num=0, keep_den=0),
@@ -71,7 +76,7 @@ def test_route_bit_exact(name):
     torch.cuda.synchronize()
     ref_l = O.router_logits(to_np(inp.x), to_np(inp.w_router), _bias_np(inp))
     assert np.array_equal(to_np(B.logits), ref_l)
-    probs, idx, gate, _ = O.route(oracle_config(w), ref_l)
+    probs, idx, gate, _ = O.route(oracle_config(w), ref_l, state_np(inp))
     assert np.array_equal(to_np(B.probs), probs)
     if w.mode == "tc":
         assert np.array_equal(to_np(B.topk_idx), idx)
@@ -85,10 +90,11 @@ def test_gate_bit_exact_from_oracle_logits(name):
     w = WORKLOADS[name]
     inp = make_inputs(w, seed=2, device="cpu", grid=False, with_weights=False)
     ref_l = O.router_logits(to_np(inp.x), to_np(inp.w_router), _bias_np(inp))
-    probs, idx, gate, _ = O.route(oracle_config(w), ref_l)
+    probs, idx, gate, _ = O.route(oracle_config(w), ref_l, state_np(inp))
     cfg = api.config_from_workload(w)
     B = api.step_buffers(cfg)
-    api.moe_gate(cfg, torch.from_numpy(ref_l).cuda(), B.probs, B.topk_idx, B.topk_gate, B.ws)
+    api.moe_gate(cfg, torch.from_numpy(ref_l).cuda(), B.probs, B.topk_idx, B.topk_gate, B.ws,
+                 route_state=state_dev(inp))
     torch.cuda.synchronize()
     assert np.array_equal(to_np(B.probs), probs)
     if w.mode == "tc":
@@ -105,7 +111,7 @@ def _permute_check(w, seed=3, bias_override=None):
     bias = _bias_np(inp) if bias_override is None else bias_override
     ref_l = O.router_logits(to_np(inp.x), to_np(inp.w_router), bias)
     oc = oracle_config(w)
-    probs, idx, gate, disp = O.route(oc, ref_l)
+    probs, idx, gate, disp = O.route(oc, ref_l, state_np(inp))
     cfg = api.config_from_workload(w)
     B = api.step_buffers(cfg)
     xg = inp.x.cuda()
@@ -190,7 +196,7 @@ def test_expert_ffn_rows(name):
     oc = oracle_config(w)
     x_np = to_np(inp.x)
     ref_l = O.router_logits(x_np, to_np(inp.w_router), _bias_np(inp))
-    probs, idx, gate, disp = O.route(oc, ref_l)
+    probs, idx, gate, disp = O.route(oc, ref_l, state_np(inp))
     cfg = api.config_from_workload(w)
     s = api.query_sizes(cfg)
     B = api.step_buffers(cfg)
@@ -222,7 +228,7 @@ def test_combine_sums_rows_in_order(name):
     inp = make_inputs(w, seed=5, device="cpu", grid=False, with_weights=False)
     oc = oracle_config(w)
     ref_l = O.router_logits(to_np(inp.x), to_np(inp.w_router), _bias_np(inp))
-    _, _, _, disp = O.route(oc, ref_l)
+    _, _, _, disp = O.route(oc, ref_l, state_np(inp))
     cfg = api.config_from_workload(w)
     s = api.query_sizes(cfg)
     dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
@@ -259,12 +265,13 @@ def _forward_check(w, seed=6, tokens=None, inp=None):
     ws = api.new_workspace(cfg)
     y = torch.empty_like(inp.x)
     counts = torch.empty(w.E, dtype=torch.int32, device="cuda")
-    api.moe_forward(cfg, inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, y, counts, ws)
+    api.moe_forward(cfg, inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, y, counts, ws,
+                    route_state=inp.route_state)
     api.moe_check_device_errors(ws)
     oc = oracle_config(w)
     x_np = to_np(inp.x)
     ref_l = O.router_logits(x_np, to_np(inp.w_router), _bias_np(inp))
-    probs, idx, gate, disp = O.route(oc, ref_l)
+    probs, idx, gate, disp = O.route(oc, ref_l, state_np(inp))
     assert np.array_equal(to_np(counts), disp.counts)
     toks = np.arange(w.T) if tokens is None else np.asarray(tokens)
     lazy = (LazyExperts(inp.w1), LazyExperts(inp.w2), LazyExperts(inp.w3))
