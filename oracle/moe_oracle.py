@@ -556,3 +556,188 @@ def forward(cfg: OracleConfig, x, w_router, bias, w1, w3, w2, tokens=None,
     tokens = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
     y = combine_tokens(cfg, x, w1, w2, w3, disp, tokens)
     return OracleResult(logits, probs, idx, gate, disp, tokens, y)
+
+
+# --------------------------------------------------------------------------
+# backward (training): gradients of L = sum(dy * y) with the routing held fixed
+# --------------------------------------------------------------------------
+# The pages train these layers (GShard, DeepSeekMoE, DeepSeek-V2/V3 on "MoE技术演进";
+# the gating network p = softmax(g) of "Adaptive Mixtures of Local Experts"):
+# gradients reach the experts through every kept row, and the router through
+# the gate of each kept row (G = p, p / sum of the selected p when
+# renormalised, s + b for DeepSeek-V3's bias routing, whose bias is a fixed
+# input).  The selection itself (top-k, capacity drops, keep-fraction,
+# expert choice, local groups) is piecewise constant in the logits and is held
+# fixed, as training frameworks do.  Everything below is float64 with the
+# softmax in exact mathematics (the fixed fp32 recipe only serves the integer
+# decisions).
+
+
+@dataclass
+class Grads:
+    dx: np.ndarray               # [T, d]
+    dw_router: np.ndarray        # [E, d]
+    dbias: np.ndarray | None     # [E] when a logit bias is given
+    dw1: np.ndarray              # [E+S, f, d]
+    dw3: np.ndarray | None       # [E+S, f, d] (SwiGLU)
+    dw2: np.ndarray              # [E+S, d, f]
+
+
+def softmax_f64(logits: np.ndarray) -> np.ndarray:
+    """p = exp(l - max l) / sum exp(l - max l) in float64."""
+    l = np.asarray(logits, dtype=np.float64)
+    e = np.exp(l - l.max(axis=1, keepdims=True))
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def softmax_backward(p: np.ndarray, dp: np.ndarray) -> np.ndarray:
+    """dL/dl from dL/dp through p = softmax(l): p * (dp - sum_j p_j dp_j)."""
+    return p * (dp - np.sum(p * dp, axis=1, keepdims=True))
+
+
+def _ffn_parts(xr, w1_e, w2_e, w3_e, act):
+    """Forward of one expert on rows xr (float64), keeping what its backward needs."""
+    a = xr @ widen(w1_e).T
+    if act == "relu":
+        h = np.maximum(a, 0.0)
+        u = None
+    else:
+        u = xr @ widen(w3_e).T
+        h = a / (1.0 + np.exp(-a)) * u
+    return a, u, h, h @ widen(w2_e).T
+
+
+def _ffn_backward(xr, a, u, h, dyr, w1_e, w2_e, w3_e, act):
+    """Backward of FFN_e for rows with output gradients dyr: returns
+    (dx rows, dW1, dW3, dW2).  ReLU: dA = dH [A > 0].  SwiGLU: with
+    s = sigmoid(A), H = A s U: dA = dH U s (1 + A (1 - s)), dU = dH A s."""
+    w2 = widen(w2_e)
+    dw2 = dyr.T @ h
+    dh = dyr @ w2
+    if act == "relu":
+        da = dh * (a > 0)
+        dw1 = da.T @ xr
+        return da @ widen(w1_e), dw1, None, dw2
+    s = 1.0 / (1.0 + np.exp(-a))
+    da = dh * u * s * (1.0 + a * (1.0 - s))
+    du = dh * a * s
+    dw1 = da.T @ xr
+    dw3 = du.T @ xr
+    return da @ widen(w1_e) + du @ widen(w3_e), dw1, dw3, dw2
+
+
+def _gates_f64(cfg: OracleConfig, logits, disp: Dispatch, idx, state):
+    """Gate of every kept row as a float64 function of the logits (the
+    selection fixed), and what its backward needs."""
+    p = softmax_f64(logits)
+    T, E = p.shape
+    if cfg.mode == "ec":
+        rows_e = np.searchsorted(disp.offsets, np.arange(len(disp.row_token)), side="right") - 1
+        return p, p[disp.row_token, rows_e], None
+    k = idx.shape[1]
+    src = p[np.arange(T)[:, None], idx]                  # gate source of the k selected
+    if cfg.rule == "bias":
+        src = src + np.asarray(state, np.float64)[idx]
+    if cfg.renormalize:
+        ssum = src.sum(axis=1, keepdims=True)
+        g_sel = src / ssum
+    else:
+        ssum = None
+        g_sel = src
+    # gate of each kept row: row of (t, j) is tok_rows[t, j]
+    row_gate = np.zeros(len(disp.row_token))
+    r = disp.tok_rows
+    kept = r >= 0
+    row_gate[r[kept]] = g_sel[kept]
+    return p, row_gate, (src, ssum, g_sel)
+
+
+def backward(cfg: OracleConfig, x, w_router, bias, w1, w3, w2, dy, state=None,
+             disp: Dispatch | None = None) -> Grads:
+    """Gradients of L = sum(dy * y) for the layer's forward, routing fixed.
+
+    ``disp`` is the forward's routing (recomputed here when not given).
+    """
+    xs = widen(x)
+    T, d = xs.shape
+    dy = np.asarray(dy, dtype=np.float64)
+    logits32 = router_logits(x, w_router, bias)
+    probs, idx, gate, disp0 = route(cfg, logits32, state)
+    disp = disp0 if disp is None else disp
+    logits = widen(x) @ widen(w_router).T + (0.0 if bias is None else widen(bias)[None, :])
+    p, row_gate, gparts = _gates_f64(cfg, logits, disp, idx, state)
+    E = cfg.E
+    G = cfg.E + cfg.S
+    f = np.asarray(w1[0]).shape[0]
+    dx = np.zeros((T, d))
+    dw1 = np.zeros((G, f, d))
+    dw3 = np.zeros((G, f, d)) if cfg.act == "swiglu" else None
+    dw2 = np.zeros((G, d, f))
+    dgate = np.zeros(len(disp.row_token))               # dL / d(gate of each kept row)
+    for e in range(G):
+        if e < E:
+            a0, a1 = int(disp.offsets[e]), int(disp.offsets[e + 1])
+            if a1 == a0:
+                continue
+            toks = disp.row_token[a0:a1].astype(np.int64)
+            g = row_gate[a0:a1]
+        else:
+            toks = np.arange(T)
+            g = np.ones(T)
+        xr = xs[toks]
+        a, u, h, yo = _ffn_parts(xr, w1[e], w2[e], None if w3 is None else w3[e], cfg.act)
+        dyr = dy[toks] * g[:, None]
+        dxr, gw1, gw3, gw2 = _ffn_backward(xr, a, u, h, dyr, w1[e], w2[e],
+                                           None if w3 is None else w3[e], cfg.act)
+        np.add.at(dx, toks, dxr)
+        dw1[e] += gw1
+        dw2[e] += gw2
+        if dw3 is not None:
+            dw3[e] += gw3
+        if e < E:
+            dgate[a0:a1] = np.sum(dy[toks] * yo, axis=1)
+    # gates -> probabilities
+    dp = np.zeros((T, E))
+    if cfg.mode == "ec":
+        rows_e = np.searchsorted(disp.offsets, np.arange(len(disp.row_token)), side="right") - 1
+        np.add.at(dp, (disp.row_token.astype(np.int64), rows_e), dgate)
+    else:
+        src, ssum, g_sel = gparts
+        k = idx.shape[1]
+        dg_sel = np.zeros((T, k))
+        r = disp.tok_rows
+        kept = r >= 0
+        dg_sel[kept] = dgate[r[kept]]
+        if cfg.renormalize:
+            dsrc = (dg_sel - np.sum(dg_sel * g_sel, axis=1, keepdims=True)) / ssum
+        else:
+            dsrc = dg_sel
+        np.add.at(dp, (np.repeat(np.arange(T), k), idx.reshape(-1)), dsrc.reshape(-1))
+    # softmax backward, then the router
+    dl = softmax_backward(p, dp)
+    dx += dl @ widen(w_router)
+    return Grads(dx, dl.T @ xs, None if bias is None else dl.sum(axis=0), dw1, dw3, dw2)
+
+
+def forward_fixed_selection(cfg: OracleConfig, x, w_router, bias, w1, w3, w2, disp: Dispatch,
+                            idx, state=None) -> np.ndarray:
+    """y [T, d] in float64 for a given selection, gates from the exact
+    softmax of the logits (what ``backward`` differentiates)."""
+    xs = widen(x)
+    T, d = xs.shape
+    logits = xs @ widen(w_router).T + (0.0 if bias is None else widen(bias)[None, :])
+    _, row_gate, _ = _gates_f64(cfg, logits, disp, idx, state)
+    y = np.zeros((T, d))
+    for e in range(cfg.E + cfg.S):
+        if e < cfg.E:
+            a0, a1 = int(disp.offsets[e]), int(disp.offsets[e + 1])
+            toks = disp.row_token[a0:a1].astype(np.int64)
+            g = row_gate[a0:a1]
+        else:
+            toks = np.arange(T)
+            g = np.ones(T)
+        if len(toks) == 0:
+            continue
+        _, _, _, yo = _ffn_parts(xs[toks], w1[e], w2[e], None if w3 is None else w3[e], cfg.act)
+        np.add.at(y, toks, yo * g[:, None])
+    return y

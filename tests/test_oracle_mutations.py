@@ -13,6 +13,7 @@ from tests import test_oracle_ffn as TF
 from tests import test_oracle_gating as TG
 from tests import test_oracle_selection as TS
 from tests import test_oracle_routing_variants as TV
+from tests import test_oracle_backward as TB
 
 
 def _expect_pin_failure(pin, *args):
@@ -186,3 +187,27 @@ def test_global_ranks_under_local_groups_are_caught(monkeypatch):
 
     monkeypatch.setattr(O, "_priority_ranks", wrong)
     _expect_pin_failure(TV.test_local_groups_are_independent_batches, 4)
+
+
+def test_backward_silu_derivative_is_caught(monkeypatch):
+    """SiLU'(a) taken as sigmoid(a) (the a * s * (1 - s) term dropped)."""
+    def wrong(xr, a, u, h, dyr, w1_e, w2_e, w3_e, act):
+        w2 = O.widen(w2_e)
+        dw2 = dyr.T @ h
+        dh = dyr @ w2
+        if act == "relu":
+            da = dh * (a > 0)
+            return da @ O.widen(w1_e), da.T @ xr, None, dw2
+        s = 1.0 / (1.0 + np.exp(-a))
+        da = dh * u * s
+        du = dh * a * s
+        return da @ O.widen(w1_e) + du @ O.widen(w3_e), da.T @ xr, du.T @ xr, dw2
+
+    monkeypatch.setattr(O, "_ffn_backward", wrong)
+    _expect_pin_failure(TB.test_backward_matches_finite_differences, "renorm_swiglu_shared")
+
+
+def test_backward_without_softmax_jacobian_is_caught(monkeypatch):
+    """dlogits = dp (the softmax Jacobian left out)."""
+    monkeypatch.setattr(O, "softmax_backward", lambda p, dp: dp)
+    _expect_pin_failure(TB.test_backward_matches_finite_differences, "capacity_relu")
