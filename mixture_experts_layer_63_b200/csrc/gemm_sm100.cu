@@ -705,7 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool gather = P.gather_rows != nullptr;
   if (tid == 32) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_bar[s], 1 + (gather ? kGatherThreads : 0));
+      mbar_init(&full_bar[s], 1 + (gather ? kGatherThreads / 32 : 0));   // + one per gather warp
       mbar_init(&empty_bar[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -868,14 +868,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (routed) gr.load(P, s_off[tl.g], s_rows[tl.g], tl.m * BM, gt);
       else gr.clear();
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+        // lane 0 waits for the stage to be free, the warp follows it
+        int okw = 1;
+        if (lane == 0) okw = mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err) ? 1 : 0;
+        __syncwarp();
+        if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
         if (routed) gr.issue(smem_u32(smem + (size_t)stage * stage_bytes), gt, kb, xs, row_bytes);
         cp_async_commit();
         ++issued;
         if (issued - arrived > kLag) {
           cp_async_wait<kLag>();
           fence_proxy_async_smem();
-          mbar_arrive(&full_bar[arrived % kStages]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full_bar[arrived % kStages]);   // one arrival per warp
           ++arrived;
         }
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -883,7 +888,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     cp_async_wait<0>();
     fence_proxy_async_smem();
-    for (; arrived < issued; ++arrived) mbar_arrive(&full_bar[arrived % kStages]);
+    __syncwarp();
+    for (; arrived < issued; ++arrived)
+      if (lane == 0) mbar_arrive(&full_bar[arrived % kStages]);
   } else if (warp >= 4) {
     // -------------------------------- epilogue --------------------------------
     const int ew = warp - 4;                     // TMEM lanes 32*ew .. 32*ew+31
@@ -972,8 +979,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const bool gather = P.gather_rows != nullptr;
   if (tid == 32) {
     for (int st = 0; st < kPairStages; ++st) {
-      // the even CTA's: its expect_tx arrival, then both CTAs' gather threads
-      mbar_init(&full_bar[st], 1 + (gather ? 2 * kGatherThreads : 0));
+      // the even CTA's: its expect_tx arrival, then both CTAs' gather warps
+      mbar_init(&full_bar[st], 1 + (gather ? 2 * kGatherThreads / 32 : 0));
       mbar_init(&empty_bar[st], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -1138,14 +1145,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (routed) gr.load(P, s_off[tl.g], s_rows[tl.g], tl.m * PM + (int)rank * BM, gt);
       else gr.clear();
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+        // lane 0 waits for the stage to be free, the warp follows it
+        int okw = 1;
+        if (lane == 0) okw = mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err) ? 1 : 0;
+        __syncwarp();
+        if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
         if (routed) gr.issue(smem_u32(smem + (size_t)stage * stage_bytes), gt, kb, xs, row_bytes);
         cp_async_commit();
         ++issued;
         if (issued - arrived > kLag) {
           cp_async_wait<kLag>();
           fence_proxy_async_smem();
-          arrive_full((int)(arrived % kPairStages));
+          __syncwarp();
+          if (lane == 0) arrive_full((int)(arrived % kPairStages));   // one arrival per warp
           ++arrived;
         }
         if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
@@ -1153,7 +1165,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     cp_async_wait<0>();
     fence_proxy_async_smem();
-    for (; arrived < issued; ++arrived) arrive_full((int)(arrived % kPairStages));
+    __syncwarp();
+    for (; arrived < issued; ++arrived)
+      if (lane == 0) arrive_full((int)(arrived % kPairStages));
   } else if (warp >= 4) {
     // -------------------------------- epilogue --------------------------------
     const int ew = warp - 4;
