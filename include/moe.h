@@ -258,6 +258,32 @@ MOE_API moe_status moe_forward_timed(const moe_config *cfg, const void *x, const
                                      void *ws, size_t ws_bytes, void *const *events,
                                      moe_stream_t stream);
 
+/* Backward pass (training) of the forward that last ran on `ws`: gradients
+ * of L = sum(dy * y) ("MoE技术演进": GShard, DeepSeekMoE and DeepSeek-V2/V3
+ * are trained this way; the gate is the softmax gating network of "Adaptive
+ * Mixtures of Local Experts").  The routing decisions of that forward (top-k,
+ * capacity drops, keep-fraction, expert choice, local groups) are held fixed;
+ * gradient reaches the experts through every kept row and the router through
+ * the gate of each kept row (G = p, p / sum of the selected p when
+ * renormalised, p + b under MOE_ROUTE_BIAS).  bf16 layers only
+ * (MOE_ERR_UNSUPPORTED for fp32).
+ *   in : the forward's x, w_router, bias, route_state, w1, w3, w2 and its
+ *        workspace ws (unchanged since moe_forward); dy [T, d] bf16.
+ *   out: dx [T, d], dw_router [E, d], dbias [E] (NULL when bias is NULL),
+ *        dw1 [E+S, f, d], dw3 [E+S, f, d] (SwiGLU; NULL for ReLU),
+ *        dw2 [E+S, d, f]: fp32, overwritten.
+ *   bws: scratch of at least moe_query_backward_size bytes (256-byte aligned).
+ *   Arithmetic: bf16 tensor-core contractions with fp32 accumulation; the
+ *   recomputed pre-activations, dA / dU and the transposed operands are
+ *   rounded to bf16; gate and router gradients in fp32. */
+MOE_API moe_status moe_query_backward_size(const moe_config *cfg, size_t *bytes);
+MOE_API moe_status moe_backward(const moe_config *cfg, const void *x, const void *w_router,
+                                const float *bias, const float *route_state, const void *w1,
+                                const void *w3, const void *w2, const void *dy, float *dx,
+                                float *dw_router, float *dbias, float *dw1, float *dw3, float *dw2,
+                                const void *ws, size_t ws_bytes, void *bws, size_t bws_bytes,
+                                moe_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the workspace's device error
  * word.  Returns MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_CHECK; *flags (if
  * not NULL) receives the raw bits.  After an error it also clears the rest

@@ -31,7 +31,7 @@ ROUTE_RULES = {"softmax": MOE_ROUTE_SOFTMAX, "bias": MOE_ROUTE_BIAS, "load": MOE
 EXPORTS = ("moe_query_sizes", "moe_route", "moe_gate", "moe_permute", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_check_device_errors", "moe_workspace_init",
            "moe_status_string", "moe_permute_noalloc", "moe_forward_timed",
-           "moe_route_bias_update")
+           "moe_route_bias_update", "moe_query_backward_size", "moe_backward")
 
 
 class MoeError(RuntimeError):
@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             "moe_route": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_gate": [cfgp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_route_bias_update": [cfgp, vp, vp, ctypes.c_float, vp],
+            "moe_query_backward_size": [cfgp, ctypes.POINTER(ctypes.c_size_t)],
+            "moe_backward": [cfgp] + [vp] * 14 + [vp, sz, vp, sz, vp],
             "moe_permute": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_expert_ffn": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_combine": [cfgp, vp, vp, vp, vp],
@@ -245,6 +247,23 @@ def moe_forward_timed(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, eve
         _ptr(w2), _ptr(y), _ptr(counts_out), wp, wn, handles, _stream(stream)))
 
 
+def query_backward_size(cfg: MoeConfig) -> int:
+    out = ctypes.c_size_t(0)
+    _check("moe_query_backward_size", lib().moe_query_backward_size(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
+
+
+def moe_backward(cfg, x, w_router, bias, w1, w3, w2, dy, dx, dw_router, dbias, dw1, dw3, dw2, ws, bws,
+                 stream=None, *, route_state=None):
+    """Gradients of sum(dy * y) for the forward that last ran on ws (routing fixed)."""
+    wp, wn = _ws(ws)
+    bp, bn = _ws(bws)
+    _check("moe_backward", lib().moe_backward(
+        ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(route_state), _ptr(w1), _ptr(w3),
+        _ptr(w2), _ptr(dy), _ptr(dx), _ptr(dw_router), _ptr(dbias), _ptr(dw1), _ptr(dw3), _ptr(dw2),
+        wp, wn, bp, bn, _stream(stream)))
+
+
 def moe_check_device_errors(ws, stream=None) -> int:
     """Blocks on the stream; returns the raw error bits and raises if any is set."""
     wp, wn = _ws(ws)
@@ -324,6 +343,24 @@ class MoELayer:
         moe_forward(self.cfg, x, self.w_router, self.bias, self.w1, self.w3, self.w2, y,
                     self.counts, self.ws, stream, route_state=self.route_state)
         return y
+
+    def backward(self, x: torch.Tensor, dy: torch.Tensor, stream=None) -> dict:
+        """Gradients of sum(dy * y) for the last ``self(x)`` (same x), routing
+        fixed: dx, dw_router, dbias (when the layer has a logit bias), dw1,
+        dw3 (SwiGLU), dw2, all fp32."""
+        if getattr(self, "bws", None) is None:
+            self.bws = torch.empty(max(query_backward_size(self.cfg), 256), dtype=torch.uint8,
+                                   device=x.device)
+        f32 = dict(dtype=torch.float32, device=x.device)
+        g = {"dx": torch.empty(x.shape, **f32), "dw_router": torch.empty(self.w_router.shape, **f32),
+             "dbias": torch.empty(self.bias.shape, **f32) if self.bias is not None else None,
+             "dw1": torch.empty(self.w1.shape, **f32),
+             "dw3": torch.empty(self.w3.shape, **f32) if self.w3 is not None else None,
+             "dw2": torch.empty(self.w2.shape, **f32)}
+        moe_backward(self.cfg, x, self.w_router, self.bias, self.w1, self.w3, self.w2, dy, g["dx"],
+                     g["dw_router"], g["dbias"], g["dw1"], g["dw3"], g["dw2"], self.ws, self.bws,
+                     stream, route_state=self.route_state)
+        return g
 
     def update_route_bias(self, gamma: float, stream=None):
         """DeepSeek-V3's bias step from the last forward's counts."""

@@ -95,8 +95,21 @@ struct Params {
   const int32_t *gather_rows;  // routed A row r = gather_src[gather_rows[r]] (null: A as stored)
   const void *gather_src;      //   bf16 [src_rows, K]
   int64_t src_rows;
+  const void *aux;          // kEpiDAct*: bf16 pre-activations [row][aux_ld]
+  int64_t aux_ld;
+  int kgroup;               // K-grouped mode (weight gradients), see GroupedGemm
+  int M;
+  const int32_t *kseg;
+  int split_m;
+  void *out2;
   uint32_t *err;
 };
+
+// B tiles of 128 gate rows (map_b) + 128 up rows (map_b3): SwiGLU and its
+// pre-activation recompute
+__host__ __device__ constexpr bool swiglu_b(int epi) {
+  return epi == kEpiSwiglu || epi == kEpiPreSwiglu;
+}
 
 // ------------------------------- PTX wrappers --------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -586,6 +599,18 @@ __device__ __forceinline__ void store_bf16x32(void *dst, const float (&v)[32]) {
   }
 }
 
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16 *src, float (&v)[32]) {
+  const uint4 *p = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 w = p[q];
+    v[8 * q + 0] = bf16_lo(w.x); v[8 * q + 1] = bf16_hi(w.x);
+    v[8 * q + 2] = bf16_lo(w.y); v[8 * q + 3] = bf16_hi(w.y);
+    v[8 * q + 4] = bf16_lo(w.z); v[8 * q + 5] = bf16_hi(w.z);
+    v[8 * q + 6] = bf16_lo(w.w); v[8 * q + 7] = bf16_hi(w.w);
+  }
+}
+
 // Epilogue of one accumulator: this thread's row (TMEM lane) of the tile,
 // BN columns from TMEM address `taddr`; the later stream-K pieces of the tile
 // added first when F is given; then activation / gate / bias, stores.
@@ -655,6 +680,79 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
                                v[4 * q + 3] * scale);
       }
     }
+  } else if (EPI == kEpiPreRelu) {
+    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
+#pragma unroll 1
+    for (int c = 0; c < P.bn / 32; ++c) {
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      if (F) add_parts(v, *F, c * 32);
+      const int col = col0 + c * 32;
+      if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
+    }
+  } else if (EPI == kEpiPreSwiglu) {
+    // a (gate half) at [row][col], u (up half) at [row][N + col]
+    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
+    const int64_t ld = 2 * (int64_t)P.N;
+#pragma unroll 1
+    for (int c = 0; c < 128 / 32; ++c) {
+      uint32_t u[32];
+      float uf[32];
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld32(taddr + 128 + c * 32, u);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        v[i] = __uint_as_float(r[i]);
+        uf[i] = __uint_as_float(u[i]);
+      }
+      if (F) {
+        add_parts(v, *F, c * 32);
+        add_parts(uf, *F, 128 + c * 32);
+      }
+      const int col = col0 + c * 32;
+      if (valid && col < P.N) {
+        store_bf16x32(out + out_row * ld + col, v);
+        store_bf16x32(out + out_row * ld + P.N + col, uf);
+      }
+    }
+  } else if (EPI == kEpiDActRelu || EPI == kEpiDActSwiglu) {
+    // dh = g * acc, then the activation's backward from the saved a (and u)
+    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
+    const __nv_bfloat16 *aux = reinterpret_cast<const __nv_bfloat16 *>(P.aux);
+    const int64_t ld = (EPI == kEpiDActSwiglu ? 2 : 1) * (int64_t)P.N;
+    const float scale = (routed && valid) ? P.row_gate[out_row] : 1.0f;
+#pragma unroll 1
+    for (int c = 0; c < P.bn / 32; ++c) {
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      if (F) add_parts(v, *F, c * 32);
+      const int col = col0 + c * 32;
+      if (!valid || col >= P.N) continue;
+      float a[32];
+      load_bf16x32(aux + out_row * P.aux_ld + col, a);
+      if (EPI == kEpiDActRelu) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = a[i] > 0.0f ? v[i] * scale : 0.0f;
+        store_bf16x32(out + out_row * ld + col, v);
+      } else {
+        float uu[32], du[32];
+        load_bf16x32(aux + out_row * P.aux_ld + P.N + col, uu);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float dh = v[i] * scale;
+          const float sg = 1.0f / (1.0f + __expf(-a[i]));
+          du[i] = dh * a[i] * sg;
+          v[i] = dh * uu[i] * sg * (1.0f + a[i] * (1.0f - sg));
+        }
+        store_bf16x32(out + out_row * ld + col, v);
+        store_bf16x32(out + out_row * ld + P.N + col, du);
+      }
+    }
   } else {  // kEpiStoreF32 (a K part when the router is split: no bias, own output)
     float *out = reinterpret_cast<float *>(P.out) + out_offset;
     const float *bias = P.ksplit > 1 ? nullptr : P.bias;
@@ -662,16 +760,51 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
     for (int c = 0; c < P.bn / 32; ++c) {
       tmem_ld32(taddr + c * 32, r);
       tmem_ld_wait();
-      if (valid) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      if (F) add_parts(v, *F, c * 32);
+      const int col0c = col0 + c * 32;
+      if (!valid) continue;
+      if (!bias && col0c + 32 <= P.N && (P.N & 3) == 0) {
+        float4 *dst = reinterpret_cast<float4 *>(out + out_row * P.N + col0c);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int col = col0 + c * 32 + i;
-          if (col < P.N) {
-            const float a = __uint_as_float(r[i]);
-            out[out_row * P.N + col] = bias ? a + bias[col] : a;
-          }
+          const int col = col0c + i;
+          if (col < P.N) out[out_row * P.N + col] = bias ? v[i] + bias[col] : v[i];
         }
       }
+    }
+  }
+}
+
+// K-grouped mode: this thread's row of a weight-gradient tile (fp32), or
+// zeros when the group has no K columns (zero is the same for the whole
+// CTA, so the warp's TMEM loads stay aligned); dst null: row past M
+__device__ __forceinline__ void epilogue_wgrad(const Params &P, uint32_t taddr, bool zero, float *dst,
+                                               int col0) {
+  uint32_t r[32];
+#pragma unroll 1
+  for (int c = 0; c < P.bn / 32; ++c) {
+    const int col = col0 + c * 32;
+    if (!zero) {
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+    }
+    if (!dst || col >= P.N) continue;
+    if (col + 32 <= P.N && (P.N & 3) == 0) {
+      float4 *d4 = reinterpret_cast<float4 *>(dst + col);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        d4[q] = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
+                     : make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                   __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (col + i < P.N) dst[col + i] = zero ? 0.0f : __uint_as_float(r[i]);
     }
   }
 }
@@ -726,7 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_map(&map_a);
     tma_prefetch_map(&map_b);
     if (P.n_static > 0) tma_prefetch_map(&map_a_static);
-    if (EPI == kEpiSwiglu) tma_prefetch_map(&map_b3);
+    if (swiglu_b(EPI)) tma_prefetch_map(&map_b3);
   }
   pdl_wait();              // what earlier kernels wrote is visible from here on
   pdl_trigger();
@@ -736,7 +869,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int base = 0; base < P.G; base += 32) {
       const int g = base + lane;
       int tiles = 0;
-      if (g < P.G) {
+      if (g < P.G && P.kgroup) {
+        // K-grouped: group g owns K columns [kseg[g], kseg[g+1]); rows = its k-blocks
+        const int k0 = P.kseg[g], k1 = P.kseg[g + 1];
+        const int kbg = (k1 - k0) / BK;
+        if (k0 < 0 || k1 < k0 || (k0 % BK) != 0 || (int64_t)k1 > P.a_rows) {
+          raise_error(P.err, kErrBadIndex);
+          s_off[g] = 0;
+          s_rows[g] = 0;
+        } else {
+          s_off[g] = k0;
+          s_rows[g] = kbg;
+        }
+        tiles = ((P.M + BM - 1) / BM) * P.nt;
+      } else if (g < P.G) {
         int off = 0, rows = 0;
         if (g < P.n_routed) {
           off = P.offsets[g];
@@ -794,7 +940,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
       int64_t a_row;
       const CUtensorMap *ma = a_of(tl, a_row);
-      const int b_row = tl.g * P.N + tl.n * P.bnh;
+      int b_row = tl.g * P.N + tl.n * P.bnh;
+      int kx = 0;                      // K coordinate of k-block 0
+      if (P.kgroup) {
+        ma = &map_a;
+        a_row = (int64_t)tl.m * BM;
+        b_row = tl.n * P.bnh;
+        kx = s_off[tl.g];
+        kb0 = 0;
+        kb1 = s_rows[tl.g];
+      }
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
         uint8_t *sa = smem + (size_t)stage * stage_bytes;
@@ -803,12 +958,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(&full_bar[stage], a_by_tma ? stage_bytes : b_bytes);
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-        if (a_by_tma) tma_load_2d(sa, ma, &full_bar[stage], kb * BK, (int)a_row);
-        if (EPI == kEpiSwiglu) {
-          tma_load_2d(sb, &map_b, &full_bar[stage], kb * BK, b_row);
-          tma_load_2d(sb + (b_bytes >> 1), &map_b3, &full_bar[stage], kb * BK, b_row);
+        if (a_by_tma) tma_load_2d(sa, ma, &full_bar[stage], kx + kb * BK, (int)a_row);
+        if (swiglu_b(EPI)) {
+          tma_load_2d(sb, &map_b, &full_bar[stage], kx + kb * BK, b_row);
+          tma_load_2d(sb + (b_bytes >> 1), &map_b3, &full_bar[stage], kx + kb * BK, b_row);
         } else {
-          tma_load_2d(sb, &map_b, &full_bar[stage], kb * BK, b_row);
+          tma_load_2d(sb, &map_b, &full_bar[stage], kx + kb * BK, b_row);
         }
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
       }
@@ -827,6 +982,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     bool ok = true;
     while (ok && sc.next(tile, kb0, kb1, part)) {
+      if (P.kgroup) {
+        const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
+        kb0 = 0;
+        kb1 = s_rows[tl.g];
+      }
       if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
@@ -903,7 +1063,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
       const bool in_tail = sk && tile >= sc.dp_limit;
-      if (in_tail && kb0 > 0) {
+      if (P.kgroup) {
+        // weight gradient tile: rows of group g's [M, N] output (split at split_m)
+        const int row = tl.m * BM + r_cta;
+        const bool zero = s_rows[tl.g] == 0;
+        float *dst = nullptr;
+        if (row < P.M)
+          dst = row < P.split_m
+                    ? reinterpret_cast<float *>(P.out) + ((int64_t)tl.g * P.split_m + row) * P.N
+                    : reinterpret_cast<float *>(P.out2) +
+                          ((int64_t)tl.g * (P.M - P.split_m) + row - P.split_m) * P.N;
+        epilogue_wgrad(P, taddr, zero, dst, tl.n * P.bnh);
+      } else if (in_tail && kb0 > 0) {
         sk_write(P, (int)blockIdx.x, r_cta, taddr);              // a later piece of the tile
       } else {
         const bool routed = tl.g < P.n_routed;
@@ -1001,7 +1172,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     tma_prefetch_map(&map_a);
     tma_prefetch_map(&map_b);
     if (P.n_static > 0) tma_prefetch_map(&map_a_static);
-    if (EPI == kEpiSwiglu) tma_prefetch_map(&map_b3);
+    if (swiglu_b(EPI)) tma_prefetch_map(&map_b3);
   }
   pdl_wait();              // what earlier kernels wrote is visible from here on
   pdl_trigger();
@@ -1057,13 +1228,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     bool ok = true;
     // B rows of this CTA: SwiGLU: even CTA the gate rows (W1), odd CTA the up
     // rows (W3); otherwise the two halves of the BN-row tile
-    const CUtensorMap *mb = (EPI == kEpiSwiglu && rank == 1) ? &map_b3 : &map_b;
+    const CUtensorMap *mb = (swiglu_b(EPI) && rank == 1) ? &map_b3 : &map_b;
     auto rows_of = [&](const Tile &tl, int64_t &a_row, int &b_row) -> const CUtensorMap * {
       const bool routed = tl.g < P.n_routed;
       a_row = (routed ? (int64_t)s_off[tl.g]
                       : P.a_static_base + (int64_t)(tl.g - P.n_routed) * P.a_static_stride) +
               (int64_t)tl.m * PM + (int64_t)rank * BM;
-      b_row = tl.g * P.N + tl.n * P.bnh + ((EPI == kEpiSwiglu) ? 0 : (int)rank * (P.bn / 2));
+      b_row = tl.g * P.N + tl.n * P.bnh + (swiglu_b(EPI) ? 0 : (int)rank * (P.bn / 2));
       return routed ? &map_a : &map_a_static;
     };
     while (ok && sc.next(tile, kb0, kb1, part)) {
@@ -1305,11 +1476,11 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   P.epi = g.epi;
   P.K = g.K;
   P.N = g.N;
-  if (g.epi == kEpiSwiglu) {
+  if (swiglu_b(g.epi)) {
     P.bn = 256;
     P.bnh = 128;
   } else if (g.epi == kEpiStoreF32) {
-    P.bn = std::max(32, (g.N + 31) / 32 * 32);
+    P.bn = std::min(256, std::max(32, (g.N + 31) / 32 * 32));
     P.bnh = P.bn;
   } else {
     P.bn = 256;
@@ -1331,37 +1502,53 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   P.bias = g.bias;
   P.ksplit = std::max(1, g.ksplit);
   P.split_stride = g.split_stride;
-  // stream-K tail for the expert GEMMs (the router splits K its own way)
-  const bool sk = MOE_STREAM_K && g.epi != kEpiStoreF32 && g.sk_part && g.sk_flags;
+  P.kgroup = g.kgroup;
+  P.M = g.M;
+  P.kseg = g.kseg;
+  P.split_m = g.out2 ? g.split_m : g.M;
+  P.out2 = g.out2;
+  P.aux = g.aux;
+  P.aux_ld = g.aux_ld;
+  // stream-K tail for the expert GEMMs (not with the router's K split or K groups)
+  const bool sk = MOE_STREAM_K && P.ksplit == 1 && !g.kgroup && g.n_routed > 0 && g.sk_part &&
+                  g.sk_flags;
   P.sk_part = sk ? g.sk_part : nullptr;
   P.sk_flags = sk ? g.sk_flags : nullptr;
   P.reverse = g.reverse;
   P.gather_rows = g.gather_rows;
   P.gather_src = g.gather_src;
   P.src_rows = g.src_rows;
-  if (g.gather_rows && (!g.gather_src || g.epi == kEpiStoreF32 || g.n_routed == 0))
+  if (g.gather_rows && (!g.gather_src || g.epi == kEpiStoreF32 || g.n_routed == 0 || g.kgroup))
     return cudaErrorInvalidValue;
   P.err = g.err;
   if (P.G <= 0 || P.G > kMaxGroups || P.bn > 256 || g.K % BK != 0) return cudaErrorInvalidValue;
   if (g.ksplit > 1 && (g.epi != kEpiStoreF32 || g.n_routed != 0)) return cudaErrorInvalidValue;
+  if ((g.epi == kEpiDActRelu || g.epi == kEpiDActSwiglu) && (!g.aux || !g.row_gate))
+    return cudaErrorInvalidValue;
+  if (g.kgroup && (g.epi != kEpiStoreF32 || g.n_routed != 0 || !g.kseg || g.M <= 0 ||
+                   (g.out2 && (g.split_m <= 0 || g.split_m >= g.M))))
+    return cudaErrorInvalidValue;
 
   // CTA pairs for the expert GEMMs whose groups are long enough that 256-row
   // tiles waste little (average routed rows per expert >= MOE_PAIR_MIN_ROWS)
-  const bool pair = g.epi != kEpiStoreF32 && g.n_routed > 0 && P.bn == 256 &&
+  const bool pair = !g.kgroup && g.n_routed > 0 && P.bn == 256 &&
                     g.max_routed_rows / g.n_routed >= MOE_PAIR_MIN_ROWS;
   CUtensorMap ma, mas, mb, mb3;
-  const uint32_t box_b = (g.epi == kEpiSwiglu || pair) ? 128u : (uint32_t)P.bn;
-  if (!make_map(&ma, g.a, (uint64_t)g.K, (uint64_t)g.a_rows, BM)) return cudaErrorInvalidValue;
-  if (!make_map(&mas, g.a_static ? g.a_static : g.a, (uint64_t)g.K,
-                (uint64_t)(g.a_static ? g.a_static_rows : g.a_rows), BM))
+  const uint32_t box_b = (swiglu_b(g.epi) || pair) ? 128u : (uint32_t)P.bn;
+  // K groups: A is [M, K] and B [N, K] with all groups' K columns side by side
+  const uint64_t a_outer = g.kgroup ? (uint64_t)g.M : (uint64_t)g.a_rows;
+  const uint64_t b_outer = g.kgroup ? (uint64_t)g.N : (uint64_t)g.b_rows;
+  if (!make_map(&ma, g.a, (uint64_t)g.K, a_outer, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&mas, g.a_static && !g.kgroup ? g.a_static : g.a, (uint64_t)g.K,
+                (uint64_t)(g.a_static && !g.kgroup ? g.a_static_rows : a_outer), BM))
     return cudaErrorInvalidValue;
-  if (!make_map(&mb, g.b, (uint64_t)g.K, (uint64_t)g.b_rows, box_b)) return cudaErrorInvalidValue;
-  if (!make_map(&mb3, g.b3 ? g.b3 : g.b, (uint64_t)g.K, (uint64_t)g.b_rows, box_b))
+  if (!make_map(&mb, g.b, (uint64_t)g.K, b_outer, box_b)) return cudaErrorInvalidValue;
+  if (!make_map(&mb3, g.b3 ? g.b3 : g.b, (uint64_t)g.K, b_outer, box_b))
     return cudaErrorInvalidValue;
 
   // grid: one CTA per SM, fewer when there are fewer tiles
   const int64_t mt_routed = (g.max_routed_rows + BM - 1) / BM + g.n_routed;
-  const int64_t mt_static = (int64_t)g.n_static * ((g.rows_static + BM - 1) / BM);
+  const int64_t mt_static = (int64_t)g.n_static * (((g.kgroup ? g.M : g.rows_static) + BM - 1) / BM);
   const int64_t max_tiles = (mt_routed + mt_static) * P.nt * P.ksplit;
   // (with stream-K, every SM: a short problem's k-blocks are spread over all)
   const int grid = std::min(kSkSlots, (int)std::max<int64_t>(1, std::min<int64_t>(
@@ -1375,20 +1562,37 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
     const int64_t pt_static = (int64_t)g.n_static * ((g.rows_static + 2 * BM - 1) / (2 * BM));
     const int64_t pair_tiles = (pt_routed + pt_static) * P.nt;
     const size_t psmem = (size_t)kPairStages * (kABytes + (size_t)(P.bn / 2) * BK * 2) + 1024;
+#define MOE_PAIR_CASE(E_)                                                            \
+  case E_:                                                                           \
+    return launch_pair<E_>(P, ma, mas, mb, mb3, pair_tiles, psmem, s);
     switch (g.epi) {
-      case kEpiRelu: return launch_pair<kEpiRelu>(P, ma, mas, mb, mb3, pair_tiles, psmem, s);
-      case kEpiSwiglu: return launch_pair<kEpiSwiglu>(P, ma, mas, mb, mb3, pair_tiles, psmem, s);
-      case kEpiScale: return launch_pair<kEpiScale>(P, ma, mas, mb, mb3, pair_tiles, psmem, s);
+      MOE_PAIR_CASE(kEpiStoreF32)
+      MOE_PAIR_CASE(kEpiRelu)
+      MOE_PAIR_CASE(kEpiSwiglu)
+      MOE_PAIR_CASE(kEpiScale)
+      MOE_PAIR_CASE(kEpiPreRelu)
+      MOE_PAIR_CASE(kEpiPreSwiglu)
+      MOE_PAIR_CASE(kEpiDActRelu)
+      MOE_PAIR_CASE(kEpiDActSwiglu)
       default: return cudaErrorInvalidValue;
     }
+#undef MOE_PAIR_CASE
   }
+#define MOE_ONE_CASE(E_)                                                             \
+  case E_:                                                                           \
+    return launch_epi<E_>(g, P, ma, mas, mb, mb3, grid, smem, s);
   switch (g.epi) {
-    case kEpiStoreF32: return launch_epi<kEpiStoreF32>(g, P, ma, mas, mb, mb3, grid, smem, s);
-    case kEpiRelu: return launch_epi<kEpiRelu>(g, P, ma, mas, mb, mb3, grid, smem, s);
-    case kEpiSwiglu: return launch_epi<kEpiSwiglu>(g, P, ma, mas, mb, mb3, grid, smem, s);
-    case kEpiScale: return launch_epi<kEpiScale>(g, P, ma, mas, mb, mb3, grid, smem, s);
+    MOE_ONE_CASE(kEpiStoreF32)
+    MOE_ONE_CASE(kEpiRelu)
+    MOE_ONE_CASE(kEpiSwiglu)
+    MOE_ONE_CASE(kEpiScale)
+    MOE_ONE_CASE(kEpiPreRelu)
+    MOE_ONE_CASE(kEpiPreSwiglu)
+    MOE_ONE_CASE(kEpiDActRelu)
+    MOE_ONE_CASE(kEpiDActSwiglu)
     default: return cudaErrorInvalidValue;
   }
+#undef MOE_ONE_CASE
 }
 
 }  // namespace moe

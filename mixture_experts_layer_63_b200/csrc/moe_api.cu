@@ -261,6 +261,267 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
   return launch_grouped_gemm(dn, s);
 }
 
+// ---- backward ----------------------------------------------------------------
+static int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+struct BwLayout {
+  size_t w2t, w1t, dy_perm, au, dau, dx_rows, kseg, kseg_r, dyT, hT, dauT, xT, dgate, dl, dl_pad, dlT,
+      xTr, wrT, dx_router, total;
+  int64_t kp_max, Ep, Tp;
+  int fw;
+};
+
+static BwLayout make_bw_layout(const moe_config *c, const WsLayout &L) {
+  BwLayout B{};
+  const int64_t T = c->T, d = c->d_model, f = c->d_ff;
+  const int G = c->E + c->S;
+  B.fw = (int)(c->act == MOE_ACT_SWIGLU ? 2 * f : f);
+  B.kp_max = round_up(L.rows_total + 64 * (int64_t)G, 64);
+  B.Ep = round_up(c->E, 64);
+  B.Tp = round_up(T, 64);
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  B.w2t = take((size_t)G * f * d * 2);
+  B.w1t = take((size_t)G * d * B.fw * 2);
+  B.dy_perm = take((size_t)L.rows_cap * d * 2);
+  B.au = take((size_t)L.rows_total * B.fw * 2);
+  B.dau = take((size_t)L.rows_total * B.fw * 2);
+  B.dx_rows = take((size_t)L.rows_total * d * 4);
+  B.kseg = take((size_t)(G + 1) * 4);
+  B.kseg_r = take(2 * 4);
+  B.dyT = take((size_t)d * B.kp_max * 2);
+  B.hT = take((size_t)f * B.kp_max * 2);
+  B.dauT = take((size_t)B.fw * B.kp_max * 2);
+  B.xT = take((size_t)d * B.kp_max * 2);
+  B.dgate = take((size_t)L.rows_cap * 4);
+  B.dl = take((size_t)T * c->E * 4);
+  B.dl_pad = take((size_t)T * B.Ep * 2);
+  B.dlT = take((size_t)c->E * B.Tp * 2);
+  B.xTr = take((size_t)d * B.Tp * 2);
+  B.wrT = take((size_t)d * B.Ep * 2);
+  B.dx_router = take((size_t)T * d * 4);
+  B.total = o;
+  return B;
+}
+
+static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const BwLayout &B,
+                                const char *ws_c, char *bw, const void *x, const void *w_router,
+                                const float *state, const void *w1, const void *w3, const void *w2,
+                                const void *dy, float *dx, float *dw_router, float *dbias,
+                                float *dw1, float *dw3, float *dw2, cudaStream_t s) {
+  char *ws = const_cast<char *>(ws_c);          // GEMM scratch and error word of the forward's workspace
+  uint32_t *err = reinterpret_cast<uint32_t *>(ws + L.err);
+  float *sk_part = reinterpret_cast<float *>(ws + L.sk_part);
+  int *sk_flags = reinterpret_cast<int *>(ws + L.err + kSkFlagsOffset);
+  const int64_t T = c->T, d = c->d_model, f = c->d_ff;
+  const int E = c->E, S = c->S, G = E + S;
+  const bool swiglu = c->act == MOE_ACT_SWIGLU;
+  const float *probs = reinterpret_cast<const float *>(ws + L.probs);
+  const int32_t *topk_idx = reinterpret_cast<const int32_t *>(ws + L.topk_idx);
+  const int32_t *offsets = reinterpret_cast<const int32_t *>(ws + L.offsets);
+  const int32_t *tok_rows = reinterpret_cast<const int32_t *>(ws + L.tok_rows);
+  const int32_t *row_token = reinterpret_cast<const int32_t *>(ws + L.row_token);
+  const float *row_gate = reinterpret_cast<const float *>(ws + L.row_gate);
+  const void *h = ws + L.h;
+  const float *y_rows = reinterpret_cast<const float *>(ws + L.y_rows);
+  const bool fused_gather = c->dtype == MOE_BF16 && MOE_FUSED_GATHER;
+  void *w2t = bw + B.w2t, *w1t = bw + B.w1t, *dy_perm = bw + B.dy_perm;
+  void *au = bw + B.au, *dau = bw + B.dau;
+  float *dx_rows = reinterpret_cast<float *>(bw + B.dx_rows);
+  int32_t *kseg = reinterpret_cast<int32_t *>(bw + B.kseg);
+  int32_t *kseg_r = reinterpret_cast<int32_t *>(bw + B.kseg_r);
+  float *dgate = reinterpret_cast<float *>(bw + B.dgate);
+  float *dl = reinterpret_cast<float *>(bw + B.dl);
+  float *dx_router = reinterpret_cast<float *>(bw + B.dx_router);
+  cudaError_t e;
+#define MOE_TRY(x_)            \
+  do {                         \
+    e = (x_);                  \
+    if (e != cudaSuccess) return e; \
+  } while (0)
+
+  // 1. transposed weights: W2^T [G][f][d]; [W1 | W3]^T [G][d][fw]
+  MOE_TRY(launch_transpose_bf16(w2, w2t, (int)d, (int)f, f, d, G, d * f, f * d, 0, s));
+  MOE_TRY(launch_transpose_bf16(w1, w1t, (int)f, (int)d, d, B.fw, G, f * d, d * B.fw, 0, s));
+  if (swiglu) MOE_TRY(launch_transpose_bf16(w3, w1t, (int)f, (int)d, d, B.fw, G, f * d, d * B.fw, (int)f, s));
+
+  // 2. pre-activations recomputed: A (| U) [rows_total][fw]
+  GroupedGemm up{};
+  up.epi = swiglu ? kEpiPreSwiglu : kEpiPreRelu;
+  up.K = (int)d;
+  up.N = (int)f;
+  up.a = fused_gather ? x : static_cast<const void *>(ws + L.x_perm);
+  up.a_rows = fused_gather ? T : L.rows_cap;
+  up.gather_rows = fused_gather ? row_token : nullptr;
+  up.gather_src = fused_gather ? x : nullptr;
+  up.src_rows = T;
+  up.a_static = x;
+  up.a_static_rows = T;
+  up.b = w1;
+  up.b3 = swiglu ? w3 : nullptr;
+  up.b_rows = (int64_t)G * f;
+  up.offsets = offsets;
+  up.n_routed = E;
+  up.n_static = S;
+  up.rows_static = T;
+  up.out_static_base = L.rows_cap;
+  up.max_routed_rows = L.rows_cap;
+  up.out = au;
+  up.sk_part = sk_part;
+  up.sk_flags = sk_flags;
+  up.err = err;
+  MOE_TRY(launch_grouped_gemm(up, s));
+
+  // 3. dY of the routed rows (ungated; the gate is applied in the epilogue)
+  MOE_TRY(launch_gather_bf16_rows(dy, dy_perm, row_token, offsets, E, T, (int)d, L.rows_cap, err, s));
+
+  // 4. dA (| dU) = act'(A, U) * (g * dY . W2)
+  GroupedGemm dh{};
+  dh.epi = swiglu ? kEpiDActSwiglu : kEpiDActRelu;
+  dh.K = (int)d;
+  dh.N = (int)f;
+  dh.a = dy_perm;
+  dh.a_rows = L.rows_cap;
+  dh.a_static = dy;
+  dh.a_static_rows = T;
+  dh.b = w2t;
+  dh.b_rows = (int64_t)G * f;
+  dh.offsets = offsets;
+  dh.n_routed = E;
+  dh.n_static = S;
+  dh.rows_static = T;
+  dh.out_static_base = L.rows_cap;
+  dh.max_routed_rows = L.rows_cap;
+  dh.out = dau;
+  dh.aux = au;
+  dh.aux_ld = B.fw;
+  dh.row_gate = row_gate;
+  dh.sk_part = sk_part;
+  dh.sk_flags = sk_flags;
+  dh.err = err;
+  MOE_TRY(launch_grouped_gemm(dh, s));
+
+  // 5. dX rows = [dA | dU] . [W1 | W3]   (fp32 rows)
+  GroupedGemm dxg{};
+  dxg.epi = kEpiStoreF32;
+  dxg.K = B.fw;
+  dxg.N = (int)d;
+  dxg.a = dau;
+  dxg.a_rows = L.rows_total;
+  dxg.a_static = dau;
+  dxg.a_static_rows = L.rows_total;
+  dxg.a_static_base = L.rows_cap;
+  dxg.a_static_stride = T;
+  dxg.b = w1t;
+  dxg.b_rows = (int64_t)G * d;
+  dxg.offsets = offsets;
+  dxg.n_routed = E;
+  dxg.n_static = S;
+  dxg.rows_static = T;
+  dxg.out_static_base = L.rows_cap;
+  dxg.max_routed_rows = L.rows_cap;
+  dxg.out = dx_rows;
+  dxg.sk_part = sk_part;
+  dxg.sk_flags = sk_flags;
+  dxg.err = err;
+  MOE_TRY(launch_grouped_gemm(dxg, s));
+
+  // 6-8. gate gradients, router logits gradient dl, bias gradient
+  MOE_TRY(launch_gate_grad(dy, y_rows, row_token, row_gate, offsets, E, (int)d, L.rows_cap, dgate, s));
+  MOE_TRY(launch_router_grad(c, probs, topk_idx, tok_rows, dgate, state, dl, s));
+  if (dbias) MOE_TRY(launch_bias_grad(dl, T, E, dbias, s));
+
+  // 9. router term of dx: dl [T, E] . W_r [E, d] (K padded to 64 with zeros)
+  MOE_TRY(launch_pad_f32_bf16(dl, bw + B.dl_pad, T, E, (int)B.Ep, s));
+  MOE_TRY(cudaMemsetAsync(bw + B.wrT, 0, (size_t)d * B.Ep * 2, s));
+  MOE_TRY(launch_transpose_bf16(w_router, bw + B.wrT, E, (int)d, d, B.Ep, 1, 0, 0, 0, s));
+  GroupedGemm rx{};
+  rx.epi = kEpiStoreF32;
+  rx.K = (int)B.Ep;
+  rx.N = (int)d;
+  rx.a = bw + B.dl_pad;
+  rx.a_rows = T;
+  rx.a_static = bw + B.dl_pad;
+  rx.a_static_rows = T;
+  rx.b = bw + B.wrT;
+  rx.b_rows = d;
+  rx.n_routed = 0;
+  rx.n_static = 1;
+  rx.rows_static = T;
+  rx.out = dx_router;
+  rx.ksplit = 1;
+  rx.err = err;
+  MOE_TRY(launch_grouped_gemm(rx, s));
+
+  // 10. dx = its dX rows + shared rows + the router term
+  MOE_TRY(launch_dx_finish(c, L.rows_cap, dx_rows, tok_rows, dx_router, dx, s));
+
+  // 11. router weights: dW_r = dl^T . x  (one K group over the tokens)
+  MOE_TRY(launch_transpose_f32_bf16(dl, bw + B.dlT, (int)T, E, (int)B.Tp, B.Tp, s));
+  MOE_TRY(cudaMemsetAsync(bw + B.xTr, 0, (size_t)d * B.Tp * 2, s));
+  MOE_TRY(launch_transpose_bf16(x, bw + B.xTr, (int)T, (int)d, d, B.Tp, 1, 0, 0, 0, s));
+  MOE_TRY(launch_seg_offsets(nullptr, 0, 1, T, kseg_r, s));
+  GroupedGemm rw{};
+  rw.epi = kEpiStoreF32;
+  rw.kgroup = 1;
+  rw.M = E;
+  rw.K = (int)B.Tp;
+  rw.N = (int)d;
+  rw.a = bw + B.dlT;
+  rw.a_rows = B.Tp;
+  rw.b = bw + B.xTr;
+  rw.b_rows = d;
+  rw.n_routed = 0;
+  rw.n_static = 1;
+  rw.kseg = kseg_r;
+  rw.out = dw_router;
+  rw.err = err;
+  MOE_TRY(launch_grouped_gemm(rw, s));
+
+  // 12. expert weights: each expert contracts over its own rows (K groups)
+  MOE_TRY(launch_seg_offsets(offsets, E, S, T, kseg, s));
+  MOE_TRY(launch_transpose_segments(dy, d, row_token, row_gate, 0, 0, T, T, offsets, kseg, E, G,
+                                    (int)d, B.kp_max, bw + B.dyT, err, s));
+  MOE_TRY(launch_transpose_segments(h, f, nullptr, nullptr, L.rows_cap, T, T, L.rows_total, offsets,
+                                    kseg, E, G, (int)f, B.kp_max, bw + B.hT, err, s));
+  MOE_TRY(launch_transpose_segments(dau, B.fw, nullptr, nullptr, L.rows_cap, T, T, L.rows_total,
+                                    offsets, kseg, E, G, B.fw, B.kp_max, bw + B.dauT, err, s));
+  MOE_TRY(launch_transpose_segments(x, d, row_token, nullptr, 0, 0, T, T, offsets, kseg, E, G,
+                                    (int)d, B.kp_max, bw + B.xT, err, s));
+  GroupedGemm w2g{};
+  w2g.epi = kEpiStoreF32;
+  w2g.kgroup = 1;
+  w2g.M = (int)d;
+  w2g.K = (int)B.kp_max;
+  w2g.N = (int)f;
+  w2g.a = bw + B.dyT;
+  w2g.a_rows = B.kp_max;
+  w2g.b = bw + B.hT;
+  w2g.b_rows = f;
+  w2g.n_routed = 0;
+  w2g.n_static = G;
+  w2g.kseg = kseg;
+  w2g.out = dw2;
+  w2g.err = err;
+  MOE_TRY(launch_grouped_gemm(w2g, s));
+  GroupedGemm w1g = w2g;
+  w1g.M = B.fw;
+  w1g.N = (int)d;
+  w1g.a = bw + B.dauT;
+  w1g.b = bw + B.xT;
+  w1g.b_rows = d;
+  w1g.out = dw1;
+  w1g.out2 = swiglu ? dw3 : nullptr;
+  w1g.split_m = (int)f;
+  MOE_TRY(launch_grouped_gemm(w1g, s));
+#undef MOE_TRY
+  return cudaSuccess;
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -448,6 +709,43 @@ moe_status moe_forward_timed(const moe_config *cfg, const void *x, const void *w
                              void *ws, size_t ws_bytes, void *const *events, moe_stream_t stream) {
   return forward_impl(cfg, x, w_router, bias, route_state, w1, w3, w2, y, counts_out, ws, ws_bytes,
                       events, stream);
+}
+
+moe_status moe_query_backward_size(const moe_config *cfg, size_t *bytes) {
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  const moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  const WsLayout L = make_layout(cfg);
+  *bytes = make_bw_layout(cfg, L).total;
+  return MOE_OK;
+}
+
+moe_status moe_backward(const moe_config *cfg, const void *x, const void *w_router,
+                        const float *bias, const float *route_state, const void *w1,
+                        const void *w3, const void *w2, const void *dy, float *dx, float *dw_router,
+                        float *dbias, float *dw1, float *dw3, float *dw2, const void *ws,
+                        size_t ws_bytes, void *bws, size_t bws_bytes, moe_stream_t stream) {
+  moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  const WsLayout L = make_layout(cfg);
+  if ((st = check_ws(L, ws, ws_bytes, L.total)) != MOE_OK) return st;
+  const BwLayout B = make_bw_layout(cfg, L);
+  if ((st = check_ws(L, bws, bws_bytes, B.total)) != MOE_OK) return st;
+  const bool swiglu = cfg->act == MOE_ACT_SWIGLU;
+  if (!x || !w_router || !w1 || !w2 || !dy || !dx || !dw_router || !dw1 || !dw2 ||
+      (swiglu && (!w3 || !dw3)) || (bias && !dbias))
+    return MOE_ERR_INVALID_ARG;
+  if (!state_ok(cfg, route_state)) return MOE_ERR_INVALID_ARG;
+  for (const void *p : {x, w_router, w1, w2, dy, static_cast<const void *>(dx),
+                        static_cast<const void *>(dw_router), static_cast<const void *>(dw1),
+                        static_cast<const void *>(dw2)})
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (swiglu && (!aligned16(w3) || !aligned16(dw3))) return MOE_ERR_INVALID_ARG;
+  return cuda_status(run_backward(cfg, L, B, static_cast<const char *>(ws), static_cast<char *>(bws),
+                                  x, w_router, route_state, w1, w3, w2, dy, dx, dw_router, dbias,
+                                  dw1, dw3, dw2, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_check_device_errors(void *ws, size_t ws_bytes, moe_stream_t stream, uint32_t *flags) {

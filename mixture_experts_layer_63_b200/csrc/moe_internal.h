@@ -136,6 +136,12 @@ enum GemmEpilogue : int {
   kEpiRelu = 1,       // out bf16 = relu(acc)                    (up-projection, ReLU)
   kEpiSwiglu = 2,     // out bf16 = silu(acc_gate) * acc_up      (gate/up projection)
   kEpiScale = 3,      // out fp32 = row_gate[row] * acc          (down-projection)
+  // backward
+  kEpiPreRelu = 4,    // out bf16 = acc                          (pre-activation a, recomputed)
+  kEpiPreSwiglu = 5,  // out bf16 [row][col] = a, [row][N+col] = u  (gate/up pre-activations)
+  kEpiDActRelu = 6,   // dh = g*acc; out bf16 = dh * [a > 0]     (a from aux [row][col])
+  kEpiDActSwiglu = 7, // dh = g*acc; s = sigmoid(a): out[row][col] = dh u s (1 + a (1 - s)),
+                      //   out[row][N+col] = dh a s              (a, u from aux, ld 2N)
 };
 
 // One grouped GEMM  out[rows_g, N] = A[rows_g, K] . B_g[N, K]^T  per group g.
@@ -172,9 +178,51 @@ struct GroupedGemm {
   const int32_t *gather_rows;  // non-null: routed A row r is gather_src[gather_rows[r]]
   const void *gather_src;      //   (the row gather done inside the GEMM; bf16 [src_rows, K])
   int64_t src_rows;
+  const void *aux;          // kEpiDAct*: bf16 pre-activations, ld aux_ld
+  int64_t aux_ld;
+  // K-grouped mode (weight gradients): group g computes out_g[M, N] =
+  // A[M, kseg[g]:kseg[g+1]] . B[N, kseg[g]:kseg[g+1]]^T over the K columns
+  // kseg gives (multiples of 64, device array of n_static + 1 entries; one
+  // group per static group, n_routed = 0); A is [M, a_rows = Kp], B [N, Kp]
+  // (row-major, K contiguous).  fp32 out: row r < split_m of group g at
+  // out + (g*split_m + r)*N, rows r >= split_m at out2 + (g*split_m + r - split_m)*N.
+  int kgroup;
+  int M;
+  const int32_t *kseg;
+  int split_m;
+  void *out2;
   uint32_t *err;
 };
 cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s);
+
+// --- backward helpers (backward.cu) ----------------------------------------
+cudaError_t launch_transpose_bf16(const void *in, void *out, int R, int C, int64_t ld_in,
+                                  int64_t ld_out, int batch, int64_t bstride_in,
+                                  int64_t bstride_out, int col_off, cudaStream_t s);
+cudaError_t launch_transpose_f32_bf16(const float *in, void *out, int R, int C, int Rpad,
+                                      int64_t ld_out, cudaStream_t s);
+cudaError_t launch_seg_offsets(const int32_t *offsets, int E, int S, int64_t T, int32_t *kseg,
+                               cudaStream_t s);
+cudaError_t launch_transpose_segments(const void *src, int64_t ld, const int32_t *map,
+                                      const float *scale, int64_t shared_base, int64_t shared_stride,
+                                      int64_t shared_len, int64_t src_rows, const int32_t *offsets,
+                                      const int32_t *kseg, int E, int G, int C, int64_t kp_max,
+                                      void *out, uint32_t *err, cudaStream_t s);
+cudaError_t launch_gather_bf16_rows(const void *src, void *dst, const int32_t *map,
+                                    const int32_t *offsets, int E, int64_t src_rows, int d,
+                                    int64_t max_rows, uint32_t *err, cudaStream_t s);
+cudaError_t launch_gate_grad(const void *dy, const float *y_rows, const int32_t *row_token,
+                             const float *row_gate, const int32_t *offsets, int E, int d,
+                             int64_t max_rows, float *dgate, cudaStream_t s);
+cudaError_t launch_router_grad(const moe_config *c, const float *probs, const int32_t *topk_idx,
+                               const int32_t *tok_rows, const float *dgate, const float *state,
+                               float *dl, cudaStream_t s);
+cudaError_t launch_bias_grad(const float *dl, int64_t T, int E, float *dbias, cudaStream_t s);
+cudaError_t launch_dx_finish(const moe_config *c, int64_t rows_cap, const float *dx_rows,
+                             const int32_t *tok_rows, const float *dx_router, float *dx,
+                             cudaStream_t s);
+cudaError_t launch_pad_f32_bf16(const float *in, void *out, int64_t R, int C, int Cp,
+                                cudaStream_t s);
 // K parts of the bf16 router GEMM: enough CTAs to fill the GPU, >= 4 k-blocks each
 inline int router_ksplit(const moe_config *c) {
   const int64_t mtiles = (c->T + 127) / 128;

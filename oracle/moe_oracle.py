@@ -581,6 +581,7 @@ class Grads:
     dw1: np.ndarray              # [E+S, f, d]
     dw3: np.ndarray | None       # [E+S, f, d] (SwiGLU)
     dw2: np.ndarray              # [E+S, d, f]
+    dlogits: np.ndarray | None = None   # [T, E]: dL/d(router logits)
 
 
 def softmax_f64(logits: np.ndarray) -> np.ndarray:
@@ -716,7 +717,7 @@ def backward(cfg: OracleConfig, x, w_router, bias, w1, w3, w2, dy, state=None,
     # softmax backward, then the router
     dl = softmax_backward(p, dp)
     dx += dl @ widen(w_router)
-    return Grads(dx, dl.T @ xs, None if bias is None else dl.sum(axis=0), dw1, dw3, dw2)
+    return Grads(dx, dl.T @ xs, None if bias is None else dl.sum(axis=0), dw1, dw3, dw2, dl)
 
 
 def forward_fixed_selection(cfg: OracleConfig, x, w_router, bias, w1, w3, w2, disp: Dispatch,
