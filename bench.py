@@ -403,7 +403,7 @@ def run_ours(args, w) -> None:
     nmat = 3 if w.act == "swiglu" else 2
     gemm_flops = 2.0 * rows * w.d_model * w.d_ff * nmat
     permute_bytes = (w.T * w.d_model + R * w.d_model) * es
-    combine_bytes = rows * w.d_model * 4 + w.T * w.d_model * es     # fp32 rows in, y out
+    combine_bytes = rows * w.d_model * es + w.T * w.d_model * es    # gated rows in, y out
     route_bytes = (w.T * w.d_model + w.E * w.d_model) * es + 2 * w.T * w.E * 4
     mean = per.mean(axis=0)                                # ms per call
     hbm, tfl, tfl_sus, peak_src = _peaks()
@@ -442,6 +442,43 @@ def run_ours(args, w) -> None:
         dist.barrier()
     e2e_value = replicas.throughput(world, w.T, args.steps, e2e_ms)
 
+    # training: forward + backward (moe_backward) per step, separate steps,
+    # not part of `value`; every rank takes the same steps
+    backward = None
+    if w.dtype == "bf16" and not args.no_backward:
+        g = torch.Generator(device="cuda")
+        g.manual_seed(args.seed + 17)
+        dy = torch.randn(w.T, w.d_model, generator=g, device="cuda").to(inp.x.dtype)
+        for _ in range(args.warmup):
+            flush.zero_()
+            layer(inp.x, out=y_dev)
+            layer.backward(inp.x, dy)
+        bev = new_events(3)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        for i in range(args.steps):
+            flush.zero_()
+            bev[i][0].record(stream)
+            layer(inp.x, out=y_dev)
+            bev[i][1].record(stream)
+            layer.backward(inp.x, dy)
+            bev[i][2].record(stream)
+        torch.cuda.synchronize()
+        api.moe_check_device_errors(layer.ws)
+        bw_ms = replicas.max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in bev), dist, device="cuda")
+        fb_ms = replicas.max_over_ranks(sum(e[0].elapsed_time(e[2]) for e in bev), dist, device="cuda")
+        # flops of the backward's contractions: recompute of the pre-activations,
+        # dH, dX, dW2, dW1 (| dW3), plus the router's dx and dW_r
+        nb = (2 + 1 + 2 + 1 + 2) if w.act == "swiglu" else (1 + 1 + 1 + 1 + 1)
+        bw_flops = 2.0 * rows * w.d_model * w.d_ff * nb + 2 * 2.0 * w.T * w.E * w.d_model
+        backward = {"ms_per_step": bw_ms / args.steps,
+                    "tokens_per_s_fwd_bwd": replicas.throughput(world, w.T, args.steps, fb_ms),
+                    "achieved_tflops": bw_flops / (bw_ms / args.steps * 1e-3) / 1e12,
+                    "algorithmic_flops": bw_flops,
+                    "note": "moe_backward after moe_forward, routing held fixed; separate steps"}
+        del layer.bws
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, args.seed, "cuda")
@@ -477,6 +514,7 @@ def run_ours(args, w) -> None:
             "gpu_launches": launches_per_step(w) * args.steps,
             "clocks": clk,
             "cpu_baseline": cpu,
+            "backward": backward,
         }
         print(json.dumps(line), flush=True)
     if dist:
@@ -547,6 +585,8 @@ def main() -> None:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the forward + backward measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm-vs-library", action="store_true",
                     help="time the expert GEMMs on this workload's dense shape next to torch.matmul")

@@ -36,9 +36,9 @@
  *   - Layout: row-major.  x [T, d]; w_router [E, d]; w1, w3 [E+S, f, d];
  *     w2 [E+S, d, f] (each output neuron's weights contiguous along its input
  *     dimension); experts 0..E-1 are routed, E..E+S-1 shared.  Element type
- *     fp32 (MOE_F32) or bf16 (MOE_BF16) for x, weights, x_perm, h and y.
- *     y_rows, router logits, probabilities and gates are always fp32 (the
- *     combine sums fp32 rows and rounds once); indices int32.
+ *     fp32 (MOE_F32) or bf16 (MOE_BF16) for x, weights, x_perm, h, y_rows
+ *     and y (the combine sums rows in fp32 and rounds once).  Router logits,
+ *     probabilities and gates are always fp32; indices int32.
  *   - Alignment: tensor pointers 16-byte aligned, the workspace 256-byte
  *     aligned.  Limits of this build (else MOE_ERR_UNSUPPORTED): E <= 256,
  *     S <= 8, k <= 8, n_groups <= 32, topk_groups <= 8, T*k and E*C below
@@ -222,7 +222,7 @@ MOE_API moe_status moe_permute_noalloc(const moe_config *cfg, const void *x, con
  *   in : x [T, d] (input of the shared experts), x_perm [rows_cap, d],
  *        offsets [E+1], row_gate [rows_cap], w1, w3 (SwiGLU; NULL for ReLU), w2.
  *   out: h [rows_total, f]  activations, layer dtype (scratch the caller may read);
- *        y_rows [rows_total, d] fp32: routed row r = row_gate[r] * FFN_e(x_perm[r]);
+ *        y_rows [rows_total, d], layer dtype: routed row r = row_gate[r] * FFN_e(x_perm[r]);
  *        shared expert s, token t at row rows_cap + s*T + t = FFN_{E+s}(x[t]).
  *   bf16: tcgen05 tensor cores, bf16 operands, fp32 accumulation, h rounded
  *   to bf16.  fp32: CUDA-core fp32 arithmetic. */
@@ -231,7 +231,7 @@ MOE_API moe_status moe_expert_ffn(const moe_config *cfg, const void *x, const vo
                           const void *w3, const void *w2, void *h, void *y_rows, void *ws,
                           size_t ws_bytes, moe_stream_t stream);
 
-/* Step 5c: y[t] = sum of t's fp32 routed rows (token choice: in k-rank order;
+/* Step 5c: y[t] = sum of t's routed rows (layer dtype; token choice: in k-rank order;
  * expert choice: ascending expert) + its shared rows, fp32 accumulation,
  * rounded once to the layer dtype.  A token with no kept row and no shared
  * expert gets 0. */

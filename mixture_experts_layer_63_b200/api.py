@@ -320,7 +320,7 @@ def step_buffers(cfg: MoeConfig, device="cuda") -> StepBuffers:
         x_perm=torch.empty(max(s.rows_cap, 1), d, dtype=dt, device=device),
         n_dropped=torch.empty(1, dtype=i32, device=device),
         h=torch.empty(s.rows_total, f, dtype=dt, device=device),
-        y_rows=torch.empty(s.rows_total, d, dtype=torch.float32, device=device),
+        y_rows=torch.empty(s.rows_total, d, dtype=dt, device=device),
         y=torch.empty(T, d, dtype=dt, device=device),
         ws=new_workspace(cfg, device, step_only=True),
     )

@@ -165,10 +165,10 @@ __global__ void __launch_bounds__(256) gather_bf16_rows_kernel(const uint4 *__re
 
 // ---- gate gradients and the router ---------------------------------------
 // dG_r = <dy[t], FFN_e(x_t)> for each kept routed row r of token t: the
-// forward's fp32 row is g_r * FFN_e(x_t), so dG_r = <dy[t], y_row> / g_r
+// forward's bf16 row is g_r * FFN_e(x_t), so dG_r = <dy[t], y_row> / g_r
 // (0 when g_r is 0: such a row contributes nothing, and neither does its gate).
 __global__ void __launch_bounds__(256) gate_grad_kernel(const __nv_bfloat16 *__restrict__ dy,
-                                                        const float *__restrict__ y_rows,
+                                                        const __nv_bfloat16 *__restrict__ y_rows,
                                                         const int32_t *__restrict__ row_token,
                                                         const float *__restrict__ row_gate,
                                                         const int32_t *__restrict__ offsets, int E,
@@ -181,12 +181,13 @@ __global__ void __launch_bounds__(256) gate_grad_kernel(const __nv_bfloat16 *__r
   for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += nw) {
     const int64_t t = row_token[r];
     const __nv_bfloat16 *a = dy + t * d;
-    const float *b = y_rows + r * d;
+    const __nv_bfloat16 *b = y_rows + r * d;
     float acc = 0.0f;
     for (int i = lane * 2; i < d; i += 64) {
       const __nv_bfloat162 av = *reinterpret_cast<const __nv_bfloat162 *>(a + i);
-      acc = fmaf(__low2float(av), b[i], acc);
-      acc = fmaf(__high2float(av), b[i + 1], acc);
+      const __nv_bfloat162 bv = *reinterpret_cast<const __nv_bfloat162 *>(b + i);
+      acc = fmaf(__low2float(av), __low2float(bv), acc);
+      acc = fmaf(__high2float(av), __high2float(bv), acc);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -358,13 +359,14 @@ cudaError_t launch_gather_bf16_rows(const void *src, void *dst, const int32_t *m
                        static_cast<uint4 *>(dst), map, offsets, E, src_rows, d / 8, err);
 }
 
-cudaError_t launch_gate_grad(const void *dy, const float *y_rows, const int32_t *row_token,
+cudaError_t launch_gate_grad(const void *dy, const void *y_rows, const int32_t *row_token,
                              const float *row_gate, const int32_t *offsets, int E, int d,
                              int64_t max_rows, float *dgate, cudaStream_t s) {
   const int64_t want = (max_rows + 7) / 8;
   const unsigned blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, 148 * 16));
   return launch_kernel(gate_grad_kernel, blocks, 256, 0, s, static_cast<const __nv_bfloat16 *>(dy),
-                       y_rows, row_token, row_gate, offsets, E, d, dgate);
+                       static_cast<const __nv_bfloat16 *>(y_rows), row_token, row_gate, offsets, E,
+                       d, dgate);
 }
 
 cudaError_t launch_router_grad(const moe_config *c, const float *probs, const int32_t *topk_idx,

@@ -1,10 +1,10 @@
 // Gate-weighted combine (GShard section 3 of "MoE技术演进": y_s = sum_e
 // G_{s,e} FFN_e(x_s); DeepSeekMoE section 2: plus the shared experts' sum).
-// The gates were applied in the down-projection epilogue, which leaves fp32
-// rows; here each token sums its rows: routed rows in the token's k-rank
-// order (expert choice: ascending expert), then shared experts 0..S-1, fp32
-// accumulation, one rounding to the output dtype.  One warp per token,
-// 16-byte vectors.
+// The gates were applied in the down-projection epilogue, which leaves rows
+// in the layer dtype; here each token sums its rows: routed rows in the
+// token's k-rank order (expert choice: ascending expert), then shared experts
+// 0..S-1, fp32 accumulation, one rounding to the output dtype.  One warp per
+// token, 16-byte vectors.
 #include "device_common.cuh"
 #include "moe_internal.h"
 
@@ -41,24 +41,26 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const void *__rest
   n += S;
   __syncwarp();
 
-  // y_rows are fp32; 8 (bf16 out) or 4 (fp32 out) elements per lane and step
+  // one 16-byte vector per lane and step: 8 bf16 or 4 fp32 elements
   constexpr int EPV = BF16 ? 8 : 4;
   const int nvec = d / EPV;
-  const float4 *src = reinterpret_cast<const float4 *>(y_rows);
-  const int64_t row_vec = d / 4;                 // float4 per fp32 row
+  const uint4 *src = reinterpret_cast<const uint4 *>(y_rows);
   for (int v = lane; v < nvec; v += 32) {
     float acc[EPV];
 #pragma unroll
     for (int i = 0; i < EPV; ++i) acc[i] = 0.f;
     for (int i = 0; i < n; ++i) {
-      const float4 *p = src + (int64_t)rows[i] * row_vec + (int64_t)v * (EPV / 4);
-#pragma unroll
-      for (int q = 0; q < EPV / 4; ++q) {
-        const float4 a = p[q];
-        acc[4 * q + 0] += a.x;
-        acc[4 * q + 1] += a.y;
-        acc[4 * q + 2] += a.z;
-        acc[4 * q + 3] += a.w;
+      const uint4 a = src[(int64_t)rows[i] * nvec + v];
+      if (BF16) {
+        acc[0] += bf16_lo(a.x); acc[1] += bf16_hi(a.x);
+        acc[2 % EPV] += bf16_lo(a.y); acc[3 % EPV] += bf16_hi(a.y);
+        acc[4 % EPV] += bf16_lo(a.z); acc[5 % EPV] += bf16_hi(a.z);
+        acc[6 % EPV] += bf16_lo(a.w); acc[7 % EPV] += bf16_hi(a.w);
+      } else {
+        acc[0] += __uint_as_float(a.x);
+        acc[1] += __uint_as_float(a.y);
+        acc[2 % EPV] += __uint_as_float(a.z);
+        acc[3 % EPV] += __uint_as_float(a.w);
       }
     }
     if (BF16) {

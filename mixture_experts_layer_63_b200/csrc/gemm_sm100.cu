@@ -661,8 +661,8 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
       if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
     }
   } else if (EPI == kEpiScale) {
-    // fp32 rows: the combine rounds once, after summing
-    float *out = reinterpret_cast<float *>(P.out);
+    // gated rows in bf16; the combine sums them in fp32 and rounds once
+    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
     const float scale = (routed && valid) ? P.row_gate[out_row] : 1.0f;
 #pragma unroll 1
     for (int c = 0; c < P.bn / 32; ++c) {
@@ -671,14 +671,10 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
 #pragma unroll
       for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
       if (F) add_parts(v, *F, c * 32);
-      const int col = col0 + c * 32;
-      if (valid && col < P.N) {
-        float4 *dst = reinterpret_cast<float4 *>(out + out_row * P.N + col);
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          dst[q] = make_float4(v[4 * q] * scale, v[4 * q + 1] * scale, v[4 * q + 2] * scale,
-                               v[4 * q + 3] * scale);
-      }
+      for (int i = 0; i < 32; ++i) v[i] *= scale;
+      const int col = col0 + c * 32;
+      if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
     }
   } else if (EPI == kEpiPreRelu) {
     __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);

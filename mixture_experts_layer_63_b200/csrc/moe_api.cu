@@ -117,7 +117,7 @@ WsLayout make_layout(const moe_config *c) {
   const bool fused_gather = c->dtype == MOE_BF16 && MOE_FUSED_GATHER;
   L.x_perm = take(fused_gather ? 0 : (size_t)L.rows_cap * c->d_model * es);
   L.h = take((size_t)L.rows_total * c->d_ff * es);
-  L.y_rows = take((size_t)L.rows_total * c->d_model * 4);      // fp32 rows
+  L.y_rows = take((size_t)L.rows_total * c->d_model * es);     // rows in the layer dtype
   L.total = o;
   return L;
 }
@@ -327,7 +327,7 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
   const int32_t *row_token = reinterpret_cast<const int32_t *>(ws + L.row_token);
   const float *row_gate = reinterpret_cast<const float *>(ws + L.row_gate);
   const void *h = ws + L.h;
-  const float *y_rows = reinterpret_cast<const float *>(ws + L.y_rows);
+  const void *y_rows = ws + L.y_rows;
   const bool fused_gather = c->dtype == MOE_BF16 && MOE_FUSED_GATHER;
   void *w2t = bw + B.w2t, *w1t = bw + B.w1t, *dy_perm = bw + B.dy_perm;
   void *au = bw + B.au, *dau = bw + B.dau;

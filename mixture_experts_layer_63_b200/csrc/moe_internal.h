@@ -211,7 +211,7 @@ cudaError_t launch_transpose_segments(const void *src, int64_t ld, const int32_t
 cudaError_t launch_gather_bf16_rows(const void *src, void *dst, const int32_t *map,
                                     const int32_t *offsets, int E, int64_t src_rows, int d,
                                     int64_t max_rows, uint32_t *err, cudaStream_t s);
-cudaError_t launch_gate_grad(const void *dy, const float *y_rows, const int32_t *row_token,
+cudaError_t launch_gate_grad(const void *dy, const void *y_rows, const int32_t *row_token,
                              const float *row_gate, const int32_t *offsets, int E, int d,
                              int64_t max_rows, float *dgate, cudaStream_t s);
 cudaError_t launch_router_grad(const moe_config *c, const float *probs, const int32_t *topk_idx,
