@@ -11,12 +11,15 @@
 // This file holds the data-movement and small arithmetic kernels; the
 // contractions run on the tcgen05 grouped GEMM (gemm_sm100.cu):
 //   recompute    A|U = X . [W1|W3]^T            (pre-activations, bf16)
-//   dact         dA|dU = act'(A, U) * (g * dY . W2)      (fused epilogue)
-//   dX rows      dX = [dA|dU] . [W1|W3]          (fp32 rows, summed per token)
+//   dact         dA|dU = act'(A, U) * (g * dY . W2)      (fused epilogue;
+//                W2 read as it is stored, MN-major)
+//   dX rows      dX = [dA|dU] . [W1;W3]          (fp32 rows, summed per token;
+//                W1, W3 read MN-major)
 //   wgrad        dW2_e = (g dY)_e^T H_e,  [dW1|dW3]_e = [dA|dU]_e^T X_e
 //                (K-grouped: each expert contracts over its own rows)
 //   router       dW_r = dl^T X,  dx += dl . W_r   (dl from the gate gradients)
-// Transposed operands are built here (the GEMM takes K-major operands only).
+// The weight-gradient operands are transposed here into 64-padded segments
+// (an expert's rows are not 64-aligned in the forward's row layout).
 #include <algorithm>
 
 #include "device_common.cuh"
@@ -25,26 +28,86 @@
 namespace moe {
 namespace {
 
-// ---- tiled transposes (32 x 32 tiles through shared memory) ---------------
-// out[b][c][col_off + r] = in[b][r][c] for r < R, c < C (bf16).
-__global__ void transpose_bf16_kernel(const uint16_t *__restrict__ in, uint16_t *__restrict__ out,
-                                      int R, int C, int64_t ld_in, int64_t ld_out,
-                                      int64_t bstride_in, int64_t bstride_out, int col_off) {
-  __shared__ uint16_t tile[32][33];
+// ---- tiled transposes (64 x 64 bf16 tiles through shared memory) ----------
+// A tile is read as 16-byte vectors along its rows (8 elements) and written
+// as 16-byte vectors along its columns; partial vectors at a ragged edge
+// fall back to single elements.
+constexpr int kTT = 64;                 // tile edge
+constexpr int kTP = kTT + 2;            // shared-memory row pitch (halfs): spreads the banks
+
+struct TileIO {
+  // source row r of the tile (-1: zeros) and its factor
+  int64_t row;
+  float scale;
+};
+
+__device__ __forceinline__ void tile_load_row(uint16_t (*tile)[kTP], int i, const uint16_t *src_row,
+                                              int c0, int C, int v, float scale) {
+  // 8 elements c0 + 8v .. c0 + 8v + 7 of one source row into tile[i][8v..]
+  const int c = c0 + 8 * v;
+  uint16_t e[8];
+  if (src_row && c + 8 <= C && ((reinterpret_cast<uintptr_t>(src_row + c) & 15) == 0)) {
+    const uint4 q = *reinterpret_cast<const uint4 *>(src_row + c);
+    e[0] = (uint16_t)(q.x & 0xffff); e[1] = (uint16_t)(q.x >> 16);
+    e[2] = (uint16_t)(q.y & 0xffff); e[3] = (uint16_t)(q.y >> 16);
+    e[4] = (uint16_t)(q.z & 0xffff); e[5] = (uint16_t)(q.z >> 16);
+    e[6] = (uint16_t)(q.w & 0xffff); e[7] = (uint16_t)(q.w >> 16);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) e[j] = (src_row && c + j < C) ? src_row[c + j] : (uint16_t)0;
+  }
+  if (scale != 1.0f) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      e[j] = __bfloat16_as_ushort(__float2bfloat16_rn(scale * __bfloat162float(__ushort_as_bfloat16(e[j]))));
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) tile[i][8 * v + j] = e[j];
+}
+
+// out row (tile column) c: 8 consecutive tile rows 8v .. 8v+7 at dst[8v..]
+__device__ __forceinline__ void tile_store_col(uint16_t (*tile)[kTP], int c, uint16_t *dst, int v,
+                                               int nrows) {
+  uint16_t e[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) e[j] = tile[8 * v + j][c];
+  if (8 * v + 8 <= nrows && ((reinterpret_cast<uintptr_t>(dst + 8 * v) & 15) == 0)) {
+    uint4 q;
+    q.x = (uint32_t)e[0] | ((uint32_t)e[1] << 16);
+    q.y = (uint32_t)e[2] | ((uint32_t)e[3] << 16);
+    q.z = (uint32_t)e[4] | ((uint32_t)e[5] << 16);
+    q.w = (uint32_t)e[6] | ((uint32_t)e[7] << 16);
+    *reinterpret_cast<uint4 *>(dst + 8 * v) = q;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (8 * v + j < nrows) dst[8 * v + j] = e[j];
+  }
+}
+
+// out[b][c][col_off + r] = in[b][r][c] for r < R, c < C (bf16), 256 threads
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const uint16_t *__restrict__ in,
+                                                             uint16_t *__restrict__ out, int R, int C,
+                                                             int64_t ld_in, int64_t ld_out,
+                                                             int64_t bstride_in, int64_t bstride_out,
+                                                             int col_off) {
+  __shared__ uint16_t tile[kTT][kTP];
   pdl_wait();
   pdl_trigger();
   const int64_t b = blockIdx.z;
-  const int r0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
+  const int r0 = blockIdx.x * kTT, c0 = blockIdx.y * kTT;
   const uint16_t *src = in + b * bstride_in;
   uint16_t *dst = out + b * bstride_out;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int r = r0 + i, c = c0 + threadIdx.x;
-    if (r < R && c < C) tile[i][threadIdx.x] = src[(int64_t)r * ld_in + c];
+  for (int k = threadIdx.x; k < kTT * 8; k += blockDim.x) {
+    const int i = k >> 3, v = k & 7;
+    const int r = r0 + i;
+    tile_load_row(tile, i, r < R ? src + (int64_t)r * ld_in : nullptr, c0, C, v, 1.0f);
   }
   __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int c = c0 + i, r = r0 + threadIdx.x;
-    if (r < R && c < C) dst[(int64_t)c * ld_out + col_off + r] = tile[threadIdx.x][i];
+  const int nrows = min(kTT, R - r0);
+  for (int k = threadIdx.x; k < kTT * 8; k += blockDim.x) {
+    const int c = k >> 3, v = k & 7;
+    if (c0 + c < C) tile_store_col(tile, c, dst + (int64_t)(c0 + c) * ld_out + col_off + r0, v, nrows);
   }
 }
 
@@ -87,6 +150,7 @@ __global__ void seg_offsets_kernel(const int32_t *__restrict__ offsets, int E, i
 // (zeros in the padding up to the next segment).  Row i of routed group e
 // is r = offsets[e] + i, read at map[r] (null: r); scale_i = scale[r] (null:
 // 1).  Row i of shared group s is read at shared_base + s * shared_stride + i.
+// 64 x 64 tiles: segments are 64-aligned, so a tile never straddles two.
 struct SegSrc {
   const __nv_bfloat16 *src;
   int64_t ld;                // elements per source row
@@ -101,10 +165,12 @@ __global__ void __launch_bounds__(256) transpose_segments_kernel(SegSrc S_, cons
                                                                  __nv_bfloat16 *__restrict__ out,
                                                                  uint32_t *err, int64_t src_rows,
                                                                  int64_t shared_len) {
-  __shared__ float tile[32][33];
+  __shared__ uint16_t tile[kTT][kTP];
+  __shared__ int64_t s_row[kTT];
+  __shared__ float s_scale[kTT];
   pdl_wait();
   pdl_trigger();
-  const int k0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
+  const int k0 = blockIdx.x * kTT, c0 = blockIdx.y * kTT;
   if (k0 >= kseg[G]) return;                            // past the last segment
   int lo = 0, hi = G - 1;                               // group holding column k0
   while (lo < hi) {
@@ -114,13 +180,11 @@ __global__ void __launch_bounds__(256) transpose_segments_kernel(SegSrc S_, cons
   }
   const int g = lo;
   const int64_t len = g < E ? (int64_t)(offsets[g + 1] - offsets[g]) : shared_len;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int64_t li = (int64_t)(k0 - kseg[g]) + i;      // row of the segment
-    const int c = c0 + threadIdx.x;
-    float v = 0.0f;
-    if (c < C && li < len) {
-      int64_t row;
-      float sc = 1.0f;
+  if (threadIdx.x < kTT) {
+    const int64_t li = (int64_t)(k0 - kseg[g]) + threadIdx.x;    // row of the segment
+    int64_t row = -1;
+    float sc = 1.0f;
+    if (li < len) {
       if (g < E) {
         const int64_t r = (int64_t)offsets[g] + li;
         row = S_.map ? S_.map[r] : r;
@@ -128,15 +192,26 @@ __global__ void __launch_bounds__(256) transpose_segments_kernel(SegSrc S_, cons
       } else {
         row = S_.shared_base + (int64_t)(g - E) * S_.shared_stride + li;
       }
-      if (row >= 0 && row < src_rows) v = sc * __bfloat162float(S_.src[row * S_.ld + c]);
-      else raise_error(err, kErrBadIndex);
+      if (row < 0 || row >= src_rows) {
+        raise_error(err, kErrBadIndex);
+        row = -1;
+      }
     }
-    tile[i][threadIdx.x] = v;
+    s_row[threadIdx.x] = row;
+    s_scale[threadIdx.x] = sc;
   }
   __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int c = c0 + i;
-    if (c < C) out[(int64_t)c * ld_out + k0 + threadIdx.x] = __float2bfloat16_rn(tile[threadIdx.x][i]);
+  const uint16_t *src = reinterpret_cast<const uint16_t *>(S_.src);
+  for (int k = threadIdx.x; k < kTT * 8; k += blockDim.x) {
+    const int i = k >> 3, v = k & 7;
+    const int64_t row = s_row[i];
+    tile_load_row(tile, i, row >= 0 ? src + row * S_.ld : nullptr, c0, C, v, s_scale[i]);
+  }
+  __syncthreads();
+  uint16_t *dst = reinterpret_cast<uint16_t *>(out);
+  for (int k = threadIdx.x; k < kTT * 8; k += blockDim.x) {
+    const int c = k >> 3, v = k & 7;
+    if (c0 + c < C) tile_store_col(tile, c, dst + (int64_t)(c0 + c) * ld_out + k0, v, kTT);
   }
 }
 
@@ -320,7 +395,8 @@ __global__ void __launch_bounds__(256) dx_finish_kernel(const float *__restrict_
 cudaError_t launch_transpose_bf16(const void *in, void *out, int R, int C, int64_t ld_in,
                                   int64_t ld_out, int batch, int64_t bstride_in,
                                   int64_t bstride_out, int col_off, cudaStream_t s) {
-  dim3 grid((unsigned)((R + 31) / 32), (unsigned)((C + 31) / 32), (unsigned)batch), block(32, 8);
+  dim3 grid((unsigned)((R + kTT - 1) / kTT), (unsigned)((C + kTT - 1) / kTT), (unsigned)batch),
+      block(256);
   return launch_kernel(transpose_bf16_kernel, grid, block, 0, s, static_cast<const uint16_t *>(in),
                        static_cast<uint16_t *>(out), R, C, ld_in, ld_out, bstride_in, bstride_out,
                        col_off);
@@ -345,7 +421,7 @@ cudaError_t launch_transpose_segments(const void *src, int64_t ld, const int32_t
                                       int E, int G, int C, int64_t kp_max, void *out, uint32_t *err,
                                       cudaStream_t s) {
   SegSrc S_{static_cast<const __nv_bfloat16 *>(src), ld, map, scale, shared_base, shared_stride};
-  dim3 grid((unsigned)(kp_max / 32), (unsigned)((C + 31) / 32)), block(32, 8);
+  dim3 grid((unsigned)(kp_max / kTT), (unsigned)((C + kTT - 1) / kTT)), block(256);
   return launch_kernel(transpose_segments_kernel, grid, block, 0, s, S_, offsets, kseg, E, G, C,
                        kp_max, static_cast<__nv_bfloat16 *>(out), err, src_rows, shared_len);
 }

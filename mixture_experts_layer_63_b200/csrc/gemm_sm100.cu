@@ -97,6 +97,9 @@ struct Params {
   int64_t src_rows;
   const void *aux;          // kEpiDAct*: bf16 pre-activations [row][aux_ld]
   int64_t aux_ld;
+  int b_mn;                 // B stored [K][N] (N contiguous) instead of [N][K]
+  int b_kb_split;           //   k-blocks read from map_b, the rest from map_b3
+  int64_t b_krows;          //   K rows per group in B's row dimension
   int kgroup;               // K-grouped mode (weight gradients), see GroupedGemm
   int M;
   const int32_t *kseg;
@@ -215,6 +218,21 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
   d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Shared-memory descriptor of an MN-major operand (B stored [K][N]) written
+// by TMA boxes of 64 N x 64 K with the 128-byte swizzle: each 128-byte row
+// holds 64 consecutive N values of one K index; 8-row atoms 1024 bytes apart
+// along K (stride byte offset), boxes 8192 bytes apart along N (leading byte
+// offset); version 1, swizzle mode 2.  A K step of 16 moves 2048 bytes.
+__device__ __forceinline__ uint64_t mn128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(8192 >> 4) << 16;
   d |= (uint64_t)(1024 >> 4) << 32;
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
@@ -955,7 +973,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         if (a_by_tma) tma_load_2d(sa, ma, &full_bar[stage], kx + kb * BK, (int)a_row);
-        if (swiglu_b(EPI)) {
+        if (P.b_mn) {
+          // B as [K][N]: bn/64 boxes of 64 N x 64 K, 8 KB apart
+          const bool first = kb < P.b_kb_split;
+          const int y = (int)(tl.g * P.b_krows) + (first ? kb : kb - P.b_kb_split) * BK;
+          for (int j = 0; j < P.bn / 64; ++j)
+            tma_load_2d(sb + j * 8192, first ? &map_b : &map_b3, &full_bar[stage],
+                        tl.n * P.bnh + j * 64, y);
+        } else if (swiglu_b(EPI)) {
           tma_load_2d(sb, &map_b, &full_bar[stage], kx + kb * BK, b_row);
           tma_load_2d(sb + (b_bytes >> 1), &map_b3, &full_bar[stage], kx + kb * BK, b_row);
         } else {
@@ -971,7 +996,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------- MMA issuer -------------------------------
-    const uint32_t idesc = idesc_bf16(BM, P.bn);
+    const uint32_t idesc = idesc_bf16(BM, P.bn) | (P.b_mn ? (1u << 16) : 0u);   // bit 16: B MN-major
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -993,8 +1018,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t b_addr = a_addr + kABytes;
 #pragma unroll
         for (int k = 0; k < BK / kUmmaK; ++k) {
-          umma_bf16(d_tmem, sw128_desc(a_addr + k * kUmmaK * 2), sw128_desc(b_addr + k * kUmmaK * 2),
-                    idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          const uint64_t bdesc = P.b_mn ? mn128_desc(b_addr + k * 2048) : sw128_desc(b_addr + k * kUmmaK * 2);
+          umma_bf16(d_tmem, sw128_desc(a_addr + k * kUmmaK * 2), bdesc, idesc,
+                    (kb > kb0 || k > 0) ? 1u : 0u);
         }
         umma_commit(&empty_bar[stage]);
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -1250,7 +1276,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         }
         if (a_by_tma) tma_load_2d_pair(sa, ma, fb, kb * BK, (int)a_row);
-        tma_load_2d_pair(sb, mb, fb, kb * BK, b_row);
+        if (P.b_mn) {
+          // this CTA's 128 N columns of B stored [K][N]: two boxes of 64 N x 64 K
+          const bool first = kb < P.b_kb_split;
+          const int y = (int)(tl.g * P.b_krows) + (first ? kb : kb - P.b_kb_split) * BK;
+          for (int j = 0; j < P.bn / 128; ++j)
+            tma_load_2d_pair(sb + j * 8192, first ? &map_b : &map_b3, fb,
+                             tl.n * P.bnh + (int)rank * (P.bn / 2) + j * 64, y);
+        } else {
+          tma_load_2d_pair(sb, mb, fb, kb * BK, b_row);
+        }
         if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
       }
     }
@@ -1260,7 +1295,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------ MMA issuer (even CTA only) ------------------------
-    const uint32_t idesc = idesc_bf16(PM, P.bn);
+    const uint32_t idesc = idesc_bf16(PM, P.bn) | (P.b_mn ? (1u << 16) : 0u);   // bit 16: B MN-major
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -1277,8 +1312,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t b_addr = a_addr + kABytes;
 #pragma unroll
         for (int k = 0; k < BK / kUmmaK; ++k) {
-          umma_bf16_pair(d_tmem, sw128_desc(a_addr + k * kUmmaK * 2),
-                         sw128_desc(b_addr + k * kUmmaK * 2), idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          const uint64_t bdesc = P.b_mn ? mn128_desc(b_addr + k * 2048) : sw128_desc(b_addr + k * kUmmaK * 2);
+          umma_bf16_pair(d_tmem, sw128_desc(a_addr + k * kUmmaK * 2), bdesc, idesc,
+                         (kb > kb0 || k > 0) ? 1u : 0u);
         }
         umma_commit_pair_both(&empty_bar[stage]);
         if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
@@ -1498,6 +1534,9 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   P.bias = g.bias;
   P.ksplit = std::max(1, g.ksplit);
   P.split_stride = g.split_stride;
+  P.b_mn = g.b_mn;
+  P.b_kb_split = g.b_mn ? (g.b_kb_split > 0 ? g.b_kb_split : g.K / BK) : 0;
+  P.b_krows = g.b_krows;
   P.kgroup = g.kgroup;
   P.M = g.M;
   P.kseg = g.kseg;
@@ -1521,6 +1560,8 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   if (g.ksplit > 1 && (g.epi != kEpiStoreF32 || g.n_routed != 0)) return cudaErrorInvalidValue;
   if ((g.epi == kEpiDActRelu || g.epi == kEpiDActSwiglu) && (!g.aux || !g.row_gate))
     return cudaErrorInvalidValue;
+  if (g.b_mn && (swiglu_b(g.epi) || g.kgroup || g.b_krows <= 0 || P.bn != 256))
+    return cudaErrorInvalidValue;
   if (g.kgroup && (g.epi != kEpiStoreF32 || g.n_routed != 0 || !g.kseg || g.M <= 0 ||
                    (g.out2 && (g.split_m <= 0 || g.split_m >= g.M))))
     return cudaErrorInvalidValue;
@@ -1538,9 +1579,16 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   if (!make_map(&mas, g.a_static && !g.kgroup ? g.a_static : g.a, (uint64_t)g.K,
                 (uint64_t)(g.a_static && !g.kgroup ? g.a_static_rows : a_outer), BM))
     return cudaErrorInvalidValue;
-  if (!make_map(&mb, g.b, (uint64_t)g.K, b_outer, box_b)) return cudaErrorInvalidValue;
-  if (!make_map(&mb3, g.b3 ? g.b3 : g.b, (uint64_t)g.K, b_outer, box_b))
-    return cudaErrorInvalidValue;
+  if (g.b_mn) {
+    // B stored [K][N]: rows of N values, boxes of 64 N x 64 K
+    if (!make_map(&mb, g.b, (uint64_t)g.N, (uint64_t)g.b_rows, 64)) return cudaErrorInvalidValue;
+    if (!make_map(&mb3, g.b3 ? g.b3 : g.b, (uint64_t)g.N, (uint64_t)g.b_rows, 64))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_map(&mb, g.b, (uint64_t)g.K, b_outer, box_b)) return cudaErrorInvalidValue;
+    if (!make_map(&mb3, g.b3 ? g.b3 : g.b, (uint64_t)g.K, b_outer, box_b))
+      return cudaErrorInvalidValue;
+  }
 
   // grid: one CTA per SM, fewer when there are fewer tiles
   const int64_t mt_routed = (g.max_routed_rows + BM - 1) / BM + g.n_routed;

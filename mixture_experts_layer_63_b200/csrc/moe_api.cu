@@ -265,7 +265,7 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
 static int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 struct BwLayout {
-  size_t w2t, w1t, dy_perm, au, dau, dx_rows, kseg, kseg_r, dyT, hT, dauT, xT, dgate, dl, dl_pad, dlT,
+  size_t dy_perm, au, dau, dx_rows, kseg, kseg_r, dyT, hT, dauT, xT, dgate, dl, dl_pad, dlT,
       xTr, wrT, dx_router, total;
   int64_t kp_max, Ep, Tp;
   int fw;
@@ -285,8 +285,6 @@ static BwLayout make_bw_layout(const moe_config *c, const WsLayout &L) {
     o = align256(o + bytes);
     return at;
   };
-  B.w2t = take((size_t)G * f * d * 2);
-  B.w1t = take((size_t)G * d * B.fw * 2);
   B.dy_perm = take((size_t)L.rows_cap * d * 2);
   B.au = take((size_t)L.rows_total * B.fw * 2);
   B.dau = take((size_t)L.rows_total * B.fw * 2);
@@ -329,7 +327,7 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
   const void *h = ws + L.h;
   const void *y_rows = ws + L.y_rows;
   const bool fused_gather = c->dtype == MOE_BF16 && MOE_FUSED_GATHER;
-  void *w2t = bw + B.w2t, *w1t = bw + B.w1t, *dy_perm = bw + B.dy_perm;
+  void *dy_perm = bw + B.dy_perm;
   void *au = bw + B.au, *dau = bw + B.dau;
   float *dx_rows = reinterpret_cast<float *>(bw + B.dx_rows);
   int32_t *kseg = reinterpret_cast<int32_t *>(bw + B.kseg);
@@ -343,11 +341,6 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
     e = (x_);                  \
     if (e != cudaSuccess) return e; \
   } while (0)
-
-  // 1. transposed weights: W2^T [G][f][d]; [W1 | W3]^T [G][d][fw]
-  MOE_TRY(launch_transpose_bf16(w2, w2t, (int)d, (int)f, f, d, G, d * f, f * d, 0, s));
-  MOE_TRY(launch_transpose_bf16(w1, w1t, (int)f, (int)d, d, B.fw, G, f * d, d * B.fw, 0, s));
-  if (swiglu) MOE_TRY(launch_transpose_bf16(w3, w1t, (int)f, (int)d, d, B.fw, G, f * d, d * B.fw, (int)f, s));
 
   // 2. pre-activations recomputed: A (| U) [rows_total][fw]
   GroupedGemm up{};
@@ -388,8 +381,10 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
   dh.a_rows = L.rows_cap;
   dh.a_static = dy;
   dh.a_static_rows = T;
-  dh.b = w2t;
-  dh.b_rows = (int64_t)G * f;
+  dh.b = w2;                       // W2 [G][d][f] read as [K = d][N = f]
+  dh.b_mn = 1;
+  dh.b_krows = d;
+  dh.b_rows = (int64_t)G * d;
   dh.offsets = offsets;
   dh.n_routed = E;
   dh.n_static = S;
@@ -405,7 +400,7 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
   dh.err = err;
   MOE_TRY(launch_grouped_gemm(dh, s));
 
-  // 5. dX rows = [dA | dU] . [W1 | W3]   (fp32 rows)
+  // 5. dX rows = [dA | dU] . [W1 ; W3]   (fp32 rows)
   GroupedGemm dxg{};
   dxg.epi = kEpiStoreF32;
   dxg.K = B.fw;
@@ -416,8 +411,12 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
   dxg.a_static_rows = L.rows_total;
   dxg.a_static_base = L.rows_cap;
   dxg.a_static_stride = T;
-  dxg.b = w1t;
-  dxg.b_rows = (int64_t)G * d;
+  dxg.b = w1;                      // W1 (| W3) [G][f][d] read as [K = f (+ f)][N = d]
+  dxg.b3 = swiglu ? w3 : nullptr;
+  dxg.b_mn = 1;
+  dxg.b_krows = f;
+  dxg.b_kb_split = (int)(f / 64);
+  dxg.b_rows = (int64_t)G * f;
   dxg.offsets = offsets;
   dxg.n_routed = E;
   dxg.n_static = S;

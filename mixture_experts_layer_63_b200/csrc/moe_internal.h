@@ -178,6 +178,12 @@ struct GroupedGemm {
   const int32_t *gather_rows;  // non-null: routed A row r is gather_src[gather_rows[r]]
   const void *gather_src;      //   (the row gather done inside the GEMM; bf16 [src_rows, K])
   int64_t src_rows;
+  // B stored [K][N] per group (N contiguous; the weights as they are, read
+  // MN-major by the tensor cores): group g's K rows start at row g * b_krows
+  // of b (k-blocks < b_kb_split) or of b3 (the rest, from k-block 0 of b3)
+  int b_mn;
+  int b_kb_split;
+  int64_t b_krows;
   const void *aux;          // kEpiDAct*: bf16 pre-activations, ld aux_ld
   int64_t aux_ld;
   // K-grouped mode (weight gradients): group g computes out_g[M, N] =
