@@ -412,35 +412,52 @@ def run_ours(args, w) -> None:
     tr = NCU_TRAFFIC.get(w.name)
     traffic = tr["bytes"] if tr and tr.get("src") == h else None
 
-    # end to end through the public layer object, host buffers
+    # end to end through the public layer object, host buffers: every step
+    # copies its batch of x from pinned host memory and its y back; the
+    # copies of neighbouring steps overlap the forward (api.HostPipeline); L2
+    # is flushed on the compute stream before every forward, inside the timed
+    # region
     layer = api.MoELayer(cfg, inp.w_router, inp.w1, inp.w2, inp.w3, inp.bias,
                          route_state=inp.route_state)
-    x_host = inp.x.cpu().pin_memory()
-    y_host = torch.empty_like(x_host).pin_memory()
+    x_host = [inp.x.cpu().pin_memory() for _ in range(2)]
+    y_host = [torch.empty_like(x_host[0]).pin_memory() for _ in range(2)]
     x_dev = torch.empty_like(inp.x)
     y_dev = torch.empty_like(inp.x)
-    for _ in range(args.warmup):
-        flush.zero_()
-        x_dev.copy_(x_host, non_blocking=True)
-        layer(x_dev, out=y_dev)
-        y_host.copy_(y_dev, non_blocking=True)
-    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    pipe = api.HostPipeline(layer, before_forward=flush.zero_)
+    for i in range(args.warmup):
+        pipe.submit(x_host[i & 1], y_host[i & 1])
+    pipe.synchronize()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(pipe.s_in)
     for i in range(args.steps):
-        flush.zero_()
-        e2e_ev[i][0].record(stream)
-        x_dev.copy_(x_host, non_blocking=True)
-        layer(x_dev, out=y_dev)
-        y_host.copy_(y_dev, non_blocking=True)
-        e2e_ev[i][1].record(stream)
-    torch.cuda.synchronize()
+        pipe.submit(x_host[i & 1], y_host[i & 1])
+    pipe.s_out.wait_stream(pipe.s_in)
+    pipe.s_out.wait_stream(pipe.s_comp)
+    e1.record(pipe.s_out)
+    pipe.synchronize()
     api.moe_check_device_errors(layer.ws)
-    e2e_ms = replicas.max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), dist, device="cuda")
+    e2e_ms = replicas.max_over_ranks(e0.elapsed_time(e1), dist, device="cuda")
     if dist:
         dist.barrier()
     e2e_value = replicas.throughput(world, w.T, args.steps, e2e_ms)
+    # the same steps one after the other (no overlap), for reference
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    seq_ms = 0.0
+    for i in range(args.steps):
+        flush.zero_()
+        s0.record(stream)
+        x_dev.copy_(x_host[i & 1], non_blocking=True)
+        layer(x_dev, out=y_dev)
+        y_host[i & 1].copy_(y_dev, non_blocking=True)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        seq_ms += s0.elapsed_time(s1)
+    e2e_seq = replicas.throughput(world, w.T, args.steps,
+                                  replicas.max_over_ranks(seq_ms, dist, device="cuda"))
 
     # training: forward + backward (moe_backward) per step, separate steps,
     # not part of `value`; every rank takes the same steps
@@ -509,8 +526,10 @@ def run_ours(args, w) -> None:
                               "hbm_peak": hbm},
             "rows": {"routed_kept": R, "shared": w.S * w.T, "capacity_rows": sizes.rows_cap},
             "e2e": {"value": e2e_value, "unit": "tokens/s",
-                    "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
-                    "d2h_bytes_per_step": int(y_host.numel() * y_host.element_size())},
+                    "h2d_bytes_per_step": int(x_host[0].numel() * x_host[0].element_size()),
+                    "d2h_bytes_per_step": int(y_host[0].numel() * y_host[0].element_size()),
+                    "sequential_value": e2e_seq,
+                    "note": "api.HostPipeline: each step's host copies overlap its neighbours' forwards"},
             "gpu_launches": launches_per_step(w) * args.steps,
             "clocks": clk,
             "cpu_baseline": cpu,

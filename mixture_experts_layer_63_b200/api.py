@@ -367,6 +367,63 @@ class MoELayer:
         moe_route_bias_update(self.cfg, self.counts, self.route_state, gamma, stream)
 
 
+class HostPipeline:
+    """Serving from host memory: batches of T tokens in pinned host buffers go
+    through ``layer`` and their outputs come back to pinned host buffers.  The
+    host-to-device copy of a batch and the device-to-host copy of the one
+    before it overlap the forward of the batch in between (three streams, two
+    device staging slots, events between them); every batch's copies and
+    forward still happen, in order.
+
+        pipe = HostPipeline(layer)
+        for x_h, y_h in batches:          # pinned [T, d] tensors
+            pipe.submit(x_h, y_h)
+        pipe.synchronize()                # every y_h is now filled
+    """
+
+    def __init__(self, layer: MoELayer, before_forward=None):
+        self.layer = layer
+        dev = layer.w1.device
+        cfg = layer.cfg
+        dt = torch.float32 if cfg.dtype == MOE_F32 else torch.bfloat16
+        self.x_dev = [torch.empty(cfg.T, cfg.d_model, dtype=dt, device=dev) for _ in range(2)]
+        self.y_dev = [torch.empty(cfg.T, cfg.d_model, dtype=dt, device=dev) for _ in range(2)]
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_comp = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        mk = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+        self.in_done, self.comp_done, self.out_done = mk(), mk(), mk()
+        self.before_forward = before_forward     # optional callable, run on the compute stream
+        self.i = 0
+
+    def submit(self, x_host: torch.Tensor, y_host: torch.Tensor) -> torch.cuda.Event:
+        """Queue one batch; returns the event recorded once y_host is filled."""
+        k = self.i & 1
+        if self.i >= 2:                      # slot k last used two batches ago
+            self.s_in.wait_event(self.comp_done[k])
+        with torch.cuda.stream(self.s_in):
+            self.x_dev[k].copy_(x_host, non_blocking=True)
+            self.in_done[k].record(self.s_in)
+        self.s_comp.wait_event(self.in_done[k])
+        if self.i >= 2:
+            self.s_comp.wait_event(self.out_done[k])
+        with torch.cuda.stream(self.s_comp):
+            if self.before_forward is not None:
+                self.before_forward()
+            self.layer(self.x_dev[k], out=self.y_dev[k], stream=self.s_comp)
+            self.comp_done[k].record(self.s_comp)
+        self.s_out.wait_event(self.comp_done[k])
+        with torch.cuda.stream(self.s_out):
+            y_host.copy_(self.y_dev[k], non_blocking=True)
+            self.out_done[k].record(self.s_out)
+        self.i += 1
+        return self.out_done[k]
+
+    def synchronize(self):
+        for st in (self.s_in, self.s_comp, self.s_out):
+            st.synchronize()
+
+
 # ---------------------------------------------------------------------------
 # moe_permute without a workspace (callers that cannot allocate device memory)
 # ---------------------------------------------------------------------------
