@@ -43,8 +43,8 @@ DEFAULT_WORKLOAD = "gshard"
 # profiles/, with the sha256 (first 16 hex digits) of the kernel source they
 # were taken at; a value is reported only while the source is unchanged.
 NCU_TRAFFIC: dict[str, dict] = {
-    # profiles/gemm_gshard_ncu.md: up 151.0 + 39.2 MB, down 207.6 + 19.5 MB
-    "gshard": {"bytes": 417_320_704, "src": "3c68e297a84446e9"},
+    # profiles/gemm_gshard_ncu.md: up 151.08 + 38.64 MB, down 207.60 + 11.16 MB
+    "gshard": {"bytes": 408_476_160, "src": "96baee379a04fed3"},
 }
 
 
