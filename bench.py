@@ -79,27 +79,6 @@ def _src_hash(name: str) -> str:
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
 
 
-def launches_per_step(w) -> int:
-    """Kernels libmoe launches for one moe_forward of this workload."""
-    # fp32 layers: the gate kernel computes the logits itself for E <= 32 when
-    # W_r (fp32) and the partial logits of 32 slices x 32 tokens fit 200 KB of
-    # shared memory; bf16 layers run the tcgen05 router GEMM first
-    fused_router = (w.dtype == "f32" and w.E <= 32
-                    and w.E * w.d_model * 4 + 32 * 32 * (w.E + 1) * 4 <= 200 * 1024)
-    n = 1 if fused_router else 2              # router GEMM (or the router inside the gate) + gate
-    if w.mode == "ec":
-        n += 2                                # transpose, expert-choice select
-    else:
-        n += 2                                # scan, rank/scatter
-        if w.capacity_factor <= 0 and w.keep_den > 0:
-            n += 1                            # per-expert affinity select
-    if w.dtype == "f32":
-        n += 1                                # row gather (bf16: inside the up-projection GEMM)
-    n += 2                                    # up- and down-projection GEMMs
-    n += 1                                    # combine
-    return n
-
-
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -364,11 +343,13 @@ def run_ours(args, w) -> None:
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
+    launches0 = api.kernel_launches()
     for i in range(args.steps):
         flush.zero_()
         evs[i][0].record(stream)
         step([None, None, evs[i][1], evs[i][2], None])
         evs[i][3].record(stream)
+    launches = api.kernel_launches() - launches0        # libmoe kernels in the timed region
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -530,7 +511,7 @@ def run_ours(args, w) -> None:
                     "d2h_bytes_per_step": int(y_host[0].numel() * y_host[0].element_size()),
                     "sequential_value": e2e_seq,
                     "note": "api.HostPipeline: each step's host copies overlap its neighbours' forwards"},
-            "gpu_launches": launches_per_step(w) * args.steps,
+            "gpu_launches": launches,
             "clocks": clk,
             "cpu_baseline": cpu,
             "backward": backward,

@@ -302,6 +302,13 @@ MOE_API moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t st
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(moe_status s);
 
+/* Number of kernels the library has launched since it was loaded, counted
+ * over all threads and devices at each successful launch (host-side
+ * counter; touches no CUDA state, so it works without a GPU).  The
+ * difference across a region of calls is the number of kernels those calls
+ * launched. */
+MOE_API uint64_t moe_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,7 +31,8 @@ ROUTE_RULES = {"softmax": MOE_ROUTE_SOFTMAX, "bias": MOE_ROUTE_BIAS, "load": MOE
 EXPORTS = ("moe_query_sizes", "moe_route", "moe_gate", "moe_permute", "moe_expert_ffn",
            "moe_combine", "moe_forward", "moe_check_device_errors", "moe_workspace_init",
            "moe_status_string", "moe_permute_noalloc", "moe_forward_timed",
-           "moe_route_bias_update", "moe_query_backward_size", "moe_backward")
+           "moe_route_bias_update", "moe_query_backward_size", "moe_backward",
+           "moe_kernel_launches")
 
 
 class MoeError(RuntimeError):
@@ -93,12 +94,19 @@ def lib() -> ctypes.CDLL:
             f.restype = ctypes.c_int
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_kernel_launches.argtypes = []
+        L.moe_kernel_launches.restype = ctypes.c_uint64
         _lib = L
     return _lib
 
 
 def status_string(status: int) -> str:
     return lib().moe_status_string(status).decode()
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched since it was loaded (host counter)."""
+    return int(lib().moe_kernel_launches())
 
 
 def _check(fn: str, status: int) -> None:

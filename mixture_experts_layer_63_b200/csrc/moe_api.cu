@@ -2,11 +2,15 @@
 // workspace layout and the launch sequence of each entry point.  All
 // arithmetic of the layer runs in the kernels of the other files.
 #include <algorithm>
+#include <atomic>
 
 #include "device_common.cuh"
 #include "moe_internal.h"
 
 namespace moe {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -780,5 +784,7 @@ const char *moe_status_string(moe_status s) {
     default: return "unknown status";
   }
 }
+
+uint64_t moe_kernel_launches(void) { return moe::g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

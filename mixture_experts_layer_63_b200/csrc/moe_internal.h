@@ -17,6 +17,9 @@ namespace moe {
 #ifndef MOE_PDL
 #define MOE_PDL 1
 #endif
+// Kernels this library has launched, all threads together (moe_kernel_launches).
+void count_launch();
+
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                                  cudaStream_t s, Args... args) {
@@ -30,7 +33,9 @@ inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = MOE_PDL ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  if (e == cudaSuccess) count_launch();
+  return e;
 }
 
 // Tokens per unit of the token-choice counting sort (one warp per unit).

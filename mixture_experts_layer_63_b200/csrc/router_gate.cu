@@ -18,8 +18,9 @@
 // permutation's scan consumes (see permute.cu).
 //
 // Router logits: for few experts (E <= 32, W_r small enough for shared
-// memory) the warp computes them itself from x and W_r in fp32 (fused
-// router); otherwise they come from the tcgen05 GEMM in gemm_sm100.cu.
+// memory) the warp computes them itself from x and W_r with fp32
+// accumulation (fused router: x is read once, no logits round trip);
+// otherwise they come from the tcgen05 GEMM in gemm_sm100.cu.
 #include <math.h>
 
 #include "device_common.cuh"
@@ -68,6 +69,32 @@ __device__ __forceinline__ float max_warp(float v) {
   return v;
 }
 
+// One halving step of a warp reduction of N values a lane: the lanes with
+// bit `o` set keep the upper N/2 values, the others the lower N/2, each
+// adding its partner's copy of the half it keeps.
+template <int N, int EMAX>
+__device__ __forceinline__ void halve(float (&a)[EMAX], int o, int lane) {
+  const bool upper = (lane & o) != 0;
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    const float send = upper ? a[i] : a[N / 2 + i];
+    const float keep = upper ? a[N / 2 + i] : a[i];
+    a[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+  }
+}
+
+// 16-byte chunk of x or W_r widened to fp32
+template <bool BF16>
+__device__ __forceinline__ void widen_chunk(const uint4 v, float (&f)[BF16 ? 8 : 4]) {
+  if constexpr (BF16) {
+    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z); f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+  } else {
+    f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+  }
+}
+
 // NV = slots per lane (ceil(E/32)); FUSED: compute logits from x and W_r
 // (requires E <= EMAX <= 32, so NV == 1); BF16: input element type of the
 // fused router.
@@ -80,94 +107,85 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_gate_kernel(const GatePa
   pdl_trigger();
   int *s_hist = reinterpret_cast<int *>(smem);                    // [k][E]
   const int hist_ints = P.hist ? k * E : 0;
-  // fused router: W_r widened to fp32 [E][d] and the partial logits of the
-  // 32 slices of the model dimension [32 slices][32 tokens][E + 1 (pad)]
-  constexpr int EPV = BF16 ? 8 : 4;                      // x elements per 16-byte chunk
+  // fused router: W_r as stored, [E][d] in 16-byte chunks
+  constexpr int EPV = BF16 ? 8 : 4;                      // elements per 16-byte chunk
   const int nchunk = P.d / EPV;
-  const int pstride = E + 1;                             // odd: conflict-free rows
-  float *s_w = reinterpret_cast<float *>(smem + ((hist_ints * 4 + 15) & ~15));
-  float *s_part = s_w + (FUSED ? (size_t)E * P.d : 0);
+  uint4 *s_w = reinterpret_cast<uint4 *>(smem + ((hist_ints * 4 + 15) & ~15));
   // per-warp buffer of the exponentials, summed in order by lane 0
-  float *s_ex = s_part + (FUSED ? (size_t)32 * kTokWarps * pstride : 0) + warp * E;
-
-  for (int i = threadIdx.x; i < hist_ints; i += blockDim.x) s_hist[i] = 0;
-  if (FUSED) {
-    const int nq = E * P.d / 4;                          // 4 consecutive elements at a time
-    for (int q = threadIdx.x; q < nq; q += blockDim.x) {
-      float4 f;
-      if (BF16) {
-        const uint2 w = reinterpret_cast<const uint2 *>(P.w_router)[q];
-        f = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
-      } else {
-        f = reinterpret_cast<const float4 *>(P.w_router)[q];
-      }
-      reinterpret_cast<float4 *>(s_w)[q] = f;
-    }
-  }
-  __syncthreads();
+  float *s_ex = reinterpret_cast<float *>(s_w + (FUSED ? (size_t)E * nchunk : 0)) + warp * E;
 
   const int64_t t = (int64_t)blockIdx.x * kTokWarps + warp;
   const bool live = t < P.T;
 
+  // fused router: this warp's token, lanes split the model dimension (lane l
+  // takes chunks l, l + 32, ...); the first NB chunks a lane are in flight
+  // while the block stages W_r
+  constexpr int NB = EMAX >= 32 ? 2 : 4;
+  const uint4 *xr = reinterpret_cast<const uint4 *>(P.x) + (live ? t : 0) * nchunk;
+  uint4 xb[NB];
+  if (FUSED) {
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+      const int c = lane + 32 * i;
+      xb[i] = (live && c < nchunk) ? xr[c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+
+  for (int i = threadIdx.x; i < hist_ints; i += blockDim.x) s_hist[i] = 0;
+  if (FUSED) {
+    const uint4 *wg = reinterpret_cast<const uint4 *>(P.w_router);
+#pragma unroll 4
+    for (int q = threadIdx.x; q < E * nchunk; q += blockDim.x) s_w[q] = wg[q];
+  }
+  __syncthreads();
+
   // ---- logits of this token: lane l holds experts l + 32 j ----------------
   float l[NV];
   if (FUSED) {
-    // slice `warp` of the model dimension for token t0 + lane: x chunks from
-    // global memory into registers, W_r chunks read by all lanes at once
-    // (shared-memory broadcast); per expert an fp32 chain in element order
-    // (experts in passes of up to 16, to stay within 64 registers a thread)
-    constexpr int EB = EMAX < 16 ? EMAX : 16;
-    for (int e0 = 0; e0 < E; e0 += EB) {
-      const int64_t tt = (int64_t)blockIdx.x * kTokWarps + lane;
-      const int c0 = warp * nchunk / 32, c1 = (warp + 1) * nchunk / 32;
-      float acc[EB];
+    // per expert an fp32 sum over this lane's chunks (chunk order, element
+    // order inside a chunk), then a halving butterfly over the 32 lanes
+    float acc[EMAX];
 #pragma unroll
-      for (int e = 0; e < EB; ++e) acc[e] = 0.f;
-      if (tt < P.T) {
-        const uint4 *xr = reinterpret_cast<const uint4 *>(P.x) + tt * nchunk;
-        for (int c = c0; c < c1; ++c) {
-          const uint4 xv = xr[c];
-          float xf[EPV];
-          if (BF16) {
-            xf[0] = bf16_lo(xv.x); xf[1] = bf16_hi(xv.x); xf[2 % EPV] = bf16_lo(xv.y); xf[3 % EPV] = bf16_hi(xv.y);
-            xf[4 % EPV] = bf16_lo(xv.z); xf[5 % EPV] = bf16_hi(xv.z); xf[6 % EPV] = bf16_lo(xv.w); xf[7 % EPV] = bf16_hi(xv.w);
-          } else {
-            xf[0] = __uint_as_float(xv.x); xf[1] = __uint_as_float(xv.y);
-            xf[2 % EPV] = __uint_as_float(xv.z); xf[3 % EPV] = __uint_as_float(xv.w);
-          }
-          const float4 *wc = reinterpret_cast<const float4 *>(s_w + (size_t)e0 * P.d + (size_t)c * EPV);
+    for (int e = 0; e < EMAX; ++e) acc[e] = 0.f;
+    for (int c0 = 0; c0 < nchunk; c0 += 32 * NB) {
+      if (c0 > 0) {
 #pragma unroll
-          for (int e = 0; e < EB; ++e) {
-            if (e0 + e < E) {
-              float a = acc[e];
+        for (int i = 0; i < NB; ++i) {
+          const int c = c0 + lane + 32 * i;
+          xb[i] = (live && c < nchunk) ? xr[c] : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
 #pragma unroll
-              for (int h = 0; h < EPV / 4; ++h) {
-                const float4 w = wc[(size_t)e * (P.d / 4) + h];
-                a = fmaf(xf[4 * h + 0], w.x, a);
-                a = fmaf(xf[4 * h + 1], w.y, a);
-                a = fmaf(xf[4 * h + 2], w.z, a);
-                a = fmaf(xf[4 * h + 3], w.w, a);
-              }
-              acc[e] = a;
-            }
+      for (int i = 0; i < NB; ++i) {
+        const int c = c0 + lane + 32 * i;
+        if (c >= nchunk) break;
+        float xf[EPV];
+        widen_chunk<BF16>(xb[i], xf);
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) {
+          if (e < E) {
+            float wf[EPV];
+            widen_chunk<BF16>(s_w[(size_t)e * nchunk + c], wf);
+            float a = acc[e];
+#pragma unroll
+            for (int h = 0; h < EPV; ++h) a = fmaf(xf[h], wf[h], a);
+            acc[e] = a;
           }
         }
       }
-      float *pp = s_part + ((size_t)warp * kTokWarps + lane) * pstride + e0;
+    }
+    // EMAX values -> one: lane l then holds expert l / (32 / EMAX)
+    halve<EMAX, EMAX>(acc, 16, lane);
+    if constexpr (EMAX >= 4) halve<EMAX / 2, EMAX>(acc, 8, lane);
+    if constexpr (EMAX >= 8) halve<EMAX / 4, EMAX>(acc, 4, lane);
+    if constexpr (EMAX >= 16) halve<EMAX / 8, EMAX>(acc, 2, lane);
+    if constexpr (EMAX >= 32) halve<EMAX / 16, EMAX>(acc, 1, lane);
+    float v = acc[0];
 #pragma unroll
-      for (int e = 0; e < EB; ++e)
-        if (e0 + e < E) pp[e] = acc[e];
-    }
-    __syncthreads();
-    // token t = this warp's token: the 32 slices summed in order, then the bias
+    for (int o = 16 / EMAX; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    v = __shfl_sync(0xffffffffu, v, (lane * (32 / EMAX)) & 31);
     float mine = -INFINITY;
-    if (lane < E) {
-      const float *pp = s_part + (size_t)warp * pstride + lane;
-      float v = pp[0];
-#pragma unroll 8
-      for (int sl = 1; sl < 32; ++sl) v = __fadd_rn(v, pp[(size_t)sl * kTokWarps * pstride]);
-      mine = P.bias ? __fadd_rn(v, P.bias[lane]) : v;
-    }
+    if (lane < E) mine = P.bias ? __fadd_rn(v, P.bias[lane]) : v;
     l[0] = mine;
     if (live && lane < E) P.logits_out[t * E + lane] = mine;
   } else {
@@ -350,25 +368,23 @@ cudaError_t launch_nv(int NV, const GateParams &P, int blocks, size_t smem, cuda
 
 }  // namespace
 
-#ifndef MOE_FUSED_ROUTER_BF16
-#define MOE_FUSED_ROUTER_BF16 0
-#endif
-
-// shared memory of the fused router: W_r widened to fp32 and the partial
-// logits of 32 slices x 32 tokens
+// shared memory of the fused router: W_r as stored
 static size_t fused_router_smem(const moe_config *c) {
-  return (size_t)c->E * c->d_model * 4 + (size_t)32 * kTokWarps * (c->E + 1) * 4;
+  return (size_t)c->E * c->d_model * (c->dtype == MOE_BF16 ? 2 : 4);
 }
 
-// fp32 layers with few experts (E <= 32) and a W_r that fits shared memory:
-// the gate kernel computes the logits itself on CUDA cores, reading x once.
-// Otherwise the tcgen05 router GEMM (bf16) or a CUDA-core kernel (fp32) runs
-// first.  (For bf16 the fused form measured slower than the router GEMM plus
-// the gate: 21 vs 18 us on the GShard-shaped layer, 78 vs 44 us on the
-// Mixtral-shaped one; MOE_FUSED_ROUTER_BF16=1 builds it.)
+// Few experts (E <= 32) and a W_r that fits shared memory: the gate kernel
+// computes the logits itself on CUDA cores, reading x once; otherwise the
+// tcgen05 router GEMM (bf16) or a CUDA-core kernel (fp32) runs first.  For
+// bf16 the fused form is used up to d = 2048: router + gate 19 vs 24 us on
+// the GShard-shaped layer (d = 1024), but 63 vs 50 us on the Mixtral-shaped
+// one (d = 4096), where each warp's serial walk along a 8 KB row loses to
+// the GEMM.
+constexpr int kFusedRouterMaxDBf16 = 2048;
+
 bool router_is_fused(const moe_config *c) {
-  if (c->dtype == MOE_BF16 && !MOE_FUSED_ROUTER_BF16) return false;
-  return c->E <= 32 && fused_router_smem(c) <= kFusedRouterSmem;
+  if (c->E > 32 || fused_router_smem(c) > kFusedRouterSmem) return false;
+  return c->dtype != MOE_BF16 || c->d_model <= kFusedRouterMaxDBf16;
 }
 
 cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float *logits_out,
@@ -407,7 +423,7 @@ cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float
   smem += (size_t)kTokWarps * c->E * 4;                     // per-warp exponentials
   const int NV = (c->E + 31) / 32;
   if (fused) {
-    smem += fused_router_smem(c);                           // W_r (fp32) + slice partials
+    smem += fused_router_smem(c);                           // W_r as stored
     const bool bf = c->dtype == MOE_BF16;
     auto kern = c->E <= 8    ? (bf ? route_gate_kernel<1, true, true, 8> : route_gate_kernel<1, true, false, 8>)
                 : c->E <= 16 ? (bf ? route_gate_kernel<1, true, true, 16> : route_gate_kernel<1, true, false, 16>)

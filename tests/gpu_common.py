@@ -40,6 +40,10 @@ SMALL = {
     # (256-row tiles); ragged M tails, partial N tiles, shared experts
     "pair_relu_s": replace(WORKLOADS["gshard"], T=2100, E=4, d_model=256, d_ff=320),
     "pair_swiglu_s": replace(WORKLOADS["deepseekmoe_tc"], T=1400, E=8, k=6, d_model=320, d_ff=192),
+    # CTA pairs, ReLU with a shared expert: last M-tiles of 24-31 rows (the
+    # even CTA's rows only) and of 122 rows (both CTAs), the shared expert's
+    # 2150 = 8 * 256 + 102 rows
+    "pair_half_s": replace(WORKLOADS["gshard"], T=2150, E=4, S=1, d_model=256, d_ff=320),
     # routing variants: DeepSeek-V3 bias routing (256 + 1 experts, top-8 of 4
     # groups), load-aware top-k, GShard local groups
     "dsv3_s": replace(WORKLOADS["deepseek_v3"], T=600, d_model=256, d_ff=128),

@@ -64,6 +64,15 @@ def test_struct_layout_matches_the_header(tmp_path):
             assert int(got[f"{cname}.{f}"]) == getattr(st, f).offset, f
 
 
+def test_launch_counter_reads_without_a_gpu(L):
+    n = api.kernel_launches()
+    assert n >= 0
+    # a call that fails host validation launches nothing
+    with pytest.raises(api.MoeError):
+        api.query_sizes(_cfg(T=0))
+    assert api.kernel_launches() == n
+
+
 def test_status_strings(L):
     for s in range(7):
         assert api.status_string(s)

@@ -49,16 +49,18 @@ def _route_gpu(cfg, inp):
 # steps 1-3a
 # ---------------------------------------------------------------------------
 
-# extra routing cases: the fused CUDA-core router (fp32, E <= 32, one and two
-# passes over the experts) and the tcgen05 router GEMM, K whole or split
+# extra routing cases: the fused CUDA-core router (E <= 32 and W_r within
+# 200 KB of shared memory; 8, 16 and 32 accumulators a lane) and the tcgen05
+# router GEMM, K whole or split
 ROUTE_EXTRA = {
-    # fp32, E <= 32: the logits come from the gate kernel's own CUDA-core
-    # router (two passes over the experts for E = 32)
+    # fp32, E <= 32: the logits come from the gate kernel's own CUDA-core router
     "fused_router_f32_s": replace(WORKLOADS["tiny_f32"], T=300, d_model=512),
     "fused_router_e32_f32_s": replace(WORKLOADS["tiny_f32"], T=200, E=32, d_model=256),
-    # bf16: tcgen05 router GEMM, one K part and 16 / 32 experts
-    "router_gemm_s": replace(WORKLOADS["gshard"], T=300),
-    "router_gemm_e32_s": replace(WORKLOADS["gshard"], T=200, E=32, d_model=512),
+    # bf16, E <= 32: the same fused router on bf16 x and W_r
+    "fused_router_bf16_s": replace(WORKLOADS["gshard"], T=300),
+    "fused_router_e32_bf16_s": replace(WORKLOADS["gshard"], T=200, E=32, d_model=512),
+    # bf16, E = 32 with a 256 KB W_r: the tcgen05 router GEMM, one K part
+    "router_gemm_e32_s": replace(WORKLOADS["gshard"], T=200, E=32, d_model=4096),
     # E > 32: the tcgen05 router GEMM with K split over CTAs
     "split_k_s": replace(WORKLOADS["deepseekmoe_tc"], T=300),
     "split_k_groups_s": replace(WORKLOADS["deepseek_v2"], T=200, d_model=1024, keep_num=0, keep_den=0),

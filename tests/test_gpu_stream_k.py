@@ -29,6 +29,8 @@ LONG_K = {
     "pair_relu": replace(SMALL["pair_relu_s"], d_ff=2048),
     # CTA pairs, SwiGLU and shared experts, K = 1024 on the down-projection
     "pair_swiglu": replace(SMALL["pair_swiglu_s"], d_ff=1024),
+    # CTA pairs, short last M-tiles cut into pieces, K = 2048
+    "pair_half": replace(SMALL["pair_half_s"], d_ff=2048),
 }
 
 
