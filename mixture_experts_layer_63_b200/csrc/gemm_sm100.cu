@@ -23,7 +23,8 @@
 //               a finished accumulator to the epilogue
 //   warp 2      TMEM allocation (512 columns = two 256-column accumulators)
 //   warps 4-7   epilogue: tcgen05.ld of its 32 rows, activation / gate /
-//               bias, bf16 pack, masked 16-byte stores (rows beyond the
+//               bias, bf16 pack; bf16 rows leave through a per-warp shared
+//               staging buffer as whole 128-byte lines (rows beyond the
 //               expert's segment are never written)
 // Tiles are ordered group by group, N-tile outer and M-tile inner, so CTAs
 // working at the same time share one expert's weight slice in L2.  Segment
@@ -629,154 +630,79 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16 *src, float (&v
   }
 }
 
+// bf16 outputs leave through a 4 KB staging buffer of the warp in shared
+// memory: each thread writes its row's PIECES 16-byte pieces there (piece c
+// of row r at slot c ^ f(r), which keeps both the writes and the reads below
+// free of bank conflicts), then every store instruction of the warp writes
+// 32 / PIECES whole rows of PIECES * 16 bytes (8 pieces: 128-byte lines).
+// Stored straight from the row-per-thread layout, a warp's 16-byte stores
+// would touch 32 rows each and fill every 32-byte sector in two halves.
+// Row r of the warp (output row row0 + r) is written when bit r of vmask is
+// set.
+constexpr int kStageBytesPerWarp = 32 * 128;
+
+template <int PIECES>
+__device__ __forceinline__ int stage_slot(int r, int c) {
+  return PIECES == 8 ? c ^ (r & 7) : c ^ ((r >> 1) & 3);
+}
+
+template <int PIECES>
+__device__ __forceinline__ void store_rows(uint8_t *stg, const uint32_t (&pk)[PIECES * 4],
+                                           __nv_bfloat16 *out, int64_t ld, int64_t row0, int col,
+                                           uint32_t vmask, int lane) {
+  static_assert(PIECES == 4 || PIECES == 8, "rows of 64 or 128 bytes");
+  constexpr int kRowBytes = PIECES * 16;
+  constexpr int kRowsPerStore = 32 / PIECES;
+  uint4 *mine = reinterpret_cast<uint4 *>(stg + lane * kRowBytes);
+#pragma unroll
+  for (int c = 0; c < PIECES; ++c)
+    mine[stage_slot<PIECES>(lane, c)] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int p = 0; p < PIECES; ++p) {
+    const int r = p * kRowsPerStore + lane / PIECES, c = lane % PIECES;
+    const uint4 w = reinterpret_cast<const uint4 *>(stg + r * kRowBytes)[stage_slot<PIECES>(r, c)];
+    if ((vmask >> r) & 1u) *reinterpret_cast<uint4 *>(out + (row0 + r) * ld + col + c * 8) = w;
+  }
+  __syncwarp();
+}
+
+// 32 fp32 values into 16 bf16x2 words at word offset 16 * H of pk
+template <int H, int N>
+__device__ __forceinline__ void pack_words(uint32_t (&pk)[N], const float (&v)[32]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) pk[16 * H + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+}
+
+// TMEM columns [c, c + 32) of this thread's row as fp32, plus the later
+// stream-K pieces of the tile when F is given
+__device__ __forceinline__ void acc_cols(uint32_t taddr, int c, const Fixup *F, float (&v)[32]) {
+  uint32_t r[32];
+  tmem_ld32(taddr + c, r);
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (F) add_parts(v, *F, c);
+}
+
 // Epilogue of one accumulator: this thread's row (TMEM lane) of the tile,
-// BN columns from TMEM address `taddr`; the later stream-K pieces of the tile
-// added first when F is given; then activation / gate / bias, stores.
+// BN columns from TMEM address `taddr` (SwiGLU forms: gate columns 0-127,
+// up 128-255), output columns from col0 on; the later stream-K pieces of the
+// tile added first when F is given; then activation / gate / bias, stores.
+// The warp's rows are consecutive (lane l: output row out_row = row0 + l);
+// `stg` is the warp's staging buffer.
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, bool valid, bool routed,
-                                              int64_t out_row, int col0, int64_t out_offset = 0,
-                                              const Fixup *F = nullptr) {
-  uint32_t r[32];
+                                              int64_t out_row, int col0, uint8_t *stg, int lane,
+                                              int64_t out_offset = 0, const Fixup *F = nullptr) {
   float v[32];
-  if (EPI == kEpiSwiglu) {
-    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
-#pragma unroll 1
-    for (int c = 0; c < 128 / 32; ++c) {
-      uint32_t u[32];
-      float uf[32];
-      tmem_ld32(taddr + c * 32, r);
-      tmem_ld32(taddr + 128 + c * 32, u);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        v[i] = __uint_as_float(r[i]);
-        uf[i] = __uint_as_float(u[i]);
-      }
-      if (F) {
-        add_parts(v, *F, c * 32);
-        add_parts(uf, *F, 128 + c * 32);
-      }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float g = v[i];
-        v[i] = g / (1.0f + __expf(-g)) * uf[i];
-      }
-      const int col = col0 + c * 32;
-      if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
-    }
-  } else if (EPI == kEpiRelu) {
-    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
-#pragma unroll 1
-    for (int c = 0; c < P.bn / 32; ++c) {
-      tmem_ld32(taddr + c * 32, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-      if (F) add_parts(v, *F, c * 32);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.0f);
-      const int col = col0 + c * 32;
-      if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
-    }
-  } else if (EPI == kEpiScale) {
-    // gated rows in bf16; the combine sums them in fp32 and rounds once
-    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
-    const float scale = (routed && valid) ? P.row_gate[out_row] : 1.0f;
-#pragma unroll 1
-    for (int c = 0; c < P.bn / 32; ++c) {
-      tmem_ld32(taddr + c * 32, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-      if (F) add_parts(v, *F, c * 32);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] *= scale;
-      const int col = col0 + c * 32;
-      if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
-    }
-  } else if (EPI == kEpiPreRelu) {
-    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
-#pragma unroll 1
-    for (int c = 0; c < P.bn / 32; ++c) {
-      tmem_ld32(taddr + c * 32, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-      if (F) add_parts(v, *F, c * 32);
-      const int col = col0 + c * 32;
-      if (valid && col < P.N) store_bf16x32(out + out_row * P.N + col, v);
-    }
-  } else if (EPI == kEpiPreSwiglu) {
-    // a (gate half) at [row][col], u (up half) at [row][N + col]
-    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
-    const int64_t ld = 2 * (int64_t)P.N;
-#pragma unroll 1
-    for (int c = 0; c < 128 / 32; ++c) {
-      uint32_t u[32];
-      float uf[32];
-      tmem_ld32(taddr + c * 32, r);
-      tmem_ld32(taddr + 128 + c * 32, u);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        v[i] = __uint_as_float(r[i]);
-        uf[i] = __uint_as_float(u[i]);
-      }
-      if (F) {
-        add_parts(v, *F, c * 32);
-        add_parts(uf, *F, 128 + c * 32);
-      }
-      const int col = col0 + c * 32;
-      if (valid && col < P.N) {
-        store_bf16x32(out + out_row * ld + col, v);
-        store_bf16x32(out + out_row * ld + P.N + col, uf);
-      }
-    }
-  } else if (EPI == kEpiDActRelu || EPI == kEpiDActSwiglu) {
-    // dh = g * acc, then the activation's backward from the saved a (and u)
-    __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
-    const __nv_bfloat16 *aux = reinterpret_cast<const __nv_bfloat16 *>(P.aux);
-    const int64_t ld = (EPI == kEpiDActSwiglu ? 2 : 1) * (int64_t)P.N;
-    const float scale = (routed && valid) ? P.row_gate[out_row] : 1.0f;
-#pragma unroll 1
-    for (int c = 0; c < P.bn / 32; ++c) {
-      tmem_ld32(taddr + c * 32, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-      if (F) add_parts(v, *F, c * 32);
-      const int col = col0 + c * 32;
-      if (!valid || col >= P.N) continue;
-      float a[32];
-      load_bf16x32(aux + out_row * P.aux_ld + col, a);
-      if (EPI == kEpiDActRelu) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = a[i] > 0.0f ? v[i] * scale : 0.0f;
-        store_bf16x32(out + out_row * ld + col, v);
-      } else {
-        float uu[32], du[32];
-        load_bf16x32(aux + out_row * P.aux_ld + P.N + col, uu);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float dh = v[i] * scale;
-          const float sg = 1.0f / (1.0f + __expf(-a[i]));
-          du[i] = dh * a[i] * sg;
-          v[i] = dh * uu[i] * sg * (1.0f + a[i] * (1.0f - sg));
-        }
-        store_bf16x32(out + out_row * ld + col, v);
-        store_bf16x32(out + out_row * ld + P.N + col, du);
-      }
-    }
-  } else {  // kEpiStoreF32 (a K part when the router is split: no bias, own output)
+  if constexpr (EPI == kEpiStoreF32) {
+    // a K part when the router is split: no bias, own output
     float *out = reinterpret_cast<float *>(P.out) + out_offset;
     const float *bias = P.ksplit > 1 ? nullptr : P.bias;
 #pragma unroll 1
     for (int c = 0; c < P.bn / 32; ++c) {
-      tmem_ld32(taddr + c * 32, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-      if (F) add_parts(v, *F, c * 32);
+      acc_cols(taddr, c * 32, F, v);
       const int col0c = col0 + c * 32;
       if (!valid) continue;
       if (!bias && col0c + 32 <= P.N && (P.N & 3) == 0) {
@@ -790,6 +716,94 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
           if (col < P.N) out[out_row * P.N + col] = bias ? v[i] + bias[col] : v[i];
         }
       }
+    }
+    return;
+  }
+  __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
+  const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+  const int64_t row0 = out_row - lane;
+  if constexpr (EPI == kEpiPreSwiglu || EPI == kEpiDActSwiglu) {
+    // two outputs: [row][col] and [row][N + col], 32 columns at a time
+    const int64_t ld = 2 * (int64_t)P.N;
+    const int ncol = EPI == kEpiPreSwiglu ? 128 : P.bn;
+    const float scale = (EPI == kEpiDActSwiglu && routed && valid) ? P.row_gate[out_row] : 1.0f;
+    const __nv_bfloat16 *aux = reinterpret_cast<const __nv_bfloat16 *>(P.aux);
+#pragma unroll 1
+    for (int c = 0; c < ncol / 32; ++c) {
+      const int col = col0 + c * 32;
+      if (col >= P.N) break;                                    // the same for the whole CTA
+      float w[32];
+      uint32_t pk[16], pk2[16];
+      if constexpr (EPI == kEpiPreSwiglu) {
+        acc_cols(taddr, c * 32, F, v);                          // a
+        acc_cols(taddr, 128 + c * 32, F, w);                    // u
+      } else {
+        // dh = g * acc, then SwiGLU's backward from the saved a and u
+        acc_cols(taddr, c * 32, F, v);
+        float a[32], uu[32];
+        if (valid) {
+          load_bf16x32(aux + out_row * P.aux_ld + col, a);
+          load_bf16x32(aux + out_row * P.aux_ld + P.N + col, uu);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = uu[i] = 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float dh = v[i] * scale;
+          const float sg = 1.0f / (1.0f + __expf(-a[i]));
+          w[i] = dh * a[i] * sg;
+          v[i] = dh * uu[i] * sg * (1.0f + a[i] * (1.0f - sg));
+        }
+      }
+      pack_words<0>(pk, v);
+      pack_words<0>(pk2, w);
+      store_rows<4>(stg, pk, out, ld, row0, col, vmask, lane);
+      store_rows<4>(stg, pk2, out, ld, row0, (int)P.N + col, vmask, lane);
+    }
+  } else {
+    // one output, 64 columns (one 128-byte line a row) at a time
+    const int ncol = EPI == kEpiSwiglu ? 128 : P.bn;
+    const int64_t ld = P.N;
+    const float scale = ((EPI == kEpiScale || EPI == kEpiDActRelu) && routed && valid) ? P.row_gate[out_row] : 1.0f;
+    const __nv_bfloat16 *aux = reinterpret_cast<const __nv_bfloat16 *>(P.aux);
+#pragma unroll 1
+    for (int c2 = 0; c2 < ncol / 64; ++c2) {
+      const int col = col0 + c2 * 64;
+      if (col >= P.N) break;                                    // the same for the whole CTA
+      uint32_t pk[32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int c = 2 * c2 + h;                               // 32-column group of the tile
+        acc_cols(taddr, c * 32, F, v);
+        if constexpr (EPI == kEpiSwiglu) {
+          float uf[32];
+          acc_cols(taddr, 128 + c * 32, F, uf);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = v[i] / (1.0f + __expf(-v[i])) * uf[i];
+        } else if constexpr (EPI == kEpiRelu) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.0f);
+        } else if constexpr (EPI == kEpiScale) {
+          // gated rows in bf16; the combine sums them in fp32 and rounds once
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= scale;
+        } else if constexpr (EPI == kEpiDActRelu) {
+          // dh = g * acc, masked where the saved pre-activation a <= 0
+          float a[32];
+          if (valid) {
+            load_bf16x32(aux + out_row * P.aux_ld + col + h * 32, a);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) a[i] = 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = a[i] > 0.0f ? v[i] * scale : 0.0f;
+        }                                                       // kEpiPreRelu: a as is
+        if (h == 0) pack_words<0>(pk, v);
+        else pack_words<1>(pk, v);
+      }
+      store_rows<8>(stg, pk, out, ld, row0, col, vmask, lane);
     }
   }
 }
@@ -1077,11 +1091,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------- epilogue --------------------------------
     const int ew = warp - 4;                     // TMEM lanes 32*ew .. 32*ew+31
     const int r_cta = ew * 32 + lane;            // row of the tile
+    uint8_t *stg = smem + (size_t)kStages * stage_bytes + (size_t)ew * kStageBytesPerWarp;
     int acc = 0;
     uint32_t acc_phase = 0;
     while (sc.next(tile, kb0, kb1, part)) {
       const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
-      if (!mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err)) break;
+      // (warp-uniform exits: the epilogue's TMEM loads and stores are warp-wide)
+      if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err))) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
       const bool in_tail = sk && tile >= sc.dp_limit;
@@ -1107,11 +1123,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int col0 = tl.n * P.bnh;
         if (in_tail && kb1 < KB) {                              // finalizer of a split tile
           const Fixup F{P.sk_part, &sc, (int)blockIdx.x + 1, sc.contributors_end(tile), 1, 0, r_cta};
-          if (!sk_wait(P, F, &s_abort)) break;
-          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, 0, &F);
+          if (!__all_sync(0xffffffffu, sk_wait(P, F, &s_abort))) break;
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F);
           sk_done(P, F);
         } else {
-          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, (int64_t)part * P.split_stride);
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane,
+                             (int64_t)part * P.split_stride);
         }
       }
       tc_fence_before();
@@ -1375,13 +1392,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // -------------------------------- epilogue --------------------------------
     const int ew = warp - 4;
     const int r_cta = ew * 32 + lane;                 // row within this CTA's half
+    uint8_t *stg = smem + (size_t)kPairStages * stage_bytes + (size_t)ew * kStageBytesPerWarp;
     const uint32_t acce_even0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
     const uint32_t acce_even1 = mapa_shared(smem_u32(&acce_bar[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
     while (sc.next(tile, kb0, kb1, part)) {
       const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
-      if (!mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err)) break;
+      // (warp-uniform exits: the epilogue's TMEM loads and stores are warp-wide)
+      if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err))) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
       const bool in_tail = sk && tile >= sc.dp_limit;
@@ -1397,11 +1416,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int col0 = tl.n * P.bnh;
         if (in_tail && kb1 < KB) {                              // finalizer of a split tile
           const Fixup F{P.sk_part, &sc, pair + 1, sc.contributors_end(tile), 2, (int)rank, r_cta};
-          if (!sk_wait(P, F, &s_abort)) break;
-          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, 0, &F);
+          if (!__all_sync(0xffffffffu, sk_wait(P, F, &s_abort))) break;
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F);
           sk_done(P, F);
         } else {
-          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0);
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane);
         }
       }
       tc_fence_before();
@@ -1598,14 +1617,16 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   const int grid = std::min(kSkSlots, (int)std::max<int64_t>(1, std::min<int64_t>(
                                           device_sms(), sk ? device_sms() : max_tiles)));
   // at least 120 KB so that one CTA (and one 512-column TMEM allocation) fits per SM
-  const size_t smem = std::max<size_t>((size_t)kStages * (kABytes + (size_t)P.bn * BK * 2) + 1024,
+  const size_t smem = std::max<size_t>((size_t)kStages * (kABytes + (size_t)P.bn * BK * 2) + 1024 +
+                                           4 * kStageBytesPerWarp,
                                        (size_t)120 * 1024);
 
   if (pair) {
     const int64_t pt_routed = (g.max_routed_rows + 2 * BM - 1) / (2 * BM) + g.n_routed;
     const int64_t pt_static = (int64_t)g.n_static * ((g.rows_static + 2 * BM - 1) / (2 * BM));
     const int64_t pair_tiles = (pt_routed + pt_static) * P.nt;
-    const size_t psmem = (size_t)kPairStages * (kABytes + (size_t)(P.bn / 2) * BK * 2) + 1024;
+    const size_t psmem = (size_t)kPairStages * (kABytes + (size_t)(P.bn / 2) * BK * 2) + 1024 +
+                         4 * kStageBytesPerWarp;
 #define MOE_PAIR_CASE(E_)                                                            \
   case E_:                                                                           \
     return launch_pair<E_>(P, ma, mas, mb, mb3, pair_tiles, psmem, s);
