@@ -240,8 +240,13 @@ MOE_API moe_status moe_combine(const moe_config *cfg, const void *y_rows, const 
 
 /* Steps 1-5 in one call; intermediates live in the workspace (at least
  * `workspace` bytes).  counts_out [E] (optional, may be NULL) receives the
- * per-expert assignment counts.  Equivalent to moe_route, moe_permute,
- * moe_expert_ffn and moe_combine in sequence. */
+ * per-expert assignment counts.  Same result as moe_route, moe_permute,
+ * moe_expert_ffn and moe_combine in sequence, bit for bit.  bf16 token
+ * choice with k + S <= 2 (at most two rows a token) folds the combine into
+ * the expert FFN: y is zeroed by the routing kernel and each gated row is
+ * added into its token's row by the down-projection (two bf16 additions onto
+ * 0, which commute), so the workspace holds no y_rows afterwards and no
+ * combine kernel runs.  y [T, d] must not overlap x (MOE_ERR_INVALID_ARG). */
 MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const void *w_router,
                        const float *bias, const float *route_state, const void *w1, const void *w3,
                        const void *w2, void *y, int32_t *counts_out, void *ws, size_t ws_bytes,
@@ -268,14 +273,16 @@ MOE_API moe_status moe_forward_timed(const moe_config *cfg, const void *x, const
  * renormalised, p + b under MOE_ROUTE_BIAS).  bf16 layers only
  * (MOE_ERR_UNSUPPORTED for fp32).
  *   in : the forward's x, w_router, bias, route_state, w1, w3, w2 and its
- *        workspace ws (unchanged since moe_forward); dy [T, d] bf16.
+ *        workspace ws (unchanged since moe_forward: the routing, x_perm and h
+ *        it holds are read); dy [T, d] bf16.
  *   out: dx [T, d], dw_router [E, d], dbias [E] (NULL when bias is NULL),
  *        dw1 [E+S, f, d], dw3 [E+S, f, d] (SwiGLU; NULL for ReLU),
  *        dw2 [E+S, d, f]: fp32, overwritten.
  *   bws: scratch of at least moe_query_backward_size bytes (256-byte aligned).
  *   Arithmetic: bf16 tensor-core contractions with fp32 accumulation; the
  *   recomputed pre-activations, dA / dU and the transposed operands are
- *   rounded to bf16; gate and router gradients in fp32. */
+ *   rounded to bf16; gate and router gradients in fp32 (a gate's gradient
+ *   <dy, FFN_e(x)> is taken as <dy W2_e, act(a)> inside the dA GEMM). */
 MOE_API moe_status moe_query_backward_size(const moe_config *cfg, size_t *bytes);
 MOE_API moe_status moe_backward(const moe_config *cfg, const void *x, const void *w_router,
                                 const float *bias, const float *route_state, const void *w1,

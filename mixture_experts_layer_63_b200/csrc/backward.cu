@@ -239,37 +239,24 @@ __global__ void __launch_bounds__(256) gather_bf16_rows_kernel(const uint4 *__re
 }
 
 // ---- gate gradients and the router ---------------------------------------
-// dG_r = <dy[t], FFN_e(x_t)> for each kept routed row r of token t: the
-// forward's bf16 row is g_r * FFN_e(x_t), so dG_r = <dy[t], y_row> / g_r
-// (0 when g_r is 0: such a row contributes nothing, and neither does its gate).
-__global__ void __launch_bounds__(256) gate_grad_kernel(const __nv_bfloat16 *__restrict__ dy,
-                                                        const __nv_bfloat16 *__restrict__ y_rows,
-                                                        const int32_t *__restrict__ row_token,
-                                                        const float *__restrict__ row_gate,
+// dG_r = <dy[t], FFN_e(x_t)> for each kept routed row r of token t.  With
+// FFN_e(x) = W2_e h, this is <dy[t] W2_e, h_r>: the dact GEMM, whose
+// accumulator holds dy[t] W2_e, multiplies it by h in its epilogue (ReLU:
+// relu of the recomputed a, which equals the forward's rounded h; SwiGLU:
+// the forward's h itself) and leaves one partial sum per 256-column N-tile;
+// here they are added in N-tile order.
+__global__ void __launch_bounds__(256) gate_grad_kernel(const float *__restrict__ dg_part, int nt,
                                                         const int32_t *__restrict__ offsets, int E,
-                                                        int d, float *__restrict__ dgate) {
+                                                        float *__restrict__ dgate) {
   pdl_wait();
   pdl_trigger();
-  const int lane = threadIdx.x & 31;
   const int64_t R = offsets[E];
-  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < R; r += nw) {
-    const int64_t t = row_token[r];
-    const __nv_bfloat16 *a = dy + t * d;
-    const __nv_bfloat16 *b = y_rows + r * d;
-    float acc = 0.0f;
-    for (int i = lane * 2; i < d; i += 64) {
-      const __nv_bfloat162 av = *reinterpret_cast<const __nv_bfloat162 *>(a + i);
-      const __nv_bfloat162 bv = *reinterpret_cast<const __nv_bfloat162 *>(b + i);
-      acc = fmaf(__low2float(av), __low2float(bv), acc);
-      acc = fmaf(__high2float(av), __high2float(bv), acc);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) {
-      const float g = row_gate[r];
-      dgate[r] = g != 0.0f ? acc / g : 0.0f;
-    }
+  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < R;
+       r += (int64_t)gridDim.x * blockDim.x) {
+    const float *p = dg_part + r * nt;
+    float acc = p[0];
+    for (int n = 1; n < nt; ++n) acc = __fadd_rn(acc, p[n]);
+    dgate[r] = acc;
   }
 }
 
@@ -435,14 +422,11 @@ cudaError_t launch_gather_bf16_rows(const void *src, void *dst, const int32_t *m
                        static_cast<uint4 *>(dst), map, offsets, E, src_rows, d / 8, err);
 }
 
-cudaError_t launch_gate_grad(const void *dy, const void *y_rows, const int32_t *row_token,
-                             const float *row_gate, const int32_t *offsets, int E, int d,
+cudaError_t launch_gate_grad(const float *dg_part, int nt, const int32_t *offsets, int E,
                              int64_t max_rows, float *dgate, cudaStream_t s) {
-  const int64_t want = (max_rows + 7) / 8;
-  const unsigned blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, 148 * 16));
-  return launch_kernel(gate_grad_kernel, blocks, 256, 0, s, static_cast<const __nv_bfloat16 *>(dy),
-                       static_cast<const __nv_bfloat16 *>(y_rows), row_token, row_gate, offsets, E,
-                       d, dgate);
+  const int64_t want = (max_rows + 255) / 256;
+  const unsigned blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, 148 * 8));
+  return launch_kernel(gate_grad_kernel, blocks, 256, 0, s, dg_part, nt, offsets, E, dgate);
 }
 
 cudaError_t launch_router_grad(const moe_config *c, const float *probs, const int32_t *topk_idx,

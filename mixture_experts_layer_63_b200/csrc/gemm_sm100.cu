@@ -98,6 +98,11 @@ struct Params {
   int64_t src_rows;
   const void *aux;          // kEpiDAct*: bf16 pre-activations [row][aux_ld]
   int64_t aux_ld;
+  float *dg_part;           // kEpiDAct*: per routed row and N-tile, sum of acc * act(a)
+  int dg_nt;
+  const void *aux2;         // kEpiDActSwiglu: the forward's h [row][aux2_ld] for dg_part
+  int64_t aux2_ld;
+  const int32_t *add_rows;  // kEpiScaleAdd: output row (token) of each routed row
   int b_mn;                 // B stored [K][N] (N contiguous) instead of [N][K]
   int b_kb_split;           //   k-blocks read from map_b, the rest from map_b3
   int64_t b_krows;          //   K rows per group in B's row dimension
@@ -667,6 +672,31 @@ __device__ __forceinline__ void store_rows(uint8_t *stg, const uint32_t (&pk)[PI
   __syncwarp();
 }
 
+// The same staging, with the rows added into out (bf16, vector reductions)
+// at rows dest of each thread's row (-1: not added) instead of stored.
+__device__ __forceinline__ void red_add_bf16x8(__nv_bfloat16 *p, const uint4 w) {
+  asm volatile("red.global.add.noftz.v4.bf16x2 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(w.x), "r"(w.y),
+               "r"(w.z), "r"(w.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void red_rows(uint8_t *stg, const uint32_t (&pk)[32], __nv_bfloat16 *out,
+                                         int64_t ld, int dest, int col, int lane) {
+  uint4 *mine = reinterpret_cast<uint4 *>(stg + lane * 128);
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    mine[stage_slot<8>(lane, c)] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int r = p * 4 + (lane >> 3), c = lane & 7;
+    const uint4 w = reinterpret_cast<const uint4 *>(stg + r * 128)[stage_slot<8>(r, c)];
+    const int dr = __shfl_sync(0xffffffffu, dest, r);
+    if (dr >= 0) red_add_bf16x8(out + (int64_t)dr * ld + col + c * 8, w);
+  }
+  __syncwarp();
+}
+
 // 32 fp32 values into 16 bf16x2 words at word offset 16 * H of pk
 template <int H, int N>
 __device__ __forceinline__ void pack_words(uint32_t (&pk)[N], const float (&v)[32]) {
@@ -690,11 +720,13 @@ __device__ __forceinline__ void acc_cols(uint32_t taddr, int c, const Fixup *F, 
 // up 128-255), output columns from col0 on; the later stream-K pieces of the
 // tile added first when F is given; then activation / gate / bias, stores.
 // The warp's rows are consecutive (lane l: output row out_row = row0 + l);
-// `stg` is the warp's staging buffer.
+// `stg` is the warp's staging buffer.  kEpiScaleAdd adds the row into output
+// row `dest` instead (-1: nothing).
 template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, bool valid, bool routed,
                                               int64_t out_row, int col0, uint8_t *stg, int lane,
-                                              int64_t out_offset = 0, const Fixup *F = nullptr) {
+                                              int64_t out_offset = 0, const Fixup *F = nullptr,
+                                              int dest = -1) {
   float v[32];
   if constexpr (EPI == kEpiStoreF32) {
     // a K part when the router is split: no bias, own output
@@ -728,6 +760,7 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
     const int ncol = EPI == kEpiPreSwiglu ? 128 : P.bn;
     const float scale = (EPI == kEpiDActSwiglu && routed && valid) ? P.row_gate[out_row] : 1.0f;
     const __nv_bfloat16 *aux = reinterpret_cast<const __nv_bfloat16 *>(P.aux);
+    float dg = 0.0f;                                            // sum of acc * h (the forward's h)
 #pragma unroll 1
     for (int c = 0; c < ncol / 32; ++c) {
       const int col = col0 + c * 32;
@@ -740,6 +773,13 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
       } else {
         // dh = g * acc, then SwiGLU's backward from the saved a and u
         acc_cols(taddr, c * 32, F, v);
+        if (P.dg_part && routed && valid) {
+          // gate-gradient piece against the forward's h (rounded once)
+          float hh[32];
+          load_bf16x32(reinterpret_cast<const __nv_bfloat16 *>(P.aux2) + out_row * P.aux2_ld + col, hh);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) dg = fmaf(v[i], hh[i], dg);
+        }
         float a[32], uu[32];
         if (valid) {
           load_bf16x32(aux + out_row * P.aux_ld + col, a);
@@ -750,8 +790,8 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float dh = v[i] * scale;
           const float sg = 1.0f / (1.0f + __expf(-a[i]));
+          const float dh = v[i] * scale;
           w[i] = dh * a[i] * sg;
           v[i] = dh * uu[i] * sg * (1.0f + a[i] * (1.0f - sg));
         }
@@ -761,12 +801,16 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
       store_rows<4>(stg, pk, out, ld, row0, col, vmask, lane);
       store_rows<4>(stg, pk2, out, ld, row0, (int)P.N + col, vmask, lane);
     }
+    if (EPI == kEpiDActSwiglu && P.dg_part && routed && valid)
+      P.dg_part[out_row * P.dg_nt + col0 / P.bnh] = dg;
   } else {
     // one output, 64 columns (one 128-byte line a row) at a time
     const int ncol = EPI == kEpiSwiglu ? 128 : P.bn;
     const int64_t ld = P.N;
-    const float scale = ((EPI == kEpiScale || EPI == kEpiDActRelu) && routed && valid) ? P.row_gate[out_row] : 1.0f;
+    const float scale = ((EPI == kEpiScale || EPI == kEpiScaleAdd || EPI == kEpiDActRelu) && routed && valid)
+                            ? P.row_gate[out_row] : 1.0f;
     const __nv_bfloat16 *aux = reinterpret_cast<const __nv_bfloat16 *>(P.aux);
+    float dg = 0.0f;                                            // sum of acc * relu(a)
 #pragma unroll 1
     for (int c2 = 0; c2 < ncol / 64; ++c2) {
       const int col = col0 + c2 * 64;
@@ -784,8 +828,9 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
         } else if constexpr (EPI == kEpiRelu) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.0f);
-        } else if constexpr (EPI == kEpiScale) {
+        } else if constexpr (EPI == kEpiScale || EPI == kEpiScaleAdd) {
           // gated rows in bf16; the combine sums them in fp32 and rounds once
+          // (kEpiScaleAdd: added into the zeroed output rows, at most two per row)
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] *= scale;
         } else if constexpr (EPI == kEpiDActRelu) {
@@ -798,14 +843,31 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
             for (int i = 0; i < 32; ++i) a[i] = 0.f;
           }
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = a[i] > 0.0f ? v[i] * scale : 0.0f;
+          for (int i = 0; i < 32; ++i) {
+            dg = fmaf(v[i], fmaxf(a[i], 0.0f), dg);
+            v[i] = a[i] > 0.0f ? v[i] * scale : 0.0f;
+          }
         }                                                       // kEpiPreRelu: a as is
         if (h == 0) pack_words<0>(pk, v);
         else pack_words<1>(pk, v);
       }
-      store_rows<8>(stg, pk, out, ld, row0, col, vmask, lane);
+      if constexpr (EPI == kEpiScaleAdd) red_rows(stg, pk, out, ld, dest, col, lane);
+      else store_rows<8>(stg, pk, out, ld, row0, col, vmask, lane);
     }
+    if (EPI == kEpiDActRelu && P.dg_part && routed && valid)
+      P.dg_part[out_row * P.dg_nt + col0 / P.bnh] = dg;
   }
+}
+
+// kEpiScaleAdd: the output row a tile row adds into (its token; a static
+// group's row t is token t), -1 when out of range (error bit raised)
+__device__ __forceinline__ int add_dest(const Params &P, bool routed, int64_t out_row, int64_t tile_row) {
+  const int64_t t = routed ? (int64_t)P.add_rows[out_row] : tile_row;
+  if (t < 0 || t >= P.src_rows) {
+    raise_error(P.err, kErrBadIndex);
+    return -1;
+  }
+  return (int)t;
 }
 
 // K-grouped mode: this thread's row of a weight-gradient tile (fp32), or
@@ -1121,14 +1183,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         : P.out_static_base + (int64_t)(tl.g - P.n_routed) * P.rows_static) +
                                 (int64_t)tl.m * BM + r_cta;
         const int col0 = tl.n * P.bnh;
+        const int dest = (EPI == kEpiScaleAdd && valid) ? add_dest(P, routed, out_row, tl.m * BM + r_cta) : -1;
         if (in_tail && kb1 < KB) {                              // finalizer of a split tile
           const Fixup F{P.sk_part, &sc, (int)blockIdx.x + 1, sc.contributors_end(tile), 1, 0, r_cta};
           if (!__all_sync(0xffffffffu, sk_wait(P, F, &s_abort))) break;
-          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F);
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F, dest);
           sk_done(P, F);
         } else {
           epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane,
-                             (int64_t)part * P.split_stride);
+                             (int64_t)part * P.split_stride, nullptr, dest);
         }
       }
       tc_fence_before();
@@ -1414,13 +1477,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                         : P.out_static_base + (int64_t)(tl.g - P.n_routed) * P.rows_static) +
                                 (int64_t)tl.m * PM + r_in;
         const int col0 = tl.n * P.bnh;
+        const int dest = (EPI == kEpiScaleAdd && valid) ? add_dest(P, routed, out_row, tl.m * PM + r_in) : -1;
         if (in_tail && kb1 < KB) {                              // finalizer of a split tile
           const Fixup F{P.sk_part, &sc, pair + 1, sc.contributors_end(tile), 2, (int)rank, r_cta};
           if (!__all_sync(0xffffffffu, sk_wait(P, F, &s_abort))) break;
-          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F);
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F, dest);
           sk_done(P, F);
         } else {
-          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane);
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, nullptr, dest);
         }
       }
       tc_fence_before();
@@ -1563,6 +1627,11 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   P.out2 = g.out2;
   P.aux = g.aux;
   P.aux_ld = g.aux_ld;
+  P.dg_part = g.dg_part;
+  P.dg_nt = g.dg_nt;
+  P.aux2 = g.aux2;
+  P.aux2_ld = g.aux2_ld;
+  P.add_rows = g.add_rows;
   // stream-K tail for the expert GEMMs (not with the router's K split or K groups)
   const bool sk = MOE_STREAM_K && P.ksplit == 1 && !g.kgroup && g.n_routed > 0 && g.sk_part &&
                   g.sk_flags;
@@ -1578,6 +1647,12 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   if (P.G <= 0 || P.G > kMaxGroups || P.bn > 256 || g.K % BK != 0) return cudaErrorInvalidValue;
   if (g.ksplit > 1 && (g.epi != kEpiStoreF32 || g.n_routed != 0)) return cudaErrorInvalidValue;
   if ((g.epi == kEpiDActRelu || g.epi == kEpiDActSwiglu) && (!g.aux || !g.row_gate))
+    return cudaErrorInvalidValue;
+  if (g.dg_part && (g.dg_nt != P.nt || (g.epi != kEpiDActRelu && g.epi != kEpiDActSwiglu) ||
+                    (g.epi == kEpiDActSwiglu && !g.aux2)))
+    return cudaErrorInvalidValue;
+  // the folded combine: gates, the row -> token map, its range
+  if (g.epi == kEpiScaleAdd && (!g.row_gate || !g.add_rows || g.src_rows <= 0 || g.N % 64 != 0))
     return cudaErrorInvalidValue;
   if (g.b_mn && (swiglu_b(g.epi) || g.kgroup || g.b_krows <= 0 || P.bn != 256))
     return cudaErrorInvalidValue;
@@ -1639,6 +1714,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
       MOE_PAIR_CASE(kEpiPreSwiglu)
       MOE_PAIR_CASE(kEpiDActRelu)
       MOE_PAIR_CASE(kEpiDActSwiglu)
+      MOE_PAIR_CASE(kEpiScaleAdd)
       default: return cudaErrorInvalidValue;
     }
 #undef MOE_PAIR_CASE
@@ -1655,6 +1731,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
     MOE_ONE_CASE(kEpiPreSwiglu)
     MOE_ONE_CASE(kEpiDActRelu)
     MOE_ONE_CASE(kEpiDActSwiglu)
+    MOE_ONE_CASE(kEpiScaleAdd)
     default: return cudaErrorInvalidValue;
   }
 #undef MOE_ONE_CASE

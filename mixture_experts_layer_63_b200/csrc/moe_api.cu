@@ -138,15 +138,29 @@ static moe_status check_ws(const WsLayout &L, const void *ws, size_t ws_bytes, s
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The combine folded into the down-projection (moe_forward): with at most
+// two rows a token (k + S <= 2, token choice), the gate zeroes y and the
+// down-projection's epilogue adds each gated bf16 row into its token's row
+// of y with bf16 vector reductions.  Two bf16 additions onto 0 commute, so
+// the result is the same in whatever order the rows arrive: y = bf16(r1 +
+// r2), as the combine kernel computes it.  No y_rows, no combine launch.
+#ifndef MOE_FOLD_COMBINE
+#define MOE_FOLD_COMBINE 1
+#endif
+static bool combine_folded(const moe_config *c) {
+  return MOE_FOLD_COMBINE && c->mode == MOE_TOKEN_CHOICE && c->dtype == MOE_BF16 && c->k + c->S <= 2;
+}
+
 // ---- step bodies, shared by the step entry points and moe_forward ----------
+// y_zero non-null: the gate also sets y to 0 (the folded combine)
 static cudaError_t run_route(const moe_config *c, const WsLayout &L, char *ws, const void *x,
                              const void *w_router, const float *bias, const float *state,
                              float *logits, float *probs, int32_t *topk_idx, float *topk_gate,
-                             cudaStream_t s) {
+                             cudaStream_t s, void *y_zero = nullptr) {
   int32_t *hist = c->mode == MOE_TOKEN_CHOICE ? reinterpret_cast<int32_t *>(ws + L.hist) : nullptr;
   if (router_is_fused(c))
     return launch_route_gate(c, nullptr, logits, x, w_router, bias, state, probs, topk_idx,
-                             topk_gate, hist, s);
+                             topk_gate, hist, s, 1, 0, y_zero);
   cudaError_t e;
   if (c->dtype == MOE_F32) {
     e = launch_router_f32(c, static_cast<const float *>(x), static_cast<const float *>(w_router),
@@ -182,7 +196,7 @@ static cudaError_t run_route(const moe_config *c, const WsLayout &L, char *ws, c
       e = launch_grouped_gemm(g, s);
       if (e != cudaSuccess) return e;
       return launch_route_gate(c, parts, logits, nullptr, nullptr, bias, state, probs, topk_idx,
-                               topk_gate, hist, s, ks, c->T * c->E);
+                               topk_gate, hist, s, ks, c->T * c->E, y_zero);
     }
     g.out = logits;
     g.bias = bias;
@@ -190,15 +204,18 @@ static cudaError_t run_route(const moe_config *c, const WsLayout &L, char *ws, c
   }
   if (e != cudaSuccess) return e;
   return launch_route_gate(c, logits, nullptr, nullptr, nullptr, nullptr, state, probs, topk_idx,
-                           topk_gate, hist, s);
+                           topk_gate, hist, s, 1, 0, y_zero);
 }
 
 // row_token non-null (bf16): the up-projection gathers the routed rows of x
-// itself and x_perm is not read
+// itself and x_perm is not read.  y_add non-null (bf16): the folded combine,
+// the down-projection adds row r into y_add[add_rows[r]] (zeroed by the gate)
+// instead of writing y_rows.
 static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, const void *x,
                            const void *x_perm, const int32_t *offsets, const float *row_gate,
                            const void *w1, const void *w3, const void *w2, void *h, void *y_rows,
-                           cudaStream_t s, const int32_t *row_token = nullptr) {
+                           cudaStream_t s, const int32_t *row_token = nullptr,
+                           void *y_add = nullptr, const int32_t *add_rows = nullptr) {
   uint32_t *err = reinterpret_cast<uint32_t *>(ws + L.err);
   if (c->dtype == MOE_F32)
     return launch_ffn_f32(c, L, err, static_cast<const float *>(x),
@@ -236,7 +253,7 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
   cudaError_t e = launch_grouped_gemm(up, s);
   if (e != cudaSuccess) return e;
   GroupedGemm dn{};
-  dn.epi = kEpiScale;
+  dn.epi = y_add ? kEpiScaleAdd : kEpiScale;
   dn.K = c->d_ff;
   dn.N = c->d_model;
   dn.a = h;
@@ -254,7 +271,9 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
   dn.a_static_stride = c->T;
   dn.out_static_base = L.rows_cap;
   dn.max_routed_rows = L.rows_cap;
-  dn.out = y_rows;
+  dn.out = y_add ? y_add : y_rows;
+  dn.add_rows = y_add ? add_rows : nullptr;
+  dn.src_rows = c->T;
   dn.row_gate = row_gate;
   // the last groups' activations are the ones still in L2 when the
   // up-projection ends: start the down-projection there
@@ -269,10 +288,11 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
 static int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 struct BwLayout {
-  size_t dy_perm, au, dau, dx_rows, kseg, kseg_r, dyT, hT, dauT, xT, dgate, dl, dl_pad, dlT,
-      xTr, wrT, dx_router, total;
+  size_t dy_perm, au, dau, dx_rows, kseg, kseg_r, dyT, hT, dauT, xT, dgate, dg_part, dl, dl_pad,
+      dlT, xTr, wrT, dx_router, total;
   int64_t kp_max, Ep, Tp;
   int fw;
+  int dg_nt;                // 256-column N-tiles of the dact GEMM (pieces of a gate gradient)
 };
 
 static BwLayout make_bw_layout(const moe_config *c, const WsLayout &L) {
@@ -300,6 +320,8 @@ static BwLayout make_bw_layout(const moe_config *c, const WsLayout &L) {
   B.dauT = take((size_t)B.fw * B.kp_max * 2);
   B.xT = take((size_t)d * B.kp_max * 2);
   B.dgate = take((size_t)L.rows_cap * 4);
+  B.dg_nt = (int)((f + 255) / 256);
+  B.dg_part = take((size_t)L.rows_cap * B.dg_nt * 4);
   B.dl = take((size_t)T * c->E * 4);
   B.dl_pad = take((size_t)T * B.Ep * 2);
   B.dlT = take((size_t)c->E * B.Tp * 2);
@@ -329,7 +351,6 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
   const int32_t *row_token = reinterpret_cast<const int32_t *>(ws + L.row_token);
   const float *row_gate = reinterpret_cast<const float *>(ws + L.row_gate);
   const void *h = ws + L.h;
-  const void *y_rows = ws + L.y_rows;
   const bool fused_gather = c->dtype == MOE_BF16 && MOE_FUSED_GATHER;
   void *dy_perm = bw + B.dy_perm;
   void *au = bw + B.au, *dau = bw + B.dau;
@@ -398,6 +419,10 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
   dh.out = dau;
   dh.aux = au;
   dh.aux_ld = B.fw;
+  dh.dg_part = reinterpret_cast<float *>(bw + B.dg_part);
+  dh.dg_nt = B.dg_nt;
+  dh.aux2 = h;                     // the forward's activations (SwiGLU's gate-gradient pieces)
+  dh.aux2_ld = f;
   dh.row_gate = row_gate;
   dh.sk_part = sk_part;
   dh.sk_flags = sk_flags;
@@ -434,7 +459,8 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
   MOE_TRY(launch_grouped_gemm(dxg, s));
 
   // 6-8. gate gradients, router logits gradient dl, bias gradient
-  MOE_TRY(launch_gate_grad(dy, y_rows, row_token, row_gate, offsets, E, (int)d, L.rows_cap, dgate, s));
+  MOE_TRY(launch_gate_grad(reinterpret_cast<const float *>(bw + B.dg_part), B.dg_nt, offsets, E,
+                           L.rows_cap, dgate, s));
   MOE_TRY(launch_router_grad(c, probs, topk_idx, tok_rows, dgate, state, dl, s));
   if (dbias) MOE_TRY(launch_bias_grad(dl, T, E, dbias, s));
 
@@ -656,6 +682,13 @@ static moe_status forward_impl(const moe_config *cfg, const void *x, const void 
   if (!aligned16(x) || !aligned16(w_router) || !aligned16(w1) || !aligned16(w2) || !aligned16(y) ||
       (swiglu && !aligned16(w3)))
     return MOE_ERR_INVALID_ARG;
+  const bool fold = combine_folded(cfg);
+  {
+    // y is written from the first kernel on (folded combine): it may not overlap x
+    const uintptr_t xb = reinterpret_cast<uintptr_t>(x), yb = reinterpret_cast<uintptr_t>(y);
+    const uintptr_t n = (uintptr_t)cfg->T * (uintptr_t)cfg->d_model * elem_size(cfg);
+    if (xb < yb + n && yb < xb + n) return MOE_ERR_INVALID_ARG;
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   char *w = static_cast<char *>(ws);
   float *logits = reinterpret_cast<float *>(w + L.logits);
@@ -677,7 +710,8 @@ static moe_status forward_impl(const moe_config *cfg, const void *x, const void 
   };
   cudaError_t e = mark(0);
   if (e == cudaSuccess)
-    e = run_route(cfg, L, w, x, w_router, bias, state, logits, probs, topk_idx, topk_gate, s);
+    e = run_route(cfg, L, w, x, w_router, bias, state, logits, probs, topk_idx, topk_gate, s,
+                  fold ? y : nullptr);
   if (e == cudaSuccess) e = mark(1);
   // token choice: the gate wrote the unit histogram into the workspace.
   // bf16: the up-projection gathers the rows of x itself (no x_perm)
@@ -689,9 +723,9 @@ static moe_status forward_impl(const moe_config *cfg, const void *x, const void 
   if (e == cudaSuccess) e = mark(2);
   if (e == cudaSuccess)
     e = run_ffn(cfg, L, w, x, x_perm, offsets, row_gate, w1, w3, w2, h, y_rows, s,
-                fused_gather ? row_token : nullptr);
+                fused_gather ? row_token : nullptr, fold ? y : nullptr, row_token);
   if (e == cudaSuccess) e = mark(3);
-  if (e == cudaSuccess) e = launch_combine(cfg, L.rows_cap, y_rows, tok_rows, y, s);
+  if (e == cudaSuccess && !fold) e = launch_combine(cfg, L.rows_cap, y_rows, tok_rows, y, s);
   if (e == cudaSuccess) e = mark(4);
   if (e == cudaSuccess && counts_out)
     e = cudaMemcpyAsync(counts_out, counts, (size_t)cfg->E * 4, cudaMemcpyDeviceToDevice, s);

@@ -113,11 +113,13 @@ bool router_is_fused(const moe_config *c);
 // logits_in may hold nsplit partial sums split_stride floats apart (summed in
 // order, then + bias when bias is given).
 // state: the per-expert routing bias or utilisation of c->route_rule (or null).
+// y_zero non-null: every token's row of y [T, d] (layer dtype) is set to 0
+// (the down-projection then adds the token's rows into it)
 cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float *logits_out,
                               const void *x, const void *w_router, const float *bias,
                               const float *state, float *probs, int32_t *topk_idx, float *topk_gate,
                               int32_t *hist, cudaStream_t s, int nsplit = 1,
-                              int64_t split_stride = 0);
+                              int64_t split_stride = 0, void *y_zero = nullptr);
 // DeepSeek-V3 routing-bias update from a step's counts (one block)
 cudaError_t launch_bias_update(const moe_config *c, const int32_t *counts, float *bias, float gamma,
                                cudaStream_t s);
@@ -140,13 +142,16 @@ enum GemmEpilogue : int {
   kEpiStoreF32 = 0,   // out fp32 = acc (+ bias[col])           (router logits)
   kEpiRelu = 1,       // out bf16 = relu(acc)                    (up-projection, ReLU)
   kEpiSwiglu = 2,     // out bf16 = silu(acc_gate) * acc_up      (gate/up projection)
-  kEpiScale = 3,      // out fp32 = row_gate[row] * acc          (down-projection)
+  kEpiScale = 3,      // out bf16 = row_gate[row] * acc          (down-projection, gated rows)
   // backward
   kEpiPreRelu = 4,    // out bf16 = acc                          (pre-activation a, recomputed)
   kEpiPreSwiglu = 5,  // out bf16 [row][col] = a, [row][N+col] = u  (gate/up pre-activations)
   kEpiDActRelu = 6,   // dh = g*acc; out bf16 = dh * [a > 0]     (a from aux [row][col])
   kEpiDActSwiglu = 7, // dh = g*acc; s = sigmoid(a): out[row][col] = dh u s (1 + a (1 - s)),
                       //   out[row][N+col] = dh a s              (a, u from aux, ld 2N)
+  // forward, combine folded into the down-projection
+  kEpiScaleAdd = 8,   // out[add_rows[row]] += bf16(row_gate[row] * acc)  (routed rows; a static
+                      //   group's row t adds into out[t]); out zeroed beforehand
 };
 
 // One grouped GEMM  out[rows_g, N] = A[rows_g, K] . B_g[N, K]^T  per group g.
@@ -191,6 +196,13 @@ struct GroupedGemm {
   int64_t b_krows;
   const void *aux;          // kEpiDAct*: bf16 pre-activations, ld aux_ld
   int64_t aux_ld;
+  // kEpiDAct*: dg_part[row * dg_nt + n] = sum over N-tile n's columns of
+  // acc * act(a) for routed rows (the gate gradient's pieces); null: none
+  float *dg_part;
+  int dg_nt;
+  const void *aux2;         // kEpiDActSwiglu with dg_part: the forward's bf16 h [row][aux2_ld]
+  int64_t aux2_ld;          //   (the gate-gradient pieces take h from there)
+  const int32_t *add_rows;  // kEpiScaleAdd: output row of each routed row (row_token)
   // K-grouped mode (weight gradients): group g computes out_g[M, N] =
   // A[M, kseg[g]:kseg[g+1]] . B[N, kseg[g]:kseg[g+1]]^T over the K columns
   // kseg gives (multiples of 64, device array of n_static + 1 entries; one
@@ -222,8 +234,7 @@ cudaError_t launch_transpose_segments(const void *src, int64_t ld, const int32_t
 cudaError_t launch_gather_bf16_rows(const void *src, void *dst, const int32_t *map,
                                     const int32_t *offsets, int E, int64_t src_rows, int d,
                                     int64_t max_rows, uint32_t *err, cudaStream_t s);
-cudaError_t launch_gate_grad(const void *dy, const void *y_rows, const int32_t *row_token,
-                             const float *row_gate, const int32_t *offsets, int E, int d,
+cudaError_t launch_gate_grad(const float *dg_part, int nt, const int32_t *offsets, int E,
                              int64_t max_rows, float *dgate, cudaStream_t s);
 cudaError_t launch_router_grad(const moe_config *c, const float *probs, const int32_t *topk_idx,
                                const int32_t *tok_rows, const float *dgate, const float *state,

@@ -49,6 +49,8 @@ struct GateParams {
   int64_t T;
   int d, E, k, n_groups, topk_groups, renormalize, nunit;
   int nbg;                    // 32-token blocks per local group (unit numbering)
+  uint4 *y_zero;              // [T, y_vecs] 16-byte vectors set to 0, or null
+  int y_vecs;
 };
 
 __device__ __forceinline__ void argmax_warp(float &v, int &i) {
@@ -116,6 +118,8 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_gate_kernel(const GatePa
 
   const int64_t t = (int64_t)blockIdx.x * kTokWarps + warp;
   const bool live = t < P.T;
+  if (P.y_zero && live)
+    for (int v = lane; v < P.y_vecs; v += 32) P.y_zero[t * P.y_vecs + v] = make_uint4(0u, 0u, 0u, 0u);
 
   // fused router: this warp's token, lanes split the model dimension (lane l
   // takes chunks l, l + 32, ...); the first NB chunks a lane are in flight
@@ -390,8 +394,11 @@ bool router_is_fused(const moe_config *c) {
 cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float *logits_out,
                               const void *x, const void *w_router, const float *bias,
                               const float *state, float *probs, int32_t *topk_idx, float *topk_gate,
-                              int32_t *hist, cudaStream_t s, int nsplit, int64_t split_stride) {
+                              int32_t *hist, cudaStream_t s, int nsplit, int64_t split_stride,
+                              void *y_zero) {
   GateParams P{};
+  P.y_zero = static_cast<uint4 *>(y_zero);
+  P.y_vecs = (int)((int64_t)c->d_model * (c->dtype == MOE_BF16 ? 2 : 4) / 16);
   P.rule = c->mode == MOE_TOKEN_CHOICE ? c->route_rule : MOE_ROUTE_SOFTMAX;
   P.state = state;
   P.alpha = c->route_alpha;

@@ -44,6 +44,10 @@ SMALL = {
     # even CTA's rows only) and of 122 rows (both CTAs), the shared expert's
     # 2150 = 8 * 256 + 102 rows
     "pair_half_s": replace(WORKLOADS["gshard"], T=2150, E=4, S=1, d_model=256, d_ff=320),
+    # one routed and one shared row a token: moe_forward adds both into y from
+    # the down-projection (the folded combine), with single CTAs and with pairs
+    "fold_shared_s": replace(WORKLOADS["gshard"], T=700, k=1, S=1, d_model=256, d_ff=320),
+    "fold_shared_pair_s": replace(WORKLOADS["gshard"], T=2100, E=4, k=1, S=1, d_model=256, d_ff=320),
     # routing variants: DeepSeek-V3 bias routing (256 + 1 experts, top-8 of 4
     # groups), load-aware top-k, GShard local groups
     "dsv3_s": replace(WORKLOADS["deepseek_v3"], T=600, d_model=256, d_ff=128),

@@ -292,6 +292,38 @@ def test_forward_small(name):
     _forward_check(SMALL[name])
 
 
+FOLDED = [n for n, w in SMALL.items()
+          if w.dtype == "bf16" and w.mode == "tc" and w.k + w.S <= 2]
+
+
+@pytest.mark.parametrize("name", FOLDED + ["full:gshard", "full:mixtral"])
+def test_folded_combine_equals_the_steps(name):
+    """With at most two rows a token, moe_forward adds the gated rows into y
+    inside the down-projection; the result is bit-identical to the step entry
+    points (gated rows written out, then the combine kernel's fp32 sum and one
+    rounding)."""
+    w = WORKLOADS[name[5:]] if name.startswith("full:") else SMALL[name]
+    inp = gpu_inputs(w, seed=12, grid=False)
+    cfg = api.config_from_workload(w)
+    ws = api.new_workspace(cfg)
+    y = torch.empty_like(inp.x)
+    api.moe_forward(cfg, inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, y, None, ws,
+                    route_state=inp.route_state)
+    B = api.step_buffers(cfg)
+    api.moe_route(cfg, inp.x, inp.w_router, inp.bias, B.logits, B.probs, B.topk_idx, B.topk_gate,
+                  B.ws, route_state=inp.route_state)
+    api.moe_permute(cfg, inp.x, B.topk_idx, B.topk_gate, B.probs, B.counts, B.offsets, B.tok_rows,
+                    B.row_token, B.row_gate, B.x_perm, B.n_dropped, B.ws)
+    api.moe_expert_ffn(cfg, inp.x, B.x_perm, B.offsets, B.row_gate, inp.w1, inp.w3, inp.w2, B.h,
+                       B.y_rows, B.ws)
+    y_steps = torch.empty_like(inp.x)
+    api.moe_combine(cfg, B.y_rows, B.tok_rows, y_steps)
+    torch.cuda.synchronize()
+    api.moe_check_device_errors(ws)
+    api.moe_check_device_errors(B.ws)
+    assert torch.equal(y.view(torch.int16), y_steps.view(torch.int16))
+
+
 @pytest.mark.parametrize("name", list(WORKLOADS))
 def test_forward_full_size_sampled(name):
     """The benchmark's launch configuration at full size: full routing bit-exact
