@@ -9,7 +9,8 @@ in HBM.  The timed loop calls moe_forward_timed (the launches of moe_forward,
 with CUDA events recorded at its phase boundaries on the launching stream);
 L2 is flushed (256 MB memset, untimed) before every step.  `e2e` times moe_forward through the public
 layer object with the host->device copy of x and the device->host copy of y
-inside the timed region.  With N > 1 (torchrun), every rank runs its own
+inside the timed region (no flush there: every step streams all expert
+weights, more than the 126 MB L2, and x arrives fresh from the host).  With N > 1 (torchrun), every rank runs its own
 replica on its own tokens (no collective in the forward: weak scaling); the
 time is the maximum over ranks.
 
@@ -386,6 +387,10 @@ def run_ours(args, w) -> None:
     permute_bytes = (w.T * w.d_model + R * w.d_model) * es
     combine_bytes = rows * w.d_model * es + w.T * w.d_model * es    # gated rows in, y out
     route_bytes = (w.T * w.d_model + w.E * w.d_model) * es + 2 * w.T * w.E * 4
+    weight_bytes = (w.E + w.S) * w.d_ff * w.d_model * nmat * es
+    # moe_forward folds the combine into the down-projection when a token has
+    # at most two rows (bf16 token choice, k + S <= 2): no combine phase then
+    folded = w.dtype == "bf16" and w.mode == "tc" and w.k + w.S <= 2
     mean = per.mean(axis=0)                                # ms per call
     hbm, tfl, tfl_sus, peak_src = _peaks()
     gemm_tflops = gemm_flops / (ffn_ms * 1e-3) / 1e12
@@ -395,16 +400,16 @@ def run_ours(args, w) -> None:
 
     # end to end through the public layer object, host buffers: every step
     # copies its batch of x from pinned host memory and its y back; the
-    # copies of neighbouring steps overlap the forward (api.HostPipeline); L2
-    # is flushed on the compute stream before every forward, inside the timed
-    # region
+    # copies of neighbouring steps overlap the forward (api.HostPipeline).  No
+    # L2 flush: every step streams the expert weights (larger than the L2 on
+    # every workload) and x arrives fresh from the host, as a caller sees it
     layer = api.MoELayer(cfg, inp.w_router, inp.w1, inp.w2, inp.w3, inp.bias,
                          route_state=inp.route_state)
     x_host = [inp.x.cpu().pin_memory() for _ in range(2)]
     y_host = [torch.empty_like(x_host[0]).pin_memory() for _ in range(2)]
     x_dev = torch.empty_like(inp.x)
     y_dev = torch.empty_like(inp.x)
-    pipe = api.HostPipeline(layer, before_forward=flush.zero_)
+    pipe = api.HostPipeline(layer)
     for i in range(args.warmup):
         pipe.submit(x_host[i & 1], y_host[i & 1])
     pipe.synchronize()
@@ -429,7 +434,6 @@ def run_ours(args, w) -> None:
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     seq_ms = 0.0
     for i in range(args.steps):
-        flush.zero_()
         s0.record(stream)
         x_dev.copy_(x_host[i & 1], non_blocking=True)
         layer(x_dev, out=y_dev)
@@ -500,16 +504,19 @@ def run_ours(args, w) -> None:
             "steps_us": {"route": mean[0] * 1e3, "permute": mean[1] * 1e3,
                          "expert_ffn": mean[2] * 1e3, "combine": mean[3] * 1e3,
                          "expert_ffn_in_timed_region": ffn_ms * 1e3,
+                         "combine_folded_into_down_gemm": folded,
                          "note": "phase split from separate steps with an event at every phase boundary"},
             "bandwidth_gbs": {"route": route_bytes / (mean[0] * 1e-3) / 1e9,
                               "permute": permute_bytes / (mean[1] * 1e-3) / 1e9,
-                              "combine": combine_bytes / (mean[3] * 1e-3) / 1e9,
+                              "combine": None if folded else combine_bytes / (mean[3] * 1e-3) / 1e9,
                               "hbm_peak": hbm},
             "rows": {"routed_kept": R, "shared": w.S * w.T, "capacity_rows": sizes.rows_cap},
             "e2e": {"value": e2e_value, "unit": "tokens/s",
                     "h2d_bytes_per_step": int(x_host[0].numel() * x_host[0].element_size()),
                     "d2h_bytes_per_step": int(y_host[0].numel() * y_host[0].element_size()),
                     "sequential_value": e2e_seq,
+                    "l2": "not flushed: each step streams %.0f MB of expert weights (L2: 126 MB)"
+                          % (weight_bytes / 1e6),
                     "note": "api.HostPipeline: each step's host copies overlap its neighbours' forwards"},
             "gpu_launches": launches,
             "clocks": clk,

@@ -54,6 +54,10 @@ constexpr int kMaxGroups = 320;
 #ifndef MOE_PAIR_MIN_ROWS
 #define MOE_PAIR_MIN_ROWS 384
 #endif
+// K-grouped weight gradients on CTA pairs as well
+#ifndef MOE_PAIR_WGRAD
+#define MOE_PAIR_WGRAD 1
+#endif
 constexpr uint32_t kABytes = BM * BK * 2;   // 16 KB
 // Gathered A rows: warps 2 and 3 copy them with cp.async (16 bytes a copy,
 // 128-byte swizzle applied by hand) and report a stage full after issuing
@@ -697,6 +701,26 @@ __device__ __forceinline__ void red_rows(uint8_t *stg, const uint32_t (&pk)[32],
   __syncwarp();
 }
 
+// Each thread's 128-byte row piece (32 words) to its own destination `dst`
+// (bytes; null: not stored), through the warp's staging buffer: every store
+// instruction of the warp then writes four whole 128-byte lines.
+__device__ __forceinline__ void store_rows_at(uint8_t *stg, const uint32_t (&pk)[32], char *dst, int lane) {
+  uint4 *mine = reinterpret_cast<uint4 *>(stg + lane * 128);
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    mine[stage_slot<8>(lane, c)] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int r = p * 4 + (lane >> 3), c = lane & 7;
+    const uint4 w = reinterpret_cast<const uint4 *>(stg + r * 128)[stage_slot<8>(r, c)];
+    char *d = reinterpret_cast<char *>(
+        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst), r));
+    if (d) *reinterpret_cast<uint4 *>(d + c * 16) = w;
+  }
+  __syncwarp();
+}
+
 // 32 fp32 values into 16 bf16x2 words at word offset 16 * H of pk
 template <int H, int N>
 __device__ __forceinline__ void pack_words(uint32_t (&pk)[N], const float (&v)[32]) {
@@ -736,12 +760,15 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
     for (int c = 0; c < P.bn / 32; ++c) {
       acc_cols(taddr, c * 32, F, v);
       const int col0c = col0 + c * 32;
-      if (!valid) continue;
+      if (col0c >= P.N) break;                                  // the same for the whole CTA
       if (!bias && col0c + 32 <= P.N && (P.N & 3) == 0) {
-        float4 *dst = reinterpret_cast<float4 *>(out + out_row * P.N + col0c);
+        // whole 32-column groups: 128-byte rows through the staging buffer
+        uint32_t w[32];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-      } else {
+        for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
+        store_rows_at(stg, w, valid ? reinterpret_cast<char *>(out + out_row * P.N + col0c) : nullptr,
+                      lane);
+      } else if (valid) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int col = col0c + i;
@@ -872,9 +899,10 @@ __device__ __forceinline__ int add_dest(const Params &P, bool routed, int64_t ou
 
 // K-grouped mode: this thread's row of a weight-gradient tile (fp32), or
 // zeros when the group has no K columns (zero is the same for the whole
-// CTA, so the warp's TMEM loads stay aligned); dst null: row past M
+// CTA, so the warp's TMEM loads stay aligned); dst null: row past M.  Whole
+// 32-column groups (128 bytes a row) leave through the staging buffer.
 __device__ __forceinline__ void epilogue_wgrad(const Params &P, uint32_t taddr, bool zero, float *dst,
-                                               int col0) {
+                                               int col0, uint8_t *stg, int lane) {
   uint32_t r[32];
 #pragma unroll 1
   for (int c = 0; c < P.bn / 32; ++c) {
@@ -882,19 +910,17 @@ __device__ __forceinline__ void epilogue_wgrad(const Params &P, uint32_t taddr, 
     if (!zero) {
       tmem_ld32(taddr + c * 32, r);
       tmem_ld_wait();
-    }
-    if (!dst || col >= P.N) continue;
-    if (col + 32 <= P.N && (P.N & 3) == 0) {
-      float4 *d4 = reinterpret_cast<float4 *>(dst + col);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        d4[q] = zero ? make_float4(0.f, 0.f, 0.f, 0.f)
-                     : make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                   __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
     } else {
 #pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = 0u;
+    }
+    if (col >= P.N) break;                                      // the same for the whole CTA
+    if (col + 32 <= P.N && (P.N & 3) == 0) {
+      store_rows_at(stg, r, dst ? reinterpret_cast<char *>(dst + col) : nullptr, lane);
+    } else if (dst) {
+#pragma unroll
       for (int i = 0; i < 32; ++i)
-        if (col + i < P.N) dst[col + i] = zero ? 0.0f : __uint_as_float(r[i]);
+        if (col + i < P.N) dst[col + i] = __uint_as_float(r[i]);
     }
   }
 }
@@ -1173,7 +1199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ? reinterpret_cast<float *>(P.out) + ((int64_t)tl.g * P.split_m + row) * P.N
                     : reinterpret_cast<float *>(P.out2) +
                           ((int64_t)tl.g * (P.M - P.split_m) + row - P.split_m) * P.N;
-        epilogue_wgrad(P, taddr, zero, dst, tl.n * P.bnh);
+        epilogue_wgrad(P, taddr, zero, dst, tl.n * P.bnh, stg, lane);
       } else if (in_tail && kb0 > 0) {
         sk_write(P, (int)blockIdx.x, r_cta, taddr);              // a later piece of the tile
       } else {
@@ -1283,7 +1309,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int base = 0; base < P.G; base += 32) {
       const int g = base + lane;
       int tiles = 0;
-      if (g < P.G) {
+      if (g < P.G && P.kgroup) {
+        // K-grouped: group g owns K columns [kseg[g], kseg[g+1]); rows = its k-blocks
+        const int k0 = P.kseg[g], k1 = P.kseg[g + 1];
+        if (k0 < 0 || k1 < k0 || (k0 % BK) != 0 || (int64_t)k1 > P.a_rows) {
+          raise_error(P.err, kErrBadIndex);
+          s_off[g] = 0;
+          s_rows[g] = 0;
+        } else {
+          s_off[g] = k0;
+          s_rows[g] = (k1 - k0) / BK;
+        }
+        tiles = ((P.M + PM - 1) / PM) * P.nt;
+      } else if (g < P.G) {
         int off = 0, rows = 0;
         if (g < P.n_routed) {
           off = P.offsets[g];
@@ -1344,6 +1382,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int64_t a_row;
       int b_row;
       const CUtensorMap *ma = rows_of(tl, a_row, b_row);
+      int kx = 0;                      // K coordinate of k-block 0
+      if (P.kgroup) {
+        // weight gradient: A [M, K] rows of this CTA, B [N, K] half of the tile
+        ma = &map_a;
+        a_row = (int64_t)tl.m * PM + (int64_t)rank * BM;
+        b_row = tl.n * P.bnh + (int)rank * (P.bn / 2);
+        kx = s_off[tl.g];
+        kb0 = 0;
+        kb1 = s_rows[tl.g];
+      }
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
         uint8_t *sa = smem + (size_t)stage * stage_bytes;
@@ -1355,7 +1403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         }
-        if (a_by_tma) tma_load_2d_pair(sa, ma, fb, kb * BK, (int)a_row);
+        if (a_by_tma) tma_load_2d_pair(sa, ma, fb, kx + kb * BK, (int)a_row);
         if (P.b_mn) {
           // this CTA's 128 N columns of B stored [K][N]: two boxes of 64 N x 64 K
           const bool first = kb < P.b_kb_split;
@@ -1364,7 +1412,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tma_load_2d_pair(sb + j * 8192, first ? &map_b : &map_b3, fb,
                              tl.n * P.bnh + (int)rank * (P.bn / 2) + j * 64, y);
         } else {
-          tma_load_2d_pair(sb, mb, fb, kb * BK, b_row);
+          tma_load_2d_pair(sb, mb, fb, kx + kb * BK, b_row);
         }
         if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
       }
@@ -1382,6 +1430,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     bool ok = true;
     while (ok && sc.next(tile, kb0, kb1, part)) {
+      if (P.kgroup) {
+        const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
+        kb0 = 0;
+        kb1 = s_rows[tl.g];
+      }
       if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
@@ -1467,7 +1520,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
       const bool in_tail = sk && tile >= sc.dp_limit;
-      if (in_tail && kb0 > 0) {
+      if (P.kgroup) {
+        // weight gradient tile: rows of group g's [M, N] output (split at split_m)
+        const int row = tl.m * PM + (int)rank * BM + r_cta;
+        const bool zero = s_rows[tl.g] == 0;
+        float *dst = nullptr;
+        if (row < P.M)
+          dst = row < P.split_m
+                    ? reinterpret_cast<float *>(P.out) + ((int64_t)tl.g * P.split_m + row) * P.N
+                    : reinterpret_cast<float *>(P.out2) +
+                          ((int64_t)tl.g * (P.M - P.split_m) + row - P.split_m) * P.N;
+        epilogue_wgrad(P, taddr, zero, dst, tl.n * P.bnh, stg, lane);
+      } else if (in_tail && kb0 > 0) {
         sk_write(P, 2 * pair + (int)rank, r_cta, taddr);        // a later piece of the tile
       } else {
         const bool routed = tl.g < P.n_routed;
@@ -1661,9 +1725,11 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
     return cudaErrorInvalidValue;
 
   // CTA pairs for the expert GEMMs whose groups are long enough that 256-row
-  // tiles waste little (average routed rows per expert >= MOE_PAIR_MIN_ROWS)
-  const bool pair = !g.kgroup && g.n_routed > 0 && P.bn == 256 &&
-                    g.max_routed_rows / g.n_routed >= MOE_PAIR_MIN_ROWS;
+  // tiles waste little (average routed rows per expert >= MOE_PAIR_MIN_ROWS),
+  // and for weight gradients of at least 256 rows
+  const bool pair = P.bn == 256 &&
+                    ((!g.kgroup && g.n_routed > 0 && g.max_routed_rows / g.n_routed >= MOE_PAIR_MIN_ROWS) ||
+                     (g.kgroup && g.M >= 2 * BM && MOE_PAIR_WGRAD));
   CUtensorMap ma, mas, mb, mb3;
   const uint32_t box_b = (swiglu_b(g.epi) || pair) ? 128u : (uint32_t)P.bn;
   // K groups: A is [M, K] and B [N, K] with all groups' K columns side by side
@@ -1698,7 +1764,8 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
 
   if (pair) {
     const int64_t pt_routed = (g.max_routed_rows + 2 * BM - 1) / (2 * BM) + g.n_routed;
-    const int64_t pt_static = (int64_t)g.n_static * ((g.rows_static + 2 * BM - 1) / (2 * BM));
+    const int64_t pt_static =
+        (int64_t)g.n_static * (((g.kgroup ? g.M : g.rows_static) + 2 * BM - 1) / (2 * BM));
     const int64_t pair_tiles = (pt_routed + pt_static) * P.nt;
     const size_t psmem = (size_t)kPairStages * (kABytes + (size_t)(P.bn / 2) * BK * 2) + 1024 +
                          4 * kStageBytesPerWarp;
