@@ -7,7 +7,9 @@
 // before any second choice, lower token first), in units of 32 tokens:
 //   hist_units    per-unit expert histogram (the gate kernel writes it when
 //                 it runs first, so moe_forward skips this launch)
-//   unit_sums     per-expert totals of each block of 32 units
+//   unit_sums     per-expert totals of each block of 32 units (skipped for
+//                 small histograms without local groups: the rank kernel's
+//                 blocks then sum all units before theirs themselves)
 //   rank_units    per block: bases from the earlier blocks' totals and an
 //                 in-block scan, counts / kept rows (min(n_e, C) or
 //                 ceil(n_e*num/den)) / row offsets; then the stable rank of
@@ -179,7 +181,19 @@ __global__ void __launch_bounds__(1024, 1) rank_units_kernel(
   // 1. totals of the blocks before this one (in its group), and of all blocks
   const int G = max(1, (int)blockDim.x / E);
   const int g = threadIdx.x / E, e_g = threadIdx.x - g * E;
-  if (lgroups == 1) {
+  if (lgroups == 1 && bsum == nullptr) {
+    // small histograms: every block sums the units itself (no unit_sums launch)
+    int pre = 0, tot = 0;
+    if (g < G) {
+      for (int u = g; u < upg; u += G) {
+        const int v = hist[(int64_t)u * E + e_g];
+        tot += v;
+        if (u < u_begin) pre += v;
+      }
+      s_part[threadIdx.x] = pre;
+      s_part2[threadIdx.x] = tot;
+    }
+  } else if (lgroups == 1) {
     int pre = 0, tot = 0;
     if (g < G) {
       for (int bb = g; bb < nb; bb += G) {
@@ -536,8 +550,13 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
                       nu, ug.nbg, hist, err);
     if (e != cudaSuccess) return e;
   }
-  e = launch_kernel(unit_sums_kernel, nb, 1024, 0, s, hist, ug.upg, ug.bpg, E, bsum);
-  if (e != cudaSuccess) return e;
+  // without local groups and with at most 16K histogram entries, the rank
+  // kernel's blocks sum the units before them themselves (one launch fewer)
+  const bool own_sums = ug.G == 1 && (int64_t)nu * E <= 16384;
+  if (!own_sums) {
+    e = launch_kernel(unit_sums_kernel, nb, 1024, 0, s, hist, ug.upg, ug.bpg, E, bsum);
+    if (e != cudaSuccess) return e;
+  }
   const size_t rank_smem = ((size_t)kUnitsPerBlock * E + 6 * E + 2 + 2048) * sizeof(int);
   if (rank_smem > 48 * 1024) {
     e = cudaFuncSetAttribute(rank_units_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -545,7 +564,8 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
     if (e != cudaSuccess) return e;
   }
   e = launch_kernel(rank_units_kernel, nb, 1024, rank_smem, s, topk_idx, topk_gate, T, c->k, E,
-                    ug.nbg, ug.upg, ug.bpg, nb, hist, bsum, c->capacity, c->keep_num, c->keep_den,
+                    ug.nbg, ug.upg, ug.bpg, nb, hist, own_sums ? nullptr : bsum, c->capacity,
+                    c->keep_num, c->keep_den,
                     keepfrac, counts,
                     cnt_off, kept, offsets, n_dropped, tok_rows, row_token, row_gate, sorted_q);
   if (e != cudaSuccess) return e;
