@@ -54,6 +54,10 @@ constexpr int kMaxGroups = 320;
 #ifndef MOE_PAIR_MIN_ROWS
 #define MOE_PAIR_MIN_ROWS 384
 #endif
+// CTA pairs: stages of two 64-wide k-blocks where K is a multiple of 128
+#ifndef MOE_PAIR_BK128
+#define MOE_PAIR_BK128 1
+#endif
 // K-grouped weight gradients on CTA pairs as well
 #ifndef MOE_PAIR_WGRAD
 #define MOE_PAIR_WGRAD 1
@@ -1246,15 +1250,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 // complete on the even CTA's full barrier; the MMA commits arrive on the
 // empty / accumulator-full barriers of both CTAs; both CTAs' epilogues arrive
 // on the even CTA's accumulator-empty barrier.  No load is multicast.
+//
+// BKS = 2: stages of two 64-wide k-blocks (three 64 KB stages instead of six
+// of 32 KB, eight MMAs and one barrier round trip per stage), for K a
+// multiple of 128 without the row gather, K-major B only.
 constexpr int kPairStages = 6;
+constexpr int kPairStages2 = 3;
 
-template <int EPI>
+template <int EPI, int BKS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
                              const __grid_constant__ CUtensorMap map_a_static,
                              const __grid_constant__ CUtensorMap map_b,
                              const __grid_constant__ CUtensorMap map_b3, const Params P) {
   constexpr int PM = 2 * BM;                         // rows per pair tile
+  constexpr int STAGES = BKS == 2 ? kPairStages2 : kPairStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ int s_prefix[kMaxGroups + 1];
   __shared__ int s_off[kMaxGroups];
@@ -1270,14 +1280,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~(uintptr_t)1023);
   const uint32_t b_bytes = (uint32_t)(P.bn / 2) * BK * 2;       // this CTA's half of B
-  const uint32_t stage_bytes = kABytes + b_bytes;
+  const uint32_t stage_bytes = BKS * (kABytes + b_bytes);       // A blocks, then B blocks
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
   const bool gather = P.gather_rows != nullptr;
   if (tid == 32) {
-    for (int st = 0; st < kPairStages; ++st) {
+    for (int st = 0; st < STAGES; ++st) {
       // the even CTA's: its expect_tx arrival, then both CTAs' gather warps
       mbar_init(&full_bar[st], 1 + (gather ? 2 * kGatherThreads / 32 : 0));
       mbar_init(&empty_bar[st], 1);
@@ -1354,7 +1364,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
 
   const uint32_t tmem_base = s_tmem_base;
-  const int KB = P.K / BK;
+  const int KB = P.K / (BK * BKS);                     // stages of K per tile
   const bool sk = P.sk_part != nullptr;
   Sched sc;
   sc.init(s_prefix[P.G], KB, npairs, pair, sk, 1);
@@ -1395,7 +1405,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
         uint8_t *sa = smem + (size_t)stage * stage_bytes;
-        uint8_t *sb = sa + kABytes;
+        uint8_t *sb = sa + BKS * kABytes;
         const uint32_t fb = smem_u32(&full_bar[stage]) & 0xFEFFFFFFu;   // the even CTA's barrier
         const bool a_by_tma = !(gather && tl.g < P.n_routed);          // else the gather warps
         if (rank == 0) {
@@ -1403,7 +1413,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         }
-        if (a_by_tma) tma_load_2d_pair(sa, ma, fb, kx + kb * BK, (int)a_row);
+        if (a_by_tma) {
+#pragma unroll
+          for (int q = 0; q < BKS; ++q)
+            tma_load_2d_pair(sa + q * kABytes, ma, fb, kx + (kb * BKS + q) * BK, (int)a_row);
+        }
         if (P.b_mn) {
           // this CTA's 128 N columns of B stored [K][N]: two boxes of 64 N x 64 K
           const bool first = kb < P.b_kb_split;
@@ -1412,13 +1426,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tma_load_2d_pair(sb + j * 8192, first ? &map_b : &map_b3, fb,
                              tl.n * P.bnh + (int)rank * (P.bn / 2) + j * 64, y);
         } else {
-          tma_load_2d_pair(sb, mb, fb, kx + kb * BK, b_row);
+#pragma unroll
+          for (int q = 0; q < BKS; ++q)
+            tma_load_2d_pair(sb + q * b_bytes, mb, fb, kx + (kb * BKS + q) * BK, b_row);
         }
-        if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
     }
     if (!ok && rank == 0) {
-      for (int st = 0; st < kPairStages; ++st)
+      for (int st = 0; st < STAGES; ++st)
         if (armed & (1u << st)) mbar_wait_drain(&full_bar[st], (armed_parity >> st) & 1u);
     }
   } else if (warp == 1 && lane == 0 && rank == 0) {
@@ -1442,15 +1458,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (!mbar_wait<true>(&full_bar[stage], phase, &s_abort, P.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + (size_t)stage * stage_bytes);
-        const uint32_t b_addr = a_addr + kABytes;
+        const uint32_t b_addr = a_addr + BKS * kABytes;
 #pragma unroll
-        for (int k = 0; k < BK / kUmmaK; ++k) {
-          const uint64_t bdesc = P.b_mn ? mn128_desc(b_addr + k * 2048) : sw128_desc(b_addr + k * kUmmaK * 2);
-          umma_bf16_pair(d_tmem, sw128_desc(a_addr + k * kUmmaK * 2), bdesc, idesc,
-                         (kb > kb0 || k > 0) ? 1u : 0u);
+        for (int q = 0; q < BKS; ++q) {
+#pragma unroll
+          for (int k = 0; k < BK / kUmmaK; ++k) {
+            const uint32_t bq = b_addr + q * b_bytes;
+            const uint64_t bdesc = P.b_mn ? mn128_desc(bq + k * 2048) : sw128_desc(bq + k * kUmmaK * 2);
+            umma_bf16_pair(d_tmem, sw128_desc(a_addr + q * kABytes + k * kUmmaK * 2), bdesc, idesc,
+                           (kb > kb0 || q > 0 || k > 0) ? 1u : 0u);
+          }
         }
         umma_commit_pair_both(&empty_bar[stage]);
-        if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
       umma_commit_pair_both(&accf_bar[acc]);
@@ -1461,7 +1481,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (gather && (warp == 2 || warp == 3)) {
     // --------------- gather of this CTA's 128 routed A rows ---------------
     constexpr int kLag = MOE_GATHER_LAG_PAIR;
-    static_assert(kLag >= 0 && kLag < kPairStages, "gather lag below the ring depth");
+    static_assert(kLag >= 0 && kLag < STAGES, "gather lag below the ring depth");
     const int gt = tid - 64;
     int stage = 0;
     uint32_t phase = 0;
@@ -1493,22 +1513,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           cp_async_wait<kLag>();
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) arrive_full((int)(arrived % kPairStages));   // one arrival per warp
+          if (lane == 0) arrive_full((int)(arrived % STAGES));   // one arrival per warp
           ++arrived;
         }
-        if (++stage == kPairStages) { stage = 0; phase ^= 1u; }
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
     }
     cp_async_wait<0>();
     fence_proxy_async_smem();
     __syncwarp();
     for (; arrived < issued; ++arrived)
-      if (lane == 0) arrive_full((int)(arrived % kPairStages));
+      if (lane == 0) arrive_full((int)(arrived % STAGES));
   } else if (warp >= 4) {
     // -------------------------------- epilogue --------------------------------
     const int ew = warp - 4;
     const int r_cta = ew * 32 + lane;                 // row within this CTA's half
-    uint8_t *stg = smem + (size_t)kPairStages * stage_bytes + (size_t)ew * kStageBytesPerWarp;
+    uint8_t *stg = smem + (size_t)STAGES * stage_bytes + (size_t)ew * kStageBytesPerWarp;
     const uint32_t acce_even0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
     const uint32_t acce_even1 = mapa_shared(smem_u32(&acce_bar[1]), 0);
     int acc = 0;
@@ -1619,11 +1639,11 @@ cudaError_t launch_epi(const GroupedGemm &g, const Params &P, const CUtensorMap 
 
 // CTA-pair launch: as many 2-CTA clusters as fit at once (one CTA per SM),
 // fewer when there are fewer tiles.
-template <int EPI>
+template <int EPI, int BKS>
 cudaError_t launch_pair(const Params &P, const CUtensorMap &ma, const CUtensorMap &mas,
                         const CUtensorMap &mb, const CUtensorMap &mb3, int64_t max_tiles,
                         size_t smem, cudaStream_t s) {
-  auto kern = grouped_gemm_pair_kernel<EPI>;
+  auto kern = grouped_gemm_pair_kernel<EPI, BKS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   static int max_clusters[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -1767,11 +1787,21 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
     const int64_t pt_static =
         (int64_t)g.n_static * (((g.kgroup ? g.M : g.rows_static) + 2 * BM - 1) / (2 * BM));
     const int64_t pair_tiles = (pt_routed + pt_static) * P.nt;
-    const size_t psmem = (size_t)kPairStages * (kABytes + (size_t)(P.bn / 2) * BK * 2) + 1024 +
-                         4 * kStageBytesPerWarp;
+    // stages of two k-blocks where K allows (no gather, K-major B, no K
+    // groups) and the GEMM is large: measured 10% faster expert GEMMs on the
+    // Mixtral shape and 5% on DeepSeekMoE's, 1% slower on the GShard shape's
+    // 3.4e10-MAC GEMMs
+    const double macs = (double)(g.max_routed_rows + (int64_t)g.n_static * g.rows_static) * g.N *
+                        g.K * (swiglu_b(g.epi) ? 2 : 1);
+    const bool bk2 = MOE_PAIR_BK128 && !g.kgroup && !g.b_mn && !g.gather_rows &&
+                     g.K % (2 * BK) == 0 && macs >= 2e11;
+    const size_t psmem = (bk2 ? (size_t)kPairStages2 * 2 : (size_t)kPairStages) *
+                             (kABytes + (size_t)(P.bn / 2) * BK * 2) +
+                         1024 + 4 * kStageBytesPerWarp;
 #define MOE_PAIR_CASE(E_)                                                            \
   case E_:                                                                           \
-    return launch_pair<E_>(P, ma, mas, mb, mb3, pair_tiles, psmem, s);
+    return bk2 ? launch_pair<E_, 2>(P, ma, mas, mb, mb3, pair_tiles, psmem, s)       \
+               : launch_pair<E_, 1>(P, ma, mas, mb, mb3, pair_tiles, psmem, s);
     switch (g.epi) {
       MOE_PAIR_CASE(kEpiStoreF32)
       MOE_PAIR_CASE(kEpiRelu)
