@@ -85,6 +85,25 @@ __device__ __forceinline__ void halve(float (&a)[EMAX], int o, int lane) {
   }
 }
 
+// acc + sum over the 8 bf16 pairs of two 16-byte chunks, in element order:
+// fma.rn.f32.bf16 multiplies the bf16 operands exactly and rounds once into
+// the fp32 accumulator, as fmaf on the widened values does, with no
+// widening instructions
+__device__ __forceinline__ float dot8_bf16(const uint4 x, const uint4 w, float acc) {
+  asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
+      "mov.b32 {xl, xh}, %1;\n\tmov.b32 {wl, wh}, %5;\n\t"
+      "fma.rn.f32.bf16 %0, xl, wl, %0;\n\tfma.rn.f32.bf16 %0, xh, wh, %0;\n\t"
+      "mov.b32 {xl, xh}, %2;\n\tmov.b32 {wl, wh}, %6;\n\t"
+      "fma.rn.f32.bf16 %0, xl, wl, %0;\n\tfma.rn.f32.bf16 %0, xh, wh, %0;\n\t"
+      "mov.b32 {xl, xh}, %3;\n\tmov.b32 {wl, wh}, %7;\n\t"
+      "fma.rn.f32.bf16 %0, xl, wl, %0;\n\tfma.rn.f32.bf16 %0, xh, wh, %0;\n\t"
+      "mov.b32 {xl, xh}, %4;\n\tmov.b32 {wl, wh}, %8;\n\t"
+      "fma.rn.f32.bf16 %0, xl, wl, %0;\n\tfma.rn.f32.bf16 %0, xh, wh, %0;\n\t}"
+      : "+f"(acc)
+      : "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w), "r"(w.x), "r"(w.y), "r"(w.z), "r"(w.w));
+  return acc;
+}
+
 // 16-byte chunk of x or W_r widened to fp32
 template <bool BF16>
 __device__ __forceinline__ void widen_chunk(const uint4 v, float (&f)[BF16 ? 8 : 4]) {
@@ -163,17 +182,23 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_gate_kernel(const GatePa
       for (int i = 0; i < NB; ++i) {
         const int c = c0 + lane + 32 * i;
         if (c >= nchunk) break;
-        float xf[EPV];
-        widen_chunk<BF16>(xb[i], xf);
+        if constexpr (BF16) {
 #pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-          if (e < E) {
-            float wf[EPV];
-            widen_chunk<BF16>(s_w[(size_t)e * nchunk + c], wf);
-            float a = acc[e];
+          for (int e = 0; e < EMAX; ++e)
+            if (e < E) acc[e] = dot8_bf16(xb[i], s_w[(size_t)e * nchunk + c], acc[e]);
+        } else {
+          float xf[EPV];
+          widen_chunk<BF16>(xb[i], xf);
 #pragma unroll
-            for (int h = 0; h < EPV; ++h) a = fmaf(xf[h], wf[h], a);
-            acc[e] = a;
+          for (int e = 0; e < EMAX; ++e) {
+            if (e < E) {
+              float wf[EPV];
+              widen_chunk<BF16>(s_w[(size_t)e * nchunk + c], wf);
+              float a = acc[e];
+#pragma unroll
+              for (int h = 0; h < EPV; ++h) a = fmaf(xf[h], wf[h], a);
+              acc[e] = a;
+            }
           }
         }
       }
