@@ -178,6 +178,25 @@ __global__ void __launch_bounds__(1024, 1) rank_units_kernel(
   const int lgroups = nb / bpg;                       // local groups
   const int my_group = b / bpg;
 
+  // this warp's unit (u = g*upg + r*nbg + bl) and its lane's assignment,
+  // loaded now so that the loads overlap the scans below
+  const int u = u_begin + warp;
+  const bool unit_live = u < u_end;
+  int r = 0, e = -1;
+  int64_t t = 0;
+  float gate = 0.f;
+  if (unit_live) {
+    const int rem = u - my_group * upg;
+    r = rem / nbg;
+    const int64_t bu = (int64_t)my_group * nbg + (rem - r * nbg);
+    t = bu * kUnitTokens + lane;
+    if (t < T) {
+      e = topk_idx[t * k + r];
+      if (e < 0 || e >= E) e = -1;                       // reported by the histogram
+      if (!keep_fraction && e >= 0) gate = topk_gate[t * k + r];
+    }
+  }
+
   // 1. totals of the blocks before this one (in its group), and of all blocks
   const int G = max(1, (int)blockDim.x / E);
   const int g = threadIdx.x / E, e_g = threadIdx.x - g * E;
@@ -295,18 +314,8 @@ __global__ void __launch_bounds__(1024, 1) rank_units_kernel(
   }
   __syncthreads();
 
-  // 4. one warp per unit (u = g*upg + r*nbg + bl)
-  const int u = u_begin + warp;
-  if (u >= u_end) return;
-  const int rem = u - my_group * upg;
-  const int r = rem / nbg;
-  const int64_t bu = (int64_t)my_group * nbg + (rem - r * nbg);
-  const int64_t t = bu * kUnitTokens + lane;
-  int e = -1;
-  if (t < T) {
-    e = topk_idx[t * k + r];
-    if (e < 0 || e >= E) e = -1;                         // reported by the histogram
-  }
+  // 4. one warp per unit: the rank of each assignment inside its expert
+  if (!unit_live) return;
   const unsigned peers = __match_any_sync(0xffffffffu, e);
   const int rank = e >= 0 ? s_base[warp * E + e] + __popc(peers & ((1u << lane) - 1u)) : 0;
   if (keep_fraction) {
@@ -318,7 +327,7 @@ __global__ void __launch_bounds__(1024, 1) rank_units_kernel(
   if (e >= 0) tok_rows[t * k + r] = slot;
   if (keep) {
     row_token[slot] = (int32_t)t;
-    row_gate[slot] = topk_gate[t * k + r];
+    row_gate[slot] = gate;
   }
 }
 
