@@ -151,6 +151,7 @@ __global__ void seg_offsets_kernel(const int32_t *__restrict__ offsets, int E, i
 // is r = offsets[e] + i, read at map[r] (null: r); scale_i = scale[r] (null:
 // 1).  Row i of shared group s is read at shared_base + s * shared_stride + i.
 // 64 x 64 tiles: segments are 64-aligned, so a tile never straddles two.
+constexpr int kMaxSegGroups = kMaxExperts + 8;         // routed + shared experts
 struct SegSrc {
   const __nv_bfloat16 *src;
   int64_t ld;                // elements per source row
@@ -168,20 +169,25 @@ __global__ void __launch_bounds__(256) transpose_segments_kernel(SegSrc S_, cons
   __shared__ uint16_t tile[kTT][kTP];
   __shared__ int64_t s_row[kTT];
   __shared__ float s_scale[kTT];
+  __shared__ int s_kseg[kMaxSegGroups + 1];
   pdl_wait();
   pdl_trigger();
   const int k0 = blockIdx.x * kTT, c0 = blockIdx.y * kTT;
-  if (k0 >= kseg[G]) return;                            // past the last segment
+  // the segment offsets into shared memory in one parallel load, so that the
+  // search below costs no chain of dependent global loads
+  for (int i = threadIdx.x; i <= G; i += blockDim.x) s_kseg[i] = kseg[i];
+  __syncthreads();
+  if (k0 >= s_kseg[G]) return;                          // past the last segment
   int lo = 0, hi = G - 1;                               // group holding column k0
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (kseg[mid] <= k0) lo = mid;
+    if (s_kseg[mid] <= k0) lo = mid;
     else hi = mid - 1;
   }
   const int g = lo;
   const int64_t len = g < E ? (int64_t)(offsets[g + 1] - offsets[g]) : shared_len;
   if (threadIdx.x < kTT) {
-    const int64_t li = (int64_t)(k0 - kseg[g]) + threadIdx.x;    // row of the segment
+    const int64_t li = (int64_t)(k0 - s_kseg[g]) + threadIdx.x;  // row of the segment
     int64_t row = -1;
     float sc = 1.0f;
     if (li < len) {
@@ -407,6 +413,7 @@ cudaError_t launch_transpose_segments(const void *src, int64_t ld, const int32_t
                                       const int32_t *kseg,
                                       int E, int G, int C, int64_t kp_max, void *out, uint32_t *err,
                                       cudaStream_t s) {
+  if (G < 1 || G > kMaxSegGroups) return cudaErrorInvalidValue;
   SegSrc S_{static_cast<const __nv_bfloat16 *>(src), ld, map, scale, shared_base, shared_stride};
   dim3 grid((unsigned)(kp_max / kTT), (unsigned)((C + kTT - 1) / kTT)), block(256);
   return launch_kernel(transpose_segments_kernel, grid, block, 0, s, S_, offsets, kseg, E, G, C,
