@@ -4,7 +4,9 @@
 // in the layer dtype; here each token sums its rows: routed rows in the
 // token's k-rank order (expert choice: ascending expert), then shared experts
 // 0..S-1, fp32 accumulation, one rounding to the output dtype.  One warp per
-// token, 16-byte vectors.
+// token, 16-byte vectors.  (moe_forward with at most two rows a token adds
+// the rows into y in the down-projection's epilogue instead, with the same
+// result; this kernel then does not run.)
 #include "device_common.cuh"
 #include "moe_internal.h"
 

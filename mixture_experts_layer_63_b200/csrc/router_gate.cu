@@ -9,8 +9,8 @@
 // Lane l of a token's warp holds experts l, l+32, l+64, ...  The arithmetic
 // is the fixed fp32 recipe shared with the oracle: m = max, z = l - m (one
 // rounded subtraction), exp_det, the denominator summed sequentially in
-// ascending expert order (a shuffle chain, so the order is that of a single
-// thread), IEEE division.  Top-k runs k rounds of a warp arg-max on the fp32
+// ascending expert order (lane 0 adds the exponentials one at a time from
+// shared memory, the order of a single thread), IEEE division.  Top-k runs k rounds of a warp arg-max on the fp32
 // logits: larger value first, lower expert index on ties.
 //
 // The kernel also counts, per 32-token unit and per rank j, how many tokens
@@ -18,9 +18,11 @@
 // permutation's scan consumes (see permute.cu).
 //
 // Router logits: for few experts (E <= 32, W_r small enough for shared
-// memory) the warp computes them itself from x and W_r with fp32
-// accumulation (fused router: x is read once, no logits round trip);
-// otherwise they come from the tcgen05 GEMM in gemm_sm100.cu.
+// memory; bf16 up to d_model = 2048) the warp computes them itself from x
+// and W_r with fp32 accumulation (fused router: x is read once, no logits
+// round trip); otherwise they come from the tcgen05 GEMM in gemm_sm100.cu.
+// With the combine folded into the down-projection the kernel also zeroes
+// its tokens' rows of y.
 #include <math.h>
 
 #include "device_common.cuh"
