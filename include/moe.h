@@ -1,6 +1,6 @@
 /*
  * moe.h - C ABI of libmoe.so: the forward pass of a sparse Mixture-of-Experts
- * FFN layer on one NVIDIA B200 (sm_100a).
+ * FFN layer on one NVIDIA B200 (sm_100a), and its backward pass (moe_backward).
  *
  * The layer, in five steps (all arithmetic runs in this library's CUDA
  * kernels):
