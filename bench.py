@@ -46,8 +46,8 @@ DEFAULT_WORKLOAD = "gshard"
 # profiles/, with the sha256 (first 16 hex digits) of the kernel source they
 # were taken at; a value is reported only while the source is unchanged.
 NCU_TRAFFIC: dict[str, dict] = {
-    # profiles/gemm_gshard_ncu.md: up 151.11 + 40.66 MB, down 220.16 + 10.15 MB
-    "gshard": {"bytes": 422_082_304, "src": "a274bdab48a8ec57"},
+    # profiles/gemm_gshard_ncu.md: up 151.09 + 41.15 MB, down 220.18 + 9.75 MB
+    "gshard": {"bytes": 422_169_088, "src": "a9de9705dc80e5bb"},
 }
 
 

@@ -618,19 +618,6 @@ __device__ __forceinline__ void sk_done(const Params &P, const Fixup &F) {
 }
 
 // --------------------------------- epilogues ---------------------------------
-__device__ __forceinline__ void store_bf16x32(void *dst, const float (&v)[32]) {
-  uint4 *p = reinterpret_cast<uint4 *>(dst);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 w;
-    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-    p[q] = w;
-  }
-}
-
 __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16 *src, float (&v)[32]) {
   const uint4 *p = reinterpret_cast<const uint4 *>(src);
 #pragma unroll
@@ -1628,7 +1615,7 @@ int device_sms() {
 }
 
 template <int EPI>
-cudaError_t launch_epi(const GroupedGemm &g, const Params &P, const CUtensorMap &ma,
+cudaError_t launch_epi(const Params &P, const CUtensorMap &ma,
                        const CUtensorMap &mas, const CUtensorMap &mb, const CUtensorMap &mb3,
                        int grid, size_t smem, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
@@ -1818,7 +1805,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   }
 #define MOE_ONE_CASE(E_)                                                             \
   case E_:                                                                           \
-    return launch_epi<E_>(g, P, ma, mas, mb, mb3, grid, smem, s);
+    return launch_epi<E_>(P, ma, mas, mb, mb3, grid, smem, s);
   switch (g.epi) {
     MOE_ONE_CASE(kEpiStoreF32)
     MOE_ONE_CASE(kEpiRelu)
