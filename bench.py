@@ -214,7 +214,8 @@ class OracleTimer:
         self.w2 = _DeviceExperts(inp.w2)
         self.w3 = _DeviceExperts(inp.w3)
         Tg = w.T // max(1, w.local_groups)
-        cap = O.capacity_from_factor(Tg, w.E, w.k, w.capacity_factor) if w.mode == "tc" else 0
+        cf = float(np.float32(w.capacity_factor))
+        cap = min(O.capacity_from_factor(Tg, w.E, w.k, cf), Tg) if w.mode == "tc" else 0
         self.state = None if inp.route_state is None else inp.route_state.cpu().numpy()
         self.cfg = O.OracleConfig(E=w.E, S=w.S, k=w.k, act=w.act, mode=w.mode, capacity=cap,
                                   keep_num=w.keep_num, keep_den=w.keep_den,

@@ -31,8 +31,11 @@
  * Conventions that hold for every entry point:
  *   - Ownership: the caller owns every buffer.  The library allocates no
  *     device memory on any path; scratch lives in the caller's workspace
- *     (moe_query_sizes gives its size).  Every tensor pointer is a DEVICE
- *     pointer on the current CUDA device; the structs are host memory.
+ *     (moe_query_sizes gives its size).  The one exception is the fixed
+ *     array of MOE_PERMUTE_NOALLOC_SCRATCH_BYTES compiled into the library
+ *     for moe_permute_noalloc, which every GPU that loads the library holds
+ *     until the process exits.  Every tensor pointer is a DEVICE pointer on
+ *     the current CUDA device; the structs are host memory.
  *   - Layout: row-major.  x [T, d]; w_router [E, d]; w1, w3 [E+S, f, d];
  *     w2 [E+S, d, f] (each output neuron's weights contiguous along its input
  *     dimension); experts 0..E-1 are routed, E..E+S-1 shared.  Element type
@@ -94,7 +97,18 @@ typedef enum moe_mode { MOE_TOKEN_CHOICE = 0, MOE_EXPERT_CHOICE = 1 } moe_mode;
  *            gate = p; u = route_state [E], the experts' utilisation. */
 typedef enum moe_route_rule { MOE_ROUTE_SOFTMAX = 0, MOE_ROUTE_BIAS = 1, MOE_ROUTE_LOAD = 2 } moe_route_rule;
 
-/* The layer.  Capacity, keep-fraction and expert choice are exclusive. */
+/* The layer.  Capacity, keep-fraction and expert choice are exclusive.
+ *
+ * Expert capacity (GShard section 1 of "MoE技术演进": each expert takes at
+ * most C = O(N/E) tokens, the overflow passes to the residual; with local
+ * group dispatching the capacity of a group of N/G tokens, 2N/(G*E) for
+ * top-2 at factor 1).  The library derives C from the factor:
+ *     C = ceil(capacity_factor * k * T / E)          (one group)
+ *     C = ceil(capacity_factor * k * (T / G) / E)    (local_groups G > 1, per group)
+ * evaluated exactly for the fp32 value given (no rounding before the
+ * ceiling; 0.1f is slightly above 0.1, so 0.1f * 10 gives 2) and clamped to
+ * the group's token count (an expert receives at most one assignment per
+ * token).  moe_sizes.capacity reports C. */
 typedef struct moe_config {
   int64_t T;           /* tokens in this call (>= 1)                                */
   int32_t d_model;     /* d                                                         */
@@ -102,7 +116,7 @@ typedef struct moe_config {
   int32_t S;           /* shared experts, gate 1 for every token (>= 0)             */
   int32_t k;           /* experts per token, token choice (1 <= k <= E)             */
   int32_t d_ff;        /* expert hidden size f (d_ff, or d_moe for SwiGLU)          */
-  int32_t capacity;    /* token choice: max rows per routed expert; <= 0 unlimited  */
+  float capacity_factor; /* token choice: expert capacity factor cf; <= 0 unlimited  */
   int32_t keep_num;    /* token choice: expert e keeps ceil(n_e*num/den) of its n_e */
   int32_t keep_den;    /*   assignments by affinity; den = 0: keep all              */
   int32_t ec_capacity; /* expert choice: tokens per expert C (1 <= C <= T)          */
@@ -115,9 +129,9 @@ typedef struct moe_config {
   int32_t route_rule;  /* moe_route_rule (token choice; SOFTMAX in expert choice)   */
   float route_alpha;   /* MOE_ROUTE_LOAD: alpha                                     */
   int32_t local_groups;/* GShard local groups G (0 or 1: one group): T/G contiguous  */
-                       /*   tokens per group, each dispatching on its own with      */
-                       /*   `capacity` rows per expert; needs capacity > 0, T % G   */
-                       /*   == 0 and (T/G) % 32 == 0                                */
+                       /*   tokens per group, each dispatching on its own with C    */
+                       /*   rows per expert; needs capacity_factor > 0, T % G == 0  */
+                       /*   and (T/G) % 32 == 0                                     */
   int32_t reserved;    /* 0                                                         */
 } moe_config;
 
@@ -128,6 +142,11 @@ typedef struct moe_sizes {
   int64_t tok_rows_len;    /* entries of tok_rows: T*k (token choice) or E*T (expert choice)     */
   size_t step_workspace;   /* bytes of workspace the step entry points need                     */
   size_t workspace;        /* bytes of workspace moe_forward needs (>= step_workspace)          */
+  int64_t capacity;        /* token choice: expert capacity C the library derived from          */
+                           /*   capacity_factor (per local group); 0: unlimited or not token    */
+                           /*   choice.  Expert choice's C is ec_capacity                       */
+  size_t permute_workspace;/* bytes of scratch moe_permute uses (<= step_workspace): what       */
+                           /*   moe_permute_noalloc needs from its fixed array                  */
 } moe_sizes;
 
 /* Sizes of every buffer for `cfg`.  Validates cfg: returns MOE_ERR_INVALID_ARG
@@ -199,11 +218,17 @@ MOE_API moe_status moe_permute(const moe_config *cfg, const void *x, const int32
  *   Arguments, outputs and results are those of moe_permute.
  *   Scratch: a fixed array of MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (8 MiB) compiled
  *   into the library, held by every GPU that loads the library until the
- *   process exits.  A configuration whose step scratch
- *   (moe_sizes.step_workspace) exceeds it returns MOE_ERR_WORKSPACE before
- *   any launch.  It calls no cudaMalloc, cudaFree or allocating routine.
+ *   process exits.  The permutation's scratch (moe_sizes.permute_workspace:
+ *   the control block, the unit histograms and their block sums, the count
+ *   and row offsets, and the keep-fraction list or the transposed
+ *   probabilities of expert choice) must fit in it, else the call returns
+ *   MOE_ERR_WORKSPACE before any launch.  It calls no cudaMalloc, cudaFree or
+ *   allocating routine.
  *   Set-up: the first call on each device looks up the array's device address
  *   with that device current; make that first call before any stream capture.
+ *   Later calls look it up again whenever `stream` is not capturing (so a
+ *   device reset, which reloads the library's device code, is picked up) and
+ *   reuse the last address while it is.
  *   Sharing: every call on a device uses the same array, which keeps the last
  *   call's contents (each call clears what must start at zero).  Calls that
  *   overlap on the GPU -- other streams or threads -- race on it and give wrong

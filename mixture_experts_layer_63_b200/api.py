@@ -44,7 +44,7 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d_model", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("S", ctypes.c_int32), ("k", ctypes.c_int32), ("d_ff", ctypes.c_int32),
-                ("capacity", ctypes.c_int32), ("keep_num", ctypes.c_int32),
+                ("capacity_factor", ctypes.c_float), ("keep_num", ctypes.c_int32),
                 ("keep_den", ctypes.c_int32), ("ec_capacity", ctypes.c_int32),
                 ("n_groups", ctypes.c_int32), ("topk_groups", ctypes.c_int32),
                 ("renormalize", ctypes.c_int32), ("act", ctypes.c_int32),
@@ -56,7 +56,8 @@ class MoeConfig(ctypes.Structure):
 class MoeSizes(ctypes.Structure):
     _fields_ = [("rows_cap", ctypes.c_int64), ("rows_total", ctypes.c_int64),
                 ("tok_rows_len", ctypes.c_int64), ("step_workspace", ctypes.c_size_t),
-                ("workspace", ctypes.c_size_t)]
+                ("workspace", ctypes.c_size_t), ("capacity", ctypes.c_int64),
+                ("permute_workspace", ctypes.c_size_t)]
 
 
 _lib = None
@@ -114,13 +115,23 @@ def _check(fn: str, status: int) -> None:
         raise MoeError(fn, status)
 
 
-def _ptr(t: torch.Tensor | None):
+def _ptr(t: torch.Tensor | None, numel: int | None = None, dtype: torch.dtype | None = None):
+    """Device pointer of a contiguous CUDA tensor on the current device; with
+    numel / dtype given, also checks that it holds at least numel elements of
+    that dtype (a short buffer would be written past its end)."""
     if t is None:
         return None
     if not t.is_cuda:
         raise ValueError("libmoe takes CUDA tensors only (no CPU path)")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device}, but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
     if not t.is_contiguous():
         raise ValueError("libmoe takes contiguous tensors")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"expected {dtype}, got {t.dtype}")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"buffer of {t.numel()} elements, {numel} needed")
     return t.data_ptr()
 
 
@@ -137,18 +148,12 @@ def _ws(ws: torch.Tensor):
 # configuration
 # ---------------------------------------------------------------------------
 
-def capacity_for(T: int, E: int, k: int, capacity_factor: float) -> int:
-    """Expert capacity ceil(cf * k * T / E) (GShard's C = O(N/E)); 0 = unlimited."""
-    if capacity_factor <= 0:
-        return 0
-    return int(math.ceil(capacity_factor * k * T / E))
-
-
 def config_from_workload(w: Workload, T: int | None = None) -> MoeConfig:
     T = w.T if T is None else T
     c = MoeConfig()
     c.T, c.d_model, c.E, c.S, c.k, c.d_ff = T, w.d_model, w.E, w.S, w.k, w.d_ff
-    c.capacity = capacity_for(T, w.E, w.k, w.capacity_factor) if w.mode == "tc" else 0
+    # the library derives the expert capacity from the factor (per local group)
+    c.capacity_factor = w.capacity_factor if w.mode == "tc" else 0.0
     c.keep_num, c.keep_den = w.keep_num, w.keep_den
     if T != w.T:
         w = w.with_tokens(T)
@@ -161,8 +166,6 @@ def config_from_workload(w: Workload, T: int | None = None) -> MoeConfig:
     c.route_rule = ROUTE_RULES[w.route_rule]
     c.route_alpha = w.route_alpha
     c.local_groups = w.local_groups
-    if w.local_groups > 1:           # capacity of one expert in one group
-        c.capacity = capacity_for(T // w.local_groups, w.E, w.k, w.capacity_factor)
     return c
 
 
@@ -173,12 +176,15 @@ class Sizes:
     tok_rows_len: int
     step_workspace: int
     workspace: int
+    capacity: int
+    permute_workspace: int
 
 
 def query_sizes(cfg: MoeConfig) -> Sizes:
     out = MoeSizes()
     _check("moe_query_sizes", lib().moe_query_sizes(ctypes.byref(cfg), ctypes.byref(out)))
-    return Sizes(out.rows_cap, out.rows_total, out.tok_rows_len, out.step_workspace, out.workspace)
+    return Sizes(out.rows_cap, out.rows_total, out.tok_rows_len, out.step_workspace, out.workspace,
+                 out.capacity, out.permute_workspace)
 
 
 def new_workspace(cfg: MoeConfig, device="cuda", step_only: bool = False) -> torch.Tensor:

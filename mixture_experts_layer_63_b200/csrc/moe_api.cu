@@ -3,6 +3,7 @@
 // arithmetic of the layer runs in the kernels of the other files.
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 
 #include "device_common.cuh"
 #include "moe_internal.h"
@@ -13,6 +14,32 @@ static std::atomic<uint64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// Expert capacity (GShard section 1 of "MoE技术演进": C = O(N/E) tokens per
+// expert; per local group of N/G tokens with group dispatching):
+// C = ceil(cf * k * Tg / E) for the fp32 factor cf, Tg = T / G tokens per
+// group, evaluated exactly: cf = m * 2^s with m a 24-bit integer, so
+// C = ceil(m * k * Tg * 2^s / E) in 128-bit integers.  Clamped to Tg (an
+// expert takes at most one assignment per token); 0 = unlimited.
+int64_t capacity_rows(const moe_config *c) {
+  if (c->mode != MOE_TOKEN_CHOICE || !(c->capacity_factor > 0.0f)) return 0;
+  const int64_t Tg = c->local_groups > 1 ? c->T / c->local_groups : c->T;
+  int ex = 0;
+  const double mant = frexp((double)c->capacity_factor, &ex);      // cf = mant * 2^ex
+  const uint64_t m = (uint64_t)ldexp(mant, 24);                     // exact: fp32 has 24 bits
+  const int s = ex - 24;                                            // cf = m * 2^s
+  unsigned __int128 num = (unsigned __int128)m * (uint64_t)c->k * (uint64_t)Tg;
+  unsigned __int128 den = (uint64_t)c->E;
+  if (s >= 0) {
+    if (s > 60) return Tg;                      // cf >= 2^60: far above Tg
+    num <<= s;
+  } else {
+    if (-s > 100) return num > 0 ? 1 : 0;       // 0 < value < 1: the ceiling is 1
+    den <<= -s;
+  }
+  const unsigned __int128 q = (num + den - 1) / den;
+  return q >= (unsigned __int128)Tg ? Tg : (int64_t)q;
+}
 
 moe_status validate(const moe_config *c) {
   if (!c) return MOE_ERR_INVALID_ARG;
@@ -28,16 +55,18 @@ moe_status validate(const moe_config *c) {
   if (c->route_rule < MOE_ROUTE_SOFTMAX || c->route_rule > MOE_ROUTE_LOAD || c->reserved != 0)
     return MOE_ERR_INVALID_ARG;
   if (!(c->route_alpha == c->route_alpha)) return MOE_ERR_INVALID_ARG;       // NaN
+  if (!std::isfinite(c->capacity_factor)) return MOE_ERR_INVALID_ARG;
+  const bool capped = c->capacity_factor > 0.0f;
   if (c->local_groups < 0) return MOE_ERR_INVALID_ARG;
   if (c->local_groups > 1) {
     // GShard local groups: capacity dispatch of contiguous 32-token-aligned groups
-    if (c->mode != MOE_TOKEN_CHOICE || c->capacity <= 0) return MOE_ERR_INVALID_ARG;
+    if (c->mode != MOE_TOKEN_CHOICE || !capped) return MOE_ERR_INVALID_ARG;
     if (c->T % c->local_groups != 0) return MOE_ERR_INVALID_ARG;
     if ((c->T / c->local_groups) % kUnitTokens != 0) return MOE_ERR_UNSUPPORTED;
   }
   if (c->mode == MOE_TOKEN_CHOICE) {
     if (c->k < 1 || c->k > c->E) return MOE_ERR_INVALID_ARG;
-    if (c->capacity > 0 && c->keep_den > 0) return MOE_ERR_INVALID_ARG;   // exclusive drop rules
+    if (capped && c->keep_den > 0) return MOE_ERR_INVALID_ARG;            // exclusive drop rules
     if (c->n_groups > 0) {
       if (c->E % c->n_groups != 0 || c->topk_groups < 1 || c->topk_groups > c->n_groups)
         return MOE_ERR_INVALID_ARG;
@@ -48,7 +77,7 @@ moe_status validate(const moe_config *c) {
     if (c->T * (int64_t)c->k > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
   } else {
     if (c->ec_capacity < 1 || c->ec_capacity > c->T) return MOE_ERR_INVALID_ARG;
-    if (c->n_groups != 0 || c->topk_groups != 0 || c->capacity > 0 || c->keep_den > 0 ||
+    if (c->n_groups != 0 || c->topk_groups != 0 || capped || c->keep_den > 0 ||
         c->renormalize || c->route_rule != MOE_ROUTE_SOFTMAX)
       return MOE_ERR_INVALID_ARG;
     if ((int64_t)c->E * c->ec_capacity > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED;
@@ -88,7 +117,7 @@ WsLayout make_layout(const moe_config *c) {
   L.tok_rows_len = tc ? T * k : (int64_t)E * T;
   L.nunit = (int)((T + kUnitTokens - 1) / kUnitTokens);
   const int64_t hist_ints = tc ? (int64_t)k * L.nunit * E : 0;
-  const bool keepfrac = tc && c->capacity <= 0 && c->keep_den > 0;
+  const bool keepfrac = tc && capacity_rows(c) == 0 && c->keep_den > 0;
   size_t o = 0;
   auto take = [&](size_t bytes) {
     const size_t at = o;
@@ -567,6 +596,8 @@ moe_status moe_query_sizes(const moe_config *cfg, moe_sizes *out) {
   out->tok_rows_len = L.tok_rows_len;
   out->step_workspace = L.step_end;
   out->workspace = L.total;
+  out->capacity = capacity_rows(cfg);
+  out->permute_workspace = L.permute_end;
   return MOE_OK;
 }
 
@@ -627,7 +658,7 @@ moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *topk
   const WsLayout L = make_layout(cfg);
   if ((st = check_ws(L, ws, ws_bytes, L.step_end)) != MOE_OK) return st;
   const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
-  const bool keepfrac = tc && cfg->capacity <= 0 && cfg->keep_den > 0;
+  const bool keepfrac = tc && capacity_rows(cfg) == 0 && cfg->keep_den > 0;
   if (!x || !counts || !offsets || !tok_rows || !row_token || !row_gate || !x_perm || !n_dropped)
     return MOE_ERR_INVALID_ARG;
   if (tc && (!topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;

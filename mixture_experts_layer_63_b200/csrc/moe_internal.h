@@ -102,6 +102,9 @@ struct WsLayout {
 
 moe_status validate(const moe_config *c);
 WsLayout make_layout(const moe_config *c);
+// expert capacity C per (local group and) routed expert from the capacity
+// factor, exact ceiling, clamped to the group's tokens; 0 = unlimited
+int64_t capacity_rows(const moe_config *c);
 
 inline size_t elem_size(const moe_config *c) { return c->dtype == MOE_F32 ? 4 : 2; }
 

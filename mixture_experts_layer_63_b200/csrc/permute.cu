@@ -549,7 +549,8 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
   int32_t *cnt_off = reinterpret_cast<int32_t *>(ws + L.cnt_off);
   int32_t *kept = reinterpret_cast<int32_t *>(ws + L.kept);
   int32_t *sorted_q = reinterpret_cast<int32_t *>(ws + L.sorted_q);
-  const int keepfrac = (c->capacity <= 0 && c->keep_den > 0) ? 1 : 0;
+  const int capacity = (int)capacity_rows(c);                // 0: unlimited
+  const int keepfrac = (capacity == 0 && c->keep_den > 0) ? 1 : 0;
   const UnitGrid ug = unit_grid(c);
   const int nu = ug.G * ug.upg;
   const int nb = ug.nb;
@@ -573,7 +574,7 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
     if (e != cudaSuccess) return e;
   }
   e = launch_kernel(rank_units_kernel, nb, 1024, rank_smem, s, topk_idx, topk_gate, T, c->k, E,
-                    ug.nbg, ug.upg, ug.bpg, nb, hist, own_sums ? nullptr : bsum, c->capacity,
+                    ug.nbg, ug.upg, ug.bpg, nb, hist, own_sums ? nullptr : bsum, capacity,
                     c->keep_num, c->keep_den,
                     keepfrac, counts,
                     cnt_off, kept, offsets, n_dropped, tok_rows, row_token, row_gate, sorted_q);
@@ -607,8 +608,10 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
 //
 // The array lives on every GPU that loads the library until the process
 // exits.  In host code its name is only a host-side stand-in, so its device
-// address is looked up once per device (with that device current) through
+// address is looked up (with the device current) through
 // cudaGetSymbolAddress and passed to the kernels like a workspace pointer.
+// Only the permutation's share of a workspace (control block, histograms,
+// scans, keep-fraction list or transposed probabilities) lives there.
 // All calls on a device share the array and it keeps the last call's
 // contents: the kernels overwrite every scratch word they read except the
 // error word, which each call clears first.  Calls that overlap on the GPU
@@ -624,14 +627,20 @@ constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 void *g_scratch_address[kMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device.
-cudaError_t static_scratch_address(char **out) {
+// Device address of g_static_scratch on the current device.  Looked up
+// again on every call whose stream is not capturing (cheap; a device reset
+// reloads the module and can move the array), the cached address reused
+// while the stream captures (a lookup may not be legal then).
+cudaError_t static_scratch_address(cudaStream_t s, char **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(s, &cap);
+  if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_address[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone || g_scratch_address[dev] == nullptr) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return e;
@@ -653,18 +662,19 @@ extern "C" moe_status moe_permute_noalloc(const moe_config *cfg, const void *x,
   const moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const WsLayout L = make_layout(cfg);
-  if (L.permute_end > kStaticScratchBytes) return MOE_ERR_WORKSPACE;   // beyond the fixed array
+  // the permutation's scratch (moe_sizes.permute_workspace) must fit the array
+  if (L.permute_end > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
   const bool tc = cfg->mode == MOE_TOKEN_CHOICE;
-  const bool keepfrac = tc && cfg->capacity <= 0 && cfg->keep_den > 0;
+  const bool keepfrac = tc && capacity_rows(cfg) == 0 && cfg->keep_den > 0;
   if (!x || !counts || !offsets || !tok_rows || !row_token || !row_gate || !x_perm || !n_dropped)
     return MOE_ERR_INVALID_ARG;
   if (tc && (!topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
   if ((!tc || keepfrac) && !probs) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_perm) & 15u))
     return MOE_ERR_INVALID_ARG;
-  char *scratch = nullptr;
-  if (static_scratch_address(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char *scratch = nullptr;
+  if (static_scratch_address(s, &scratch) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaMemsetAsync(scratch + L.err, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
   const cudaError_t e = launch_permute(cfg, L, scratch, false, x, topk_idx, topk_gate, probs, counts,
                                        offsets, tok_rows, row_token, row_gate, x_perm, n_dropped, s);

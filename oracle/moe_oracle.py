@@ -64,6 +64,7 @@ soft mixture, and invariants; none is "parity unpinned".
 from __future__ import annotations
 
 import math
+from fractions import Fraction
 from dataclasses import dataclass
 
 import numpy as np
@@ -293,10 +294,16 @@ class Dispatch:
 
 
 def capacity_from_factor(T: int, E: int, k: int, capacity_factor: float) -> int:
-    """C = ceil(cf * k * T / E); 0 means unlimited (cf <= 0)."""
+    """C = ceil(cf * k * T / E); 0 means unlimited (cf <= 0).
+
+    GShard section 1 of "MoE技术演进" fixes only C = O(N/E) (2N/(G*E) per
+    group for top-2); the factor form is the workloads'.  The ceiling is taken
+    of the exact product for the binary value of cf (a fraction, no rounding
+    before the ceiling): a floating-point product could land on either side
+    of an integer."""
     if capacity_factor <= 0:
         return 0
-    return int(math.ceil(capacity_factor * k * T / E))
+    return int(math.ceil(Fraction(capacity_factor) * k * T / E))
 
 
 def keep_count(n: np.ndarray, keep_num: int, keep_den: int) -> np.ndarray:

@@ -58,9 +58,9 @@ SMALL = {
 
 
 def oracle_config(w: Workload) -> O.OracleConfig:
-    cap = O.capacity_from_factor(w.T, w.E, w.k, w.capacity_factor) if w.mode == "tc" else 0
-    if w.mode == "tc" and w.local_groups > 1:        # capacity of one expert in one group
-        cap = O.capacity_from_factor(w.T // w.local_groups, w.E, w.k, w.capacity_factor)
+    cf = float(np.float32(w.capacity_factor))       # the fp32 factor the library takes
+    Tg = w.T // max(1, w.local_groups)              # capacity of one expert in one group
+    cap = min(O.capacity_from_factor(Tg, w.E, w.k, cf), Tg) if w.mode == "tc" else 0
     return O.OracleConfig(E=w.E, S=w.S, k=w.k, act=w.act, mode=w.mode, capacity=cap,
                           keep_num=w.keep_num, keep_den=w.keep_den,
                           ec_capacity=w.ec_capacity if w.mode == "ec" else 0,

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(L):
 
 def test_struct_sizes(L):
     assert ctypes.sizeof(api.MoeConfig) == 88
-    assert ctypes.sizeof(api.MoeSizes) == 40
+    assert ctypes.sizeof(api.MoeSizes) == 56
 
 
 def test_struct_layout_matches_the_header(tmp_path):
@@ -115,6 +115,8 @@ def _cfg(**kw):
     ("local_groups", 3, api.MOE_ERR_INVALID_ARG),   # 4096 tokens do not split into 3 groups
     ("local_groups", 256, api.MOE_ERR_UNSUPPORTED), # groups of 16 tokens: below one 32-token unit
     ("local_groups", -1, api.MOE_ERR_INVALID_ARG),
+    ("capacity_factor", float("nan"), api.MOE_ERR_INVALID_ARG),
+    ("capacity_factor", float("inf"), api.MOE_ERR_INVALID_ARG),
 ])
 def test_invalid_configs_rejected(L, field, value, status):
     c = _cfg(**{field: value})
@@ -124,9 +126,9 @@ def test_invalid_configs_rejected(L, field, value, status):
 
 
 def test_group_limit_needs_enough_experts(L):
-    c = _cfg(n_groups=8, topk_groups=1, k=2, capacity=0)   # 1 group of 2 experts holds k=2: ok
+    c = _cfg(n_groups=8, topk_groups=1, k=2, capacity_factor=0.0)   # 1 group of 2 experts holds k=2: ok
     api.query_sizes(c)
-    c = _cfg(n_groups=8, topk_groups=1, k=3, capacity=0)
+    c = _cfg(n_groups=8, topk_groups=1, k=3, capacity_factor=0.0)
     with pytest.raises(api.MoeError):
         api.query_sizes(c)
 
@@ -147,7 +149,7 @@ def test_expert_choice_options(L):
 def test_local_groups_need_a_capacity(L):
     c = _cfg(local_groups=4)
     api.query_sizes(c)
-    c = _cfg(local_groups=4, capacity=0)
+    c = _cfg(local_groups=4, capacity_factor=0.0)
     with pytest.raises(api.MoeError):
         api.query_sizes(c)
 
@@ -169,7 +171,7 @@ def test_null_pointers_rejected_before_any_launch(L):
                        s.workspace, None)
     assert st == api.MOE_ERR_INVALID_ARG
     # a routing rule that reads route_state, without one
-    c2 = _cfg(T=64, d_model=64, d_ff=64, capacity=8)
+    c2 = _cfg(T=64, d_model=64, d_ff=64, capacity_factor=1.0)
     c2.route_rule = api.MOE_ROUTE_BIAS
     ws = ctypes.create_string_buffer(api.query_sizes(c2).workspace + 256)
     wa = (ctypes.addressof(ws) + 255) & ~255
@@ -188,3 +190,59 @@ def test_cpu_tensors_refused(L):
     x = torch.zeros(c.T, c.d_model, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         api.moe_combine(c, x, x, x)
+
+
+def _lib_capacity(w, T=None, cf=None):
+    c = api.config_from_workload(w, T)
+    if cf is not None:
+        c.capacity_factor = cf
+    return api.query_sizes(c).capacity
+
+
+def test_library_capacity_matches_the_oracle(L):
+    """The expert capacity the library derives from capacity_factor (GShard
+    section 1: C = O(N/E), per local group with group dispatching) equals the
+    oracle's ceil(cf * k * T / E) for the fp32 factor, clamped to the tokens
+    of a group."""
+    import numpy as np
+    from dataclasses import replace
+
+    from oracle import moe_oracle as O
+
+    def oracle_c(T, E, k, cf):
+        return min(O.capacity_from_factor(T, E, k, float(np.float32(cf))), T)
+
+    tiny, gshard, local = WORKLOADS["tiny_f32"], WORKLOADS["gshard"], WORKLOADS["gshard_local"]
+    assert _lib_capacity(tiny) == oracle_c(256, 8, 2, 1.25) == 80
+    assert _lib_capacity(gshard) == oracle_c(4096, 16, 2, 1.25) == 640
+    G = local.local_groups
+    assert _lib_capacity(local) == oracle_c(4096 // G, 16, 2, 1.25) == 160
+    # factor 1, top-2: 2N/(G*E) per group (GShard's local-group capacity)
+    assert _lib_capacity(replace(local, capacity_factor=1.0)) == 2 * 4096 // (G * 16)
+    # factors whose product is not an integer, or not exact in binary
+    rng = np.random.default_rng(5)
+    for cf in [0.1, 0.3, 1.1, 1.3, 2.7, 1e-3, 1e-30, 7.0, 100.0, 3e9]:
+        for T in (96, 1000, 4096):
+            w = replace(gshard, T=T, capacity_factor=cf)
+            assert _lib_capacity(w) == oracle_c(T, 16, 2, cf), (cf, T)
+    for _ in range(200):
+        T, E = int(rng.integers(1, 5000)), int(rng.integers(1, 257))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        cf = float(np.float32(rng.uniform(0.01, 4.0)))
+        w = replace(gshard, T=T, E=E, k=k, capacity_factor=cf)
+        assert _lib_capacity(w) == oracle_c(T, E, k, cf), (T, E, k, cf)
+    # no capacity: 0; expert choice: 0 (its C is ec_capacity)
+    assert _lib_capacity(replace(gshard, capacity_factor=0.0)) == 0
+    assert _lib_capacity(WORKLOADS["deepseekmoe_ec"]) == 0
+
+
+def test_permute_workspace_is_the_permutation_share(L):
+    """moe_sizes.permute_workspace: the scratch moe_permute uses (what
+    moe_permute_noalloc needs in its fixed array), within step_workspace."""
+    for name, w in WORKLOADS.items():
+        s = api.query_sizes(api.config_from_workload(w))
+        assert 4096 <= s.permute_workspace <= s.step_workspace, name
+    # the bf16 layers' step workspace holds the GEMMs' 24 MiB stream-K slab
+    # as well, which the permutation does not use
+    s = api.query_sizes(api.config_from_workload(WORKLOADS["gshard"]))
+    assert s.step_workspace - s.permute_workspace >= 24 << 20

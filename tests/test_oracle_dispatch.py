@@ -116,6 +116,22 @@ def test_capacity_formula():
     assert O.capacity_from_factor(100, 3, 2, 0.0) == 0
 
 
+def test_capacity_is_the_exact_ceiling():
+    """For a factor num / 2^p (exact in binary) the capacity is the integer
+    ceiling -(-(num * k * T) // (2^p * E)), with no rounding before it: e.g.
+    1.1 * 2 * 500 / 10 = 110 exactly for the decimal 1.1, but the binary
+    double 1.1 lies above it, so the exact ceiling is 111."""
+    rng = np.random.default_rng(3)
+    for _ in range(2000):
+        p = int(rng.integers(0, 30))
+        num = int(rng.integers(1, 1 << 24))
+        T, E, k = int(rng.integers(1, 100000)), int(rng.integers(1, 300)), int(rng.integers(1, 9))
+        want = -(-(num * k * T) // ((1 << p) * E))
+        assert O.capacity_from_factor(T, E, k, num / (1 << p)) == want
+    assert O.capacity_from_factor(500, 10, 2, 1.1) == 111
+    assert O.capacity_from_factor(500, 10, 2, 1.25) == 125
+
+
 def test_keep_fraction_golden():
     g = _load("keep_fraction_worked.json")
     idx = np.array(g["topk_idx"], np.int32)
