@@ -40,13 +40,16 @@ import torch  # noqa: E402
 from mixture_experts_layer_63_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "MoE-layer fwd tokens/s on 1 B200; grouped-GEMM % bf16 peak; permute GB/s"
-DEFAULT_WORKLOAD = "gshard"
+# the largest of the five layers (DeepSeek-V2-shaped: 160 + 2 experts, 7.6 GB
+# of expert weights); --workload selects the others
+DEFAULT_WORKLOAD = "deepseek_v2"
 
-# dram bytes (read + write) per launch, from ncu captures summarised under
-# profiles/, with the sha256 (first 16 hex digits) of the kernel source they
-# were taken at; a value is reported only while the source is unchanged.
+# DRAM bytes (read + write) of the two expert GEMMs of one forward, from an
+# ncu capture of the same kernels, with the sha256 (first 16 hex digits) of
+# the GEMM source they were taken at; reported only while the source is
+# unchanged (null otherwise).
 NCU_TRAFFIC: dict[str, dict] = {
-    # profiles/gemm_gshard_ncu.md: up 151.09 + 41.15 MB, down 220.18 + 9.75 MB
+    # up 151.09 + 41.15 MB, down 220.18 + 9.75 MB
     "gshard": {"bytes": 422_169_088, "src": "a9de9705dc80e5bb"},
 }
 
@@ -413,6 +416,9 @@ def run_ours(args, w) -> None:
     mean = per.mean(axis=0)                                # ms per call
     hbm, tfl, tfl_sus, peak_src = _peaks()
     gemm_tflops = gemm_flops / (ffn_ms * 1e-3) / 1e12
+    # the expert GEMMs' floor: their flops at the tensor peak, or streaming
+    # every expert's weights once at the HBM peak, whichever is longer
+    floor_ms = max(gemm_flops / (tfl * 1e12), weight_bytes / (hbm * 1e9)) * 1e3
     h = _src_hash("gemm_sm100.cu")
     tr = NCU_TRAFFIC.get(w.name)
     traffic = tr["bytes"] if tr and tr.get("src") == h else None
@@ -520,7 +526,11 @@ def run_ours(args, w) -> None:
                          "achieved": gemm_tflops, "peak": tfl, "unit": "TFLOP/s",
                          "frac": gemm_tflops / tfl, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16 burst", "algorithmic_flops": gemm_flops,
-                         "frac_of_sustained": gemm_tflops / tfl_sus if tfl_sus else None},
+                         "frac_of_sustained": gemm_tflops / tfl_sus if tfl_sus else None,
+                         "weight_bytes": weight_bytes,
+                         "floor_ms": floor_ms, "floor_bound": "tensor" if gemm_flops / (tfl * 1e12)
+                         >= weight_bytes / (hbm * 1e9) else "hbm (weights)",
+                         "frac_of_floor": floor_ms / ffn_ms},
             "steps_us": {"route": mean[0] * 1e3, "permute": mean[1] * 1e3,
                          "expert_ffn": mean[2] * 1e3, "combine": mean[3] * 1e3,
                          "expert_ffn_in_timed_region": ffn_ms * 1e3,
@@ -617,9 +627,20 @@ def main() -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm-vs-library", action="store_true",
                     help="time the expert GEMMs on this workload's dense shape next to torch.matmul")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="profiling shape: this many tokens instead of the workload's")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="profiling shape: this many routed experts instead of the workload's")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
+    if args.experts:
+        from dataclasses import replace
+        w = replace(w, E=args.experts, name=f"{w.name}[E={args.experts}]",
+                    ec_capacity=w.T * w.k // args.experts if w.mode == "ec" else 0)
+    if args.tokens:
+        from dataclasses import replace
+        w = replace(w.with_tokens(args.tokens), name=f"{w.name}[T={args.tokens}]")
     if args.gemm_vs_library:
         run_gemm_vs_library(args, w)
     elif args.impl == "reference":

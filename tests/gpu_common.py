@@ -110,6 +110,46 @@ def assert_close_rms(y: np.ndarray, ref: np.ndarray, dtype: str, what: str = "y"
     return float(diff.max()) / rms
 
 
+def round_to_format(ref: np.ndarray, dtype: str) -> np.ndarray:
+    """ref rounded once, to nearest even, to the output format (bf16 or fp32)."""
+    r32 = ref.astype(np.float32)
+    if dtype == "f32":
+        return r32.astype(np.float64)
+    return torch.from_numpy(r32).to(torch.bfloat16).double().numpy()
+
+
+def output_margins(y: np.ndarray, ref: np.ndarray, dtype: str) -> dict:
+    """How close an output is to the oracle, relative to rms(ref):
+    excess_over_rms         max(|y - ref| - half an ulp of ref) / rms, the
+                            quantity the tolerance rule bounds (P17);
+    plain_over_rms          max |y - ref| / rms;
+    vs_rounded_ref_over_rms max(|y - r| - ulp(ref)) / rms with r = ref rounded
+                            once to the output format: y may sit on the
+                            neighbouring representable value of r, no further;
+    identical_to_rounded    share of elements equal to r bit for bit."""
+    ref = ref.astype(np.float64)
+    y = y.astype(np.float64)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    hu = half_ulp(ref, dtype)
+    r = round_to_format(ref, dtype)
+    return {"excess_over_rms": float(np.max(np.abs(y - ref) - hu)) / rms,
+            "plain_over_rms": float(np.max(np.abs(y - ref))) / rms,
+            "vs_rounded_ref_over_rms": float(np.max(np.abs(y - r) - 2 * hu)) / rms,
+            "identical_to_rounded": float(np.mean(y == r)),
+            "tol": TOL[dtype]}
+
+
+def record_margin(case: str, m: dict) -> None:
+    """Append the margins of one case as a JSON line to the file named by
+    MOE_MARGIN_LOG (if set), for the design notes' tolerance table."""
+    import json
+    import os
+    path = os.environ.get("MOE_MARGIN_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": case, **m}) + "\n")
+
+
 def gpu_inputs(w: Workload, seed: int = 0, grid: bool = True):
     return make_inputs(w, seed=seed, device="cuda", grid=grid)
 

@@ -13,10 +13,14 @@ leading dimension (one token of dx, one expert of each weight gradient):
 (an element's error is measured against the slice's largest value: a
 lightly loaded expert's gradient is a sum of a few outer products, heavy
 tailed, and its largest elements carry the largest roundings).  With ReLU
-the bound on single elements is 1e-1 max |g_ref|: where a pre-activation
-lies within its bf16 rounding of zero, the recomputed value and the exact
-one may fall on opposite sides, both correct, and the ReLU mask (the
-derivative is discontinuous there) takes or drops a whole term dh * x.  Slices, because experts differ in load,
+the same 3e-2 element bound holds everywhere except where a mask can
+legitimately differ: a pre-activation whose exact value lies within the
+accumulation error of its fp32 recomputation (|a| <= K * 2^-22 * sum |x_i w_i|,
+four fp32 roundings per added term) may come out on the other side of
+zero, both correct, and the ReLU mask (the derivative is discontinuous
+there) then takes or drops a whole term dh * x.  Only the elements such a
+position feeds -- the row j of dW1_e, and the token's row of dx -- are held
+to the looser 1e-1 max |g_ref|.  Slices, because experts differ in load,
 so their gradients differ in scale by an order of magnitude or more, and
 each slice carries its own rounding at its own scale.  An all-zero reference slice (an
 expert without rows) must come out exactly zero.  The router's gradients are
@@ -44,7 +48,13 @@ TOL_MAX = 3e-2      # per slice, max error over the largest reference value
 BF16_SMALL = [n for n, w in SMALL.items() if w.dtype == "bf16"]
 
 
-def _check(name, got, ref, tol_max=TOL_MAX):
+TOL_MAX_MASK = 1e-1  # ReLU: elements fed by a pre-activation whose sign may differ
+
+
+def _check(name, got, ref, loose=None):
+    """Per slice of the leading dimension: relative Frobenius error within
+    TOL_FRO, every element within TOL_MAX of the slice's largest value, or
+    within TOL_MAX_MASK where `loose` (a boolean array of ref's shape) is set."""
     ref = np.asarray(ref, dtype=np.float64)
     got = np.asarray(got, dtype=np.float64).reshape(ref.shape)
     n = ref.shape[0]
@@ -52,16 +62,43 @@ def _check(name, got, ref, tol_max=TOL_MAX):
     g2 = got.reshape(n, -1)
     rms = np.sqrt(np.mean(r2 ** 2, axis=1))
     top = np.abs(r2).max(axis=1)
+    tol = np.full(r2.shape, TOL_MAX)
+    if loose is not None:
+        tol[np.asarray(loose).reshape(n, -1)] = TOL_MAX_MASK
+    over = (np.abs(g2 - r2) / (tol * top[:, None] + 1e-300)).max(axis=1)   # > 1: out of bound
     err = np.abs(g2 - r2).max(axis=1)
     fro = np.sqrt(np.mean((g2 - r2) ** 2, axis=1))
     zero = rms == 0
     assert np.all(err[zero] == 0), f"{name}: nonzero gradient where the reference is zero"
     nz = np.flatnonzero(~zero)
-    bad = nz[(fro[nz] > TOL_FRO * rms[nz]) | (err[nz] > tol_max * top[nz])]
+    bad = nz[(fro[nz] > TOL_FRO * rms[nz]) | (over[nz] > 1.0)]
     if len(bad):
         i = bad[0]
         raise AssertionError(f"{name}[{i}]: rel. error {fro[i] / rms[i]:.3e}, max|err| / max|ref| "
                              f"{err[i] / top[i]:.3e}")
+
+
+def _relu_ambiguous(w, x_np, w1, disp):
+    """Where the sign of a ReLU pre-activation is within rounding: returns
+    (rows_of_dw1 [E+S, f] bool, tokens [T] bool) of the elements it feeds."""
+    xs = O.widen(x_np)
+    K = xs.shape[1]
+    amb_w = np.zeros((w.E + w.S, w.d_ff), dtype=bool)
+    amb_t = np.zeros(w.T, dtype=bool)
+    for e in range(w.E + w.S):
+        if e < w.E:
+            toks = disp.row_token[disp.offsets[e]:disp.offsets[e + 1]]
+        else:
+            toks = np.arange(w.T)
+        if len(toks) == 0:
+            continue
+        we = O.widen(w1[e])
+        a = xs[toks] @ we.T
+        bound = K * 2.0 ** -22 * (np.abs(xs[toks]) @ np.abs(we).T)
+        near = np.abs(a) <= bound
+        amb_w[e] |= near.any(axis=0)
+        amb_t[toks[near.any(axis=1)]] = True
+    return amb_w, amb_t
 
 
 def _backward_check(w, seed=21):
@@ -87,8 +124,12 @@ def _backward_check(w, seed=21):
     w2 = [to_np(inp.w2[e]) for e in range(G)]
     w3 = [to_np(inp.w3[e]) for e in range(G)] if inp.w3 is not None else None
     ref = O.backward(oc, x_np, to_np(inp.w_router), bias, w1, w3, w2, to_f64(dy), st, disp)
-    tm = TOL_MAX if w.act == "swiglu" else 1e-1
-    _check("dx", to_f64(grads["dx"]), ref.dx, tm)
+    loose_w1 = loose_x = None
+    if w.act == "relu":
+        amb_w, amb_t = _relu_ambiguous(w, x_np, w1, disp)
+        loose_w1 = np.broadcast_to(amb_w[:, :, None], ref.dw1.shape)
+        loose_x = np.broadcast_to(amb_t[:, None], ref.dx.shape)
+    _check("dx", to_f64(grads["dx"]), ref.dx, loose_x)
     dl = ref.dlogits
     xs = O.widen(x_np)
     rss_w = np.sqrt((dl ** 2).T @ (xs ** 2))             # [E, d]
@@ -100,10 +141,10 @@ def _backward_check(w, seed=21):
         err_b = np.abs(to_f64(grads["dbias"]) - ref.dbias)
         assert np.all(err_b <= TOL * rss_b + 1e-12), \
             f"dbias: worst err / rss {float((err_b / (rss_b + 1e-30)).max()):.3e}"
-    _check("dw1", to_f64(grads["dw1"]), ref.dw1, tm)
-    _check("dw2", to_f64(grads["dw2"]), ref.dw2, tm)
+    _check("dw1", to_f64(grads["dw1"]), ref.dw1, loose_w1)
+    _check("dw2", to_f64(grads["dw2"]), ref.dw2)
     if w3 is not None:
-        _check("dw3", to_f64(grads["dw3"]), ref.dw3, tm)
+        _check("dw3", to_f64(grads["dw3"]), ref.dw3)
 
 
 @pytest.mark.parametrize("name", BF16_SMALL)

@@ -1,9 +1,12 @@
 """The expert GEMMs' stream-K tail (tiles cut into k-block pieces spread over
 all CTAs, summed by the CTA holding each tile's first k-block).
 
-* Long contractions on few tiles: every tile is cut into several pieces, so
-  each finalizer adds three or more partial tiles (1-CTA and CTA-pair
-  kernels, ReLU and SwiGLU up-projections, gate-scaled down-projection).
+* Long contractions on few tiles: every tile of the CTA-pair kernel is cut
+  into several pieces, so each finalizer adds three or more partial tiles
+  (ReLU and SwiGLU up-projections, gate-scaled down-projection); the same
+  contractions on the token-N tiles of short experts, which have no tail.
+  (The single-CTA kernel's tail runs in the backward pass, covered by its
+  tests.)
 * The sum order is fixed by the tile count and the grid: two calls give the
   same bits.
 """
@@ -21,10 +24,10 @@ from tests.test_gpu_parity import _forward_check
 pytestmark = pytest.mark.gpu
 
 LONG_K = {
-    # 1-CTA tiles (128 rows): down-projection K = 2048 -> 32 k-blocks on 3 tiles
-    "one_cta_relu": replace(SMALL["gshard_s"], T=300, E=1, k=1, capacity_factor=0.0, d_ff=2048),
-    # 1-CTA, SwiGLU with shared experts, K = 1536 on the down-projection
-    "one_cta_swiglu": replace(SMALL["dsv2_s"], T=260, d_ff=1536),
+    # short experts: token-N tiles (no stream-K tail), down-projection K = 2048
+    # on 3 tiles and K = 1536 with SwiGLU and shared experts
+    "token_n_relu": replace(SMALL["gshard_s"], T=300, E=1, k=1, capacity_factor=0.0, d_ff=2048),
+    "token_n_swiglu": replace(SMALL["dsv2_s"], T=260, d_ff=1536),
     # CTA pairs (256-row tiles): about 1050 rows per expert, K = 2048
     "pair_relu": replace(SMALL["pair_relu_s"], d_ff=2048),
     # CTA pairs, SwiGLU and shared experts, K = 1024 on the down-projection
