@@ -331,6 +331,19 @@ MOE_API moe_status moe_check_device_errors(void *ws, size_t ws_bytes, moe_stream
  * it reports an error. */
 MOE_API moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Set the time limit of every device-side wait of the launches that use
+ * `ws` (bytes 8-15 of its control block): limit_ns nanoseconds, 0 for the
+ * default of 2 s.  A wait that runs out sets the timeout bit of the error
+ * word and its kernel returns early (its outputs are then incomplete);
+ * moe_check_device_errors reports MOE_ERR_TIMEOUT, and clears the control
+ * block, which restores the default.  The drains that let a timed-out
+ * kernel's copies land always take the default.  Asynchronous on `stream`
+ * (a copy from host memory).  Meant for failure detection: a short limit
+ * turns a wait that can never finish into an error status within that
+ * time. */
+MOE_API moe_status moe_workspace_set_wait_limit(void *ws, size_t ws_bytes, uint64_t limit_ns,
+                                                moe_stream_t stream);
+
 /* Static text for a status code. */
 MOE_API const char *moe_status_string(moe_status s);
 

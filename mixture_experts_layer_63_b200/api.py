@@ -32,7 +32,7 @@ EXPORTS = ("moe_query_sizes", "moe_route", "moe_gate", "moe_permute", "moe_exper
            "moe_combine", "moe_forward", "moe_check_device_errors", "moe_workspace_init",
            "moe_status_string", "moe_permute_noalloc", "moe_forward_timed",
            "moe_route_bias_update", "moe_query_backward_size", "moe_backward",
-           "moe_kernel_launches")
+           "moe_kernel_launches", "moe_workspace_set_wait_limit")
 
 
 class MoeError(RuntimeError):
@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
                                   ctypes.POINTER(ctypes.c_void_p), vp],
             "moe_check_device_errors": [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)],
             "moe_workspace_init": [vp, sz, vp],
+            "moe_workspace_set_wait_limit": [vp, sz, ctypes.c_uint64, vp],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -290,6 +291,13 @@ def moe_check_device_errors(ws, stream=None) -> int:
 def moe_workspace_init(ws, stream=None):
     wp, wn = _ws(ws)
     _check("moe_workspace_init", lib().moe_workspace_init(wp, wn, _stream(stream)))
+
+
+def moe_workspace_set_wait_limit(ws, limit_ns: int, stream=None):
+    """Time limit of the device-side waits of launches on ws (0: default 2 s)."""
+    wp, wn = _ws(ws)
+    _check("moe_workspace_set_wait_limit",
+           lib().moe_workspace_set_wait_limit(wp, wn, int(limit_ns), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------

@@ -11,8 +11,21 @@ namespace moe {
 constexpr uint32_t kErrTimeout = 1u;      // a bounded wait ran out
 constexpr uint32_t kErrBadIndex = 2u;     // an index failed a kernel's own check
 
-// Time limit of every device-side wait, in nanoseconds of %globaltimer.
+// Time limit of every device-side wait, in nanoseconds of %globaltimer: the
+// workspace's control block holds it at byte kWaitLimitOffset (uint64,
+// moe_workspace_set_wait_limit); 0 there means this default.  The drains
+// after an abort always take the default.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr size_t kWaitLimitOffset = 8;
+
+// The wait limit of the launch whose control block starts at `err` (read
+// after pdl_wait: a copy before the launch may have set it).
+__device__ __forceinline__ uint64_t wait_limit_ns(const uint32_t *err) {
+  if (!err) return kWaitLimitNs;
+  const uint64_t v = *reinterpret_cast<const volatile uint64_t *>(
+      reinterpret_cast<const char *>(err) + kWaitLimitOffset);
+  return v ? v : kWaitLimitNs;
+}
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;

@@ -174,11 +174,11 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t pa
 }
 
 // Bounded wait for the phase of parity `parity` to complete.  Returns false
-// when the CTA is aborting or the time limit passed (then it raises the
-// timeout bit and starts the abort).
+// when the CTA is aborting or the time limit (`limit` ns) passed (then it
+// raises the timeout bit and starts the abort).
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          uint32_t *err) {
+                                          uint32_t *err, uint64_t limit) {
   auto try_wait = [&]() {
     return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
   };
@@ -188,7 +188,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (try_wait()) return true;
     if ((i & 63u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit) {
         raise_error(err, kErrTimeout);
         *abort_flag = 1;
         return false;
@@ -389,6 +389,23 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
       : "memory");
 }
 
+// Four rows r0..r3 of a 2-D tensor (each a box of 64 columns from column c0;
+// the tensor map's box is one row high) into four consecutive 128-byte rows
+// of this CTA's shared memory at `dst`, with the map's 128-byte swizzle
+// (which follows the shared-memory address, so rows placed at a 512-byte
+// offset of a 1024-byte-aligned tile land as rows 4..7 of an 8-row tile
+// load would), completing on the mbarrier at `bar_cluster` (the even CTA's
+// barrier of the pair).
+__device__ __forceinline__ void tma_gather4_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster,
+                                                 int c0, int4 rows) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(rows.x), "r"(rows.y),
+      "r"(rows.z), "r"(rows.w)
+      : "memory");
+}
+
 __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                                uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -586,7 +603,8 @@ __device__ __forceinline__ void sk_write(const Params &P, int slot, int row, uin
 
 // Finalizer thread: bounded wait until every later piece of the tile is
 // published.  False when the CTA is aborting (timeout bit raised here).
-__device__ __forceinline__ bool sk_wait(const Params &P, const Fixup &F, volatile int *abort_flag) {
+__device__ __forceinline__ bool sk_wait(const Params &P, const Fixup &F, volatile int *abort_flag,
+                                        uint64_t limit) {
   for (int q = F.q0; q < F.q1; ++q) {
     if (!F.sc->nonempty(q)) continue;
     const int *flag = P.sk_flags + q * F.slot_mul + F.slot_add;
@@ -596,7 +614,7 @@ __device__ __forceinline__ bool sk_wait(const Params &P, const Fixup &F, volatil
       if (ld_acquire_gpu(flag) >= kEpiThreads) break;
       if ((it & 63u) == 0) {
         if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit) {
           raise_error(P.err, kErrTimeout);
           *abort_flag = 1;
           return false;
@@ -934,6 +952,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t s_tmem_base;
   __shared__ volatile int s_abort;
+  __shared__ uint64_t s_limit_sh;
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~(uintptr_t)1023);
@@ -970,6 +989,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   pdl_wait();              // what earlier kernels wrote is visible from here on
   pdl_trigger();
+  if (tid == 0) s_limit_sh = wait_limit_ns(P.err);
   // group table: rows and tile prefix, warp 0
   if (warp == 0) {
     int carry = 0;
@@ -1022,6 +1042,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
 
   const uint32_t tmem_base = s_tmem_base;
+  const uint64_t s_limit = s_limit_sh;
   const int KB = P.K / BK;
   const bool sk = EPI != kEpiStoreF32 && P.sk_part != nullptr;
   Sched sc;
@@ -1058,7 +1079,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         kb1 = s_rows[tl.g];
       }
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err, s_limit)) { ok = false; break; }
         uint8_t *sa = smem + (size_t)stage * stage_bytes;
         uint8_t *sb = sa + kABytes;
         const bool a_by_tma = !(gather && tl.g < P.n_routed);   // else the gather warps
@@ -1101,11 +1122,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         kb0 = 0;
         kb1 = s_rows[tl.g];
       }
-      if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+      if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err, s_limit)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&full_bar[stage], phase, &s_abort, P.err)) { ok = false; break; }
+        if (!mbar_wait(&full_bar[stage], phase, &s_abort, P.err, s_limit)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + (size_t)stage * stage_bytes);
         const uint32_t b_addr = a_addr + kABytes;
@@ -1145,7 +1166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = kb0; kb < kb1; ++kb) {
         // lane 0 waits for the stage to be free, the warp follows it
         int okw = 1;
-        if (lane == 0) okw = mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err) ? 1 : 0;
+        if (lane == 0) okw = mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err, s_limit) ? 1 : 0;
         __syncwarp();
         if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
         if (routed) gr.issue(smem_u32(smem + (size_t)stage * stage_bytes), gt, kb, xs, row_bytes);
@@ -1176,7 +1197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (sc.next(tile, kb0, kb1, part)) {
       const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
       // (warp-uniform exits: the epilogue's TMEM loads and stores are warp-wide)
-      if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err, s_limit))) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
       const bool in_tail = sk && tile >= sc.dp_limit;
@@ -1203,7 +1224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int dest = (EPI == kEpiScaleAdd && valid) ? add_dest(P, routed, out_row, tl.m * BM + r_cta) : -1;
         if (in_tail && kb1 < KB) {                              // finalizer of a split tile
           const Fixup F{P.sk_part, &sc, (int)blockIdx.x + 1, sc.contributors_end(tile), 1, 0, r_cta};
-          if (!__all_sync(0xffffffffu, sk_wait(P, F, &s_abort))) break;
+          if (!__all_sync(0xffffffffu, sk_wait(P, F, &s_abort, s_limit))) break;
           epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F, dest);
           sk_done(P, F);
         } else {
@@ -1263,6 +1284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t s_tmem_base;
   __shared__ volatile int s_abort;
+  __shared__ uint64_t s_limit_sh;
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~(uintptr_t)1023);
@@ -1301,6 +1323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
   pdl_wait();              // what earlier kernels wrote is visible from here on
   pdl_trigger();
+  if (tid == 0) s_limit_sh = wait_limit_ns(P.err);
   if (warp == 0) {
     int carry = 0;
     for (int base = 0; base < P.G; base += 32) {
@@ -1351,6 +1374,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
 
   const uint32_t tmem_base = s_tmem_base;
+  const uint64_t s_limit = s_limit_sh;
   const int KB = P.K / (BK * BKS);                     // stages of K per tile
   const bool sk = P.sk_part != nullptr;
   Sched sc;
@@ -1390,7 +1414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         kb1 = s_rows[tl.g];
       }
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err, s_limit)) { ok = false; break; }
         uint8_t *sa = smem + (size_t)stage * stage_bytes;
         uint8_t *sb = sa + BKS * kABytes;
         const uint32_t fb = smem_u32(&full_bar[stage]) & 0xFEFFFFFFu;   // the even CTA's barrier
@@ -1438,11 +1462,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         kb0 = 0;
         kb1 = s_rows[tl.g];
       }
-      if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err)) { ok = false; break; }
+      if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err, s_limit)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait<true>(&full_bar[stage], phase, &s_abort, P.err)) { ok = false; break; }
+        if (!mbar_wait<true>(&full_bar[stage], phase, &s_abort, P.err, s_limit)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + (size_t)stage * stage_bytes);
         const uint32_t b_addr = a_addr + BKS * kABytes;
@@ -1490,7 +1514,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int kb = kb0; kb < kb1; ++kb) {
         // lane 0 waits for the stage to be free, the warp follows it
         int okw = 1;
-        if (lane == 0) okw = mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err) ? 1 : 0;
+        if (lane == 0) okw = mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err, s_limit) ? 1 : 0;
         __syncwarp();
         if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
         if (routed) gr.issue(smem_u32(smem + (size_t)stage * stage_bytes), gt, kb, xs, row_bytes);
@@ -1523,7 +1547,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     while (sc.next(tile, kb0, kb1, part)) {
       const Tile tl = decode_tile(P.reverse ? s_prefix[P.G] - 1 - tile : tile, s_prefix, P.G, P.nt);
       // (warp-uniform exits: the epilogue's TMEM loads and stores are warp-wide)
-      if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err, s_limit))) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
       const bool in_tail = sk && tile >= sc.dp_limit;
@@ -1551,13 +1575,446 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int dest = (EPI == kEpiScaleAdd && valid) ? add_dest(P, routed, out_row, tl.m * PM + r_in) : -1;
         if (in_tail && kb1 < KB) {                              // finalizer of a split tile
           const Fixup F{P.sk_part, &sc, pair + 1, sc.contributors_end(tile), 2, (int)rank, r_cta};
-          if (!__all_sync(0xffffffffu, sk_wait(P, F, &s_abort))) break;
+          if (!__all_sync(0xffffffffu, sk_wait(P, F, &s_abort, s_limit))) break;
           epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F, dest);
           sk_done(P, F);
         } else {
           epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, nullptr, dest);
         }
       }
+      tc_fence_before();
+      mbar_arrive_cluster(acc == 0 ? acce_even0 : acce_even1);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();              // neither CTA leaves while the pair may still touch it
+  tc_fence_after();
+  if (warp == 2) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols));
+  }
+}
+
+// ------------------ the kernel, token-N version (CTA pairs) ------------------
+// The forward expert GEMMs (kEpiRelu, kEpiSwiglu, kEpiScale, kEpiScaleAdd)
+// with the operands' roles swapped: the weights are the MMA's M side (256
+// rows a pair tile, 128 a CTA) and a group's token rows its N side, in tiles
+// of at most 256 rows cut to multiples of 32.  A group of n rows runs
+// ceil(n / 256) token tiles of nearly equal width, so a tile computes at most
+// 31 padding rows: an expert of 277 rows costs 288 rows of MMA work instead
+// of 384 on 128-row tiles or 512 on 256-row tiles.  The accumulator holds one
+// weight row (output column) per TMEM lane and one token per column; the
+// epilogue transposes it through shared memory into whole output rows.
+//   A (weights): ReLU and the down-projection take 128 consecutive rows of W
+//     per CTA; SwiGLU takes 64 rows of W1 (gate) and the same 64 rows of W3
+//     (up), so a CTA's accumulator holds both halves of its 64 outputs.
+//   B (tokens): the tile's N rows, N / 2 per CTA, in TMA boxes of 16 rows;
+//     or, with gather_rows (the up-projection of moe_forward), the routed
+//     rows straight from x: row r of a group is x[gather_rows[off + r]],
+//     four rows per TMA tile::gather4 load, so no permuted copy of x is
+//     written or read.  Warp 3 stages each tile's row indices in shared
+//     memory (two slots, mbarrier handshakes) ahead of the producer.
+// Tiles run group by group, weight tile outer and token tile inner, so the
+// pairs working at once share a weight tile in L2; they are dealt
+// round-robin (no stream-K tail).
+constexpr int kTnTokBox = 16;            // token rows per TMA box
+constexpr int kTnMaxN = 256;             // token rows per tile (the MMA's N)
+constexpr int kTnGran = 32;              // tile widths are multiples of this
+constexpr int kTnStgBytes = 2304;        // per epilogue warp: 33 rows of 64 bytes (+ pad)
+constexpr int kTnXchBytes = 16384;       // SwiGLU: 2 warp pairs x 2 buffers x 4 KB
+
+struct TnTile {
+  int g, wt, n0, n, valid;               // group, weight tile, first token, MMA N, rows stored
+};
+
+// tiles per group: weight tiles x token tiles
+__device__ __forceinline__ int tn_token_tiles(int rows) { return (rows + kTnMaxN - 1) / kTnMaxN; }
+
+__device__ __forceinline__ TnTile tn_decode(int tile, const int *prefix, const int *rows, int G) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {                      // largest g with prefix[g] <= tile
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= tile) lo = mid;
+    else hi = mid - 1;
+  }
+  TnTile t;
+  t.g = lo;
+  const int r = rows[lo];
+  const int nn = tn_token_tiles(r);
+  const int width = ((r + nn - 1) / nn + kTnGran - 1) / kTnGran * kTnGran;
+  const int local = tile - prefix[lo];
+  t.wt = local / nn;
+  t.n0 = (local - t.wt * nn) * width;
+  t.valid = min(width, r - t.n0);
+  t.n = (t.valid + kTnGran - 1) / kTnGran * kTnGran;        // the last tile may be narrower
+  return t;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// NT tokens x this warp's 32 output columns (lane l: column col_base + l;
+// vals[i]: token tok0 + i of the tile) into the output rows, as 16-byte
+// pieces of whole 64-byte row segments.  Adjacent lanes first trade halves
+// (even lanes keep columns l, l+1 of the first NT/2 tokens, odd lanes
+// columns l-1, l of the others) and write packed bf16 pairs into a staging
+// area of one 64-byte row per token (the second half of the tokens one row
+// further on, so that the two halves fall on different banks); then every
+// lane reads back 16-byte pieces and stores them.  Tokens at or past
+// `valid` and columns past the output width are not written.  kEpiScaleAdd
+// adds the piece into the token's row of y (routed: add_rows[out row];
+// static group: its token index) with bf16 vector reductions instead.
+template <int NT, int EPI>
+__device__ __forceinline__ void store_tn(const Params &P, const float (&vals)[NT], int64_t row0,
+                                         int tok0, int valid, bool routed, int64_t static_tok0,
+                                         int col_base, uint8_t *stg, int lane) {
+  __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
+  const int64_t ld = P.N;
+  const bool odd = (lane & 1) != 0;
+  uint32_t *sw = reinterpret_cast<uint32_t *>(stg);
+#pragma unroll
+  for (int i = 0; i < NT / 2; ++i) {
+    const float send = odd ? vals[i] : vals[NT / 2 + i];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    const uint32_t w = odd ? pack_bf16x2(recv, vals[NT / 2 + i]) : pack_bf16x2(vals[i], recv);
+    const int srow = odd ? NT / 2 + i + 1 : i;
+    sw[srow * 16 + (lane >> 1)] = w;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < NT / 8; ++it) {
+    const int n = it * 8 + (lane >> 2), p = lane & 3;
+    const int srow = n + (n >= NT / 2 ? 1 : 0);
+    const uint4 w = *reinterpret_cast<const uint4 *>(stg + srow * 64 + p * 16);
+    const int tok = tok0 + n;
+    const int col = col_base + p * 8;
+    if (tok < valid && col < P.N) {
+      if constexpr (EPI == kEpiScaleAdd) {
+        const int64_t dest = routed ? (int64_t)P.add_rows[row0 + tok] : static_tok0 + tok;
+        if (dest >= 0 && dest < P.src_rows) red_add_bf16x8(out + dest * ld + col, w);
+        else raise_error(P.err, kErrBadIndex);
+      } else {
+        *reinterpret_cast<uint4 *>(out + (row0 + tok) * ld + col) = w;
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// Epilogue of one token-N tile, this warp's 32 TMEM lanes (weight rows) x
+// the tile's tokens, 32 tokens (TMEM columns) at a time.  SwiGLU: warps
+// ew and ew + 2 hold the gate and up rows of the same 32 outputs; they trade
+// half of each 32-token chunk through `xch` (two buffers, so one barrier of
+// the two warps per chunk suffices) and each stores 16 tokens of h.
+template <int EPI>
+__device__ __forceinline__ void epilogue_tn(const Params &P, uint32_t taddr, const TnTile &tl,
+                                            bool routed, int64_t row0, int64_t static_tok0,
+                                            int col_base, uint8_t *stg, float *xch, int ew, int lane,
+                                            int &xpar) {
+  for (int c = 0; c < tl.n / 32; ++c) {
+    if (32 * c >= tl.valid) break;                            // the same for the whole tile
+    float v[32];
+    acc_cols(taddr, 32 * c, nullptr, v);
+    if constexpr (EPI == kEpiSwiglu) {
+      const int pr = ew & 1;                                  // warps pr (gate) and pr + 2 (up)
+      const bool gate_warp = ew < 2;
+      float *xg = xch + (size_t)(pr * 2 + xpar) * 1024;       // gate values of tokens 16..31
+      float *xu = xg + 512;                                   // up values of tokens 0..15
+      if (gate_warp) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xg[i * 32 + lane] = v[16 + i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xu[i * 32 + lane] = v[i];
+      }
+      named_bar_sync(1 + pr, 64);
+      float h[16];
+      if (gate_warp) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) h[i] = v[i] / (1.0f + __expf(-v[i])) * xu[i * 32 + lane];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float g = xg[i * 32 + lane];
+          h[i] = g / (1.0f + __expf(-g)) * v[16 + i];
+        }
+      }
+      xpar ^= 1;
+      store_tn<16, EPI>(P, h, row0, 32 * c + (gate_warp ? 0 : 16), tl.valid, routed, static_tok0,
+                        col_base, stg, lane);
+    } else {
+      if constexpr (EPI == kEpiRelu) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.0f);
+      } else {
+        // gated rows: the gate of token 32c + i (routed groups; static: 1)
+        float gm = 1.0f;
+        if (routed && 32 * c + lane < tl.valid) gm = P.row_gate[row0 + 32 * c + lane];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= __shfl_sync(0xffffffffu, gm, i);
+      }
+      store_tn<32, EPI>(P, v, row0, 32 * c, tl.valid, routed, static_tok0, col_base, stg, lane);
+    }
+  }
+}
+
+template <int EPI, int BKS>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap map_tok,
+                           const __grid_constant__ CUtensorMap map_tok_static,
+                           const __grid_constant__ CUtensorMap map_w,
+                           const __grid_constant__ CUtensorMap map_w3, const Params P) {
+  constexpr bool kSwiglu = EPI == kEpiSwiglu;
+  constexpr int STAGES = BKS == 2 ? kPairStages2 : kPairStages;
+  constexpr uint32_t kWBytes = BM * BK * 2;                     // weights: 16 KB a k-block and CTA
+  constexpr uint32_t kTokBytes = (kTnMaxN / 2) * BK * 2;        // token rows: up to 16 KB
+  constexpr uint32_t stage_bytes = BKS * (kWBytes + kTokBytes);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ int s_prefix[kMaxGroups + 1];
+  __shared__ int s_off[kMaxGroups];
+  __shared__ int s_rows[kMaxGroups];
+  __shared__ __align__(8) uint64_t full_bar[kPairStages];
+  __shared__ __align__(8) uint64_t empty_bar[kPairStages];
+  __shared__ __align__(8) uint64_t accf_bar[2];
+  __shared__ __align__(8) uint64_t acce_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t s_tmem_base;
+  __shared__ volatile int s_abort;
+  __shared__ uint64_t s_limit_sh;
+  __shared__ __align__(16) int s_idx[2][kTnMaxN / 2];  // gathered rows of a tile (two slots)
+  __shared__ __align__(8) uint64_t idx_full[2];
+  __shared__ __align__(8) uint64_t idx_empty[2];
+
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~(uintptr_t)1023);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const bool gather = P.gather_rows != nullptr;
+
+  if (tid == 32) {
+    for (int st = 0; st < STAGES; ++st) {
+      mbar_init(&full_bar[st], 1);                     // the even CTA's expect_tx arrival
+      mbar_init(&empty_bar[st], 1);
+    }
+    for (int sl = 0; sl < 2; ++sl) {
+      mbar_init(&idx_full[sl], 1);
+      mbar_init(&idx_empty[sl], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&accf_bar[a], 1);
+      mbar_init(&acce_bar[a], 2 * 4 * 32);
+    }
+    mbar_init(&drain_bar, 1);
+    s_abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  if (tid == 0) {
+    tma_prefetch_map(&map_tok);
+    tma_prefetch_map(&map_w);
+    if (P.n_static > 0) tma_prefetch_map(&map_tok_static);
+    if (kSwiglu) tma_prefetch_map(&map_w3);
+  }
+  pdl_wait();              // what earlier kernels wrote is visible from here on
+  pdl_trigger();
+  if (tid == 0) s_limit_sh = wait_limit_ns(P.err);
+  if (warp == 0) {
+    // group table: rows of each group and the tile prefix (weight tiles x token tiles)
+    int carry = 0;
+    for (int base = 0; base < P.G; base += 32) {
+      const int g = base + lane;
+      int tiles = 0;
+      if (g < P.G) {
+        int off = 0, rows = 0;
+        if (g < P.n_routed) {
+          off = P.offsets[g];
+          rows = P.offsets[g + 1] - off;
+          if (rows < 0 || off < 0 || (int64_t)off + rows > P.seg_rows) {
+            raise_error(P.err, kErrBadIndex);
+            rows = 0;
+            off = 0;
+          }
+        } else {
+          rows = (int)P.rows_static;
+        }
+        s_off[g] = off;
+        s_rows[g] = rows;
+        tiles = tn_token_tiles(rows) * P.nt;
+      }
+      int x = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (g < P.G) s_prefix[g] = carry + x - tiles;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) s_prefix[P.G] = carry;
+  }
+  tc_fence_before();
+  cluster_sync_all();              // barriers of both CTAs initialised before any remote use
+  tc_fence_after();
+
+  const uint32_t tmem_base = s_tmem_base;
+  const uint64_t s_limit = s_limit_sh;
+  const int KB = P.K / (BK * BKS);                     // stages of K per tile
+  const int total = s_prefix[P.G];
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0, armed_parity = 0;
+    int islot = 0;
+    uint32_t iphase = 0;
+    bool ok = true;
+    for (int tile = pair; ok && tile < total; tile += npairs) {
+      const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G);
+      const bool routed = tl.g < P.n_routed;
+      const bool gathered = gather && routed;
+      if (gathered && !mbar_wait(&idx_full[islot], iphase, &s_abort, P.err, s_limit)) { ok = false; break; }
+      const CUtensorMap *mt = routed ? &map_tok : &map_tok_static;
+      const int64_t tok_row =
+          (routed ? (int64_t)s_off[tl.g]
+                  : P.a_static_base + (int64_t)(tl.g - P.n_routed) * P.a_static_stride) +
+          tl.n0 + (int64_t)rank * (tl.n / 2);
+      const int w_row = kSwiglu ? tl.g * P.N + tl.wt * 128 + (int)rank * 64
+                                : tl.g * P.N + tl.wt * 256 + (int)rank * 128;
+      const int nbox = tl.n / 2 / kTnTokBox;
+      const uint32_t tx = 2u * BKS * (kWBytes + (uint32_t)(tl.n / 2) * BK * 2);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err, s_limit)) { ok = false; break; }
+        uint8_t *sa = smem + (size_t)stage * stage_bytes;
+        uint8_t *sb = sa + BKS * kWBytes;
+        const uint32_t fb = smem_u32(&full_bar[stage]) & 0xFEFFFFFFu;   // the even CTA's barrier
+        if (rank == 0) {
+          mbar_expect_tx(&full_bar[stage], tx);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        }
+#pragma unroll
+        for (int q = 0; q < BKS; ++q) {
+          const int kx = (kb * BKS + q) * BK;
+          if (kSwiglu) {
+            tma_load_2d_pair(sa + q * kWBytes, &map_w, fb, kx, w_row);
+            tma_load_2d_pair(sa + q * kWBytes + kWBytes / 2, &map_w3, fb, kx, w_row);
+          } else {
+            tma_load_2d_pair(sa + q * kWBytes, &map_w, fb, kx, w_row);
+          }
+          if (gathered) {
+            const int4 *ix = reinterpret_cast<const int4 *>(s_idx[islot]);
+            for (int j = 0; j < tl.n / 8; ++j)
+              tma_gather4_pair(sb + q * kTokBytes + j * 512, mt, fb, kx, ix[j]);
+          } else {
+            for (int j = 0; j < nbox; ++j)
+              tma_load_2d_pair(sb + q * kTokBytes + j * (kTnTokBox * 128), mt, fb, kx,
+                               (int)(tok_row + j * kTnTokBox));
+          }
+        }
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (gathered && ok) {
+        mbar_arrive(&idx_empty[islot]);         // the coordinates were taken at issue
+        if (++islot == 2) { islot = 0; iphase ^= 1u; }
+      }
+    }
+    if (!ok && rank == 0) {
+      for (int st = 0; st < STAGES; ++st)
+        if (armed & (1u << st)) mbar_wait_drain(&full_bar[st], (armed_parity >> st) & 1u);
+    }
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------ MMA issuer (even CTA only) ------------------------
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int tile = pair; ok && tile < total; tile += npairs) {
+      const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G);
+      const uint32_t idesc = idesc_bf16(2 * BM, tl.n);
+      if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err, s_limit)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait<true>(&full_bar[stage], phase, &s_abort, P.err, s_limit)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + (size_t)stage * stage_bytes);
+        const uint32_t b_addr = a_addr + BKS * kWBytes;
+#pragma unroll
+        for (int q = 0; q < BKS; ++q) {
+#pragma unroll
+          for (int k = 0; k < BK / kUmmaK; ++k)
+            umma_bf16_pair(d_tmem, sw128_desc(a_addr + q * kWBytes + k * kUmmaK * 2),
+                           sw128_desc(b_addr + q * kTokBytes + k * kUmmaK * 2), idesc,
+                           (kb > 0 || q > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit_pair_both(&empty_bar[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      umma_commit_pair_both(&accf_bar[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    umma_commit_pair_local(&drain_bar);
+    mbar_wait_drain(&drain_bar, 0);
+  } else if (gather && warp == 3) {
+    // ------------- row indices of the gathered tiles, one tile ahead -------------
+    int islot = 0;
+    uint32_t iphase = 0;
+    for (int tile = pair; tile < total; tile += npairs) {
+      const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G);
+      if (tl.g >= P.n_routed) continue;                 // static groups read x as stored
+      int okw = 1;
+      if (lane == 0) okw = mbar_wait(&idx_empty[islot], iphase ^ 1u, &s_abort, P.err, s_limit) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+      const int rows = s_rows[tl.g], off = s_off[tl.g];
+      const int half = tl.n / 2, r0 = tl.n0 + (int)rank * half;
+      for (int i = lane; i < half; i += 32) {
+        const int r = min(r0 + i, rows - 1);           // padding rows repeat the last row
+        int t = P.gather_rows[off + r];
+        if (t < 0 || t >= P.src_rows) {
+          raise_error(P.err, kErrBadIndex);
+          t = 0;
+        }
+        s_idx[islot][i] = t;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&idx_full[islot]);
+      if (++islot == 2) { islot = 0; iphase ^= 1u; }
+    }
+  } else if (warp >= 4) {
+    // -------------------------------- epilogue --------------------------------
+    const int ew = warp - 4;                           // TMEM lanes 32 ew .. 32 ew + 31
+    uint8_t *stg = smem + (size_t)STAGES * stage_bytes + (size_t)ew * kTnStgBytes;
+    float *xch = reinterpret_cast<float *>(smem + (size_t)STAGES * stage_bytes + 4 * kTnStgBytes);
+    const uint32_t acce_even0 = mapa_shared(smem_u32(&acce_bar[0]), 0);
+    const uint32_t acce_even1 = mapa_shared(smem_u32(&acce_bar[1]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int xpar = 0;
+    for (int tile = pair; tile < total; tile += npairs) {
+      const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G);
+      // (warp-uniform exits: the epilogue's TMEM loads and stores are warp-wide)
+      if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err, s_limit))) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (uint32_t)(acc * kAccCols) + ((uint32_t)(ew * 32) << 16);
+      const bool routed = tl.g < P.n_routed;
+      const int64_t row0 = (routed ? (int64_t)s_off[tl.g]
+                                   : P.out_static_base + (int64_t)(tl.g - P.n_routed) * P.rows_static) +
+                           tl.n0;
+      const int col_base = kSwiglu ? tl.wt * 128 + (int)rank * 64 + 32 * (ew & 1)
+                                   : tl.wt * 256 + (int)rank * 128 + 32 * ew;
+      epilogue_tn<EPI>(P, taddr, tl, routed, row0, (int64_t)tl.n0, col_base, stg, xch, ew, lane, xpar);
       tc_fence_before();
       mbar_arrive_cluster(acc == 0 ? acce_even0 : acce_even1);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
@@ -1655,6 +2112,36 @@ cudaError_t launch_pair(const Params &P, const CUtensorMap &ma, const CUtensorMa
   return launch_kernel(kern, 2 * pairs, kThreads, smem, s, ma, mas, mb, mb3, P);
 }
 
+// Token-N launch: as many 2-CTA clusters as fit at once, fewer when there are
+// fewer tiles.
+template <int EPI, int BKS>
+cudaError_t launch_tn(const Params &P, const CUtensorMap &mt, const CUtensorMap &mts,
+                      const CUtensorMap &mw, const CUtensorMap &mw3, int64_t max_tiles, size_t smem,
+                      cudaStream_t s) {
+  auto kern = grouped_gemm_tn_kernel<EPI, BKS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  static int max_clusters[8][4] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int &mc = max_clusters[dev & 7][(EPI == kEpiSwiglu ? 2 : 0) + (BKS - 1)];
+  if (mc == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = device_sms() / 2;
+    }
+    mc = n;
+  }
+  const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(mc, max_tiles));
+  return launch_kernel(kern, 2 * pairs, kThreads, smem, s, mt, mts, mw, mw3, P);
+}
+
 }  // namespace
 
 cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
@@ -1730,6 +2217,55 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   if (g.kgroup && (g.epi != kEpiStoreF32 || g.n_routed != 0 || !g.kseg || g.M <= 0 ||
                    (g.out2 && (g.split_m <= 0 || g.split_m >= g.M))))
     return cudaErrorInvalidValue;
+
+  // token-N tiles (weights on the MMA's M side) for the forward expert GEMMs
+  // of short groups
+  const bool tn_epi = g.epi == kEpiRelu || g.epi == kEpiSwiglu || g.epi == kEpiScale ||
+                      g.epi == kEpiScaleAdd;
+  if (tn_epi && !g.kgroup && g.n_routed > 0 && !g.b_mn && g.ksplit <= 1 &&
+      g.max_routed_rows / g.n_routed < MOE_TN_MAX_ROWS) {
+    const bool swiglu = g.epi == kEpiSwiglu;
+    Params Q = P;
+    Q.nt = swiglu ? (g.N + 127) / 128 : (g.N + 255) / 256;     // weight tiles per group
+    Q.sk_part = nullptr;
+    Q.sk_flags = nullptr;
+    CUtensorMap mt, mts, mw, mw3;
+    // routed rows: x_perm in 16-row boxes, or x itself in one-row boxes for
+    // the tile::gather4 loads
+    if (g.gather_rows) {
+      if (!make_map(&mt, g.gather_src, (uint64_t)g.K, (uint64_t)g.src_rows, 1)) return cudaErrorInvalidValue;
+    } else if (!make_map(&mt, g.a, (uint64_t)g.K, (uint64_t)g.a_rows, kTnTokBox)) {
+      return cudaErrorInvalidValue;
+    }
+    if (!make_map(&mts, g.a_static ? g.a_static : g.a, (uint64_t)g.K,
+                  (uint64_t)(g.a_static ? g.a_static_rows : g.a_rows), kTnTokBox))
+      return cudaErrorInvalidValue;
+    const uint32_t wbox = swiglu ? 64u : 128u;
+    if (!make_map(&mw, g.b, (uint64_t)g.K, (uint64_t)g.b_rows, wbox)) return cudaErrorInvalidValue;
+    if (!make_map(&mw3, swiglu ? g.b3 : g.b, (uint64_t)g.K, (uint64_t)g.b_rows, wbox))
+      return cudaErrorInvalidValue;
+    const int64_t tt_routed = (g.max_routed_rows + kTnMaxN - 1) / kTnMaxN + g.n_routed;
+    const int64_t tt_static = (int64_t)g.n_static * ((g.rows_static + kTnMaxN - 1) / kTnMaxN);
+    const int64_t max_tiles = (tt_routed + tt_static) * Q.nt;
+    const double macs = (double)(g.max_routed_rows + (int64_t)g.n_static * g.rows_static) * g.N *
+                        g.K * (swiglu ? 2 : 1);
+    const bool bk2 = MOE_PAIR_BK128 && g.K % (2 * BK) == 0 && macs >= 2e11;
+    const size_t stage = (size_t)(bk2 ? 2 : 1) * (kABytes + (size_t)(kTnMaxN / 2) * BK * 2);
+    const size_t tsmem = (bk2 ? (size_t)kPairStages2 : (size_t)kPairStages) * stage + 1024 +
+                         4 * (size_t)kTnStgBytes + (swiglu ? (size_t)kTnXchBytes : 0);
+#define MOE_TN_CASE(E_)                                                                  \
+  case E_:                                                                               \
+    return bk2 ? launch_tn<E_, 2>(Q, mt, mts, mw, mw3, max_tiles, tsmem, s)              \
+               : launch_tn<E_, 1>(Q, mt, mts, mw, mw3, max_tiles, tsmem, s);
+    switch (g.epi) {
+      MOE_TN_CASE(kEpiRelu)
+      MOE_TN_CASE(kEpiSwiglu)
+      MOE_TN_CASE(kEpiScale)
+      MOE_TN_CASE(kEpiScaleAdd)
+      default: return cudaErrorInvalidValue;
+    }
+#undef MOE_TN_CASE
+  }
 
   // CTA pairs for the expert GEMMs whose groups are long enough that 256-row
   // tiles waste little (average routed rows per expert >= MOE_PAIR_MIN_ROWS),

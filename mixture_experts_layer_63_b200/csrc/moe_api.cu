@@ -95,11 +95,16 @@ moe_status validate(const moe_config *c) {
   return MOE_OK;
 }
 
-// moe_forward gathers the routed rows inside the up-projection GEMM (bf16);
-// MOE_FUSED_GATHER=0 at build time runs the separate gather kernel instead
+// MOE_FUSED_GATHER=1 at build time: moe_forward's up-projection gathers the
+// routed rows of x itself on every tile kernel (16-byte cp.async copies);
+// by default only the token-N kernel does (TMA tile::gather4), and the
+// others read x_perm written by the gather kernel.
 #ifndef MOE_FUSED_GATHER
 #define MOE_FUSED_GATHER 0
 #endif
+static bool forward_gathers(const moe_config *c, int64_t rows_cap) {
+  return c->dtype == MOE_BF16 && (MOE_FUSED_GATHER || expert_gemm_gathers(c, rows_cap));
+}
 
 #ifndef MOE_DOWN_REVERSE
 #define MOE_DOWN_REVERSE 0
@@ -147,7 +152,7 @@ WsLayout make_layout(const moe_config *c) {
   L.row_token = take((size_t)L.rows_cap * 4);
   L.row_gate = take((size_t)L.rows_cap * 4);
   // moe_forward's x_perm: bf16 layers gather inside the up-projection GEMM
-  const bool fused_gather = c->dtype == MOE_BF16 && MOE_FUSED_GATHER;
+  const bool fused_gather = forward_gathers(c, L.rows_cap);
   L.x_perm = take(fused_gather ? 0 : (size_t)L.rows_cap * c->d_model * es);
   L.h = take((size_t)L.rows_total * c->d_ff * es);
   L.y_rows = take((size_t)L.rows_total * c->d_model * es);     // rows in the layer dtype
@@ -317,6 +322,7 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
 static int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 struct BwLayout {
+  size_t x_perm;            // the routed rows of x, when the forward left no x_perm
   size_t dy_perm, au, dau, dx_rows, kseg, kseg_r, dyT, hT, dauT, xT, dgate, dg_part, dl, dl_pad,
       dlT, xTr, wrT, dx_router, total;
   int64_t kp_max, Ep, Tp;
@@ -338,6 +344,7 @@ static BwLayout make_bw_layout(const moe_config *c, const WsLayout &L) {
     o = align256(o + bytes);
     return at;
   };
+  B.x_perm = take(forward_gathers(c, L.rows_cap) ? (size_t)L.rows_cap * d * 2 : 0);
   B.dy_perm = take((size_t)L.rows_cap * d * 2);
   B.au = take((size_t)L.rows_total * B.fw * 2);
   B.dau = take((size_t)L.rows_total * B.fw * 2);
@@ -380,7 +387,7 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
   const int32_t *row_token = reinterpret_cast<const int32_t *>(ws + L.row_token);
   const float *row_gate = reinterpret_cast<const float *>(ws + L.row_gate);
   const void *h = ws + L.h;
-  const bool fused_gather = c->dtype == MOE_BF16 && MOE_FUSED_GATHER;
+  const bool fused_gather = forward_gathers(c, L.rows_cap);
   void *dy_perm = bw + B.dy_perm;
   void *au = bw + B.au, *dau = bw + B.dau;
   float *dx_rows = reinterpret_cast<float *>(bw + B.dx_rows);
@@ -396,15 +403,21 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
     if (e != cudaSuccess) return e; \
   } while (0)
 
+  // 1. the routed rows of x: the forward's x_perm, or gathered here when the
+  // forward's up-projection read them from x itself
+  const void *xp = ws + L.x_perm;
+  if (fused_gather) {
+    MOE_TRY(launch_gather_bf16_rows(x, bw + B.x_perm, row_token, offsets, E, T, (int)d, L.rows_cap,
+                                    err, s));
+    xp = bw + B.x_perm;
+  }
   // 2. pre-activations recomputed: A (| U) [rows_total][fw]
   GroupedGemm up{};
   up.epi = swiglu ? kEpiPreSwiglu : kEpiPreRelu;
   up.K = (int)d;
   up.N = (int)f;
-  up.a = fused_gather ? x : static_cast<const void *>(ws + L.x_perm);
-  up.a_rows = fused_gather ? T : L.rows_cap;
-  up.gather_rows = fused_gather ? row_token : nullptr;
-  up.gather_src = fused_gather ? x : nullptr;
+  up.a = xp;
+  up.a_rows = L.rows_cap;
   up.src_rows = T;
   up.a_static = x;
   up.a_static_rows = T;
@@ -746,7 +759,7 @@ static moe_status forward_impl(const moe_config *cfg, const void *x, const void 
   if (e == cudaSuccess) e = mark(1);
   // token choice: the gate wrote the unit histogram into the workspace.
   // bf16: the up-projection gathers the rows of x itself (no x_perm)
-  const bool fused_gather = cfg->dtype == MOE_BF16 && MOE_FUSED_GATHER;
+  const bool fused_gather = forward_gathers(cfg, L.rows_cap);
   if (e == cudaSuccess)
     e = launch_permute(cfg, L, w, cfg->mode == MOE_TOKEN_CHOICE, x, topk_idx, topk_gate, probs,
                        counts, offsets, tok_rows, row_token, row_gate, x_perm, n_dropped, s,
@@ -834,6 +847,16 @@ moe_status moe_check_device_errors(void *ws, size_t ws_bytes, moe_stream_t strea
 moe_status moe_workspace_init(void *ws, size_t ws_bytes, moe_stream_t stream) {
   if (!ws || ws_bytes < 256) return MOE_ERR_INVALID_ARG;
   return cuda_status(cudaMemsetAsync(ws, 0, std::min(ws_bytes, kCtrlBytes),
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_workspace_set_wait_limit(void *ws, size_t ws_bytes, uint64_t limit_ns,
+                                        moe_stream_t stream) {
+  if (!ws || ws_bytes < kCtrlBytes || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return MOE_ERR_INVALID_ARG;
+  // from host memory: the value is staged before the call returns
+  return cuda_status(cudaMemcpyAsync(static_cast<char *>(ws) + kWaitLimitOffset, &limit_ns,
+                                     sizeof(limit_ns), cudaMemcpyHostToDevice,
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -401,6 +401,10 @@ __device__ uint64_t block_select_kth_largest(int n, int m, KeyOf key_of, int *hi
 // ---------------------------------------------------------------------------
 // token choice, keep-fraction: per-expert affinity selection
 // ---------------------------------------------------------------------------
+// lists of at most this many assignments select by counting (n^2 / 1024
+// compares a thread) instead of the 8-pass radix select
+constexpr int kKeepCountMax = 2048;
+
 __global__ void __launch_bounds__(1024) keep_select_kernel(
     const int32_t *__restrict__ sorted_q, const int32_t *__restrict__ cnt_off,
     const int32_t *__restrict__ kept, const int32_t *__restrict__ offsets,
@@ -410,6 +414,7 @@ __global__ void __launch_bounds__(1024) keep_select_kernel(
   __shared__ int scratch[32];
   __shared__ uint64_t s_prefix;
   __shared__ int s_remaining;
+  __shared__ uint64_t s_keys[kKeepCountMax];
   pdl_wait();
   pdl_trigger();
   const int e = blockIdx.x;
@@ -424,7 +429,25 @@ __global__ void __launch_bounds__(1024) keep_select_kernel(
   };
   uint64_t thr = 0ull;          // keep keys >= thr
   bool keep_all = m >= n, keep_none = m <= 0;
-  if (!keep_all && !keep_none) thr = block_select_kth_largest(n, m, key_of, hist, &s_prefix, &s_remaining);
+  if (!keep_all && !keep_none) {
+    if (n <= kKeepCountMax) {
+      // short lists: the m-th largest key by counting, for each key, the keys
+      // above it (keys are distinct: each token appears once in a list); the
+      // key with exactly m - 1 above it is the threshold
+      for (int i = threadIdx.x; i < n; i += blockDim.x) s_keys[i] = key_of(i);
+      __syncthreads();
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const uint64_t ki = s_keys[i];
+        int above = 0;
+        for (int j = 0; j < n; ++j) above += s_keys[j] > ki ? 1 : 0;
+        if (above == m - 1) s_prefix = ki;
+      }
+      __syncthreads();
+      thr = s_prefix;
+    } else {
+      thr = block_select_kth_largest(n, m, key_of, hist, &s_prefix, &s_remaining);
+    }
+  }
   const int row0 = offsets[e];
   int done = 0;
   for (int c = 0; c < n; c += blockDim.x) {

@@ -32,6 +32,9 @@ namespace moe {
 namespace {
 
 constexpr int kTokWarps = kUnitTokens;     // one warp per token, one unit per block
+#ifndef MOE_GATE8
+#define MOE_GATE8 1
+#endif
 
 struct GateParams {
   const float *logits_in;     // [T, E] (null when the router is fused)
@@ -372,6 +375,233 @@ __global__ void __launch_bounds__(kTokWarps * 32) route_gate_kernel(const GatePa
   }
 }
 
+// ---------------------------------------------------------------------------
+// Gate for more than 32 experts: eight lanes per token, four tokens a warp,
+// one 32-token unit a block (256 threads).  Lane s of a token's eight holds
+// the contiguous experts [s * EPL, s * EPL + EPL) (EPL >= E / 8), so
+//   * the softmax denominator, summed one fp32 add at a time in ascending
+//     expert order, runs along the eight lanes in turn (each lane extends
+//     the running sum with its own experts and hands it to the next);
+//   * maxima and arg-maxima take three shuffle steps;
+//   * a token costs a quarter of the instructions of one warp per token.
+// Same arithmetic as route_gate_kernel, so the same bits.
+// ---------------------------------------------------------------------------
+template <int EPL>
+__global__ void __launch_bounds__(256) gate8_kernel(const GateParams P) {
+  __shared__ int s_hist[kMaxTopK * kMaxExperts];          // [k][E] of this unit
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int s = lane & 7;                                  // sub-lane of the token
+  const int gbase = lane & ~7;
+  const int E = P.E, k = P.k;
+  pdl_wait();
+  pdl_trigger();
+  const int64_t t = (int64_t)blockIdx.x * kUnitTokens + warp * 4 + (lane >> 3);
+  const bool live = t < P.T;
+  const int hist_ints = P.hist ? k * E : 0;
+  for (int i = threadIdx.x; i < hist_ints; i += blockDim.x) s_hist[i] = 0;
+  if (P.hist) __syncthreads();
+  if (P.y_zero && live)
+    for (int v = s; v < P.y_vecs; v += 8) P.y_zero[t * P.y_vecs + v] = make_uint4(0u, 0u, 0u, 0u);
+  const int e0 = s * EPL;
+
+  // ---- logits: partial sums of the K parts added in order, then the bias --
+  float l[EPL];
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const int e = e0 + j;
+    float v = -INFINITY;
+    if (live && e < E) {
+      v = P.logits_in[t * E + e];
+      for (int sp = 1; sp < P.nsplit; ++sp) v = __fadd_rn(v, P.logits_in[sp * P.split_stride + t * E + e]);
+      if (P.bias) v = __fadd_rn(v, P.bias[e]);
+      if (P.logits_out) P.logits_out[t * E + e] = v;
+    }
+    l[j] = v;
+  }
+
+  // ---- max, exps, the sequential sum, probabilities -------------------------
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) m = fmaxf(m, l[j]);
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float p[EPL];
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) p[j] = (e0 + j < E) ? exp_det(__fsub_rn(l[j], m)) : 0.f;
+  float S = 0.f;
+#pragma unroll 1
+  for (int step = 0; step < 8; ++step) {
+    const float prev = __shfl_sync(0xffffffffu, S, gbase | ((step + 7) & 7));
+    if (s == step) {
+      float acc = prev;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (e0 + j < E) acc = (step == 0 && j == 0) ? p[0] : __fadd_rn(acc, p[j]);
+      S = acc;
+    }
+  }
+  S = __shfl_sync(0xffffffffu, S, gbase | 7);
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const int e = e0 + j;
+    p[j] = __fdiv_rn(p[j], S);
+    if (live && e < E && P.probs) P.probs[t * E + e] = p[j];
+  }
+  if (P.topk_idx == nullptr) return;          // expert choice: probabilities only
+
+  // ---- selection keys and gate values of the routing rule -------------------
+  float key[EPL], gsrc[EPL];
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const int e = e0 + j;
+    key[j] = l[j];
+    gsrc[j] = p[j];
+    if (P.rule != 0 && e < E) {
+      const float st = P.state[e];
+      if (P.rule == 1) {
+        key[j] = __fadd_rn(p[j], st);
+        gsrc[j] = key[j];
+      } else {
+        key[j] = __fadd_rn(l[j], __fmul_rn(P.alpha, __fsub_rn(1.0f, st)));
+      }
+    }
+  }
+
+  // ---- group limit: groups of E/n_groups experts, keep the best topk_groups --
+  uint32_t allowed = 0xffffffffu;
+  int grp[EPL];
+  const int gsz = P.n_groups > 0 ? E / P.n_groups : E;
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) grp[j] = (e0 + j) / gsz;
+  if (P.n_groups > 0) {
+    float gs0 = -INFINITY, gs1 = -INFINITY, gs2 = -INFINITY, gs3 = -INFINITY;   // groups s + 8 i
+#pragma unroll 1
+    for (int g = 0; g < P.n_groups; ++g) {
+      float v = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (e0 + j < E && grp[j] == g) v = fmaxf(v, key[j]);
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+      if ((g & 7) == s) {
+        const int i = g >> 3;
+        if (i == 0) gs0 = v;
+        else if (i == 1) gs1 = v;
+        else if (i == 2) gs2 = v;
+        else gs3 = v;
+      }
+    }
+    allowed = 0;
+    uint32_t gtaken = 0;                          // bit i: group s + 8 i chosen
+#pragma unroll 1
+    for (int r = 0; r < P.topk_groups; ++r) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int g = s + 8 * i;
+        const float sc = i == 0 ? gs0 : i == 1 ? gs1 : i == 2 ? gs2 : gs3;
+        if (g < P.n_groups && !((gtaken >> i) & 1u) && (sc > bv || (sc == bv && g < bi))) {
+          bv = sc;
+          bi = g;
+        }
+      }
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      allowed |= 1u << bi;
+      if ((bi & 7) == s) gtaken |= 1u << (bi >> 3);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) grp[j] = 0;
+  }
+
+  // ---- top-k: k rounds of an arg-max over the eight lanes --------------------
+  uint32_t taken = 0;                             // bit j: expert e0 + j chosen
+  float gates[kMaxTopK];
+  int idxs[kMaxTopK];
+  float gsum = 0.f;
+#pragma unroll
+  for (int r = 0; r < kMaxTopK; ++r) {
+    gates[r] = 0.f;
+    idxs[r] = 0;
+    if (r < k) {
+      float bv = -INFINITY, bg = 0.f;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) {
+        const int e = e0 + j;
+        const bool ok = e < E && !((taken >> j) & 1u) && ((allowed >> grp[j]) & 1u);
+        if (ok && (key[j] > bv || (key[j] == bv && e < bi))) {
+          bv = key[j];
+          bi = e;
+          bg = gsrc[j];
+        }
+      }
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        const float og = __shfl_xor_sync(0xffffffffu, bg, o);
+        if (ov > bv || (ov == bv && oi < bi)) {
+          bv = ov;
+          bi = oi;
+          bg = og;
+        }
+      }
+      if (bi >= e0 && bi < e0 + EPL) taken |= 1u << (bi - e0);
+      idxs[r] = bi;
+      gates[r] = bg;
+      gsum = (r == 0) ? bg : __fadd_rn(gsum, bg);
+    }
+  }
+  int my_idx = 0;
+  float my_gate = 0.f;
+#pragma unroll
+  for (int r = 0; r < kMaxTopK; ++r) {
+    if (r < k && s == r) {
+      my_idx = idxs[r];
+      my_gate = P.renormalize ? __fdiv_rn(gates[r], gsum) : gates[r];
+    }
+  }
+  if (live && s < k) {
+    P.topk_idx[t * k + s] = my_idx;
+    P.topk_gate[t * k + s] = my_gate;
+    if (P.hist && my_idx >= 0 && my_idx < E) atomicAdd(&s_hist[s * E + my_idx], 1);
+  }
+  if (P.hist) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < hist_ints; i += blockDim.x) {
+      const int r = i / E, e = i - r * E;
+      // unit of (rank r, this block): group-major numbering, see unit_grid
+      const int g = blockIdx.x / P.nbg, bl = blockIdx.x - g * P.nbg;
+      const int64_t u = ((int64_t)g * P.k + r) * P.nbg + bl;
+      P.hist[u * E + e] = s_hist[i];
+    }
+  }
+}
+
+cudaError_t launch_gate8(const GateParams &P, int blocks, cudaStream_t s) {
+  const int epl = (P.E + 7) / 8;
+#define MOE_GATE8_CASE(n)                                                          \
+  if (epl <= n) return launch_kernel(gate8_kernel<n>, blocks, 256, 0, s, P);
+  MOE_GATE8_CASE(8)
+  MOE_GATE8_CASE(12)
+  MOE_GATE8_CASE(16)
+  MOE_GATE8_CASE(20)
+  MOE_GATE8_CASE(24)
+  MOE_GATE8_CASE(32)
+#undef MOE_GATE8_CASE
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_nv(int NV, const GateParams &P, int blocks, size_t smem, cudaStream_t s) {
 #define MOE_GATE_CASE(n)                                                                       \
   case n: {                                                                                    \
@@ -469,6 +699,9 @@ cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float
     }
     return launch_kernel(kern, blocks, kTokWarps * 32, smem, s, P);
   }
+  // more than 32 experts: eight lanes a token (MOE_GATE8=0 at build time: a
+  // warp a token)
+  if (NV > 1 && MOE_GATE8) return launch_gate8(P, blocks, s);
   return launch_nv(NV, P, blocks, smem, s);
 }
 
