@@ -423,16 +423,16 @@ def run_ours(args, w) -> None:
     tr = NCU_TRAFFIC.get(w.name)
     traffic = tr["bytes"] if tr and tr.get("src") == h else None
 
-    # end to end through the public layer object, host buffers: every step
-    # copies its batch of x from pinned host memory and its y back; the
-    # copies of neighbouring steps overlap the forward (api.HostPipeline).  No
-    # L2 flush: every step streams the expert weights (larger than the L2 on
+    # end to end through the C-ABI call on host buffers (moe_forward_host, via
+    # api.HostPipeline): every step copies its batch of x from pinned host
+    # memory and its y back; two workspaces in turn and copy streams of their
+    # own let the copies of neighbouring steps overlap the forward.  No L2
+    # flush: every step streams the expert weights (larger than the L2 on
     # every workload) and x arrives fresh from the host, as a caller sees it
     layer = api.MoELayer(cfg, inp.w_router, inp.w1, inp.w2, inp.w3, inp.bias,
                          route_state=inp.route_state)
     x_host = [inp.x.cpu().pin_memory() for _ in range(2)]
     y_host = [torch.empty_like(x_host[0]).pin_memory() for _ in range(2)]
-    x_dev = torch.empty_like(inp.x)
     y_dev = torch.empty_like(inp.x)
     pipe = api.HostPipeline(layer)
     for i in range(args.warmup):
@@ -449,23 +449,27 @@ def run_ours(args, w) -> None:
     pipe.s_out.wait_stream(pipe.s_comp)
     e1.record(pipe.s_out)
     pipe.synchronize()
-    api.moe_check_device_errors(layer.ws)
+    for pws in pipe.ws:
+        api.moe_check_device_errors(pws)
     e2e_ms = replicas.max_over_ranks(e0.elapsed_time(e1), dist, device="cuda")
     if dist:
         dist.barrier()
     e2e_value = replicas.throughput(world, w.T, args.steps, e2e_ms)
-    # the same steps one after the other (no overlap), for reference
+    # the same calls one after the other on one stream (no overlap), for reference
+    del pipe
+    hws = api.new_workspace(cfg, host=True)
     torch.cuda.synchronize()
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     seq_ms = 0.0
     for i in range(args.steps):
         s0.record(stream)
-        x_dev.copy_(x_host[i & 1], non_blocking=True)
-        layer(x_dev, out=y_dev)
-        y_host[i & 1].copy_(y_dev, non_blocking=True)
+        api.moe_forward_host(cfg, x_host[i & 1], inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2,
+                             y_host[i & 1], None, hws, route_state=inp.route_state)
         s1.record(stream)
         torch.cuda.synchronize()
         seq_ms += s0.elapsed_time(s1)
+    api.moe_check_device_errors(hws)
+    del hws
     e2e_seq = replicas.throughput(world, w.T, args.steps,
                                   replicas.max_over_ranks(seq_ms, dist, device="cuda"))
 
@@ -547,7 +551,8 @@ def run_ours(args, w) -> None:
                     "sequential_value": e2e_seq,
                     "l2": "not flushed: each step streams %.0f MB of expert weights (L2: 126 MB)"
                           % (weight_bytes / 1e6),
-                    "note": "api.HostPipeline: each step's host copies overlap its neighbours' forwards"},
+                    "note": "moe_forward_host (C ABI, host buffers) with two workspaces and copy "
+                            "streams: each step's host copies overlap its neighbours' forwards"},
             "gpu_launches": launches,
             "clocks": clk,
             "cpu_baseline": cpu,

@@ -147,6 +147,8 @@ typedef struct moe_sizes {
                            /*   choice.  Expert choice's C is ec_capacity                       */
   size_t permute_workspace;/* bytes of scratch moe_permute uses (<= step_workspace): what       */
                            /*   moe_permute_noalloc needs from its fixed array                  */
+  size_t host_workspace;   /* bytes of workspace moe_forward_host needs (>= workspace): the     */
+                           /*   forward's, plus device staging rows for x and y                  */
 } moe_sizes;
 
 /* Sizes of every buffer for `cfg`.  Validates cfg: returns MOE_ERR_INVALID_ARG
@@ -276,6 +278,32 @@ MOE_API moe_status moe_forward(const moe_config *cfg, const void *x, const void 
                        const float *bias, const float *route_state, const void *w1, const void *w3,
                        const void *w2, void *y, int32_t *counts_out, void *ws, size_t ws_bytes,
                        moe_stream_t stream);
+
+/* moe_forward on HOST buffers: x_host [T, d] is copied into the workspace,
+ * the layer runs as moe_forward does, and y comes back to y_host [T, d] (both
+ * in the layer dtype; page-locked host memory lets the copies run
+ * asynchronously at full speed).  Everything is queued without a host sync:
+ * the host buffers must stay untouched until y_host's copy has completed
+ * (synchronise `copy_out`, or `stream` when copy_out is NULL).
+ *   stream: the forward's kernels.  copy_in / copy_out: streams for the
+ *   host-to-device and device-to-host copies (NULL: `stream`).  With two
+ *   copy streams and two workspaces used in turn, the copies of one call
+ *   overlap the forward of the call before and after it; the forwards
+ *   themselves stay in order on `stream`.
+ *   The library orders the calls that share a workspace itself: a call's
+ *   input copy waits for the previous forward on that workspace, its forward
+ *   for the previous output copy.  For that it keeps three CUDA events per
+ *   workspace used here (host objects, no device memory) until the process
+ *   exits.
+ *   ws: at least moe_sizes.host_workspace bytes.  counts_out as moe_forward
+ *   (device memory or NULL).  Errors as moe_forward; MOE_ERR_INVALID_ARG for
+ *   a NULL host buffer. */
+MOE_API moe_status moe_forward_host(const moe_config *cfg, const void *x_host, const void *w_router,
+                                    const float *bias, const float *route_state, const void *w1,
+                                    const void *w3, const void *w2, void *y_host,
+                                    int32_t *counts_out, void *ws, size_t ws_bytes,
+                                    moe_stream_t stream, moe_stream_t copy_in,
+                                    moe_stream_t copy_out);
 
 /* moe_forward that also records caller-created CUDA events on `stream` at
  * its phase boundaries: events[0] before step 1, [1] after steps 1-3a

@@ -32,7 +32,7 @@ EXPORTS = ("moe_query_sizes", "moe_route", "moe_gate", "moe_permute", "moe_exper
            "moe_combine", "moe_forward", "moe_check_device_errors", "moe_workspace_init",
            "moe_status_string", "moe_permute_noalloc", "moe_forward_timed",
            "moe_route_bias_update", "moe_query_backward_size", "moe_backward",
-           "moe_kernel_launches", "moe_workspace_set_wait_limit")
+           "moe_kernel_launches", "moe_workspace_set_wait_limit", "moe_forward_host")
 
 
 class MoeError(RuntimeError):
@@ -57,7 +57,7 @@ class MoeSizes(ctypes.Structure):
     _fields_ = [("rows_cap", ctypes.c_int64), ("rows_total", ctypes.c_int64),
                 ("tok_rows_len", ctypes.c_int64), ("step_workspace", ctypes.c_size_t),
                 ("workspace", ctypes.c_size_t), ("capacity", ctypes.c_int64),
-                ("permute_workspace", ctypes.c_size_t)]
+                ("permute_workspace", ctypes.c_size_t), ("host_workspace", ctypes.c_size_t)]
 
 
 _lib = None
@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "moe_forward": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
             "moe_forward_timed": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                   ctypes.POINTER(ctypes.c_void_p), vp],
+            "moe_forward_host": [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp],
             "moe_check_device_errors": [vp, sz, vp, ctypes.POINTER(ctypes.c_uint32)],
             "moe_workspace_init": [vp, sz, vp],
             "moe_workspace_set_wait_limit": [vp, sz, ctypes.c_uint64, vp],
@@ -179,19 +180,22 @@ class Sizes:
     workspace: int
     capacity: int
     permute_workspace: int
+    host_workspace: int
 
 
 def query_sizes(cfg: MoeConfig) -> Sizes:
     out = MoeSizes()
     _check("moe_query_sizes", lib().moe_query_sizes(ctypes.byref(cfg), ctypes.byref(out)))
     return Sizes(out.rows_cap, out.rows_total, out.tok_rows_len, out.step_workspace, out.workspace,
-                 out.capacity, out.permute_workspace)
+                 out.capacity, out.permute_workspace, out.host_workspace)
 
 
-def new_workspace(cfg: MoeConfig, device="cuda", step_only: bool = False) -> torch.Tensor:
-    """A zeroed workspace tensor (uint8) of the size the configuration needs."""
+def new_workspace(cfg: MoeConfig, device="cuda", step_only: bool = False,
+                  host: bool = False) -> torch.Tensor:
+    """A zeroed workspace tensor (uint8) of the size the configuration needs
+    (step entry points, moe_forward, or moe_forward_host)."""
     s = query_sizes(cfg)
-    n = s.step_workspace if step_only else s.workspace
+    n = s.step_workspace if step_only else (s.host_workspace if host else s.workspace)
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
 
@@ -247,6 +251,32 @@ def moe_forward(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, stream=No
     _check("moe_forward", lib().moe_forward(
         ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(route_state), _ptr(w1), _ptr(w3),
         _ptr(w2), _ptr(y), _ptr(counts_out), wp, wn, _stream(stream)))
+
+
+def _host_ptr(t: torch.Tensor, numel: int, dtype: torch.dtype):
+    """Address of a contiguous host (CPU) tensor of at least numel elements."""
+    if t.is_cuda:
+        raise ValueError("moe_forward_host takes host (CPU) tensors for x and y")
+    if not t.is_contiguous() or t.dtype != dtype or t.numel() < numel:
+        raise ValueError(f"expected a contiguous {dtype} host tensor of {numel} elements")
+    return t.data_ptr()
+
+
+def moe_forward_host(cfg, x_host, w_router, bias, w1, w3, w2, y_host, counts_out, ws, stream=None,
+                     copy_in=None, copy_out=None, *, route_state=None):
+    """moe_forward on host buffers: x_host is copied in, y comes back to
+    y_host, queued on the streams without a host sync (page-locked tensors
+    make the copies asynchronous).  copy_in / copy_out: streams for the two
+    copies (None: `stream`)."""
+    wp, wn = _ws(ws)
+    dt = torch.float32 if cfg.dtype == MOE_F32 else torch.bfloat16
+    n = cfg.T * cfg.d_model
+    cin = None if copy_in is None else copy_in.cuda_stream
+    cout = None if copy_out is None else copy_out.cuda_stream
+    _check("moe_forward_host", lib().moe_forward_host(
+        ctypes.byref(cfg), _host_ptr(x_host, n, dt), _ptr(w_router), _ptr(bias), _ptr(route_state),
+        _ptr(w1), _ptr(w3), _ptr(w2), _host_ptr(y_host, n, dt), _ptr(counts_out), wp, wn,
+        _stream(stream), cin, cout))
 
 
 def moe_forward_timed(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, events, stream=None, *,
@@ -390,12 +420,13 @@ class MoELayer:
 
 
 class HostPipeline:
-    """Serving from host memory: batches of T tokens in pinned host buffers go
-    through ``layer`` and their outputs come back to pinned host buffers.  The
-    host-to-device copy of a batch and the device-to-host copy of the one
-    before it overlap the forward of the batch in between (three streams, two
-    device staging slots, events between them); every batch's copies and
-    forward still happen, in order.
+    """Serving from host memory through moe_forward_host: batches of T tokens
+    in page-locked host buffers go through ``layer`` and their outputs come
+    back to page-locked host buffers.  Two workspaces are used in turn and
+    the copies run on their own streams, so the host-to-device copy of a
+    batch and the device-to-host copy of the one before it overlap the
+    forward in between; the forwards stay in order on one stream (the library
+    orders the calls that share a workspace).
 
         pipe = HostPipeline(layer)
         for x_h, y_h in batches:          # pinned [T, d] tensors
@@ -406,40 +437,23 @@ class HostPipeline:
     def __init__(self, layer: MoELayer, before_forward=None):
         self.layer = layer
         dev = layer.w1.device
-        cfg = layer.cfg
-        dt = torch.float32 if cfg.dtype == MOE_F32 else torch.bfloat16
-        self.x_dev = [torch.empty(cfg.T, cfg.d_model, dtype=dt, device=dev) for _ in range(2)]
-        self.y_dev = [torch.empty(cfg.T, cfg.d_model, dtype=dt, device=dev) for _ in range(2)]
+        self.ws = [new_workspace(layer.cfg, dev, host=True) for _ in range(2)]
         self.s_in = torch.cuda.Stream(device=dev)
         self.s_comp = torch.cuda.Stream(device=dev)
         self.s_out = torch.cuda.Stream(device=dev)
-        mk = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
-        self.in_done, self.comp_done, self.out_done = mk(), mk(), mk()
         self.before_forward = before_forward     # optional callable, run on the compute stream
         self.i = 0
 
-    def submit(self, x_host: torch.Tensor, y_host: torch.Tensor) -> torch.cuda.Event:
-        """Queue one batch; returns the event recorded once y_host is filled."""
-        k = self.i & 1
-        if self.i >= 2:                      # slot k last used two batches ago
-            self.s_in.wait_event(self.comp_done[k])
-        with torch.cuda.stream(self.s_in):
-            self.x_dev[k].copy_(x_host, non_blocking=True)
-            self.in_done[k].record(self.s_in)
-        self.s_comp.wait_event(self.in_done[k])
-        if self.i >= 2:
-            self.s_comp.wait_event(self.out_done[k])
-        with torch.cuda.stream(self.s_comp):
-            if self.before_forward is not None:
+    def submit(self, x_host: torch.Tensor, y_host: torch.Tensor) -> None:
+        """Queue one batch (the host tensors must stay untouched until synchronize)."""
+        L = self.layer
+        if self.before_forward is not None:
+            with torch.cuda.stream(self.s_comp):
                 self.before_forward()
-            self.layer(self.x_dev[k], out=self.y_dev[k], stream=self.s_comp)
-            self.comp_done[k].record(self.s_comp)
-        self.s_out.wait_event(self.comp_done[k])
-        with torch.cuda.stream(self.s_out):
-            y_host.copy_(self.y_dev[k], non_blocking=True)
-            self.out_done[k].record(self.s_out)
+        moe_forward_host(L.cfg, x_host, L.w_router, L.bias, L.w1, L.w3, L.w2, y_host, L.counts,
+                         self.ws[self.i & 1], self.s_comp, self.s_in, self.s_out,
+                         route_state=L.route_state)
         self.i += 1
-        return self.out_done[k]
 
     def synchronize(self):
         for st in (self.s_in, self.s_comp, self.s_out):

@@ -4,11 +4,24 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <mutex>
+#include <unordered_map>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "device_common.cuh"
 #include "moe_internal.h"
 
 namespace moe {
+
+// NVTX range around an entry point or a phase of moe_forward (host-side
+// markers for profilers; header-only, inert when no tool is attached).
+struct Range {
+  explicit Range(const char *name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range &) = delete;
+  Range &operator=(const Range &) = delete;
+};
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -157,6 +170,9 @@ WsLayout make_layout(const moe_config *c) {
   L.h = take((size_t)L.rows_total * c->d_ff * es);
   L.y_rows = take((size_t)L.rows_total * c->d_model * es);     // rows in the layer dtype
   L.total = o;
+  L.x_stage = take((size_t)T * c->d_model * es);
+  L.y_stage = take((size_t)T * c->d_model * es);
+  L.host_total = o;
   return L;
 }
 
@@ -597,6 +613,33 @@ static cudaError_t run_backward(const moe_config *c, const WsLayout &L, const Bw
 
 using namespace moe;
 
+// Per-workspace ordering of moe_forward_host calls: the input copy of a call
+// waits for the previous forward on the workspace (which read the staged x),
+// the forward for the previous output copy (which read the staged y).
+namespace {
+struct HostEvents {
+  cudaEvent_t in_done = nullptr, fwd_done = nullptr, out_done = nullptr;
+};
+std::mutex g_host_mutex;
+std::unordered_map<const void *, HostEvents> g_host_events;
+
+cudaError_t host_events(const void *ws, HostEvents *out) {
+  std::lock_guard<std::mutex> lock(g_host_mutex);
+  HostEvents &h = g_host_events[ws];
+  for (cudaEvent_t *e : {&h.in_done, &h.fwd_done, &h.out_done}) {
+    if (*e == nullptr) {
+      const cudaError_t r = cudaEventCreateWithFlags(e, cudaEventDisableTiming);
+      if (r != cudaSuccess) {
+        *e = nullptr;
+        return r;
+      }
+    }
+  }
+  *out = h;
+  return cudaSuccess;
+}
+}  // namespace
+
 extern "C" {
 
 moe_status moe_query_sizes(const moe_config *cfg, moe_sizes *out) {
@@ -611,6 +654,7 @@ moe_status moe_query_sizes(const moe_config *cfg, moe_sizes *out) {
   out->workspace = L.total;
   out->capacity = capacity_rows(cfg);
   out->permute_workspace = L.permute_end;
+  out->host_workspace = L.host_total;
   return MOE_OK;
 }
 
@@ -622,6 +666,7 @@ static bool state_ok(const moe_config *c, const float *state) {
 moe_status moe_route(const moe_config *cfg, const void *x, const void *w_router, const float *bias,
                      const float *route_state, float *logits, float *probs, int32_t *topk_idx,
                      float *topk_gate, void *ws, size_t ws_bytes, moe_stream_t stream) {
+  Range range("moe_route");
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const WsLayout L = make_layout(cfg);
@@ -640,6 +685,7 @@ moe_status moe_route(const moe_config *cfg, const void *x, const void *w_router,
 moe_status moe_gate(const moe_config *cfg, const float *logits, const float *route_state,
                     float *probs, int32_t *topk_idx, float *topk_gate, void *ws, size_t ws_bytes,
                     moe_stream_t stream) {
+  Range range("moe_gate");
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const WsLayout L = make_layout(cfg);
@@ -666,6 +712,7 @@ moe_status moe_permute(const moe_config *cfg, const void *x, const int32_t *topk
                        const float *topk_gate, const float *probs, int32_t *counts, int32_t *offsets,
                        int32_t *tok_rows, int32_t *row_token, float *row_gate, void *x_perm,
                        int32_t *n_dropped, void *ws, size_t ws_bytes, moe_stream_t stream) {
+  Range range("moe_permute");
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const WsLayout L = make_layout(cfg);
@@ -686,6 +733,7 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x, const void *x_pe
                           const int32_t *offsets, const float *row_gate, const void *w1,
                           const void *w3, const void *w2, void *h, void *y_rows, void *ws,
                           size_t ws_bytes, moe_stream_t stream) {
+  Range range("moe_expert_ffn");
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const WsLayout L = make_layout(cfg);
@@ -702,6 +750,7 @@ moe_status moe_expert_ffn(const moe_config *cfg, const void *x, const void *x_pe
 
 moe_status moe_combine(const moe_config *cfg, const void *y_rows, const int32_t *tok_rows, void *y,
                        moe_stream_t stream) {
+  Range range("moe_combine");
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   if (!y_rows || !tok_rows || !y) return MOE_ERR_INVALID_ARG;
@@ -716,6 +765,7 @@ static moe_status forward_impl(const moe_config *cfg, const void *x, const void 
                                const void *w3, const void *w2, void *y, int32_t *counts_out,
                                void *ws, size_t ws_bytes, void *const *events,
                                moe_stream_t stream) {
+  Range range("moe_forward");
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   const WsLayout L = make_layout(cfg);
@@ -753,23 +803,32 @@ static moe_status forward_impl(const moe_config *cfg, const void *x, const void 
     return cudaSuccess;
   };
   cudaError_t e = mark(0);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess) {
+    Range r("route");
     e = run_route(cfg, L, w, x, w_router, bias, state, logits, probs, topk_idx, topk_gate, s,
                   fold ? y : nullptr);
+  }
   if (e == cudaSuccess) e = mark(1);
   // token choice: the gate wrote the unit histogram into the workspace.
   // bf16: the up-projection gathers the rows of x itself (no x_perm)
   const bool fused_gather = forward_gathers(cfg, L.rows_cap);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess) {
+    Range r("permute");
     e = launch_permute(cfg, L, w, cfg->mode == MOE_TOKEN_CHOICE, x, topk_idx, topk_gate, probs,
                        counts, offsets, tok_rows, row_token, row_gate, x_perm, n_dropped, s,
                        !fused_gather);
+  }
   if (e == cudaSuccess) e = mark(2);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess) {
+    Range r("expert_ffn");
     e = run_ffn(cfg, L, w, x, x_perm, offsets, row_gate, w1, w3, w2, h, y_rows, s,
                 fused_gather ? row_token : nullptr, fold ? y : nullptr, row_token);
+  }
   if (e == cudaSuccess) e = mark(3);
-  if (e == cudaSuccess && !fold) e = launch_combine(cfg, L.rows_cap, y_rows, tok_rows, y, s);
+  if (e == cudaSuccess && !fold) {
+    Range r("combine");
+    e = launch_combine(cfg, L.rows_cap, y_rows, tok_rows, y, s);
+  }
   if (e == cudaSuccess) e = mark(4);
   if (e == cudaSuccess && counts_out)
     e = cudaMemcpyAsync(counts_out, counts, (size_t)cfg->E * 4, cudaMemcpyDeviceToDevice, s);
@@ -782,6 +841,41 @@ moe_status moe_forward(const moe_config *cfg, const void *x, const void *w_route
                        moe_stream_t stream) {
   return forward_impl(cfg, x, w_router, bias, route_state, w1, w3, w2, y, counts_out, ws, ws_bytes,
                       nullptr, stream);
+}
+
+
+moe_status moe_forward_host(const moe_config *cfg, const void *x_host, const void *w_router,
+                            const float *bias, const float *route_state, const void *w1,
+                            const void *w3, const void *w2, void *y_host, int32_t *counts_out,
+                            void *ws, size_t ws_bytes, moe_stream_t stream, moe_stream_t copy_in,
+                            moe_stream_t copy_out) {
+  Range range("moe_forward_host");
+  moe_status st = validate(cfg);
+  if (st != MOE_OK) return st;
+  const WsLayout L = make_layout(cfg);
+  if ((st = check_ws(L, ws, ws_bytes, L.host_total)) != MOE_OK) return st;
+  if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t cin = copy_in ? reinterpret_cast<cudaStream_t>(copy_in) : s;
+  cudaStream_t cout = copy_out ? reinterpret_cast<cudaStream_t>(copy_out) : s;
+  HostEvents ev;
+  if (host_events(ws, &ev) != cudaSuccess) return MOE_ERR_CUDA;
+  char *w = static_cast<char *>(ws);
+  const size_t bytes = (size_t)cfg->T * cfg->d_model * elem_size(cfg);
+  cudaError_t e = cudaStreamWaitEvent(cin, ev.fwd_done, 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(w + L.x_stage, x_host, bytes, cudaMemcpyHostToDevice, cin);
+  if (e == cudaSuccess) e = cudaEventRecord(ev.in_done, cin);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev.in_done, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev.out_done, 0);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  st = forward_impl(cfg, w + L.x_stage, w_router, bias, route_state, w1, w3, w2, w + L.y_stage,
+                    counts_out, ws, ws_bytes, nullptr, stream);
+  if (st != MOE_OK) return st;
+  e = cudaEventRecord(ev.fwd_done, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(cout, ev.fwd_done, 0);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(y_host, w + L.y_stage, bytes, cudaMemcpyDeviceToHost, cout);
+  if (e == cudaSuccess) e = cudaEventRecord(ev.out_done, cout);
+  return cuda_status(e);
 }
 
 moe_status moe_forward_timed(const moe_config *cfg, const void *x, const void *w_router,
@@ -807,6 +901,7 @@ moe_status moe_backward(const moe_config *cfg, const void *x, const void *w_rout
                         const void *w3, const void *w2, const void *dy, float *dx, float *dw_router,
                         float *dbias, float *dw1, float *dw3, float *dw2, const void *ws,
                         size_t ws_bytes, void *bws, size_t bws_bytes, moe_stream_t stream) {
+  Range range("moe_backward");
   moe_status st = validate(cfg);
   if (st != MOE_OK) return st;
   if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;

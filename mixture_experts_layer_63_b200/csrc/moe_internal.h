@@ -96,6 +96,8 @@ struct WsLayout {
   size_t logits, probs, topk_idx, topk_gate, counts, offsets, n_dropped;
   size_t tok_rows, row_token, row_gate, x_perm, h, y_rows;
   size_t total;
+  // moe_forward_host staging rows of x and y (after everything moe_forward uses)
+  size_t x_stage, y_stage, host_total;
   int nunit;         // 32-token units: ceil(T / 32)
   int64_t rows_cap, rows_total, tok_rows_len;
 };

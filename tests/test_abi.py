@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(L):
 
 def test_struct_sizes(L):
     assert ctypes.sizeof(api.MoeConfig) == 88
-    assert ctypes.sizeof(api.MoeSizes) == 56
+    assert ctypes.sizeof(api.MoeSizes) == 64
 
 
 def test_struct_layout_matches_the_header(tmp_path):
@@ -88,6 +88,8 @@ def test_sizes_of_the_workloads(L):
             assert s.rows_cap == w.T * w.k and s.tok_rows_len == w.T * w.k
         assert s.rows_total == s.rows_cap + w.S * w.T
         assert s.workspace >= s.step_workspace >= 256
+        es = 4 if w.dtype == "f32" else 2
+        assert s.host_workspace >= s.workspace + 2 * w.T * w.d_model * es
 
 
 def _cfg(**kw):

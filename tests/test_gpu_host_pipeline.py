@@ -1,6 +1,8 @@
-"""api.HostPipeline: batches from pinned host memory through the layer with
-overlapped copies give the same outputs, bit for bit, as one forward per
-batch on resident tensors."""
+"""moe_forward_host (the C-ABI call on host buffers) and api.HostPipeline
+built on it: batches from pinned host memory through the layer, with copies
+on their own streams overlapping the forwards and two workspaces in turn,
+give the same outputs, bit for bit, as one forward per batch on resident
+tensors; so does the plain call on one stream, pinned or pageable."""
 import pytest
 import torch
 
@@ -30,4 +32,39 @@ def test_pipeline_matches_direct_forwards(name):
     pipe.synchronize()
     for i, (yh, yw) in enumerate(zip(y_host, want)):
         assert torch.equal(yh, yw.cpu()), i
-    api.moe_check_device_errors(layer.ws)
+    for ws in pipe.ws:
+        api.moe_check_device_errors(ws)
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+def test_forward_host_on_one_stream(pinned):
+    w = SMALL["dsv2_s"]
+    inp = gpu_inputs(w, seed=32, grid=False)
+    cfg = api.config_from_workload(w)
+    layer = api.MoELayer(cfg, inp.w_router, inp.w1, inp.w2, inp.w3, inp.bias)
+    want = layer(inp.x).cpu()
+    ws = api.new_workspace(cfg, host=True)
+    xh = inp.x.cpu()
+    yh = torch.full_like(xh, float("nan"))
+    if pinned:
+        xh, yh = xh.pin_memory(), yh.pin_memory()
+    counts = torch.empty(w.E, dtype=torch.int32, device="cuda")
+    for _ in range(2):                       # the second call reuses the workspace's events
+        api.moe_forward_host(cfg, xh, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2, yh, counts, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(yh, want)
+    assert torch.equal(counts, layer.counts)
+    api.moe_check_device_errors(ws)
+
+
+def test_forward_host_refuses_device_buffers_and_a_short_workspace():
+    w = SMALL["gshard_s"]
+    inp = gpu_inputs(w, seed=33, grid=False)
+    cfg = api.config_from_workload(w)
+    with pytest.raises(ValueError):
+        api.moe_forward_host(cfg, inp.x, inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2,
+                             inp.x.cpu(), None, api.new_workspace(cfg, host=True))
+    with pytest.raises(api.MoeError) as ei:
+        api.moe_forward_host(cfg, inp.x.cpu(), inp.w_router, inp.bias, inp.w1, inp.w3, inp.w2,
+                             inp.x.cpu(), None, api.new_workspace(cfg))
+    assert ei.value.status == api.MOE_ERR_WORKSPACE
