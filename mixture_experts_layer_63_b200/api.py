@@ -183,11 +183,37 @@ class Sizes:
     host_workspace: int
 
 
+_sizes_cache: dict[bytes, Sizes] = {}
+
+
 def query_sizes(cfg: MoeConfig) -> Sizes:
+    key = bytes(cfg)
+    hit = _sizes_cache.get(key)
+    if hit is not None:
+        return hit
     out = MoeSizes()
     _check("moe_query_sizes", lib().moe_query_sizes(ctypes.byref(cfg), ctypes.byref(out)))
-    return Sizes(out.rows_cap, out.rows_total, out.tok_rows_len, out.step_workspace, out.workspace,
-                 out.capacity, out.permute_workspace, out.host_workspace)
+    s = Sizes(out.rows_cap, out.rows_total, out.tok_rows_len, out.step_workspace, out.workspace,
+              out.capacity, out.permute_workspace, out.host_workspace)
+    if len(_sizes_cache) < 256:
+        _sizes_cache[key] = s
+    return s
+
+
+class _Need:
+    """Element counts and dtypes of a configuration's buffers, for the size
+    checks of the bindings (a short output buffer would be written past its
+    end by the kernels)."""
+
+    def __init__(self, cfg: MoeConfig):
+        s = query_sizes(cfg)
+        self.dt = torch.float32 if cfg.dtype == MOE_F32 else torch.bfloat16
+        T, E, d, f = cfg.T, cfg.E, cfg.d_model, cfg.d_ff
+        k = cfg.k if cfg.mode == MOE_TOKEN_CHOICE else 0
+        self.td, self.te, self.tk, self.e = T * d, T * E, T * k, E
+        self.rows_cap, self.tok_rows = max(s.rows_cap, 1), s.tok_rows_len
+        self.x_perm = max(s.rows_cap, 1) * d
+        self.h, self.y_rows = s.rows_total * f, s.rows_total * d
 
 
 def new_workspace(cfg: MoeConfig, device="cuda", step_only: bool = False,
@@ -206,15 +232,21 @@ def new_workspace(cfg: MoeConfig, device="cuda", step_only: bool = False,
 def moe_route(cfg, x, w_router, bias, logits, probs, topk_idx, topk_gate, ws, stream=None, *,
               route_state=None):
     wp, wn = _ws(ws)
-    _check("moe_route", lib().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias),
-                                        _ptr(route_state), _ptr(logits), _ptr(probs), _ptr(topk_idx),
-                                        _ptr(topk_gate), wp, wn, _stream(stream)))
+    n = _Need(cfg)
+    _check("moe_route", lib().moe_route(ctypes.byref(cfg), _ptr(x, n.td, n.dt), _ptr(w_router),
+                                        _ptr(bias), _ptr(route_state), _ptr(logits, n.te, torch.float32),
+                                        _ptr(probs, n.te, torch.float32),
+                                        _ptr(topk_idx, n.tk, torch.int32),
+                                        _ptr(topk_gate, n.tk, torch.float32), wp, wn, _stream(stream)))
 
 
 def moe_gate(cfg, logits, probs, topk_idx, topk_gate, ws, stream=None, *, route_state=None):
     wp, wn = _ws(ws)
-    _check("moe_gate", lib().moe_gate(ctypes.byref(cfg), _ptr(logits), _ptr(route_state), _ptr(probs),
-                                      _ptr(topk_idx), _ptr(topk_gate), wp, wn, _stream(stream)))
+    n = _Need(cfg)
+    _check("moe_gate", lib().moe_gate(ctypes.byref(cfg), _ptr(logits, n.te, torch.float32),
+                                      _ptr(route_state), _ptr(probs, n.te, torch.float32),
+                                      _ptr(topk_idx, n.tk, torch.int32),
+                                      _ptr(topk_gate, n.tk, torch.float32), wp, wn, _stream(stream)))
 
 
 def moe_route_bias_update(cfg, counts, route_bias, gamma: float, stream=None):
@@ -227,30 +259,44 @@ def moe_route_bias_update(cfg, counts, route_bias, gamma: float, stream=None):
 def moe_permute(cfg, x, topk_idx, topk_gate, probs, counts, offsets, tok_rows, row_token, row_gate,
                 x_perm, n_dropped, ws, stream=None):
     wp, wn = _ws(ws)
+    n = _Need(cfg)
     _check("moe_permute", lib().moe_permute(
-        ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(topk_gate), _ptr(probs), _ptr(counts),
-        _ptr(offsets), _ptr(tok_rows), _ptr(row_token), _ptr(row_gate), _ptr(x_perm),
-        _ptr(n_dropped), wp, wn, _stream(stream)))
+        ctypes.byref(cfg), _ptr(x, n.td, n.dt), _ptr(topk_idx), _ptr(topk_gate), _ptr(probs),
+        *_permute_outputs(n, counts, offsets, tok_rows, row_token, row_gate, x_perm, n_dropped),
+        wp, wn, _stream(stream)))
+
+
+def _permute_outputs(n: _Need, counts, offsets, tok_rows, row_token, row_gate, x_perm, n_dropped):
+    i32 = torch.int32
+    return (_ptr(counts, n.e, i32), _ptr(offsets, n.e + 1, i32), _ptr(tok_rows, n.tok_rows, i32),
+            _ptr(row_token, n.rows_cap, i32), _ptr(row_gate, n.rows_cap, torch.float32),
+            _ptr(x_perm, n.x_perm, n.dt), _ptr(n_dropped, 1, i32))
 
 
 def moe_expert_ffn(cfg, x, x_perm, offsets, row_gate, w1, w3, w2, h, y_rows, ws, stream=None):
     wp, wn = _ws(ws)
+    n = _Need(cfg)
     _check("moe_expert_ffn", lib().moe_expert_ffn(
-        ctypes.byref(cfg), _ptr(x), _ptr(x_perm), _ptr(offsets), _ptr(row_gate), _ptr(w1), _ptr(w3),
-        _ptr(w2), _ptr(h), _ptr(y_rows), wp, wn, _stream(stream)))
+        ctypes.byref(cfg), _ptr(x, n.td, n.dt), _ptr(x_perm, None, n.dt), _ptr(offsets), _ptr(row_gate),
+        _ptr(w1, None, n.dt), _ptr(w3, None, n.dt), _ptr(w2, None, n.dt), _ptr(h, n.h, n.dt),
+        _ptr(y_rows, n.y_rows, n.dt), wp, wn, _stream(stream)))
 
 
 def moe_combine(cfg, y_rows, tok_rows, y, stream=None):
-    _check("moe_combine", lib().moe_combine(ctypes.byref(cfg), _ptr(y_rows), _ptr(tok_rows), _ptr(y),
-                                            _stream(stream)))
+    n = _Need(cfg)
+    _check("moe_combine", lib().moe_combine(ctypes.byref(cfg), _ptr(y_rows, n.y_rows, n.dt),
+                                            _ptr(tok_rows, n.tok_rows, torch.int32),
+                                            _ptr(y, n.td, n.dt), _stream(stream)))
 
 
 def moe_forward(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, stream=None, *,
                 route_state=None):
     wp, wn = _ws(ws)
+    n = _Need(cfg)
     _check("moe_forward", lib().moe_forward(
-        ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(route_state), _ptr(w1), _ptr(w3),
-        _ptr(w2), _ptr(y), _ptr(counts_out), wp, wn, _stream(stream)))
+        ctypes.byref(cfg), _ptr(x, n.td, n.dt), _ptr(w_router), _ptr(bias), _ptr(route_state),
+        _ptr(w1, None, n.dt), _ptr(w3, None, n.dt), _ptr(w2, None, n.dt), _ptr(y, n.td, n.dt),
+        _ptr(counts_out, n.e, torch.int32), wp, wn, _stream(stream)))
 
 
 def _host_ptr(t: torch.Tensor, numel: int, dtype: torch.dtype):
@@ -287,9 +333,11 @@ def moe_forward_timed(cfg, x, w_router, bias, w1, w3, w2, y, counts_out, ws, eve
     that its CUDA handle exists."""
     wp, wn = _ws(ws)
     handles = (ctypes.c_void_p * 5)(*[ev.cuda_event if ev is not None else None for ev in events])
+    n = _Need(cfg)
     _check("moe_forward_timed", lib().moe_forward_timed(
-        ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(route_state), _ptr(w1), _ptr(w3),
-        _ptr(w2), _ptr(y), _ptr(counts_out), wp, wn, handles, _stream(stream)))
+        ctypes.byref(cfg), _ptr(x, n.td, n.dt), _ptr(w_router), _ptr(bias), _ptr(route_state),
+        _ptr(w1, None, n.dt), _ptr(w3, None, n.dt), _ptr(w2, None, n.dt), _ptr(y, n.td, n.dt),
+        _ptr(counts_out, n.e, torch.int32), wp, wn, handles, _stream(stream)))
 
 
 def query_backward_size(cfg: MoeConfig) -> int:
@@ -488,7 +536,8 @@ def moe_permute_noalloc(cfg, x, topk_idx, topk_gate, probs, counts, offsets, tok
     The first call on a device looks up the array's address: make it before
     any stream capture.  Calls that overlap on the GPU race on the array.
     """
+    n = _Need(cfg)
     _check("moe_permute_noalloc", _noalloc()(
-        ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(topk_gate), _ptr(probs), _ptr(counts),
-        _ptr(offsets), _ptr(tok_rows), _ptr(row_token), _ptr(row_gate), _ptr(x_perm),
-        _ptr(n_dropped), _stream(stream)))
+        ctypes.byref(cfg), _ptr(x, n.td, n.dt), _ptr(topk_idx), _ptr(topk_gate), _ptr(probs),
+        *_permute_outputs(n, counts, offsets, tok_rows, row_token, row_gate, x_perm, n_dropped),
+        _stream(stream)))

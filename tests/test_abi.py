@@ -248,3 +248,34 @@ def test_permute_workspace_is_the_permutation_share(L):
     # as well, which the permutation does not use
     s = api.query_sizes(api.config_from_workload(WORKLOADS["gshard"]))
     assert s.step_workspace - s.permute_workspace >= 24 << 20
+
+
+def test_new_entry_points_validate_on_the_host(L):
+    """moe_forward_host refuses NULL host buffers and a workspace below
+    host_workspace, moe_workspace_set_wait_limit a workspace below its 4 KiB
+    control block: both before any CUDA call."""
+    c = _cfg(T=64, d_model=64, d_ff=64)
+    s = api.query_sizes(c)
+    assert s.host_workspace > s.workspace
+    buf = ctypes.create_string_buffer(s.host_workspace + 256)
+    addr = (ctypes.addressof(buf) + 255) & ~255
+    st = L.moe_forward_host(ctypes.byref(c), None, 16, None, None, 16, None, 16, None, None, addr,
+                            s.host_workspace, None, None, None)
+    assert st == api.MOE_ERR_INVALID_ARG
+    st = L.moe_forward_host(ctypes.byref(c), 16, 16, None, None, 16, None, 16, 16, None, addr,
+                            s.workspace, None, None, None)
+    assert st == api.MOE_ERR_WORKSPACE
+    assert L.moe_workspace_set_wait_limit(addr, 1024, 1000, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_workspace_set_wait_limit(None, 1 << 20, 1000, None) == api.MOE_ERR_INVALID_ARG
+
+
+def test_binding_checks_buffer_sizes():
+    """A short output buffer is a Python error, not a write past its end
+    (checked before the pointer is handed to the library)."""
+    import torch
+    c = _cfg(T=64, d_model=64, d_ff=64)
+    n = api._Need(c)
+    assert n.td == 64 * 64 and n.tok_rows == 64 * 2
+    t = torch.empty(8)
+    with pytest.raises(ValueError):
+        api._ptr(t)                      # not a CUDA tensor
