@@ -389,20 +389,15 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
       : "memory");
 }
 
-// Four rows r0..r3 of a 2-D tensor (each a box of 64 columns from column c0;
-// the tensor map's box is one row high) into four consecutive 128-byte rows
-// of this CTA's shared memory at `dst`, with the map's 128-byte swizzle
-// (which follows the shared-memory address, so rows placed at a 512-byte
-// offset of a 1024-byte-aligned tile land as rows 4..7 of an 8-row tile
-// load would), completing on the mbarrier at `bar_cluster` (the even CTA's
-// barrier of the pair).
-__device__ __forceinline__ void tma_gather4_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster,
-                                                 int c0, int4 rows) {
+// The same from a 3-D tensor map {64 columns, rows, k-blocks} (a 2-D bf16
+// matrix viewed as its 64-column k-blocks): one copy brings several
+// consecutive k-blocks of the same rows, landing one tile after another.
+__device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster,
+                                                 int c0, int c1, int c2) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(rows.x), "r"(rows.y),
-      "r"(rows.z), "r"(rows.w)
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
 
@@ -1610,16 +1605,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 //   A (weights): ReLU and the down-projection take 128 consecutive rows of W
 //     per CTA; SwiGLU takes 64 rows of W1 (gate) and the same 64 rows of W3
 //     (up), so a CTA's accumulator holds both halves of its 64 outputs.
-//   B (tokens): the tile's N rows, N / 2 per CTA, in TMA boxes of 16 rows;
-//     or, with gather_rows (the up-projection of moe_forward), the routed
-//     rows straight from x: row r of a group is x[gather_rows[off + r]],
-//     four rows per TMA tile::gather4 load, so no permuted copy of x is
-//     written or read.  Warp 3 stages each tile's row indices in shared
-//     memory (two slots, mbarrier handshakes) ahead of the producer.
+//   B (tokens): the tile's N rows, N / 2 per CTA, in one TMA load: a tensor
+//     map per box height (16, 32, ..., 128 rows), so a k-block costs one
+//     copy of the weights (two for SwiGLU) and one of the tokens.  (Each TMA
+//     instruction has a fixed cost: with 16-row boxes the tensor pipe sat
+//     idle 64% of the time on the DeepSeek-V2 shape, with one box 42%.)
 // Tiles run group by group, weight tile outer and token tile inner, so the
 // pairs working at once share a weight tile in L2; they are dealt
 // round-robin (no stream-K tail).
-constexpr int kTnTokBox = 16;            // token rows per TMA box
+constexpr int kTnTokBox = 16;            // token box heights are multiples of this
+constexpr int kTnBoxes = 8;              // one tensor map per height 16, 32, ..., 128
 constexpr int kTnMaxN = 256;             // token rows per tile (the MMA's N)
 constexpr int kTnGran = 32;              // tile widths are multiples of this
 constexpr int kTnStgBytes = 2304;        // per epilogue warp: 33 rows of 64 bytes (+ pad)
@@ -1627,6 +1622,17 @@ constexpr int kTnXchBytes = 16384;       // SwiGLU: 2 warp pairs x 2 buffers x 4
 
 struct TnTile {
   int g, wt, n0, n, valid;               // group, weight tile, first token, MMA N, rows stored
+};
+
+// The token-N kernel's tensor maps: token rows of the routed segments (x_perm
+// or h) and of the static groups (x or h), one map per box height
+// 16 (i + 1) rows, 3-D (one copy brings the stage's BKS k-blocks); the
+// weights: 3-D boxes of 128 rows, or (SwiGLU) 2-D boxes of 64 rows of W1 and
+// of W3, which must interleave k-block by k-block.
+struct TnMaps {
+  CUtensorMap tok[kTnBoxes];
+  CUtensorMap tok_static[kTnBoxes];
+  CUtensorMap w, w3;
 };
 
 // tiles per group: weight tiles x token tiles
@@ -1763,10 +1769,7 @@ __device__ __forceinline__ void epilogue_tn(const Params &P, uint32_t taddr, con
 
 template <int EPI, int BKS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    grouped_gemm_tn_kernel(const __grid_constant__ CUtensorMap map_tok,
-                           const __grid_constant__ CUtensorMap map_tok_static,
-                           const __grid_constant__ CUtensorMap map_w,
-                           const __grid_constant__ CUtensorMap map_w3, const Params P) {
+    grouped_gemm_tn_kernel(const __grid_constant__ TnMaps M, const Params P) {
   constexpr bool kSwiglu = EPI == kEpiSwiglu;
   constexpr int STAGES = BKS == 2 ? kPairStages2 : kPairStages;
   constexpr uint32_t kWBytes = BM * BK * 2;                     // weights: 16 KB a k-block and CTA
@@ -1784,25 +1787,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   __shared__ uint32_t s_tmem_base;
   __shared__ volatile int s_abort;
   __shared__ uint64_t s_limit_sh;
-  __shared__ __align__(16) int s_idx[2][kTnMaxN / 2];  // gathered rows of a tile (two slots)
-  __shared__ __align__(8) uint64_t idx_full[2];
-  __shared__ __align__(8) uint64_t idx_empty[2];
 
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~(uintptr_t)1023);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const bool gather = P.gather_rows != nullptr;
 
   if (tid == 32) {
     for (int st = 0; st < STAGES; ++st) {
       mbar_init(&full_bar[st], 1);                     // the even CTA's expect_tx arrival
       mbar_init(&empty_bar[st], 1);
-    }
-    for (int sl = 0; sl < 2; ++sl) {
-      mbar_init(&idx_full[sl], 1);
-      mbar_init(&idx_empty[sl], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&accf_bar[a], 1);
@@ -1819,10 +1814,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
   }
   if (tid == 0) {
-    tma_prefetch_map(&map_tok);
-    tma_prefetch_map(&map_w);
-    if (P.n_static > 0) tma_prefetch_map(&map_tok_static);
-    if (kSwiglu) tma_prefetch_map(&map_w3);
+    tma_prefetch_map(&M.w);
+    if (kSwiglu) tma_prefetch_map(&M.w3);
   }
   pdl_wait();              // what earlier kernels wrote is visible from here on
   pdl_trigger();
@@ -1875,23 +1868,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     uint32_t armed = 0, armed_parity = 0;
-    int islot = 0;
-    uint32_t iphase = 0;
     bool ok = true;
     for (int tile = pair; ok && tile < total; tile += npairs) {
       const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G);
       const bool routed = tl.g < P.n_routed;
-      const bool gathered = gather && routed;
-      if (gathered && !mbar_wait(&idx_full[islot], iphase, &s_abort, P.err, s_limit)) { ok = false; break; }
-      const CUtensorMap *mt = routed ? &map_tok : &map_tok_static;
-      const int64_t tok_row =
-          (routed ? (int64_t)s_off[tl.g]
-                  : P.a_static_base + (int64_t)(tl.g - P.n_routed) * P.a_static_stride) +
-          tl.n0 + (int64_t)rank * (tl.n / 2);
+      const int half = tl.n / 2;                       // this CTA's token rows: one box
+      const CUtensorMap *mt = routed ? &M.tok[half / kTnTokBox - 1] : &M.tok_static[half / kTnTokBox - 1];
+      const int tok_row =
+          (int)((routed ? (int64_t)s_off[tl.g]
+                        : P.a_static_base + (int64_t)(tl.g - P.n_routed) * P.a_static_stride) +
+                tl.n0 + (int64_t)rank * half);
       const int w_row = kSwiglu ? tl.g * P.N + tl.wt * 128 + (int)rank * 64
                                 : tl.g * P.N + tl.wt * 256 + (int)rank * 128;
-      const int nbox = tl.n / 2 / kTnTokBox;
-      const uint32_t tx = 2u * BKS * (kWBytes + (uint32_t)(tl.n / 2) * BK * 2);
+      const uint32_t tx = 2u * BKS * (kWBytes + (uint32_t)half * BK * 2);
+      const int kz = 0;                                // 3-D maps: k-block coordinate below
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &s_abort, P.err, s_limit)) { ok = false; break; }
         uint8_t *sa = smem + (size_t)stage * stage_bytes;
@@ -1902,30 +1892,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           armed |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         }
+        (void)kz;
+        if (kSwiglu) {
 #pragma unroll
-        for (int q = 0; q < BKS; ++q) {
-          const int kx = (kb * BKS + q) * BK;
-          if (kSwiglu) {
-            tma_load_2d_pair(sa + q * kWBytes, &map_w, fb, kx, w_row);
-            tma_load_2d_pair(sa + q * kWBytes + kWBytes / 2, &map_w3, fb, kx, w_row);
-          } else {
-            tma_load_2d_pair(sa + q * kWBytes, &map_w, fb, kx, w_row);
+          for (int q = 0; q < BKS; ++q) {
+            const int kx = (kb * BKS + q) * BK;
+            tma_load_2d_pair(sa + q * kWBytes, &M.w, fb, kx, w_row);
+            tma_load_2d_pair(sa + q * kWBytes + kWBytes / 2, &M.w3, fb, kx, w_row);
           }
-          if (gathered) {
-            const int4 *ix = reinterpret_cast<const int4 *>(s_idx[islot]);
-            for (int j = 0; j < tl.n / 8; ++j)
-              tma_gather4_pair(sb + q * kTokBytes + j * 512, mt, fb, kx, ix[j]);
-          } else {
-            for (int j = 0; j < nbox; ++j)
-              tma_load_2d_pair(sb + q * kTokBytes + j * (kTnTokBox * 128), mt, fb, kx,
-                               (int)(tok_row + j * kTnTokBox));
-          }
+        } else {
+          tma_load_3d_pair(sa, &M.w, fb, 0, w_row, kb * BKS);            // BKS tiles of 16 KB
         }
+        tma_load_3d_pair(sb, mt, fb, 0, tok_row, kb * BKS);               // BKS tiles of half rows
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-      }
-      if (gathered && ok) {
-        mbar_arrive(&idx_empty[islot]);         // the coordinates were taken at issue
-        if (++islot == 2) { islot = 0; iphase ^= 1u; }
       }
     }
     if (!ok && rank == 0) {
@@ -1950,12 +1929,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t a_addr = smem_u32(smem + (size_t)stage * stage_bytes);
         const uint32_t b_addr = a_addr + BKS * kWBytes;
+        const uint32_t b_chunk = (uint32_t)(tl.n / 2) * BK * 2;   // token tiles lie back to back
 #pragma unroll
         for (int q = 0; q < BKS; ++q) {
 #pragma unroll
           for (int k = 0; k < BK / kUmmaK; ++k)
             umma_bf16_pair(d_tmem, sw128_desc(a_addr + q * kWBytes + k * kUmmaK * 2),
-                           sw128_desc(b_addr + q * kTokBytes + k * kUmmaK * 2), idesc,
+                           sw128_desc(b_addr + q * b_chunk + k * kUmmaK * 2), idesc,
                            (kb > 0 || q > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit_pair_both(&empty_bar[stage]);
@@ -1967,31 +1947,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     umma_commit_pair_local(&drain_bar);
     mbar_wait_drain(&drain_bar, 0);
-  } else if (gather && warp == 3) {
-    // ------------- row indices of the gathered tiles, one tile ahead -------------
-    int islot = 0;
-    uint32_t iphase = 0;
-    for (int tile = pair; tile < total; tile += npairs) {
-      const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G);
-      if (tl.g >= P.n_routed) continue;                 // static groups read x as stored
-      int okw = 1;
-      if (lane == 0) okw = mbar_wait(&idx_empty[islot], iphase ^ 1u, &s_abort, P.err, s_limit) ? 1 : 0;
-      if (!__shfl_sync(0xffffffffu, okw, 0)) break;
-      const int rows = s_rows[tl.g], off = s_off[tl.g];
-      const int half = tl.n / 2, r0 = tl.n0 + (int)rank * half;
-      for (int i = lane; i < half; i += 32) {
-        const int r = min(r0 + i, rows - 1);           // padding rows repeat the last row
-        int t = P.gather_rows[off + r];
-        if (t < 0 || t >= P.src_rows) {
-          raise_error(P.err, kErrBadIndex);
-          t = 0;
-        }
-        s_idx[islot][i] = t;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&idx_full[islot]);
-      if (++islot == 2) { islot = 0; iphase ^= 1u; }
-    }
   } else if (warp >= 4) {
     // -------------------------------- epilogue --------------------------------
     const int ew = warp - 4;                           // TMEM lanes 32 ew .. 32 ew + 31
@@ -2064,6 +2019,25 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D view {64 columns, rows, K / 64 k-blocks} of a bf16 matrix [rows][K]
+// (strides: K * 2 bytes between rows, 128 bytes between k-blocks), box
+// {64, box_rows, chunks}: one copy brings `chunks` consecutive k-blocks of
+// box_rows rows, landing as `chunks` [box_rows][64] tiles one after another,
+// each 128-byte swizzled like a 2-D box.
+bool make_map3(CUtensorMap *m, const void *base, uint64_t K, uint64_t rows, uint32_t box_rows,
+               uint32_t chunks) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  if (rows == 0) rows = 1;
+  cuuint64_t dims[3] = {(cuuint64_t)BK, rows, K / BK};
+  cuuint64_t strides[2] = {K * 2, (cuuint64_t)BK * 2};
+  cuuint32_t box[3] = {(cuuint32_t)BK, box_rows, chunks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int device_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -2115,8 +2089,7 @@ cudaError_t launch_pair(const Params &P, const CUtensorMap &ma, const CUtensorMa
 // Token-N launch: as many 2-CTA clusters as fit at once, fewer when there are
 // fewer tiles.
 template <int EPI, int BKS>
-cudaError_t launch_tn(const Params &P, const CUtensorMap &mt, const CUtensorMap &mts,
-                      const CUtensorMap &mw, const CUtensorMap &mw3, int64_t max_tiles, size_t smem,
+cudaError_t launch_tn(const Params &P, const TnMaps &maps, int64_t max_tiles, size_t smem,
                       cudaStream_t s) {
   auto kern = grouped_gemm_tn_kernel<EPI, BKS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -2139,7 +2112,7 @@ cudaError_t launch_tn(const Params &P, const CUtensorMap &mt, const CUtensorMap 
     mc = n;
   }
   const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(mc, max_tiles));
-  return launch_kernel(kern, 2 * pairs, kThreads, smem, s, mt, mts, mw, mw3, P);
+  return launch_kernel(kern, 2 * pairs, kThreads, smem, s, maps, P);
 }
 
 }  // namespace
@@ -2222,41 +2195,45 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   // of short groups
   const bool tn_epi = g.epi == kEpiRelu || g.epi == kEpiSwiglu || g.epi == kEpiScale ||
                       g.epi == kEpiScaleAdd;
-  if (tn_epi && !g.kgroup && g.n_routed > 0 && !g.b_mn && g.ksplit <= 1 &&
+  if (tn_epi && !g.kgroup && g.n_routed > 0 && !g.gather_rows && !g.b_mn && g.ksplit <= 1 &&
       g.max_routed_rows / g.n_routed < MOE_TN_MAX_ROWS) {
     const bool swiglu = g.epi == kEpiSwiglu;
     Params Q = P;
     Q.nt = swiglu ? (g.N + 127) / 128 : (g.N + 255) / 256;     // weight tiles per group
     Q.sk_part = nullptr;
     Q.sk_flags = nullptr;
-    CUtensorMap mt, mts, mw, mw3;
-    // routed rows: x_perm in 16-row boxes, or x itself in one-row boxes for
-    // the tile::gather4 loads
-    if (g.gather_rows) {
-      if (!make_map(&mt, g.gather_src, (uint64_t)g.K, (uint64_t)g.src_rows, 1)) return cudaErrorInvalidValue;
-    } else if (!make_map(&mt, g.a, (uint64_t)g.K, (uint64_t)g.a_rows, kTnTokBox)) {
-      return cudaErrorInvalidValue;
+    const double macs_tn = (double)(g.max_routed_rows + (int64_t)g.n_static * g.rows_static) * g.N *
+                           g.K * (swiglu ? 2 : 1);
+    const bool bk2_tn = MOE_PAIR_BK128 && g.K % (2 * BK) == 0 && macs_tn >= 2e11;
+    const uint32_t chunks = bk2_tn ? 2u : 1u;
+    TnMaps maps;
+    for (int i = 0; i < kTnBoxes; ++i) {
+      const uint32_t h = (uint32_t)(kTnTokBox * (i + 1));
+      if (!make_map3(&maps.tok[i], g.a, (uint64_t)g.K, (uint64_t)g.a_rows, h, chunks))
+        return cudaErrorInvalidValue;
+      if (!make_map3(&maps.tok_static[i], g.a_static ? g.a_static : g.a, (uint64_t)g.K,
+                     (uint64_t)(g.a_static ? g.a_static_rows : g.a_rows), h, chunks))
+        return cudaErrorInvalidValue;
     }
-    if (!make_map(&mts, g.a_static ? g.a_static : g.a, (uint64_t)g.K,
-                  (uint64_t)(g.a_static ? g.a_static_rows : g.a_rows), kTnTokBox))
-      return cudaErrorInvalidValue;
-    const uint32_t wbox = swiglu ? 64u : 128u;
-    if (!make_map(&mw, g.b, (uint64_t)g.K, (uint64_t)g.b_rows, wbox)) return cudaErrorInvalidValue;
-    if (!make_map(&mw3, swiglu ? g.b3 : g.b, (uint64_t)g.K, (uint64_t)g.b_rows, wbox))
-      return cudaErrorInvalidValue;
+    if (swiglu) {
+      if (!make_map(&maps.w, g.b, (uint64_t)g.K, (uint64_t)g.b_rows, 64)) return cudaErrorInvalidValue;
+      if (!make_map(&maps.w3, g.b3, (uint64_t)g.K, (uint64_t)g.b_rows, 64)) return cudaErrorInvalidValue;
+    } else {
+      if (!make_map3(&maps.w, g.b, (uint64_t)g.K, (uint64_t)g.b_rows, 128, chunks))
+        return cudaErrorInvalidValue;
+      maps.w3 = maps.w;
+    }
     const int64_t tt_routed = (g.max_routed_rows + kTnMaxN - 1) / kTnMaxN + g.n_routed;
     const int64_t tt_static = (int64_t)g.n_static * ((g.rows_static + kTnMaxN - 1) / kTnMaxN);
     const int64_t max_tiles = (tt_routed + tt_static) * Q.nt;
-    const double macs = (double)(g.max_routed_rows + (int64_t)g.n_static * g.rows_static) * g.N *
-                        g.K * (swiglu ? 2 : 1);
-    const bool bk2 = MOE_PAIR_BK128 && g.K % (2 * BK) == 0 && macs >= 2e11;
+    const bool bk2 = bk2_tn;
     const size_t stage = (size_t)(bk2 ? 2 : 1) * (kABytes + (size_t)(kTnMaxN / 2) * BK * 2);
     const size_t tsmem = (bk2 ? (size_t)kPairStages2 : (size_t)kPairStages) * stage + 1024 +
                          4 * (size_t)kTnStgBytes + (swiglu ? (size_t)kTnXchBytes : 0);
 #define MOE_TN_CASE(E_)                                                                  \
   case E_:                                                                               \
-    return bk2 ? launch_tn<E_, 2>(Q, mt, mts, mw, mw3, max_tiles, tsmem, s)              \
-               : launch_tn<E_, 1>(Q, mt, mts, mw, mw3, max_tiles, tsmem, s);
+    return bk2 ? launch_tn<E_, 2>(Q, maps, max_tiles, tsmem, s)                          \
+               : launch_tn<E_, 1>(Q, maps, max_tiles, tsmem, s);
     switch (g.epi) {
       MOE_TN_CASE(kEpiRelu)
       MOE_TN_CASE(kEpiSwiglu)

@@ -109,14 +109,14 @@ moe_status validate(const moe_config *c) {
 }
 
 // MOE_FUSED_GATHER=1 at build time: moe_forward's up-projection gathers the
-// routed rows of x itself on every tile kernel (16-byte cp.async copies);
-// by default only the token-N kernel does (TMA tile::gather4), and the
-// others read x_perm written by the gather kernel.
+// routed rows of x itself (16-byte cp.async copies in the tile kernels;
+// measured slower than the gather kernel, so off by default).
 #ifndef MOE_FUSED_GATHER
 #define MOE_FUSED_GATHER 0
 #endif
 static bool forward_gathers(const moe_config *c, int64_t rows_cap) {
-  return c->dtype == MOE_BF16 && (MOE_FUSED_GATHER || expert_gemm_gathers(c, rows_cap));
+  (void)rows_cap;
+  return c->dtype == MOE_BF16 && MOE_FUSED_GATHER;
 }
 
 #ifndef MOE_DOWN_REVERSE

@@ -230,14 +230,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s);
 #ifndef MOE_TN_MAX_ROWS
 #define MOE_TN_MAX_ROWS 384
 #endif
-// ... and then gathers the routed rows of x itself in moe_forward's
-// up-projection (TMA tile::gather4; MOE_TN_GATHER=0: x_perm as usual)
-#ifndef MOE_TN_GATHER
-#define MOE_TN_GATHER 1
-#endif
-inline bool expert_gemm_gathers(const moe_config *c, int64_t rows_cap) {
-  return MOE_TN_GATHER && c->dtype == MOE_BF16 && rows_cap / c->E < MOE_TN_MAX_ROWS;
-}
+
 
 // --- backward helpers (backward.cu) ----------------------------------------
 cudaError_t launch_transpose_bf16(const void *in, void *out, int R, int C, int64_t ld_in,

@@ -450,37 +450,41 @@ __global__ void __launch_bounds__(256) gate8_kernel(const GateParams P) {
   if (P.topk_idx == nullptr) return;          // expert choice: probabilities only
 
   // ---- selection keys and gate values of the routing rule -------------------
-  float key[EPL], gsrc[EPL];
+  // in place: l becomes the key, p the gate source
+  //   softmax: key = logit, gate = p
+  //   bias   : key = p + b_e (one fp32 add), gate = key   (DeepSeek-V3)
+  //   load   : key = logit + alpha * (1 - u_e), gate = p   (load-aware top-k)
+  if (P.rule != 0) {
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) {
-    const int e = e0 + j;
-    key[j] = l[j];
-    gsrc[j] = p[j];
-    if (P.rule != 0 && e < E) {
-      const float st = P.state[e];
-      if (P.rule == 1) {
-        key[j] = __fadd_rn(p[j], st);
-        gsrc[j] = key[j];
-      } else {
-        key[j] = __fadd_rn(l[j], __fmul_rn(P.alpha, __fsub_rn(1.0f, st)));
+    for (int j = 0; j < EPL; ++j) {
+      const int e = e0 + j;
+      if (e < E) {
+        const float st = P.state[e];
+        if (P.rule == 1) {
+          l[j] = __fadd_rn(p[j], st);
+          p[j] = l[j];
+        } else {
+          l[j] = __fadd_rn(l[j], __fmul_rn(P.alpha, __fsub_rn(1.0f, st)));
+        }
       }
     }
   }
+  float *key = l, *gsrc = p;
 
   // ---- group limit: groups of E/n_groups experts, keep the best topk_groups --
-  uint32_t allowed = 0xffffffffu;
-  int grp[EPL];
-  const int gsz = P.n_groups > 0 ? E / P.n_groups : E;
-#pragma unroll
-  for (int j = 0; j < EPL; ++j) grp[j] = (e0 + j) / gsz;
+  // amask bit j: expert e0 + j may be chosen
+  const uint32_t all_mine = EPL >= 32 ? 0xffffffffu : ((1u << EPL) - 1u);
+  uint32_t amask = all_mine;
   if (P.n_groups > 0) {
+    const int gsz = E / P.n_groups;
     float gs0 = -INFINITY, gs1 = -INFINITY, gs2 = -INFINITY, gs3 = -INFINITY;   // groups s + 8 i
 #pragma unroll 1
     for (int g = 0; g < P.n_groups; ++g) {
+      const int lo = g * gsz - e0, hi = lo + gsz;          // my slots in group g: [lo, hi)
       float v = -INFINITY;
 #pragma unroll
       for (int j = 0; j < EPL; ++j)
-        if (e0 + j < E && grp[j] == g) v = fmaxf(v, key[j]);
+        if (j >= lo && j < hi && e0 + j < E) v = fmaxf(v, key[j]);
 #pragma unroll
       for (int o = 1; o < 8; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
       if ((g & 7) == s) {
@@ -491,7 +495,7 @@ __global__ void __launch_bounds__(256) gate8_kernel(const GateParams P) {
         else gs3 = v;
       }
     }
-    allowed = 0;
+    amask = 0;
     uint32_t gtaken = 0;                          // bit i: group s + 8 i chosen
 #pragma unroll 1
     for (int r = 0; r < P.topk_groups; ++r) {
@@ -515,62 +519,55 @@ __global__ void __launch_bounds__(256) gate8_kernel(const GateParams P) {
           bi = oi;
         }
       }
-      allowed |= 1u << bi;
       if ((bi & 7) == s) gtaken |= 1u << (bi >> 3);
+      // my slots of group bi
+      const int lo = max(bi * gsz - e0, 0), hi = min(bi * gsz - e0 + gsz, EPL);
+      if (lo < hi) {
+        const uint32_t upto_hi = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+        amask |= upto_hi & ~((1u << lo) - 1u);
+      }
     }
-  } else {
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) grp[j] = 0;
   }
 
   // ---- top-k: k rounds of an arg-max over the eight lanes --------------------
+  // (a loop, not unrolled: the round's result goes to lane r of the eight,
+  // so no per-round arrays; keeps the code small for the instruction cache)
   uint32_t taken = 0;                             // bit j: expert e0 + j chosen
-  float gates[kMaxTopK];
-  int idxs[kMaxTopK];
-  float gsum = 0.f;
-#pragma unroll
-  for (int r = 0; r < kMaxTopK; ++r) {
-    gates[r] = 0.f;
-    idxs[r] = 0;
-    if (r < k) {
-      float bv = -INFINITY, bg = 0.f;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        const int e = e0 + j;
-        const bool ok = e < E && !((taken >> j) & 1u) && ((allowed >> grp[j]) & 1u);
-        if (ok && (key[j] > bv || (key[j] == bv && e < bi))) {
-          bv = key[j];
-          bi = e;
-          bg = gsrc[j];
-        }
-      }
-#pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        const float og = __shfl_xor_sync(0xffffffffu, bg, o);
-        if (ov > bv || (ov == bv && oi < bi)) {
-          bv = ov;
-          bi = oi;
-          bg = og;
-        }
-      }
-      if (bi >= e0 && bi < e0 + EPL) taken |= 1u << (bi - e0);
-      idxs[r] = bi;
-      gates[r] = bg;
-      gsum = (r == 0) ? bg : __fadd_rn(gsum, bg);
-    }
-  }
   int my_idx = 0;
-  float my_gate = 0.f;
+  float my_gate = 0.f, gsum = 0.f;
+#pragma unroll 1
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY, bg = 0.f;
+    int bi = 0x7fffffff;
 #pragma unroll
-  for (int r = 0; r < kMaxTopK; ++r) {
-    if (r < k && s == r) {
-      my_idx = idxs[r];
-      my_gate = P.renormalize ? __fdiv_rn(gates[r], gsum) : gates[r];
+    for (int j = 0; j < EPL; ++j) {
+      const int e = e0 + j;
+      const bool ok = e < E && !((taken >> j) & 1u) && ((amask >> j) & 1u);
+      if (ok && (key[j] > bv || (key[j] == bv && e < bi))) {
+        bv = key[j];
+        bi = e;
+        bg = gsrc[j];
+      }
     }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      const float og = __shfl_xor_sync(0xffffffffu, bg, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+        bg = og;
+      }
+    }
+    if (bi >= e0 && bi < e0 + EPL) taken |= 1u << (bi - e0);
+    if (s == r) {
+      my_idx = bi;
+      my_gate = bg;
+    }
+    gsum = (r == 0) ? bg : __fadd_rn(gsum, bg);
   }
+  if (P.renormalize) my_gate = __fdiv_rn(my_gate, gsum);
   if (live && s < k) {
     P.topk_idx[t * k + s] = my_idx;
     P.topk_gate[t * k + s] = my_gate;
@@ -699,9 +696,12 @@ cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float
     }
     return launch_kernel(kern, blocks, kTokWarps * 32, smem, s, P);
   }
-  // more than 32 experts: eight lanes a token (MOE_GATE8=0 at build time: a
-  // warp a token)
-  if (NV > 1 && MOE_GATE8) return launch_gate8(P, blocks, s);
+  // 33 to 64 experts: eight lanes a token (8 experts a lane, 60 registers);
+  // beyond that a warp a token, whose registers stay few enough for 32
+  // warps an SM (measured: DeepSeekMoE's 64 experts route 50 vs 65 us; 160
+  // experts 95 vs 83 us and 256 experts 191 vs 108 us the other way).
+  // MOE_GATE8=0 at build time: a warp a token throughout.
+  if (NV > 1 && MOE_GATE8 && c->E <= 64) return launch_gate8(P, blocks, s);
   return launch_nv(NV, P, blocks, smem, s);
 }
 

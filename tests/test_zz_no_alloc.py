@@ -101,8 +101,9 @@ def test_noalloc_limit_is_the_permutation_scratch():
     w2 = WORKLOADS["deepseekmoe_ec"].with_tokens(T + 32)
     cfg2 = api.config_from_workload(w2)
     assert api.query_sizes(cfg2).permute_workspace > api.NOALLOC_SCRATCH_BYTES
-    dummy = torch.empty(16, dtype=torch.int32, device="cuda")
-    with pytest.raises(api.MoeError) as ei:
-        api.moe_permute_noalloc(cfg2, dummy, None, None, dummy, dummy, dummy, dummy, dummy,
-                                dummy.float(), dummy, dummy)
-    assert ei.value.status == api.MOE_ERR_WORKSPACE
+    # refused by the library before it touches any buffer (the C call directly:
+    # the binding's own size checks would refuse these stand-in pointers first)
+    import ctypes
+    st = api._noalloc()(ctypes.byref(cfg2), 256, None, None, 256, 256, 256, 256, 256, 256, 256, 256,
+                        None)
+    assert st == api.MOE_ERR_WORKSPACE
