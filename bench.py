@@ -636,6 +636,8 @@ def main() -> None:
                     help="profiling shape: this many tokens instead of the workload's")
     ap.add_argument("--experts", type=int, default=0,
                     help="profiling shape: this many routed experts instead of the workload's")
+    ap.add_argument("--d-ff", type=int, default=0,
+                    help="profiling shape: this expert hidden size instead of the workload's")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
@@ -646,6 +648,9 @@ def main() -> None:
     if args.tokens:
         from dataclasses import replace
         w = replace(w.with_tokens(args.tokens), name=f"{w.name}[T={args.tokens}]")
+    if args.d_ff:
+        from dataclasses import replace
+        w = replace(w, d_ff=args.d_ff, name=f"{w.name}[d_ff={args.d_ff}]")
     if args.gemm_vs_library:
         run_gemm_vs_library(args, w)
     elif args.impl == "reference":

@@ -1614,6 +1614,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // pairs working at once share a weight tile in L2; they are dealt
 // round-robin (no stream-K tail).
 constexpr int kTnTokBox = 16;            // token box heights are multiples of this
+// stages of two k-blocks (one 3-D copy each) for large token-N GEMMs;
+// MOE_TN_BK2=0 at build time: six stages of one k-block
+#ifndef MOE_TN_BK2
+#define MOE_TN_BK2 1
+#endif
 constexpr int kTnBoxes = 8;              // one tensor map per height 16, 32, ..., 128
 constexpr int kTnMaxN = 256;             // token rows per tile (the MMA's N)
 constexpr int kTnGran = 32;              // tile widths are multiples of this
@@ -1635,10 +1640,11 @@ struct TnMaps {
   CUtensorMap w, w3;
 };
 
-// tiles per group: weight tiles x token tiles
-__device__ __forceinline__ int tn_token_tiles(int rows) { return (rows + kTnMaxN - 1) / kTnMaxN; }
+// tiles per group: weight tiles x token tiles of at most maxn rows
+__device__ __forceinline__ int tn_token_tiles(int rows, int maxn) { return (rows + maxn - 1) / maxn; }
 
-__device__ __forceinline__ TnTile tn_decode(int tile, const int *prefix, const int *rows, int G) {
+__device__ __forceinline__ TnTile tn_decode(int tile, const int *prefix, const int *rows, int G,
+                                            int maxn) {
   int lo = 0, hi = G - 1;
   while (lo < hi) {                      // largest g with prefix[g] <= tile
     const int mid = (lo + hi + 1) >> 1;
@@ -1648,7 +1654,7 @@ __device__ __forceinline__ TnTile tn_decode(int tile, const int *prefix, const i
   TnTile t;
   t.g = lo;
   const int r = rows[lo];
-  const int nn = tn_token_tiles(r);
+  const int nn = tn_token_tiles(r, maxn);
   const int width = ((r + nn - 1) / nn + kTnGran - 1) / kTnGran * kTnGran;
   const int local = tile - prefix[lo];
   t.wt = local / nn;
@@ -1771,9 +1777,10 @@ template <int EPI, int BKS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_tn_kernel(const __grid_constant__ TnMaps M, const Params P) {
   constexpr bool kSwiglu = EPI == kEpiSwiglu;
+  constexpr int kMaxN = kTnMaxN;                                // token rows per tile
   constexpr int STAGES = BKS == 2 ? kPairStages2 : kPairStages;
   constexpr uint32_t kWBytes = BM * BK * 2;                     // weights: 16 KB a k-block and CTA
-  constexpr uint32_t kTokBytes = (kTnMaxN / 2) * BK * 2;        // token rows: up to 16 KB
+  constexpr uint32_t kTokBytes = (kMaxN / 2) * BK * 2;          // token rows: up to 16 KB
   constexpr uint32_t stage_bytes = BKS * (kWBytes + kTokBytes);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ int s_prefix[kMaxGroups + 1];
@@ -1841,7 +1848,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         s_off[g] = off;
         s_rows[g] = rows;
-        tiles = tn_token_tiles(rows) * P.nt;
+        tiles = tn_token_tiles(rows, kMaxN) * P.nt;
       }
       int x = tiles;
 #pragma unroll
@@ -1870,7 +1877,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t armed = 0, armed_parity = 0;
     bool ok = true;
     for (int tile = pair; ok && tile < total; tile += npairs) {
-      const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G);
+      const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G, kMaxN);
       const bool routed = tl.g < P.n_routed;
       const int half = tl.n / 2;                       // this CTA's token rows: one box
       const CUtensorMap *mt = routed ? &M.tok[half / kTnTokBox - 1] : &M.tok_static[half / kTnTokBox - 1];
@@ -1919,7 +1926,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     bool ok = true;
     for (int tile = pair; ok && tile < total; tile += npairs) {
-      const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G);
+      const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G, kMaxN);
       const uint32_t idesc = idesc_bf16(2 * BM, tl.n);
       if (!mbar_wait(&acce_bar[acc], acc_phase ^ 1u, &s_abort, P.err, s_limit)) { ok = false; break; }
       tc_fence_after();
@@ -1958,7 +1965,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     int xpar = 0;
     for (int tile = pair; tile < total; tile += npairs) {
-      const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G);
+      const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G, kMaxN);
       // (warp-uniform exits: the epilogue's TMEM loads and stores are warp-wide)
       if (!__all_sync(0xffffffffu, mbar_wait(&accf_bar[acc], acc_phase, &s_abort, P.err, s_limit))) break;
       tc_fence_after();
@@ -2198,13 +2205,14 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   if (tn_epi && !g.kgroup && g.n_routed > 0 && !g.gather_rows && !g.b_mn && g.ksplit <= 1 &&
       g.max_routed_rows / g.n_routed < MOE_TN_MAX_ROWS) {
     const bool swiglu = g.epi == kEpiSwiglu;
+    const int maxn = kTnMaxN;
     Params Q = P;
     Q.nt = swiglu ? (g.N + 127) / 128 : (g.N + 255) / 256;     // weight tiles per group
     Q.sk_part = nullptr;
     Q.sk_flags = nullptr;
     const double macs_tn = (double)(g.max_routed_rows + (int64_t)g.n_static * g.rows_static) * g.N *
                            g.K * (swiglu ? 2 : 1);
-    const bool bk2_tn = MOE_PAIR_BK128 && g.K % (2 * BK) == 0 && macs_tn >= 2e11;
+    const bool bk2_tn = MOE_TN_BK2 && g.K % (2 * BK) == 0 && macs_tn >= 2e11;
     const uint32_t chunks = bk2_tn ? 2u : 1u;
     TnMaps maps;
     for (int i = 0; i < kTnBoxes; ++i) {
@@ -2223,13 +2231,14 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
         return cudaErrorInvalidValue;
       maps.w3 = maps.w;
     }
-    const int64_t tt_routed = (g.max_routed_rows + kTnMaxN - 1) / kTnMaxN + g.n_routed;
-    const int64_t tt_static = (int64_t)g.n_static * ((g.rows_static + kTnMaxN - 1) / kTnMaxN);
+    const int64_t tt_routed = (g.max_routed_rows + maxn - 1) / maxn + g.n_routed;
+    const int64_t tt_static = (int64_t)g.n_static * ((g.rows_static + maxn - 1) / maxn);
     const int64_t max_tiles = (tt_routed + tt_static) * Q.nt;
     const bool bk2 = bk2_tn;
-    const size_t stage = (size_t)(bk2 ? 2 : 1) * (kABytes + (size_t)(kTnMaxN / 2) * BK * 2);
-    const size_t tsmem = (bk2 ? (size_t)kPairStages2 : (size_t)kPairStages) * stage + 1024 +
-                         4 * (size_t)kTnStgBytes + (swiglu ? (size_t)kTnXchBytes : 0);
+    const size_t stage = (size_t)(bk2 ? 2 : 1) * ((size_t)kABytes + (size_t)(maxn / 2) * BK * 2);
+    const size_t nstages = bk2 ? (size_t)kPairStages2 : (size_t)kPairStages;
+    const size_t tsmem = nstages * stage + 1024 + 4 * (size_t)kTnStgBytes +
+                         (swiglu ? (size_t)kTnXchBytes : 0);
 #define MOE_TN_CASE(E_)                                                                  \
   case E_:                                                                               \
     return bk2 ? launch_tn<E_, 2>(Q, maps, max_tiles, tsmem, s)                          \
