@@ -33,15 +33,7 @@
 #include "device_common.cuh"
 #include "moe_internal.h"
 
-// the row gather by TMA bulk copies (MOE_GATHER_TMA=0 at build time: one
-// warp a row with 16-byte vectors)
-#ifndef MOE_GATHER_TMA
-#define MOE_GATHER_TMA 1
-#endif
-
 namespace moe {
-
-constexpr int kGatherTmaMaxSlots = 32;
 
 // ---------------------------------------------------------------------------
 // row gather: x_perm[r] = x[row_token[r]] for r < offsets[E], one warp per
@@ -75,119 +67,6 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
     }
     for (; v < vpr; v += 32) dst[v] = src[v];
   }
-}
-
-// ---------------------------------------------------------------------------
-// row gather with TMA bulk copies: one CTA per SM, one thread issuing.  Each
-// row is one contiguous copy x[row_token[r]] -> shared slot (completing on
-// the slot's mbarrier) and one copy slot -> x_perm[r] (a bulk async-group),
-// two instructions a row instead of a vector load and store per 16 bytes.
-// A ring of 2H slots: after the store of row i is issued, waiting until at
-// most H stores are still reading shared memory frees the slot of row
-// i - H, which is reloaded with row i + H, so H loads and H stores stay in
-// flight.  Waits on the slots' barriers are bounded.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-template <int H>
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(H) : "memory");
-}
-
-__global__ void __launch_bounds__(32, 1) gather_rows_tma_kernel(
-    const char *__restrict__ x, char *__restrict__ x_perm, const int32_t *__restrict__ row_token,
-    const int32_t *__restrict__ offsets, int E, int64_t T, uint32_t row_bytes, int slots,
-    uint32_t *err) {
-  extern __shared__ __align__(128) uint8_t ring[];
-  __shared__ __align__(8) uint64_t bar[kGatherTmaMaxSlots];
-  const int lane = threadIdx.x;
-  pdl_wait();
-  pdl_trigger();
-  if (lane != 0) return;
-  const int H = slots / 2;
-  for (int i = 0; i < slots; ++i)
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bar[i])));
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  const int64_t R = offsets[E];
-  const int64_t first = blockIdx.x, step = gridDim.x;
-  const int64_t mine = first < R ? (R - 1 - first) / step + 1 : 0;     // rows of this CTA
-  auto issue_load = [&](int64_t i) {
-    const int64_t r = first + i * step;
-    int64_t t = row_token[r];
-    if (t < 0 || t >= T) {
-      raise_error(err, kErrBadIndex);
-      t = 0;
-    }
-    const int sl = (int)(i % slots);
-    const uint32_t b = smem_addr(&bar[sl]);
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(row_bytes)
-                 : "memory");
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_addr(ring + (size_t)sl * row_bytes)),
-        "l"(x + t * row_bytes), "r"(row_bytes), "r"(b)
-        : "memory");
-  };
-  for (int64_t i = 0; i < mine && i < H; ++i) issue_load(i);
-  for (int64_t i = 0; i < mine; ++i) {
-    const int sl = (int)(i % slots);
-    const uint32_t parity = (uint32_t)((i / slots) & 1);
-    const uint32_t b = smem_addr(&bar[sl]);
-    // bounded wait for the row's load
-    const uint64_t t0 = global_timer_ns();
-    for (;;) {
-      uint32_t ok;
-      asm volatile(
-          "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-          "selp.u32 %0, 1, 0, p;\n\t}"
-          : "=r"(ok)
-          : "r"(b), "r"(parity)
-          : "memory");
-      if (ok) break;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        raise_error(err, kErrTimeout);
-        // let the loads still in flight (rows i .. i + H - 1) and the stores land
-        for (int64_t j = i; j < mine && j < i + H; ++j) {
-          const uint32_t bj = smem_addr(&bar[j % slots]);
-          const uint32_t pj = (uint32_t)((j / slots) & 1);
-          const uint64_t t1 = global_timer_ns();
-          for (;;) {
-            uint32_t done;
-            asm volatile(
-                "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                "selp.u32 %0, 1, 0, p;\n\t}"
-                : "=r"(done)
-                : "r"(bj), "r"(pj)
-                : "memory");
-            if (done || global_timer_ns() - t1 > kWaitLimitNs) break;
-          }
-        }
-        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-        return;
-      }
-    }
-    const int64_t r = first + i * step;
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                     x_perm + r * row_bytes),
-                 "r"(smem_addr(ring + (size_t)sl * row_bytes)), "r"(row_bytes)
-                 : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    // at most H stores still reading: the slot of row i - H + 1 ... is free
-    // once the store of row i + 1 - H has read it; reload it with row i + H
-    if (i + H < mine) {
-      switch (H) {                                    // the instruction takes a constant
-        case 1: bulk_wait_read<0>(); break;
-        case 2: bulk_wait_read<1>(); break;
-        case 4: bulk_wait_read<3>(); break;
-        case 8: bulk_wait_read<7>(); break;
-        default: bulk_wait_read<15>(); break;
-      }
-      issue_load(i + H);
-    }
-  }
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");          // x_perm written
 }
 
 // ---------------------------------------------------------------------------
@@ -733,23 +612,6 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const uint32_t row_bytes = (uint32_t)(c->d_model * elem_size(c));
-  if (MOE_GATHER_TMA && row_bytes % 16 == 0) {
-    // a ring of 2H row slots within 192 KB of shared memory, H a power of two <= 16
-    int slots = 2;
-    while (slots * 2 <= kGatherTmaMaxSlots && (size_t)slots * 2 * row_bytes <= (size_t)192 * 1024)
-      slots *= 2;
-    if ((size_t)slots * row_bytes <= (size_t)192 * 1024) {
-      const size_t smem = (size_t)slots * row_bytes;
-      cudaError_t e = cudaFuncSetAttribute(gather_rows_tma_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(L.rows_cap, sms));
-      return launch_kernel(gather_rows_tma_kernel, blocks, 32, smem, s,
-                           static_cast<const char *>(x), static_cast<char *>(x_perm), row_token,
-                           offsets, E, T, row_bytes, slots, err);
-    }
-  }
   const int64_t want = (L.rows_cap + 7) / 8;
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 8));
   return launch_kernel(gather_rows_kernel, blocks, 256, 0, s, xv, xp, row_token, offsets, E, T, vpr,
