@@ -51,6 +51,10 @@ DEFAULT_WORKLOAD = "deepseek_v2"
 NCU_TRAFFIC: dict[str, dict] = {
     # up 151.09 + 41.15 MB, down 220.18 + 9.75 MB
     "gshard": {"bytes": 422_169_088, "src": "a9de9705dc80e5bb"},
+    # captured on a 40-expert cut of the layer and scaled to 160 + 2 experts
+    # (weights) and 60693 kept rows (h, y_rows): up 1497.0 + 39.8 MB, down
+    # 707.5 + 122.4 MB at the cut
+    "deepseek_v2": {"bytes": 9_159_220_990, "src": "70e87a5ed947693e"},
 }
 
 
