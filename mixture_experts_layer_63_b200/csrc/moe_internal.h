@@ -2,6 +2,7 @@
 // workspace layout.  Not part of the public ABI (include/moe.h is).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -268,6 +269,25 @@ inline int router_ksplit(const moe_config *c) {
   while (ks > 1 && kb / ks < 4) --ks;
   return ks < 1 ? 1 : ks;
 }
+// --- tensor maps (gemm_sm100.cu) ---------------------------------------------
+// TMA descriptor of a bf16 matrix [outer][inner] (inner contiguous) read in
+// boxes of box_outer rows x 64 columns with the 128-byte swizzle; false when
+// the driver refuses it.
+bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+              uint32_t box_outer);
+int device_sms();
+
+// --- router GEMM with the gate in its epilogue (router_tc.cu) ---------------
+// true when moe_route / moe_forward run the bf16 router through it
+bool router_tc_used(const moe_config *c);
+// logits_out may be null (not written); topk_idx null: expert choice
+// (probabilities only); hist null: no unit histogram; y_zero as for
+// launch_route_gate
+cudaError_t launch_router_tc(const moe_config *c, const void *x, const void *w_router,
+                             const float *bias, const float *state, float *logits_out, float *probs,
+                             int32_t *topk_idx, float *topk_gate, int32_t *hist, void *y_zero,
+                             uint32_t *err, cudaStream_t s);
+
 // --- fp32 CUDA-core expert FFN (ffn_f32.cu) ----------------------------------
 cudaError_t launch_ffn_f32(const moe_config *c, const WsLayout &L, uint32_t *err, const float *x,
                            const float *x_perm,

@@ -35,6 +35,9 @@ constexpr int kTokWarps = kUnitTokens;     // one warp per token, one unit per b
 #ifndef MOE_GATE8
 #define MOE_GATE8 1
 #endif
+#ifndef MOE_GATE_WIDE
+#define MOE_GATE_WIDE 1
+#endif
 
 struct GateParams {
   const float *logits_in;     // [T, E] (null when the router is fused)
@@ -599,6 +602,214 @@ cudaError_t launch_gate8(const GateParams &P, int blocks, cudaStream_t s) {
   return cudaErrorInvalidValue;
 }
 
+// ---------------------------------------------------------------------------
+// Gate for more than 64 experts: a warp a token (lane l holding experts l,
+// l + 32, ...), 32 tokens a block, with the two serial parts moved off the
+// token's warp:
+//   * the softmax denominators: every warp stores its token's exponentials
+//     in shared memory, then one warp sums them with a lane per token, each
+//     lane adding its token's E values one at a time in ascending expert
+//     order (rows padded to E + 1 floats: the 32 lanes read different banks);
+//   * the group scores: lane g takes the maximum of group g's keys from the
+//     token's row in shared memory, instead of one warp-wide reduction per
+//     group.
+// Same operations in the same order as route_gate_kernel, so the same bits.
+// ---------------------------------------------------------------------------
+template <int NV>
+__global__ void __launch_bounds__(kTokWarps * 32, 1) gate_wide_kernel(const GateParams P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int E = P.E, k = P.k, ld = E + 1;
+  int *s_hist = reinterpret_cast<int *>(smem);                                // [k][E]
+  const int hist_ints = P.hist ? k * E : 0;
+  float *s_ex = reinterpret_cast<float *>(smem + ((kMaxTopK * kMaxExperts * 4 + 15) & ~15));
+  float *s_key = s_ex + kTokWarps * ld;                                       // [32][E + 1]
+  float *s_sum = s_key + kTokWarps * ld;                                      // [32]
+  pdl_wait();
+  pdl_trigger();
+  const int64_t t = (int64_t)blockIdx.x * kTokWarps + warp;
+  const bool live = t < P.T;
+  for (int i = threadIdx.x; i < hist_ints; i += blockDim.x) s_hist[i] = 0;
+  if (P.y_zero && live)
+    for (int v = lane; v < P.y_vecs; v += 32) P.y_zero[t * P.y_vecs + v] = make_uint4(0u, 0u, 0u, 0u);
+
+  // ---- logits (K parts added in order, then the bias), max, exponentials ----
+  float l[NV], ex[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int e = lane + 32 * j;
+    float v = -INFINITY;
+    if (live && e < E) {
+      v = P.logits_in[t * E + e];
+      for (int sp = 1; sp < P.nsplit; ++sp) v = __fadd_rn(v, P.logits_in[sp * P.split_stride + t * E + e]);
+      if (P.bias) v = __fadd_rn(v, P.bias[e]);
+      if (P.logits_out) P.logits_out[t * E + e] = v;
+    }
+    l[j] = v;
+  }
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) m = fmaxf(m, l[j]);
+  m = max_warp(m);
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int e = lane + 32 * j;
+    ex[j] = (live && e < E) ? exp_det(__fsub_rn(l[j], m)) : 0.f;
+    if (e < E) s_ex[warp * ld + e] = ex[j];
+  }
+  __syncthreads();
+  // ---- S = sum of a token's exponentials in ascending expert order, one
+  //      fp32 add at a time: warp 0, a lane per token ------------------------
+  if (warp == 0) {
+    const float *row = s_ex + lane * ld;
+    float S = row[0];
+#pragma unroll 8
+    for (int e = 1; e < E; ++e) S = __fadd_rn(S, row[e]);
+    s_sum[lane] = S;
+  }
+  __syncthreads();
+  const float S = s_sum[warp];
+  float p[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int e = lane + 32 * j;
+    p[j] = __fdiv_rn(ex[j], S);
+    if (live && e < E && P.probs) P.probs[t * E + e] = p[j];
+  }
+  if (P.topk_idx == nullptr) return;          // expert choice: probabilities only (no barrier follows)
+
+  // ---- selection keys and gate values of the routing rule -------------------
+  //   softmax: key = logit, gate = p
+  //   bias   : key = p + b_e (one fp32 add), gate = key   (DeepSeek-V3)
+  //   load   : key = logit + alpha * (1 - u_e), gate = p   (load-aware top-k)
+  float key[NV], gsrc[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = l[j];
+    gsrc[j] = p[j];
+    if (P.rule != 0 && e < E) {
+      const float st = P.state[e];
+      if (P.rule == 1) {
+        key[j] = __fadd_rn(p[j], st);
+        gsrc[j] = key[j];
+      } else {
+        key[j] = __fadd_rn(l[j], __fmul_rn(P.alpha, __fsub_rn(1.0f, st)));
+      }
+    }
+  }
+
+  // ---- group limit: lane g scores group g from the token's keys -------------
+  uint32_t allowed = 0xffffffffu;
+  const int gsz = P.n_groups > 0 ? E / P.n_groups : E;
+  if (P.n_groups > 0) {
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E) s_key[warp * ld + e] = key[j];
+    }
+    __syncwarp();
+    float sc = -INFINITY;
+    if (lane < P.n_groups) {
+      const float *row = s_key + warp * ld + lane * gsz;
+      for (int i = 0; i < gsz; ++i) sc = fmaxf(sc, row[i]);
+    }
+    allowed = 0;
+    int gtaken = 0;
+    for (int r = 0; r < P.topk_groups; ++r) {
+      float v = (lane < P.n_groups && !gtaken) ? sc : -INFINITY;
+      int i = (lane < P.n_groups && !gtaken) ? lane : 0x7fffffff;
+      argmax_warp(v, i);
+      allowed |= 1u << i;
+      if (lane == i) gtaken = 1;
+    }
+  }
+
+  // ---- top-k: k rounds of warp arg-max --------------------------------------
+  // open: bit j set while slot j (expert lane + 32 j) exists, is in an
+  // allowed group and has not been chosen
+  uint32_t open = 0;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int e = lane + 32 * j;
+    if (e < E && ((allowed >> (e / gsz)) & 1u)) open |= 1u << j;
+  }
+  int my_idx = 0;
+  float my_gate = 0.f, gsum = 0.f;
+#pragma unroll 1
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY, bg = 0.f;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int e = lane + 32 * j;
+      const bool ok = (open >> j) & 1u;
+      if (ok && (key[j] > bv || (key[j] == bv && e < bi))) {
+        bv = key[j];
+        bi = e;
+        bg = gsrc[j];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      const float og = __shfl_xor_sync(0xffffffffu, bg, o);
+      if (ov > bv || (ov == bv && oi < bi)) {
+        bv = ov;
+        bi = oi;
+        bg = og;
+      }
+    }
+    if (lane == (bi & 31)) open &= ~(1u << (bi >> 5));
+    if (lane == r) {
+      my_idx = bi;
+      my_gate = bg;
+    }
+    gsum = (r == 0) ? bg : __fadd_rn(gsum, bg);
+  }
+  if (P.renormalize) my_gate = __fdiv_rn(my_gate, gsum);
+  if (live && lane < k) {
+    P.topk_idx[t * k + lane] = my_idx;
+    P.topk_gate[t * k + lane] = my_gate;
+    if (P.hist && my_idx >= 0 && my_idx < E) atomicAdd(&s_hist[lane * E + my_idx], 1);
+  }
+  if (P.hist) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < hist_ints; i += blockDim.x) {
+      const int r = i / E, e = i - r * E;
+      // unit of (rank r, this block): group-major numbering, see unit_grid
+      const int g = blockIdx.x / P.nbg, bl = blockIdx.x - g * P.nbg;
+      const int64_t u = ((int64_t)g * P.k + r) * P.nbg + bl;
+      P.hist[u * E + e] = s_hist[i];
+    }
+  }
+}
+
+cudaError_t launch_gate_wide(const GateParams &P, int blocks, cudaStream_t s) {
+  const int NV = (P.E + 31) / 32;
+  const size_t smem = (size_t)((kMaxTopK * kMaxExperts * 4 + 15) & ~15) +
+                      (size_t)2 * kTokWarps * (P.E + 1) * 4 + kTokWarps * 4;
+#define MOE_GATE_WIDE_CASE(n)                                                              \
+  case n: {                                                                                \
+    auto kern = gate_wide_kernel<n>;                                                       \
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                         (int)smem);                                       \
+    if (e != cudaSuccess) return e;                                                        \
+    return launch_kernel(kern, blocks, kTokWarps * 32, smem, s, P);                        \
+  }
+  switch (NV) {
+    MOE_GATE_WIDE_CASE(3)
+    MOE_GATE_WIDE_CASE(4)
+    MOE_GATE_WIDE_CASE(5)
+    MOE_GATE_WIDE_CASE(6)
+    MOE_GATE_WIDE_CASE(7)
+    MOE_GATE_WIDE_CASE(8)
+    default: return cudaErrorInvalidValue;
+  }
+#undef MOE_GATE_WIDE_CASE
+}
+
 cudaError_t launch_nv(int NV, const GateParams &P, int blocks, size_t smem, cudaStream_t s) {
 #define MOE_GATE_CASE(n)                                                                       \
   case n: {                                                                                    \
@@ -702,6 +913,8 @@ cudaError_t launch_route_gate(const moe_config *c, const float *logits_in, float
   // experts 95 vs 83 us and 256 experts 191 vs 108 us the other way).
   // MOE_GATE8=0 at build time: a warp a token throughout.
   if (NV > 1 && MOE_GATE8 && c->E <= 64) return launch_gate8(P, blocks, s);
+  // more than 64 experts: a warp a token, sums and group scores off the warp
+  if (NV > 2 && MOE_GATE_WIDE) return launch_gate_wide(P, blocks, s);
   return launch_nv(NV, P, blocks, smem, s);
 }
 
