@@ -20,7 +20,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
 
 SOURCES = ["moe_api.cu", "router_gate.cu", "permute.cu", "gemm_sm100.cu", "ffn_f32.cu",
-           "combine.cu", "backward.cu"]
+           "combine.cu", "backward.cu", "router_tc.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -150,7 +150,7 @@ WsLayout make_layout(const moe_config *c) {
   L.sorted_q = take(keepfrac ? (size_t)T * k * 4 : 0);
   L.probs_t = take(tc ? 0 : (size_t)E * T * 4);
   L.permute_end = o;
-  const int ks = (c->dtype == MOE_BF16 && !router_is_fused(c)) ? router_ksplit(c) : 1;
+  const int ks = (c->dtype == MOE_BF16 && !router_is_fused(c) && !router_tc_used(c)) ? router_ksplit(c) : 1;
   L.logits_part = take(ks > 1 ? (size_t)ks * T * E * 4 : 0);
   L.sk_part = take(c->dtype == MOE_BF16 ? (size_t)kSkSlots * kSkSlotFloats * 4 : 0);
   L.step_end = o;
@@ -211,6 +211,11 @@ static cudaError_t run_route(const moe_config *c, const WsLayout &L, char *ws, c
   if (router_is_fused(c))
     return launch_route_gate(c, nullptr, logits, x, w_router, bias, state, probs, topk_idx,
                              topk_gate, hist, s, 1, 0, y_zero);
+  // bf16: the tcgen05 router GEMM with the gate in its epilogue (logits
+  // written only when the caller wants them)
+  if (router_tc_used(c))
+    return launch_router_tc(c, x, w_router, bias, state, logits, probs, topk_idx, topk_gate, hist,
+                            y_zero, reinterpret_cast<uint32_t *>(ws + L.err), s);
   cudaError_t e;
   if (c->dtype == MOE_F32) {
     e = launch_router_f32(c, static_cast<const float *>(x), static_cast<const float *>(w_router),
@@ -805,8 +810,9 @@ static moe_status forward_impl(const moe_config *cfg, const void *x, const void 
   cudaError_t e = mark(0);
   if (e == cudaSuccess) {
     Range r("route");
-    e = run_route(cfg, L, w, x, w_router, bias, state, logits, probs, topk_idx, topk_gate, s,
-                  fold ? y : nullptr);
+    // (the forward's logits have no reader: the fused router skips them)
+    e = run_route(cfg, L, w, x, w_router, bias, state, router_tc_used(cfg) ? nullptr : logits, probs,
+                  topk_idx, topk_gate, s, fold ? y : nullptr);
   }
   if (e == cudaSuccess) e = mark(1);
   // token choice: the gate wrote the unit histogram into the workspace.

@@ -54,6 +54,9 @@ SMALL = {
     "load_aware_s": replace(WORKLOADS["gshard"], T=700, d_model=256, d_ff=320, route_rule="load",
                             route_alpha=0.75, capacity_factor=0.0),
     "local_groups_s": replace(WORKLOADS["gshard_local"], T=768, d_model=256, d_ff=320),
+    # 64 experts, two rows a token: the router GEMM's epilogue gates and zeroes
+    # y, the down-projection adds the rows into it (folded combine)
+    "fold_tc_s": replace(WORKLOADS["gshard"], T=700, E=64, d_model=256, d_ff=320),
 }
 
 

@@ -18,13 +18,13 @@ CASES = {
     # router+gate, rank (own unit sums), gather, up, down (combine folded)
     "gshard": (WORKLOADS["gshard"], 5),
     "gshard_s": (SMALL["gshard_s"], 5),
-    # d = 4096: the tcgen05 router GEMM first
-    "mixtral": (WORKLOADS["mixtral"], 6),
-    # E = 64, k = 6 with shared experts: router GEMM, gate, rank, gather, up, down, combine;
+    # d = 4096: the tcgen05 router GEMM with the gate in its epilogue
+    "mixtral": (WORKLOADS["mixtral"], 5),
+    # E = 64, k = 6 with shared experts: router GEMM + gate, rank, gather, up, down, combine;
     # the 3072-unit histogram is summed by its own kernel
-    "deepseekmoe_tc": (WORKLOADS["deepseekmoe_tc"], 8),
+    "deepseekmoe_tc": (WORKLOADS["deepseekmoe_tc"], 7),
     # a small histogram with k + S > 2: the combine runs
-    "dsmoe_tc_s": (SMALL["dsmoe_tc_s"], 7),
+    "dsmoe_tc_s": (SMALL["dsmoe_tc_s"], 6),
 }
 
 

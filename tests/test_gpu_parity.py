@@ -65,6 +65,27 @@ ROUTE_EXTRA = {
     # E > 32: the tcgen05 router GEMM with K split over CTAs
     "split_k_s": replace(WORKLOADS["deepseekmoe_tc"], T=300),
     "split_k_groups_s": replace(WORKLOADS["deepseek_v2"], T=200, d_model=1024, keep_num=0, keep_den=0),
+    # the router GEMM with the gate in its epilogue (clusters of 4 or 2 K
+    # parts): a last 256-token tile with no second half (T = 800), two K
+    # parts (K / 64 not a multiple of 4; more tiles than a wave of clusters
+    # of 4), every expert count a lane is built for (E = 8 ... 256), lanes
+    # past E, groups across lanes and of two a lane, the three routing
+    # rules, renormalisation, expert choice
+    "tc_tail_groups_s": replace(WORKLOADS["deepseek_v2"], T=800, d_model=1024, keep_num=0, keep_den=0),
+    "tc_ks2_s": replace(WORKLOADS["deepseekmoe_tc"], T=300, d_model=384),
+    "tc_ks2_many_tiles_s": replace(WORKLOADS["deepseekmoe_tc"], T=9700, d_model=256),
+    "tc_e8_s": replace(WORKLOADS["mixtral"], T=300),
+    "tc_e33_s": replace(WORKLOADS["deepseekmoe_tc"], T=300, E=33, S=0, k=4, d_model=256),
+    "tc_e96_ec_s": replace(WORKLOADS["deepseekmoe_ec"], T=320, E=96, S=0, d_model=256, ec_capacity=20),
+    "tc_e128_renorm_s": replace(WORKLOADS["deepseekmoe_tc"], T=300, E=128, S=0, k=8, d_model=256,
+                                renormalize=True),
+    "tc_e192_load_s": replace(WORKLOADS["deepseekmoe_tc"], T=300, E=192, S=0, k=2, d_model=256,
+                              route_rule="load", route_alpha=0.5),
+    "tc_e100_groups_s": replace(WORKLOADS["deepseek_v2"], T=300, E=100, n_groups=4, topk_groups=2, k=5,
+                                d_model=256, keep_num=0, keep_den=0),
+    "tc_e64_groups16_s": replace(WORKLOADS["deepseek_v2"], T=300, E=64, n_groups=16, topk_groups=3, k=6,
+                                 d_model=256, keep_num=0, keep_den=0),
+    "tc_e224_bias_s": replace(WORKLOADS["deepseek_v3"], T=300, E=224, d_model=512),
 }
 
 
@@ -161,6 +182,34 @@ def test_gate_ties_go_to_the_lower_expert():
     assert np.array_equal(to_np(B.probs), probs)
     assert np.array_equal(to_np(B.topk_idx), idx)
     assert np.array_equal(to_np(B.topk_gate), gate)
+
+
+@pytest.mark.parametrize("groups", [False, True])
+def test_fused_router_gate_ties_go_to_the_lower_expert(groups):
+    """The gate inside the router GEMM's epilogue on logits with many exact
+    ties: x carries the wanted logits (quarters, exact in bf16) in its first
+    E columns and W_r is the identity on them, so l = x W_r^T is exactly
+    those values; moe_route must then route like the oracle, bit for bit,
+    with the lower expert (and group) index winning every tie."""
+    w = replace(WORKLOADS["deepseek_v2"], T=600, d_model=256, keep_num=0, keep_den=0,
+                **({} if groups else {"n_groups": 0, "topk_groups": 0}))
+    rng = np.random.default_rng(29)
+    ref_l = (rng.integers(-4, 5, size=(w.T, w.E)) / 4.0).astype(np.float32)
+    x = torch.zeros(w.T, w.d_model, dtype=torch.float32)
+    x[:, :w.E] = torch.from_numpy(ref_l)
+    wr = torch.zeros(w.E, w.d_model, dtype=torch.float32)
+    wr[:, :w.E] = torch.eye(w.E)
+    x, wr = x.to(torch.bfloat16).cuda(), wr.to(torch.bfloat16).cuda()
+    probs, idx, gate, _ = O.route(oracle_config(w), ref_l, None)
+    cfg = api.config_from_workload(w)
+    B = api.step_buffers(cfg)
+    api.moe_route(cfg, x, wr, None, B.logits, B.probs, B.topk_idx, B.topk_gate, B.ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(B.logits), ref_l)
+    assert np.array_equal(to_np(B.probs), probs)
+    assert np.array_equal(to_np(B.topk_idx), idx)
+    assert np.array_equal(to_np(B.topk_gate), gate)
+    api.moe_check_device_errors(B.ws)
 
 
 # ---------------------------------------------------------------------------
