@@ -134,26 +134,45 @@ __device__ __forceinline__ void gate8(const RtParams &P, float *lg, int r, int N
   for (int j = 0; j < EPL; ++j) m = fmaxf(m, l[j]);
 #pragma unroll
   for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  // slots past E hold -inf: exp_det gives exactly 0 there, and adding 0 to
+  // the running sum leaves it unchanged, so neither needs a guard
   float p[EPL];
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) p[j] = j < mine ? exp_det(__fsub_rn(l[j], m)) : 0.f;
+  for (int j = 0; j < EPL; ++j) p[j] = exp_det(__fsub_rn(l[j], m));
   // the denominator: one fp32 add at a time in ascending expert order, lane
-  // s extending the running sum of lanes 0 .. s-1 with its own experts
+  // s extending the running sum of lanes 0 .. s-1 with its own experts (lane
+  // 0 starts from 0: 0 + p_0 = p_0 exactly)
   float S = 0.f;
 #pragma unroll 1
   for (int step = 0; step < 8; ++step) {
-    const float prev = __shfl_sync(0xffffffffu, S, gb | ((step + 7) & 7));
-    if (s == step) {
-      float acc = prev;
+    float acc = __shfl_sync(0xffffffffu, S, gb | ((step + 7) & 7));
 #pragma unroll
-      for (int j = 0; j < EPL; ++j)
-        if (j < mine) acc = (step == 0 && j == 0) ? p[0] : __fadd_rn(acc, p[j]);
-      S = acc;
-    }
+    for (int j = 0; j < EPL; ++j) acc = __fadd_rn(acc, p[j]);
+    S = s == step ? acc : S;                   // (no branch: every lane adds, one keeps)
   }
   S = __shfl_sync(0xffffffffu, S, gb | 7);
+  // p_j = RN(e_j / S), the fp32 quotient rounded once, without a division a
+  // slot: with y = RN64(1 / S), RN32(RN64(e_j * y)) is that quotient whenever
+  // it is a normal fp32 number.  The fp64 value is within 2^-52 (relative)
+  // of e_j / S, and a normal fp32 quotient of normal operands is never
+  // closer than 2^-49 to a midpoint between fp32 values (a midpoint is an odd
+  // 25-bit multiple of a power of two, and e_j = S * m would then need 25
+  // significant bits), so both round to the same value.  A quotient below
+  // 2^-126 (e_j < S * 2^-126, e_j != 0: a logit about 87 below the
+  // maximum) has fewer significant bits and can sit on a midpoint: if any
+  // lane of the warp has one, the warp divides instead.
+  bool tiny = false;
+  const float t_min = S * 0x1p-126f;                 // exact: S >= 1
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) p[j] = __fdiv_rn(p[j], S);
+  for (int j = 0; j < EPL; ++j) tiny |= p[j] < t_min && p[j] != 0.f;
+  if (__any_sync(0xffffffffu, tiny)) {
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) p[j] = __fdiv_rn(p[j], S);
+  } else {
+    const double y = __drcp_rn((double)S);
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) p[j] = __double2float_rn((double)p[j] * y);
+  }
   if (live && P.probs) {
     float *pr = P.probs + t * E + e0;
     if ((E & 3) == 0) {
@@ -193,7 +212,10 @@ __device__ __forceinline__ void gate8(const RtParams &P, float *lg, int r, int N
     // group g = experts [g gsz, (g+1) gsz); score = its largest key.  Lane s
     // scores groups s, s + 8, s + 16, s + 24 from the keys in shared memory.
     const int ng = P.n_groups, gsz = E / ng;
-    if (P.rule != 0) {
+    // groups that are exactly one lane's experts (E = 8 EPL, eight groups):
+    // lane s's score is its own maximum key
+    const bool lane_groups = gsz == EPL && ng == 8;
+    if (P.rule != 0 && !lane_groups) {
 #pragma unroll
       for (int j = 0; j < EPL; j += 4)
         if (j < mine)
@@ -201,13 +223,21 @@ __device__ __forceinline__ void gate8(const RtParams &P, float *lg, int r, int N
       __syncwarp();
     }
     float gsc[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int g = s + 8 * i;
+    if (lane_groups) {
       float v = -INFINITY;
-      if (g < ng)
-        for (int e = g * gsz; e < g * gsz + gsz; ++e) v = fmaxf(v, lg[blk_off(r, e, NC)]);
-      gsc[i] = v;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) v = fmaxf(v, l[j]);
+      gsc[0] = v;
+      gsc[1] = gsc[2] = gsc[3] = -INFINITY;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int g = s + 8 * i;
+        float v = -INFINITY;
+        if (g < ng)
+          for (int e = g * gsz; e < g * gsz + gsz; ++e) v = fmaxf(v, lg[blk_off(r, e, NC)]);
+        gsc[i] = v;
+      }
     }
     uint32_t gtaken = 0, allowed = 0;
 #pragma unroll 1
@@ -254,12 +284,12 @@ __device__ __forceinline__ void gate8(const RtParams &P, float *lg, int r, int N
     int bj = -1;
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
-      // ascending experts: a strict > keeps the lower index on ties
-      if (((open >> j) & 1u) && l[j] > bv) {
-        bv = l[j];
-        bj = j;
-        bg = p[j];
-      }
+      // ascending experts: a strict > keeps the lower index on ties (no
+      // branch: a select a value)
+      const bool take = ((open >> j) & 1u) != 0u && l[j] > bv;
+      bv = take ? l[j] : bv;
+      bj = take ? j : bj;
+      bg = take ? p[j] : bg;
     }
     int bi = bj >= 0 ? e0 + bj : 0x7fffffff;
 #pragma unroll

@@ -184,6 +184,44 @@ def test_gate_ties_go_to_the_lower_expert():
     assert np.array_equal(to_np(B.topk_gate), gate)
 
 
+def _route_exact_logits(w, ref_l):
+    """moe_route on x carrying `ref_l` (exact in bf16) in its first E columns
+    and W_r the identity on them, so that l = x W_r^T is exactly ref_l."""
+    x = torch.zeros(w.T, w.d_model, dtype=torch.float32)
+    x[:, :w.E] = torch.from_numpy(ref_l)
+    wr = torch.zeros(w.E, w.d_model, dtype=torch.float32)
+    wr[:, :w.E] = torch.eye(w.E)
+    x, wr = x.to(torch.bfloat16).cuda(), wr.to(torch.bfloat16).cuda()
+    assert torch.equal(x[:, :w.E].float().cpu(), torch.from_numpy(ref_l))
+    cfg = api.config_from_workload(w)
+    B = api.step_buffers(cfg)
+    api.moe_route(cfg, x, wr, None, B.logits, B.probs, B.topk_idx, B.topk_gate, B.ws)
+    torch.cuda.synchronize()
+    api.moe_check_device_errors(B.ws)
+    return B
+
+
+def test_fused_router_gate_quotients_below_the_normal_range():
+    """Probabilities below 2^-126 (logits 82-87 below the token's maximum):
+    the fused gate's division then takes the IEEE quotient instead of the
+    fp64-reciprocal product; both must round exactly as the oracle's fp32
+    division, subnormal results included."""
+    w = replace(WORKLOADS["deepseek_v2"], T=300, d_model=256, keep_num=0, keep_den=0)
+    rng = np.random.default_rng(31)
+    ref_l = np.zeros((w.T, w.E), dtype=np.float32)
+    far = np.float32([-82.0, -83.0, -84.5, -85.0, -86.0, -86.5, -87.0, -88.0, -90.0])
+    ref_l[:] = far[rng.integers(0, len(far), size=(w.T, w.E))]
+    ref_l[np.arange(w.T), rng.integers(0, w.E, size=w.T)] = 0.0      # one maximum a token
+    ref_l[: w.T // 2] = np.where(rng.random((w.T // 2, w.E)) < 0.5, ref_l[: w.T // 2],
+                                 (rng.integers(-8, 1, size=(w.T // 2, w.E)) / 2.0).astype(np.float32))
+    probs, idx, gate, _ = O.route(oracle_config(w), ref_l, None)
+    assert (probs[probs > 0] < 2.0 ** -126).any(), "some probabilities must be subnormal"
+    B = _route_exact_logits(w, ref_l)
+    assert np.array_equal(to_np(B.probs), probs)
+    assert np.array_equal(to_np(B.topk_idx), idx)
+    assert np.array_equal(to_np(B.topk_gate), gate)
+
+
 @pytest.mark.parametrize("groups", [False, True])
 def test_fused_router_gate_ties_go_to_the_lower_expert(groups):
     """The gate inside the router GEMM's epilogue on logits with many exact
@@ -195,21 +233,12 @@ def test_fused_router_gate_ties_go_to_the_lower_expert(groups):
                 **({} if groups else {"n_groups": 0, "topk_groups": 0}))
     rng = np.random.default_rng(29)
     ref_l = (rng.integers(-4, 5, size=(w.T, w.E)) / 4.0).astype(np.float32)
-    x = torch.zeros(w.T, w.d_model, dtype=torch.float32)
-    x[:, :w.E] = torch.from_numpy(ref_l)
-    wr = torch.zeros(w.E, w.d_model, dtype=torch.float32)
-    wr[:, :w.E] = torch.eye(w.E)
-    x, wr = x.to(torch.bfloat16).cuda(), wr.to(torch.bfloat16).cuda()
     probs, idx, gate, _ = O.route(oracle_config(w), ref_l, None)
-    cfg = api.config_from_workload(w)
-    B = api.step_buffers(cfg)
-    api.moe_route(cfg, x, wr, None, B.logits, B.probs, B.topk_idx, B.topk_gate, B.ws)
-    torch.cuda.synchronize()
+    B = _route_exact_logits(w, ref_l)
     assert np.array_equal(to_np(B.logits), ref_l)
     assert np.array_equal(to_np(B.probs), probs)
     assert np.array_equal(to_np(B.topk_idx), idx)
     assert np.array_equal(to_np(B.topk_gate), gate)
-    api.moe_check_device_errors(B.ws)
 
 
 # ---------------------------------------------------------------------------
