@@ -46,15 +46,15 @@ DEFAULT_WORKLOAD = "deepseek_v2"
 
 # DRAM bytes (read + write) of the two expert GEMMs of one forward, from an
 # ncu capture of the same kernels, with the sha256 (first 16 hex digits) of
-# the GEMM source they were taken at; reported only while the source is
-# unchanged (null otherwise).
+# the GEMM sources (the kernel file, then its PTX wrappers) they were taken
+# at; reported only while the sources are unchanged (null otherwise).
 NCU_TRAFFIC: dict[str, dict] = {
-    # up 151.09 + 41.15 MB, down 220.18 + 9.75 MB
-    "gshard": {"bytes": 422_169_088, "src": "a9de9705dc80e5bb"},
+    # up 151.10 + 40.43 MB, down 220.13 + 9.89 MB
+    "gshard": {"bytes": 421_551_616, "src": "ca21efa7a723b0d4"},
     # captured on a 40-expert cut of the layer and scaled to 160 + 2 experts
-    # (weights) and 60693 kept rows (h, y_rows): up 1497.0 + 39.8 MB, down
-    # 707.5 + 122.4 MB at the cut
-    "deepseek_v2": {"bytes": 9_159_220_990, "src": "70e87a5ed947693e"},
+    # (weights) and 60693 kept rows (h, y_rows): up 1496.9 + 39.7 MB, down
+    # 707.4 + 122.4 MB at the cut
+    "deepseek_v2": {"bytes": 9_159_220_990, "src": "ca21efa7a723b0d4"},
 }
 
 
@@ -84,9 +84,11 @@ def _describe(w) -> str:
     return s
 
 
-def _src_hash(name: str) -> str:
-    p = os.path.join(ROOT, "mixture_experts_layer_63_b200", "csrc", name)
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+def _src_hash(*names: str) -> str:
+    h = hashlib.sha256()
+    for name in names:
+        h.update(open(os.path.join(ROOT, "mixture_experts_layer_63_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
 
 
 # ---------------------------------------------------------------------------
@@ -423,7 +425,7 @@ def run_ours(args, w) -> None:
     # the expert GEMMs' floor: their flops at the tensor peak, or streaming
     # every expert's weights once at the HBM peak, whichever is longer
     floor_ms = max(gemm_flops / (tfl * 1e12), weight_bytes / (hbm * 1e9)) * 1e3
-    h = _src_hash("gemm_sm100.cu")
+    h = _src_hash("gemm_sm100.cu", "sm100_ptx.cuh")
     tr = NCU_TRAFFIC.get(w.name)
     traffic = tr["bytes"] if tr and tr.get("src") == h else None
 
