@@ -569,6 +569,47 @@ def run_ours(args, w) -> None:
         dist.destroy_process_group()
 
 
+def run_route_only(args, w) -> None:
+    """The routing step alone (moe_route: router logits, softmax, group limit,
+    top-k), L2 flushed before every call, timed with CUDA events: the
+    number a profile of the router kernel refers to.  Algorithmic bytes: x
+    and W_r read, logits and probabilities written (fp32), top-k written."""
+    from mixture_experts_layer_63_b200 import api
+    torch.cuda.set_device(0)
+    inp = make_inputs(w, seed=args.seed, device="cuda", with_weights=False)
+    cfg = api.config_from_workload(w)
+    B = api.step_buffers(cfg)
+    flush = L2Flush()
+
+    def route():
+        api.moe_route(cfg, inp.x, inp.w_router, inp.bias, B.logits, B.probs, B.topk_idx, B.topk_gate,
+                      B.ws, route_state=inp.route_state)
+
+    for _ in range(args.warmup):
+        flush()
+        route()
+    torch.cuda.synchronize()
+    api.moe_check_device_errors(B.ws)
+    ts = []
+    for _ in range(args.steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        route()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    api.moe_check_device_errors(B.ws)
+    es = 4 if w.dtype == "f32" else 2
+    k = w.k if w.mode == "tc" else 0
+    nbytes = (w.T + w.E) * w.d_model * es + 2 * w.T * w.E * 4 + 2 * w.T * k * 4
+    us = float(np.median(ts))
+    hbm = _peaks()[0]
+    print(json.dumps({"mode": "route-only", "workload": w.name, "steps": args.steps,
+                      "route_us": round(us, 2), "route_gbs": round(nbytes / us / 1e3, 1),
+                      "hbm_frac": round(nbytes / us / 1e3 / hbm, 3), "algorithmic_bytes": nbytes}))
+
+
 def run_gemm_vs_library(args, w) -> None:
     """The expert GEMMs of this workload's shape, all rows on one expert (a
     dense problem), through moe_expert_ffn, next to torch.matmul (cuBLAS) on
@@ -638,6 +679,8 @@ def main() -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm-vs-library", action="store_true",
                     help="time the expert GEMMs on this workload's dense shape next to torch.matmul")
+    ap.add_argument("--route-only", action="store_true",
+                    help="time the routing step (moe_route) alone on this workload")
     ap.add_argument("--tokens", type=int, default=0,
                     help="profiling shape: this many tokens instead of the workload's")
     ap.add_argument("--experts", type=int, default=0,
@@ -659,6 +702,8 @@ def main() -> None:
         w = replace(w, d_ff=args.d_ff, name=f"{w.name}[d_ff={args.d_ff}]")
     if args.gemm_vs_library:
         run_gemm_vs_library(args, w)
+    elif args.route_only:
+        run_route_only(args, w)
     elif args.impl == "reference":
         run_reference(args, w)
     else:
