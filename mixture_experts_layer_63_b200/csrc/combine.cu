@@ -15,6 +15,10 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kMaxRows = kMaxExperts + 16;
+#ifndef MOE_COMBINE_BATCH
+#define MOE_COMBINE_BATCH 8
+#endif
+constexpr int kRowBatch = MOE_COMBINE_BATCH;    // rows loaded before they are added
 
 template <bool BF16>
 __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const void *__restrict__ y_rows,
@@ -43,7 +47,9 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const void *__rest
   n += S;
   __syncwarp();
 
-  // one 16-byte vector per lane and step: 8 bf16 or 4 fp32 elements
+  // one 16-byte vector per lane and step: 8 bf16 or 4 fp32 elements; the
+  // token's rows are loaded eight at a time before they are added (in row
+  // order), so a lane keeps up to eight loads in flight
   constexpr int EPV = BF16 ? 8 : 4;
   const int nvec = d / EPV;
   const uint4 *src = reinterpret_cast<const uint4 *>(y_rows);
@@ -51,18 +57,26 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const void *__rest
     float acc[EPV];
 #pragma unroll
     for (int i = 0; i < EPV; ++i) acc[i] = 0.f;
-    for (int i = 0; i < n; ++i) {
-      const uint4 a = src[(int64_t)rows[i] * nvec + v];
-      if (BF16) {
-        acc[0] += bf16_lo(a.x); acc[1] += bf16_hi(a.x);
-        acc[2 % EPV] += bf16_lo(a.y); acc[3 % EPV] += bf16_hi(a.y);
-        acc[4 % EPV] += bf16_lo(a.z); acc[5 % EPV] += bf16_hi(a.z);
-        acc[6 % EPV] += bf16_lo(a.w); acc[7 % EPV] += bf16_hi(a.w);
-      } else {
-        acc[0] += __uint_as_float(a.x);
-        acc[1] += __uint_as_float(a.y);
-        acc[2 % EPV] += __uint_as_float(a.z);
-        acc[3 % EPV] += __uint_as_float(a.w);
+    for (int i0 = 0; i0 < n; i0 += kRowBatch) {
+      uint4 a[kRowBatch];
+#pragma unroll
+      for (int i = 0; i < kRowBatch; ++i)
+        if (i0 + i < n) a[i] = src[(int64_t)rows[i0 + i] * nvec + v];
+#pragma unroll
+      for (int i = 0; i < kRowBatch; ++i) {
+        if (i0 + i < n) {
+          if (BF16) {
+            acc[0] += bf16_lo(a[i].x); acc[1] += bf16_hi(a[i].x);
+            acc[2 % EPV] += bf16_lo(a[i].y); acc[3 % EPV] += bf16_hi(a[i].y);
+            acc[4 % EPV] += bf16_lo(a[i].z); acc[5 % EPV] += bf16_hi(a[i].z);
+            acc[6 % EPV] += bf16_lo(a[i].w); acc[7 % EPV] += bf16_hi(a[i].w);
+          } else {
+            acc[0] += __uint_as_float(a[i].x);
+            acc[1] += __uint_as_float(a[i].y);
+            acc[2 % EPV] += __uint_as_float(a[i].z);
+            acc[3 % EPV] += __uint_as_float(a[i].w);
+          }
+        }
       }
     }
     if (BF16) {
