@@ -25,9 +25,10 @@
 // Both selections use an exact radix select over the 64-bit key
 // (p bits << 32 | ~t), so "larger p first, lower t on ties" is decided by
 // integer comparisons alone.
-//   gather_rows   x_perm[r] = x[row_token[r]], one warp per row, 16-byte
-//                 vectors (expert choice); token choice writes the same rows
-//                 token by token (scatter_rows: x read once).
+//   scatter_rows  x_perm[r] = x[row_token[r]], written token by token: one
+//                 warp per token reads its row of x once and writes it to
+//                 each of its rows (16-byte vectors).  (gather_rows, one
+//                 warp per row, is the build-time alternative.)
 #include <algorithm>
 #include <mutex>
 
@@ -71,34 +72,44 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint4 *__restric
 }
 
 // ---------------------------------------------------------------------------
-// token choice: the same rows written token by token.  One warp per token
-// reads x[t] once (8 16-byte vectors a lane at a time) and writes it to the
-// row of each kept choice, x_perm[tok_rows[t * k + j]] (-1: dropped).  Every
-// row of x crosses HBM once; the row-by-row gather above re-reads a token's
-// row for each of its choices, and the repeats mostly miss L2 while the
-// x_perm writes stream through it.
+// The same rows written token by token.  One warp per token collects the
+// rows of its kept choices (token choice: tok_rows[t * k + j]; expert
+// choice: tok_rows[e * T + t] over the experts; -1: not kept), then reads
+// x[t] once, 8 16-byte vectors a lane at a time, and writes each piece to
+// every one of those rows.  Every row of x crosses HBM once; the row-by-row
+// gather above re-reads a token's row for each of its rows, and the repeats
+// mostly miss L2 while the x_perm writes stream through it.
 // ---------------------------------------------------------------------------
 #ifndef MOE_SCATTER
 #define MOE_SCATTER 1
 #endif
-__global__ void __launch_bounds__(256) scatter_rows_kernel(const uint4 *__restrict__ x,
-                                                           uint4 *__restrict__ x_perm,
-                                                           const int32_t *__restrict__ tok_rows,
-                                                           int64_t T, int k, int vpr,
-                                                           int64_t rows_cap, uint32_t *err) {
-  const int lane = threadIdx.x & 31;
+constexpr int kScatterWarps = 8;
+__global__ void __launch_bounds__(kScatterWarps * 32) scatter_rows_kernel(
+    const uint4 *__restrict__ x, uint4 *__restrict__ x_perm, const int32_t *__restrict__ tok_rows,
+    int64_t T, int W, int expert_major, int vpr, int64_t rows_cap, uint32_t *err) {
+  __shared__ int s_rows[kScatterWarps][kMaxExperts];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int *rows = s_rows[warp];
   pdl_wait();
   pdl_trigger();
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nwarps) {
-    int slot = -1;
-    if (lane < k) {
-      slot = tok_rows[t * k + lane];
-      if (slot >= rows_cap) {
-        raise_error(err, kErrBadIndex);
-        slot = -1;
+  const int64_t nwarps = (int64_t)gridDim.x * kScatterWarps;
+  for (int64_t t = (int64_t)blockIdx.x * kScatterWarps + warp; t < T; t += nwarps) {
+    int n = 0;
+    for (int c = 0; c < W; c += 32) {
+      const int w = c + lane;
+      int r = -1;
+      if (w < W) {
+        r = expert_major ? tok_rows[(int64_t)w * T + t] : tok_rows[t * W + w];
+        if (r >= rows_cap) {
+          raise_error(err, kErrBadIndex);
+          r = -1;
+        }
       }
+      const unsigned valid = __ballot_sync(0xffffffffu, r >= 0);
+      if (r >= 0) rows[n + __popc(valid & ((1u << lane) - 1u))] = r;
+      n += __popc(valid);
     }
+    __syncwarp();
     const uint4 *src = x + t * vpr;
     for (int v0 = 0; v0 < vpr; v0 += 32 * 8) {
       uint4 buf[8];
@@ -107,10 +118,8 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const uint4 *__restri
         const int v = v0 + i * 32 + lane;
         if (v < vpr) buf[i] = src[v];
       }
-      for (int j = 0; j < k; ++j) {
-        const int sj = __shfl_sync(0xffffffffu, slot, j);
-        if (sj < 0) continue;                               // (the whole warp)
-        uint4 *dst = x_perm + (int64_t)sj * vpr;
+      for (int j = 0; j < n; ++j) {
+        uint4 *dst = x_perm + (int64_t)rows[j] * vpr;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int v = v0 + i * 32 + lane;
@@ -118,6 +127,7 @@ __global__ void __launch_bounds__(256) scatter_rows_kernel(const uint4 *__restri
         }
       }
     }
+    __syncwarp();
   }
 }
 
@@ -664,11 +674,13 @@ cudaError_t launch_permute(const moe_config *c, const WsLayout &L, char *ws, boo
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (MOE_SCATTER && c->mode == MOE_TOKEN_CHOICE) {
-    const int64_t tw = (T + 7) / 8;
+  if (MOE_SCATTER) {
+    const bool ec = c->mode == MOE_EXPERT_CHOICE;
+    const int64_t tw = (T + kScatterWarps - 1) / kScatterWarps;
     const int tblocks = (int)std::max<int64_t>(1, std::min<int64_t>(tw, (int64_t)sms * 8));
-    return launch_kernel(scatter_rows_kernel, tblocks, 256, 0, s, xv, xp,
-                         static_cast<const int32_t *>(tok_rows), T, c->k, vpr, L.rows_cap, err);
+    return launch_kernel(scatter_rows_kernel, tblocks, kScatterWarps * 32, 0, s, xv, xp,
+                         static_cast<const int32_t *>(tok_rows), T, ec ? E : c->k, ec ? 1 : 0, vpr,
+                         L.rows_cap, err);
   }
   const int64_t want = (L.rows_cap + 7) / 8;
   const int blocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 8));
