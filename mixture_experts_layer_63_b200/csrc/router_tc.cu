@@ -282,14 +282,32 @@ __device__ __forceinline__ void gate8(const RtParams &P, float *lg, int r, int N
   for (int rr = 0; rr < k; ++rr) {
     float bv = -INFINITY, bg = 0.f;
     int bj = -1;
+    // a tournament over the open slots, pairs (a, a + w) at width w = 1, 2,
+    // 4, ...: the right one wins only with a strictly larger key, so the
+    // lowest slot of the maximum wins (as a left-to-right scan), in log2(EPL)
+    // dependent steps instead of EPL
+    float tv[EPL], tg[EPL];
+    int tj[EPL];
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
-      // ascending experts: a strict > keeps the lower index on ties (no
-      // branch: a select a value)
-      const bool take = ((open >> j) & 1u) != 0u && l[j] > bv;
-      bv = take ? l[j] : bv;
-      bj = take ? j : bj;
-      bg = take ? p[j] : bg;
+      tv[j] = ((open >> j) & 1u) != 0u ? l[j] : -INFINITY;
+      tg[j] = p[j];
+      tj[j] = j;
+    }
+#pragma unroll
+    for (int w = 1; w < EPL; w <<= 1) {
+#pragma unroll
+      for (int a = 0; a + w < EPL; a += 2 * w) {
+        const bool take = tv[a + w] > tv[a];
+        tv[a] = take ? tv[a + w] : tv[a];
+        tg[a] = take ? tg[a + w] : tg[a];
+        tj[a] = take ? tj[a + w] : tj[a];
+      }
+    }
+    if (tv[0] != -INFINITY) {
+      bv = tv[0];
+      bj = tj[0];
+      bg = tg[0];
     }
     int bi = bj >= 0 ? e0 + bj : 0x7fffffff;
 #pragma unroll
