@@ -107,6 +107,16 @@ __device__ __forceinline__ float exp_det(float z) {
   return z < -87.0f ? 0.0f : out;
 }
 
+// SiLU(x) = x / (1 + e^-x) for the SwiGLU epilogues, with the fast
+// reciprocal-based division (about 2 ulp in fp32; the result is rounded to
+// bf16 next).  For x below about -88, e^-x is +inf and the quotient -0.
+#ifndef MOE_FAST_SILU
+#define MOE_FAST_SILU 1
+#endif
+__device__ __forceinline__ float silu_f(float x) {
+  return MOE_FAST_SILU ? __fdividef(x, 1.0f + __expf(-x)) : x / (1.0f + __expf(-x));
+}
+
 // Composite selection key: larger probability first, then lower token.
 __device__ __forceinline__ uint64_t affinity_key(float p, uint32_t t) {
   return ((uint64_t)__float_as_uint(p) << 32) | (uint64_t)(0xffffffffu - t);

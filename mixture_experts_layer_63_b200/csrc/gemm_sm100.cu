@@ -602,7 +602,7 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
           float uf[32];
           acc_cols(taddr, 128 + c * 32, F, uf);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = v[i] / (1.0f + __expf(-v[i])) * uf[i];
+          for (int i = 0; i < 32; ++i) v[i] = silu_f(v[i]) * uf[i];
         } else if constexpr (EPI == kEpiRelu) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.0f);
@@ -1493,12 +1493,12 @@ __device__ __forceinline__ void epilogue_tn(const Params &P, uint32_t taddr, con
       float h[16];
       if (gate_warp) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) h[i] = v[i] / (1.0f + __expf(-v[i])) * xu[i * 32 + lane];
+        for (int i = 0; i < 16; ++i) h[i] = silu_f(v[i]) * xu[i * 32 + lane];
       } else {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float g = xg[i * 32 + lane];
-          h[i] = g / (1.0f + __expf(-g)) * v[16 + i];
+          h[i] = silu_f(g) * v[16 + i];
         }
       }
       xpar ^= 1;
