@@ -52,9 +52,9 @@ NCU_TRAFFIC: dict[str, dict] = {
     # up 151.10 + 40.43 MB, down 220.13 + 9.89 MB
     "gshard": {"bytes": 421_551_616, "src": "ca21efa7a723b0d4"},
     # captured on a 40-expert cut of the layer and scaled to 160 + 2 experts
-    # (weights) and 60693 kept rows (h, y_rows): up 1496.9 + 39.7 MB, down
-    # 707.4 + 122.4 MB at the cut
-    "deepseek_v2": {"bytes": 9_159_220_990, "src": "ca21efa7a723b0d4"},
+    # (weights) and 60693 kept rows (h, y_rows): up 1495.8 + 40.6 MB, down
+    # 707.4 + 122.1 MB at the cut
+    "deepseek_v2": {"bytes": 9_157_548_175, "src": "ee4df9bbdfaf5e7e"},
 }
 
 
