@@ -108,13 +108,17 @@ __device__ __forceinline__ float exp_det(float z) {
 }
 
 // SiLU(x) = x / (1 + e^-x) for the SwiGLU epilogues, with the fast
-// reciprocal-based division (about 2 ulp in fp32; the result is rounded to
-// bf16 next).  For x below about -88, e^-x is +inf and the quotient -0.
+// reciprocal-based division (about 2 ulp in fp32; the results are rounded
+// to bf16 next).  For x below about -88, e^-x is +inf and the quotient -0.
 #ifndef MOE_FAST_SILU
 #define MOE_FAST_SILU 1
 #endif
 __device__ __forceinline__ float silu_f(float x) {
   return MOE_FAST_SILU ? __fdividef(x, 1.0f + __expf(-x)) : x / (1.0f + __expf(-x));
+}
+// its sigmoid factor 1 / (1 + e^-x) (the SwiGLU derivative), the same way
+__device__ __forceinline__ float sigmoid_f(float x) {
+  return MOE_FAST_SILU ? __fdividef(1.0f, 1.0f + __expf(-x)) : 1.0f / (1.0f + __expf(-x));
 }
 
 // Composite selection key: larger probability first, then lower token.

@@ -568,7 +568,7 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
         }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float sg = 1.0f / (1.0f + __expf(-a[i]));
+          const float sg = sigmoid_f(a[i]);
           const float dh = v[i] * scale;
           w[i] = dh * a[i] * sg;
           v[i] = dh * uu[i] * sg * (1.0f + a[i] * (1.0f - sg));
