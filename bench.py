@@ -52,9 +52,9 @@ NCU_TRAFFIC: dict[str, dict] = {
     # up 151.08 + 40.36 MB, down 220.13 + 6.13 MB
     "gshard": {"bytes": 417_699_840, "src": "31f89d5a39211448"},
     # captured on a 40-expert cut of the layer and scaled to 160 + 2 experts
-    # (weights) and 60693 kept rows (h, y_rows): up 1495.8 + 40.6 MB, down
-    # 707.4 + 122.1 MB at the cut
-    "deepseek_v2": {"bytes": 9_157_548_175, "src": "ee4df9bbdfaf5e7e"},
+    # (weights) and 60693 kept rows (h, y_rows): up 1488.6 + 40.2 MB, down
+    # 707.4 + 118.3 MB at the cut
+    "deepseek_v2": {"bytes": 9_113_835_476, "src": "31f89d5a39211448"},
 }
 
 
