@@ -86,6 +86,10 @@ ROUTE_EXTRA = {
     "tc_e64_groups16_s": replace(WORKLOADS["deepseek_v2"], T=300, E=64, n_groups=16, topk_groups=3, k=6,
                                  d_model=256, keep_num=0, keep_den=0),
     "tc_e224_bias_s": replace(WORKLOADS["deepseek_v3"], T=300, E=224, d_model=512),
+    # one token (three of a cluster's four CTAs own no token), and a ragged
+    # 32-token unit
+    "tc_t1_s": replace(WORKLOADS["deepseek_v2"], T=1, d_model=256, keep_num=0, keep_den=0),
+    "tc_t33_s": replace(WORKLOADS["deepseek_v2"], T=33, d_model=512, keep_num=0, keep_den=0),
 }
 
 
