@@ -119,6 +119,7 @@ struct Params {
   int M;
   const int32_t *kseg;
   int split_m;
+  int tma_store;            // token-N: whole boxes of output rows leave by TMA stores
   void *out2;
   uint32_t *err;
 };
@@ -1362,6 +1363,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 // round-robin (no stream-K tail).
 constexpr int kTnTokBox = 16;            // token box heights are multiples of this
 // stages of two k-blocks (one 3-D copy each) for large token-N GEMMs;
+// token-N epilogue: whole 32-column x NT-token pieces of the output leave
+// through TMA stores from the staging buffer (a tile's ragged last tokens
+// by plain stores); 0: plain stores throughout
+#ifndef MOE_TN_TMA_STORE
+#define MOE_TN_TMA_STORE 1
+#endif
 // MOE_TN_BK2=0 at build time: six stages of one k-block
 #ifndef MOE_TN_BK2
 #define MOE_TN_BK2 1
@@ -1385,6 +1392,7 @@ struct TnMaps {
   CUtensorMap tok[kTnBoxes];
   CUtensorMap tok_static[kTnBoxes];
   CUtensorMap w, w3;
+  CUtensorMap out;            // output rows, boxes of 32 columns x NT tokens (tma_store)
 };
 
 // tiles per group: weight tiles x token tiles of at most maxn rows
@@ -1429,10 +1437,45 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
 template <int NT, int EPI>
 __device__ __forceinline__ void store_tn(const Params &P, const float (&vals)[NT], int64_t row0,
                                          int tok0, int valid, bool routed, int64_t static_tok0,
-                                         int col_base, uint8_t *stg, int lane) {
+                                         int col_base, uint8_t *stg, int lane,
+                                         const CUtensorMap *omap, int &spar) {
   __nv_bfloat16 *out = reinterpret_cast<__nv_bfloat16 *>(P.out);
   const int64_t ld = P.N;
   const bool odd = (lane & 1) != 0;
+  // a whole box of NT tokens x 32 columns: packed into the staging buffer as
+  // NT rows of 64 bytes and stored by one TMA store (two buffers in turn
+  // when they fit, so the next chunk need not wait for this store)
+  constexpr int kBoxBytes = NT * 64;
+  constexpr int kBufs = 2 * kBoxBytes <= kTnStgBytes ? 2 : 1;
+  if (EPI != kEpiScaleAdd && MOE_TN_TMA_STORE && P.tma_store && tok0 + NT <= valid &&
+      col_base + 32 <= P.N) {
+    uint8_t *buf = stg + (kBufs == 2 ? spar * kBoxBytes : 0);
+    if (lane == 0) {                                  // the store that read this buffer last is done reading
+      if (kBufs == 2) bulk_wait_read<1>();
+      else bulk_wait_read<0>();
+    }
+    __syncwarp();
+    uint32_t *sw = reinterpret_cast<uint32_t *>(buf);
+#pragma unroll
+    for (int i = 0; i < NT / 2; ++i) {
+      const float send = odd ? vals[i] : vals[NT / 2 + i];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+      const uint32_t w = odd ? pack_bf16x2(recv, vals[NT / 2 + i]) : pack_bf16x2(vals[i], recv);
+      sw[(odd ? NT / 2 + i : i) * 16 + (lane >> 1)] = w;
+    }
+    fence_proxy_async_smem();                         // the tensor store reads through the async proxy
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(omap, buf, col_base, (int)(row0 + tok0));
+      bulk_commit();
+    }
+    spar ^= kBufs - 1;
+    return;
+  }
+  if (MOE_TN_TMA_STORE && P.tma_store) {              // the staging buffer is read no more
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
+  }
   uint32_t *sw = reinterpret_cast<uint32_t *>(stg);
 #pragma unroll
   for (int i = 0; i < NT / 2; ++i) {
@@ -1472,7 +1515,7 @@ template <int EPI>
 __device__ __forceinline__ void epilogue_tn(const Params &P, uint32_t taddr, const TnTile &tl,
                                             bool routed, int64_t row0, int64_t static_tok0,
                                             int col_base, uint8_t *stg, float *xch, int ew, int lane,
-                                            int &xpar) {
+                                            int &xpar, const CUtensorMap *omap, int &spar) {
   for (int c = 0; c < tl.n / 32; ++c) {
     if (32 * c >= tl.valid) break;                            // the same for the whole tile
     float v[32];
@@ -1503,7 +1546,7 @@ __device__ __forceinline__ void epilogue_tn(const Params &P, uint32_t taddr, con
       }
       xpar ^= 1;
       store_tn<16, EPI>(P, h, row0, 32 * c + (gate_warp ? 0 : 16), tl.valid, routed, static_tok0,
-                        col_base, stg, lane);
+                        col_base, stg, lane, omap, spar);
     } else {
       if constexpr (EPI == kEpiRelu) {
 #pragma unroll
@@ -1515,7 +1558,8 @@ __device__ __forceinline__ void epilogue_tn(const Params &P, uint32_t taddr, con
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] *= __shfl_sync(0xffffffffu, gm, i);
       }
-      store_tn<32, EPI>(P, v, row0, 32 * c, tl.valid, routed, static_tok0, col_base, stg, lane);
+      store_tn<32, EPI>(P, v, row0, 32 * c, tl.valid, routed, static_tok0, col_base, stg, lane,
+                        omap, spar);
     }
   }
 }
@@ -1710,7 +1754,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t acce_even1 = mapa_shared(smem_u32(&acce_bar[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    int xpar = 0;
+    int xpar = 0, spar = 0;
     for (int tile = pair; tile < total; tile += npairs) {
       const TnTile tl = tn_decode(tile, s_prefix, s_rows, P.G, kMaxN);
       // (warp-uniform exits: the epilogue's TMEM loads and stores are warp-wide)
@@ -1723,11 +1767,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                            tl.n0;
       const int col_base = kSwiglu ? tl.wt * 128 + (int)rank * 64 + 32 * (ew & 1)
                                    : tl.wt * 256 + (int)rank * 128 + 32 * ew;
-      epilogue_tn<EPI>(P, taddr, tl, routed, row0, (int64_t)tl.n0, col_base, stg, xch, ew, lane, xpar);
+      epilogue_tn<EPI>(P, taddr, tl, routed, row0, (int64_t)tl.n0, col_base, stg, xch, ew, lane, xpar,
+                       &M.out, spar);
       tc_fence_before();
       mbar_arrive_cluster(acc == 0 ? acce_even0 : acce_even1);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait_all();                 // this warp's TMA stores written before the CTA ends
   }
 
   tc_fence_before();
@@ -1792,6 +1838,22 @@ bool make_map3(CUtensorMap *m, const void *base, uint64_t K, uint64_t rows, uint
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D bf16 tensor [outer][inner] (inner contiguous) in boxes of box_outer
+// rows x box_inner columns, no swizzle: the token-N epilogue's TMA stores
+// (rows of box_inner * 2 bytes in shared memory).
+bool make_map_box(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                  uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int device_sms() {
@@ -1982,6 +2044,12 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
         return cudaErrorInvalidValue;
       maps.w3 = maps.w;
     }
+    // TMA stores of the outputs: boxes of 32 columns x 16 (SwiGLU) or 32 tokens
+    Q.tma_store = 0;
+    if (MOE_TN_TMA_STORE && g.epi != kEpiScaleAdd && g.out_rows > 0 && g.out_rows < ((int64_t)1 << 31) &&
+        g.N % 32 == 0 &&
+        make_map_box(&maps.out, g.out, (uint64_t)g.N, (uint64_t)g.out_rows, 32, swiglu ? 16u : 32u))
+      Q.tma_store = 1;
     const int64_t tt_routed = (g.max_routed_rows + maxn - 1) / maxn + g.n_routed;
     const int64_t tt_static = (int64_t)g.n_static * ((g.rows_static + maxn - 1) / maxn);
     const int64_t max_tiles = (tt_routed + tt_static) * Q.nt;

@@ -302,6 +302,7 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
   up.out_static_base = L.rows_cap;
   up.max_routed_rows = L.rows_cap;
   up.out = h;
+  up.out_rows = L.rows_total;
   up.sk_part = reinterpret_cast<float *>(ws + L.sk_part);
   up.sk_flags = reinterpret_cast<int *>(ws + L.err + kSkFlagsOffset);
   up.err = err;
@@ -327,6 +328,7 @@ static cudaError_t run_ffn(const moe_config *c, const WsLayout &L, char *ws, con
   dn.out_static_base = L.rows_cap;
   dn.max_routed_rows = L.rows_cap;
   dn.out = y_add ? y_add : y_rows;
+  dn.out_rows = y_add ? 0 : L.rows_total;
   dn.add_rows = y_add ? add_rows : nullptr;
   dn.src_rows = c->T;
   dn.row_gate = row_gate;

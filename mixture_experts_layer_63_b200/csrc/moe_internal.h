@@ -184,6 +184,7 @@ struct GroupedGemm {
   int64_t out_static_base;
   int64_t max_routed_rows;  // host upper bound of offsets[n_routed] (grid sizing)
   void *out;                // [*, N] row-major, ld = N
+  int64_t out_rows;         // rows of out (token-N kernel: > 0 enables TMA stores of whole boxes)
   const float *row_gate;    // kEpiScale: gate per routed output row
   const float *bias;        // kEpiStoreF32: [N] or null (ignored when ksplit > 1)
   int ksplit;               // kEpiStoreF32, one static group: split K into ksplit parts and
