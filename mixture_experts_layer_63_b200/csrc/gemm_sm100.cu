@@ -428,6 +428,26 @@ __device__ __forceinline__ void store_rows(uint8_t *stg, const uint32_t (&pk)[PI
   __syncwarp();
 }
 
+// store_rows<8> for a warp whose 32 rows are all to be written, through
+// one TMA store: the staging above already holds piece c of row r at slot
+// c ^ (r mod 8), the layout of a 128-byte-swizzled box of 32 rows x 64
+// columns (the staging buffer is 1024-byte aligned).  The next use of the
+// staging waits until the store has read it.
+__device__ __forceinline__ void store_rows_tma(uint8_t *stg, const uint32_t (&pk)[32],
+                                               const CUtensorMap *omap, int64_t row0, int col,
+                                               int lane) {
+  uint4 *mine = reinterpret_cast<uint4 *>(stg + lane * 128);
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    mine[stage_slot<8>(lane, c)] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(omap, stg, col, (int)row0);
+    bulk_commit();
+  }
+}
+
 // The same staging, with the rows added into out (bf16, vector reductions)
 // at rows dest of each thread's row (-1: not added) instead of stored.
 __device__ __forceinline__ void red_add_bf16x8(__nv_bfloat16 *p, const uint4 w) {
@@ -502,7 +522,7 @@ template <int EPI>
 __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, bool valid, bool routed,
                                               int64_t out_row, int col0, uint8_t *stg, int lane,
                                               int64_t out_offset = 0, const Fixup *F = nullptr,
-                                              int dest = -1) {
+                                              int dest = -1, const CUtensorMap *omap = nullptr) {
   float v[32];
   if constexpr (EPI == kEpiStoreF32) {
     // a K part when the router is split: no bias, own output
@@ -630,7 +650,12 @@ __device__ __forceinline__ void epilogue_tile(const Params &P, uint32_t taddr, b
         if (h == 0) pack_words<0>(pk, v);
         else pack_words<1>(pk, v);
       }
+      if (P.tma_store) {                                       // the last TMA store has read stg
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+      }
       if constexpr (EPI == kEpiScaleAdd) red_rows(stg, pk, out, ld, dest, col, lane);
+      else if (P.tma_store && omap && vmask == 0xffffffffu) store_rows_tma(stg, pk, omap, row0, col, lane);
       else store_rows<8>(stg, pk, out, ld, row0, col, vmask, lane);
     }
     if (EPI == kEpiDActRelu && P.dg_part && routed && valid)
@@ -683,7 +708,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                         const __grid_constant__ CUtensorMap map_a_static,
                         const __grid_constant__ CUtensorMap map_b,
-                        const __grid_constant__ CUtensorMap map_b3, const Params P) {
+                        const __grid_constant__ CUtensorMap map_b3,
+                        const __grid_constant__ CUtensorMap map_out, const Params P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ int s_prefix[kMaxGroups + 1];
   __shared__ int s_off[kMaxGroups];
@@ -968,17 +994,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (in_tail && kb1 < KB) {                              // finalizer of a split tile
           const Fixup F{P.sk_part, &sc, (int)blockIdx.x + 1, sc.contributors_end(tile), 1, 0, r_cta};
           if (!__all_sync(0xffffffffu, sk_wait(P, F, &s_abort, s_limit))) break;
-          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F, dest);
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F, dest, &map_out);
           sk_done(P, F);
         } else {
           epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane,
-                             (int64_t)part * P.split_stride, nullptr, dest);
+                             (int64_t)part * P.split_stride, nullptr, dest, &map_out);
         }
       }
       tc_fence_before();
       mbar_arrive(&acce_bar[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (P.tma_store && lane == 0) bulk_wait_all();     // this warp's TMA stores written
   }
 
   tc_fence_before();
@@ -1013,7 +1040,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a,
                              const __grid_constant__ CUtensorMap map_a_static,
                              const __grid_constant__ CUtensorMap map_b,
-                             const __grid_constant__ CUtensorMap map_b3, const Params P) {
+                             const __grid_constant__ CUtensorMap map_b3,
+                             const __grid_constant__ CUtensorMap map_out, const Params P) {
   constexpr int PM = 2 * BM;                         // rows per pair tile
   constexpr int STAGES = BKS == 2 ? kPairStages2 : kPairStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1319,16 +1347,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (in_tail && kb1 < KB) {                              // finalizer of a split tile
           const Fixup F{P.sk_part, &sc, pair + 1, sc.contributors_end(tile), 2, (int)rank, r_cta};
           if (!__all_sync(0xffffffffu, sk_wait(P, F, &s_abort, s_limit))) break;
-          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F, dest);
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, &F, dest, &map_out);
           sk_done(P, F);
         } else {
-          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, nullptr, dest);
+          epilogue_tile<EPI>(P, taddr, valid, routed, out_row, col0, stg, lane, 0, nullptr, dest, &map_out);
         }
       }
       tc_fence_before();
       mbar_arrive_cluster(acc == 0 ? acce_even0 : acce_even1);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (P.tma_store && lane == 0) bulk_wait_all();     // this warp's TMA stores written
   }
 
   tc_fence_before();
@@ -1368,6 +1397,10 @@ constexpr int kTnTokBox = 16;            // token box heights are multiples of t
 // by plain stores); 0: plain stores throughout
 #ifndef MOE_TN_TMA_STORE
 #define MOE_TN_TMA_STORE 1
+#endif
+// the same for the single-CTA and CTA-pair kernels' bf16 forward outputs
+#ifndef MOE_PAIR_TMA_STORE
+#define MOE_PAIR_TMA_STORE 1
 #endif
 // MOE_TN_BK2=0 at build time: six stages of one k-block
 #ifndef MOE_TN_BK2
@@ -1868,19 +1901,19 @@ namespace {
 template <int EPI>
 cudaError_t launch_epi(const Params &P, const CUtensorMap &ma,
                        const CUtensorMap &mas, const CUtensorMap &mb, const CUtensorMap &mb3,
-                       int grid, size_t smem, cudaStream_t s) {
+                       const CUtensorMap &mo, int grid, size_t smem, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_kernel(grouped_gemm_kernel<EPI>, grid, kThreads, smem, s, ma, mas, mb, mb3, P);
+  return launch_kernel(grouped_gemm_kernel<EPI>, grid, kThreads, smem, s, ma, mas, mb, mb3, mo, P);
 }
 
 // CTA-pair launch: as many 2-CTA clusters as fit at once (one CTA per SM),
 // fewer when there are fewer tiles.
 template <int EPI, int BKS>
 cudaError_t launch_pair(const Params &P, const CUtensorMap &ma, const CUtensorMap &mas,
-                        const CUtensorMap &mb, const CUtensorMap &mb3, int64_t max_tiles,
-                        size_t smem, cudaStream_t s) {
+                        const CUtensorMap &mb, const CUtensorMap &mb3, const CUtensorMap &mo,
+                        int64_t max_tiles, size_t smem, cudaStream_t s) {
   auto kern = grouped_gemm_pair_kernel<EPI, BKS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -1903,7 +1936,7 @@ cudaError_t launch_pair(const Params &P, const CUtensorMap &ma, const CUtensorMa
   }
   const int64_t want = P.sk_part ? mc : std::min<int64_t>(mc, max_tiles);
   const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(want, kSkSlots / 2));
-  return launch_kernel(kern, 2 * pairs, kThreads, smem, s, ma, mas, mb, mb3, P);
+  return launch_kernel(kern, 2 * pairs, kThreads, smem, s, ma, mas, mb, mb3, mo, P);
 }
 
 // Token-N launch: as many 2-CTA clusters as fit at once, fewer when there are
@@ -2078,12 +2111,20 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   const bool pair = P.bn == 256 &&
                     ((!g.kgroup && g.n_routed > 0 && g.max_routed_rows / g.n_routed >= MOE_PAIR_MIN_ROWS) ||
                      (g.kgroup && g.M >= 2 * BM && MOE_PAIR_WGRAD));
-  CUtensorMap ma, mas, mb, mb3;
+  CUtensorMap ma, mas, mb, mb3, mo;
+  // bf16 forward outputs: whole 32-row x 64-column pieces by TMA stores
+  // (boxes of the 128-byte-swizzled staging)
+  P.tma_store = 0;
+  if (MOE_PAIR_TMA_STORE && (g.epi == kEpiRelu || g.epi == kEpiSwiglu || g.epi == kEpiScale) &&
+      !g.kgroup && g.out_rows > 0 && g.out_rows < ((int64_t)1 << 31) && g.N % 64 == 0 &&
+      make_map(&mo, g.out, (uint64_t)g.N, (uint64_t)g.out_rows, 32))
+    P.tma_store = 1;
   const uint32_t box_b = (swiglu_b(g.epi) || pair) ? 128u : (uint32_t)P.bn;
   // K groups: A is [M, K] and B [N, K] with all groups' K columns side by side
   const uint64_t a_outer = g.kgroup ? (uint64_t)g.M : (uint64_t)g.a_rows;
   const uint64_t b_outer = g.kgroup ? (uint64_t)g.N : (uint64_t)g.b_rows;
   if (!make_map(&ma, g.a, (uint64_t)g.K, a_outer, BM)) return cudaErrorInvalidValue;
+  if (!P.tma_store) mo = ma;                                 // (not read)
   if (!make_map(&mas, g.a_static && !g.kgroup ? g.a_static : g.a, (uint64_t)g.K,
                 (uint64_t)(g.a_static && !g.kgroup ? g.a_static_rows : a_outer), BM))
     return cudaErrorInvalidValue;
@@ -2128,8 +2169,8 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
                          1024 + 4 * kStageBytesPerWarp;
 #define MOE_PAIR_CASE(E_)                                                            \
   case E_:                                                                           \
-    return bk2 ? launch_pair<E_, 2>(P, ma, mas, mb, mb3, pair_tiles, psmem, s)       \
-               : launch_pair<E_, 1>(P, ma, mas, mb, mb3, pair_tiles, psmem, s);
+    return bk2 ? launch_pair<E_, 2>(P, ma, mas, mb, mb3, mo, pair_tiles, psmem, s)   \
+               : launch_pair<E_, 1>(P, ma, mas, mb, mb3, mo, pair_tiles, psmem, s);
     switch (g.epi) {
       MOE_PAIR_CASE(kEpiStoreF32)
       MOE_PAIR_CASE(kEpiRelu)
@@ -2146,7 +2187,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
   }
 #define MOE_ONE_CASE(E_)                                                             \
   case E_:                                                                           \
-    return launch_epi<E_>(P, ma, mas, mb, mb3, grid, smem, s);
+    return launch_epi<E_>(P, ma, mas, mb, mb3, mo, grid, smem, s);
   switch (g.epi) {
     MOE_ONE_CASE(kEpiStoreF32)
     MOE_ONE_CASE(kEpiRelu)
