@@ -49,12 +49,12 @@ DEFAULT_WORKLOAD = "deepseek_v2"
 # the GEMM sources (the kernel file, then its PTX wrappers) they were taken
 # at; reported only while the sources are unchanged (null otherwise).
 NCU_TRAFFIC: dict[str, dict] = {
-    # up 151.08 + 40.36 MB, down 220.13 + 6.13 MB
-    "gshard": {"bytes": 417_699_840, "src": "31f89d5a39211448"},
+    # up 151.09 + 39.97 MB, down 220.03 + 6.44 MB
+    "gshard": {"bytes": 417_516_800, "src": "185a493843fb085a"},
     # captured on a 40-expert cut of the layer and scaled to 160 + 2 experts
-    # (weights) and 60693 kept rows (h, y_rows): up 1488.6 + 40.2 MB, down
-    # 707.4 + 118.3 MB at the cut
-    "deepseek_v2": {"bytes": 9_113_835_476, "src": "31f89d5a39211448"},
+    # (weights) and 60693 kept rows (h, y_rows): up 1496.2 + 40.0 MB, down
+    # 707.4 + 118.8 MB at the cut
+    "deepseek_v2": {"bytes": 9_144_011_170, "src": "185a493843fb085a"},
 }
 
 
