@@ -557,6 +557,14 @@ def test_single_expert_dense_ffn():
     _forward_check(w)
 
 
+@pytest.mark.parametrize("base,S", [("dsv3_s", 8), ("dsmoe_tc_s", 8), ("tiny_f32", 3)])
+def test_forward_most_shared_experts(base, S):
+    """The largest shared-expert count the library takes (8): with the V3
+    shape's 256 routed experts that is 264 weight groups in one grouped GEMM;
+    and shared experts on the fp32 path."""
+    _forward_check(replace(SMALL[base], S=S, T=300))
+
+
 def test_all_routed_dropped_leaves_shared_experts():
     w = replace(SMALL["dsv2_s"], T=300, keep_num=0, keep_den=1)
     rel, disp = _forward_check(w)
