@@ -678,8 +678,13 @@ __device__ __forceinline__ int add_dest(const Params &P, bool routed, int64_t ou
 // zeros when the group has no K columns (zero is the same for the whole
 // CTA, so the warp's TMEM loads stay aligned); dst null: row past M.  Whole
 // 32-column groups (128 bytes a row) leave through the staging buffer.
+// `om`: the fp32 tensor map of the output part that holds all 32 rows of
+// this warp, `orow` the first of them there; whole 32-row x 32-column pieces
+// then leave by TMA stores from the 128-byte-swizzled staging (the pieces
+// of the last columns by plain stores).  Null: plain stores throughout.
 __device__ __forceinline__ void epilogue_wgrad(const Params &P, uint32_t taddr, bool zero, float *dst,
-                                               int col0, uint8_t *stg, int lane) {
+                                               int col0, uint8_t *stg, int lane,
+                                               const CUtensorMap *om = nullptr, int64_t orow = 0) {
   uint32_t r[32];
 #pragma unroll 1
   for (int c = 0; c < P.bn / 32; ++c) {
@@ -692,7 +697,22 @@ __device__ __forceinline__ void epilogue_wgrad(const Params &P, uint32_t taddr, 
       for (int i = 0; i < 32; ++i) r[i] = 0u;
     }
     if (col >= P.N) break;                                      // the same for the whole CTA
-    if (col + 32 <= P.N && (P.N & 3) == 0) {
+    if (P.tma_store) {                                          // the last TMA store has read stg
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+    }
+    if (om && col + 32 <= P.N) {
+      uint4 *mine = reinterpret_cast<uint4 *>(stg + lane * 128);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        mine[stage_slot<8>(lane, q)] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(om, stg, col, (int)orow);
+        bulk_commit();
+      }
+    } else if (col + 32 <= P.N && (P.N & 3) == 0) {
       store_rows_at(stg, r, dst ? reinterpret_cast<char *>(dst + col) : nullptr, lane);
     } else if (dst) {
 #pragma unroll
@@ -1041,7 +1061,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                              const __grid_constant__ CUtensorMap map_a_static,
                              const __grid_constant__ CUtensorMap map_b,
                              const __grid_constant__ CUtensorMap map_b3,
-                             const __grid_constant__ CUtensorMap map_out, const Params P) {
+                             const __grid_constant__ CUtensorMap map_out,
+                             const __grid_constant__ CUtensorMap map_out2, const Params P) {
   constexpr int PM = 2 * BM;                         // rows per pair tile
   constexpr int STAGES = BKS == 2 ? kPairStages2 : kPairStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1332,7 +1353,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     ? reinterpret_cast<float *>(P.out) + ((int64_t)tl.g * P.split_m + row) * P.N
                     : reinterpret_cast<float *>(P.out2) +
                           ((int64_t)tl.g * (P.M - P.split_m) + row - P.split_m) * P.N;
-        epilogue_wgrad(P, taddr, zero, dst, tl.n * P.bnh, stg, lane);
+        // the warp's 32 rows by TMA stores when they lie in one output part
+        const int row0w = tl.m * PM + (int)rank * BM + ew * 32;
+        const CUtensorMap *om = nullptr;
+        int64_t orow = 0;
+        if (P.tma_store && row0w + 32 <= P.M) {
+          if (row0w + 32 <= P.split_m) {
+            om = &map_out;
+            orow = (int64_t)tl.g * P.split_m + row0w;
+          } else if (row0w >= P.split_m) {
+            om = &map_out2;
+            orow = (int64_t)tl.g * (P.M - P.split_m) + row0w - P.split_m;
+          }
+        }
+        epilogue_wgrad(P, taddr, zero, dst, tl.n * P.bnh, stg, lane, om, orow);
       } else if (in_tail && kb0 > 0) {
         sk_write(P, 2 * pair + (int)rank, r_cta, taddr);        // a later piece of the tile
       } else {
@@ -1889,6 +1923,21 @@ bool make_map_box(CUtensorMap *m, const void *base, uint64_t inner, uint64_t out
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor [outer][inner] (inner contiguous) in boxes of 32 rows x
+// 32 columns (128 bytes), 128-byte swizzled: the weight-gradient epilogue's
+// TMA stores from its swizzled staging.
+bool make_map_f32(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || outer == 0) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int device_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -1913,7 +1962,7 @@ cudaError_t launch_epi(const Params &P, const CUtensorMap &ma,
 template <int EPI, int BKS>
 cudaError_t launch_pair(const Params &P, const CUtensorMap &ma, const CUtensorMap &mas,
                         const CUtensorMap &mb, const CUtensorMap &mb3, const CUtensorMap &mo,
-                        int64_t max_tiles, size_t smem, cudaStream_t s) {
+                        const CUtensorMap &mo2, int64_t max_tiles, size_t smem, cudaStream_t s) {
   auto kern = grouped_gemm_pair_kernel<EPI, BKS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -1936,7 +1985,7 @@ cudaError_t launch_pair(const Params &P, const CUtensorMap &ma, const CUtensorMa
   }
   const int64_t want = P.sk_part ? mc : std::min<int64_t>(mc, max_tiles);
   const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(want, kSkSlots / 2));
-  return launch_kernel(kern, 2 * pairs, kThreads, smem, s, ma, mas, mb, mb3, mo, P);
+  return launch_kernel(kern, 2 * pairs, kThreads, smem, s, ma, mas, mb, mb3, mo, mo2, P);
 }
 
 // Token-N launch: as many 2-CTA clusters as fit at once, fewer when there are
@@ -2119,12 +2168,26 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
       !g.kgroup && g.out_rows > 0 && g.out_rows < ((int64_t)1 << 31) && g.N % 64 == 0 &&
       make_map(&mo, g.out, (uint64_t)g.N, (uint64_t)g.out_rows, 32))
     P.tma_store = 1;
+  // weight gradients (fp32, K groups) on CTA pairs: whole 32-row x 32-column
+  // pieces by TMA stores, one map per output part (rows below split_m, and
+  // the rest); a warp's rows never straddle the two when split_m is a
+  // multiple of 32
+  CUtensorMap mo2;
+  if (MOE_PAIR_TMA_STORE && g.kgroup && pair && g.epi == kEpiStoreF32 && g.N % 4 == 0 &&
+      (!g.out2 || P.split_m % 32 == 0) &&
+      make_map_f32(&mo, g.out, (uint64_t)g.N, (uint64_t)P.G * P.split_m) &&
+      (!g.out2 || make_map_f32(&mo2, g.out2, (uint64_t)g.N, (uint64_t)P.G * (g.M - P.split_m))))
+    P.tma_store = 1;
+  if (!g.out2 || !P.tma_store) mo2 = mo;
   const uint32_t box_b = (swiglu_b(g.epi) || pair) ? 128u : (uint32_t)P.bn;
   // K groups: A is [M, K] and B [N, K] with all groups' K columns side by side
   const uint64_t a_outer = g.kgroup ? (uint64_t)g.M : (uint64_t)g.a_rows;
   const uint64_t b_outer = g.kgroup ? (uint64_t)g.N : (uint64_t)g.b_rows;
   if (!make_map(&ma, g.a, (uint64_t)g.K, a_outer, BM)) return cudaErrorInvalidValue;
-  if (!P.tma_store) mo = ma;                                 // (not read)
+  if (!P.tma_store) {                                        // (not read)
+    mo = ma;
+    mo2 = ma;
+  }
   if (!make_map(&mas, g.a_static && !g.kgroup ? g.a_static : g.a, (uint64_t)g.K,
                 (uint64_t)(g.a_static && !g.kgroup ? g.a_static_rows : a_outer), BM))
     return cudaErrorInvalidValue;
@@ -2169,8 +2232,8 @@ cudaError_t launch_grouped_gemm(const GroupedGemm &g, cudaStream_t s) {
                          1024 + 4 * kStageBytesPerWarp;
 #define MOE_PAIR_CASE(E_)                                                            \
   case E_:                                                                           \
-    return bk2 ? launch_pair<E_, 2>(P, ma, mas, mb, mb3, mo, pair_tiles, psmem, s)   \
-               : launch_pair<E_, 1>(P, ma, mas, mb, mb3, mo, pair_tiles, psmem, s);
+    return bk2 ? launch_pair<E_, 2>(P, ma, mas, mb, mb3, mo, mo2, pair_tiles, psmem, s)   \
+               : launch_pair<E_, 1>(P, ma, mas, mb, mb3, mo, mo2, pair_tiles, psmem, s);
     switch (g.epi) {
       MOE_PAIR_CASE(kEpiStoreF32)
       MOE_PAIR_CASE(kEpiRelu)
