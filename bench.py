@@ -51,12 +51,13 @@ SUSTAINED_MIN_MS = 1.0
 # the GEMM sources (the kernel file, then its PTX wrappers) they were taken
 # at; reported only while the sources are unchanged (null otherwise).
 NCU_TRAFFIC: dict[str, dict] = {
-    # up 151.09 + 39.97 MB, down 220.03 + 6.44 MB
-    "gshard": {"bytes": 417_516_800, "src": "185a493843fb085a"},
-    # captured on a 40-expert cut of the layer and scaled to 160 + 2 experts
-    # (weights) and 60693 kept rows (h, y_rows): up 1496.2 + 40.0 MB, down
-    # 707.4 + 118.8 MB at the cut
-    "deepseek_v2": {"bytes": 9_144_011_170, "src": "185a493843fb085a"},
+    # up 151.11 + 40.05 MB, down 220.19 + 6.10 MB
+    "gshard": {"bytes": 417_442_304, "src": "1f89c012e2ab7a21"},
+    # captured on a 40 + 2-expert cut of the layer (15173 kept rows): up
+    # 1496.68 + 40.32 MB, down 707.72 + 119.18 MB; scaled to the whole layer
+    # as every expert's weights read once (7644 MB) plus the cut's other
+    # bytes (382.1 MB) times the kept rows' ratio (60693 / 15173)
+    "deepseek_v2": {"bytes": 9_172_527_711, "src": "1f89c012e2ab7a21"},
 }
 
 
