@@ -484,10 +484,11 @@ __global__ void __launch_bounds__(1024) keep_select_kernel(
   const int n = cnt_off[e + 1] - start;
   const int m = kept[e];
   const int32_t *list = sorted_q + start;
+  // q = j * T + t < T * k <= 2^31 - 1 (validated): 32-bit division is exact
+  const uint32_t T32 = (uint32_t)T;
   auto key_of = [&](int i) -> uint64_t {
-    const int64_t q = list[i];
-    const int64_t t = q % T;
-    return affinity_key(probs[t * E + e], (uint32_t)t);
+    const uint32_t t = (uint32_t)list[i] % T32;
+    return affinity_key(probs[(int64_t)t * E + e], t);
   };
   uint64_t thr = 0ull;          // keep keys >= thr
   bool keep_all = m >= n, keep_none = m <= 0;
@@ -523,7 +524,7 @@ __global__ void __launch_bounds__(1024) keep_select_kernel(
     int total;
     const int r = block_exclusive_scan(keep ? 1 : 0, scratch, &total);
     if (i < n) {
-      const int64_t j = q / T, t = q - j * T;
+      const int64_t j = (uint32_t)q / T32, t = q - j * T;
       if (keep) {
         const int slot = row0 + done + r;
         tok_rows[t * k + j] = slot;
